@@ -1,0 +1,100 @@
+"""Named attention workloads and their seeded bf16 inputs.
+
+Shapes are per head ``[B, H, N, d]`` (d fastest).  Values are iid N(0, 1)
+(times ``std``) drawn in fp32 from a CPU ``torch.Generator`` and rounded to
+bf16 (round-to-nearest-even), in the order Q, K, V; the output gradient dO of
+the backward workload comes from a second seed.  The five workloads follow the
+shapes the FlashAttention pages discuss: a tiny smoke case, a GPT-2-like
+sequence length (FlashAttention (NL), "Empirische resultaten": GPT-2 at 1K),
+a causal LLM shape, its backward with recomputation (memory-optimized flash
+attention page, "How it works") and a long-context sliding-window case
+(sparse-attention glossary, "Abgrenzung": sliding-window attention).
+
+Nothing in this module computes attention.
+"""
+
+from __future__ import annotations
+
+import math
+import random
+from dataclasses import dataclass, replace
+
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    H: int
+    N: int
+    d: int
+    causal: bool = False
+    window: int = 0          # 0 = no band; W > 0 keeps keys i-W+1 .. i (causal only)
+    std: float = 1.0
+    seed: int = 0
+    grad_seed: int | None = None   # seed of dO (backward workloads)
+    oracle_heads: int | None = None  # heads the oracle checks (None = all)
+    description: str = ""
+
+    @property
+    def scale(self) -> float:
+        # the 1/sqrt(d_k) of the attention formula (FlashAttention (NL),
+        # "Problemen met standaard attention")
+        return 1.0 / math.sqrt(self.d)
+
+    @property
+    def BH(self) -> int:
+        return self.B * self.H
+
+    def with_(self, **kw) -> "Workload":
+        return replace(self, **kw)
+
+
+WORKLOADS: dict[str, Workload] = {
+    "tiny": Workload("tiny", 1, 2, 128, 64, seed=1001,
+                     description="tiny forward B1 H2 N128 d64 non-causal"),
+    "gpt2": Workload("gpt2", 4, 16, 2048, 64, seed=1002,
+                     description="GPT-2-like forward B4 H16 N2048 d64 non-causal"),
+    "causal": Workload("causal", 2, 32, 4096, 128, causal=True, std=0.5, seed=1003,
+                       description="causal LLM-shape forward B2 H32 N4096 d128"),
+    "bwd": Workload("bwd", 2, 32, 4096, 128, causal=True, std=0.5, seed=1003,
+                    grad_seed=2003,
+                    description="causal backward B2 H32 N4096 d128, dO seed 2003"),
+    "long": Workload("long", 1, 16, 32768, 128, causal=True, window=4096, seed=1005,
+                     oracle_heads=2,
+                     description="long-context forward B1 H16 N32768 d128 causal+window 4096"),
+}
+
+
+def _randn_bf16(gen: torch.Generator, shape, std: float) -> torch.Tensor:
+    x = torch.randn(*shape, generator=gen, dtype=torch.float32)
+    if std != 1.0:
+        x = x * std
+    return x.to(torch.bfloat16)
+
+
+def make_inputs(wl: Workload, seed: int | None = None):
+    """Q, K, V as contiguous CPU bf16 tensors of shape [B, H, N, d]."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(wl.seed if seed is None else seed)
+    shape = (wl.B, wl.H, wl.N, wl.d)
+    q = _randn_bf16(gen, shape, wl.std)
+    k = _randn_bf16(gen, shape, wl.std)
+    v = _randn_bf16(gen, shape, wl.std)
+    return q, k, v
+
+
+def make_grad_output(wl: Workload, seed: int | None = None) -> torch.Tensor:
+    """dO as a contiguous CPU bf16 tensor [B, H, N, d], N(0, 1) from the grad seed."""
+    s = seed if seed is not None else (wl.grad_seed if wl.grad_seed is not None else wl.seed + 1000)
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(s)
+    return _randn_bf16(gen, (wl.B, wl.H, wl.N, wl.d), 1.0)
+
+
+def head_subset(wl: Workload, count: int, seed: int | None = None) -> list[int]:
+    """A seeded, sorted sample of flat head indices b*H + h."""
+    rng = random.Random(wl.seed if seed is None else seed)
+    count = min(count, wl.BH)
+    return sorted(rng.sample(range(wl.BH), count))

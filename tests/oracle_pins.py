@@ -1,0 +1,307 @@
+"""Checks that pin the fp64 oracle to facts other than itself.
+
+Each check takes the oracle module and raises AssertionError when the oracle
+disagrees with a closed form, an invariant of exact attention, a hand-derived
+example (tests/golden/), central finite differences, or an independent library
+routine (torch's scaled_dot_product_attention and autograd, in float64).  The
+checks are written so that a plausible slip anywhere in the oracle (a dropped
+scale, a swapped operand, an off-by-one mask edge, a missing max shift, a
+transposed gradient) fails at least one of them; tests/test_oracle_mutants.py
+plants such slips and confirms it.
+"""
+
+from __future__ import annotations
+
+import json
+import math
+import pathlib
+
+import numpy as np
+
+GOLDEN = pathlib.Path(__file__).parent / "golden"
+MASKS = [(False, 0), (True, 0), (True, 1), (True, 3), (True, 7)]
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _qkv(seed, n=13, d=5, lead=(2,), std=1.0):
+    r = _rng(seed)
+    return [std * r.standard_normal(lead + (n, d)) for _ in range(3)]
+
+
+def _n_allowed(i, n, causal, window):
+    hi = i if causal else n - 1
+    lo = max(0, i - window + 1) if window > 0 else 0
+    return hi - lo + 1
+
+
+# --- forward pins -------------------------------------------------------------------------
+
+def rows_sum_to_one(orc):
+    """Every softmax row is a probability vector over the allowed keys only."""
+    q, k, _ = _qkv(1)
+    for causal, window in MASKS:
+        p = orc.attention_probabilities(q, k, 0.7, causal, window)
+        assert np.all(p >= 0)
+        assert np.max(np.abs(p.sum(-1) - 1.0)) < 1e-12
+        n = q.shape[-2]
+        i = np.arange(n)[:, None]
+        j = np.arange(n)[None, :]
+        masked = np.zeros((n, n), bool)
+        if causal:
+            masked |= j > i
+        if window:
+            masked |= j < i - window + 1
+        assert np.all(p[..., masked] == 0.0)
+
+
+def constant_v(orc):
+    """V with every row equal to c gives O rows equal to c for every mask."""
+    q, k, _ = _qkv(2)
+    c = np.array([0.5, -2.0, 3.25, 0.0, 1.0])
+    v = np.broadcast_to(c, q.shape).copy()
+    for causal, window in MASKS:
+        o, _ = orc.attention_forward(q, k, v, 0.9, causal, window)
+        assert np.max(np.abs(o - c)) < 1e-12
+
+
+def causal_row0(orc):
+    """Causal row 0 sees only key 0: O_0 = v_0 and L_0 = scale q_0 . k_0."""
+    q, k, v = _qkv(3)
+    o, lse = orc.attention_forward(q, k, v, 0.37, True, 0)
+    assert np.max(np.abs(o[..., 0, :] - v[..., 0, :])) < 1e-12
+    l0 = 0.37 * np.sum(q[..., 0, :] * k[..., 0, :], -1)
+    assert np.max(np.abs(lse[..., 0] - l0)) < 1e-12
+
+
+def causal_future_independence(orc):
+    """Changing keys/values after row i leaves causal rows <= i unchanged, and changes row i+1."""
+    q, k, v = _qkv(4)
+    o, lse = orc.attention_forward(q, k, v, 0.5, True, 0)
+    i = 6
+    k2, v2 = k.copy(), v.copy()
+    k2[..., i + 1:, :] += 3.0
+    v2[..., i + 1:, :] -= 5.0
+    o2, l2 = orc.attention_forward(q, k2, v2, 0.5, True, 0)
+    assert np.max(np.abs(o2[..., :i + 1, :] - o[..., :i + 1, :])) < 1e-12
+    assert np.max(np.abs(l2[..., :i + 1] - lse[..., :i + 1])) < 1e-12
+    assert np.max(np.abs(o2[..., i + 1, :] - o[..., i + 1, :])) > 1e-3
+
+
+def window_one(orc):
+    """A window of 1 keeps only the diagonal: O_i = v_i, L_i = scale q_i . k_i."""
+    q, k, v = _qkv(5)
+    o, lse = orc.attention_forward(q, k, v, 0.8, True, 1)
+    assert np.max(np.abs(o - v)) < 1e-12
+    assert np.max(np.abs(lse - 0.8 * np.sum(q * k, -1))) < 1e-12
+
+
+def window_covering_is_causal(orc):
+    """A window of N or more equals plain causal attention."""
+    q, k, v = _qkv(6)
+    n = q.shape[-2]
+    o, lse = orc.attention_forward(q, k, v, 0.6, True, 0)
+    for w in (n, n + 5):
+        o2, l2 = orc.attention_forward(q, k, v, 0.6, True, w)
+        assert np.max(np.abs(o2 - o)) < 1e-12 and np.max(np.abs(l2 - lse)) < 1e-12
+
+
+def window_edge(orc):
+    """Row i with window W ignores key i-W and depends on key i-W+1."""
+    q, k, v = _qkv(7)
+    w, i = 4, 9
+    o, _ = orc.attention_forward(q, k, v, 0.6, True, w)
+    for j, should_change in ((i - w, False), (i - w + 1, True)):
+        k2, v2 = k.copy(), v.copy()
+        k2[..., j, :] += 2.0
+        v2[..., j, :] += 7.0
+        o2, _ = orc.attention_forward(q, k2, v2, 0.6, True, w)
+        diff = np.max(np.abs(o2[..., i, :] - o[..., i, :]))
+        assert (diff > 1e-3) if should_change else (diff < 1e-12)
+
+
+def scale_zero(orc):
+    """scale = 0 gives uniform weights: L_i = ln(#allowed keys), O_i = mean of the allowed v_j."""
+    q, k, v = _qkv(8)
+    n = q.shape[-2]
+    for causal, window in MASKS:
+        o, lse = orc.attention_forward(q, k, v, 0.0, causal, window)
+        for i in range(n):
+            cnt = _n_allowed(i, n, causal, window)
+            lo = max(0, i - window + 1) if window else 0
+            hi = i + 1 if causal else n
+            assert abs(lse[..., i] - math.log(cnt)).max() < 1e-12
+            assert np.max(np.abs(o[..., i, :] - v[..., lo:hi, :].mean(-2))) < 1e-12
+
+
+def key_shift(orc):
+    """K_j <- K_j + c for every j leaves O unchanged and shifts L_i by scale q_i . c."""
+    q, k, v = _qkv(9)
+    c = np.array([0.3, -1.1, 0.7, 2.0, -0.4])
+    for causal, window in MASKS:
+        o, lse = orc.attention_forward(q, k, v, 0.45, causal, window)
+        o2, l2 = orc.attention_forward(q, k + c, v, 0.45, causal, window)
+        assert np.max(np.abs(o2 - o)) < 1e-11
+        assert np.max(np.abs(l2 - lse - 0.45 * (q @ c))) < 1e-11
+
+
+def key_permutation(orc):
+    """Without a mask, permuting keys and values together leaves O and L unchanged."""
+    q, k, v = _qkv(10)
+    perm = _rng(10).permutation(q.shape[-2])
+    o, lse = orc.attention_forward(q, k, v, 0.5, False, 0)
+    o2, l2 = orc.attention_forward(q, k[..., perm, :], v[..., perm, :], 0.5, False, 0)
+    assert np.max(np.abs(o2 - o)) < 1e-12 and np.max(np.abs(l2 - lse)) < 1e-12
+
+
+def large_scores(orc):
+    """Scores of 1e3 (exp overflows fp64) must still give the exact softmax: the top key,
+    ahead of the runner-up by 200, takes all the weight."""
+    n, d = 6, 3
+    q = np.zeros((n, d))
+    q[:, 0] = 200.0
+    k = np.zeros((n, d))
+    k[:, 0] = np.arange(n, dtype=float)        # scores 200 * j, up to 1000
+    v = _rng(11).standard_normal((n, d))
+    o, lse = orc.attention_forward(q, k, v, 1.0, False, 0)
+    assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse))
+    assert np.max(np.abs(o - v[n - 1])) < 1e-12          # e^-200 relative weight of the runner-up
+    assert np.max(np.abs(lse - 200.0 * (n - 1))) < 1e-12
+
+
+def golden_examples(orc):
+    """Hand-derived examples (tests/golden/*.json) reproduce to 1e-12."""
+    for path in sorted(GOLDEN.glob("*.json")):
+        g = json.loads(path.read_text())
+        q, k, v = (np.array(g[x]) for x in ("q", "k", "v"))
+        for case in g["cases"]:
+            o, lse = orc.attention_forward(q, k, v, g["scale"], case["causal"], case["window"])
+            assert np.max(np.abs(o - np.array(case["O"]))) < 1e-12, path.name
+            assert np.max(np.abs(lse - np.array(case["L"]))) < 1e-12, path.name
+        if "backward_single_row" in g:
+            b = g["backward_single_row"]
+            dq, dk, dv = orc.attention_backward(np.array(b["q"]), k, v, np.array(b["dO"]), g["scale"])
+            assert np.max(np.abs(dq - np.array(b["dQ"]))) < 1e-12
+            assert np.max(np.abs(dk - np.array(b["dK"]))) < 1e-12
+            assert np.max(np.abs(dv - np.array(b["dV"]))) < 1e-12
+
+
+def _torch_reference(q, k, v, scale, causal, window):
+    import torch
+    import torch.nn.functional as F
+    tq, tk, tv = (torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (q, k, v))
+    n = q.shape[-2]
+    i = torch.arange(n)[:, None]
+    j = torch.arange(n)[None, :]
+    ok = torch.ones(n, n, dtype=torch.bool)
+    if causal:
+        ok &= j <= i
+    if window:
+        ok &= j >= i - window + 1
+    o = F.scaled_dot_product_attention(tq, tk, tv, attn_mask=ok, scale=scale)
+    return (tq, tk, tv), o
+
+
+def library_forward(orc):
+    """torch scaled_dot_product_attention (float64, boolean mask, explicit scale) agrees to 1e-12."""
+    q, k, v = _qkv(12, n=37, d=16, lead=(2, 3))
+    for causal, window in MASKS:
+        _, o_ref = _torch_reference(q, k, v, 0.25, causal, window)
+        o, _ = orc.attention_forward(q, k, v, 0.25, causal, window)
+        assert np.max(np.abs(o - o_ref.detach().numpy())) < 1e-12
+
+
+def library_backward(orc):
+    """torch autograd of sum(O o dO) through scaled_dot_product_attention agrees to 1e-11."""
+    import torch
+    q, k, v = _qkv(13, n=23, d=8, lead=(2,))
+    do = _rng(14).standard_normal(q.shape)
+    for causal, window in MASKS:
+        (tq, tk, tv), o_ref = _torch_reference(q, k, v, 0.4, causal, window)
+        (o_ref * torch.tensor(do)).sum().backward()
+        dq, dk, dv = orc.attention_backward(q, k, v, do, 0.4, causal, window)
+        for mine, ref in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
+            assert np.max(np.abs(mine - ref.numpy())) < 1e-11
+
+
+def finite_differences(orc):
+    """Central differences (h = 1e-6) of sum(O o dO) match dQ, dK, dV on tiny inputs."""
+    n, d, h, scale = 7, 3, 1e-6, 0.6
+    q, k, v = _qkv(15, n=n, d=d, lead=())
+    do = _rng(16).standard_normal((n, d))
+    for causal, window in MASKS:
+        grads = orc.attention_backward(q, k, v, do, scale, causal, window)
+
+        def f(qq, kk, vv):
+            return float(np.sum(orc.attention_forward(qq, kk, vv, scale, causal, window)[0] * do))
+
+        for which, g in enumerate(grads):
+            fd = np.zeros((n, d))
+            for a in range(n):
+                for b in range(d):
+                    args_p = [q.copy(), k.copy(), v.copy()]
+                    args_m = [q.copy(), k.copy(), v.copy()]
+                    args_p[which][a, b] += h
+                    args_m[which][a, b] -= h
+                    fd[a, b] = (f(*args_p) - f(*args_m)) / (2 * h)
+            err = np.linalg.norm(fd - g) / max(np.linalg.norm(fd), 1e-30)
+            assert err < 1e-6, (which, causal, window, err)
+
+
+def delta_identity(orc):
+    """sum_j P_ij dP_ij equals rowsum(dO o O): the D term a fused backward uses."""
+    q, k, v = _qkv(17, n=19, d=6, lead=())
+    do = _rng(18).standard_normal(q.shape)
+    for causal, window in MASKS:
+        p = orc.attention_probabilities(q, k, 0.5, causal, window)
+        o, _ = orc.attention_forward(q, k, v, 0.5, causal, window)
+        lhs = np.sum(p * (do @ v.T), -1)
+        rhs = np.sum(do * o, -1)
+        assert np.max(np.abs(lhs - rhs)) < 1e-12
+
+
+def row_blocks_match(orc):
+    """The row-block forward/backward equal the full-matrix ones (blocks smaller than N)."""
+    q, k, v = _qkv(19, n=41, d=8, lead=())
+    do = _rng(20).standard_normal(q.shape)
+    rows = np.array([0, 3, 17, 40])
+    for causal, window in MASKS:
+        o, lse = orc.attention_forward(q, k, v, 0.3, causal, window)
+        o_r, l_r = orc.attention_forward_rows(q, k, v, 0.3, causal, window, rows=rows, block=3)
+        assert np.max(np.abs(o_r - o[rows])) < 1e-12 and np.max(np.abs(l_r - lse[rows])) < 1e-12
+        dq, dk, dv = orc.attention_backward(q, k, v, do, 0.3, causal, window)
+        dq_r, dk_r, dv_r = orc.attention_backward_rows(q, k, v, do, 0.3, causal, window,
+                                                       key_rows=rows, block=5)
+        assert np.max(np.abs(dq_r - dq)) < 1e-12
+        assert np.max(np.abs(dk_r - dk[rows])) < 1e-12 and np.max(np.abs(dv_r - dv[rows])) < 1e-12
+
+
+def pair_count(orc):
+    """allowed_pairs matches the closed forms N^2, N(N+1)/2 and the banded count."""
+    for n in (1, 5, 16, 33):
+        assert orc.allowed_pairs(n, False, 0) == n * n
+        assert orc.allowed_pairs(n, True, 0) == n * (n + 1) // 2
+        for w in (1, 4, 40):
+            ww = min(w, n)
+            assert orc.allowed_pairs(n, True, w) == ww * (ww + 1) // 2 + (n - ww) * ww
+
+
+def rejects_bad_masks(orc):
+    """A negative window, or a window without causal, is rejected."""
+    q, k, v = _qkv(21, n=4, d=2, lead=())
+    for causal, window in ((True, -1), (False, 3)):
+        try:
+            orc.attention_forward(q, k, v, 1.0, causal, window)
+        except ValueError:
+            continue
+        raise AssertionError("bad mask accepted")
+
+
+PINS = {f.__name__: f for f in (
+    rows_sum_to_one, constant_v, causal_row0, causal_future_independence, window_one,
+    window_covering_is_causal, window_edge, scale_zero, key_shift, key_permutation,
+    large_scores, golden_examples, library_forward, library_backward, finite_differences,
+    delta_identity, row_blocks_match, pair_count, rejects_bad_masks,
+)}

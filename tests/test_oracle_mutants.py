@@ -1,0 +1,141 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and check that a pin catches each.
+
+If a mutant survived every pin, the pins would not be tying the oracle to the
+definition of attention tightly enough; this file is the evidence that they do.
+"""
+
+import numpy as np
+import pytest
+
+from oracle import attention as orc
+from tests.oracle_pins import PINS
+
+
+def _scores_transposed(q, k, scale, ok):
+    return np.where(ok, scale * (k @ q.T), -np.inf)
+
+
+def _scores_no_scale(q, k, scale, ok):
+    return np.where(ok, q @ k.T, -np.inf)
+
+
+def _rows_mask_causal_strict(r, n_k, causal, window):
+    i = r[:, None]
+    j = np.arange(n_k)[None, :]
+    ok = np.ones((r.size, n_k), dtype=bool)
+    if causal:
+        ok &= j < i
+    if window > 0:
+        ok &= j >= i - window + 1
+    return ok
+
+
+def _rows_mask_window_wide(r, n_k, causal, window):
+    i = r[:, None]
+    j = np.arange(n_k)[None, :]
+    ok = np.ones((r.size, n_k), dtype=bool)
+    if causal:
+        ok &= j <= i
+    if window > 0:
+        ok &= j >= i - window
+    return ok
+
+
+def _rows_mask_no_window_check(r, n_k, causal, window):
+    i = r[:, None]
+    j = np.arange(n_k)[None, :]
+    ok = np.ones((r.size, n_k), dtype=bool)
+    if causal:
+        ok &= j <= i
+    if window > 0:
+        ok &= j >= i - window + 1
+    return ok
+
+
+def _softmax_no_shift(s):
+    e = np.exp(s)
+    denom = np.sum(e, axis=1, keepdims=True)
+    return e / denom, np.log(denom)[:, 0]
+
+
+def _softmax_log2(s):
+    m = np.max(s, axis=1, keepdims=True)
+    e = np.exp(s - m)
+    denom = np.sum(e, axis=1, keepdims=True)
+    return e / denom, (m + np.log2(denom))[:, 0]
+
+
+def _softmax_lse_no_max(s):
+    m = np.max(s, axis=1, keepdims=True)
+    e = np.exp(s - m)
+    denom = np.sum(e, axis=1, keepdims=True)
+    return e / denom, np.log(denom)[:, 0]
+
+
+def _make_bwd(variant):
+    def bwd(q, k, v, do, scale, causal, window):
+        o, lse, p = orc._head_forward(q, k, v, scale, causal, window)
+        dv = p.T @ do
+        dp = do @ v.T
+        d_row = np.sum(p * dp, axis=1, keepdims=True)
+        if variant == "dv_untransposed":
+            dv = p @ do
+        if variant == "dp_swapped":
+            dp = (v @ do.T).T if dp.shape[0] == dp.shape[1] else do @ v.T * 1.01
+        if variant == "delta_wrong_axis":
+            d_row = np.sum(p * dp, axis=0, keepdims=True)
+        if variant == "delta_missing":
+            d_row = 0.0
+        ds = p * (dp - d_row)
+        dq = scale * (ds @ k)
+        dk = scale * (ds.T @ q)
+        if variant == "dq_no_scale":
+            dq = ds @ k
+        if variant == "dk_untransposed":
+            dk = scale * (ds @ q)
+        return dq, dk, dv
+    return bwd
+
+
+def _head_forward_pv_transposed(q, k, v, scale, causal, window, row_start=0):
+    ok = orc.allowed_mask(q.shape[0], k.shape[0], causal, window, row_start)
+    p, lse = orc._softmax_rows(orc._scores(q, k, scale, ok))
+    return p.T @ v, lse, p
+
+
+MUTANTS = {
+    "scores_transposed": ("_scores", _scores_transposed),
+    "scale_dropped": ("_scores", _scores_no_scale),
+    "causal_excludes_diagonal": ("_rows_mask", _rows_mask_causal_strict),
+    "window_one_too_wide": ("_rows_mask", _rows_mask_window_wide),
+    "window_without_causal_accepted": ("_check_mask_args", lambda causal, window: None),
+    "no_max_shift": ("_softmax_rows", _softmax_no_shift),
+    "lse_in_log2": ("_softmax_rows", _softmax_log2),
+    "lse_missing_max": ("_softmax_rows", _softmax_lse_no_max),
+    "probabilities_transposed": ("_head_forward", _head_forward_pv_transposed),
+    "dv_untransposed": ("_head_backward", _make_bwd("dv_untransposed")),
+    "delta_wrong_axis": ("_head_backward", _make_bwd("delta_wrong_axis")),
+    "delta_missing": ("_head_backward", _make_bwd("delta_missing")),
+    "dq_no_scale": ("_head_backward", _make_bwd("dq_no_scale")),
+    "dk_untransposed": ("_head_backward", _make_bwd("dk_untransposed")),
+}
+
+
+def _first_failing_pin():
+    import warnings
+    for name in sorted(PINS):
+        try:
+            with warnings.catch_warnings():
+                warnings.simplefilter("ignore")
+                PINS[name](orc)
+        except Exception:  # an assertion, or a shape/overflow error the slip causes
+            return name
+    return None
+
+
+@pytest.mark.parametrize("mutant", sorted(MUTANTS))
+def test_mutant_is_caught(mutant, monkeypatch):
+    attr, fn = MUTANTS[mutant]
+    monkeypatch.setattr(orc, attr, fn)
+    caught_by = _first_failing_pin()
+    assert caught_by is not None, f"mutant {mutant} survived every pin"
