@@ -1,0 +1,452 @@
+#!/usr/bin/env python
+"""Throughput of the exact-attention hot path on B200, one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one pass of the whole path over the causal LLM-shape workload
+(B=2, H=32, N=4096, d=128, causal; inputs N(0,1)*0.5 in bf16): the forward
+kernel (O and logsumexp) followed, when the library has it, by the backward
+with recomputation (dQ, dK, dV from Q, K, V, O, dO and L).  Throughput is
+TFLOP/s with the usual convention: forward 4*B*H*N^2*d, halved for causal;
+backward 2.5x the forward.
+
+Timing: W untimed warm-up steps, then K steps bracketed by a barrier and a
+device synchronise; every step is timed with CUDA events on the launching
+stream and L2 is flushed (256 MB write) between steps, outside the events.
+With N > 1 ranks (torchrun, NCCL) every rank runs its own copy of the
+workload (independent heads: weak scaling, no collective on the data path)
+and the time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle (the definition of the result,
+not a GPU program) on a bounded row-block sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+WORKLOAD = "causal"          # forward workload; the backward uses the same shape
+GRAD_WORKLOAD = "bwd"
+FLUSH_BYTES = 256 << 20      # > 126 MB L2
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- FLOPs
+def fwd_flops(B, H, N, d, causal) -> float:
+    f = 4.0 * B * H * N * N * d
+    return f / 2 if causal else f
+
+
+def bwd_flops(B, H, N, d, causal) -> float:
+    return 2.5 * fwd_flops(B, H, N, d, causal)
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return FALLBACK_PEAKS, "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples (every 100 ms) of SM clock and throttle reasons."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.samples = []
+        self.proc = None
+        self.thread = None
+        self.window = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm, smax = float(parts[1]), float(parts[2])
+            except ValueError:
+                continue
+            self.samples.append((time.time(), sm, smax, parts[5:9]))
+
+    def mark(self, t0, t1):
+        self.window = (t0, t1)
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        t0, t1 = self.window or (0, float("inf"))
+        inside = [s for s in self.samples if t0 - 0.05 <= s[0] <= t1 + 0.05]
+        used = inside if inside else self.samples
+        reasons = sorted({name for s in used for name, flag in zip(self.REASONS, s[3])
+                          if flag.lower() == "active"})
+        return {"sm_mhz": statistics.median(s[1] for s in used),
+                "sm_max_mhz": max(s[2] for s in used), "reasons": reasons,
+                "samples": len(inside), "samples_total": len(self.samples)}
+
+
+def gpu_id_for(dev_index: int) -> str:
+    import torch
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev_index).uuid)
+        return uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    except Exception:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        if vis:
+            return vis.split(",")[dev_index]
+        return str(dev_index)
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_sample(seconds: float, rows_per_block: int = 512, with_bwd: bool = True,
+                  max_blocks: int | None = None):
+    """Time the fp64 oracle on contiguous query-row blocks of head 0 of the workload.
+
+    Returns (flops credited, seconds, blocks, cores).  A block of R rows is credited
+    R/N of one head's conventional forward (+ backward) FLOPs.
+    """
+    import numpy as np
+    from oracle import attention as orc
+    from synthetic import WORKLOADS, make_grad_output, make_inputs
+    wl = WORKLOADS[WORKLOAD]
+    sub = wl.with_(B=1, H=1)
+    q, k, v = (x[0, 0] for x in make_inputs(sub))
+    do = make_grad_output(WORKLOADS[GRAD_WORKLOAD].with_(B=1, H=1))[0, 0]
+    q, k, v, do = (x.double().numpy() for x in (q, k, v, do))
+    per_row = fwd_flops(1, 1, wl.N, wl.d, wl.causal) / wl.N
+    if with_bwd:
+        per_row += bwd_flops(1, 1, wl.N, wl.d, wl.causal) / wl.N
+    t0 = time.perf_counter()
+    blocks = 0
+    start = 0
+    while True:
+        rows = np.arange(start, start + rows_per_block) % wl.N
+        orc.attention_forward_rows(q, k, v, wl.scale, wl.causal, wl.window, rows=rows)
+        if with_bwd:
+            orc.attention_backward_rows(q, k, v, do, wl.scale, wl.causal, wl.window, query_rows=rows)
+        blocks += 1
+        start = (start + rows_per_block) % wl.N
+        el = time.perf_counter() - t0
+        if el >= seconds or (max_blocks is not None and blocks >= max_blocks):
+            break
+    return per_row * rows_per_block * blocks, el, blocks, blas_threads()
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=300))
+
+    import exact_io_aware_77_b200 as fa
+    fa.load()                                    # no library, no bench: fails loudly
+    from synthetic import WORKLOADS, make_grad_output, make_inputs
+
+    wl = WORKLOADS[WORKLOAD]
+    B, H, N, d = wl.B, wl.H, wl.N, wl.d
+    has_bwd = hasattr(fa, "backward")
+    q_h, k_h, v_h = make_inputs(wl)
+    do_h = make_grad_output(WORKLOADS[GRAD_WORKLOAD])
+    q, k, v, do = (x.to(dev) for x in (q_h, k_h, v_h, do_h))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    grads = (torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)) if has_bwd else None
+    ws = None
+    if has_bwd:
+        ws = torch.empty(fa.bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    f_fwd = fwd_flops(B, H, N, d, wl.causal)
+    f_bwd = bwd_flops(B, H, N, d, wl.causal) if has_bwd else 0.0
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        fa.forward(q, k, v, wl.scale, wl.causal, wl.window, out=o, lse=lse)
+        if ev:
+            ev[1].record(stream)
+        if has_bwd:
+            fa.backward(q, k, v, o, lse, do, wl.scale, wl.causal, wl.window, grads=grads, workspace=ws)
+            if ev:
+                ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    st = fa.check_status(dev)
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {fa.STATUS_NAMES.get(st, st)}")
+
+    sampler = ClockSampler(gpu_id_for(local))
+    sampler.start()
+    time.sleep(0.3)
+    n_ev = 3 if has_bwd else 2
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    wall0 = time.time()
+    for i in range(args.steps):
+        flush.zero_()
+        step(events[i])
+    torch.cuda.synchronize(dev)
+    wall1 = time.time()
+    if world > 1:
+        dist.barrier()
+    sampler.mark(wall0, wall1)
+    time.sleep(0.25)
+    sampler.stop()
+    st = fa.check_status(dev)
+    if st != 0:
+        raise RuntimeError(f"device status after timing: {fa.STATUS_NAMES.get(st, st)}")
+
+    fwd_ms = [e[0].elapsed_time(e[1]) for e in events]
+    bwd_ms = [e[1].elapsed_time(e[2]) for e in events] if has_bwd else [0.0] * args.steps
+    step_ms_total = sum(f + b for f, b in zip(fwd_ms, bwd_ms))
+    fwd_total, bwd_total = sum(fwd_ms), sum(bwd_ms)
+    if world > 1:
+        t = torch.tensor([step_ms_total, fwd_total, bwd_total], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        step_ms_total, fwd_total, bwd_total = t.tolist()
+    ms_per_step = step_ms_total / args.steps
+    value = world * (f_fwd + f_bwd) / (ms_per_step * 1e-3) / 1e12
+
+    # end to end through the public API: pinned host inputs -> device -> path -> host outputs
+    e2e = None
+    if not args.no_e2e:
+        e2e = measure_e2e(fa, torch, wl, dev, stream, q_h, k_h, v_h, do_h, has_bwd, args.e2e_steps,
+                          f_fwd + f_bwd, world)
+
+    peaks, peak_kind = load_peaks()
+    fwd_ms_avg = fwd_total / args.steps
+    bwd_ms_avg = bwd_total / args.steps
+    if has_bwd and bwd_ms_avg > fwd_ms_avg:
+        dom, dom_flops, dom_ms = "fa_bwd (3 kernels)", f_bwd, bwd_ms_avg
+    else:
+        dom, dom_flops, dom_ms = "fa_fwd_kernel<128>", f_fwd, fwd_ms_avg
+    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 1),
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(achieved / peaks["bf16_tflops"], 4),
+                "peak_source": f"{peak_kind} burst bf16 (MEASURED_PEAKS.json)" if peak_kind == "measured"
+                else "fallback 1.59 PFLOP/s",
+                "traffic": load_traffic(dom)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        flops, secs, blocks, cores = oracle_sample(args.cpu_seconds, with_bwd=has_bwd)
+        cpu = {"value": round(flops / secs / 1e12, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+               "sample": f"{blocks} blocks of 512 query rows of head 0 of the B2 H32 N4096 d128 causal "
+                         f"workload through the fp64 oracle ({'fwd+bwd' if has_bwd else 'fwd'}), "
+                         f"{secs:.1f} s, credited rows/N of a head's conventional FLOPs"}
+
+    clocks = sampler.summary()
+    line = {
+        "metric": "attention fwd/bwd TFLOP/s at 1 B200; % of dense BF16 tensor peak",
+        "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": ("causal LLM shape forward+backward" if has_bwd else
+                                "causal LLM shape forward (backward not built yet)") +
+                   f": B={B} H={H} N={N} d={d} causal, inputs N(0,1)*0.5 bf16 seeded",
+                   "global_batch": B * world, "seq_len": N, "parallelism": f"replicas{world}",
+                   "l2": "flushed (256 MB write) between timed steps, outside the events"},
+        "fwd_tflops": round(world * f_fwd / (fwd_ms_avg * 1e-3) / 1e12, 2),
+        "fwd_ms": round(fwd_ms_avg, 4),
+        "pct_of_measured_peak": round(100 * value / world / peaks["bf16_tflops"], 2),
+        "pct_of_spec_peak_2250": round(100 * value / world / 2250.0, 2),
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": args.steps * (1 + (3 if has_bwd else 0)),
+        "clocks": clocks,
+    }
+    if has_bwd:
+        line["bwd_tflops"] = round(world * f_bwd / (bwd_ms_avg * 1e-3) / 1e12, 2)
+        line["bwd_ms"] = round(bwd_ms_avg, 4)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def measure_e2e(fa, torch, wl, dev, stream, q_h, k_h, v_h, do_h, has_bwd, steps, flops, world):
+    pin = [x.pin_memory() for x in (q_h, k_h, v_h, do_h if has_bwd else q_h[:0])]
+    q, k, v = (torch.empty_like(x, device=dev) for x in pin[:3])
+    do = torch.empty_like(pin[3], device=dev) if has_bwd else None
+    o = torch.empty_like(q)
+    lse = torch.empty((wl.B, wl.H, wl.N), dtype=torch.float32, device=dev)
+    o_h = torch.empty_like(pin[0]).pin_memory()
+    l_h = torch.empty((wl.B, wl.H, wl.N), dtype=torch.float32).pin_memory()
+    grads = grads_h = ws = None
+    if has_bwd:
+        grads = tuple(torch.empty_like(q) for _ in range(3))
+        grads_h = tuple(torch.empty_like(pin[0]).pin_memory() for _ in range(3))
+        ws = torch.empty(fa.bwd_workspace_size(wl.B, wl.H, wl.N, wl.d), dtype=torch.uint8, device=dev)
+    h2d = sum(x.numel() * x.element_size() for x in pin)
+    d2h = o_h.numel() * 2 + l_h.numel() * 4 + (3 * o_h.numel() * 2 if has_bwd else 0)
+
+    def one():
+        for dst, src in zip((q, k, v) + ((do,) if has_bwd else ()), pin):
+            dst.copy_(src, non_blocking=True)
+        fa.forward(q, k, v, wl.scale, wl.causal, wl.window, out=o, lse=lse)
+        if has_bwd:
+            fa.backward(q, k, v, o, lse, do, wl.scale, wl.causal, wl.window, grads=grads, workspace=ws)
+        o_h.copy_(o, non_blocking=True)
+        l_h.copy_(lse, non_blocking=True)
+        if has_bwd:
+            for h, g in zip(grads_h, grads):
+                h.copy_(g, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / steps
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = t.item()
+    return {"value": round(world * flops / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 3)}
+
+
+def load_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it is for this kernel build."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+        return t.get(kernel)
+    except Exception:
+        return None
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from synthetic import WORKLOADS
+    wl = WORKLOADS[WORKLOAD]
+    import exact_io_aware_77_b200 as fa_pkg   # only to learn whether the path has a backward
+    with_bwd = hasattr(fa_pkg, "backward")
+    times, flops = [], []
+    for i in range(args.warmup + args.steps):
+        f, s, _, cores = oracle_sample(0.0, rows_per_block=128, with_bwd=with_bwd, max_blocks=1)
+        if i >= args.warmup:
+            times.append(s)
+            flops.append(f)
+    secs = sum(times)
+    value = sum(flops) / secs / 1e12
+    sample = (f"each step: 128 query rows of head 0 of the B2 H32 N4096 d128 causal workload through "
+              f"the fp64 oracle ({'fwd+bwd' if with_bwd else 'fwd'}), credited rows/N of a head's "
+              f"conventional FLOPs")
+    line = {
+        "metric": "attention fwd/bwd TFLOP/s at 1 B200; % of dense BF16 tensor peak",
+        "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * secs / args.steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": f"causal LLM shape {'forward+backward' if with_bwd else 'forward'}: "
+                               f"B={wl.B} H={wl.H} N={wl.N} d={wl.d} causal (row-block sample)",
+                   "global_batch": wl.B, "seq_len": wl.N, "parallelism": "cpu"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,95 @@
+"""ctypes binding of libfa_b200.so: the C-ABI entry points under the same names.
+
+Argument marshalling only -- every step of the attention path runs in the CUDA
+kernels behind these calls.  Loading fails loudly when the library has not been
+built; there is no fallback implementation.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa_b200.so")
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "fa.h")
+
+FA_OK = 0
+STATUS_NAMES = {
+    0: "FA_OK", 1: "FA_ERR_NULL", 2: "FA_ERR_SHAPE", 3: "FA_ERR_HEADDIM", 4: "FA_ERR_ALIGN",
+    5: "FA_ERR_MASK", 6: "FA_ERR_WORKSPACE", 7: "FA_ERR_CUDA", 8: "FA_ERR_DEVICE",
+    9: "FA_ERR_TIMEOUT", 10: "FA_ERR_SCALE",
+}
+STATUS = {v: k for k, v in STATUS_NAMES.items()}
+
+_c_int, _c_float, _c_void_p, _c_size_t = ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
+_c_ull = ctypes.c_ulonglong
+
+# name -> (restype, argtypes); mirrors include/fa.h
+SIGNATURES = {
+    "fa_fwd": (_c_int, [_c_void_p] * 5 + [_c_int] * 4 + [_c_float, _c_int, _c_int, _c_void_p]),
+    "fa_status_string": (ctypes.c_char_p, [_c_int]),
+    "fa_check_status": (_c_int, [_c_void_p]),
+    "fa_set_wait_limit_ns": (None, [_c_ull]),
+    "fa_selftest_timeout": (_c_int, [_c_ull, _c_void_p]),
+}
+
+
+class FAError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {STATUS_NAMES.get(status, status)} ({status_string(status)})")
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load the built library (raises if it is missing)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is not built; run `python -m exact_io_aware_77_b200.build` (needs nvcc)")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def header_symbols() -> list[str]:
+    """Every function include/fa.h declares (FA_EXPORT lines)."""
+    text = open(HEADER).read()
+    return re.findall(r"FA_EXPORT\s+[\w\s\*]+?\b(fa_\w+)\s*\(", text)
+
+
+def status_string(status: int) -> str:
+    return load().fa_status_string(int(status)).decode()
+
+
+def _call(name, *args) -> int:
+    return getattr(load(), name)(*args)
+
+
+def fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, window, stream) -> int:
+    return _call("fa_fwd", q, k, v, o, lse, B, H, N, d, scale, causal, window, stream)
+
+
+def fa_status_string(status: int) -> str:
+    return status_string(status)
+
+
+def fa_check_status(stream) -> int:
+    return _call("fa_check_status", stream)
+
+
+def fa_set_wait_limit_ns(limit_ns: int) -> None:
+    _call("fa_set_wait_limit_ns", limit_ns)
+
+
+def fa_selftest_timeout(limit_ns: int, stream) -> int:
+    return _call("fa_selftest_timeout", limit_ns, stream)

@@ -1,0 +1,189 @@
+// C ABI of the exact-attention library: argument validation, TMA tensor maps, launches
+// and the device status word.  The kernels are included here so that the whole library
+// is one translation unit (the status word needs no relocatable device code).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/fa.h"
+
+#include "fwd_kernel.cuh"
+
+namespace fa {
+namespace {
+
+constexpr unsigned long long kDefaultWaitLimitNs = 4000000000ull;
+unsigned long long g_wait_limit_ns = kDefaultWaitLimitNs;
+
+// ---------------------------------------------------------------- tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// [BH, rows, d] bf16 viewed as a 3-D tensor (d, rows, BH); box = 64 columns x box_rows rows
+// of one head, 128-byte swizzled.  Rows past the end of a head read as zero.
+bool make_map_bf16(CUtensorMap* map, const void* base, int d, int rows, int bh, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(rows), cuuint64_t(bh)};
+  cuuint64_t strides[2] = {cuuint64_t(d) * 2, cuuint64_t(d) * 2 * cuuint64_t(rows)};
+  cuuint32_t box[3] = {64, cuuint32_t(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------- validation
+constexpr int kMaxDevices = 64;
+
+int check_device() {
+  static int ok_cache[kMaxDevices] = {0};  // 0 unknown, 1 ok, 2 wrong device
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_DEVICE;
+  if (ok_cache[dev] == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return FA_ERR_CUDA;
+    ok_cache[dev] = (major == 10 && minor == 0) ? 1 : 2;
+  }
+  return ok_cache[dev] == 1 ? FA_OK : FA_ERR_DEVICE;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_problem(int B, int H, int N, int d, float scale, int causal, int window) {
+  if (B < 1 || H < 1 || N < 1) return FA_ERR_SHAPE;
+  const long long bh = (long long)B * H;
+  const long long tiles = (N + kBlockM - 1) / kBlockM;
+  if (bh > 0x7fffffffLL || bh * tiles > 0x7fffffffLL) return FA_ERR_SHAPE;
+  if (d != 64 && d != 128) return FA_ERR_HEADDIM;
+  if (!(causal == 0 || causal == 1) || window < 0 || (window > 0 && !causal)) return FA_ERR_MASK;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_SCALE;
+  return FA_OK;
+}
+
+template <class Kernel>
+int set_smem(Kernel k, int bytes) {
+  return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess ? FA_OK
+                                                                                                     : FA_ERR_CUDA;
+}
+
+template <int D>
+int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int BH, int N, float scale,
+               int causal, int window, cudaStream_t stream) {
+  CUtensorMap tq, tk, tv;
+  if (!make_map_bf16(&tq, q, D, N, BH, kBlockM) || !make_map_bf16(&tk, k, D, N, BH, kBlockN) ||
+      !make_map_bf16(&tv, v, D, N, BH, kBlockN))
+    return FA_ERR_CUDA;
+  FwdParams prm;
+  prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.lse = lse;
+  prm.N = N;
+  prm.BH = BH;
+  prm.n_q_tiles = (N + kBlockM - 1) / kBlockM;
+  prm.causal = causal;
+  prm.window = window;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.wait_limit_ns = g_wait_limit_ns;
+  // at least 120 KB so that one CTA (and its 512 TMEM columns) owns the SM
+  const int smem = int(sizeof(FwdSmem<D>)) + 1024 > 120 * 1024 ? int(sizeof(FwdSmem<D>)) + 1024 : 120 * 1024;
+  if (set_smem(fa_fwd_kernel<D>, smem) != FA_OK) return FA_ERR_CUDA;
+  const unsigned grid = unsigned(prm.n_q_tiles) * unsigned(BH);
+  fa_fwd_kernel<D><<<grid, kFwdThreads, smem, stream>>>(tq, tk, tv, prm);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- self-test kernel
+__global__ void selftest_timeout_kernel(unsigned long long limit_ns) {
+  __shared__ alignas(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(smem_u32(&bar), 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, &abort_flag, limit_ns);  // nothing ever arrives
+  __syncthreads();
+}
+
+}  // namespace
+}  // namespace fa
+
+using namespace fa;
+
+extern "C" {
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+           float scale, int causal, int window, void* stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
+  int st = check_problem(B, H, N, d, scale, causal, window);
+  if (st != FA_OK) return st;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+    return FA_ERR_ALIGN;
+  if ((st = check_device()) != FA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  return d == 64 ? launch_fwd<64>(q, k, v, o, lse, BH, N, scale, causal, window, s)
+                 : launch_fwd<128>(q, k, v, o, lse, BH, N, scale, causal, window, s);
+}
+
+const char* fa_status_string(int status) {
+  switch (status) {
+    case FA_OK: return "ok";
+    case FA_ERR_NULL: return "null pointer";
+    case FA_ERR_SHAPE: return "bad shape (B, H, N must be >= 1 and within launch limits)";
+    case FA_ERR_HEADDIM: return "unsupported head dimension (64 or 128)";
+    case FA_ERR_ALIGN: return "misaligned pointer (bf16 arrays 16 B, L 4 B)";
+    case FA_ERR_MASK: return "bad mask (causal 0/1, window >= 0, window needs causal)";
+    case FA_ERR_WORKSPACE: return "backward workspace missing or too small";
+    case FA_ERR_CUDA: return "CUDA runtime or launch error";
+    case FA_ERR_DEVICE: return "device is not compute capability 10.0 (B200)";
+    case FA_ERR_TIMEOUT: return "a kernel-side wait timed out";
+    case FA_ERR_SCALE: return "scale must be finite and > 0";
+    default: return "unknown status";
+  }
+}
+
+int fa_check_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
+  int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+  if (v != 0 && cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+  return v ? FA_ERR_TIMEOUT : FA_OK;
+}
+
+void fa_set_wait_limit_ns(unsigned long long limit_ns) {
+  g_wait_limit_ns = limit_ns ? limit_ns : kDefaultWaitLimitNs;
+}
+
+int fa_selftest_timeout(unsigned long long limit_ns, void* stream) {
+  int st = check_device();
+  if (st != FA_OK) return st;
+  if (limit_ns < 1000ull) limit_ns = 1000ull;
+  if (limit_ns > 1000000000ull) limit_ns = 1000000000ull;
+  selftest_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // extern "C"

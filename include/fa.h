@@ -1,0 +1,104 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) exact-attention library (libfa_b200.so).
+ *
+ * The library computes exact scaled-dot-product attention
+ *
+ *     O = softmax(scale * Q K^T + mask) V,      L_i = ln sum_j exp(scale * q_i . k_j + mask_ij)
+ *
+ * block by block with an online softmax, so the N x N score matrix never reaches
+ * device memory.  The formula is the one the FlashAttention pages print
+ * (FlashAttention (NL), "Problemen met standaard attention", with 1/sqrt(d_k) as the
+ * usual scale); the tiling, the online softmax (running row maximum and running sum of
+ * exponentials) and the single fused kernel are that page's "Tiling en blokgewijze
+ * verwerking", "Online berekening van Softmax" and "Samensmelting van bewerkingen in een
+ * CUDA-kernel"; the backward recomputes the probabilities from L instead of storing them
+ * (memory-optimized flash attention page, "How it works").
+ *
+ * Conventions shared by every entry point
+ *   Layout     Q, K, V, O, dO, dQ, dK, dV are contiguous bf16 arrays [B, H, N, d] (d fastest,
+ *              row stride d elements, head stride N*d); L is contiguous fp32 [B, H, N].
+ *              Self-attention: queries and keys have the same length N.
+ *   Pointers   every array argument is a DEVICE pointer of the current CUDA device; the
+ *              caller allocates, owns and frees all of them.  The library allocates no
+ *              device memory and keeps no pointer after a call returns.
+ *   Streams    `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *              Every call only enqueues work on that stream and returns; it never
+ *              synchronises (fa_check_status excepted).
+ *   Masks      causal = 1 keeps key j for query i iff j <= i.  window = W > 0 (needs
+ *              causal = 1) also requires j >= i - W + 1, so the band counts the diagonal
+ *              and W = 1 keeps only key i.  window = 0 means no band.  Keys j >= N never
+ *              exist.  Every query keeps its diagonal, so no row is empty.
+ *   Scale      applied inside: S = scale * Q K^T.  Must be finite and > 0.
+ *   Errors     arguments are validated before anything is enqueued; a rejected call
+ *              returns its FA_ERR_* code and touches no memory.  A failed launch returns
+ *              FA_ERR_CUDA.  Kernel-side waits are bounded: one that runs out records a
+ *              timeout in a device status word that fa_check_status() reports.
+ *   Device     a compute-capability 10.0 GPU (B200, sm_100a); others give FA_ERR_DEVICE.
+ */
+#ifndef FA_B200_H
+#define FA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FA_EXPORT __attribute__((visibility("default")))
+#else
+#define FA_EXPORT
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_NULL = 1,       /* a required pointer is NULL */
+  FA_ERR_SHAPE = 2,      /* B, H or N < 1, or the problem exceeds the launch limits */
+  FA_ERR_HEADDIM = 3,    /* d is not 64 or 128 */
+  FA_ERR_ALIGN = 4,      /* a bf16 array is not 16-byte aligned, or L not 4-byte aligned */
+  FA_ERR_MASK = 5,       /* causal not 0/1, window < 0, or window > 0 without causal */
+  FA_ERR_WORKSPACE = 6,  /* backward workspace missing or smaller than fa_bwd_workspace_size */
+  FA_ERR_CUDA = 7,       /* a CUDA runtime call or kernel launch failed */
+  FA_ERR_DEVICE = 8,     /* the current device is not compute capability 10.0 */
+  FA_ERR_TIMEOUT = 9,    /* a kernel-side wait ran out of time (reported by fa_check_status) */
+  FA_ERR_SCALE = 10      /* scale is not finite and > 0 */
+} fa_status;
+
+/*
+ * Forward pass.  Writes O (bf16 [B,H,N,d]) and L (fp32 [B,H,N], natural-log logsumexp of
+ * the masked, scaled scores of each query row).  Reads q, k, v (bf16 [B,H,N,d]).
+ * d must be 64 or 128.  Extra device memory: none beyond O and L.
+ */
+FA_EXPORT int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+           float scale, int causal, int window, void* stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+FA_EXPORT const char* fa_status_string(int status);
+
+/*
+ * Synchronises `stream`, then reads and clears the device status word of the current
+ * device.  Returns FA_ERR_TIMEOUT if any kernel since the last check gave up on a
+ * bounded wait, FA_ERR_CUDA if the synchronisation failed, FA_OK otherwise.
+ */
+FA_EXPORT int fa_check_status(void* stream);
+
+/*
+ * Time limit, in nanoseconds, of every kernel-side wait launched after this call
+ * (process-wide; default 4e9 = 4 s).  0 restores the default.
+ */
+FA_EXPORT void fa_set_wait_limit_ns(unsigned long long limit_ns);
+
+/*
+ * Failure-detection self-test: enqueues one small kernel that waits on a barrier nothing
+ * ever completes, under a limit of `limit_ns` nanoseconds (clamped to [1 us, 1 s]).  The
+ * wait runs out, the kernel records a timeout and exits, and the next fa_check_status()
+ * returns FA_ERR_TIMEOUT.  No memory is touched besides the status word.
+ */
+FA_EXPORT int fa_selftest_timeout(unsigned long long limit_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_H */

@@ -189,28 +189,31 @@ def _rows_mask(r: np.ndarray, n_k: int, causal: bool, window: int) -> np.ndarray
 
 
 def attention_backward_rows(q, k, v, do, scale: float, causal: bool = False, window: int = 0,
-                            key_rows=None, block: int = 512):
+                            key_rows=None, block: int = 512, query_rows=None):
     """Backward of ONE head for a subset of outputs, without an N x N buffer.
 
-    dQ is returned for every row; dK and dV only for ``key_rows`` (all if None).
-    It is the same chain rule as ``attention_backward`` evaluated over
-    full-width row blocks: each block of query rows contributes its part of
-    dK and dV = sum over rows of (dS^T Q, P^T dO).
+    dQ is returned for the query rows processed (all rows unless ``query_rows``
+    is given); dK and dV for ``key_rows`` (all if None).  It is the same chain
+    rule as ``attention_backward`` evaluated over full-width row blocks: each
+    block of query rows contributes its part of dK and dV (dS^T Q and P^T dO).
+    With ``query_rows`` the dK/dV returned are those rows' contributions only.
     """
     q, k, v, do = _as64(q), _as64(k), _as64(v), _as64(do)
     n = q.shape[0]
     key_rows = np.arange(n) if key_rows is None else np.asarray(key_rows, dtype=np.int64)
-    dq = np.empty_like(q)
+    qrows = np.arange(n) if query_rows is None else np.asarray(query_rows, dtype=np.int64)
+    dq = np.empty((qrows.size, q.shape[1]))
     dk = np.zeros((key_rows.size, q.shape[1]))
     dv = np.zeros((key_rows.size, q.shape[1]))
-    for b0 in range(0, n, block):
-        r = np.arange(b0, min(n, b0 + block))
+    for b0 in range(0, qrows.size, block):
+        sel = slice(b0, min(qrows.size, b0 + block))
+        r = qrows[sel]
         ok = _rows_mask(r, n, causal, window)
         p, _ = _softmax_rows(_scores(q[r], k, scale, ok))
         dp = do[r] @ v.T
         d_row = np.sum(p * dp, axis=1, keepdims=True)
         ds = p * (dp - d_row)
-        dq[r] = scale * (ds @ k)
+        dq[sel] = scale * (ds @ k)
         dk += scale * (ds[:, key_rows].T @ q[r])
         dv += p[:, key_rows].T @ do[r]
     return dq, dk, dv

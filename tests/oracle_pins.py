@@ -276,6 +276,15 @@ def row_blocks_match(orc):
                                                        key_rows=rows, block=5)
         assert np.max(np.abs(dq_r - dq)) < 1e-12
         assert np.max(np.abs(dk_r - dk[rows])) < 1e-12 and np.max(np.abs(dv_r - dv[rows])) < 1e-12
+        # disjoint query-row subsets: their dQ rows, and dK/dV contributions summing to the whole
+        parts = [np.arange(0, 20), np.arange(20, 41)]
+        acc_k, acc_v = 0.0, 0.0
+        for qr in parts:
+            dq_p, dk_p, dv_p = orc.attention_backward_rows(q, k, v, do, 0.3, causal, window,
+                                                           block=7, query_rows=qr)
+            assert np.max(np.abs(dq_p - dq[qr])) < 1e-12
+            acc_k, acc_v = acc_k + dk_p, acc_v + dv_p
+        assert np.max(np.abs(acc_k - dk)) < 1e-12 and np.max(np.abs(acc_v - dv)) < 1e-12
 
 
 def pair_count(orc):

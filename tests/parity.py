@@ -1,0 +1,49 @@
+"""Shared helpers of the GPU parity tests: tolerances and comparisons against the oracle.
+
+Tolerances (fixed for this method): bf16 O max-abs <= 2e-2 and mean-abs <= 2e-3;
+fp32 logsumexp max-abs <= 1e-3; gradients relative L2 <= 1e-2.  The GPU result is
+widened to fp64 and compared with the unrounded fp64 oracle.
+"""
+
+import numpy as np
+import torch
+
+O_MAX_ABS = 2e-2
+O_MEAN_ABS = 2e-3
+L_MAX_ABS = 1e-3
+GRAD_REL_L2 = 1e-2
+
+
+def to64(t) -> np.ndarray:
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def forward_errors(o_gpu, l_gpu, o_ref, l_ref) -> dict:
+    o_gpu, l_gpu = to64(o_gpu), to64(l_gpu)
+    assert np.all(np.isfinite(o_gpu)) and np.all(np.isfinite(l_gpu)), "non-finite output"
+    e = np.abs(o_gpu - o_ref)
+    return {"o_max": float(e.max()), "o_mean": float(e.mean()),
+            "l_max": float(np.abs(l_gpu - l_ref).max())}
+
+
+def assert_forward_close(o_gpu, l_gpu, o_ref, l_ref, what=""):
+    err = forward_errors(o_gpu, l_gpu, o_ref, l_ref)
+    assert err["o_max"] <= O_MAX_ABS, (what, err)
+    assert err["o_mean"] <= O_MEAN_ABS, (what, err)
+    assert err["l_max"] <= L_MAX_ABS, (what, err)
+    return err
+
+
+def rel_l2(a, ref) -> float:
+    a = to64(a) if isinstance(a, torch.Tensor) else a
+    return float(np.linalg.norm(a - ref) / max(np.linalg.norm(ref), 1e-30))
+
+
+def assert_grads_close(grads_gpu, grads_ref, what=""):
+    errs = {}
+    for name, g, r in zip(("dq", "dk", "dv"), grads_gpu, grads_ref):
+        gg = to64(g)
+        assert np.all(np.isfinite(gg)), (what, name, "non-finite")
+        errs[name] = rel_l2(gg, r)
+        assert errs[name] <= GRAD_REL_L2, (what, errs)
+    return errs

@@ -1,0 +1,65 @@
+"""The C-ABI library: it builds, loads, exports every declared symbol, and rejects bad
+arguments on the host before touching a device (no GPU needed for any of this)."""
+
+import ctypes
+
+import pytest
+
+from exact_io_aware_77_b200 import _lib
+from exact_io_aware_77_b200.build import build
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return _lib.load()
+
+
+def test_exports_every_header_symbol(lib):
+    names = _lib.header_symbols()
+    assert "fa_fwd" in names and "fa_check_status" in names
+    for name in names:
+        assert hasattr(lib, name), name
+        assert name in _lib.SIGNATURES, f"{name} has no ctypes signature"
+
+
+def test_status_strings(lib):
+    for code in _lib.STATUS_NAMES:
+        s = _lib.status_string(code)
+        assert s and s != "unknown status"
+    assert _lib.status_string(999) == "unknown status"
+
+
+A = 0x10000   # fake, 16-byte-aligned addresses: validation must fail before any use
+GOOD = dict(B=1, H=2, N=128, d=64, scale=0.125, causal=0, window=0)
+
+
+def _fwd(**kw):
+    a = dict(GOOD)
+    ptrs = kw.pop("ptrs", [A, A + 4096, A + 8192, A + 12288, A + 16384])
+    a.update(kw)
+    return _lib.fa_fwd(*ptrs, a["B"], a["H"], a["N"], a["d"], a["scale"], a["causal"], a["window"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(ptrs=[0, A, A, A, A]), "FA_ERR_NULL"),
+    (dict(ptrs=[A, A, A, A, 0]), "FA_ERR_NULL"),
+    (dict(B=0), "FA_ERR_SHAPE"),
+    (dict(H=-1), "FA_ERR_SHAPE"),
+    (dict(N=0), "FA_ERR_SHAPE"),
+    (dict(B=1 << 20, H=1 << 20), "FA_ERR_SHAPE"),
+    (dict(d=96), "FA_ERR_HEADDIM"),
+    (dict(d=256), "FA_ERR_HEADDIM"),
+    (dict(window=-1, causal=1), "FA_ERR_MASK"),
+    (dict(window=4, causal=0), "FA_ERR_MASK"),
+    (dict(causal=2), "FA_ERR_MASK"),
+    (dict(scale=0.0), "FA_ERR_SCALE"),
+    (dict(scale=-1.0), "FA_ERR_SCALE"),
+    (dict(scale=float("inf")), "FA_ERR_SCALE"),
+    (dict(scale=float("nan")), "FA_ERR_SCALE"),
+    (dict(ptrs=[A + 8, A, A, A, A]), "FA_ERR_ALIGN"),
+    (dict(ptrs=[A, A, A, A + 2, A]), "FA_ERR_ALIGN"),
+    (dict(ptrs=[A, A, A, A, A + 2]), "FA_ERR_ALIGN"),
+])
+def test_fwd_rejects_bad_arguments(lib, kw, code):
+    assert _lib.STATUS_NAMES[_fwd(**kw)] == code
