@@ -52,11 +52,15 @@ def test_small_shapes_elementwise(fa, B, H, N, d, causal, window):
 
 
 def test_large_magnitude_scores(fa):
-    """Scores up to ~±90 (log2 domain ~130): the running max keeps exp in range."""
+    """Q, K with std 3 give scores of std 9 (peaked rows, |S| up to ~40): the running max
+    keeps exp2 in range.  V stays N(0, 1) so |O| stays where the absolute bf16 bound applies."""
     wl = Workload("big", 1, 2, 384, 128, True, 0, std=3.0, seed=99)
-    (q, k, v), o, lse = _run(fa, wl)
+    q, k, _ = make_inputs(wl)
+    v = make_inputs(wl.with_(std=1.0), seed=100)[2]
+    o, lse = fa.forward(q.cuda(), k.cuda(), v.cuda(), wl.scale, True, 0)
+    assert fa.check_status() == 0
     o_ref, l_ref = orc.attention_forward(q, k, v, wl.scale, True, 0)
-    assert_forward_close(o, lse, o_ref, l_ref, "std=3")
+    assert_forward_close(o.cpu(), lse.cpu(), o_ref, l_ref, "qk std=3")
 
 
 def test_tiny_scale(fa):
