@@ -12,7 +12,7 @@ import math
 from . import _lib
 from ._lib import FAError, STATUS, STATUS_NAMES, load
 
-__all__ = ["forward", "check_status", "FAError", "STATUS", "STATUS_NAMES", "load", "default_scale"]
+__all__ = ["forward", "backward", "bwd_workspace_size", "check_status", "FAError", "STATUS", "STATUS_NAMES", "load", "default_scale"]
 
 
 def default_scale(d: int) -> float:
@@ -55,6 +55,37 @@ def forward(q, k, v, scale: float | None = None, causal: bool = False, window: i
                      B, H, N, d, scale, int(bool(causal)), int(window), _stream_handle(q.device))
     _raise("fa_fwd", st)
     return out, lse
+
+
+def bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
+    """Bytes of scratch device memory backward() needs (O(N*d))."""
+    n = _lib.fa_bwd_workspace_size(B, H, N, d)
+    if n == 0:
+        raise ValueError("invalid shape")
+    return n
+
+
+def backward(q, k, v, o, lse, do, scale: float | None = None, causal: bool = False, window: int = 0,
+             grads=None, workspace=None):
+    """dQ, dK, dV (bf16 [B,H,N,d]) of sum(O o dO), recomputing P from the forward's L."""
+    import torch
+    _check_qkv(q, k, v, o, do)
+    B, H, N, d = q.shape
+    if not (lse.is_cuda and lse.dtype == torch.float32 and lse.is_contiguous() and lse.numel() == B * H * N):
+        raise ValueError("lse must be a contiguous fp32 CUDA tensor of B*H*N elements")
+    scale = default_scale(d) if scale is None else float(scale)
+    if grads is None:
+        grads = (torch.empty_like(q), torch.empty_like(q), torch.empty_like(q))
+    need = bwd_workspace_size(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    dq, dk, dv = grads
+    st = _lib.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                     do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, scale,
+                     int(bool(causal)), int(window), workspace.data_ptr(),
+                     workspace.numel() * workspace.element_size(), _stream_handle(q.device))
+    _raise("fa_bwd", st)
+    return dq, dk, dv
 
 
 def check_status(device=None) -> int:

@@ -28,6 +28,9 @@ _c_ull = ctypes.c_ulonglong
 # name -> (restype, argtypes); mirrors include/fa.h
 SIGNATURES = {
     "fa_fwd": (_c_int, [_c_void_p] * 5 + [_c_int] * 4 + [_c_float, _c_int, _c_int, _c_void_p]),
+    "fa_bwd_workspace_size": (_c_size_t, [_c_int] * 4),
+    "fa_bwd": (_c_int, [_c_void_p] * 9 + [_c_int] * 4 + [_c_float, _c_int, _c_int, _c_void_p, _c_size_t,
+                                                         _c_void_p]),
     "fa_status_string": (ctypes.c_char_p, [_c_int]),
     "fa_check_status": (_c_int, [_c_void_p]),
     "fa_set_wait_limit_ns": (None, [_c_ull]),
@@ -77,6 +80,16 @@ def _call(name, *args) -> int:
 
 def fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, window, stream) -> int:
     return _call("fa_fwd", q, k, v, o, lse, B, H, N, d, scale, causal, window, stream)
+
+
+def fa_bwd_workspace_size(B, H, N, d) -> int:
+    return _call("fa_bwd_workspace_size", B, H, N, d)
+
+
+def fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal, window, workspace,
+           workspace_bytes, stream) -> int:
+    return _call("fa_bwd", q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal, window,
+                 workspace, workspace_bytes, stream)
 
 
 def fa_status_string(status: int) -> str:

@@ -12,6 +12,7 @@
 #include "../../include/fa.h"
 
 #include "fwd_kernel.cuh"
+#include "bwd_kernel.cuh"
 
 namespace fa {
 namespace {
@@ -113,6 +114,63 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------- backward
+long long padded_rows(int N) { return ((long long)N + kBwdRows - 1) / kBwdRows * kBwdRows; }
+
+size_t bwd_workspace_bytes(long long BH, int N, int d) {
+  return size_t(4) * size_t(BH) * size_t(padded_rows(N)) * size_t(2 + d);
+}
+
+template <int D>
+int launch_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+               void* dq, void* dk, void* dv, int BH, int N, float scale, int causal, int window, void* ws,
+               cudaStream_t stream) {
+  const long long Np = padded_rows(N);
+  float* lp = static_cast<float*>(ws);
+  float* dd = lp + size_t(BH) * Np;
+  float* dq_acc = dd + size_t(BH) * Np;
+  constexpr int G = D / 8;
+  {
+    const long long rows = (long long)BH * Np;
+    const long long blocks = (rows + (256 / G) - 1) / (256 / G);
+    fa_bwd_prep<D><<<unsigned(blocks), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, lp, dd, dq_acc, N,
+        int(Np), rows);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_map_bf16(&tq, q, D, N, BH, kBwdRows) || !make_map_bf16(&tk, k, D, N, BH, kBwdKeys) ||
+      !make_map_bf16(&tv, v, D, N, BH, kBwdKeys) || !make_map_bf16(&tdo, dout, D, N, BH, kBwdRows))
+    return FA_ERR_CUDA;
+  BwdParams prm;
+  prm.lp = lp;
+  prm.dd = dd;
+  prm.dq_acc = dq_acc;
+  prm.dk = static_cast<__nv_bfloat16*>(dk);
+  prm.dv = static_cast<__nv_bfloat16*>(dv);
+  prm.N = N;
+  prm.Np = int(Np);
+  prm.BH = BH;
+  prm.n_kv_tiles = (N + kBwdKeys - 1) / kBwdKeys;
+  prm.causal = causal;
+  prm.window = window;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.scale = scale;
+  prm.wait_limit_ns = g_wait_limit_ns;
+  const int smem = int(sizeof(BwdSmem<D>)) + 1024;
+  if (set_smem(fa_bwd_kernel<D>, smem) != FA_OK) return FA_ERR_CUDA;
+  fa_bwd_kernel<D><<<unsigned(prm.n_kv_tiles) * unsigned(BH), kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, prm);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  {
+    const long long rows = (long long)BH * N;
+    const long long blocks = (rows + (256 / G) - 1) / (256 / G);
+    fa_bwd_dq_final<D><<<unsigned(blocks), 256, 0, stream>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), N, int(Np),
+                                                             scale, rows);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
+
 // ---------------------------------------------------------------- self-test kernel
 __global__ void selftest_timeout_kernel(unsigned long long limit_ns) {
   __shared__ alignas(8) uint64_t bar;
@@ -146,6 +204,30 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   const int BH = B * H;
   return d == 64 ? launch_fwd<64>(q, k, v, o, lse, BH, N, scale, causal, window, s)
                  : launch_fwd<128>(q, k, v, o, lse, BH, N, scale, causal, window, s);
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
+  if (check_problem(B, H, N, d, 1.f, 0, 0) != FA_OK) return 0;
+  return bwd_workspace_bytes((long long)B * H, N, d);
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout, void* dq,
+           void* dk, void* dv, int B, int H, int N, int d, float scale, int causal, int window, void* workspace,
+           size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FA_ERR_NULL;
+  int st = check_problem(B, H, N, d, scale, causal, window);
+  if (st != FA_OK) return st;
+  const long long BH = (long long)B * H;
+  if (BH * ((N + kBwdKeys - 1) / kBwdKeys) > 0x7fffffffLL || BH * padded_rows(N) > 0x7fffffffLL) return FA_ERR_SHAPE;
+  if (!workspace || workspace_bytes < bwd_workspace_bytes(BH, N, d)) return FA_ERR_WORKSPACE;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dout, 16) ||
+      !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4) || !aligned(workspace, 16))
+    return FA_ERR_ALIGN;
+  if ((st = check_device()) != FA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, int(BH), N, scale, causal, window, workspace, s)
+                 : launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, int(BH), N, scale, causal, window, workspace,
+                                   s);
 }
 
 const char* fa_status_string(int status) {

@@ -73,6 +73,26 @@ typedef enum {
 FA_EXPORT int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
            float scale, int causal, int window, void* stream);
 
+/*
+ * Bytes of device workspace fa_bwd needs: 4 * B*H * Np * (d + 2) with Np = N rounded up to
+ * a multiple of 64 (per row: D, L in log2 units, and a d-wide fp32 dQ accumulator).
+ * Returns 0 when the shape itself is invalid.  O(N * d): no N x N buffer.
+ */
+FA_EXPORT size_t fa_bwd_workspace_size(int B, int H, int N, int d);
+
+/*
+ * Backward pass with recomputation.  From q, k, v, the forward's o and lse, and the output
+ * gradient dO (bf16 [B,H,N,d]) it writes dQ, dK, dV (bf16 [B,H,N,d]): the gradients of
+ * sum(O o dO).  Same mask, scale and shape arguments as the forward that produced o and lse.
+ * `workspace` (device, caller-owned, 16-byte aligned, at least fa_bwd_workspace_size bytes)
+ * is scratch: it is overwritten and may be reused once the call's work has completed on
+ * `stream`.  Three kernels are enqueued: D = rowsum(dO o O) with a cleared accumulator, the
+ * fused recompute kernel, and the dQ scaling.
+ */
+FA_EXPORT int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                     void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal, int window,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 FA_EXPORT const char* fa_status_string(int status);
 

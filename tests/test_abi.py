@@ -63,3 +63,36 @@ def _fwd(**kw):
 ])
 def test_fwd_rejects_bad_arguments(lib, kw, code):
     assert _lib.STATUS_NAMES[_fwd(**kw)] == code
+
+
+def _bwd(ws_bytes=1 << 30, **kw):
+    a = dict(GOOD)
+    ptrs = kw.pop("ptrs", [A + 4096 * i for i in range(9)])
+    ws = kw.pop("ws", A + 65536)
+    a.update(kw)
+    return _lib.fa_bwd(*ptrs, a["B"], a["H"], a["N"], a["d"], a["scale"], a["causal"], a["window"],
+                       ws, ws_bytes, None)
+
+
+def test_workspace_size_formula(lib):
+    for B, H, N, d in ((1, 1, 1, 64), (2, 32, 4096, 128), (1, 16, 32768, 128), (3, 5, 65, 64)):
+        np_ = (N + 63) // 64 * 64
+        assert _lib.fa_bwd_workspace_size(B, H, N, d) == 4 * B * H * np_ * (d + 2)
+    assert _lib.fa_bwd_workspace_size(1, 1, 0, 64) == 0
+    assert _lib.fa_bwd_workspace_size(1, 1, 16, 80) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(ptrs=[A] * 8 + [0]), "FA_ERR_NULL"),
+    (dict(ptrs=[0] + [A] * 8), "FA_ERR_NULL"),
+    (dict(N=0), "FA_ERR_SHAPE"),
+    (dict(d=32), "FA_ERR_HEADDIM"),
+    (dict(window=3), "FA_ERR_MASK"),
+    (dict(scale=0.0), "FA_ERR_SCALE"),
+    (dict(ws=0), "FA_ERR_WORKSPACE"),
+    (dict(ws_bytes=100), "FA_ERR_WORKSPACE"),
+    (dict(ws=A + 8), "FA_ERR_ALIGN"),
+    (dict(ptrs=[A] * 5 + [A + 2] + [A] * 3), "FA_ERR_ALIGN"),
+])
+def test_bwd_rejects_bad_arguments(lib, kw, code):
+    assert _lib.STATUS_NAMES[_bwd(**kw)] == code

@@ -22,6 +22,7 @@ def fa():
     build()
     import exact_io_aware_77_b200 as fa
     fa.load()
+    fa._lib.fa_set_wait_limit_ns(1_000_000_000)   # a correct pipeline never waits this long
     return fa
 
 
