@@ -34,9 +34,19 @@ def assert_forward_close(o_gpu, l_gpu, o_ref, l_ref, what=""):
     return err
 
 
+GRAD_RMS_FLOOR = 1e-3
+
+
 def rel_l2(a, ref) -> float:
+    """||a - ref|| / max(||ref||, 1e-3 * sqrt(n)).
+
+    The floor matters only for gradients that are zero by the mathematics (a window of 1
+    makes dS, hence dQ and dK, exactly 0); there the relative error has no meaning and the
+    check becomes an absolute RMS error of at most 1e-5 per element.
+    """
     a = to64(a) if isinstance(a, torch.Tensor) else a
-    return float(np.linalg.norm(a - ref) / max(np.linalg.norm(ref), 1e-30))
+    floor = GRAD_RMS_FLOOR * np.sqrt(ref.size)
+    return float(np.linalg.norm(a - ref) / max(np.linalg.norm(ref), floor))
 
 
 def assert_grads_close(grads_gpu, grads_ref, what=""):
