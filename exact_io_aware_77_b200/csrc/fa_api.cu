@@ -171,6 +171,28 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   return FA_OK;
 }
 
+// ---------------------------------------------------------------- backward without caller memory
+// Built-in scratch for fa_bwd_noalloc.  It lives in the module's global memory, so every GPU
+// that loads this library holds these 64 MiB until the process exits.  Host code must not
+// use the array's name as a device address (on the host it is only a stand-in); the device
+// address comes from cudaGetSymbolAddress, looked up once per device.
+constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch on the current device (nullptr on failure).  Called
+// with the device already current; the first call on a device does the lookup.
+void* noalloc_scratch(int dev) {
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {nullptr};
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return nullptr;
+    addr[dev] = p;
+  }
+  return addr[dev];
+}
+
 // ---------------------------------------------------------------- self-test kernel
 __global__ void selftest_timeout_kernel(unsigned long long limit_ns) {
   __shared__ alignas(8) uint64_t bar;
@@ -243,6 +265,7 @@ const char* fa_status_string(int status) {
     case FA_ERR_DEVICE: return "device is not compute capability 10.0 (B200)";
     case FA_ERR_TIMEOUT: return "a kernel-side wait timed out";
     case FA_ERR_SCALE: return "scale must be finite and > 0";
+    case FA_ERR_NOALLOC_LIMIT: return "problem needs more than the 64 MiB built-in scratch of fa_bwd_noalloc";
     default: return "unknown status";
   }
 }
@@ -266,6 +289,30 @@ int fa_selftest_timeout(unsigned long long limit_ns, void* stream) {
   if (limit_ns > 1000000000ull) limit_ns = 1000000000ull;
   selftest_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                   void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal, int window,
+                   void* stream) {
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FA_ERR_NULL;
+  int st = check_problem(B, H, N, d, scale, causal, window);
+  if (st != FA_OK) return st;
+  const long long BH = (long long)B * H;
+  if (BH * ((N + kBwdKeys - 1) / kBwdKeys) > 0x7fffffffLL || BH * padded_rows(N) > 0x7fffffffLL) return FA_ERR_SHAPE;
+  if (bwd_workspace_bytes(BH, N, d) > kNoAllocScratchBytes) return FA_ERR_NOALLOC_LIMIT;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dout, 16) ||
+      !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4))
+    return FA_ERR_ALIGN;
+  if ((st = check_device()) != FA_OK) return st;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  void* ws = noalloc_scratch(dev);
+  if (ws == nullptr) return FA_ERR_CUDA;
+  // every byte of the scratch the kernels read is rewritten first by fa_bwd_prep (D, L and a
+  // zeroed dQ accumulator), so what an earlier call left there does not leak in
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, int(BH), N, scale, causal, window, ws, s)
+                 : launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, int(BH), N, scale, causal, window, ws, s);
 }
 
 }  // extern "C"

@@ -62,7 +62,8 @@ typedef enum {
   FA_ERR_CUDA = 7,       /* a CUDA runtime call or kernel launch failed */
   FA_ERR_DEVICE = 8,     /* the current device is not compute capability 10.0 */
   FA_ERR_TIMEOUT = 9,    /* a kernel-side wait ran out of time (reported by fa_check_status) */
-  FA_ERR_SCALE = 10      /* scale is not finite and > 0 */
+  FA_ERR_SCALE = 10,     /* scale is not finite and > 0 */
+  FA_ERR_NOALLOC_LIMIT = 11 /* fa_bwd_noalloc: fa_bwd_workspace_size(...) exceeds its 64 MiB scratch */
 } fa_status;
 
 /*
@@ -116,6 +117,31 @@ FA_EXPORT void fa_set_wait_limit_ns(unsigned long long limit_ns);
  * returns FA_ERR_TIMEOUT.  No memory is touched besides the status word.
  */
 FA_EXPORT int fa_selftest_timeout(unsigned long long limit_ns, void* stream);
+
+/*
+ * Backward pass for callers that cannot allocate device memory.  The FlashAttention pages
+ * have no counterpart of this entry point; it exists for code that may not call cudaMalloc
+ * and has no allocator to ask: for example an operator running as a plugin inside a host
+ * framework that owns all device memory, or a latency-critical service that forbids
+ * allocation (which can synchronise the device) once it has started.
+ *
+ * Same arguments and results as fa_bwd, without the workspace: the scratch (D, L and the
+ * fp32 dQ accumulator) lives in one 64 MiB array inside the library, which every GPU that
+ * loads the library holds until the process exits.  Problems whose
+ * fa_bwd_workspace_size(B, H, N, d) exceeds 64 MiB (67108864 bytes) are rejected with
+ * FA_ERR_NOALLOC_LIMIT before anything is enqueued; for d = 128 that allows
+ * B*H*ceil(N/64)*64 <= 129055 rows, e.g. 31 heads of N = 4096.
+ *
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress,
+ * with that device current), so make that first call before any stream capture begins.
+ * The call itself allocates nothing (no cudaMalloc, cudaFree or allocating library call);
+ * every scratch byte the kernels read is rewritten at the start of each call.  All calls
+ * share the one array: two calls whose work overlaps on the GPU (different streams, or
+ * several host threads) race on it and give wrong results -- serialise them.
+ */
+FA_EXPORT int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                             const void* dO, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                             float scale, int causal, int window, void* stream);
 
 #ifdef __cplusplus
 }
