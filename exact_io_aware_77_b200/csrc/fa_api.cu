@@ -101,7 +101,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   prm.lse = lse;
   prm.N = N;
   prm.BH = BH;
-  prm.n_q_tiles = (N + kBlockM - 1) / kBlockM;
+  prm.n_pairs = ((N + kBlockM - 1) / kBlockM + kQTiles - 1) / kQTiles;
   prm.causal = causal;
   prm.window = window;
   prm.scale_log2 = scale * 1.4426950408889634f;
@@ -109,7 +109,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   // at least 120 KB so that one CTA (and its 512 TMEM columns) owns the SM
   const int smem = int(sizeof(FwdSmem<D>)) + 1024 > 120 * 1024 ? int(sizeof(FwdSmem<D>)) + 1024 : 120 * 1024;
   if (set_smem(fa_fwd_kernel<D>, smem) != FA_OK) return FA_ERR_CUDA;
-  const unsigned grid = unsigned(prm.n_q_tiles) * unsigned(BH);
+  const unsigned grid = unsigned(prm.n_pairs) * unsigned(BH);
   fa_fwd_kernel<D><<<grid, kFwdThreads, smem, stream>>>(tq, tk, tv, prm);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }

@@ -9,35 +9,47 @@
 // final result (same page, "Samensmelting van bewerkingen in een CUDA-kernel").  The
 // N x N score matrix never leaves the SM.
 //
-// sm_100a mapping (one CTA per 128-row query tile of one head):
-//   warp 4      TMA producer: Q tile once, then K_j / V_j tiles into 2-stage rings.
-//   warp 5      MMA issuer:   S_j = Q K_j^T into TMEM (double-buffered), O += P_j V_j in TMEM.
-//   warps 0-3   softmax:      thread t owns query row t = TMEM lane t; reads S_j with
-//                              tcgen05.ld, applies scale/mask, updates the running max m and
-//                              sum l, writes P_j (bf16) to shared memory, rescales O in TMEM
-//                              when m grows, and finally writes O / l and L.
-// TMEM columns: [0,128) S buffer 0, [128,256) S buffer 1, [256, 256 + D) O accumulator.
+// sm_100a mapping: one CTA per pair of adjacent 128-row query tiles of one head, so every
+// K/V tile brought on chip serves 256 query rows.
+//   warp 8      TMA producer: both Q tiles once, then K_j, V_j through a 4-slot ring.
+//   warp 9      MMA issuer (one thread), in the order
+//                 PV0(j), S0(j+1), PV1(j), S1(j+1)
+//               so the tensor pipe computes one tile's products while the other tile's
+//               softmax runs (ping-pong).  S = Q K^T lands in TMEM; P is written back over
+//               the consumed S columns as bf16 and O += P V reads it from TMEM.
+//   warps 0-3   softmax of query tile 0, warps 4-7 of tile 1: thread t owns row t (TMEM
+//               lane t).  Each tile: tcgen05.ld S, scale and mask, running max m and sum l,
+//               P = exp2(S c - m) packed to bf16 and stored to TMEM, then the epilogue
+//               O / l -> bf16 and L = (m + log2 l) ln 2.
+// The running max is updated lazily: O in TMEM is rescaled only when a row's max grows by
+// more than 2^8; otherwise the stale max keeps being used (P <= 256, exact after the final
+// division by l).  Because S(j) is issued after PV(j-1) and tcgen05 MMAs of one thread run in
+// order, S(j) completing means PV(j-1) has completed, so a rescale never races an MMA and the
+// softmax warps never wait on P V.
+// TMEM columns: S0 [0,128), S1 [128,256), O0 [256, 256+D), O1 [384, 384+D); P_w occupies
+// the first 64 columns of S_w.
 #pragma once
 
 #include "sm100.cuh"
 
 namespace fa {
 
-constexpr int kBlockM = 128;   // query rows per CTA
+constexpr int kBlockM = 128;   // query rows per tile (one per TMEM lane)
 constexpr int kBlockN = 128;   // keys per KV tile
-constexpr int kStages = 2;     // K/V shared-memory ring depth
-constexpr int kFwdThreads = 192;
-constexpr int kWarpTma = 4;
-constexpr int kWarpMma = 5;
+constexpr int kQTiles = 2;     // query tiles per CTA
+constexpr int kSlots = 4;      // K/V shared-memory ring slots (K and V alternate)
+constexpr int kFwdThreads = 320;
+constexpr int kWarpTma = 8;
+constexpr int kWarpMma = 9;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemO = 256;
+constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only when m grows by > 2^8
 
 struct FwdParams {
   __nv_bfloat16* o;   // [BH, N, D]
   float* lse;         // [BH, N]
   int N;
   int BH;
-  int n_q_tiles;
+  int n_pairs;        // ceil(ceil(N / 128) / 2)
   int causal;
   int window;
   float scale_log2;   // scale * log2(e)
@@ -46,24 +58,25 @@ struct FwdParams {
 
 template <int D>
 struct FwdSmem {
-  static constexpr int kChunks = D / 64;                 // 64-element (128-byte) column chunks
+  static constexpr int kChunks = D / 64;                   // 64-element (128-byte) column chunks
   static constexpr uint32_t kTileBytes = kBlockN * D * 2;  // one Q, K or V tile
-  alignas(1024) uint8_t q[kBlockM * D * 2];
-  alignas(1024) uint8_t k[kStages][kTileBytes];
-  alignas(1024) uint8_t v[kStages][kTileBytes];
-  alignas(1024) uint8_t p[kBlockM * kBlockN * 2];
+  alignas(1024) uint8_t q[kQTiles][kTileBytes];
+  alignas(1024) uint8_t kv[kSlots][kTileBytes];
   alignas(8) uint64_t q_full;
-  uint64_t k_full[kStages], k_empty[kStages];
-  uint64_t v_full[kStages], v_empty[kStages];
-  uint64_t s_full[2], s_empty[2];
-  uint64_t p_full, o_done, mma_drain;
+  uint64_t slot_full[kSlots], slot_empty[kSlots];
+  uint64_t s_full[kQTiles], p_full[kQTiles], o_final[kQTiles];
+  uint64_t mma_drain;
   uint32_t tmem_base;
   int abort;
 };
 
-// Range of KV tiles a query tile needs: causal stops at the diagonal, a window starts at
-// the first tile that holds key q0 - W + 1.
+// KV tiles [t_begin, t_end) one query tile starting at q0 needs: causal stops at the diagonal,
+// a window starts at the tile holding key q0 - W + 1.  Empty when the tile is past N.
 __device__ __forceinline__ void kv_tile_range(int q0, int N, int causal, int window, int& t_begin, int& t_end) {
+  if (q0 >= N) {
+    t_begin = t_end = 0;
+    return;
+  }
   const int kv_end = causal ? min(N, q0 + kBlockM) : N;
   t_end = (kv_end + kBlockN - 1) / kBlockN;
   const int kv_begin = window > 0 ? max(0, q0 - window + 1) : 0;
@@ -80,30 +93,31 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int q_tile = prm.n_q_tiles - 1 - int(blockIdx.x / prm.BH);   // longest causal tiles first
-  const int bh = int(blockIdx.x % prm.BH);
-  const int q0 = q_tile * kBlockM;
-  int t_begin, t_end;
-  kv_tile_range(q0, prm.N, prm.causal, prm.window, t_begin, t_end);
-  const int n_tiles = t_end - t_begin;   // >= 1: the diagonal tile is always needed
+  // head-major order keeps a head's K/V hot in L2; longest causal pairs first within a head
+  const int bh = int(blockIdx.x / prm.n_pairs);
+  const int pair = prm.n_pairs - 1 - int(blockIdx.x % prm.n_pairs);
+  const int q0 = pair * (kQTiles * kBlockM);
+  int b0, e0, b1, e1;
+  kv_tile_range(q0, prm.N, prm.causal, prm.window, b0, e0);
+  kv_tile_range(q0 + kBlockM, prm.N, prm.causal, prm.window, b1, e1);
+  if (e1 == 0) b1 = e1 = b0;   // second tile entirely past N: no work for it
+  const int t_begin = b0;       // b1 >= b0 and e1 >= e0 whenever tile 1 has work
+  const int t_end = max(e0, e1);
   volatile int* abort = &sm.abort;
   const uint64_t lim = prm.wait_limit_ns;
 
   if (threadIdx.x == 0) {
     sm.abort = 0;
     mbar_init(smem_u32(&sm.q_full), 1);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(smem_u32(&sm.k_full[s]), 1);
-      mbar_init(smem_u32(&sm.k_empty[s]), 1);
-      mbar_init(smem_u32(&sm.v_full[s]), 1);
-      mbar_init(smem_u32(&sm.v_empty[s]), 1);
+    for (int s = 0; s < kSlots; ++s) {
+      mbar_init(smem_u32(&sm.slot_full[s]), 1);
+      mbar_init(smem_u32(&sm.slot_empty[s]), 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(smem_u32(&sm.s_full[b]), 1);
-      mbar_init(smem_u32(&sm.s_empty[b]), kBlockM);
+    for (int w = 0; w < kQTiles; ++w) {
+      mbar_init(smem_u32(&sm.s_full[w]), 1);
+      mbar_init(smem_u32(&sm.p_full[w]), kBlockM);
+      mbar_init(smem_u32(&sm.o_final[w]), 1);
     }
-    mbar_init(smem_u32(&sm.p_full), kBlockM);
-    mbar_init(smem_u32(&sm.o_done), 1);
     mbar_init(smem_u32(&sm.mma_drain), 1);
     fence_mbar_init();
   }
@@ -125,101 +139,120 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       const uint32_t qb = smem_u32(&sm.q_full);
-      int k_issued = 0, v_issued = 0;
-      mbar_expect_tx(qb, Smem::kTileBytes);
-      for (int c = 0; c < Smem::kChunks; ++c)
-        tma_load_3d(smem_u32(sm.q) + c * 16384, &tm_q, qb, c * 64, q0, bh);
-      for (int t = 0; t < n_tiles; ++t) {
-        const int s = t & 1;
-        const uint32_t ph = (t >> 1) & 1;
-        const int kv0 = (t_begin + t) * kBlockN;
-        if (!mbar_wait(smem_u32(&sm.k_empty[s]), ph ^ 1, abort, lim)) break;
-        const uint32_t kb = smem_u32(&sm.k_full[s]);
-        mbar_expect_tx(kb, Smem::kTileBytes);
+      mbar_expect_tx(qb, kQTiles * Smem::kTileBytes);
+      for (int w = 0; w < kQTiles; ++w)
         for (int c = 0; c < Smem::kChunks; ++c)
-          tma_load_3d(smem_u32(sm.k[s]) + c * 16384, &tm_k, kb, c * 64, kv0, bh);
-        k_issued = t + 1;
-        if (!mbar_wait(smem_u32(&sm.v_empty[s]), ph ^ 1, abort, lim)) break;
-        const uint32_t vb = smem_u32(&sm.v_full[s]);
-        mbar_expect_tx(vb, Smem::kTileBytes);
-        for (int c = 0; c < Smem::kChunks; ++c)
-          tma_load_3d(smem_u32(sm.v[s]) + c * 16384, &tm_v, vb, c * 64, kv0, bh);
-        v_issued = t + 1;
+          tma_load_3d(smem_u32(sm.q[w]) + c * 16384, &tm_q, qb, c * 64, q0 + w * kBlockM, bh);
+      int issued = 0;   // loads issued: K_t is load 2(t - t_begin), V_t the next one
+      const int n_loads = 2 * (t_end - t_begin);
+      for (int L = 0; L < n_loads; ++L) {
+        const int slot = L % kSlots;
+        if (!mbar_wait(smem_u32(&sm.slot_empty[slot]), ((L / kSlots) & 1) ^ 1, abort, lim)) break;
+        const uint32_t fb = smem_u32(&sm.slot_full[slot]);
+        const int kv0 = (t_begin + (L >> 1)) * kBlockN;
+        const CUtensorMap* map = (L & 1) ? &tm_v : &tm_k;
+        mbar_expect_tx(fb, Smem::kTileBytes);
+        for (int c = 0; c < Smem::kChunks; ++c) tma_load_3d(smem_u32(sm.kv[slot]) + c * 16384, map, fb, c * 64, kv0, bh);
+        issued = L + 1;
       }
-      // Let every copy this CTA started land before the CTA can exit (matters only when
-      // aborting; on the normal path each one has been consumed already).
+      // let every copy this CTA started land before the CTA may exit
       mbar_wait_drain(qb, 0, lim);
-      for (int t = max(0, k_issued - kStages); t < k_issued; ++t)
-        mbar_wait_drain(smem_u32(&sm.k_full[t & 1]), (t >> 1) & 1, lim);
-      for (int t = max(0, v_issued - kStages); t < v_issued; ++t)
-        mbar_wait_drain(smem_u32(&sm.v_full[t & 1]), (t >> 1) & 1, lim);
+      for (int L = max(0, issued - kSlots); L < issued; ++L)
+        mbar_wait_drain(smem_u32(&sm.slot_full[L % kSlots]), (L / kSlots) & 1, lim);
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(kBlockM, kBlockN, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(kBlockM, D, false, true);
-      const uint32_t q_addr = smem_u32(sm.q);
-      const uint32_t p_addr = smem_u32(sm.p);
-      bool ok = mbar_wait(smem_u32(&sm.q_full), 0, abort, lim);
-      for (int t = 0; ok && t <= n_tiles; ++t) {
-        if (t < n_tiles) {
-          const int s = t & 1;
-          const uint32_t ph = (t >> 1) & 1;
-          if (!mbar_wait(smem_u32(&sm.k_full[s]), ph, abort, lim)) break;
-          if (!mbar_wait(smem_u32(&sm.s_empty[s]), ph ^ 1, abort, lim)) break;
-          tc_fence_after();
-          const uint32_t k_addr = smem_u32(sm.k[s]);
+      const int bw[2] = {b0, b1}, ew[2] = {e0, e1};
+      auto active = [&](int w, int t) { return t >= bw[w] && t < ew[w]; };
+      int pv_count[2] = {0, 0};
+      auto issue_s = [&](int w, uint32_t k_addr) {
+        const uint32_t q_addr = smem_u32(sm.q[w]);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            // K-major operands: 16-element k-steps are 32 bytes apart inside a 128-byte row,
-            // 64-element chunks are separate 16 KB tiles.
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            mma_bf16_ss(tmem + s * kBlockN, sw128_desc(q_addr + off, 16, 1024), sw128_desc(k_addr + off, 16, 1024),
-                        idesc_s, kk > 0);
-          }
-          mma_commit(smem_u32(&sm.s_full[s]));
-          mma_commit(smem_u32(&sm.k_empty[s]));
+        for (int kk = 0; kk < D / 16; ++kk) {
+          // K-major operands: 16-element k-steps are 32 bytes apart inside a 128-byte row,
+          // 64-element chunks are separate 16 KB tiles
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_bf16_ss(tmem + w * 128, sw128_desc(q_addr + off, 16, 1024), sw128_desc(k_addr + off, 16, 1024),
+                      idesc_s, kk > 0);
         }
-        if (t > 0) {
-          const int u = t - 1;
-          const int su = u & 1;
-          if (!mbar_wait(smem_u32(&sm.p_full), u & 1, abort, lim)) break;
-          if (!mbar_wait(smem_u32(&sm.v_full[su]), (u >> 1) & 1, abort, lim)) break;
-          tc_fence_after();
-          const uint32_t v_addr = smem_u32(sm.v[su]);
+        mma_commit(smem_u32(&sm.s_full[w]));
+      };
+      auto issue_pv = [&](int w, uint32_t v_addr) {
 #pragma unroll
-          for (int kk = 0; kk < kBlockN / 16; ++kk) {
-            // A = P (K-major, like Q); B = V is MN-major: 16 keys = 16 rows of 128 bytes,
-            // the next 64 head-dim columns sit one 16 KB chunk (LBO) further.
-            const uint32_t a_off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            mma_bf16_ss(tmem + kTmemO, sw128_desc(p_addr + a_off, 16, 1024),
-                        sw128_desc(v_addr + kk * 2048, 16384, 1024), idesc_o, (u > 0 || kk > 0));
-          }
-          mma_commit(smem_u32(&sm.o_done));
-          mma_commit(smem_u32(&sm.v_empty[su]));
+        for (int kk = 0; kk < kBlockN / 16; ++kk) {
+          // A = P from TMEM (16 keys = 8 packed columns per k-step); B = V MN-major: 16 keys =
+          // 16 rows of 128 bytes, the next 64 head-dim columns one 16 KB chunk (LBO) further
+          mma_bf16_ts(tmem + 256 + w * 128, tmem + w * 128 + kk * 8, sw128_desc(v_addr + kk * 2048, 16384, 1024),
+                      idesc_o, (pv_count[w] > 0 || kk > 0));
+        }
+        ++pv_count[w];
+      };
+      bool ok = mbar_wait(smem_u32(&sm.q_full), 0, abort, lim);
+      // prologue: S of the first KV tile
+      if (ok) {
+        const int Lk = 0;
+        ok = mbar_wait(smem_u32(&sm.slot_full[Lk % kSlots]), (Lk / kSlots) & 1, abort, lim);
+        if (ok) {
+          tc_fence_after();
+          const uint32_t k_addr = smem_u32(sm.kv[Lk % kSlots]);
+#pragma unroll
+          for (int w = 0; w < kQTiles; ++w)
+            if (active(w, t_begin)) issue_s(w, k_addr);
+          mma_commit(smem_u32(&sm.slot_empty[Lk % kSlots]));
         }
       }
+      for (int t = t_begin; ok && t < t_end; ++t) {
+        const int Lv = 2 * (t - t_begin) + 1;
+        const int Lk = Lv + 1;   // K of tile t + 1
+        const bool has_next = t + 1 < t_end;
+        if (!mbar_wait(smem_u32(&sm.slot_full[Lv % kSlots]), (Lv / kSlots) & 1, abort, lim)) break;
+        if (has_next && !mbar_wait(smem_u32(&sm.slot_full[Lk % kSlots]), (Lk / kSlots) & 1, abort, lim)) break;
+        const uint32_t v_addr = smem_u32(sm.kv[Lv % kSlots]);
+        const uint32_t k_addr = smem_u32(sm.kv[Lk % kSlots]);
+#pragma unroll
+        for (int w = 0; w < kQTiles; ++w) {
+          if (active(w, t)) {
+            if (!mbar_wait(smem_u32(&sm.p_full[w]), pv_count[w] & 1, abort, lim)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_pv(w, v_addr);
+          }
+          if (has_next && active(w, t + 1)) issue_s(w, k_addr);
+        }
+        if (!ok) break;
+        if (has_next) mma_commit(smem_u32(&sm.slot_empty[Lk % kSlots]));
+        mma_commit(smem_u32(&sm.slot_empty[Lv % kSlots]));
+      }
+#pragma unroll
+      for (int w = 0; w < kQTiles; ++w) mma_commit(smem_u32(&sm.o_final[w]));
       // every MMA issued above completes before TMEM is released
       mma_commit(smem_u32(&sm.mma_drain));
       mbar_wait_drain(smem_u32(&sm.mma_drain), 0, lim);
     }
   } else {
-    // ------------------------------------------------------------------ softmax warps 0-3
-    const int row = threadIdx.x;                 // 0..127 == TMEM lane
-    const int qi = q0 + row;
-    const uint32_t lane_base = uint32_t(warp * 32) << 16;
+    // ------------------------------------------------------------------ softmax warpgroups
+    const int w = warp >> 2;                     // query tile of this warpgroup
+    const int row = threadIdx.x & 127;           // == TMEM lane
+    const int qw0 = q0 + w * kBlockM;
+    const int qi = qw0 + row;
+    const int tb = w == 0 ? b0 : b1;
+    const int n_tiles = (w == 0 ? e0 : e1) - tb;
+    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+    const uint32_t s_col = tmem + lane_base + w * 128;
+    const uint32_t o_col = tmem + lane_base + 256 + w * 128;
     const float c = prm.scale_log2;
     float m = -INFINITY;                         // running max of scaled scores (log2 units)
     float l = 0.f;                               // running sum of exponentials
-    const uint32_t p_row = smem_u32(sm.p) + row * 128;
-    const uint32_t sw = row & 7;
     bool ok = true;
-    for (int t = 0; t < n_tiles; ++t) {
-      const int s = t & 1;
-      const int kv0 = (t_begin + t) * kBlockN;
+    for (int k = 0; k < n_tiles; ++k) {
+      const int kv0 = (tb + k) * kBlockN;
       // the vote keeps every lane of the warp on the same path into the .sync.aligned TMEM ops
-      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.s_full[s]), (t >> 1) & 1, abort, lim))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.s_full[w]), k & 1, abort, lim))) {
         ok = false;
         break;
       }
@@ -228,18 +261,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
       for (int ch = 0; ch < kBlockN / 32; ++ch) {
         uint32_t r[32];
-        tmem_ld32(tmem + lane_base + s * kBlockN + ch * 32, r);
+        tmem_ld32(s_col + ch * 32, r);
 #pragma unroll
         for (int j = 0; j < 32; ++j) sv[ch * 32 + j] = __uint_as_float(r[j]);
       }
-      tc_fence_before();
-      mbar_arrive(smem_u32(&sm.s_empty[s]));
-
-      const bool need_mask = (kv0 + kBlockN > prm.N) || (prm.causal && kv0 + kBlockN - 1 > q0) ||
-                             (prm.window > 0 && kv0 < q0 + kBlockM - prm.window);
+      const bool need_mask = (kv0 + kBlockN > prm.N) || (prm.causal && kv0 + kBlockN - 1 > qw0) ||
+                             (prm.window > 0 && kv0 < qw0 + kBlockM - prm.window);
       if (need_mask) {
-        const int hi = prm.causal ? min(qi, prm.N - 1) : prm.N - 1;       // last allowed key
-        const int lo = prm.window > 0 ? qi - prm.window + 1 : 0;           // first allowed key
+        const int hi = prm.causal ? min(qi, prm.N - 1) : prm.N - 1;   // last allowed key
+        const int lo = prm.window > 0 ? qi - prm.window + 1 : 0;       // first allowed key
 #pragma unroll
         for (int j = 0; j < kBlockN; ++j) {
           const int key = kv0 + j;
@@ -249,52 +279,44 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       float mx = sv[0];
 #pragma unroll
       for (int j = 1; j < kBlockN; ++j) mx = fmaxf(mx, sv[j]);
-      const float m_new = fmaxf(m, mx * c);
-      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;   // a row with no key yet stays at 0
-      const float alpha = ex2_approx(m - m_use);
+      const float m_cand = fmaxf(m, mx * c);
+      const bool grow = m_cand > m + kRescaleThreshold;   // false while the row has no key
+      const float m_new = grow ? m_cand : m;
+      const float alpha = grow ? ex2_approx(m - m_new) : 1.f;   // 0 for the first keys of a row
+      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;   // a row with no key yet gives P = 0
       float sum = 0.f;
-      uint32_t pk[kBlockN / 2];
 #pragma unroll
-      for (int j = 0; j < kBlockN; j += 2) {
-        const float p0 = ex2_approx(fmaf(sv[j], c, -m_use));
-        const float p1 = ex2_approx(fmaf(sv[j + 1], c, -m_use));
-        sum += p0 + p1;
-        pk[j / 2] = pack_bf16x2(p0, p1);
+      for (int ch = 0; ch < kBlockN / 32; ++ch) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          const float p0 = ex2_approx(fmaf(sv[ch * 32 + j], c, -m_use));
+          const float p1 = ex2_approx(fmaf(sv[ch * 32 + j + 1], c, -m_use));
+          sum += p0 + p1;
+          pk[j / 2] = pack_bf16x2(p0, p1);
+        }
+        // P overwrites the S columns already read: keys 32ch.. -> packed columns 16ch..
+        tmem_st16(s_col + ch * 16, pk);
       }
       l = l * alpha + sum;
       m = m_new;
-
-      if (t > 0) {
-        // PV of the previous tile must be complete: it read the P buffer, and O is rescaled now.
-        if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.o_done), (t - 1) & 1, abort, lim))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-      }
-      // P row -> shared memory, 128B-swizzled K-major layout (two 64-key chunks of 16 KB)
-#pragma unroll
-      for (int c16 = 0; c16 < kBlockN / 8; ++c16) {
-        const uint32_t addr = p_row + (c16 >> 3) * 16384 + (((c16 & 7) ^ sw) << 4);
-        st_shared_v4(addr, pk[c16 * 4 + 0], pk[c16 * 4 + 1], pk[c16 * 4 + 2], pk[c16 * 4 + 3]);
-      }
-      if (t > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+      if (k > 0 && __any_sync(0xffffffffu, grow)) {
+        // PV of the previous tile is complete (it was issued before this S), so O is stable;
+        // done after P so that the S registers are free
 #pragma unroll
         for (int ch = 0; ch < D / 32; ++ch) {
           uint32_t r[32];
-          const uint32_t ta = tmem + lane_base + kTmemO + ch * 32;
-          tmem_ld32(ta, r);
+          tmem_ld32(o_col + ch * 32, r);
 #pragma unroll
           for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha);
-          tmem_st32(ta, r);
+          tmem_st32(o_col + ch * 32, r);
         }
-        tmem_st_wait();
       }
-      fence_proxy_async_smem();
+      tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(smem_u32(&sm.p_full));
+      mbar_arrive(smem_u32(&sm.p_full[w]));
     }
-    if (ok && __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.o_done), (n_tiles - 1) & 1, abort, lim))) {
+    if (ok && n_tiles > 0 && __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.o_final[w]), 0, abort, lim))) {
       tc_fence_after();
       const float inv_l = 1.f / l;
       const bool in_range = qi < prm.N;
@@ -302,15 +324,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
       for (int ch = 0; ch < D / 32; ++ch) {
         uint32_t r[32];
-        tmem_ld32(tmem + lane_base + kTmemO + ch * 32, r);
-        uint32_t w[16];
+        tmem_ld32(o_col + ch * 32, r);
+        uint32_t wv[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j)
-          w[j] = pack_bf16x2(__uint_as_float(r[2 * j]) * inv_l, __uint_as_float(r[2 * j + 1]) * inv_l);
+          wv[j] = pack_bf16x2(__uint_as_float(r[2 * j]) * inv_l, __uint_as_float(r[2 * j + 1]) * inv_l);
         if (in_range) {
           uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+          for (int j = 0; j < 4; ++j) dst[j] = make_uint4(wv[4 * j], wv[4 * j + 1], wv[4 * j + 2], wv[4 * j + 3]);
         }
       }
       if (in_range) prm.lse[size_t(bh) * prm.N + qi] = (m + lg2_approx(l)) * 0.69314718055994531f;
