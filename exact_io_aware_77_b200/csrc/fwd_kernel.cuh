@@ -11,21 +11,21 @@
 //
 // sm_100a mapping: one CTA per pair of adjacent 128-row query tiles of one head, so every
 // K/V tile brought on chip serves 256 query rows.
-//   warp 8      TMA producer: both Q tiles once, then K_j, V_j through a 4-slot ring.
-//   warp 9      MMA issuer (one thread), in the order
-//                 PV0(j), S0(j+1), PV1(j), S1(j+1)
-//               so the tensor pipe computes one tile's products while the other tile's
-//               softmax runs (ping-pong).  S = Q K^T lands in TMEM; P is written back over
-//               the consumed S columns as bf16 and O += P V reads it from TMEM.
+//   warp 8      TMA producer (and TMEM owner): both Q tiles once, then K_j, V_j through a
+//               4-slot ring.
+//   warp 9      MMA issuer (one thread), in the order PV0(j), S0(j+1), PV1(j), S1(j+1), so
+//               the tensor pipe computes one tile's products while the other tile's softmax
+//               runs (ping-pong).  S = Q K^T lands in TMEM; P is written back over the
+//               consumed S columns as bf16 and O += P V reads it from TMEM.
 //   warps 0-3   softmax of query tile 0, warps 4-7 of tile 1: thread t owns row t (TMEM
-//               lane t).  Each tile: tcgen05.ld S, scale and mask, running max m and sum l,
-//               P = exp2(S c - m) packed to bf16 and stored to TMEM, then the epilogue
-//               O / l -> bf16 and L = (m + log2 l) ln 2.
+//               lane t): tcgen05.ld of S, scale and mask, running max m and sum l,
+//               P = 2^(S c - m) packed to bf16 and stored to TMEM, and at the end O / l ->
+//               bf16 and L = (m + log2 l) ln 2.
 // The running max is updated lazily: O in TMEM is rescaled only when a row's max grows by
 // more than 2^8; otherwise the stale max keeps being used (P <= 256, exact after the final
-// division by l).  Because S(j) is issued after PV(j-1) and tcgen05 MMAs of one thread run in
-// order, S(j) completing means PV(j-1) has completed, so a rescale never races an MMA and the
-// softmax warps never wait on P V.
+// division by l).  MMAs issued by one thread execute in order, so S(j) completing means
+// PV(j-1) of the same tile has completed: a rescale never races an MMA, and S(j+1) may be
+// issued right behind PV(j) although it overwrites the TMEM columns PV(j) reads P from.
 // TMEM columns: S0 [0,128), S1 [128,256), O0 [256, 256+D), O1 [384, 384+D); P_w occupies
 // the first 64 columns of S_w.
 #pragma once
@@ -43,6 +43,10 @@ constexpr int kWarpTma = 8;
 constexpr int kWarpMma = 9;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only when m grows by > 2^8
+#ifndef FA_FWD_EMU_PAIRS
+#define FA_FWD_EMU_PAIRS 2
+#endif
+constexpr int kEmuPairs = FA_FWD_EMU_PAIRS;   // of every 16 exponential pairs, this many use the FMA pipe
 
 struct FwdParams {
   __nv_bfloat16* o;   // [BH, N, D]
@@ -121,12 +125,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     mbar_init(smem_u32(&sm.mma_drain), 1);
     fence_mbar_init();
   }
-  if (warp == kWarpTma && lane == 0) {
-    tma_prefetch_desc(&tm_q);
-    tma_prefetch_desc(&tm_k);
-    tma_prefetch_desc(&tm_v);
-  }
-  if (warp == kWarpMma) {
+  if (warp == kWarpTma) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+    }
+    __syncwarp();
     tmem_alloc(smem_u32(&sm.tmem_base), kTmemCols);
     tmem_relinquish();
   }
@@ -152,7 +157,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const int kv0 = (t_begin + (L >> 1)) * kBlockN;
         const CUtensorMap* map = (L & 1) ? &tm_v : &tm_k;
         mbar_expect_tx(fb, Smem::kTileBytes);
-        for (int c = 0; c < Smem::kChunks; ++c) tma_load_3d(smem_u32(sm.kv[slot]) + c * 16384, map, fb, c * 64, kv0, bh);
+        for (int c = 0; c < Smem::kChunks; ++c)
+          tma_load_3d(smem_u32(sm.kv[slot]) + c * 16384, map, fb, c * 64, kv0, bh);
         issued = L + 1;
       }
       // let every copy this CTA started land before the CTA may exit
@@ -168,50 +174,51 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const int bw[2] = {b0, b1}, ew[2] = {e0, e1};
       auto active = [&](int w, int t) { return t >= bw[w] && t < ew[w]; };
       int pv_count[2] = {0, 0};
-      auto issue_s = [&](int w, uint32_t k_addr) {
-        const uint32_t q_addr = smem_u32(sm.q[w]);
+      // descriptors are built once; each k-step only adds a constant to the start field
+      const uint64_t dq[2] = {sw128_desc(smem_u32(sm.q[0]), 16, 1024), sw128_desc(smem_u32(sm.q[1]), 16, 1024)};
+      const uint64_t dkv0 = sw128_desc(smem_u32(sm.kv[0]), 16, 1024);
+      const uint64_t dv0 = sw128_desc(smem_u32(sm.kv[0]), 16384, 1024);
+      auto issue_s = [&](int w, uint32_t slot) {
+        const uint64_t dk = desc_advance(dkv0, slot * Smem::kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           // K-major operands: 16-element k-steps are 32 bytes apart inside a 128-byte row,
           // 64-element chunks are separate 16 KB tiles
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_bf16_ss(tmem + w * 128, sw128_desc(q_addr + off, 16, 1024), sw128_desc(k_addr + off, 16, 1024),
-                      idesc_s, kk > 0);
+          mma_bf16_ss(tmem + w * 128, desc_advance(dq[w], off), desc_advance(dk, off), idesc_s, kk > 0);
         }
         mma_commit(smem_u32(&sm.s_full[w]));
       };
-      auto issue_pv = [&](int w, uint32_t v_addr) {
+      auto issue_pv = [&](int w, uint32_t slot) {
+        const uint64_t dv = desc_advance(dv0, slot * Smem::kTileBytes);
+        const uint32_t acc = pv_count[w] > 0;
 #pragma unroll
         for (int kk = 0; kk < kBlockN / 16; ++kk) {
           // A = P from TMEM (16 keys = 8 packed columns per k-step); B = V MN-major: 16 keys =
           // 16 rows of 128 bytes, the next 64 head-dim columns one 16 KB chunk (LBO) further
-          mma_bf16_ts(tmem + 256 + w * 128, tmem + w * 128 + kk * 8, sw128_desc(v_addr + kk * 2048, 16384, 1024),
-                      idesc_o, (pv_count[w] > 0 || kk > 0));
+          mma_bf16_ts(tmem + 256 + w * 128, tmem + w * 128 + kk * 8, desc_advance(dv, kk * 2048), idesc_o,
+                      kk > 0 ? 1u : acc);
         }
         ++pv_count[w];
       };
       bool ok = mbar_wait(smem_u32(&sm.q_full), 0, abort, lim);
       // prologue: S of the first KV tile
       if (ok) {
-        const int Lk = 0;
-        ok = mbar_wait(smem_u32(&sm.slot_full[Lk % kSlots]), (Lk / kSlots) & 1, abort, lim);
+        ok = mbar_wait(smem_u32(&sm.slot_full[0]), 0, abort, lim);
         if (ok) {
           tc_fence_after();
-          const uint32_t k_addr = smem_u32(sm.kv[Lk % kSlots]);
 #pragma unroll
           for (int w = 0; w < kQTiles; ++w)
-            if (active(w, t_begin)) issue_s(w, k_addr);
-          mma_commit(smem_u32(&sm.slot_empty[Lk % kSlots]));
+            if (active(w, t_begin)) issue_s(w, 0);
+          mma_commit(smem_u32(&sm.slot_empty[0]));
         }
       }
       for (int t = t_begin; ok && t < t_end; ++t) {
-        const int Lv = 2 * (t - t_begin) + 1;
-        const int Lk = Lv + 1;   // K of tile t + 1
+        const int Lv = 2 * (t - t_begin) + 1;   // V of tile t
+        const int Lk = Lv + 1;                  // K of tile t + 1
         const bool has_next = t + 1 < t_end;
         if (!mbar_wait(smem_u32(&sm.slot_full[Lv % kSlots]), (Lv / kSlots) & 1, abort, lim)) break;
         if (has_next && !mbar_wait(smem_u32(&sm.slot_full[Lk % kSlots]), (Lk / kSlots) & 1, abort, lim)) break;
-        const uint32_t v_addr = smem_u32(sm.kv[Lv % kSlots]);
-        const uint32_t k_addr = smem_u32(sm.kv[Lk % kSlots]);
 #pragma unroll
         for (int w = 0; w < kQTiles; ++w) {
           if (active(w, t)) {
@@ -220,9 +227,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               break;
             }
             tc_fence_after();
-            issue_pv(w, v_addr);
+            issue_pv(w, Lv % kSlots);
           }
-          if (has_next && active(w, t + 1)) issue_s(w, k_addr);
+          if (has_next && active(w, t + 1)) issue_s(w, Lk % kSlots);
         }
         if (!ok) break;
         if (has_next) mma_commit(smem_u32(&sm.slot_empty[Lk % kSlots]));
@@ -241,82 +248,110 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const int qw0 = q0 + w * kBlockM;
     const int qi = qw0 + row;
     const int tb = w == 0 ? b0 : b1;
-    const int n_tiles = (w == 0 ? e0 : e1) - tb;
+    const int te = w == 0 ? e0 : e1;
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
     const uint32_t s_col = tmem + lane_base + w * 128;
     const uint32_t o_col = tmem + lane_base + 256 + w * 128;
     const float c = prm.scale_log2;
-    float m = -INFINITY;                         // running max of scaled scores (log2 units)
-    float l = 0.f;                               // running sum of exponentials
     bool ok = true;
-    for (int k = 0; k < n_tiles; ++k) {
-      const int kv0 = (tb + k) * kBlockN;
-      // the vote keeps every lane of the warp on the same path into the .sync.aligned TMEM ops
-      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.s_full[w]), k & 1, abort, lim))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      float sv[kBlockN];
+    float m = -INFINITY;   // running max of scaled scores (log2 units)
+    float l = 0.f;         // running sum of exponentials
+    for (int t = tb; t < te; ++t) {
+      {
+        const int k = t - tb;
+        const int kv0 = t * kBlockN;
+        // the vote keeps every lane of the warp on the same path into the .sync.aligned TMEM ops
+        if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.s_full[w]), k & 1, abort, lim))) ok = false;
+        if (!ok) break;
+        tc_fence_after();
+        float sv[kBlockN];
+        {
+          uint32_t r[kBlockN];
 #pragma unroll
-      for (int ch = 0; ch < kBlockN / 32; ++ch) {
-        uint32_t r[32];
-        tmem_ld32(s_col + ch * 32, r);
+          for (int ch = 0; ch < kBlockN / 32; ++ch) tmem_ld32_async(s_col + ch * 32, r + ch * 32);
+          tmem_ld_wait();
+          reg_fence<kBlockN>(r);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) sv[ch * 32 + j] = __uint_as_float(r[j]);
-      }
-      const bool need_mask = (kv0 + kBlockN > prm.N) || (prm.causal && kv0 + kBlockN - 1 > qw0) ||
-                             (prm.window > 0 && kv0 < qw0 + kBlockM - prm.window);
-      if (need_mask) {
-        const int hi = prm.causal ? min(qi, prm.N - 1) : prm.N - 1;   // last allowed key
-        const int lo = prm.window > 0 ? qi - prm.window + 1 : 0;       // first allowed key
-#pragma unroll
-        for (int j = 0; j < kBlockN; ++j) {
-          const int key = kv0 + j;
-          if (key > hi || key < lo) sv[j] = -INFINITY;
+          for (int j = 0; j < kBlockN; ++j) sv[j] = __uint_as_float(r[j]);
         }
-      }
-      float mx = sv[0];
+        const bool need_mask = (kv0 + kBlockN > prm.N) || (prm.causal && kv0 + kBlockN - 1 > qw0) ||
+                               (prm.window > 0 && kv0 < qw0 + kBlockM - prm.window);
+        if (need_mask) {
+          const int hi = prm.causal ? min(qi, prm.N - 1) : prm.N - 1;   // last allowed key
+          const int lo = prm.window > 0 ? qi - prm.window + 1 : 0;       // first allowed key
 #pragma unroll
-      for (int j = 1; j < kBlockN; ++j) mx = fmaxf(mx, sv[j]);
-      const float m_cand = fmaxf(m, mx * c);
-      const bool grow = m_cand > m + kRescaleThreshold;   // false while the row has no key
-      const float m_new = grow ? m_cand : m;
-      const float alpha = grow ? ex2_approx(m - m_new) : 1.f;   // 0 for the first keys of a row
-      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;   // a row with no key yet gives P = 0
-      float sum = 0.f;
-#pragma unroll
-      for (int ch = 0; ch < kBlockN / 32; ++ch) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          const float p0 = ex2_approx(fmaf(sv[ch * 32 + j], c, -m_use));
-          const float p1 = ex2_approx(fmaf(sv[ch * 32 + j + 1], c, -m_use));
-          sum += p0 + p1;
-          pk[j / 2] = pack_bf16x2(p0, p1);
+          for (int j = 0; j < kBlockN; ++j) {
+            const int key = kv0 + j;
+            if (key > hi || key < lo) sv[j] = -INFINITY;
+          }
         }
-        // P overwrites the S columns already read: keys 32ch.. -> packed columns 16ch..
-        tmem_st16(s_col + ch * 16, pk);
-      }
-      l = l * alpha + sum;
-      m = m_new;
-      if (k > 0 && __any_sync(0xffffffffu, grow)) {
-        // PV of the previous tile is complete (it was issued before this S), so O is stable;
-        // done after P so that the S registers are free
+        // row max: 3-input max in 8 independent chains (one chain would be 127 dependent steps)
+        float mx8[8];
 #pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch) {
-          uint32_t r[32];
-          tmem_ld32(o_col + ch * 32, r);
+        for (int i = 0; i < 8; ++i) mx8[i] = fmaxf(sv[2 * i], sv[2 * i + 1]);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha);
-          tmem_st32(o_col + ch * 32, r);
+        for (int j = 16; j < kBlockN; j += 16)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mx8[i] = max3f(mx8[i], sv[j + 2 * i], sv[j + 2 * i + 1]);
+        const float mx = max3f(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
+        const float m_cand = fmaxf(m, mx * c);
+        const bool grow = m_cand > m + kRescaleThreshold;   // false while the row has no key
+        const float m_new = grow ? m_cand : m;
+        const float alpha = grow ? ex2_approx(m - m_new) : 1.f;   // 0 for the first keys of a row
+        const float m_use = (m_new == -INFINITY) ? 0.f : m_new;   // a row with no key yet gives P = 0
+        // P = 2^(S c - m): in every 16 pairs the first kEmuPairs go through the FMA-pipe
+        // polynomial, the rest through MUFU ex2, so that neither unit limits the tile
+        const uint64_t c2 = f2(c, c), nm2 = f2(-m_use, -m_use);
+        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+        for (int ch = 0; ch < kBlockN / 32; ++ch) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int jp = 0; jp < 16; ++jp) {
+            const int j = ch * 32 + 2 * jp;
+            const uint64_t x = f2_fma(f2(sv[j], sv[j + 1]), c2, nm2);
+            float p0, p1;
+            if (jp < kEmuPairs) {
+              exp2_poly_x2(x, p0, p1);
+            } else {
+              float x0, x1;
+              f2_split(x, x0, x1);
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
+            }
+            acc[jp & 3] = f2_add(acc[jp & 3], f2(p0, p1));
+            pk[jp] = pack_bf16x2(p0, p1);
+          }
+          // P overwrites the S columns already read: keys 32ch.. -> packed columns 16ch..
+          tmem_st16(s_col + ch * 16, pk);
         }
+        float sum;
+        {
+          const uint64_t a = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+          float lo, hi;
+          f2_split(a, lo, hi);
+          sum = lo + hi;
+        }
+        l = l * alpha + sum;
+        m = m_new;
+        if (k > 0 && __any_sync(0xffffffffu, grow)) {
+          // PV of the previous tile is complete (it was issued before this S), so O is stable;
+          // done after P so that the S registers are free
+#pragma unroll
+          for (int ch = 0; ch < D / 32; ++ch) {
+            uint32_t r[32];
+            tmem_ld32(o_col + ch * 32, r);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha);
+            tmem_st32(o_col + ch * 32, r);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(smem_u32(&sm.p_full[w]));
       }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(smem_u32(&sm.p_full[w]));
     }
-    if (ok && n_tiles > 0 && __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.o_final[w]), 0, abort, lim))) {
+    if (ok && te > tb && __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.o_final[w]), 0, abort, lim))) {
       tc_fence_after();
       const float inv_l = 1.f / l;
       const bool in_range = qi < prm.N;
@@ -341,7 +376,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kWarpMma) {
+  if (warp == kWarpTma) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);

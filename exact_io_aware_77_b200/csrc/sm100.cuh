@@ -166,6 +166,10 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo_byte
          (uint64_t((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
+// Descriptor `d` moved `bytes` further along (k-steps inside a tile).  Only the 14-bit start
+// field changes; shared-memory addresses stay below 256 KB, so the add never carries out.
+__device__ __forceinline__ uint64_t desc_advance(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
+
 // 32 lanes x 32 consecutive 32-bit columns: thread t of the warp gets lane (base + t), columns
 // [col, col + 32).  The wait is in the same statement so the registers are valid on return.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
@@ -182,6 +186,30 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr)
       : "memory");
 }
+// Same load without the wait: several can be in flight; call tmem_ld_wait() and then
+// reg_fence() on each destination before reading it.
+__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]),
+        "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
+        "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// Ties registers written by an async TMEM load to a point after tmem_ld_wait(): the empty
+// volatile statement "modifies" them, so no use can be scheduled before it.
+template <int N>
+__device__ __forceinline__ void reg_fence(uint32_t* r) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i])::"memory");
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -214,6 +242,58 @@ __device__ __forceinline__ float lg2_approx(float x) {
   asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// ---------------------------------------------------------------- packed fp32 pairs (f32x2)
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// 2^x for a pair of arguments on the FMA pipe instead of the MUFU unit.
+// Cody-Waite style reduction x = n + f with n = round(x), f in [-1/2, 1/2]: adding
+// 1.5 * 2^23 leaves round(x) in the low mantissa bits (valid for |x| < 2^22).  2^f is a
+// degree-3 polynomial whose coefficients minimise the maximum relative error on
+// [-1/2, 1/2] (Remez exchange; csrc/gen_exp2_poly.py regenerates them; max relative error
+// 7.5e-5, below half a bf16 ulp).  2^n is applied by adding n to the exponent field.
+// Arguments are clamped to >= -125 so that the exponent never leaves the normal range;
+// 2^-125 stands in for 0 (masked scores, -inf, give 2^-125 instead of 0).
+__device__ __forceinline__ void exp2_poly_x2(uint64_t x, float& y0, float& y1) {
+  constexpr float kRound = 12582912.0f;   // 1.5 * 2^23
+  float x0, x1;
+  f2_split(x, x0, x1);
+  x = f2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t t = f2_add(x, f2(kRound, kRound));
+  const uint64_t r = f2_add(t, f2(-kRound, -kRound));          // round(x) as a float
+  const uint64_t f = f2_fma(r, f2(-1.f, -1.f), x);              // x - round(x)
+  uint64_t p = f2_fma(f, f2(0.05517167f, 0.05517167f), f2(0.24261113f, 0.24261113f));
+  p = f2_fma(p, f, f2(0.69326097f, 0.69326097f));
+  p = f2_fma(p, f, f2(0.99992806f, 0.99992806f));
+  float p0, p1, t0, t1;
+  f2_split(p, p0, p1);
+  f2_split(t, t0, t1);
+  y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
