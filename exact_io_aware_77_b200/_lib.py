@@ -19,6 +19,7 @@ STATUS_NAMES = {
     0: "FA_OK", 1: "FA_ERR_NULL", 2: "FA_ERR_SHAPE", 3: "FA_ERR_HEADDIM", 4: "FA_ERR_ALIGN",
     5: "FA_ERR_MASK", 6: "FA_ERR_WORKSPACE", 7: "FA_ERR_CUDA", 8: "FA_ERR_DEVICE",
     9: "FA_ERR_TIMEOUT", 10: "FA_ERR_SCALE", 11: "FA_ERR_NOALLOC_LIMIT",
+    12: "FA_ERR_INTERNAL",
 }
 STATUS = {v: k for k, v in STATUS_NAMES.items()}
 

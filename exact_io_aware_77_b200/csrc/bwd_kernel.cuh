@@ -11,22 +11,26 @@
 // Three kernels on one stream:
 //   fa_bwd_prep      D (fp32), L in log2 units (padded rows get +inf so their P is 0),
 //                    and a zeroed fp32 dQ accumulator.
-//   fa_bwd_kernel    one CTA per 128-key tile of one head; loops over 64-row query tiles.
+//   fa_bwd_kernel    one CTA per 128-key tile of one head; loops over 128-row query tiles.
 //   fa_bwd_dq_final  dQ = scale * accumulator, rounded to bf16.
 //
-// fa_bwd_kernel roles (320 threads):
-//   warp 8      TMA producer: K_j, V_j once; Q_i, dO_i (+ their L and D rows) into a 3-stage ring.
-//   warp 9      MMA issuer:   S^T = K Q_i^T and dP^T = V dO_i^T (N = 64), then
-//                              dV += P^T dO_i and dK += dS^T Q_i with A read from TMEM,
-//                              and dQ_i^T = K^T dS^T (A, B from shared memory).
-//   warps 0-3   thread t owns key kv0 + t (TMEM lane t): P^T = exp2(S^T c - L), dS^T =
-//               P^T o (dP^T - D) with the causal/window mask; P^T and dS^T go back to TMEM
-//               as bf16 (A operands of the dV/dK MMAs) and dS^T also to shared memory (B
-//               operand of the dQ^T MMA).  At the end they write dK and dV.
-//   warps 4-7   thread t owns head-dim column t of dQ_i^T (TMEM lane t) and adds its 64
-//               values into the fp32 accumulator with coalesced reductions.
-// TMEM columns: [0,128) dK, [128,256) dV, [256,320)/[320,384) S^T buffers (later P^T in the
-// first 32 columns and dS^T in the next 32), [384,448) dP^T, [448,512) dQ^T.
+// fa_bwd_kernel roles (320 threads), every MMA 128 x 128 (narrower ones cost as much time):
+//   warp 8      TMA producer: K, V once; Q_i, dO_i (+ their L and D rows) into a 2-stage ring.
+//   warp 9      MMA issuer, per query tile i in the order
+//                 dV += P_i^T dO_i, S_{i+1}^T = K Q_{i+1}^T, dK += dS_i^T Q_i, dQ_i = dS_i K,
+//                 dP_{i+1}^T = V dO_{i+1}^T
+//               (dV and dK read their A operand from TMEM), so that the exponentials of tile
+//               i+1 run while dK_i and dQ_i are computed, and dS of tile i+1 while dV_{i+1}
+//               and S_{i+2} are.
+//   warps 0-3   thread t owns key kv0 + t (TMEM lane t).  Phase A: P^T = exp2(S^T c - L) with
+//               the causal/window mask, stored to TMEM as bf16.  Phase B: dS^T = P^T o (dP^T - D)
+//               to TMEM (A of dK) and to shared memory (A of dQ).  At the end: dK, dV.
+//   warps 4-7   thread t owns query q0 + t of dQ_i (TMEM lane t) and adds its row into the fp32
+//               accumulator with 16-byte vector reductions.
+// TMEM columns: dK [0,128), dV [128,256), S^T [256,384) with P^T in [256,320) once read,
+// dP^T [384,512) with dS^T in [384,448) once read, and dQ in [384,512).  MMAs of one thread
+// run in order, which makes each reuse safe: S_{i+1} is issued after dV_i read P_i, dQ_i after
+// dK_i read dS_i; only dP_{i+1} waits until warps 4-7 have read dQ_i out.
 #pragma once
 
 #include "sm100.cuh"
@@ -34,12 +38,13 @@
 namespace fa {
 
 constexpr int kBwdKeys = 128;    // keys per CTA
-constexpr int kBwdRows = 64;     // queries per iteration
-constexpr int kBwdQStages = 3;
+constexpr int kBwdRows = 128;    // queries per iteration
+constexpr int kBwdQStages = 2;
 constexpr int kBwdThreads = 320;
 constexpr int kBwdWarpTma = 8;
 constexpr int kBwdWarpMma = 9;
-constexpr uint32_t kTdK = 0, kTdV = 128, kTS = 256, kTdP = 384, kTdQ = 448;
+constexpr uint32_t kTdK = 0, kTdV = 128, kTS = 256, kTP = 256, kTdP = 384, kTdS = 384, kTdQ = 384;
+constexpr int FA_DEVICE_SMEM_ALIGN = 2;   // status bit: dynamic shared memory not 1 KB aligned
 
 struct BwdParams {
   const float* lp;        // [BH, Np] L * log2(e), +inf on padded rows
@@ -56,20 +61,17 @@ struct BwdParams {
 template <int D>
 struct BwdSmem {
   static constexpr int kChunks = D / 64;
-  static constexpr uint32_t kKVBytes = kBwdKeys * D * 2;   // K or V tile
-  static constexpr uint32_t kQBytes = kBwdRows * D * 2;    // Q or dO tile
-  static constexpr uint32_t kDsBytes = kBwdKeys * kBwdRows * 2;
-  alignas(1024) uint8_t k[kKVBytes];
-  alignas(1024) uint8_t v[kKVBytes];
-  alignas(1024) uint8_t q[kBwdQStages][kQBytes];
-  alignas(1024) uint8_t dout[kBwdQStages][kQBytes];
-  alignas(1024) uint8_t ds[2][kDsBytes];
+  static constexpr uint32_t kTileBytes = 128 * D * 2;      // K, V, Q or dO tile
+  alignas(1024) uint8_t k[kTileBytes];
+  alignas(1024) uint8_t v[kTileBytes];
+  alignas(1024) uint8_t q[kBwdQStages][kTileBytes];
+  alignas(1024) uint8_t dout[kBwdQStages][kTileBytes];
+  alignas(1024) uint8_t ds[kBwdKeys * kBwdRows * 2];       // dS^T: [key][query], 64-query chunks
   alignas(16) float lp[kBwdQStages][kBwdRows];
   alignas(16) float dd[kBwdQStages][kBwdRows];
   alignas(8) uint64_t kv_full;
   uint64_t q_full[kBwdQStages], q_empty[kBwdQStages];
-  uint64_t s_full[2], s_free[2], ds_full[2], ds_free[2];
-  uint64_t dp_full, dp_free, dq_full, dq_free, mma_final, mma_drain;
+  uint64_t s_full, dp_full, pa_full, ds_full, ds_free, dq_full, dq_free, mma_final, mma_drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -79,8 +81,13 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
                "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
                : "memory");
 }
+__device__ __forceinline__ void red_add_f4(float* addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(__uint_as_float(a)),
+               "f"(__uint_as_float(b)), "f"(__uint_as_float(c)), "f"(__uint_as_float(d))
+               : "memory");
+}
 
-// query tiles (of 64 rows) that can see some key of the tile [kv0, kv0 + 128)
+// query tiles (of 128 rows) that can see some key of the tile [kv0, kv0 + 128)
 __device__ __forceinline__ void q_tile_range(int kv0, int N, int causal, int window, int& i_begin, int& i_end) {
   const int n_q = (N + kBwdRows - 1) / kBwdRows;
   i_begin = causal ? kv0 / kBwdRows : 0;
@@ -159,13 +166,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                   const BwdParams prm) {
   using Smem = BwdSmem<D>;
-  extern __shared__ uint8_t smem_raw[];
-  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // the layout fills almost all 227 KB, so no slack is left for realigning the base
+  if (smem_u32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) atomicOr(&g_status, FA_DEVICE_SMEM_ALIGN);
+    return;
+  }
+  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int bh = int(blockIdx.x / prm.n_kv_tiles);
-  const int kv_tile = int(blockIdx.x % prm.n_kv_tiles);    // longest causal tiles first within a head
+  const int kv_tile = int(blockIdx.x % prm.n_kv_tiles);
   const int kv0 = kv_tile * kBwdKeys;
   int i_begin, i_end;
   q_tile_range(kv0, prm.N, prm.causal, prm.window, i_begin, i_end);
@@ -180,16 +192,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(smem_u32(&sm.q_full[s]), 1);
       mbar_init(smem_u32(&sm.q_empty[s]), 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(smem_u32(&sm.s_full[b]), 1);
-      mbar_init(smem_u32(&sm.s_free[b]), 1);
-      mbar_init(smem_u32(&sm.ds_full[b]), 128);
-      mbar_init(smem_u32(&sm.ds_free[b]), 1);
-    }
+    mbar_init(smem_u32(&sm.s_full), 1);
     mbar_init(smem_u32(&sm.dp_full), 1);
-    mbar_init(smem_u32(&sm.dp_free), 128);
+    mbar_init(smem_u32(&sm.pa_full), 128);
+    mbar_init(smem_u32(&sm.ds_full), 128);
+    mbar_init(smem_u32(&sm.ds_free), 1);
     mbar_init(smem_u32(&sm.dq_full), 1);
-    mbar_init(smem_u32(&sm.dq_free), D);
+    mbar_init(smem_u32(&sm.dq_free), 128);
     mbar_init(smem_u32(&sm.mma_final), 1);
     mbar_init(smem_u32(&sm.mma_drain), 1);
     fence_mbar_init();
@@ -213,7 +222,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       const uint32_t kvb = smem_u32(&sm.kv_full);
-      mbar_expect_tx(kvb, 2 * Smem::kKVBytes);
+      mbar_expect_tx(kvb, 2 * Smem::kTileBytes);
       for (int c = 0; c < Smem::kChunks; ++c) {
         tma_load_3d(smem_u32(sm.k) + c * 16384, &tm_k, kvb, c * 64, kv0, bh);
         tma_load_3d(smem_u32(sm.v) + c * 16384, &tm_v, kvb, c * 64, kv0, bh);
@@ -225,10 +234,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int q0 = (i_begin + it) * kBwdRows;
         if (!mbar_wait(smem_u32(&sm.q_empty[qs]), ph ^ 1, abort, lim)) break;
         const uint32_t qb = smem_u32(&sm.q_full[qs]);
-        mbar_expect_tx(qb, 2 * Smem::kQBytes + 2 * kBwdRows * 4);
+        mbar_expect_tx(qb, 2 * Smem::kTileBytes + 2 * kBwdRows * 4);
         for (int c = 0; c < Smem::kChunks; ++c) {
-          tma_load_3d(smem_u32(sm.q[qs]) + c * 8192, &tm_q, qb, c * 64, q0, bh);
-          tma_load_3d(smem_u32(sm.dout[qs]) + c * 8192, &tm_do, qb, c * 64, q0, bh);
+          tma_load_3d(smem_u32(sm.q[qs]) + c * 16384, &tm_q, qb, c * 64, q0, bh);
+          tma_load_3d(smem_u32(sm.dout[qs]) + c * 16384, &tm_do, qb, c * 64, q0, bh);
         }
         const size_t row = size_t(bh) * prm.Np + q0;
         bulk_load(smem_u32(sm.lp[qs]), prm.lp + row, kBwdRows * 4, qb);
@@ -242,74 +251,70 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else if (warp == kBwdWarpMma) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, kBwdRows, false, false);   // S^T, dP^T
+      constexpr uint32_t idesc_t = idesc_bf16_f32(128, kBwdRows, false, false);   // S^T, dP^T
       constexpr uint32_t idesc_kv = idesc_bf16_f32(128, D, false, true);          // dV, dK (A in TMEM)
-      constexpr uint32_t idesc_q = idesc_bf16_f32(128, kBwdRows, true, true);     // dQ^T
-      const uint32_t k_addr = smem_u32(sm.k);
-      const uint32_t v_addr = smem_u32(sm.v);
-      bool ok = mbar_wait(smem_u32(&sm.kv_full), 0, abort, lim);
-      for (int it = 0; ok && it <= n_it; ++it) {
-        if (it < n_it) {
-          const int qs = it % kBwdQStages;
-          const int st = it & 1;
-          if (!mbar_wait(smem_u32(&sm.q_full[qs]), (it / kBwdQStages) & 1, abort, lim)) break;
-          if (!mbar_wait(smem_u32(&sm.s_free[st]), ((it >> 1) & 1) ^ 1, abort, lim)) break;
-          tc_fence_after();
-          const uint32_t q_addr = smem_u32(sm.q[qs]);
-          const uint32_t do_addr = smem_u32(sm.dout[qs]);
+      constexpr uint32_t idesc_q = idesc_bf16_f32(kBwdRows, D, true, true);       // dQ
+      const uint64_t dk_kmaj = sw128_desc(smem_u32(sm.k), 16, 1024);
+      const uint64_t dv_kmaj = sw128_desc(smem_u32(sm.v), 16, 1024);
+      const uint64_t dk_mn = sw128_desc(smem_u32(sm.k), 16384, 1024);
+      const uint64_t dds_mn = sw128_desc(smem_u32(sm.ds), 16384, 1024);
+      // X^T = M_tile N_i^T with both operands K-major over the head dim (S^T and dP^T)
+      auto issue_t = [&](uint64_t a, const uint8_t* b_tile, uint32_t d_col) {
+        const uint64_t b = sw128_desc(smem_u32(b_tile), 16, 1024);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t a_off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            const uint32_t b_off = (kk >> 2) * 8192 + (kk & 3) * 32;
-            mma_bf16_ss(tmem + kTS + st * 64, sw128_desc(k_addr + a_off, 16, 1024),
-                        sw128_desc(q_addr + b_off, 16, 1024), idesc_s, kk > 0);
-          }
-          mma_commit(smem_u32(&sm.s_full[st]));
-          if (!mbar_wait(smem_u32(&sm.dp_free), (it & 1) ^ 1, abort, lim)) break;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t a_off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            const uint32_t b_off = (kk >> 2) * 8192 + (kk & 3) * 32;
-            mma_bf16_ss(tmem + kTdP, sw128_desc(v_addr + a_off, 16, 1024), sw128_desc(do_addr + b_off, 16, 1024),
-                        idesc_s, kk > 0);
-          }
-          mma_commit(smem_u32(&sm.dp_full));
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_bf16_ss(tmem + d_col, desc_advance(a, off), desc_advance(b, off), idesc_t, kk > 0);
         }
-        if (it > 0) {
-          const int u = it - 1;
-          const int qsu = u % kBwdQStages;
-          const int su = u & 1;
-          if (!mbar_wait(smem_u32(&sm.ds_full[su]), (u >> 1) & 1, abort, lim)) break;
+      };
+      // acc += A(TMEM, 128 x 128 queries) * B (MN-major Q_i or dO_i: 16 queries = 2 KB per k-step)
+      auto issue_kv = [&](uint32_t a_col, const uint8_t* b_tile, uint32_t d_col, bool first) {
+        const uint64_t b = sw128_desc(smem_u32(b_tile), 16384, 1024);
+#pragma unroll
+        for (int kk = 0; kk < kBwdRows / 16; ++kk)
+          mma_bf16_ts(tmem + d_col, tmem + a_col + kk * 8, desc_advance(b, kk * 2048), idesc_kv,
+                      (first && kk == 0) ? 0u : 1u);
+      };
+      bool ok = mbar_wait(smem_u32(&sm.kv_full), 0, abort, lim) && mbar_wait(smem_u32(&sm.q_full[0]), 0, abort, lim);
+      if (ok) {
+        tc_fence_after();
+        issue_t(dk_kmaj, sm.q[0], kTS);
+        mma_commit(smem_u32(&sm.s_full));
+        issue_t(dv_kmaj, sm.dout[0], kTdP);
+        mma_commit(smem_u32(&sm.dp_full));
+      }
+      for (int it = 0; ok && it < n_it; ++it) {
+        const int qs = it % kBwdQStages;
+        const bool has_next = it + 1 < n_it;
+        const int qn = (it + 1) % kBwdQStages;
+        // dV += P^T dO_i
+        if (!mbar_wait(smem_u32(&sm.pa_full), it & 1, abort, lim)) break;
+        tc_fence_after();
+        issue_kv(kTP, sm.dout[qs], kTdV, it == 0);
+        // S^T of the next tile (overwrites P^T only after dV above has read it)
+        if (has_next) {
+          if (!mbar_wait(smem_u32(&sm.q_full[qn]), ((it + 1) / kBwdQStages) & 1, abort, lim)) break;
+          issue_t(dk_kmaj, sm.q[qn], kTS);
+          mma_commit(smem_u32(&sm.s_full));
+        }
+        // dK += dS^T Q_i, then dQ_i = dS_i K (A = dS^T from shared memory, MN-major over queries)
+        if (!mbar_wait(smem_u32(&sm.ds_full), it & 1, abort, lim)) break;
+        tc_fence_after();
+        issue_kv(kTdS, sm.q[qs], kTdK, it == 0);
+        if (!mbar_wait(smem_u32(&sm.dq_free), (it & 1) ^ 1, abort, lim)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kBwdKeys / 16; ++kk)
+          mma_bf16_ss(tmem + kTdQ, desc_advance(dds_mn, kk * 2048), desc_advance(dk_mn, kk * 2048), idesc_q, kk > 0);
+        mma_commit(smem_u32(&sm.dq_full));
+        mma_commit(smem_u32(&sm.ds_free));
+        mma_commit(smem_u32(&sm.q_empty[qs]));
+        // dP^T of the next tile once dQ_i has been read out of the same columns
+        if (has_next) {
+          if (!mbar_wait(smem_u32(&sm.dq_free), it & 1, abort, lim)) break;
           tc_fence_after();
-          const uint32_t q_addr = smem_u32(sm.q[qsu]);
-          const uint32_t do_addr = smem_u32(sm.dout[qsu]);
-#pragma unroll
-          for (int kk = 0; kk < kBwdRows / 16; ++kk) {
-            // B = dO_i / Q_i as MN-major [queries x D]: 16 queries per k-step = 2 KB, the next
-            // 64 head-dim columns one 8 KB chunk (LBO) further.
-            mma_bf16_ts(tmem + kTdV, tmem + kTS + su * 64 + kk * 8, sw128_desc(do_addr + kk * 2048, 8192, 1024),
-                        idesc_kv, (u > 0 || kk > 0));
-          }
-#pragma unroll
-          for (int kk = 0; kk < kBwdRows / 16; ++kk) {
-            mma_bf16_ts(tmem + kTdK, tmem + kTS + su * 64 + 32 + kk * 8,
-                        sw128_desc(q_addr + kk * 2048, 8192, 1024), idesc_kv, (u > 0 || kk > 0));
-          }
-          mma_commit(smem_u32(&sm.s_free[su]));
-          if (!mbar_wait(smem_u32(&sm.dq_free), (u & 1) ^ 1, abort, lim)) break;
-          tc_fence_after();
-          const uint32_t ds_addr = smem_u32(sm.ds[su]);
-#pragma unroll
-          for (int kk = 0; kk < kBwdKeys / 16; ++kk) {
-            // A = K^T (MN-major over the head dim: 64-column chunks 16 KB apart), B = dS^T
-            // (MN-major over the 64 queries); 16 keys per k-step = 2 KB in both.
-            mma_bf16_ss(tmem + kTdQ, sw128_desc(k_addr + kk * 2048, 16384, 1024),
-                        sw128_desc(ds_addr + kk * 2048, 8192, 1024), idesc_q, kk > 0);
-          }
-          mma_commit(smem_u32(&sm.dq_full));
-          mma_commit(smem_u32(&sm.ds_free[su]));
-          mma_commit(smem_u32(&sm.q_empty[qsu]));
+          issue_t(dv_kmaj, sm.dout[qn], kTdP);
+          mma_commit(smem_u32(&sm.dp_full));
         }
       }
       mma_commit(smem_u32(&sm.mma_final));
@@ -322,80 +327,99 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int key = kv0 + r;
     const uint32_t lane_base = uint32_t(warp * 32) << 16;
     const float c = prm.scale_log2;
+    const uint32_t ds_row = smem_u32(sm.ds) + r * 128;
+    const uint32_t sw = r & 7;
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
       const int qs = it % kBwdQStages;
-      const int st = it & 1;
       const int q0 = (i_begin + it) * kBwdRows;
+      // ---- phase A: P^T = 2^(S^T c - L) -> TMEM (bf16)
       bool w_ok = mbar_wait(smem_u32(&sm.q_full[qs]), (it / kBwdQStages) & 1, abort, lim);
-      w_ok = w_ok && mbar_wait(smem_u32(&sm.s_full[st]), (it >> 1) & 1, abort, lim);
+      w_ok = w_ok && mbar_wait(smem_u32(&sm.s_full), it & 1, abort, lim);
       if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
       tc_fence_after();
-      float s[kBwdRows], dp[kBwdRows];
-      {
-        uint32_t ra[32], rb[32];
-        tmem_ld32(tmem + lane_base + kTS + st * 64, ra);
-        tmem_ld32(tmem + lane_base + kTS + st * 64 + 32, rb);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          s[j] = __uint_as_float(ra[j]);
-          s[32 + j] = __uint_as_float(rb[j]);
-        }
-      }
-      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.dp_full), it & 1, abort, lim))) { ok = false; break; }
-      tc_fence_after();
-      {
-        uint32_t ra[32], rb[32];
-        tmem_ld32(tmem + lane_base + kTdP, ra);
-        tmem_ld32(tmem + lane_base + kTdP + 32, rb);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          dp[j] = __uint_as_float(ra[j]);
-          dp[32 + j] = __uint_as_float(rb[j]);
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(smem_u32(&sm.dp_free));
-
-      const float* lp = sm.lp[qs];
-      const float* dd = sm.dd[qs];
       const bool need_mask = (prm.causal && kv0 + kBwdKeys - 1 > q0) ||
                              (prm.window > 0 && kv0 < q0 + kBwdRows - prm.window) || (kv0 + kBwdKeys > prm.N);
-      uint32_t pp[kBwdRows / 2], pd[kBwdRows / 2];
+      const float* lp = sm.lp[qs];
+      uint32_t pk_all[64];   // packed P^T of this tile, kept for phase B (S_{i+1} may overwrite TMEM)
 #pragma unroll
-      for (int j = 0; j < kBwdRows; j += 2) {
-        float p0 = ex2_approx(fmaf(s[j], c, -lp[j]));
-        float p1 = ex2_approx(fmaf(s[j + 1], c, -lp[j + 1]));
-        if (need_mask) {
-          const int qa = q0 + j, qb = q0 + j + 1;
-          const bool oka = key < prm.N && (!prm.causal || key <= qa) && (prm.window == 0 || key > qa - prm.window);
-          const bool okb = key < prm.N && (!prm.causal || key <= qb) && (prm.window == 0 || key > qb - prm.window);
-          p0 = oka ? p0 : 0.f;
-          p1 = okb ? p1 : 0.f;
+      for (int half = 0; half < 2; ++half) {
+        uint32_t sr[64];
+        tmem_ld32_async(tmem + lane_base + kTS + half * 64, sr);
+        tmem_ld32_async(tmem + lane_base + kTS + half * 64 + 32, sr + 32);
+        tmem_ld_wait();
+        reg_fence<64>(sr);
+        // arguments first; the mask (diagonal, window edge and tail tiles only) is one branch
+        // around a separate loop that sets masked arguments to -inf, so exp2 gives exactly 0
+        float x[64];
+#pragma unroll
+        for (int j4 = 0; j4 < 16; ++j4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(lp + half * 64 + 4 * j4);
+          x[4 * j4 + 0] = fmaf(__uint_as_float(sr[4 * j4 + 0]), c, -l4.x);
+          x[4 * j4 + 1] = fmaf(__uint_as_float(sr[4 * j4 + 1]), c, -l4.y);
+          x[4 * j4 + 2] = fmaf(__uint_as_float(sr[4 * j4 + 2]), c, -l4.z);
+          x[4 * j4 + 3] = fmaf(__uint_as_float(sr[4 * j4 + 3]), c, -l4.w);
         }
-        const float d0 = p0 * (dp[j] - dd[j]);
-        const float d1 = p1 * (dp[j + 1] - dd[j + 1]);
-        pp[j / 2] = pack_bf16x2(p0, p1);
-        pd[j / 2] = pack_bf16x2(d0, d1);
-      }
-      // P^T and dS^T into this S buffer's columns (A operands of the dV / dK MMAs)
-      tmem_st32(tmem + lane_base + kTS + st * 64, pp);
-      tmem_st32(tmem + lane_base + kTS + st * 64 + 32, pd);
-      // dS^T into shared memory for the dQ^T MMA; the buffer is free once the dQ^T MMA of
-      // iteration it - 2 has completed
-      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.ds_free[st]), ((it >> 1) & 1) ^ 1, abort, lim))) {
-        ok = false;
-        break;
-      }
-      const uint32_t row_addr = smem_u32(sm.ds[st]) + r * 128;
+        if (need_mask) {
+          const int qbase = q0 + half * 64;
 #pragma unroll
-      for (int c16 = 0; c16 < 8; ++c16)
-        st_shared_v4(row_addr + ((c16 ^ (r & 7)) << 4), pd[4 * c16], pd[4 * c16 + 1], pd[4 * c16 + 2],
-                     pd[4 * c16 + 3]);
+          for (int j = 0; j < 64; ++j) {
+            const int qq = qbase + j;
+            const bool okk = key < prm.N && (!prm.causal || key <= qq) && (prm.window == 0 || key > qq - prm.window);
+            x[j] = okk ? x[j] : -INFINITY;
+          }
+        }
+        uint32_t* pk = pk_all + half * 32;
+#pragma unroll
+        for (int j2 = 0; j2 < 32; ++j2) pk[j2] = pack_bf16x2(ex2_approx(x[2 * j2]), ex2_approx(x[2 * j2 + 1]));
+        // 64 queries -> 32 packed columns of the (already read) S^T columns
+        tmem_st16(tmem + lane_base + kTP + half * 32, pk);
+        tmem_st16(tmem + lane_base + kTP + half * 32 + 16, pk + 16);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&sm.pa_full));
+
+      // ---- phase B: dS^T = P^T o (dP^T - D) -> TMEM (bf16) and shared memory
+      w_ok = mbar_wait(smem_u32(&sm.dp_full), it & 1, abort, lim);
+      // dS buffer free once the dQ MMA of the previous tile has completed
+      w_ok = w_ok && mbar_wait(smem_u32(&sm.ds_free), (it & 1) ^ 1, abort, lim);
+      if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+      tc_fence_after();
+      const float* ddp = sm.dd[qs];
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        // 32 queries per step: dP^T columns 384 + 32 q4 .. (read before any dS^T lands on them)
+        uint32_t dr[32];
+        tmem_ld32(tmem + lane_base + kTdP + q4 * 32, dr);
+        uint32_t pd[16];
+#pragma unroll
+        for (int j4 = 0; j4 < 8; ++j4) {
+          const float4 d4 = *reinterpret_cast<const float4*>(ddp + q4 * 32 + 4 * j4);
+          const uint32_t w01 = pk_all[q4 * 16 + 2 * j4], w23 = pk_all[q4 * 16 + 2 * j4 + 1];
+          const float2 pa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w01));
+          const float2 pb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w23));
+          const float s0 = pa.x * (__uint_as_float(dr[4 * j4]) - d4.x);
+          const float s1 = pa.y * (__uint_as_float(dr[4 * j4 + 1]) - d4.y);
+          const float s2 = pb.x * (__uint_as_float(dr[4 * j4 + 2]) - d4.z);
+          const float s3 = pb.y * (__uint_as_float(dr[4 * j4 + 3]) - d4.w);
+          pd[2 * j4] = pack_bf16x2(s0, s1);
+          pd[2 * j4 + 1] = pack_bf16x2(s2, s3);
+        }
+        // TMEM copy for the dK MMA: packed columns kTdS + 16 q4 (inside dP^T columns already read)
+        tmem_st16(tmem + lane_base + kTdS + q4 * 16, pd);
+        // shared-memory copy for the dQ MMA: queries 32 q4.. = half a 128-byte row of chunk q4 / 2
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          const int piece = (q4 & 1) * 4 + c4;
+          st_shared_v4(ds_row + (q4 >> 1) * 16384 + ((piece ^ sw) << 4), pd[4 * c4], pd[4 * c4 + 1],
+                       pd[4 * c4 + 2], pd[4 * c4 + 3]);
+        }
+      }
       tmem_st_wait();
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(smem_u32(&sm.ds_full[st]));
+      mbar_arrive(smem_u32(&sm.ds_full));
     }
     // epilogue: dK = scale * acc, dV = acc, rows of keys < N
     if (ok && __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.mma_final), 0, abort, lim))) {
@@ -423,24 +447,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       }
     }
-  } else if (warp < 8 && (warp - 4) * 32 < D) {
+  } else if (warp < 8) {
     // ------------------------------------------------------------------ dQ warps
-    const int dcol = (warp - 4) * 32 + lane;    // head-dim column == TMEM lane of dQ^T
+    const int qr = (warp - 4) * 32 + lane;     // query row within the tile == TMEM lane of dQ_i
     const uint32_t lane_base = uint32_t((warp - 4) * 32) << 16;
     for (int it = 0; it < n_it; ++it) {
       if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.dq_full), it & 1, abort, lim))) break;
       tc_fence_after();
-      uint32_t ra[32], rb[32];
-      tmem_ld32(tmem + lane_base + kTdQ, ra);
-      tmem_ld32(tmem + lane_base + kTdQ + 32, rb);
+      uint32_t v[D];
+#pragma unroll
+      for (int ch = 0; ch < D / 32; ++ch) tmem_ld32_async(tmem + lane_base + kTdQ + ch * 32, v + ch * 32);
+      tmem_ld_wait();
+      reg_fence<D>(v);
       tc_fence_before();
       mbar_arrive(smem_u32(&sm.dq_free));
       const int q0 = (i_begin + it) * kBwdRows;
-      float* acc = prm.dq_acc + (size_t(bh) * prm.Np + q0) * D + dcol;
+      float* acc = prm.dq_acc + (size_t(bh) * prm.Np + q0 + qr) * D;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) atomicAdd(acc + size_t(j) * D, __uint_as_float(ra[j]));
-#pragma unroll
-      for (int j = 0; j < 32; ++j) atomicAdd(acc + size_t(32 + j) * D, __uint_as_float(rb[j]));
+      for (int j = 0; j < D / 4; ++j) red_add_f4(acc + 4 * j, v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
     }
   }
 

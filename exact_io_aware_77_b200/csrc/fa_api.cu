@@ -157,7 +157,8 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.scale = scale;
   prm.wait_limit_ns = g_wait_limit_ns;
-  const int smem = int(sizeof(BwdSmem<D>)) + 1024;
+  static_assert(sizeof(BwdSmem<D>) <= 232448, "backward shared memory exceeds 227 KB");
+  const int smem = int(sizeof(BwdSmem<D>));   // the kernel checks that the base is 1 KB aligned
   if (set_smem(fa_bwd_kernel<D>, smem) != FA_OK) return FA_ERR_CUDA;
   fa_bwd_kernel<D><<<unsigned(prm.n_kv_tiles) * unsigned(BH), kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, prm);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
@@ -265,6 +266,7 @@ const char* fa_status_string(int status) {
     case FA_ERR_DEVICE: return "device is not compute capability 10.0 (B200)";
     case FA_ERR_TIMEOUT: return "a kernel-side wait timed out";
     case FA_ERR_SCALE: return "scale must be finite and > 0";
+    case FA_ERR_INTERNAL: return "kernel could not run as built (dynamic shared memory not 1 KB aligned)";
     case FA_ERR_NOALLOC_LIMIT: return "problem needs more than the 64 MiB built-in scratch of fa_bwd_noalloc";
     default: return "unknown status";
   }
@@ -275,6 +277,7 @@ int fa_check_status(void* stream) {
   int v = 0, zero = 0;
   if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
   if (v != 0 && cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+  if (v & FA_DEVICE_SMEM_ALIGN) return FA_ERR_INTERNAL;
   return v ? FA_ERR_TIMEOUT : FA_OK;
 }
 

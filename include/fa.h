@@ -63,7 +63,8 @@ typedef enum {
   FA_ERR_DEVICE = 8,     /* the current device is not compute capability 10.0 */
   FA_ERR_TIMEOUT = 9,    /* a kernel-side wait ran out of time (reported by fa_check_status) */
   FA_ERR_SCALE = 10,     /* scale is not finite and > 0 */
-  FA_ERR_NOALLOC_LIMIT = 11 /* fa_bwd_noalloc: fa_bwd_workspace_size(...) exceeds its 64 MiB scratch */
+  FA_ERR_NOALLOC_LIMIT = 11, /* fa_bwd_noalloc: fa_bwd_workspace_size(...) exceeds its 64 MiB scratch */
+  FA_ERR_INTERNAL = 12   /* a kernel found it could not run as built (reported by fa_check_status) */
 } fa_status;
 
 /*
@@ -76,7 +77,7 @@ FA_EXPORT int fa_fwd(const void* q, const void* k, const void* v, void* o, float
 
 /*
  * Bytes of device workspace fa_bwd needs: 4 * B*H * Np * (d + 2) with Np = N rounded up to
- * a multiple of 64 (per row: D, L in log2 units, and a d-wide fp32 dQ accumulator).
+ * a multiple of 128 (per row: D, L in log2 units, and a d-wide fp32 dQ accumulator).
  * Returns 0 when the shape itself is invalid.  O(N * d): no N x N buffer.
  */
 FA_EXPORT size_t fa_bwd_workspace_size(int B, int H, int N, int d);
@@ -99,7 +100,8 @@ FA_EXPORT const char* fa_status_string(int status);
 
 /*
  * Synchronises `stream`, then reads and clears the device status word of the current
- * device.  Returns FA_ERR_TIMEOUT if any kernel since the last check gave up on a
+ * device.  Returns FA_ERR_INTERNAL if a kernel since the last check refused to run (its
+ * dynamic shared memory was not 1 KB aligned), else FA_ERR_TIMEOUT if one gave up on a
  * bounded wait, FA_ERR_CUDA if the synchronisation failed, FA_OK otherwise.
  */
 FA_EXPORT int fa_check_status(void* stream);
@@ -130,7 +132,7 @@ FA_EXPORT int fa_selftest_timeout(unsigned long long limit_ns, void* stream);
  * loads the library holds until the process exits.  Problems whose
  * fa_bwd_workspace_size(B, H, N, d) exceeds 64 MiB (67108864 bytes) are rejected with
  * FA_ERR_NOALLOC_LIMIT before anything is enqueued; for d = 128 that allows
- * B*H*ceil(N/64)*64 <= 129055 rows, e.g. 31 heads of N = 4096.
+ * B*H*ceil(N/128)*128 <= 129055 rows, e.g. 31 heads of N = 4096.
  *
  * The first call on a device looks up the array's device address (cudaGetSymbolAddress,
  * with that device current), so make that first call before any stream capture begins.

@@ -76,7 +76,7 @@ def _bwd(ws_bytes=1 << 30, **kw):
 
 def test_workspace_size_formula(lib):
     for B, H, N, d in ((1, 1, 1, 64), (2, 32, 4096, 128), (1, 16, 32768, 128), (3, 5, 65, 64)):
-        np_ = (N + 63) // 64 * 64
+        np_ = (N + 127) // 128 * 128
         assert _lib.fa_bwd_workspace_size(B, H, N, d) == 4 * B * H * np_ * (d + 2)
     assert _lib.fa_bwd_workspace_size(1, 1, 0, 64) == 0
     assert _lib.fa_bwd_workspace_size(1, 1, 16, 80) == 0

@@ -97,7 +97,7 @@ def test_workspace_and_guard_bands(fa):
     bufs = [torch.full((n + 2 * pad,), 7.0, dtype=torch.bfloat16, device="cuda") for _ in range(3)]
     grads = tuple(b[pad:pad + n].view_as(q) for b in bufs)
     need = fa.bwd_workspace_size(1, 2, 300, 128)
-    assert need == 4 * 2 * 320 * (128 + 2)
+    assert need == 4 * 2 * 384 * (128 + 2)
     ws = torch.empty(need, dtype=torch.uint8, device="cuda")
     torch.cuda.synchronize()
     base = torch.cuda.memory_allocated()
