@@ -352,13 +352,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // arguments first; the mask (diagonal, window edge and tail tiles only) is one branch
         // around a separate loop that sets masked arguments to -inf, so exp2 gives exactly 0
         float x[64];
+        const uint64_t c2 = f2(c, c);
 #pragma unroll
-        for (int j4 = 0; j4 < 16; ++j4) {
-          const float4 l4 = *reinterpret_cast<const float4*>(lp + half * 64 + 4 * j4);
-          x[4 * j4 + 0] = fmaf(__uint_as_float(sr[4 * j4 + 0]), c, -l4.x);
-          x[4 * j4 + 1] = fmaf(__uint_as_float(sr[4 * j4 + 1]), c, -l4.y);
-          x[4 * j4 + 2] = fmaf(__uint_as_float(sr[4 * j4 + 2]), c, -l4.z);
-          x[4 * j4 + 3] = fmaf(__uint_as_float(sr[4 * j4 + 3]), c, -l4.w);
+        for (int j2 = 0; j2 < 32; ++j2) {
+          const float2 l2 = *reinterpret_cast<const float2*>(lp + half * 64 + 2 * j2);
+          f2_split(f2_fma(f2(__uint_as_float(sr[2 * j2]), __uint_as_float(sr[2 * j2 + 1])), c2, f2(-l2.x, -l2.y)),
+                   x[2 * j2], x[2 * j2 + 1]);
         }
         if (need_mask) {
           const int qbase = q0 + half * 64;
@@ -388,33 +387,33 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after();
       const float* ddp = sm.dd[qs];
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        // 32 queries per step: dP^T columns 384 + 32 q4 .. (read before any dS^T lands on them)
-        uint32_t dr[32];
-        tmem_ld32(tmem + lane_base + kTdP + q4 * 32, dr);
-        uint32_t pd[16];
+      for (int half = 0; half < 2; ++half) {
+        // 64 queries per step: dP^T columns 384 + 64 half .. (read before any dS^T lands on them)
+        uint32_t dr[64];
+        tmem_ld32_async(tmem + lane_base + kTdP + half * 64, dr);
+        tmem_ld32_async(tmem + lane_base + kTdP + half * 64 + 32, dr + 32);
+        tmem_ld_wait();
+        reg_fence<64>(dr);
+        uint32_t pd[32];
 #pragma unroll
-        for (int j4 = 0; j4 < 8; ++j4) {
-          const float4 d4 = *reinterpret_cast<const float4*>(ddp + q4 * 32 + 4 * j4);
-          const uint32_t w01 = pk_all[q4 * 16 + 2 * j4], w23 = pk_all[q4 * 16 + 2 * j4 + 1];
-          const float2 pa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w01));
-          const float2 pb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w23));
-          const float s0 = pa.x * (__uint_as_float(dr[4 * j4]) - d4.x);
-          const float s1 = pa.y * (__uint_as_float(dr[4 * j4 + 1]) - d4.y);
-          const float s2 = pb.x * (__uint_as_float(dr[4 * j4 + 2]) - d4.z);
-          const float s3 = pb.y * (__uint_as_float(dr[4 * j4 + 3]) - d4.w);
-          pd[2 * j4] = pack_bf16x2(s0, s1);
-          pd[2 * j4 + 1] = pack_bf16x2(s2, s3);
+        for (int j2 = 0; j2 < 32; ++j2) {
+          // (dP - D) * P on pairs; P comes back from its packed bf16 form (a shift per half)
+          const float2 d2 = *reinterpret_cast<const float2*>(ddp + half * 64 + 2 * j2);
+          const uint32_t w = pk_all[half * 32 + j2];
+          const uint64_t p2 = f2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+          const uint64_t t2 = f2_add(f2(__uint_as_float(dr[2 * j2]), __uint_as_float(dr[2 * j2 + 1])), f2(-d2.x, -d2.y));
+          float s0, s1;
+          f2_split(f2_mul(t2, p2), s0, s1);
+          pd[j2] = pack_bf16x2(s0, s1);
         }
-        // TMEM copy for the dK MMA: packed columns kTdS + 16 q4 (inside dP^T columns already read)
-        tmem_st16(tmem + lane_base + kTdS + q4 * 16, pd);
-        // shared-memory copy for the dQ MMA: queries 32 q4.. = half a 128-byte row of chunk q4 / 2
+        // TMEM copy for the dK MMA: packed columns kTdS + 32 half (inside dP^T columns already read)
+        tmem_st16(tmem + lane_base + kTdS + half * 32, pd);
+        tmem_st16(tmem + lane_base + kTdS + half * 32 + 16, pd + 16);
+        // shared-memory copy for the dQ MMA: queries 64 half.. = one 128-byte row of chunk `half`
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          const int piece = (q4 & 1) * 4 + c4;
-          st_shared_v4(ds_row + (q4 >> 1) * 16384 + ((piece ^ sw) << 4), pd[4 * c4], pd[4 * c4 + 1],
-                       pd[4 * c4 + 2], pd[4 * c4 + 3]);
-        }
+        for (int c16 = 0; c16 < 8; ++c16)
+          st_shared_v4(ds_row + half * 16384 + ((c16 ^ sw) << 4), pd[4 * c16], pd[4 * c16 + 1], pd[4 * c16 + 2],
+                       pd[4 * c16 + 3]);
       }
       tmem_st_wait();
       fence_proxy_async_smem();
