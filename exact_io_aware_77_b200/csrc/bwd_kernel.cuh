@@ -250,7 +250,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else if (warp == kBwdWarpMma) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // the whole warp runs this loop (uniformly); each tcgen05 op is issued by one elected lane
+    {
+      auto wait = [&](uint32_t bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, lim));
+      };
       constexpr uint32_t idesc_t = idesc_bf16_f32(128, kBwdRows, false, false);   // S^T, dP^T
       constexpr uint32_t idesc_kv = idesc_bf16_f32(128, D, false, true);          // dV, dK (A in TMEM)
       constexpr uint32_t idesc_q = idesc_bf16_f32(kBwdRows, D, true, true);       // dQ
@@ -264,7 +268,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_bf16_ss(tmem + d_col, desc_advance(a, off), desc_advance(b, off), idesc_t, kk > 0);
+          mma_bf16_ss_w(tmem + d_col, desc_advance(a, off), desc_advance(b, off), idesc_t, kk > 0);
         }
       };
       // acc += A(TMEM, 128 x 128 queries) * B (MN-major Q_i or dO_i: 16 queries = 2 KB per k-step)
@@ -272,53 +276,53 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint64_t b = sw128_desc(smem_u32(b_tile), 16384, 1024);
 #pragma unroll
         for (int kk = 0; kk < kBwdRows / 16; ++kk)
-          mma_bf16_ts(tmem + d_col, tmem + a_col + kk * 8, desc_advance(b, kk * 2048), idesc_kv,
+          mma_bf16_ts_w(tmem + d_col, tmem + a_col + kk * 8, desc_advance(b, kk * 2048), idesc_kv,
                       (first && kk == 0) ? 0u : 1u);
       };
-      bool ok = mbar_wait(smem_u32(&sm.kv_full), 0, abort, lim) && mbar_wait(smem_u32(&sm.q_full[0]), 0, abort, lim);
+      bool ok = wait(smem_u32(&sm.kv_full), 0) && wait(smem_u32(&sm.q_full[0]), 0);
       if (ok) {
         tc_fence_after();
         issue_t(dk_kmaj, sm.q[0], kTS);
-        mma_commit(smem_u32(&sm.s_full));
+        mma_commit_w(smem_u32(&sm.s_full));
         issue_t(dv_kmaj, sm.dout[0], kTdP);
-        mma_commit(smem_u32(&sm.dp_full));
+        mma_commit_w(smem_u32(&sm.dp_full));
       }
       for (int it = 0; ok && it < n_it; ++it) {
         const int qs = it % kBwdQStages;
         const bool has_next = it + 1 < n_it;
         const int qn = (it + 1) % kBwdQStages;
         // dV += P^T dO_i
-        if (!mbar_wait(smem_u32(&sm.pa_full), it & 1, abort, lim)) break;
+        if (!wait(smem_u32(&sm.pa_full), it & 1)) break;
         tc_fence_after();
         issue_kv(kTP, sm.dout[qs], kTdV, it == 0);
         // S^T of the next tile (overwrites P^T only after dV above has read it)
         if (has_next) {
-          if (!mbar_wait(smem_u32(&sm.q_full[qn]), ((it + 1) / kBwdQStages) & 1, abort, lim)) break;
+          if (!wait(smem_u32(&sm.q_full[qn]), ((it + 1) / kBwdQStages) & 1)) break;
           issue_t(dk_kmaj, sm.q[qn], kTS);
-          mma_commit(smem_u32(&sm.s_full));
+          mma_commit_w(smem_u32(&sm.s_full));
         }
         // dK += dS^T Q_i, then dQ_i = dS_i K (A = dS^T from shared memory, MN-major over queries)
-        if (!mbar_wait(smem_u32(&sm.ds_full), it & 1, abort, lim)) break;
+        if (!wait(smem_u32(&sm.ds_full), it & 1)) break;
         tc_fence_after();
         issue_kv(kTdS, sm.q[qs], kTdK, it == 0);
-        if (!mbar_wait(smem_u32(&sm.dq_free), (it & 1) ^ 1, abort, lim)) break;
+        if (!wait(smem_u32(&sm.dq_free), (it & 1) ^ 1)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kBwdKeys / 16; ++kk)
-          mma_bf16_ss(tmem + kTdQ, desc_advance(dds_mn, kk * 2048), desc_advance(dk_mn, kk * 2048), idesc_q, kk > 0);
-        mma_commit(smem_u32(&sm.dq_full));
-        mma_commit(smem_u32(&sm.ds_free));
-        mma_commit(smem_u32(&sm.q_empty[qs]));
+          mma_bf16_ss_w(tmem + kTdQ, desc_advance(dds_mn, kk * 2048), desc_advance(dk_mn, kk * 2048), idesc_q, kk > 0);
+        mma_commit_w(smem_u32(&sm.dq_full));
+        mma_commit_w(smem_u32(&sm.ds_free));
+        mma_commit_w(smem_u32(&sm.q_empty[qs]));
         // dP^T of the next tile once dQ_i has been read out of the same columns
         if (has_next) {
-          if (!mbar_wait(smem_u32(&sm.dq_free), it & 1, abort, lim)) break;
+          if (!wait(smem_u32(&sm.dq_free), it & 1)) break;
           tc_fence_after();
           issue_t(dv_kmaj, sm.dout[qn], kTdP);
-          mma_commit(smem_u32(&sm.dp_full));
+          mma_commit_w(smem_u32(&sm.dp_full));
         }
       }
-      mma_commit(smem_u32(&sm.mma_final));
-      mma_commit(smem_u32(&sm.mma_drain));
+      mma_commit_w(smem_u32(&sm.mma_final));
+      mma_commit_w(smem_u32(&sm.mma_drain));
       mbar_wait_drain(smem_u32(&sm.mma_drain), 0, lim);
     }
   } else if (warp < 4) {

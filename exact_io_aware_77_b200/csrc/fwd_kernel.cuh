@@ -168,7 +168,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // the whole warp runs this loop (uniformly); each tcgen05 op is issued by one elected lane
+    {
+      auto wait = [&](uint32_t bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, lim));
+      };
       constexpr uint32_t idesc_s = idesc_bf16_f32(kBlockM, kBlockN, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(kBlockM, D, false, true);
       const int bw[2] = {b0, b1}, ew[2] = {e0, e1};
@@ -185,9 +189,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           // K-major operands: 16-element k-steps are 32 bytes apart inside a 128-byte row,
           // 64-element chunks are separate 16 KB tiles
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_bf16_ss(tmem + w * 128, desc_advance(dq[w], off), desc_advance(dk, off), idesc_s, kk > 0);
+          mma_bf16_ss_w(tmem + w * 128, desc_advance(dq[w], off), desc_advance(dk, off), idesc_s, kk > 0);
         }
-        mma_commit(smem_u32(&sm.s_full[w]));
+        mma_commit_w(smem_u32(&sm.s_full[w]));
       };
       auto issue_pv = [&](int w, uint32_t slot) {
         const uint64_t dv = desc_advance(dv0, slot * Smem::kTileBytes);
@@ -196,33 +200,33 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int kk = 0; kk < kBlockN / 16; ++kk) {
           // A = P from TMEM (16 keys = 8 packed columns per k-step); B = V MN-major: 16 keys =
           // 16 rows of 128 bytes, the next 64 head-dim columns one 16 KB chunk (LBO) further
-          mma_bf16_ts(tmem + 256 + w * 128, tmem + w * 128 + kk * 8, desc_advance(dv, kk * 2048), idesc_o,
+          mma_bf16_ts_w(tmem + 256 + w * 128, tmem + w * 128 + kk * 8, desc_advance(dv, kk * 2048), idesc_o,
                       kk > 0 ? 1u : acc);
         }
         ++pv_count[w];
       };
-      bool ok = mbar_wait(smem_u32(&sm.q_full), 0, abort, lim);
+      bool ok = wait(smem_u32(&sm.q_full), 0);
       // prologue: S of the first KV tile
       if (ok) {
-        ok = mbar_wait(smem_u32(&sm.slot_full[0]), 0, abort, lim);
+        ok = wait(smem_u32(&sm.slot_full[0]), 0);
         if (ok) {
           tc_fence_after();
 #pragma unroll
           for (int w = 0; w < kQTiles; ++w)
             if (active(w, t_begin)) issue_s(w, 0);
-          mma_commit(smem_u32(&sm.slot_empty[0]));
+          mma_commit_w(smem_u32(&sm.slot_empty[0]));
         }
       }
       for (int t = t_begin; ok && t < t_end; ++t) {
         const int Lv = 2 * (t - t_begin) + 1;   // V of tile t
         const int Lk = Lv + 1;                  // K of tile t + 1
         const bool has_next = t + 1 < t_end;
-        if (!mbar_wait(smem_u32(&sm.slot_full[Lv % kSlots]), (Lv / kSlots) & 1, abort, lim)) break;
-        if (has_next && !mbar_wait(smem_u32(&sm.slot_full[Lk % kSlots]), (Lk / kSlots) & 1, abort, lim)) break;
+        if (!wait(smem_u32(&sm.slot_full[Lv % kSlots]), (Lv / kSlots) & 1)) break;
+        if (has_next && !wait(smem_u32(&sm.slot_full[Lk % kSlots]), (Lk / kSlots) & 1)) break;
 #pragma unroll
         for (int w = 0; w < kQTiles; ++w) {
           if (active(w, t)) {
-            if (!mbar_wait(smem_u32(&sm.p_full[w]), pv_count[w] & 1, abort, lim)) {
+            if (!wait(smem_u32(&sm.p_full[w]), pv_count[w] & 1)) {
               ok = false;
               break;
             }
@@ -232,13 +236,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           if (has_next && active(w, t + 1)) issue_s(w, Lk % kSlots);
         }
         if (!ok) break;
-        if (has_next) mma_commit(smem_u32(&sm.slot_empty[Lk % kSlots]));
-        mma_commit(smem_u32(&sm.slot_empty[Lv % kSlots]));
+        if (has_next) mma_commit_w(smem_u32(&sm.slot_empty[Lk % kSlots]));
+        mma_commit_w(smem_u32(&sm.slot_empty[Lv % kSlots]));
       }
 #pragma unroll
-      for (int w = 0; w < kQTiles; ++w) mma_commit(smem_u32(&sm.o_final[w]));
+      for (int w = 0; w < kQTiles; ++w) mma_commit_w(smem_u32(&sm.o_final[w]));
       // every MMA issued above completes before TMEM is released
-      mma_commit(smem_u32(&sm.mma_drain));
+      mma_commit_w(smem_u32(&sm.mma_drain));
       mbar_wait_drain(smem_u32(&sm.mma_drain), 0, lim);
     }
   } else {
