@@ -66,8 +66,12 @@ def bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
 
 
 def backward(q, k, v, o, lse, do, scale: float | None = None, causal: bool = False, window: int = 0,
-             grads=None, workspace=None):
-    """dQ, dK, dV (bf16 [B,H,N,d]) of sum(O o dO), recomputing P from the forward's L."""
+             grads=None, workspace=None, phases: int = 7):
+    """dQ, dK, dV (bf16 [B,H,N,d]) of sum(O o dO), recomputing P from the forward's L.
+
+    ``phases`` selects the steps of the backward (1 preprocess, 2 recompute kernel, 4 dQ
+    finalise); running 1, 2, 4 in turn with the same workspace equals the default 7.
+    """
     import torch
     _check_qkv(q, k, v, o, do)
     B, H, N, d = q.shape
@@ -80,11 +84,13 @@ def backward(q, k, v, o, lse, do, scale: float | None = None, causal: bool = Fal
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     dq, dk, dv = grads
-    st = _lib.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                     do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, scale,
-                     int(bool(causal)), int(window), workspace.data_ptr(),
-                     workspace.numel() * workspace.element_size(), _stream_handle(q.device))
-    _raise("fa_bwd", st)
+    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+            dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, scale, int(bool(causal)), int(window),
+            workspace.data_ptr(), workspace.numel() * workspace.element_size())
+    if phases == 7:
+        _raise("fa_bwd", _lib.fa_bwd(*args, _stream_handle(q.device)))
+    else:
+        _raise("fa_bwd_phases", _lib.fa_bwd_phases(*args, int(phases), _stream_handle(q.device)))
     return dq, dk, dv
 
 

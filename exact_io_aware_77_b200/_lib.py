@@ -19,7 +19,7 @@ STATUS_NAMES = {
     0: "FA_OK", 1: "FA_ERR_NULL", 2: "FA_ERR_SHAPE", 3: "FA_ERR_HEADDIM", 4: "FA_ERR_ALIGN",
     5: "FA_ERR_MASK", 6: "FA_ERR_WORKSPACE", 7: "FA_ERR_CUDA", 8: "FA_ERR_DEVICE",
     9: "FA_ERR_TIMEOUT", 10: "FA_ERR_SCALE", 11: "FA_ERR_NOALLOC_LIMIT",
-    12: "FA_ERR_INTERNAL",
+    12: "FA_ERR_INTERNAL", 13: "FA_ERR_PHASES",
 }
 STATUS = {v: k for k, v in STATUS_NAMES.items()}
 
@@ -32,6 +32,8 @@ SIGNATURES = {
     "fa_bwd_workspace_size": (_c_size_t, [_c_int] * 4),
     "fa_bwd": (_c_int, [_c_void_p] * 9 + [_c_int] * 4 + [_c_float, _c_int, _c_int, _c_void_p, _c_size_t,
                                                          _c_void_p]),
+    "fa_bwd_phases": (_c_int, [_c_void_p] * 9 + [_c_int] * 4 + [_c_float, _c_int, _c_int, _c_void_p, _c_size_t,
+                                                                _c_int, _c_void_p]),
     "fa_bwd_noalloc": (_c_int, [_c_void_p] * 9 + [_c_int] * 4 + [_c_float, _c_int, _c_int, _c_void_p]),
     "fa_status_string": (ctypes.c_char_p, [_c_int]),
     "fa_check_status": (_c_int, [_c_void_p]),
@@ -92,6 +94,12 @@ def fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal, window, w
            workspace_bytes, stream) -> int:
     return _call("fa_bwd", q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal, window,
                  workspace, workspace_bytes, stream)
+
+
+def fa_bwd_phases(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal, window, workspace,
+                  workspace_bytes, phases, stream) -> int:
+    return _call("fa_bwd_phases", q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal, window,
+                 workspace, workspace_bytes, phases, stream)
 
 
 def fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal, window, stream) -> int:

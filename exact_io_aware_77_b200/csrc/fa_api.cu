@@ -115,6 +115,8 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
 }
 
 // ---------------------------------------------------------------- backward
+constexpr int kBwdPhasePrep = 1, kBwdPhaseMain = 2, kBwdPhaseFinal = 4, kBwdAllPhases = 7;
+
 long long padded_rows(int N) { return ((long long)N + kBwdRows - 1) / kBwdRows * kBwdRows; }
 
 size_t bwd_workspace_bytes(long long BH, int N, int d) {
@@ -124,13 +126,13 @@ size_t bwd_workspace_bytes(long long BH, int N, int d) {
 template <int D>
 int launch_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
                void* dq, void* dk, void* dv, int BH, int N, float scale, int causal, int window, void* ws,
-               cudaStream_t stream) {
+               cudaStream_t stream, int phases = kBwdAllPhases) {
   const long long Np = padded_rows(N);
   float* lp = static_cast<float*>(ws);
   float* dd = lp + size_t(BH) * Np;
   float* dq_acc = dd + size_t(BH) * Np;
   constexpr int G = D / 8;
-  {
+  if (phases & kBwdPhasePrep) {
     const long long rows = (long long)BH * Np;
     const long long blocks = (rows + (256 / G) - 1) / (256 / G);
     fa_bwd_prep<D><<<unsigned(blocks), 256, 0, stream>>>(
@@ -138,6 +140,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
         int(Np), rows);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
+  if (phases & kBwdPhaseMain) {
   CUtensorMap tq, tk, tv, tdo;
   if (!make_map_bf16(&tq, q, D, N, BH, kBwdRows) || !make_map_bf16(&tk, k, D, N, BH, kBwdKeys) ||
       !make_map_bf16(&tv, v, D, N, BH, kBwdKeys) || !make_map_bf16(&tdo, dout, D, N, BH, kBwdRows))
@@ -162,7 +165,8 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   if (set_smem(fa_bwd_kernel<D>, smem) != FA_OK) return FA_ERR_CUDA;
   fa_bwd_kernel<D><<<unsigned(prm.n_kv_tiles) * unsigned(BH), kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, prm);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
-  {
+  }
+  if (phases & kBwdPhaseFinal) {
     const long long rows = (long long)BH * N;
     const long long blocks = (rows + (256 / G) - 1) / (256 / G);
     fa_bwd_dq_final<D><<<unsigned(blocks), 256, 0, stream>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), N, int(Np),
@@ -237,6 +241,14 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout, void* dq,
            void* dk, void* dv, int B, int H, int N, int d, float scale, int causal, int window, void* workspace,
            size_t workspace_bytes, void* stream) {
+  return fa_bwd_phases(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, window, workspace,
+                       workspace_bytes, kBwdAllPhases, stream);
+}
+
+int fa_bwd_phases(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                  void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal, int window,
+                  void* workspace, size_t workspace_bytes, int phases, void* stream) {
+  if (phases < 1 || phases > kBwdAllPhases) return FA_ERR_PHASES;
   if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FA_ERR_NULL;
   int st = check_problem(B, H, N, d, scale, causal, window);
   if (st != FA_OK) return st;
@@ -248,9 +260,10 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
     return FA_ERR_ALIGN;
   if ((st = check_device()) != FA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return d == 64 ? launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, int(BH), N, scale, causal, window, workspace, s)
+  return d == 64 ? launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, int(BH), N, scale, causal, window, workspace, s,
+                                  phases)
                  : launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, int(BH), N, scale, causal, window, workspace,
-                                   s);
+                                   s, phases);
 }
 
 const char* fa_status_string(int status) {
@@ -266,6 +279,7 @@ const char* fa_status_string(int status) {
     case FA_ERR_DEVICE: return "device is not compute capability 10.0 (B200)";
     case FA_ERR_TIMEOUT: return "a kernel-side wait timed out";
     case FA_ERR_SCALE: return "scale must be finite and > 0";
+    case FA_ERR_PHASES: return "phase mask must be a non-empty subset of 1 | 2 | 4";
     case FA_ERR_INTERNAL: return "kernel could not run as built (dynamic shared memory not 1 KB aligned)";
     case FA_ERR_NOALLOC_LIMIT: return "problem needs more than the 64 MiB built-in scratch of fa_bwd_noalloc";
     default: return "unknown status";

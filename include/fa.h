@@ -64,7 +64,8 @@ typedef enum {
   FA_ERR_TIMEOUT = 9,    /* a kernel-side wait ran out of time (reported by fa_check_status) */
   FA_ERR_SCALE = 10,     /* scale is not finite and > 0 */
   FA_ERR_NOALLOC_LIMIT = 11, /* fa_bwd_noalloc: fa_bwd_workspace_size(...) exceeds its 64 MiB scratch */
-  FA_ERR_INTERNAL = 12   /* a kernel found it could not run as built (reported by fa_check_status) */
+  FA_ERR_INTERNAL = 12,  /* a kernel found it could not run as built (reported by fa_check_status) */
+  FA_ERR_PHASES = 13     /* fa_bwd_phases: phase mask outside 1..7 */
 } fa_status;
 
 /*
@@ -94,6 +95,22 @@ FA_EXPORT size_t fa_bwd_workspace_size(int B, int H, int N, int d);
 FA_EXPORT int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
                      void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal, int window,
                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * The backward pass split into its three phases, so that a caller can time or interleave
+ * them.  `phases` is a mask of
+ *   1  preprocess: D = rowsum(dO o O), L in log2 units and a cleared fp32 dQ accumulator,
+ *      all in `workspace`;
+ *   2  the recompute kernel: dK and dV written, dQ accumulated in `workspace`;
+ *   4  finalise: dQ = scale * accumulator, written as bf16.
+ * Calling it with 1, then 2, then 4 on one stream with the same arguments and workspace
+ * does exactly what one fa_bwd call (mask 7) does.  Arguments, validation and errors are
+ * fa_bwd's; a mask outside 1..7 gives FA_ERR_PHASES.
+ */
+FA_EXPORT int fa_bwd_phases(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                            const void* dO, void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale,
+                            int causal, int window, void* workspace, size_t workspace_bytes, int phases,
+                            void* stream);
 
 /* Human-readable name of a status code (static string, never NULL). */
 FA_EXPORT const char* fa_status_string(int status);

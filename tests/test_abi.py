@@ -96,3 +96,10 @@ def test_workspace_size_formula(lib):
 ])
 def test_bwd_rejects_bad_arguments(lib, kw, code):
     assert _lib.STATUS_NAMES[_bwd(**kw)] == code
+
+
+@pytest.mark.parametrize("phases", [0, 8, -1])
+def test_bwd_phases_rejects_bad_mask(lib, phases):
+    ptrs = [A + 4096 * i for i in range(9)]
+    st = _lib.fa_bwd_phases(*ptrs, 1, 2, 128, 64, 0.125, 0, 0, A + 65536, 1 << 30, phases, None)
+    assert _lib.STATUS_NAMES[st] == "FA_ERR_PHASES"
