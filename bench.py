@@ -67,6 +67,25 @@ def bwd_flops(B, H, N, d, causal) -> float:
     return 2.5 * fwd_flops(B, H, N, d, causal)
 
 
+def max_over_ranks(values, device=None):
+    """Element-wise max of a list of floats over all ranks (identity without a process group).
+
+    Every rank calls it with the same number of values at the same point of the program.
+    """
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return list(values)
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(world: int, flops_per_rank_step: float, ms_per_step: float) -> float:
+    """Whole-job TFLOP/s: every rank processed its own copy of the workload in ms_per_step."""
+    return world * flops_per_rank_step / (ms_per_step * 1e-3) / 1e12
+
+
 def load_peaks():
     try:
         with open(PEAKS_FILE) as f:
@@ -284,12 +303,10 @@ def run_ours(args):
     main_ms = [e[2].elapsed_time(e[3]) for e in events] if has_bwd else [0.0] * args.steps
     step_ms_total = sum(f + b for f, b in zip(fwd_ms, bwd_ms))
     fwd_total, bwd_total, main_total = sum(fwd_ms), sum(bwd_ms), sum(main_ms)
-    if world > 1:
-        t = torch.tensor([step_ms_total, fwd_total, bwd_total, main_total], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        step_ms_total, fwd_total, bwd_total, main_total = t.tolist()
+    step_ms_total, fwd_total, bwd_total, main_total = max_over_ranks(
+        [step_ms_total, fwd_total, bwd_total, main_total], dev)
     ms_per_step = step_ms_total / args.steps
-    value = world * (f_fwd + f_bwd) / (ms_per_step * 1e-3) / 1e12
+    value = job_throughput(world, f_fwd + f_bwd, ms_per_step)
 
     # end to end through the public API: pinned host inputs -> device -> path -> host outputs
     e2e = None
@@ -333,7 +350,7 @@ def run_ours(args):
                    f": B={B} H={H} N={N} d={d} causal, inputs N(0,1)*0.5 bf16 seeded",
                    "global_batch": B * world, "seq_len": N, "parallelism": f"replicas{world}",
                    "l2": "flushed (256 MB write) between timed steps, outside the events"},
-        "fwd_tflops": round(world * f_fwd / (fwd_ms_avg * 1e-3) / 1e12, 2),
+        "fwd_tflops": round(job_throughput(world, f_fwd, fwd_ms_avg), 2),
         "fwd_ms": round(fwd_ms_avg, 4),
         "pct_of_measured_peak": round(100 * value / world / peaks["bf16_tflops"], 2),
         "pct_of_spec_peak_2250": round(100 * value / world / 2250.0, 2),
@@ -347,7 +364,7 @@ def run_ours(args):
         "clocks": clocks,
     }
     if has_bwd:
-        line["bwd_tflops"] = round(world * f_bwd / (bwd_ms_avg * 1e-3) / 1e12, 2)
+        line["bwd_tflops"] = round(job_throughput(world, f_bwd, bwd_ms_avg), 2)
         line["bwd_ms"] = round(bwd_ms_avg, 4)
     if world > 1:
         dist.barrier()
@@ -393,13 +410,8 @@ def measure_e2e(fa, torch, wl, dev, stream, q_h, k_h, v_h, do_h, has_bwd, steps,
         one()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    ms = e0.elapsed_time(e1) / steps
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = t.item()
-    return {"value": round(world * flops / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+    ms = max_over_ranks([e0.elapsed_time(e1) / steps], dev)[0]
+    return {"value": round(job_throughput(world, flops, ms), 3), "unit": "TFLOP/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 3)}
 
 
