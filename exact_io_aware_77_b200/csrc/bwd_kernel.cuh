@@ -22,13 +22,16 @@
 //               (dV and dK read their A operand from TMEM), so that the exponentials of tile
 //               i+1 run while dK_i and dQ_i are computed, and dS of tile i+1 while dV_{i+1}
 //               and S_{i+2} are.
-//   warps 0-3   thread t owns key kv0 + t (TMEM lane t).  Phase A: P^T = exp2(S^T c - L) with
-//               the causal/window mask, stored to TMEM as bf16.  Phase B: dS^T = P^T o (dP^T - D)
-//               to TMEM (A of dK) and to shared memory (A of dQ).  At the end: dK, dV.
-//   warps 4-7   thread t owns query q0 + t of dQ_i (TMEM lane t) and adds its row into the fp32
-//               accumulator with 16-byte vector reductions.
-// TMEM columns: dK [0,128), dV [128,256), S^T [256,384) with P^T in [256,320) once read,
-// dP^T [384,512) with dS^T in [384,448) once read, and dQ in [384,512).  MMAs of one thread
+//   warps 0-7   two per TMEM lane quadrant; warp w owns lanes 32 (w % 4).. and the query half
+//               w / 4 of each tile.  Phase A: P^T = exp2(S^T c - L) with the causal/window mask,
+//               stored to TMEM as bf16.  Phase B: dS^T = P^T o (dP^T - D) to TMEM (A of dK) and
+//               to shared memory (A of dQ).  Readout: its half of the dQ_i rows of its 32
+//               queries, staged in shared memory and added into the fp32 accumulator by a TMA
+//               tensor reduce-add.
+//               Order per tile: B(i), A(i+1), readout(i).  At the end: dK (half 0), dV (half 1).
+// TMEM columns: dK [0,128), dV [128,256), S^T [256,384) with P^T in [256,288) and [320,352)
+// once read, dP^T [384,512) with dS^T in [384,416) and [448,480) once read, and dQ in
+// [384,512).  MMAs of one thread
 // run in order, which makes each reuse safe: S_{i+1} is issued after dV_i read P_i, dQ_i after
 // dK_i read dS_i; only dP_{i+1} waits until warps 4-7 have read dQ_i out.
 #pragma once
@@ -72,6 +75,7 @@ struct BwdSmem {
   alignas(8) uint64_t kv_full;
   uint64_t q_full[kBwdQStages], q_empty[kBwdQStages];
   uint64_t s_full, dp_full, pa_full, ds_full, ds_free, dq_full, dq_free, mma_final, mma_drain;
+  uint64_t slice_free[4], staging_done;   // dQ staging in the dS buffer (see the readout)
   uint32_t tmem_base;
   int abort;
 };
@@ -79,11 +83,6 @@ struct BwdSmem {
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
                "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
-               : "memory");
-}
-__device__ __forceinline__ void red_add_f4(float* addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(__uint_as_float(a)),
-               "f"(__uint_as_float(b)), "f"(__uint_as_float(c)), "f"(__uint_as_float(d))
                : "memory");
 }
 
@@ -164,7 +163,7 @@ template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                  const BwdParams prm) {
+                  const __grid_constant__ CUtensorMap tm_dq, const BwdParams prm) {
   using Smem = BwdSmem<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // the layout fills almost all 227 KB, so no slack is left for realigning the base
@@ -194,13 +193,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     mbar_init(smem_u32(&sm.s_full), 1);
     mbar_init(smem_u32(&sm.dp_full), 1);
-    mbar_init(smem_u32(&sm.pa_full), 128);
-    mbar_init(smem_u32(&sm.ds_full), 128);
+    mbar_init(smem_u32(&sm.pa_full), 256);
+    mbar_init(smem_u32(&sm.ds_full), 256);
     mbar_init(smem_u32(&sm.ds_free), 1);
     mbar_init(smem_u32(&sm.dq_full), 1);
-    mbar_init(smem_u32(&sm.dq_free), 128);
+    mbar_init(smem_u32(&sm.dq_free), 256);
     mbar_init(smem_u32(&sm.mma_final), 1);
     mbar_init(smem_u32(&sm.mma_drain), 1);
+    for (int qd = 0; qd < 4; ++qd) mbar_init(smem_u32(&sm.slice_free[qd]), 1);
+    mbar_init(smem_u32(&sm.staging_done), 4);
     fence_mbar_init();
   }
   if (warp == kBwdWarpTma && lane == 0) {
@@ -208,6 +209,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
     tma_prefetch_desc(&tm_do);
+    tma_prefetch_desc(&tm_dq);
   }
   if (warp == kBwdWarpMma) {
     tmem_alloc(smem_u32(&sm.tmem_base), 512);
@@ -272,12 +274,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       };
       // acc += A(TMEM, 128 x 128 queries) * B (MN-major Q_i or dO_i: 16 queries = 2 KB per k-step)
+      // A (P^T or dS^T) sits in TMEM as two 32-column halves, one per query half, at a_col and
+      // a_col + 64; each 16-query k-step takes 8 of those columns
       auto issue_kv = [&](uint32_t a_col, const uint8_t* b_tile, uint32_t d_col, bool first) {
         const uint64_t b = sw128_desc(smem_u32(b_tile), 16384, 1024);
 #pragma unroll
         for (int kk = 0; kk < kBwdRows / 16; ++kk)
-          mma_bf16_ts_w(tmem + d_col, tmem + a_col + kk * 8, desc_advance(b, kk * 2048), idesc_kv,
-                      (first && kk == 0) ? 0u : 1u);
+          mma_bf16_ts_w(tmem + d_col, tmem + a_col + (kk >> 2) * 64 + (kk & 3) * 8, desc_advance(b, kk * 2048),
+                        idesc_kv, (first && kk == 0) ? 0u : 1u);
       };
       bool ok = wait(smem_u32(&sm.kv_full), 0) && wait(smem_u32(&sm.q_full[0]), 0);
       if (ok) {
@@ -325,149 +329,179 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mma_commit_w(smem_u32(&sm.mma_drain));
       mbar_wait_drain(smem_u32(&sm.mma_drain), 0, lim);
     }
-  } else if (warp < 4) {
-    // ------------------------------------------------------------------ P^T / dS^T warps
-    const int r = threadIdx.x;                 // key row within the tile == TMEM lane
+  } else if (warp < 8) {
+    // ------------------------------------------------------------------ compute warps
+    // Two warps per TMEM lane quadrant: warp w owns lanes 32 (w % 4) .. (keys for S^T, dP^T;
+    // queries for dQ) and query half hq = w / 4 (queries 64 hq .. 64 hq + 63 of each tile).
+    const int quad = warp & 3;
+    const int hq = warp >> 2;
+    const int r = quad * 32 + lane;            // key row of S^T / dP^T, query row of dQ
     const int key = kv0 + r;
-    const uint32_t lane_base = uint32_t(warp * 32) << 16;
+    const uint32_t lane_base = uint32_t(quad * 32) << 16;
     const float c = prm.scale_log2;
-    const uint32_t ds_row = smem_u32(sm.ds) + r * 128;
+    const uint32_t col_s = kTS + hq * 64;      // my S^T columns; P^T goes to the first 32 of them
+    const uint32_t col_dp = kTdP + hq * 64;    // my dP^T columns; dS^T goes to the first 32 of them
+    const uint32_t col_dq = kTdQ + hq * (D / 2);
+    const uint32_t ds_row = smem_u32(sm.ds) + hq * 16384 + r * 128;   // 64 queries = one 128-byte row
     const uint32_t sw = r & 7;
+    uint32_t pk[32];                           // packed P^T of the current tile (phase A -> phase B)
     bool ok = true;
-    for (int it = 0; it < n_it; ++it) {
+
+    // phase A: P^T = 2^(S^T c - L) for my 64 queries -> TMEM (bf16) and pk
+    auto phase_a = [&](int it) -> bool {
       const int qs = it % kBwdQStages;
       const int q0 = (i_begin + it) * kBwdRows;
-      // ---- phase A: P^T = 2^(S^T c - L) -> TMEM (bf16)
       bool w_ok = mbar_wait(smem_u32(&sm.q_full[qs]), (it / kBwdQStages) & 1, abort, lim);
       w_ok = w_ok && mbar_wait(smem_u32(&sm.s_full), it & 1, abort, lim);
-      if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, w_ok)) return false;
       tc_fence_after();
-      const bool need_mask = (prm.causal && kv0 + kBwdKeys - 1 > q0) ||
-                             (prm.window > 0 && kv0 < q0 + kBwdRows - prm.window) || (kv0 + kBwdKeys > prm.N);
-      const float* lp = sm.lp[qs];
-      uint32_t pk_all[64];   // packed P^T of this tile, kept for phase B (S_{i+1} may overwrite TMEM)
+      uint32_t sr[64];
+      tmem_ld32_async(tmem + lane_base + col_s, sr);
+      tmem_ld32_async(tmem + lane_base + col_s + 32, sr + 32);
+      tmem_ld_wait();
+      reg_fence<64>(sr);
+      const float* lp = sm.lp[qs] + hq * 64;
+      float x[64];
+      const uint64_t c2 = f2(c, c);
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t sr[64];
-        tmem_ld32_async(tmem + lane_base + kTS + half * 64, sr);
-        tmem_ld32_async(tmem + lane_base + kTS + half * 64 + 32, sr + 32);
-        tmem_ld_wait();
-        reg_fence<64>(sr);
-        // arguments first; the mask (diagonal, window edge and tail tiles only) is one branch
-        // around a separate loop that sets masked arguments to -inf, so exp2 gives exactly 0
-        float x[64];
-        const uint64_t c2 = f2(c, c);
-#pragma unroll
-        for (int j2 = 0; j2 < 32; ++j2) {
-          const float2 l2 = *reinterpret_cast<const float2*>(lp + half * 64 + 2 * j2);
-          f2_split(f2_fma(f2(__uint_as_float(sr[2 * j2]), __uint_as_float(sr[2 * j2 + 1])), c2, f2(-l2.x, -l2.y)),
-                   x[2 * j2], x[2 * j2 + 1]);
-        }
-        if (need_mask) {
-          const int qbase = q0 + half * 64;
-#pragma unroll
-          for (int j = 0; j < 64; ++j) {
-            const int qq = qbase + j;
-            const bool okk = key < prm.N && (!prm.causal || key <= qq) && (prm.window == 0 || key > qq - prm.window);
-            x[j] = okk ? x[j] : -INFINITY;
-          }
-        }
-        uint32_t* pk = pk_all + half * 32;
-#pragma unroll
-        for (int j2 = 0; j2 < 32; ++j2) pk[j2] = pack_bf16x2(ex2_approx(x[2 * j2]), ex2_approx(x[2 * j2 + 1]));
-        // 64 queries -> 32 packed columns of the (already read) S^T columns
-        tmem_st16(tmem + lane_base + kTP + half * 32, pk);
-        tmem_st16(tmem + lane_base + kTP + half * 32 + 16, pk + 16);
+      for (int j2 = 0; j2 < 32; ++j2) {
+        const float2 l2 = *reinterpret_cast<const float2*>(lp + 2 * j2);
+        f2_split(f2_fma(f2(__uint_as_float(sr[2 * j2]), __uint_as_float(sr[2 * j2 + 1])), c2, f2(-l2.x, -l2.y)),
+                 x[2 * j2], x[2 * j2 + 1]);
       }
+      // the mask (diagonal, window edge and tail tiles only) is one branch around its own loop
+      const int qbase = q0 + hq * 64;
+      const bool need_mask = (prm.causal && kv0 + kBwdKeys - 1 > qbase) ||
+                             (prm.window > 0 && kv0 < qbase + 64 - prm.window) || (kv0 + kBwdKeys > prm.N);
+      if (need_mask) {
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          const int qq = qbase + j;
+          const bool okk = key < prm.N && (!prm.causal || key <= qq) && (prm.window == 0 || key > qq - prm.window);
+          x[j] = okk ? x[j] : -INFINITY;
+        }
+      }
+#pragma unroll
+      for (int j2 = 0; j2 < 32; ++j2) pk[j2] = pack_bf16x2(ex2_approx(x[2 * j2]), ex2_approx(x[2 * j2 + 1]));
+      tmem_st16(tmem + lane_base + col_s, pk);
+      tmem_st16(tmem + lane_base + col_s + 16, pk + 16);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(smem_u32(&sm.pa_full));
-
-      // ---- phase B: dS^T = P^T o (dP^T - D) -> TMEM (bf16) and shared memory
-      w_ok = mbar_wait(smem_u32(&sm.dp_full), it & 1, abort, lim);
-      // dS buffer free once the dQ MMA of the previous tile has completed
+      return true;
+    };
+    // phase B: dS^T = P^T o (dP^T - D) for my 64 queries -> TMEM (bf16) and shared memory
+    auto phase_b = [&](int it) -> bool {
+      const int qs = it % kBwdQStages;
+      bool w_ok = mbar_wait(smem_u32(&sm.dp_full), it & 1, abort, lim);
+      // the dS buffer is free once the dQ MMA of the previous tile has completed and the TMA has
+      // read the dQ staged in it
       w_ok = w_ok && mbar_wait(smem_u32(&sm.ds_free), (it & 1) ^ 1, abort, lim);
-      if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+      w_ok = w_ok && mbar_wait(smem_u32(&sm.staging_done), (it & 1) ^ 1, abort, lim);
+      if (!__all_sync(0xffffffffu, w_ok)) return false;
       tc_fence_after();
-      const float* ddp = sm.dd[qs];
+      uint32_t dr[64];
+      tmem_ld32_async(tmem + lane_base + col_dp, dr);
+      tmem_ld32_async(tmem + lane_base + col_dp + 32, dr + 32);
+      tmem_ld_wait();
+      reg_fence<64>(dr);
+      const float* ddp = sm.dd[qs] + hq * 64;
+      uint32_t pd[32];
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        // 64 queries per step: dP^T columns 384 + 64 half .. (read before any dS^T lands on them)
-        uint32_t dr[64];
-        tmem_ld32_async(tmem + lane_base + kTdP + half * 64, dr);
-        tmem_ld32_async(tmem + lane_base + kTdP + half * 64 + 32, dr + 32);
-        tmem_ld_wait();
-        reg_fence<64>(dr);
-        uint32_t pd[32];
-#pragma unroll
-        for (int j2 = 0; j2 < 32; ++j2) {
-          // (dP - D) * P on pairs; P comes back from its packed bf16 form (a shift per half)
-          const float2 d2 = *reinterpret_cast<const float2*>(ddp + half * 64 + 2 * j2);
-          const uint32_t w = pk_all[half * 32 + j2];
-          const uint64_t p2 = f2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
-          const uint64_t t2 = f2_add(f2(__uint_as_float(dr[2 * j2]), __uint_as_float(dr[2 * j2 + 1])), f2(-d2.x, -d2.y));
-          float s0, s1;
-          f2_split(f2_mul(t2, p2), s0, s1);
-          pd[j2] = pack_bf16x2(s0, s1);
-        }
-        // TMEM copy for the dK MMA: packed columns kTdS + 32 half (inside dP^T columns already read)
-        tmem_st16(tmem + lane_base + kTdS + half * 32, pd);
-        tmem_st16(tmem + lane_base + kTdS + half * 32 + 16, pd + 16);
-        // shared-memory copy for the dQ MMA: queries 64 half.. = one 128-byte row of chunk `half`
-#pragma unroll
-        for (int c16 = 0; c16 < 8; ++c16)
-          st_shared_v4(ds_row + half * 16384 + ((c16 ^ sw) << 4), pd[4 * c16], pd[4 * c16 + 1], pd[4 * c16 + 2],
-                       pd[4 * c16 + 3]);
+      for (int j2 = 0; j2 < 32; ++j2) {
+        // (dP - D) * P on pairs; P comes back from its packed bf16 form (a shift per half)
+        const float2 d2 = *reinterpret_cast<const float2*>(ddp + 2 * j2);
+        const uint32_t w = pk[j2];
+        const uint64_t p2 = f2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+        const uint64_t t2 = f2_add(f2(__uint_as_float(dr[2 * j2]), __uint_as_float(dr[2 * j2 + 1])), f2(-d2.x, -d2.y));
+        float s0, s1;
+        f2_split(f2_mul(t2, p2), s0, s1);
+        pd[j2] = pack_bf16x2(s0, s1);
       }
+      tmem_st16(tmem + lane_base + col_dp, pd);
+      tmem_st16(tmem + lane_base + col_dp + 16, pd + 16);
+#pragma unroll
+      for (int c16 = 0; c16 < 8; ++c16)
+        st_shared_v4(ds_row + ((c16 ^ sw) << 4), pd[4 * c16], pd[4 * c16 + 1], pd[4 * c16 + 2], pd[4 * c16 + 3]);
       tmem_st_wait();
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(smem_u32(&sm.ds_full));
+      return true;
+    };
+    // dQ readout: my query row, head-dim columns D/2 hq ...  The block of this warp (32 query
+    // rows x D/2 columns, fp32) is staged in its quadrant's 8 KB slice of the dS buffer (idle
+    // between the dQ MMA and the next phase B) in the 128-byte-swizzled layout of a 32 x 32
+    // box, and added into the accumulator by the TMA engine (cp.reduce.async.bulk.tensor),
+    // which reduces whole lines in L2 instead of 32 scattered 16-byte pieces per instruction.
+    // The query-half-0 warp of a quadrant goes first; its partner reuses the slice once the
+    // TMA has read it, then reports the buffer free for the next phase B.
+    const uint32_t slice = smem_u32(sm.ds) + quad * 8192;
+    auto readout = [&](int it) -> bool {
+      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.dq_full), it & 1, abort, lim))) return false;
+      tc_fence_after();
+      uint32_t v[D / 2];
+#pragma unroll
+      for (int ch = 0; ch < D / 64; ++ch) tmem_ld32_async(tmem + lane_base + col_dq + ch * 32, v + ch * 32);
+      tmem_ld_wait();
+      reg_fence<D / 2>(v);
+      tc_fence_before();
+      mbar_arrive(smem_u32(&sm.dq_free));
+      if (hq == 1 && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.slice_free[quad]), it & 1, abort, lim)))
+        return false;
+      // box b holds columns 32 b .. 32 b + 31 of my half: row `lane` at lane * 128, 16-byte
+      // chunk c at (c ^ (lane & 7)) * 16
+#pragma unroll
+      for (int b = 0; b < D / 64; ++b)
+#pragma unroll
+        for (int c16 = 0; c16 < 8; ++c16)
+          st_shared_v4(slice + b * 4096 + lane * 128 + ((c16 ^ (lane & 7)) << 4), v[32 * b + 4 * c16],
+                       v[32 * b + 4 * c16 + 1], v[32 * b + 4 * c16 + 2], v[32 * b + 4 * c16 + 3]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        const int q0 = (i_begin + it) * kBwdRows;
+#pragma unroll
+        for (int b = 0; b < D / 64; ++b)
+          tma_reduce_add_3d(&tm_dq, slice + b * 4096, hq * (D / 2) + 32 * b, q0 + quad * 32, bh);
+        bulk_commit();
+        bulk_wait_read_all();
+        mbar_arrive(smem_u32(hq == 0 ? &sm.slice_free[quad] : &sm.staging_done));
+      }
+      __syncwarp();
+      return true;
+    };
+
+    // order: B(i), A(i+1), R(i): the dQ readout of tile i hides behind the exponentials of i+1
+    ok = phase_a(0);
+    for (int it = 0; ok && it < n_it; ++it) {
+      if (!phase_b(it)) { ok = false; break; }
+      if (it + 1 < n_it && !phase_a(it + 1)) { ok = false; break; }
+      if (!readout(it)) { ok = false; break; }
     }
-    // epilogue: dK = scale * acc, dV = acc, rows of keys < N
+    if (lane == 0) bulk_wait_all();   // the dQ reductions this thread issued have landed
+    // epilogue: warps of query half 0 write dK = scale * acc, those of half 1 write dV = acc
     if (ok && __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.mma_final), 0, abort, lim))) {
       tc_fence_after();
       const bool in_range = key < prm.N;
       const size_t row_off = (size_t(bh) * prm.N + (in_range ? key : 0)) * D;
+      __nv_bfloat16* dst_row = (hq == 0 ? prm.dk : prm.dv) + row_off;
+      const float mul = hq == 0 ? prm.scale : 1.f;
+      const uint32_t col0 = hq == 0 ? kTdK : kTdV;
 #pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        __nv_bfloat16* dst_row = (which == 0 ? prm.dk : prm.dv) + row_off;
-        const float mul = which == 0 ? prm.scale : 1.f;
-        const uint32_t col0 = which == 0 ? kTdK : kTdV;
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t rr[32];
+        tmem_ld32(tmem + lane_base + col0 + ch * 32, rr);
+        uint32_t w[16];
 #pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch) {
-          uint32_t rr[32];
-          tmem_ld32(tmem + lane_base + col0 + ch * 32, rr);
-          uint32_t w[16];
+        for (int j = 0; j < 16; ++j)
+          w[j] = pack_bf16x2(__uint_as_float(rr[2 * j]) * mul, __uint_as_float(rr[2 * j + 1]) * mul);
+        if (in_range) {
+          uint4* dst = reinterpret_cast<uint4*>(dst_row + ch * 32);
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            w[j] = pack_bf16x2(__uint_as_float(rr[2 * j]) * mul, __uint_as_float(rr[2 * j + 1]) * mul);
-          if (in_range) {
-            uint4* dst = reinterpret_cast<uint4*>(dst_row + ch * 32);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
-          }
+          for (int j = 0; j < 4; ++j) dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
         }
       }
-    }
-  } else if (warp < 8) {
-    // ------------------------------------------------------------------ dQ warps
-    const int qr = (warp - 4) * 32 + lane;     // query row within the tile == TMEM lane of dQ_i
-    const uint32_t lane_base = uint32_t((warp - 4) * 32) << 16;
-    for (int it = 0; it < n_it; ++it) {
-      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.dq_full), it & 1, abort, lim))) break;
-      tc_fence_after();
-      uint32_t v[D];
-#pragma unroll
-      for (int ch = 0; ch < D / 32; ++ch) tmem_ld32_async(tmem + lane_base + kTdQ + ch * 32, v + ch * 32);
-      tmem_ld_wait();
-      reg_fence<D>(v);
-      tc_fence_before();
-      mbar_arrive(smem_u32(&sm.dq_free));
-      const int q0 = (i_begin + it) * kBwdRows;
-      float* acc = prm.dq_acc + (size_t(bh) * prm.Np + q0 + qr) * D;
-#pragma unroll
-      for (int j = 0; j < D / 4; ++j) red_add_f4(acc + 4 * j, v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
     }
   }
 
