@@ -33,7 +33,7 @@
 // once read, dP^T [384,512) with dS^T in [384,416) and [448,480) once read, and dQ in
 // [384,512).  MMAs of one thread
 // run in order, which makes each reuse safe: S_{i+1} is issued after dV_i read P_i, dQ_i after
-// dK_i read dS_i; only dP_{i+1} waits until warps 4-7 have read dQ_i out.
+// dK_i read dS_i; only dP_{i+1} waits until the compute warps have read dQ_i out.
 #pragma once
 
 #include "sm100.cuh"

@@ -30,6 +30,8 @@
 // the first 64 columns of S_w.
 #pragma once
 
+#include <type_traits>
+
 #include "sm100.cuh"
 
 namespace fa {
@@ -44,7 +46,7 @@ constexpr int kWarpMma = 9;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only when m grows by > 2^8
 #ifndef FA_FWD_EMU_PAIRS
-#define FA_FWD_EMU_PAIRS 2
+#define FA_FWD_EMU_PAIRS 4
 #endif
 constexpr int kEmuPairs = FA_FWD_EMU_PAIRS;   // of every 16 exponential pairs, this many use the FMA pipe
 
@@ -260,13 +262,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     bool ok = true;
     float m = -INFINITY;   // running max of scaled scores (log2 units)
     float l = 0.f;         // running sum of exponentials
-    for (int t = tb; t < te; ++t) {
+    // One KV tile.  The masked and the unmasked form are separate instantiations: folded into
+    // one body, the masking code is predicated rather than branched around and costs issue
+    // slots on every tile.
+    auto step = [&](const int t, auto masked) -> bool {
       {
         const int k = t - tb;
         const int kv0 = t * kBlockN;
         // the vote keeps every lane of the warp on the same path into the .sync.aligned TMEM ops
-        if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.s_full[w]), k & 1, abort, lim))) ok = false;
-        if (!ok) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.s_full[w]), k & 1, abort, lim))) return false;
         tc_fence_after();
         float sv[kBlockN];
         {
@@ -278,26 +282,34 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
           for (int j = 0; j < kBlockN; ++j) sv[j] = __uint_as_float(r[j]);
         }
-        const bool need_mask = (kv0 + kBlockN > prm.N) || (prm.causal && kv0 + kBlockN - 1 > qw0) ||
-                               (prm.window > 0 && kv0 < qw0 + kBlockM - prm.window);
-        if (need_mask) {
-          const int hi = prm.causal ? min(qi, prm.N - 1) : prm.N - 1;   // last allowed key
-          const int lo = prm.window > 0 ? qi - prm.window + 1 : 0;       // first allowed key
+        if constexpr (decltype(masked)::value) {
+          // allowed keys of this row form one range [lo, hi]; as columns of the tile, [a, b)
+          const int hi = prm.causal ? min(qi, prm.N - 1) : prm.N - 1;
+          const int lo = prm.window > 0 ? qi - prm.window + 1 : 0;
+          const int a = lo - kv0, b = hi - kv0 + 1;
 #pragma unroll
-          for (int j = 0; j < kBlockN; ++j) {
-            const int key = kv0 + j;
-            if (key > hi || key < lo) sv[j] = -INFINITY;
+          for (int wd = 0; wd < kBlockN / 32; ++wd) {
+            const int aw = min(max(a - 32 * wd, 0), 32), bw = min(max(b - 32 * wd, 0), 32);
+            const uint32_t below_b = bw >= 32 ? 0xffffffffu : ((1u << bw) - 1u);
+            const uint32_t below_a = aw >= 32 ? 0xffffffffu : ((1u << aw) - 1u);
+            const uint32_t bits = below_b & ~below_a;   // allowed columns 32wd + j
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (!((bits >> j) & 1u)) sv[32 * wd + j] = -INFINITY;
           }
         }
-        // row max: 3-input max in 8 independent chains (one chain would be 127 dependent steps)
-        float mx8[8];
+        // row max in 16 independent chains (one chain would be 127 dependent steps)
+        float mx16[16];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) mx8[i] = fmaxf(sv[2 * i], sv[2 * i + 1]);
+        for (int i = 0; i < 16; ++i) mx16[i] = sv[i];
 #pragma unroll
         for (int j = 16; j < kBlockN; j += 16)
 #pragma unroll
-          for (int i = 0; i < 8; ++i) mx8[i] = max3f(mx8[i], sv[j + 2 * i], sv[j + 2 * i + 1]);
-        const float mx = max3f(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
+          for (int i = 0; i < 16; ++i) mx16[i] = fmaxf(mx16[i], sv[j + i]);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx16[i] = fmaxf(mx16[i], mx16[i + 8]);
+        const float mx = max3f(max3f(mx16[0], mx16[1], mx16[2]), max3f(mx16[3], mx16[4], mx16[5]),
+                               fmaxf(mx16[6], mx16[7]));
         const float m_cand = fmaxf(m, mx * c);
         const bool grow = m_cand > m + kRescaleThreshold;   // false while the row has no key
         const float m_new = grow ? m_cand : m;
@@ -354,6 +366,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         tc_fence_before();
         mbar_arrive(smem_u32(&sm.p_full[w]));
       }
+      return true;
+    };
+    for (int t = tb; t < te; ++t) {
+      const int kv0 = t * kBlockN;
+      const bool need_mask = (kv0 + kBlockN > prm.N) || (prm.causal && kv0 + kBlockN - 1 > qw0) ||
+                             (prm.window > 0 && kv0 < qw0 + kBlockM - prm.window);
+      ok = need_mask ? step(t, std::true_type{}) : step(t, std::false_type{});
+      if (!ok) break;
     }
     if (ok && te > tb && __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.o_final[w]), 0, abort, lim))) {
       tc_fence_after();
