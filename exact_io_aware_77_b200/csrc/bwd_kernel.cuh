@@ -36,6 +36,8 @@
 // dK_i read dS_i; only dP_{i+1} waits until the compute warps have read dQ_i out.
 #pragma once
 
+#include <type_traits>
+
 #include "sm100.cuh"
 
 namespace fa {
@@ -348,7 +350,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bool ok = true;
 
     // phase A: P^T = 2^(S^T c - L) for my 64 queries -> TMEM (bf16) and pk
-    auto phase_a = [&](int it) -> bool {
+    // The masked and the unmasked form of phase A are separate instantiations: folded into one
+    // body, the masking code is predicated rather than branched around and costs issue slots on
+    // every tile.
+    auto phase_a = [&](int it, auto masked) -> bool {
       const int qs = it % kBwdQStages;
       const int q0 = (i_begin + it) * kBwdRows;
       bool w_ok = mbar_wait(smem_u32(&sm.q_full[qs]), (it / kBwdQStages) & 1, abort, lim);
@@ -369,16 +374,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         f2_split(f2_fma(f2(__uint_as_float(sr[2 * j2]), __uint_as_float(sr[2 * j2 + 1])), c2, f2(-l2.x, -l2.y)),
                  x[2 * j2], x[2 * j2 + 1]);
       }
-      // the mask (diagonal, window edge and tail tiles only) is one branch around its own loop
-      const int qbase = q0 + hq * 64;
-      const bool need_mask = (prm.causal && kv0 + kBwdKeys - 1 > qbase) ||
-                             (prm.window > 0 && kv0 < qbase + 64 - prm.window) || (kv0 + kBwdKeys > prm.N);
-      if (need_mask) {
+      if constexpr (decltype(masked)::value) {
+        // the queries that may attend to this key form one range [key, key + W - 1] (causal:
+        // W unbounded without a window; no range at all for a padded key); as columns, [a, b)
+        const int qbase = q0 + hq * 64;
+        const int a = prm.causal ? key - qbase : 0;
+        const int b = key >= prm.N ? a : (prm.window > 0 ? key + prm.window - qbase : 64);
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          const int qq = qbase + j;
-          const bool okk = key < prm.N && (!prm.causal || key <= qq) && (prm.window == 0 || key > qq - prm.window);
-          x[j] = okk ? x[j] : -INFINITY;
+        for (int wd = 0; wd < 2; ++wd) {
+          const int aw = min(max(a - 32 * wd, 0), 32), bw = min(max(b - 32 * wd, 0), 32);
+          const uint32_t below_b = bw >= 32 ? 0xffffffffu : ((1u << bw) - 1u);
+          const uint32_t below_a = aw >= 32 ? 0xffffffffu : ((1u << aw) - 1u);
+          const uint32_t bits = below_b & ~below_a;
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (!((bits >> j) & 1u)) x[32 * wd + j] = -INFINITY;
         }
       }
 #pragma unroll
@@ -473,10 +483,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     };
 
     // order: B(i), A(i+1), R(i): the dQ readout of tile i hides behind the exponentials of i+1
-    ok = phase_a(0);
+    // phase A masks only on the diagonal, the window's far edge and the tail key tile
+    auto run_a = [&](int it) -> bool {
+      const int qbase = (i_begin + it) * kBwdRows + hq * 64;
+      const bool need_mask = (prm.causal && kv0 + kBwdKeys - 1 > qbase) ||
+                             (prm.window > 0 && kv0 < qbase + 64 - prm.window) || (kv0 + kBwdKeys > prm.N);
+      return need_mask ? phase_a(it, std::true_type{}) : phase_a(it, std::false_type{});
+    };
+    ok = run_a(0);
     for (int it = 0; ok && it < n_it; ++it) {
       if (!phase_b(it)) { ok = false; break; }
-      if (it + 1 < n_it && !phase_a(it + 1)) { ok = false; break; }
+      if (it + 1 < n_it && !run_a(it + 1)) { ok = false; break; }
       if (!readout(it)) { ok = false; break; }
     }
     if (lane == 0) bulk_wait_all();   // the dQ reductions this thread issued have landed
