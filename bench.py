@@ -419,12 +419,12 @@ def measure_e2e(fa, torch, wl, dev, stream, q_h, k_h, v_h, do_h, has_bwd, steps,
 # the causal B2 H32 N4096 d128 workload, keyed by kernel, with the SHA-1 of the kernel's sources
 # when the counters were taken (profiles/ holds the summaries).  A changed source reports null.
 NCU_TRAFFIC = {
-    "fa_fwd_kernel<128>": {"bytes": 253879296,
-                           "sources": {"fwd_kernel.cuh": "e35511c1c60c436c64a9df2632136123791a6a84",
-                                       "sm100.cuh": "29b768c7857f6963a8d0d84283bdbebae4fd4aab"}},
-    "fa_bwd_kernel<128>": {"bytes": 630191616,
-                           "sources": {"bwd_kernel.cuh": "de5b41104ddfc88b930ea5b7232df652f3ca2883",
-                                       "sm100.cuh": "29b768c7857f6963a8d0d84283bdbebae4fd4aab"}},
+    "fa_fwd_kernel<128>": {"bytes": 252712192,
+                           "sources": {"fwd_kernel.cuh": "ca257a75df8e68d629bb8ce734914350a093971a",
+                                       "sm100.cuh": "3f997d2b018b2617b6f28d5c697ffcab44851b33"}},
+    "fa_bwd_kernel<128>": {"bytes": 628727296,
+                           "sources": {"bwd_kernel.cuh": "41c6cf29c6cc4acc5a665149cb46ddf53390027f",
+                                       "sm100.cuh": "3f997d2b018b2617b6f28d5c697ffcab44851b33"}},
 }
 
 

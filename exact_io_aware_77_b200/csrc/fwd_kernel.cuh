@@ -46,7 +46,7 @@ constexpr int kWarpMma = 9;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only when m grows by > 2^8
 #ifndef FA_FWD_EMU_PAIRS
-#define FA_FWD_EMU_PAIRS 4
+#define FA_FWD_EMU_PAIRS 7
 #endif
 constexpr int kEmuPairs = FA_FWD_EMU_PAIRS;   // of every 16 exponential pairs, this many use the FMA pipe
 
