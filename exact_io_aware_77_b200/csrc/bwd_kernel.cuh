@@ -26,8 +26,8 @@
 //               w / 4 of each tile.  Phase A: P^T = exp2(S^T c - L) with the causal/window mask,
 //               stored to TMEM as bf16.  Phase B: dS^T = P^T o (dP^T - D) to TMEM (A of dK) and
 //               to shared memory (A of dQ).  Readout: its half of the dQ_i rows of its 32
-//               queries, staged in shared memory and added into the fp32 accumulator by a TMA
-//               tensor reduce-add.
+//               queries, through its own rows of the dS buffer into vector reductions on the
+//               fp32 accumulator.
 //               Order per tile: B(i), A(i+1), readout(i).  At the end: dK (half 0), dV (half 1).
 // TMEM columns: dK [0,128), dV [128,256), S^T [256,384) with P^T in [256,288) and [320,352)
 // once read, dP^T [384,512) with dS^T in [384,416) and [448,480) once read, and dQ in
@@ -76,8 +76,7 @@ struct BwdSmem {
   alignas(16) float dd[kBwdQStages][kBwdRows];
   alignas(8) uint64_t kv_full;
   uint64_t q_full[kBwdQStages], q_empty[kBwdQStages];
-  uint64_t s_full, dp_full, pa_full, ds_full, ds_free, dq_full, dq_free, mma_final, mma_drain;
-  uint64_t slice_free[4], staging_done;   // dQ staging in the dS buffer (see the readout)
+  uint64_t s_full, dp_full, pa_full, ds_full, dq_full, dq_free, mma_final, mma_drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -165,7 +164,7 @@ template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                  const __grid_constant__ CUtensorMap tm_dq, const BwdParams prm) {
+                  const BwdParams prm) {
   using Smem = BwdSmem<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // the layout fills almost all 227 KB, so no slack is left for realigning the base
@@ -197,13 +196,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(smem_u32(&sm.dp_full), 1);
     mbar_init(smem_u32(&sm.pa_full), 256);
     mbar_init(smem_u32(&sm.ds_full), 256);
-    mbar_init(smem_u32(&sm.ds_free), 1);
     mbar_init(smem_u32(&sm.dq_full), 1);
     mbar_init(smem_u32(&sm.dq_free), 256);
     mbar_init(smem_u32(&sm.mma_final), 1);
     mbar_init(smem_u32(&sm.mma_drain), 1);
-    for (int qd = 0; qd < 4; ++qd) mbar_init(smem_u32(&sm.slice_free[qd]), 1);
-    mbar_init(smem_u32(&sm.staging_done), 4);
     fence_mbar_init();
   }
   if (warp == kBwdWarpTma && lane == 0) {
@@ -211,7 +207,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
     tma_prefetch_desc(&tm_do);
-    tma_prefetch_desc(&tm_dq);
   }
   if (warp == kBwdWarpMma) {
     tmem_alloc(smem_u32(&sm.tmem_base), 512);
@@ -317,7 +312,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int kk = 0; kk < kBwdKeys / 16; ++kk)
           mma_bf16_ss_w(tmem + kTdQ, desc_advance(dds_mn, kk * 2048), desc_advance(dk_mn, kk * 2048), idesc_q, kk > 0);
         mma_commit_w(smem_u32(&sm.dq_full));
-        mma_commit_w(smem_u32(&sm.ds_free));
         mma_commit_w(smem_u32(&sm.q_empty[qs]));
         // dP^T of the next tile once dQ_i has been read out of the same columns
         if (has_next) {
@@ -403,11 +397,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // phase B: dS^T = P^T o (dP^T - D) for my 64 queries -> TMEM (bf16) and shared memory
     auto phase_b = [&](int it) -> bool {
       const int qs = it % kBwdQStages;
-      bool w_ok = mbar_wait(smem_u32(&sm.dp_full), it & 1, abort, lim);
-      // the dS buffer is free once the dQ MMA of the previous tile has completed and the TMA has
-      // read the dQ staged in it
-      w_ok = w_ok && mbar_wait(smem_u32(&sm.ds_free), (it & 1) ^ 1, abort, lim);
-      w_ok = w_ok && mbar_wait(smem_u32(&sm.staging_done), (it & 1) ^ 1, abort, lim);
+      // my rows of the dS buffer are free: the readout of the previous tile, earlier in this
+      // warp's program, waited for the dQ MMA that read them and then used them as staging
+      const bool w_ok = mbar_wait(smem_u32(&sm.dp_full), it & 1, abort, lim);
       if (!__all_sync(0xffffffffu, w_ok)) return false;
       tc_fence_after();
       uint32_t dr[64];
@@ -439,14 +431,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_arrive(smem_u32(&sm.ds_full));
       return true;
     };
-    // dQ readout: my query row, head-dim columns D/2 hq ...  The block of this warp (32 query
-    // rows x D/2 columns, fp32) is staged in its quadrant's 8 KB slice of the dS buffer (idle
-    // between the dQ MMA and the next phase B) in the 128-byte-swizzled layout of a 32 x 32
-    // box, and added into the accumulator by the TMA engine (cp.reduce.async.bulk.tensor),
-    // which reduces whole lines in L2 instead of 32 scattered 16-byte pieces per instruction.
-    // The query-half-0 warp of a quadrant goes first; its partner reuses the slice once the
-    // TMA has read it, then reports the buffer free for the next phase B.
-    const uint32_t slice = smem_u32(sm.ds) + quad * 8192;
+    // dQ readout: my 32 query rows, head-dim columns D/2 hq ...  In passes of 32 columns the
+    // block goes from TMEM through my own 4 KB of the dS buffer (free once the dQ MMA has
+    // read it) and is read back so that each vector reduction covers four whole 128-byte row
+    // segments of the fp32 accumulator: red.global.add.v4.f32, 32 lanes x 16 bytes.
+    const uint32_t stage = smem_u32(sm.ds) + hq * 16384 + quad * 4096;   // = my dS rows
     auto readout = [&](int it) -> bool {
       if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.dq_full), it & 1, abort, lim))) return false;
       tc_fence_after();
@@ -457,28 +446,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       reg_fence<D / 2>(v);
       tc_fence_before();
       mbar_arrive(smem_u32(&sm.dq_free));
-      if (hq == 1 && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.slice_free[quad]), it & 1, abort, lim)))
-        return false;
-      // box b holds columns 32 b .. 32 b + 31 of my half: row `lane` at lane * 128, 16-byte
-      // chunk c at (c ^ (lane & 7)) * 16
+      const int q0 = (i_begin + it) * kBwdRows + quad * 32;
+      float* acc = prm.dq_acc + (size_t(bh) * prm.Np + q0) * D + hq * (D / 2);
 #pragma unroll
-      for (int b = 0; b < D / 64; ++b)
+      for (int ps = 0; ps < D / 64; ++ps) {
+        // row `lane`, 16-byte chunk c at lane * 128 + (c ^ (lane & 7)) * 16
 #pragma unroll
         for (int c16 = 0; c16 < 8; ++c16)
-          st_shared_v4(slice + b * 4096 + lane * 128 + ((c16 ^ (lane & 7)) << 4), v[32 * b + 4 * c16],
-                       v[32 * b + 4 * c16 + 1], v[32 * b + 4 * c16 + 2], v[32 * b + 4 * c16 + 3]);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        const int q0 = (i_begin + it) * kBwdRows;
+          st_shared_v4(stage + lane * 128 + ((c16 ^ (lane & 7)) << 4), v[32 * ps + 4 * c16],
+                       v[32 * ps + 4 * c16 + 1], v[32 * ps + 4 * c16 + 2], v[32 * ps + 4 * c16 + 3]);
+        __syncwarp();
 #pragma unroll
-        for (int b = 0; b < D / 64; ++b)
-          tma_reduce_add_3d(&tm_dq, slice + b * 4096, hq * (D / 2) + 32 * b, q0 + quad * 32, bh);
-        bulk_commit();
-        bulk_wait_read_all();
-        mbar_arrive(smem_u32(hq == 0 ? &sm.slice_free[quad] : &sm.staging_done));
+        for (int j = 0; j < 8; ++j) {
+          const int row = 4 * j + (lane >> 3), c = lane & 7;   // 8 lanes cover one 128-byte row
+          const uint4 x = ld_shared_v4(stage + row * 128 + ((c ^ (row & 7)) << 4));
+          red_add_v4(acc + size_t(row) * D + 32 * ps + 4 * c, x);
+        }
+        __syncwarp();
       }
-      __syncwarp();
       return true;
     };
 
@@ -496,7 +481,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (it + 1 < n_it && !run_a(it + 1)) { ok = false; break; }
       if (!readout(it)) { ok = false; break; }
     }
-    if (lane == 0) bulk_wait_all();   // the dQ reductions this thread issued have landed
     // epilogue: warps of query half 0 write dK = scale * acc, those of half 1 write dV = acc
     if (ok && __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.mma_final), 0, abort, lim))) {
       tc_fence_after();

@@ -52,20 +52,6 @@ bool make_map_bf16(CUtensorMap* map, const void* base, int d, int rows, int bh, 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// fp32 [bh, rows, d] as a 3-D tensor (d, rows, bh); 32 x 32 boxes, 128-byte swizzled (the dQ
-// accumulator, written by tensor reduce-add)
-bool make_map_f32(CUtensorMap* map, const void* base, int d, int rows, int bh) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
-  cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(rows), cuuint64_t(bh)};
-  cuuint64_t strides[2] = {cuuint64_t(d) * 4, cuuint64_t(d) * 4 * cuuint64_t(rows)};
-  cuuint32_t box[3] = {32, 32, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // ---------------------------------------------------------------- validation
 constexpr int kMaxDevices = 64;
 
@@ -155,10 +141,9 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   if (phases & kBwdPhaseMain) {
-  CUtensorMap tq, tk, tv, tdo, tdq;
+  CUtensorMap tq, tk, tv, tdo;
   if (!make_map_bf16(&tq, q, D, N, BH, kBwdRows) || !make_map_bf16(&tk, k, D, N, BH, kBwdKeys) ||
-      !make_map_bf16(&tv, v, D, N, BH, kBwdKeys) || !make_map_bf16(&tdo, dout, D, N, BH, kBwdRows) ||
-      !make_map_f32(&tdq, dq_acc, D, int(Np), BH))
+      !make_map_bf16(&tv, v, D, N, BH, kBwdKeys) || !make_map_bf16(&tdo, dout, D, N, BH, kBwdRows))
     return FA_ERR_CUDA;
   BwdParams prm;
   prm.lp = lp;
@@ -178,8 +163,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   static_assert(sizeof(BwdSmem<D>) <= 232448, "backward shared memory exceeds 227 KB");
   const int smem = int(sizeof(BwdSmem<D>));   // the kernel checks that the base is 1 KB aligned
   if (set_smem(fa_bwd_kernel<D>, smem) != FA_OK) return FA_ERR_CUDA;
-  fa_bwd_kernel<D><<<unsigned(prm.n_kv_tiles) * unsigned(BH), kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, tdq,
-                                                                                            prm);
+  fa_bwd_kernel<D><<<unsigned(prm.n_kv_tiles) * unsigned(BH), kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, prm);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   if (phases & kBwdPhaseFinal) {
