@@ -14,8 +14,9 @@
 //   fa_bwd_kernel    one CTA per 128-key tile of one head; loops over 128-row query tiles.
 //   fa_bwd_dq_final  dQ = scale * accumulator, rounded to bf16.
 //
-// fa_bwd_kernel roles (320 threads), every MMA 128 x 128 (narrower ones cost as much time):
-//   warp 8      TMA producer: K, V once; Q_i, dO_i (+ their L and D rows) into a 2-stage ring.
+// fa_bwd_kernel roles (384 threads), every MMA 128 x 128 (narrower ones cost as much time):
+//   warp 8      TMA producer: K, V once; Q_i (+ its L and D rows) into a 2-stage ring, dO_i into
+//               one stage.
 //   warp 9      MMA issuer, per query tile i in the order
 //                 dV += P_i^T dO_i, S_{i+1}^T = K Q_{i+1}^T, dK += dS_i^T Q_i, dQ_i = dS_i K,
 //                 dP_{i+1}^T = V dO_{i+1}^T
@@ -26,9 +27,11 @@
 //               w / 4 of each tile.  Phase A: P^T = exp2(S^T c - L) with the causal/window mask,
 //               stored to TMEM as bf16.  Phase B: dS^T = P^T o (dP^T - D) to TMEM (A of dK) and
 //               to shared memory (A of dQ).  Readout: its half of the dQ_i rows of its 32
-//               queries, through its own rows of the dS buffer into vector reductions on the
-//               fp32 accumulator.
+//               queries, from TMEM into its shared-memory staging slot, 32 columns at a time.
 //               Order per tile: B(i), A(i+1), readout(i).  At the end: dK (half 0), dV (half 1).
+//   warps 10-11 reduction: read the staged dQ blocks back (so that each vector reduction
+//               covers whole 128-byte row segments) and add them into the fp32 accumulator
+//               with red.global.add.v4.f32, so that no compute warp waits on the reductions.
 // TMEM columns: dK [0,128), dV [128,256), S^T [256,384) with P^T in [256,288) and [320,352)
 // once read, dP^T [384,512) with dS^T in [384,416) and [448,480) once read, and dQ in
 // [384,512).  MMAs of one thread
@@ -45,7 +48,7 @@ namespace fa {
 constexpr int kBwdKeys = 128;    // keys per CTA
 constexpr int kBwdRows = 128;    // queries per iteration
 constexpr int kBwdQStages = 2;
-constexpr int kBwdThreads = 320;
+constexpr int kBwdThreads = 384;   // 8 compute warps, TMA, MMA, 2 reduction warps
 constexpr int kBwdWarpTma = 8;
 constexpr int kBwdWarpMma = 9;
 constexpr uint32_t kTdK = 0, kTdV = 128, kTS = 256, kTP = 256, kTdP = 384, kTdS = 384, kTdQ = 384;
@@ -70,13 +73,15 @@ struct BwdSmem {
   alignas(1024) uint8_t k[kTileBytes];
   alignas(1024) uint8_t v[kTileBytes];
   alignas(1024) uint8_t q[kBwdQStages][kTileBytes];
-  alignas(1024) uint8_t dout[kBwdQStages][kTileBytes];
+  alignas(1024) uint8_t dout[kTileBytes];                  // one stage: see the producer
   alignas(1024) uint8_t ds[kBwdKeys * kBwdRows * 2];       // dS^T: [key][query], 64-query chunks
+  alignas(1024) uint8_t stage[8][32 * 32 * 4];             // dQ staging: 32 rows x 32 fp32 per compute warp
   alignas(16) float lp[kBwdQStages][kBwdRows];
   alignas(16) float dd[kBwdQStages][kBwdRows];
   alignas(8) uint64_t kv_full;
-  uint64_t q_full[kBwdQStages], q_empty[kBwdQStages];
+  uint64_t q_full[kBwdQStages], q_empty[kBwdQStages], do_full, do_empty;
   uint64_t s_full, dp_full, pa_full, ds_full, dq_full, dq_free, mma_final, mma_drain;
+  uint64_t st_full[8], st_free[8];   // dQ staging of each compute warp: filled / read back
   uint32_t tmem_base;
   int abort;
 };
@@ -200,6 +205,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(smem_u32(&sm.dq_free), 256);
     mbar_init(smem_u32(&sm.mma_final), 1);
     mbar_init(smem_u32(&sm.mma_drain), 1);
+    mbar_init(smem_u32(&sm.do_full), 1);
+    mbar_init(smem_u32(&sm.do_empty), 1);
+    for (int w = 0; w < 8; ++w) {
+      mbar_init(smem_u32(&sm.st_full[w]), 32);
+      mbar_init(smem_u32(&sm.st_free[w]), 32);
+    }
     fence_mbar_init();
   }
   if (warp == kBwdWarpTma && lane == 0) {
@@ -227,25 +238,34 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tma_load_3d(smem_u32(sm.v) + c * 16384, &tm_v, kvb, c * 64, kv0, bh);
       }
       int issued = 0;
+      // Q_i (with its L and D rows) through two stages; dO_i through one: its last reader,
+      // dV_i, comes first in tile i and its next reader, dP_{i+1}, last, so one stage leaves
+      // the load of dO_{i+1} most of a tile to land
+      int issued_do = 0;
       for (int it = 0; it < n_it; ++it) {
         const int qs = it % kBwdQStages;
         const uint32_t ph = (it / kBwdQStages) & 1;
         const int q0 = (i_begin + it) * kBwdRows;
         if (!mbar_wait(smem_u32(&sm.q_empty[qs]), ph ^ 1, abort, lim)) break;
         const uint32_t qb = smem_u32(&sm.q_full[qs]);
-        mbar_expect_tx(qb, 2 * Smem::kTileBytes + 2 * kBwdRows * 4);
-        for (int c = 0; c < Smem::kChunks; ++c) {
+        mbar_expect_tx(qb, Smem::kTileBytes + 2 * kBwdRows * 4);
+        for (int c = 0; c < Smem::kChunks; ++c)
           tma_load_3d(smem_u32(sm.q[qs]) + c * 16384, &tm_q, qb, c * 64, q0, bh);
-          tma_load_3d(smem_u32(sm.dout[qs]) + c * 16384, &tm_do, qb, c * 64, q0, bh);
-        }
         const size_t row = size_t(bh) * prm.Np + q0;
         bulk_load(smem_u32(sm.lp[qs]), prm.lp + row, kBwdRows * 4, qb);
         bulk_load(smem_u32(sm.dd[qs]), prm.dd + row, kBwdRows * 4, qb);
         issued = it + 1;
+        if (!mbar_wait(smem_u32(&sm.do_empty), (it & 1) ^ 1, abort, lim)) break;
+        const uint32_t db = smem_u32(&sm.do_full);
+        mbar_expect_tx(db, Smem::kTileBytes);
+        for (int c = 0; c < Smem::kChunks; ++c)
+          tma_load_3d(smem_u32(sm.dout) + c * 16384, &tm_do, db, c * 64, q0, bh);
+        issued_do = it + 1;
       }
       mbar_wait_drain(kvb, 0, lim);
       for (int it = max(0, issued - kBwdQStages); it < issued; ++it)
         mbar_wait_drain(smem_u32(&sm.q_full[it % kBwdQStages]), (it / kBwdQStages) & 1, lim);
+      if (issued_do > 0) mbar_wait_drain(smem_u32(&sm.do_full), (issued_do - 1) & 1, lim);
     }
   } else if (warp == kBwdWarpMma) {
     // ------------------------------------------------------------------ MMA issuer
@@ -285,7 +305,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_after();
         issue_t(dk_kmaj, sm.q[0], kTS);
         mma_commit_w(smem_u32(&sm.s_full));
-        issue_t(dv_kmaj, sm.dout[0], kTdP);
+        ok = wait(smem_u32(&sm.do_full), 0);
+      }
+      if (ok) {
+        tc_fence_after();
+        issue_t(dv_kmaj, sm.dout, kTdP);
         mma_commit_w(smem_u32(&sm.dp_full));
       }
       for (int it = 0; ok && it < n_it; ++it) {
@@ -295,7 +319,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // dV += P^T dO_i
         if (!wait(smem_u32(&sm.pa_full), it & 1)) break;
         tc_fence_after();
-        issue_kv(kTP, sm.dout[qs], kTdV, it == 0);
+        issue_kv(kTP, sm.dout, kTdV, it == 0);
+        mma_commit_w(smem_u32(&sm.do_empty));   // dV_i was dO_i's last reader
         // S^T of the next tile (overwrites P^T only after dV above has read it)
         if (has_next) {
           if (!wait(smem_u32(&sm.q_full[qn]), ((it + 1) / kBwdQStages) & 1)) break;
@@ -316,8 +341,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // dP^T of the next tile once dQ_i has been read out of the same columns
         if (has_next) {
           if (!wait(smem_u32(&sm.dq_free), it & 1)) break;
+          if (!wait(smem_u32(&sm.do_full), (it + 1) & 1)) break;
           tc_fence_after();
-          issue_t(dv_kmaj, sm.dout[qn], kTdP);
+          issue_t(dv_kmaj, sm.dout, kTdP);
           mma_commit_w(smem_u32(&sm.dp_full));
         }
       }
@@ -432,10 +458,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       return true;
     };
     // dQ readout: my 32 query rows, head-dim columns D/2 hq ...  In passes of 32 columns the
-    // block goes from TMEM through my own 4 KB of the dS buffer (free once the dQ MMA has
-    // read it) and is read back so that each vector reduction covers four whole 128-byte row
-    // segments of the fp32 accumulator: red.global.add.v4.f32, 32 lanes x 16 bytes.
-    const uint32_t stage = smem_u32(sm.ds) + hq * 16384 + quad * 4096;   // = my dS rows
+    // block goes from TMEM into my 4 KB staging slot; a reduction warp reads it back and issues
+    // the vector reductions, so this warp never waits on them.
+    const uint32_t stage = smem_u32(sm.stage[warp]);
+    int n_pass = 0;   // blocks staged so far: their parity is the slot barriers' phase
     auto readout = [&](int it) -> bool {
       if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.dq_full), it & 1, abort, lim))) return false;
       tc_fence_after();
@@ -446,23 +472,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       reg_fence<D / 2>(v);
       tc_fence_before();
       mbar_arrive(smem_u32(&sm.dq_free));
-      const int q0 = (i_begin + it) * kBwdRows + quad * 32;
-      float* acc = prm.dq_acc + (size_t(bh) * prm.Np + q0) * D + hq * (D / 2);
 #pragma unroll
-      for (int ps = 0; ps < D / 64; ++ps) {
+      for (int ps = 0; ps < D / 64; ++ps, ++n_pass) {
+        // the reduction warp has read the previous block out of the slot
+        if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.st_free[warp]), (n_pass & 1) ^ 1, abort, lim)))
+          return false;
         // row `lane`, 16-byte chunk c at lane * 128 + (c ^ (lane & 7)) * 16
 #pragma unroll
         for (int c16 = 0; c16 < 8; ++c16)
           st_shared_v4(stage + lane * 128 + ((c16 ^ (lane & 7)) << 4), v[32 * ps + 4 * c16],
                        v[32 * ps + 4 * c16 + 1], v[32 * ps + 4 * c16 + 2], v[32 * ps + 4 * c16 + 3]);
-        __syncwarp();
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int row = 4 * j + (lane >> 3), c = lane & 7;   // 8 lanes cover one 128-byte row
-          const uint4 x = ld_shared_v4(stage + row * 128 + ((c ^ (row & 7)) << 4));
-          red_add_v4(acc + size_t(row) * D + 32 * ps + 4 * c, x);
-        }
-        __syncwarp();
+        mbar_arrive(smem_u32(&sm.st_full[warp]));
       }
       return true;
     };
@@ -503,6 +523,43 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           for (int j = 0; j < 4; ++j) dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
         }
       }
+    }
+  }
+
+  if (warp >= 10) {
+    // ------------------------------------------------------------------ reduction warps
+    // Warp 10 serves compute warps 0-3, warp 11 warps 4-7, block by block in the order they
+    // stage them: read the block back so that each red.global.add.v4.f32 covers four whole
+    // 128-byte row segments of the fp32 accumulator, free the slot, then issue the reductions.
+    const int first = (warp - 10) * 4;
+    const int hq = first / 4;   // query half (= head-dim column half) of the warps served
+    for (int it = 0; it < n_it; ++it) {
+      for (int ps = 0; ps < D / 64; ++ps) {
+        const int n = it * (D / 64) + ps;
+        bool ok = true;
+        for (int qd = 0; qd < 4 && ok; ++qd) {
+          const int w = first + qd;
+          ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.st_full[w]), n & 1, abort, lim));
+          if (!ok) break;
+          const uint32_t slot = smem_u32(sm.stage[w]);
+          uint4 x[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int row = 4 * j + (lane >> 3), c = lane & 7;   // 8 lanes cover one 128-byte row
+            x[j] = ld_shared_v4(slot + row * 128 + ((c ^ (row & 7)) << 4));
+          }
+          mbar_arrive(smem_u32(&sm.st_free[w]));
+          const int q0 = (i_begin + it) * kBwdRows + qd * 32;
+          float* acc = prm.dq_acc + (size_t(bh) * prm.Np + q0) * D + hq * (D / 2) + 32 * ps;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int row = 4 * j + (lane >> 3), c = lane & 7;
+            red_add_v4(acc + size_t(row) * D + 4 * c, x[j]);
+          }
+        }
+        if (!ok) break;
+      }
+      if (*abort) break;
     }
   }
 
