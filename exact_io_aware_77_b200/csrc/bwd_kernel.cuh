@@ -424,7 +424,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     auto phase_b = [&](int it) -> bool {
       const int qs = it % kBwdQStages;
       // my rows of the dS buffer are free: the readout of the previous tile, earlier in this
-      // warp's program, waited for the dQ MMA that read them and then used them as staging
+      // warp's program, waited for the dQ MMA that read them
       const bool w_ok = mbar_wait(smem_u32(&sm.dp_full), it & 1, abort, lim);
       if (!__all_sync(0xffffffffu, w_ok)) return false;
       tc_fence_after();
