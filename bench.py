@@ -423,7 +423,7 @@ NCU_TRAFFIC = {
                            "sources": {"fwd_kernel.cuh": "ca257a75df8e68d629bb8ce734914350a093971a",
                                        "sm100.cuh": "f5bfef53a203d01b5f2fa38e4a691ac48c3cc963"}},
     "fa_bwd_kernel<128>": {"bytes": 628685568,
-                           "sources": {"bwd_kernel.cuh": "daf2a7c83dc8072a604c2f6db933293ecacf7927",
+                           "sources": {"bwd_kernel.cuh": "99106479f0620aa9dfa5440abac1d6927ee71678",
                                        "sm100.cuh": "f5bfef53a203d01b5f2fa38e4a691ac48c3cc963"}},
 }
 
