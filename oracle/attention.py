@@ -27,11 +27,14 @@ What it computes, and where that is defined:
   the identity D_i = rowsum(dO o O) that a fused backward uses, so the two
   sides check each other.
 
-Mask readings (the pages name masking and sliding-window attention but fix no
-convention; sparse-attention glossary, "Abgrenzung"):
+Mask readings (the pages name masking and sliding-window attention, a purely
+local window, but fix no convention; sparse-attention glossary, "Abgrenzung &
+Vergleiche"):
   causal:   key j is allowed for query i iff j <= i (square self-attention);
   window W: additionally j >= i - W + 1 (the window counts the diagonal, so
-            W = 1 keeps only key i); a window needs causal (one-sided band);
+            W = 1 keeps only key i);
+  window W without causal: the local window on both sides, |i - j| <= W - 1
+            (the same count convention: W = 1 keeps only key i);
   W = 0:    no band.
 Every row keeps its diagonal, so no row is ever fully masked.
 
@@ -57,8 +60,6 @@ __all__ = [
 def _check_mask_args(causal: bool, window: int) -> None:
     if window < 0:
         raise ValueError("window must be >= 0")
-    if window > 0 and not causal:
-        raise ValueError("a sliding window is one-sided here and needs causal=True")
 
 
 def allowed_mask(n_q: int, n_k: int, causal: bool, window: int, row_start: int = 0) -> np.ndarray:
@@ -185,6 +186,8 @@ def _rows_mask(r: np.ndarray, n_k: int, causal: bool, window: int) -> np.ndarray
         ok &= j <= i
     if window > 0:
         ok &= j >= i - window + 1
+        if not causal:
+            ok &= j <= i + window - 1
     return ok
 
 
@@ -228,5 +231,7 @@ def allowed_pairs(n: int, causal: bool, window: int) -> int:
         hi = i if causal else n - 1
         if window > 0:
             lo = max(0, i - window + 1)
+            if not causal:
+                hi = min(n - 1, i + window - 1)
         total += hi - lo + 1
     return total

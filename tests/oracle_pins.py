@@ -19,7 +19,7 @@ import pathlib
 import numpy as np
 
 GOLDEN = pathlib.Path(__file__).parent / "golden"
-MASKS = [(False, 0), (True, 0), (True, 1), (True, 3), (True, 7)]
+MASKS = [(False, 0), (True, 0), (True, 1), (True, 3), (True, 7), (False, 1), (False, 3), (False, 7)]
 
 
 def _rng(seed):
@@ -31,9 +31,20 @@ def _qkv(seed, n=13, d=5, lead=(2,), std=1.0):
     return [std * r.standard_normal(lead + (n, d)) for _ in range(3)]
 
 
-def _n_allowed(i, n, causal, window):
-    hi = i if causal else n - 1
+def _band(i, n, causal, window):
+    """[lo, hi] of the keys row i may attend (closed interval), written from the mask readings."""
     lo = max(0, i - window + 1) if window > 0 else 0
+    if causal:
+        hi = i
+    elif window > 0:
+        hi = min(n - 1, i + window - 1)
+    else:
+        hi = n - 1
+    return lo, hi
+
+
+def _n_allowed(i, n, causal, window):
+    lo, hi = _band(i, n, causal, window)
     return hi - lo + 1
 
 
@@ -54,7 +65,10 @@ def rows_sum_to_one(orc):
             masked |= j > i
         if window:
             masked |= j < i - window + 1
+            if not causal:
+                masked |= j > i + window - 1
         assert np.all(p[..., masked] == 0.0)
+        assert np.all(p[..., ~masked] > 0.0)
 
 
 def constant_v(orc):
@@ -130,10 +144,9 @@ def scale_zero(orc):
         o, lse = orc.attention_forward(q, k, v, 0.0, causal, window)
         for i in range(n):
             cnt = _n_allowed(i, n, causal, window)
-            lo = max(0, i - window + 1) if window else 0
-            hi = i + 1 if causal else n
+            lo, hi = _band(i, n, causal, window)
             assert abs(lse[..., i] - math.log(cnt)).max() < 1e-12
-            assert np.max(np.abs(o[..., i, :] - v[..., lo:hi, :].mean(-2))) < 1e-12
+            assert np.max(np.abs(o[..., i, :] - v[..., lo:hi + 1, :].mean(-2))) < 1e-12
 
 
 def key_shift(orc):
@@ -199,7 +212,7 @@ def _torch_reference(q, k, v, scale, causal, window):
     if causal:
         ok &= j <= i
     if window:
-        ok &= j >= i - window + 1
+        ok &= (j - i).abs() <= window - 1 if not causal else j >= i - window + 1
     o = F.scaled_dot_product_attention(tq, tk, tv, attn_mask=ok, scale=scale)
     return (tq, tk, tv), o
 
@@ -288,19 +301,46 @@ def row_blocks_match(orc):
 
 
 def pair_count(orc):
-    """allowed_pairs matches the closed forms N^2, N(N+1)/2 and the banded count."""
+    """allowed_pairs matches the closed forms N^2, N(N+1)/2 and the banded counts: one-sided
+    W(W+1)/2 + (N-W)W, two-sided N(2W-1) - W(W-1) (each edge loses 1 + 2 + ... + (W-1))."""
     for n in (1, 5, 16, 33):
         assert orc.allowed_pairs(n, False, 0) == n * n
         assert orc.allowed_pairs(n, True, 0) == n * (n + 1) // 2
         for w in (1, 4, 40):
             ww = min(w, n)
             assert orc.allowed_pairs(n, True, w) == ww * (ww + 1) // 2 + (n - ww) * ww
+            two = n * n if w >= n else n * (2 * w - 1) - w * (w - 1)
+            assert orc.allowed_pairs(n, False, w) == two
+
+
+def two_sided_window(orc):
+    """Without causal, a window W keeps |i - j| <= W - 1: W = 1 gives O_i = v_i and
+    L_i = scale q_i . k_i; W >= N equals unmasked attention; row i ignores keys i - W and
+    i + W and depends on keys i - W + 1 and i + W - 1."""
+    q, k, v = _qkv(22)
+    n = q.shape[-2]
+    o, lse = orc.attention_forward(q, k, v, 0.8, False, 1)
+    assert np.max(np.abs(o - v)) < 1e-12
+    assert np.max(np.abs(lse - 0.8 * np.sum(q * k, -1))) < 1e-12
+    o, lse = orc.attention_forward(q, k, v, 0.6, False, 0)
+    for w in (n, n + 3):
+        o2, l2 = orc.attention_forward(q, k, v, 0.6, False, w)
+        assert np.max(np.abs(o2 - o)) < 1e-12 and np.max(np.abs(l2 - lse)) < 1e-12
+    w, i = 4, 6
+    o, _ = orc.attention_forward(q, k, v, 0.6, False, w)
+    for j, should_change in ((i - w, False), (i + w, False), (i - w + 1, True), (i + w - 1, True)):
+        k2, v2 = k.copy(), v.copy()
+        k2[..., j, :] += 2.0
+        v2[..., j, :] += 7.0
+        o2, _ = orc.attention_forward(q, k2, v2, 0.6, False, w)
+        diff = np.max(np.abs(o2[..., i, :] - o[..., i, :]))
+        assert (diff > 1e-3) if should_change else (diff < 1e-12), (j, diff)
 
 
 def rejects_bad_masks(orc):
-    """A negative window, or a window without causal, is rejected."""
+    """A negative window is rejected, with or without causal."""
     q, k, v = _qkv(21, n=4, d=2, lead=())
-    for causal, window in ((True, -1), (False, 3)):
+    for causal, window in ((True, -1), (False, -1)):
         try:
             orc.attention_forward(q, k, v, 1.0, causal, window)
         except ValueError:
@@ -312,5 +352,5 @@ PINS = {f.__name__: f for f in (
     rows_sum_to_one, constant_v, causal_row0, causal_future_independence, window_one,
     window_covering_is_causal, window_edge, scale_zero, key_shift, key_permutation,
     large_scores, golden_examples, library_forward, library_backward, finite_differences,
-    delta_identity, row_blocks_match, pair_count, rejects_bad_masks,
+    delta_identity, row_blocks_match, pair_count, two_sided_window, rejects_bad_masks,
 )}

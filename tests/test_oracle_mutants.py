@@ -41,7 +41,20 @@ def _rows_mask_window_wide(r, n_k, causal, window):
     return ok
 
 
-def _rows_mask_no_window_check(r, n_k, causal, window):
+def _rows_mask_two_sided_wide(r, n_k, causal, window):
+    i = r[:, None]
+    j = np.arange(n_k)[None, :]
+    ok = np.ones((r.size, n_k), dtype=bool)
+    if causal:
+        ok &= j <= i
+    if window > 0:
+        ok &= j >= i - window + 1
+        if not causal:
+            ok &= j <= i + window
+    return ok
+
+
+def _rows_mask_one_sided_only(r, n_k, causal, window):
     i = r[:, None]
     j = np.arange(n_k)[None, :]
     ok = np.ones((r.size, n_k), dtype=bool)
@@ -108,7 +121,9 @@ MUTANTS = {
     "scale_dropped": ("_scores", _scores_no_scale),
     "causal_excludes_diagonal": ("_rows_mask", _rows_mask_causal_strict),
     "window_one_too_wide": ("_rows_mask", _rows_mask_window_wide),
-    "window_without_causal_accepted": ("_check_mask_args", lambda causal, window: None),
+    "negative_window_accepted": ("_check_mask_args", lambda causal, window: None),
+    "two_sided_window_one_too_wide": ("_rows_mask", _rows_mask_two_sided_wide),
+    "two_sided_window_upper_edge_missing": ("_rows_mask", _rows_mask_one_sided_only),
     "no_max_shift": ("_softmax_rows", _softmax_no_shift),
     "lse_in_log2": ("_softmax_rows", _softmax_log2),
     "lse_missing_max": ("_softmax_rows", _softmax_lse_no_max),
