@@ -95,7 +95,8 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
 // query tiles (of 128 rows) that can see some key of the tile [kv0, kv0 + 128)
 __device__ __forceinline__ void q_tile_range(int kv0, int N, int causal, int window, int& i_begin, int& i_end) {
   const int n_q = (N + kBwdRows - 1) / kBwdRows;
-  i_begin = causal ? kv0 / kBwdRows : 0;
+  // causal: from the diagonal; a two-sided window: from the first query whose band reaches kv0
+  i_begin = causal ? kv0 / kBwdRows : (window > 0 ? max(0, kv0 - window + 1) / kBwdRows : 0);
   i_end = n_q;
   if (window > 0) {
     const long long last_q = (long long)kv0 + kBwdKeys - 1 + window - 1;   // last query whose band reaches the tile
@@ -395,10 +396,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                  x[2 * j2], x[2 * j2 + 1]);
       }
       if constexpr (decltype(masked)::value) {
-        // the queries that may attend to this key form one range [key, key + W - 1] (causal:
-        // W unbounded without a window; no range at all for a padded key); as columns, [a, b)
+        // the queries that may attend to this key form one range: [key, key + W - 1] (causal;
+        // W unbounded without a window), [key - W + 1, key + W - 1] (two-sided window), or all;
+        // none for a padded key.  As columns, [a, b)
         const int qbase = q0 + hq * 64;
-        const int a = prm.causal ? key - qbase : 0;
+        const int a = prm.causal ? key - qbase : (prm.window > 0 ? key - prm.window + 1 - qbase : 0);
         const int b = key >= prm.N ? a : (prm.window > 0 ? key + prm.window - qbase : 64);
 #pragma unroll
         for (int wd = 0; wd < 2; ++wd) {
@@ -492,7 +494,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     auto run_a = [&](int it) -> bool {
       const int qbase = (i_begin + it) * kBwdRows + hq * 64;
       const bool need_mask = (prm.causal && kv0 + kBwdKeys - 1 > qbase) ||
-                             (prm.window > 0 && kv0 < qbase + 64 - prm.window) || (kv0 + kBwdKeys > prm.N);
+                             (prm.window > 0 && kv0 < qbase + 64 - prm.window) || (kv0 + kBwdKeys > prm.N) ||
+                             (!prm.causal && prm.window > 0 && qbase + prm.window - 1 < kv0 + kBwdKeys - 1);
       return need_mask ? phase_a(it, std::true_type{}) : phase_a(it, std::false_type{});
     };
     ok = run_a(0);

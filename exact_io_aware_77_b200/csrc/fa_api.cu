@@ -78,7 +78,7 @@ int check_problem(int B, int H, int N, int d, float scale, int causal, int windo
   const long long tiles = (N + kBlockM - 1) / kBlockM;
   if (bh > 0x7fffffffLL || bh * tiles > 0x7fffffffLL) return FA_ERR_SHAPE;
   if (d != 64 && d != 128) return FA_ERR_HEADDIM;
-  if (!(causal == 0 || causal == 1) || window < 0 || (window > 0 && !causal)) return FA_ERR_MASK;
+  if (!(causal == 0 || causal == 1) || window < 0) return FA_ERR_MASK;
   if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_SCALE;
   return FA_OK;
 }
@@ -103,7 +103,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   prm.BH = BH;
   prm.n_pairs = ((N + kBlockM - 1) / kBlockM + kQTiles - 1) / kQTiles;
   prm.causal = causal;
-  prm.window = window;
+  prm.window = window > N ? N : window;   // a band of N or more keys is no band at all
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.wait_limit_ns = g_wait_limit_ns;
   // at least 120 KB so that one CTA (and its 512 TMEM columns) owns the SM
@@ -156,7 +156,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   prm.BH = BH;
   prm.n_kv_tiles = (N + kBwdKeys - 1) / kBwdKeys;
   prm.causal = causal;
-  prm.window = window;
+  prm.window = window > N ? N : window;   // a band of N or more keys is no band at all
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.scale = scale;
   prm.wait_limit_ns = g_wait_limit_ns;
@@ -273,7 +273,7 @@ const char* fa_status_string(int status) {
     case FA_ERR_SHAPE: return "bad shape (B, H, N must be >= 1 and within launch limits)";
     case FA_ERR_HEADDIM: return "unsupported head dimension (64 or 128)";
     case FA_ERR_ALIGN: return "misaligned pointer (bf16 arrays 16 B, L 4 B)";
-    case FA_ERR_MASK: return "bad mask (causal 0/1, window >= 0, window needs causal)";
+    case FA_ERR_MASK: return "bad mask (causal must be 0 or 1, window >= 0)";
     case FA_ERR_WORKSPACE: return "backward workspace missing or too small";
     case FA_ERR_CUDA: return "CUDA runtime or launch error";
     case FA_ERR_DEVICE: return "device is not compute capability 10.0 (B200)";

@@ -83,7 +83,9 @@ __device__ __forceinline__ void kv_tile_range(int q0, int N, int causal, int win
     t_begin = t_end = 0;
     return;
   }
-  const int kv_end = causal ? min(N, q0 + kBlockM) : N;
+  // the tile's last query attends keys up to itself (causal), up to itself + W - 1 (two-sided
+  // window), or all of them
+  const int kv_end = causal ? min(N, q0 + kBlockM) : (window > 0 ? min(N, q0 + kBlockM - 1 + window) : N);
   t_end = (kv_end + kBlockN - 1) / kBlockN;
   const int kv_begin = window > 0 ? max(0, q0 - window + 1) : 0;
   t_begin = kv_begin / kBlockN;
@@ -284,7 +286,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
         if constexpr (decltype(masked)::value) {
           // allowed keys of this row form one range [lo, hi]; as columns of the tile, [a, b)
-          const int hi = prm.causal ? min(qi, prm.N - 1) : prm.N - 1;
+          const int hi = prm.causal ? min(qi, prm.N - 1)
+                                    : (prm.window > 0 ? min(qi + prm.window - 1, prm.N - 1) : prm.N - 1);
           const int lo = prm.window > 0 ? qi - prm.window + 1 : 0;
           const int a = lo - kv0, b = hi - kv0 + 1;
 #pragma unroll
@@ -371,7 +374,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     for (int t = tb; t < te; ++t) {
       const int kv0 = t * kBlockN;
       const bool need_mask = (kv0 + kBlockN > prm.N) || (prm.causal && kv0 + kBlockN - 1 > qw0) ||
-                             (prm.window > 0 && kv0 < qw0 + kBlockM - prm.window);
+                             (prm.window > 0 && kv0 < qw0 + kBlockM - prm.window) ||
+                             (!prm.causal && prm.window > 0 && kv0 + kBlockN - 1 > qw0 + prm.window - 1);
       ok = need_mask ? step(t, std::true_type{}) : step(t, std::false_type{});
       if (!ok) break;
     }

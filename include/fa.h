@@ -24,10 +24,13 @@
  *   Streams    `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *              Every call only enqueues work on that stream and returns; it never
  *              synchronises (fa_check_status excepted).
- *   Masks      causal = 1 keeps key j for query i iff j <= i.  window = W > 0 (needs
- *              causal = 1) also requires j >= i - W + 1, so the band counts the diagonal
- *              and W = 1 keeps only key i.  window = 0 means no band.  Keys j >= N never
- *              exist.  Every query keeps its diagonal, so no row is empty.
+ *   Masks      causal = 1 keeps key j for query i iff j <= i.  window = W > 0 with
+ *              causal = 1 also requires j >= i - W + 1 (one-sided band); with causal = 0
+ *              it keeps |i - j| <= W - 1 (the local window on both sides).  Either band
+ *              counts the diagonal, so W = 1 keeps only key i; window = 0 means no band.
+ *              (The sparse-attention glossary, "Abgrenzung & Vergleiche", names sliding-
+ *              window attention as a purely local window and fixes no convention.)  Keys
+ *              j >= N never exist.  Every query keeps its diagonal, so no row is empty.
  *   Scale      applied inside: S = scale * Q K^T.  Must be finite and > 0.
  *   Errors     arguments are validated before anything is enqueued; a rejected call
  *              returns its FA_ERR_* code and touches no memory.  A failed launch returns
@@ -57,7 +60,7 @@ typedef enum {
   FA_ERR_SHAPE = 2,      /* B, H or N < 1, or the problem exceeds the launch limits */
   FA_ERR_HEADDIM = 3,    /* d is not 64 or 128 */
   FA_ERR_ALIGN = 4,      /* a bf16 array is not 16-byte aligned, or L not 4-byte aligned */
-  FA_ERR_MASK = 5,       /* causal not 0/1, window < 0, or window > 0 without causal */
+  FA_ERR_MASK = 5,       /* causal not 0/1, or window < 0 */
   FA_ERR_WORKSPACE = 6,  /* backward workspace missing or smaller than fa_bwd_workspace_size */
   FA_ERR_CUDA = 7,       /* a CUDA runtime call or kernel launch failed */
   FA_ERR_DEVICE = 8,     /* the current device is not compute capability 10.0 */

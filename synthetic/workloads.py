@@ -30,7 +30,7 @@ class Workload:
     N: int
     d: int
     causal: bool = False
-    window: int = 0          # 0 = no band; W > 0 keeps keys i-W+1 .. i (causal only)
+    window: int = 0          # 0 = no band; W > 0 keeps keys i-W+1 .. i (causal) or |i-j| <= W-1
     std: float = 1.0
     seed: int = 0
     grad_seed: int | None = None   # seed of dO (backward workloads)
@@ -64,6 +64,9 @@ WORKLOADS: dict[str, Workload] = {
     "long": Workload("long", 1, 16, 32768, 128, causal=True, window=4096, seed=1005,
                      oracle_heads=2,
                      description="long-context forward B1 H16 N32768 d128 causal+window 4096"),
+    # the same length with the local window on both sides (non-causal sliding-window attention)
+    "swa": Workload("swa", 1, 16, 32768, 128, window=4096, seed=1006, grad_seed=2006, oracle_heads=2,
+                    description="long-context two-sided window B1 H16 N32768 d128, |i-j| < 4096"),
 }
 
 

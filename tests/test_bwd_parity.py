@@ -41,6 +41,9 @@ EDGE = [
     (1, 2, 300, 64, True, 7), (1, 2, 300, 128, True, 1), (1, 2, 640, 128, True, 129),
     (1, 2, 1000, 128, True, 200), (1, 1, 1000, 64, True, 2000), (2, 1, 777, 128, False, 0),
     (1, 2, 1024, 128, True, 0), (1, 1, 1536, 64, False, 0),
+    # two-sided local windows (causal = 0)
+    (1, 2, 300, 128, False, 1), (1, 2, 300, 64, False, 7), (1, 2, 1000, 128, False, 200),
+    (1, 1, 640, 128, False, 129), (2, 1, 777, 64, False, 2000),
 ]
 
 
@@ -65,10 +68,11 @@ def test_workload_bwd_full_size_head_sample(fa):
     assert_grads_close([sel(g) for g in grads], refs, ("bwd", heads))
 
 
-def test_long_window_backward_sampled(fa):
-    """N = 32768 with a 4096 window (the long-context shape, 2 heads): dK/dV on sampled key rows
-    and dQ on one row block, against the oracle's row-block backward."""
-    wl = WORKLOADS["long"].with_(H=2)
+@pytest.mark.parametrize("name", ["long", "swa"])
+def test_long_window_backward_sampled(fa, name):
+    """N = 32768 with a 4096 window (one-sided and two-sided long-context shapes, 2 heads): dK/dV
+    on sampled key rows and dQ on one row block, against the oracle's row-block backward."""
+    wl = WORKLOADS[name].with_(H=2)
     q, k, v = make_inputs(wl)
     do = make_grad_output(wl, seed=2005)
     dq, dk, dv = _gpu_grads(fa, wl, q, k, v, do)
@@ -79,12 +83,12 @@ def test_long_window_backward_sampled(fa):
     h = 1
     qh, kh, vh, doh = (x[0, h] for x in (q, k, v, do))
     # dK/dV need every query row; dQ only its own rows
-    _, dk_ref, dv_ref = orc.attention_backward_rows(qh, kh, vh, doh, wl.scale, True, wl.window,
+    _, dk_ref, dv_ref = orc.attention_backward_rows(qh, kh, vh, doh, wl.scale, wl.causal, wl.window,
                                                     key_rows=key_rows)
-    dq_ref, _, _ = orc.attention_backward_rows(qh, kh, vh, doh, wl.scale, True, wl.window,
+    dq_ref, _, _ = orc.attention_backward_rows(qh, kh, vh, doh, wl.scale, wl.causal, wl.window,
                                                key_rows=key_rows[:1], query_rows=qrows)
     assert_grads_close([dq[0, h][qrows], dk[0, h][key_rows], dv[0, h][key_rows]],
-                       [dq_ref, dk_ref, dv_ref], "long")
+                       [dq_ref, dk_ref, dv_ref], name)
 
 
 def test_workspace_and_guard_bands(fa):

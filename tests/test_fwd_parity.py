@@ -41,6 +41,9 @@ EDGE = [
     (1, 2, 300, 64, True, 1), (1, 3, 1000, 128, True, 128), (1, 2, 1000, 64, True, 200),
     (1, 2, 777, 128, True, 2000), (1, 1, 640, 128, True, 129), (2, 2, 513, 64, False, 0),
     (1, 2, 1024, 128, True, 0), (1, 1, 2048, 64, False, 0), (1, 2, 900, 128, True, 256),
+    # two-sided local windows (causal = 0): narrower, equal to and wider than a tile, ragged N
+    (1, 2, 300, 128, False, 1), (1, 2, 300, 64, False, 5), (2, 2, 1000, 128, False, 128),
+    (1, 2, 777, 64, False, 200), (1, 1, 640, 128, False, 129), (1, 2, 513, 128, False, 2000),
 ]
 
 
@@ -93,8 +96,9 @@ def test_workload_full_size_head_sample(fa, name, n_heads):
                          o_ref, l_ref, (name, heads))
 
 
-def test_workload_long_window_sampled_rows(fa):
-    wl = WORKLOADS["long"]
+@pytest.mark.parametrize("name", ["long", "swa"])
+def test_workload_long_window_sampled_rows(fa, name):
+    wl = WORKLOADS[name]
     (q, k, v), o, lse = _run(fa, wl)
     rng = np.random.default_rng(wl.seed)
     rows = np.unique(np.concatenate([
@@ -104,7 +108,7 @@ def test_workload_long_window_sampled_rows(fa):
         qh, kh, vh = (x.reshape(wl.BH, wl.N, wl.d)[h] for x in (q, k, v))
         o_ref, l_ref = orc.attention_forward_rows(qh, kh, vh, wl.scale, wl.causal, wl.window, rows=rows)
         assert_forward_close(o.reshape(wl.BH, wl.N, wl.d)[h][rows], lse.reshape(wl.BH, wl.N)[h][rows],
-                             o_ref, l_ref, ("long", h))
+                             o_ref, l_ref, (name, h))
 
 
 def test_guard_bands_untouched(fa):
