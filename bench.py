@@ -39,6 +39,8 @@ if ROOT not in sys.path:
 
 WORKLOAD = "causal"          # forward workload; the backward uses the same shape
 GRAD_WORKLOAD = "bwd"
+# --workload choices: the forward workload and the one whose dO seed the backward uses
+BENCH_WORKLOADS = {"causal": ("causal", "bwd"), "long": ("long", "long"), "swa": ("swa", "swa")}
 FLUSH_BYTES = 256 << 20      # > 126 MB L2
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -54,17 +56,31 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--workload", choices=sorted(BENCH_WORKLOADS), default="causal",
+                    help="causal: B2 H32 N4096 d128 (the default line); long / swa: N32768 with a "
+                         "one- / two-sided window of 4096, FLOPs counted over the pairs the band keeps")
     return ap.parse_args()
 
 
 # ----------------------------------------------------------------------------- FLOPs
-def fwd_flops(B, H, N, d, causal) -> float:
+def band_pairs(N, causal, window) -> int:
+    """(query, key) pairs a banded mask keeps in N x N self-attention (closed forms)."""
+    w = min(window, N)
+    if causal:
+        return w * (w + 1) // 2 + (N - w) * w
+    return N * (2 * w - 1) - w * (w - 1)
+
+
+def fwd_flops(B, H, N, d, causal, window=0) -> float:
+    """4 B H N^2 d, halved if causal; with a window, 4 d per pair the band keeps."""
+    if window > 0:
+        return 4.0 * B * H * d * band_pairs(N, causal, window)
     f = 4.0 * B * H * N * N * d
     return f / 2 if causal else f
 
 
-def bwd_flops(B, H, N, d, causal) -> float:
-    return 2.5 * fwd_flops(B, H, N, d, causal)
+def bwd_flops(B, H, N, d, causal, window=0) -> float:
+    return 2.5 * fwd_flops(B, H, N, d, causal, window)
 
 
 def max_over_ranks(values, device=None):
@@ -188,9 +204,9 @@ def oracle_sample(seconds: float, rows_per_block: int = 512, with_bwd: bool = Tr
     q, k, v = (x[0, 0] for x in make_inputs(sub))
     do = make_grad_output(WORKLOADS[GRAD_WORKLOAD].with_(B=1, H=1))[0, 0]
     q, k, v, do = (x.double().numpy() for x in (q, k, v, do))
-    per_row = fwd_flops(1, 1, wl.N, wl.d, wl.causal) / wl.N
+    per_row = fwd_flops(1, 1, wl.N, wl.d, wl.causal, wl.window) / wl.N
     if with_bwd:
-        per_row += bwd_flops(1, 1, wl.N, wl.d, wl.causal) / wl.N
+        per_row += bwd_flops(1, 1, wl.N, wl.d, wl.causal, wl.window) / wl.N
     t0 = time.perf_counter()
     blocks = 0
     start = 0
@@ -250,8 +266,8 @@ def run_ours(args):
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    f_fwd = fwd_flops(B, H, N, d, wl.causal)
-    f_bwd = bwd_flops(B, H, N, d, wl.causal) if has_bwd else 0.0
+    f_fwd = fwd_flops(B, H, N, d, wl.causal, wl.window)
+    f_bwd = bwd_flops(B, H, N, d, wl.causal, wl.window) if has_bwd else 0.0
 
     def step(ev=None):
         # forward, then the backward as its three phases (exactly fa_bwd) so that the recompute
@@ -329,15 +345,17 @@ def run_ours(args):
                 "frac": round(achieved / peaks["bf16_tflops"], 4),
                 "peak_source": f"{peak_kind} burst bf16 (MEASURED_PEAKS.json)" if peak_kind == "measured"
                 else "fallback 1.59 PFLOP/s",
-                "traffic": load_traffic(dom)}
+                # the ncu counters were taken on the default causal workload only
+                "traffic": load_traffic(dom) if WORKLOAD == "causal" else None}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         flops, secs, blocks, cores = oracle_sample(args.cpu_seconds, with_bwd=has_bwd)
         cpu = {"value": round(flops / secs / 1e12, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-               "sample": f"{blocks} blocks of 512 query rows of head 0 of the B2 H32 N4096 d128 causal "
-                         f"workload through the fp64 oracle ({'fwd+bwd' if has_bwd else 'fwd'}), "
-                         f"{secs:.1f} s, credited rows/N of a head's conventional FLOPs"}
+               "sample": f"{blocks} blocks of 512 query rows of head 0 of the {wl.name} workload "
+                         f"(B{wl.B} H{wl.H} N{wl.N} d{wl.d}) through the fp64 oracle "
+                         f"({'fwd+bwd' if has_bwd else 'fwd'}), {secs:.1f} s, credited rows/N of a "
+                         f"head's FLOPs"}
 
     clocks = sampler.summary()
     line = {
@@ -345,9 +363,7 @@ def run_ours(args):
         "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": ("causal LLM shape forward+backward" if has_bwd else
-                                "causal LLM shape forward (backward not built yet)") +
-                   f": B={B} H={H} N={N} d={d} causal, inputs N(0,1)*0.5 bf16 seeded",
+        "config": {"workload": workload_text(wl, has_bwd),
                    "global_batch": B * world, "seq_len": N, "parallelism": f"replicas{world}",
                    "l2": "flushed (256 MB write) between timed steps, outside the events"},
         "fwd_tflops": round(job_throughput(world, f_fwd, fwd_ms_avg), 2),
@@ -461,17 +477,16 @@ def run_reference(args):
             flops.append(f)
     secs = sum(times)
     value = sum(flops) / secs / 1e12
-    sample = (f"each step: 128 query rows of head 0 of the B2 H32 N4096 d128 causal workload through "
-              f"the fp64 oracle ({'fwd+bwd' if with_bwd else 'fwd'}), credited rows/N of a head's "
-              f"conventional FLOPs")
+    sample = (f"each step: 128 query rows of head 0 of the {wl.name} workload (B{wl.B} H{wl.H} N{wl.N} "
+              f"d{wl.d}) through the fp64 oracle ({'fwd+bwd' if with_bwd else 'fwd'}), credited rows/N "
+              f"of a head's FLOPs")
     line = {
         "metric": "attention fwd/bwd TFLOP/s at 1 B200; % of dense BF16 tensor peak",
         "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * secs / args.steps, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "impl": "reference",
-        "config": {"workload": f"causal LLM shape {'forward+backward' if with_bwd else 'forward'}: "
-                               f"B={wl.B} H={wl.H} N={wl.N} d={wl.d} causal (row-block sample)",
+        "config": {"workload": workload_text(wl, with_bwd) + " (row-block sample)",
                    "global_batch": wl.B, "seq_len": wl.N, "parallelism": "cpu"},
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
@@ -480,8 +495,21 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def workload_text(wl, with_bwd: bool) -> str:
+    if wl.window:
+        band = (f"{'causal' if wl.causal else 'two-sided'} window {wl.window}, FLOPs over the "
+                f"{band_pairs(wl.N, wl.causal, wl.window)} kept pairs per head")
+        kind = "long-context"
+    else:
+        band, kind = ("causal" if wl.causal else "no mask"), "causal LLM shape"
+    return (f"{kind} {'forward+backward' if with_bwd else 'forward'}: B={wl.B} H={wl.H} N={wl.N} "
+            f"d={wl.d} {band}, inputs N(0,1)*{wl.std:g} bf16 seeded")
+
+
 def main():
+    global WORKLOAD, GRAD_WORKLOAD
     args = parse_args()
+    WORKLOAD, GRAD_WORKLOAD = BENCH_WORKLOADS[args.workload]
     if args.impl == "reference":
         run_reference(args)
     else:
