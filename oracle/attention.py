@@ -38,6 +38,13 @@ Vergleiche"):
   W = 0:    no band.
 Every row keeps its diagonal, so no row is ever fully masked.
 
+Shared K/V heads.  The pages list Multi-Query Attention among what FlashAttention-2
+supports (FlashAttention (NL), "Evolutie en verdere ontwikkelingen",
+FlashAttention-2): several query heads read one K/V head.  Reading, generalised to
+H_kv K/V heads for H query heads (H a multiple of H_kv; H_kv = 1 is MQA): query head
+h reads K/V head h // (H / H_kv), so each K/V head serves a contiguous group of query
+heads, and its gradient is the sum over that group.
+
 Arithmetic is numpy float64 with ``@`` (BLAS DGEMM) as the only library step.
 Parity of every function here is pinned by tests/test_oracle.py.
 """
@@ -54,6 +61,9 @@ __all__ = [
     "attention_forward_rows",
     "attention_backward_rows",
     "allowed_pairs",
+    "kv_head_of",
+    "attention_forward_shared_kv",
+    "attention_backward_shared_kv",
 ]
 
 
@@ -219,6 +229,33 @@ def attention_backward_rows(q, k, v, do, scale: float, causal: bool = False, win
         dq[sel] = scale * (ds @ k)
         dk += scale * (ds[:, key_rows].T @ q[r])
         dv += p[:, key_rows].T @ do[r]
+    return dq, dk, dv
+
+
+def kv_head_of(n_heads: int, n_kv_heads: int) -> np.ndarray:
+    """K/V head read by each of n_heads query heads (contiguous groups)."""
+    if n_kv_heads < 1 or n_heads % n_kv_heads:
+        raise ValueError("the query heads must be a whole multiple of the K/V heads")
+    return np.arange(n_heads) // (n_heads // n_kv_heads)
+
+
+def attention_forward_shared_kv(q, k, v, scale: float, causal: bool = False, window: int = 0):
+    """Forward with shared K/V heads: q [..., H, N, d]; k, v [..., H_kv, N, d]."""
+    q, k, v = _as64(q), _as64(k), _as64(v)
+    idx = kv_head_of(q.shape[-3], k.shape[-3])
+    return attention_forward(q, k[..., idx, :, :], v[..., idx, :, :], scale, causal, window)
+
+
+def attention_backward_shared_kv(q, k, v, do, scale: float, causal: bool = False, window: int = 0):
+    """Gradients with shared K/V heads: dQ [..., H, N, d]; dK, dV [..., H_kv, N, d], each K/V
+    head's gradient summed over the query heads that read it."""
+    q, k, v, do = _as64(q), _as64(k), _as64(v), _as64(do)
+    h, h_kv = q.shape[-3], k.shape[-3]
+    idx = kv_head_of(h, h_kv)
+    dq, dk, dv = attention_backward(q, k[..., idx, :, :], v[..., idx, :, :], do, scale, causal, window)
+    group = (h_kv, h // h_kv)
+    dk = dk.reshape(dk.shape[:-3] + group + dk.shape[-2:]).sum(axis=-3)
+    dv = dv.reshape(dv.shape[:-3] + group + dv.shape[-2:]).sum(axis=-3)
     return dq, dk, dv
 
 

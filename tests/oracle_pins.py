@@ -337,6 +337,59 @@ def two_sided_window(orc):
         assert (diff > 1e-3) if should_change else (diff < 1e-12), (j, diff)
 
 
+def shared_kv_library(orc):
+    """Shared K/V heads (MQA: 1 K/V head; GQA: 2 for 4 query heads) agree with torch
+    scaled_dot_product_attention(enable_gqa=True) and its autograd in float64, for every mask."""
+    import torch
+    import torch.nn.functional as F
+    r = _rng(23)
+    for h_kv in (1, 2, 4):
+        q = r.standard_normal((2, 4, 11, 5))
+        k, v = (r.standard_normal((2, h_kv, 11, 5)) for _ in range(2))
+        do = r.standard_normal(q.shape)
+        n = q.shape[-2]
+        i = torch.arange(n)[:, None]
+        j = torch.arange(n)[None, :]
+        for causal, window in MASKS:
+            ok = torch.ones(n, n, dtype=torch.bool)
+            if causal:
+                ok &= j <= i
+            if window:
+                ok &= (j - i).abs() <= window - 1 if not causal else j >= i - window + 1
+            tq, tk, tv = (torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (q, k, v))
+            o_ref = F.scaled_dot_product_attention(tq, tk, tv, attn_mask=ok, scale=0.35, enable_gqa=True)
+            (o_ref * torch.tensor(do)).sum().backward()
+            o, _ = orc.attention_forward_shared_kv(q, k, v, 0.35, causal, window)
+            assert np.max(np.abs(o - o_ref.detach().numpy())) < 1e-12, (h_kv, causal, window)
+            grads = orc.attention_backward_shared_kv(q, k, v, do, 0.35, causal, window)
+            for mine, ref in zip(grads, (tq.grad, tk.grad, tv.grad)):
+                assert mine.shape == ref.shape
+                assert np.max(np.abs(mine - ref.numpy())) < 1e-11, (h_kv, causal, window)
+
+
+def shared_kv_finite_differences(orc):
+    """Central differences of sum(O o dO) with respect to a shared K/V head match dK and dV."""
+    r = _rng(24)
+    q = r.standard_normal((3, 6, 3))
+    k, v = (r.standard_normal((1, 6, 3)) for _ in range(2))
+    do = r.standard_normal(q.shape)
+    h = 1e-6
+    for causal, window in ((True, 0), (False, 2)):
+        _, dk, dv = orc.attention_backward_shared_kv(q, k, v, do, 0.7, causal, window)
+
+        def f(kk, vv):
+            return float(np.sum(orc.attention_forward_shared_kv(q, kk, vv, 0.7, causal, window)[0] * do))
+
+        for which, g in ((0, dk), (1, dv)):
+            fd = np.zeros_like(g)
+            for idx in np.ndindex(g.shape):
+                plus, minus = [k.copy(), v.copy()], [k.copy(), v.copy()]
+                plus[which][idx] += h
+                minus[which][idx] -= h
+                fd[idx] = (f(*plus) - f(*minus)) / (2 * h)
+            assert np.linalg.norm(fd - g) / np.linalg.norm(fd) < 1e-6, (which, causal, window)
+
+
 def rejects_bad_masks(orc):
     """A negative window is rejected, with or without causal."""
     q, k, v = _qkv(21, n=4, d=2, lead=())
@@ -352,5 +405,6 @@ PINS = {f.__name__: f for f in (
     rows_sum_to_one, constant_v, causal_row0, causal_future_independence, window_one,
     window_covering_is_causal, window_edge, scale_zero, key_shift, key_permutation,
     large_scores, golden_examples, library_forward, library_backward, finite_differences,
-    delta_identity, row_blocks_match, pair_count, two_sided_window, rejects_bad_masks,
+    delta_identity, row_blocks_match, pair_count, two_sided_window, shared_kv_library,
+    shared_kv_finite_differences, rejects_bad_masks,
 )}

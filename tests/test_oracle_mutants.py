@@ -116,6 +116,18 @@ def _head_forward_pv_transposed(q, k, v, scale, causal, window, row_start=0):
     return p.T @ v, lse, p
 
 
+def _kv_head_interleaved(n_heads, n_kv_heads):
+    return np.arange(n_heads) % n_kv_heads
+
+
+def _backward_shared_kv_first_only(q, k, v, do, scale, causal=False, window=0):
+    q, k, v, do = orc._as64(q), orc._as64(k), orc._as64(v), orc._as64(do)
+    idx = orc.kv_head_of(q.shape[-3], k.shape[-3])
+    dq, dk, dv = orc.attention_backward(q, k[..., idx, :, :], v[..., idx, :, :], do, scale, causal, window)
+    g = q.shape[-3] // k.shape[-3]
+    return dq, dk[..., ::g, :, :], dv[..., ::g, :, :]
+
+
 MUTANTS = {
     "scores_transposed": ("_scores", _scores_transposed),
     "scale_dropped": ("_scores", _scores_no_scale),
@@ -133,6 +145,8 @@ MUTANTS = {
     "delta_missing": ("_head_backward", _make_bwd("delta_missing")),
     "dq_no_scale": ("_head_backward", _make_bwd("dq_no_scale")),
     "dk_untransposed": ("_head_backward", _make_bwd("dk_untransposed")),
+    "kv_heads_interleaved": ("kv_head_of", _kv_head_interleaved),
+    "shared_kv_grad_not_summed": ("attention_backward_shared_kv", _backward_shared_kv_first_only),
 }
 
 
