@@ -40,7 +40,8 @@ if ROOT not in sys.path:
 WORKLOAD = "causal"          # forward workload; the backward uses the same shape
 GRAD_WORKLOAD = "bwd"
 # --workload choices: the forward workload and the one whose dO seed the backward uses
-BENCH_WORKLOADS = {"causal": ("causal", "bwd"), "long": ("long", "long"), "swa": ("swa", "swa")}
+BENCH_WORKLOADS = {"causal": ("causal", "bwd"), "long": ("long", "long"), "swa": ("swa", "swa"),
+                   "gqa": ("gqa", "gqa")}
 FLUSH_BYTES = 256 << 20      # > 126 MB L2
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -57,8 +58,9 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--workload", choices=sorted(BENCH_WORKLOADS), default="causal",
-                    help="causal: B2 H32 N4096 d128 (the default line); long / swa: N32768 with a "
-                         "one- / two-sided window of 4096, FLOPs counted over the pairs the band keeps")
+                    help="causal: B2 H32 N4096 d128 (the default line); gqa: the same with 8 K/V heads; "
+                         "long / swa: N32768 with a one- / two-sided window of 4096, FLOPs counted over "
+                         "the pairs the band keeps")
     return ap.parse_args()
 
 
@@ -200,9 +202,9 @@ def oracle_sample(seconds: float, rows_per_block: int = 512, with_bwd: bool = Tr
     from oracle import attention as orc
     from synthetic import WORKLOADS, make_grad_output, make_inputs
     wl = WORKLOADS[WORKLOAD]
-    sub = wl.with_(B=1, H=1)
+    sub = wl.with_(B=1, H=1, H_kv=None)
     q, k, v = (x[0, 0] for x in make_inputs(sub))
-    do = make_grad_output(WORKLOADS[GRAD_WORKLOAD].with_(B=1, H=1))[0, 0]
+    do = make_grad_output(WORKLOADS[GRAD_WORKLOAD].with_(B=1, H=1, H_kv=None))[0, 0]
     q, k, v, do = (x.double().numpy() for x in (q, k, v, do))
     per_row = fwd_flops(1, 1, wl.N, wl.d, wl.causal, wl.window) / wl.N
     if with_bwd:
@@ -259,7 +261,7 @@ def run_ours(args):
     q, k, v, do = (x.to(dev) for x in (q_h, k_h, v_h, do_h))
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
-    grads = (torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)) if has_bwd else None
+    grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)) if has_bwd else None
     ws = None
     if has_bwd:
         ws = torch.empty(fa.bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
@@ -399,11 +401,11 @@ def measure_e2e(fa, torch, wl, dev, stream, q_h, k_h, v_h, do_h, has_bwd, steps,
     l_h = torch.empty((wl.B, wl.H, wl.N), dtype=torch.float32).pin_memory()
     grads = grads_h = ws = None
     if has_bwd:
-        grads = tuple(torch.empty_like(q) for _ in range(3))
-        grads_h = tuple(torch.empty_like(pin[0]).pin_memory() for _ in range(3))
+        grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+        grads_h = tuple(torch.empty_like(pin[i]).pin_memory() for i in range(3))
         ws = torch.empty(fa.bwd_workspace_size(wl.B, wl.H, wl.N, wl.d), dtype=torch.uint8, device=dev)
     h2d = sum(x.numel() * x.element_size() for x in pin)
-    d2h = o_h.numel() * 2 + l_h.numel() * 4 + (3 * o_h.numel() * 2 if has_bwd else 0)
+    d2h = o_h.numel() * 2 + l_h.numel() * 4 + (sum(g.numel() * 2 for g in grads_h) if has_bwd else 0)
 
     def one():
         for dst, src in zip((q, k, v) + ((do,) if has_bwd else ()), pin):
@@ -502,7 +504,8 @@ def workload_text(wl, with_bwd: bool) -> str:
         kind = "long-context"
     else:
         band, kind = ("causal" if wl.causal else "no mask"), "causal LLM shape"
-    return (f"{kind} {'forward+backward' if with_bwd else 'forward'}: B={wl.B} H={wl.H} N={wl.N} "
+    heads = f"H={wl.H}" + (f" (K/V heads {wl.kv_heads})" if wl.kv_heads != wl.H else "")
+    return (f"{kind} {'forward+backward' if with_bwd else 'forward'}: B={wl.B} {heads} N={wl.N} "
             f"d={wl.d} {band}, inputs N(0,1)*{wl.std:g} bf16 seeded")
 
 

@@ -1,8 +1,10 @@
 """Exact, IO-aware attention for B200 (sm_100a).
 
 ``forward`` and ``backward`` take contiguous bf16 CUDA tensors of shape
-[B, H, N, d] and run the hand-written kernels of libfa_b200.so on the current
-torch stream.  torch supplies device memory and streams only.
+[B, H, N, d] (K and V may have fewer heads, H_kv, with H a multiple of H_kv:
+multi-query / grouped-query attention) and run the hand-written kernels of
+libfa_b200.so on the current torch stream.  torch supplies device memory and
+streams only.
 """
 
 from __future__ import annotations
@@ -25,14 +27,20 @@ def _stream_handle(device) -> int:
     return torch.cuda.current_stream(device).cuda_stream
 
 
-def _check_qkv(*ts):
+def _check_qkv(q, k, v, *rest):
+    """q (and o, dO in rest): [B, H, N, d]; k, v: [B, H_kv, N, d] with H a multiple of H_kv."""
     import torch
-    t0 = ts[0]
-    for t in ts:
+    for t in (q, k, v) + rest:
         if not (t.is_cuda and t.dtype == torch.bfloat16 and t.dim() == 4 and t.is_contiguous()):
             raise ValueError("expected contiguous bf16 CUDA tensors of shape [B, H, N, d]")
-        if t.shape != t0.shape or t.device != t0.device:
-            raise ValueError("shape/device mismatch")
+        if t.device != q.device:
+            raise ValueError("device mismatch")
+    if any(t.shape != q.shape for t in rest) or k.shape != v.shape:
+        raise ValueError("shape mismatch")
+    B, H, N, d = q.shape
+    if k.shape[0] != B or k.shape[2:] != (N, d) or k.shape[1] < 1 or H % k.shape[1]:
+        raise ValueError("k and v must be [B, H_kv, N, d] with H a multiple of H_kv")
+    return int(k.shape[1])
 
 
 def _raise(name, st):
@@ -44,16 +52,19 @@ def forward(q, k, v, scale: float | None = None, causal: bool = False, window: i
             out=None, lse=None):
     """O, L = attention(Q, K, V); O bf16 [B,H,N,d], L fp32 [B,H,N] (natural-log logsumexp)."""
     import torch
-    _check_qkv(q, k, v)
+    H_kv = _check_qkv(q, k, v)
     B, H, N, d = q.shape
     scale = default_scale(d) if scale is None else float(scale)
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    st = _lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                     B, H, N, d, scale, int(bool(causal)), int(window), _stream_handle(q.device))
-    _raise("fa_fwd", st)
+    ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr())
+    mask = (scale, int(bool(causal)), int(window), _stream_handle(q.device))
+    if H_kv == H:
+        _raise("fa_fwd", _lib.fa_fwd(*ptrs, B, H, N, d, *mask))
+    else:
+        _raise("fa_fwd_gqa", _lib.fa_fwd_gqa(*ptrs, B, H, H_kv, N, d, *mask))
     return out, lse
 
 
@@ -67,26 +78,31 @@ def bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
 
 def backward(q, k, v, o, lse, do, scale: float | None = None, causal: bool = False, window: int = 0,
              grads=None, workspace=None, phases: int = 7):
-    """dQ, dK, dV (bf16 [B,H,N,d]) of sum(O o dO), recomputing P from the forward's L.
+    """dQ (like q), dK, dV (like k) of sum(O o dO), recomputing P from the forward's L.
 
     ``phases`` selects the steps of the backward (1 preprocess, 2 recompute kernel, 4 dQ
     finalise); running 1, 2, 4 in turn with the same workspace equals the default 7.
     """
     import torch
-    _check_qkv(q, k, v, o, do)
+    H_kv = _check_qkv(q, k, v, o, do)
     B, H, N, d = q.shape
     if not (lse.is_cuda and lse.dtype == torch.float32 and lse.is_contiguous() and lse.numel() == B * H * N):
         raise ValueError("lse must be a contiguous fp32 CUDA tensor of B*H*N elements")
     scale = default_scale(d) if scale is None else float(scale)
     if grads is None:
-        grads = (torch.empty_like(q), torch.empty_like(q), torch.empty_like(q))
+        grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
     need = bwd_workspace_size(B, H, N, d)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     dq, dk, dv = grads
-    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
-            dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, scale, int(bool(causal)), int(window),
-            workspace.data_ptr(), workspace.numel() * workspace.element_size())
+    ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+            dq.data_ptr(), dk.data_ptr(), dv.data_ptr())
+    rest = (d, scale, int(bool(causal)), int(window), workspace.data_ptr(),
+            workspace.numel() * workspace.element_size())
+    if H_kv != H:
+        _raise("fa_bwd_gqa", _lib.fa_bwd_gqa(*ptrs, B, H, H_kv, N, *rest, int(phases), _stream_handle(q.device)))
+        return dq, dk, dv
+    args = ptrs + (B, H, N) + rest
     if phases == 7:
         _raise("fa_bwd", _lib.fa_bwd(*args, _stream_handle(q.device)))
     else:

@@ -35,6 +35,9 @@ SIGNATURES = {
     "fa_bwd_phases": (_c_int, [_c_void_p] * 9 + [_c_int] * 4 + [_c_float, _c_int, _c_int, _c_void_p, _c_size_t,
                                                                 _c_int, _c_void_p]),
     "fa_bwd_noalloc": (_c_int, [_c_void_p] * 9 + [_c_int] * 4 + [_c_float, _c_int, _c_int, _c_void_p]),
+    "fa_fwd_gqa": (_c_int, [_c_void_p] * 5 + [_c_int] * 5 + [_c_float, _c_int, _c_int, _c_void_p]),
+    "fa_bwd_gqa": (_c_int, [_c_void_p] * 9 + [_c_int] * 5 + [_c_float, _c_int, _c_int, _c_void_p, _c_size_t,
+                                                             _c_int, _c_void_p]),
     "fa_status_string": (ctypes.c_char_p, [_c_int]),
     "fa_check_status": (_c_int, [_c_void_p]),
     "fa_set_wait_limit_ns": (None, [_c_ull]),
@@ -106,6 +109,18 @@ def fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal, w
     """fa_bwd with the library's built-in 64 MiB scratch instead of a caller workspace."""
     return _call("fa_bwd_noalloc", q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal, window,
                  stream)
+
+
+def fa_fwd_gqa(q, k, v, o, lse, B, H, H_kv, N, d, scale, causal, window, stream) -> int:
+    """fa_fwd with H_kv K/V heads shared by contiguous groups of the H query heads."""
+    return _call("fa_fwd_gqa", q, k, v, o, lse, B, H, H_kv, N, d, scale, causal, window, stream)
+
+
+def fa_bwd_gqa(q, k, v, o, lse, dO, dq, dk, dv, B, H, H_kv, N, d, scale, causal, window, workspace,
+               workspace_bytes, phases, stream) -> int:
+    """fa_bwd_phases with H_kv shared K/V heads; dk, dv are [B, H_kv, N, d]."""
+    return _call("fa_bwd_gqa", q, k, v, o, lse, dO, dq, dk, dv, B, H, H_kv, N, d, scale, causal, window,
+                 workspace, workspace_bytes, phases, stream)
 
 
 def fa_status_string(status: int) -> str:

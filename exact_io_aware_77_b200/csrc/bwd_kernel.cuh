@@ -61,6 +61,7 @@ struct BwdParams {
   __nv_bfloat16* dk;      // [BH, N, D]
   __nv_bfloat16* dv;      // [BH, N, D]
   int N, Np, BH, n_kv_tiles, causal, window;
+  int H, H_kv, group;     // query heads, K/V heads per batch entry; group = H / H_kv
   float scale_log2;       // scale * log2(e)
   float scale;
   unsigned long long wait_limit_ns;
@@ -182,12 +183,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // this CTA's K/V head; with shared K/V heads it runs the query tiles of every query head of
+  // its group in turn (dK and dV accumulate over all of them)
   const int bh = int(blockIdx.x / prm.n_kv_tiles);
   const int kv_tile = int(blockIdx.x % prm.n_kv_tiles);
   const int kv0 = kv_tile * kBwdKeys;
   int i_begin, i_end;
   q_tile_range(kv0, prm.N, prm.causal, prm.window, i_begin, i_end);
-  const int n_it = i_end - i_begin;                        // >= 1
+  const int n_i = i_end - i_begin;                         // query tiles per query head, >= 1
+  const int n_it = n_i * prm.group;
+  const int bh_q0 = (bh / prm.H_kv) * prm.H + (bh % prm.H_kv) * prm.group;   // first query head
+  auto q_tile = [&](int it) { return i_begin + it % n_i; };
+  auto q_head = [&](int it) { return bh_q0 + it / n_i; };
   volatile int* abort = &sm.abort;
   const uint64_t lim = prm.wait_limit_ns;
 
@@ -246,13 +253,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int it = 0; it < n_it; ++it) {
         const int qs = it % kBwdQStages;
         const uint32_t ph = (it / kBwdQStages) & 1;
-        const int q0 = (i_begin + it) * kBwdRows;
+        const int q0 = q_tile(it) * kBwdRows;
+        const int bq = q_head(it);
         if (!mbar_wait(smem_u32(&sm.q_empty[qs]), ph ^ 1, abort, lim)) break;
         const uint32_t qb = smem_u32(&sm.q_full[qs]);
         mbar_expect_tx(qb, Smem::kTileBytes + 2 * kBwdRows * 4);
         for (int c = 0; c < Smem::kChunks; ++c)
-          tma_load_3d(smem_u32(sm.q[qs]) + c * 16384, &tm_q, qb, c * 64, q0, bh);
-        const size_t row = size_t(bh) * prm.Np + q0;
+          tma_load_3d(smem_u32(sm.q[qs]) + c * 16384, &tm_q, qb, c * 64, q0, bq);
+        const size_t row = size_t(bq) * prm.Np + q0;
         bulk_load(smem_u32(sm.lp[qs]), prm.lp + row, kBwdRows * 4, qb);
         bulk_load(smem_u32(sm.dd[qs]), prm.dd + row, kBwdRows * 4, qb);
         issued = it + 1;
@@ -260,7 +268,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t db = smem_u32(&sm.do_full);
         mbar_expect_tx(db, Smem::kTileBytes);
         for (int c = 0; c < Smem::kChunks; ++c)
-          tma_load_3d(smem_u32(sm.dout) + c * 16384, &tm_do, db, c * 64, q0, bh);
+          tma_load_3d(smem_u32(sm.dout) + c * 16384, &tm_do, db, c * 64, q0, bq);
         issued_do = it + 1;
       }
       mbar_wait_drain(kvb, 0, lim);
@@ -376,7 +384,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // every tile.
     auto phase_a = [&](int it, auto masked) -> bool {
       const int qs = it % kBwdQStages;
-      const int q0 = (i_begin + it) * kBwdRows;
+      const int q0 = q_tile(it) * kBwdRows;
       bool w_ok = mbar_wait(smem_u32(&sm.q_full[qs]), (it / kBwdQStages) & 1, abort, lim);
       w_ok = w_ok && mbar_wait(smem_u32(&sm.s_full), it & 1, abort, lim);
       if (!__all_sync(0xffffffffu, w_ok)) return false;
@@ -492,7 +500,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // order: B(i), A(i+1), R(i): the dQ readout of tile i hides behind the exponentials of i+1
     // phase A masks only on the diagonal, the window's far edge and the tail key tile
     auto run_a = [&](int it) -> bool {
-      const int qbase = (i_begin + it) * kBwdRows + hq * 64;
+      const int qbase = q_tile(it) * kBwdRows + hq * 64;
       const bool need_mask = (prm.causal && kv0 + kBwdKeys - 1 > qbase) ||
                              (prm.window > 0 && kv0 < qbase + 64 - prm.window) || (kv0 + kBwdKeys > prm.N) ||
                              (!prm.causal && prm.window > 0 && qbase + prm.window - 1 < kv0 + kBwdKeys - 1);
@@ -552,8 +560,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             x[j] = ld_shared_v4(slot + row * 128 + ((c ^ (row & 7)) << 4));
           }
           mbar_arrive(smem_u32(&sm.st_free[w]));
-          const int q0 = (i_begin + it) * kBwdRows + qd * 32;
-          float* acc = prm.dq_acc + (size_t(bh) * prm.Np + q0) * D + hq * (D / 2) + 32 * ps;
+          const int q0 = q_tile(it) * kBwdRows + qd * 32;
+          float* acc = prm.dq_acc + (size_t(q_head(it)) * prm.Np + q0) * D + hq * (D / 2) + 32 * ps;
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const int row = 4 * j + (lane >> 3), c = lane & 7;

@@ -83,6 +83,9 @@ int check_problem(int B, int H, int N, int d, float scale, int causal, int windo
   return FA_OK;
 }
 
+// query heads H read K/V heads H_kv in contiguous groups
+int check_kv_heads(int H, int H_kv) { return (H_kv >= 1 && H_kv <= H && H % H_kv == 0) ? FA_OK : FA_ERR_SHAPE; }
+
 template <class Kernel>
 int set_smem(Kernel k, int bytes) {
   return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess ? FA_OK
@@ -90,17 +93,20 @@ int set_smem(Kernel k, int bytes) {
 }
 
 template <int D>
-int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int BH, int N, float scale,
-               int causal, int window, cudaStream_t stream) {
+int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv, int N,
+               float scale, int causal, int window, cudaStream_t stream) {
+  const int BH = B * H, BH_kv = B * H_kv;
   CUtensorMap tq, tk, tv;
-  if (!make_map_bf16(&tq, q, D, N, BH, kBlockM) || !make_map_bf16(&tk, k, D, N, BH, kBlockN) ||
-      !make_map_bf16(&tv, v, D, N, BH, kBlockN))
+  if (!make_map_bf16(&tq, q, D, N, BH, kBlockM) || !make_map_bf16(&tk, k, D, N, BH_kv, kBlockN) ||
+      !make_map_bf16(&tv, v, D, N, BH_kv, kBlockN))
     return FA_ERR_CUDA;
   FwdParams prm;
   prm.o = static_cast<__nv_bfloat16*>(o);
   prm.lse = lse;
   prm.N = N;
   prm.BH = BH;
+  prm.H = H;
+  prm.group = H / H_kv;
   prm.n_pairs = ((N + kBlockM - 1) / kBlockM + kQTiles - 1) / kQTiles;
   prm.causal = causal;
   prm.window = window > N ? N : window;   // a band of N or more keys is no band at all
@@ -125,8 +131,9 @@ size_t bwd_workspace_bytes(long long BH, int N, int d) {
 
 template <int D>
 int launch_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
-               void* dq, void* dk, void* dv, int BH, int N, float scale, int causal, int window, void* ws,
-               cudaStream_t stream, int phases = kBwdAllPhases) {
+               void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, float scale, int causal, int window,
+               void* ws, cudaStream_t stream, int phases = kBwdAllPhases) {
+  const int BH = B * H, BH_kv = B * H_kv;
   const long long Np = padded_rows(N);
   float* lp = static_cast<float*>(ws);
   float* dd = lp + size_t(BH) * Np;
@@ -142,8 +149,8 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   }
   if (phases & kBwdPhaseMain) {
   CUtensorMap tq, tk, tv, tdo;
-  if (!make_map_bf16(&tq, q, D, N, BH, kBwdRows) || !make_map_bf16(&tk, k, D, N, BH, kBwdKeys) ||
-      !make_map_bf16(&tv, v, D, N, BH, kBwdKeys) || !make_map_bf16(&tdo, dout, D, N, BH, kBwdRows))
+  if (!make_map_bf16(&tq, q, D, N, BH, kBwdRows) || !make_map_bf16(&tk, k, D, N, BH_kv, kBwdKeys) ||
+      !make_map_bf16(&tv, v, D, N, BH_kv, kBwdKeys) || !make_map_bf16(&tdo, dout, D, N, BH, kBwdRows))
     return FA_ERR_CUDA;
   BwdParams prm;
   prm.lp = lp;
@@ -154,6 +161,9 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   prm.N = N;
   prm.Np = int(Np);
   prm.BH = BH;
+  prm.H = H;
+  prm.H_kv = H_kv;
+  prm.group = H / H_kv;
   prm.n_kv_tiles = (N + kBwdKeys - 1) / kBwdKeys;
   prm.causal = causal;
   prm.window = window > N ? N : window;   // a band of N or more keys is no band at all
@@ -163,7 +173,8 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   static_assert(sizeof(BwdSmem<D>) <= 232448, "backward shared memory exceeds 227 KB");
   const int smem = int(sizeof(BwdSmem<D>));   // the kernel checks that the base is 1 KB aligned
   if (set_smem(fa_bwd_kernel<D>, smem) != FA_OK) return FA_ERR_CUDA;
-  fa_bwd_kernel<D><<<unsigned(prm.n_kv_tiles) * unsigned(BH), kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, prm);
+  // one CTA per (K/V head, key tile)
+  fa_bwd_kernel<D><<<unsigned(prm.n_kv_tiles) * unsigned(BH_kv), kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, prm);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   if (phases & kBwdPhaseFinal) {
@@ -219,18 +230,27 @@ using namespace fa;
 
 extern "C" {
 
+static int bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                    void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, int d, float scale, int causal,
+                    int window, void* workspace, size_t workspace_bytes, int phases, void* stream);
+
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
            float scale, int causal, int window, void* stream) {
+  return fa_fwd_gqa(q, k, v, o, lse, B, H, H, N, d, scale, causal, window, stream);
+}
+
+int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv, int N,
+               int d, float scale, int causal, int window, void* stream) {
   if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
   int st = check_problem(B, H, N, d, scale, causal, window);
+  if (st == FA_OK) st = check_kv_heads(H, H_kv);
   if (st != FA_OK) return st;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
     return FA_ERR_ALIGN;
   if ((st = check_device()) != FA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int BH = B * H;
-  return d == 64 ? launch_fwd<64>(q, k, v, o, lse, BH, N, scale, causal, window, s)
-                 : launch_fwd<128>(q, k, v, o, lse, BH, N, scale, causal, window, s);
+  return d == 64 ? launch_fwd<64>(q, k, v, o, lse, B, H, H_kv, N, scale, causal, window, s)
+                 : launch_fwd<128>(q, k, v, o, lse, B, H, H_kv, N, scale, causal, window, s);
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
@@ -248,9 +268,24 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
 int fa_bwd_phases(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
                   void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal, int window,
                   void* workspace, size_t workspace_bytes, int phases, void* stream) {
+  return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, B, H, H, N, d, scale, causal, window, workspace,
+                  workspace_bytes, phases, stream);
+}
+
+int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+               void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, int d, float scale, int causal,
+               int window, void* workspace, size_t workspace_bytes, int phases, void* stream) {
+  return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, d, scale, causal, window, workspace,
+                  workspace_bytes, phases, stream);
+}
+
+static int bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                    void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, int d, float scale, int causal,
+                    int window, void* workspace, size_t workspace_bytes, int phases, void* stream) {
   if (phases < 1 || phases > kBwdAllPhases) return FA_ERR_PHASES;
   if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FA_ERR_NULL;
   int st = check_problem(B, H, N, d, scale, causal, window);
+  if (st == FA_OK) st = check_kv_heads(H, H_kv);
   if (st != FA_OK) return st;
   const long long BH = (long long)B * H;
   if (BH * ((N + kBwdKeys - 1) / kBwdKeys) > 0x7fffffffLL || BH * padded_rows(N) > 0x7fffffffLL) return FA_ERR_SHAPE;
@@ -260,10 +295,10 @@ int fa_bwd_phases(const void* q, const void* k, const void* v, const void* o, co
     return FA_ERR_ALIGN;
   if ((st = check_device()) != FA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return d == 64 ? launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, int(BH), N, scale, causal, window, workspace, s,
-                                  phases)
-                 : launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, int(BH), N, scale, causal, window, workspace,
-                                   s, phases);
+  return d == 64 ? launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, scale, causal, window,
+                                  workspace, s, phases)
+                 : launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, scale, causal, window,
+                                   workspace, s, phases);
 }
 
 const char* fa_status_string(int status) {
@@ -328,8 +363,8 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
   // every byte of the scratch the kernels read is rewritten first by fa_bwd_prep (D, L and a
   // zeroed dQ accumulator), so what an earlier call left there does not leak in
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return d == 64 ? launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, int(BH), N, scale, causal, window, ws, s)
-                 : launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, int(BH), N, scale, causal, window, ws, s);
+  return d == 64 ? launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H, N, scale, causal, window, ws, s)
+                 : launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H, N, scale, causal, window, ws, s);
 }
 
 }  // extern "C"

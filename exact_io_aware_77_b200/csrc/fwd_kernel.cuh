@@ -54,7 +54,9 @@ struct FwdParams {
   __nv_bfloat16* o;   // [BH, N, D]
   float* lse;         // [BH, N]
   int N;
-  int BH;
+  int BH;             // query heads, B * H
+  int H;              // query heads per batch entry
+  int group;          // query heads per K/V head (H / H_kv)
   int n_pairs;        // ceil(ceil(N / 128) / 2)
   int causal;
   int window;
@@ -103,6 +105,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const int lane = threadIdx.x & 31;
   // head-major order keeps a head's K/V hot in L2; longest causal pairs first within a head
   const int bh = int(blockIdx.x / prm.n_pairs);
+  // K/V head this query head reads: heads share K/V in contiguous groups of prm.group
+  const int bh_kv = (bh / prm.H) * (prm.H / prm.group) + (bh % prm.H) / prm.group;
   const int pair = prm.n_pairs - 1 - int(blockIdx.x % prm.n_pairs);
   const int q0 = pair * (kQTiles * kBlockM);
   int b0, e0, b1, e1;
@@ -162,7 +166,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const CUtensorMap* map = (L & 1) ? &tm_v : &tm_k;
         mbar_expect_tx(fb, Smem::kTileBytes);
         for (int c = 0; c < Smem::kChunks; ++c)
-          tma_load_3d(smem_u32(sm.kv[slot]) + c * 16384, map, fb, c * 64, kv0, bh);
+          tma_load_3d(smem_u32(sm.kv[slot]) + c * 16384, map, fb, c * 64, kv0, bh_kv);
         issued = L + 1;
       }
       // let every copy this CTA started land before the CTA may exit

@@ -115,6 +115,25 @@ FA_EXPORT int fa_bwd_phases(const void* q, const void* k, const void* v, const v
                             int causal, int window, void* workspace, size_t workspace_bytes, int phases,
                             void* stream);
 
+/*
+ * Shared K/V heads (multi-query and grouped-query attention).  The FlashAttention (NL) page
+ * lists Multi-Query Attention among what FlashAttention-2 supports ("Evolutie en verdere
+ * ontwikkelingen"); here H query heads read H_kv K/V heads (H a multiple of H_kv; H_kv = 1 is
+ * multi-query, H_kv = H is fa_fwd / fa_bwd), in contiguous groups: query head h reads K/V
+ * head h / (H / H_kv).  q, o, dO, dq: bf16 [B,H,N,d]; k, v, dk, dv: bf16 [B,H_kv,N,d]; lse:
+ * fp32 [B,H,N].  dk and dv are the sums over each K/V head's query heads.  Everything else
+ * (masks, scale, ownership, errors, streams) is as for fa_fwd / fa_bwd; the workspace is
+ * fa_bwd_workspace_size(B, H, N, d) bytes (it scales with the query heads), and `phases` is
+ * as for fa_bwd_phases (7 = the whole backward).  FA_ERR_SHAPE also when H_kv < 1 or H is not
+ * a multiple of H_kv.
+ */
+FA_EXPORT int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv,
+                         int N, int d, float scale, int causal, int window, void* stream);
+FA_EXPORT int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                         const void* dO, void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, int d,
+                         float scale, int causal, int window, void* workspace, size_t workspace_bytes,
+                         int phases, void* stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 FA_EXPORT const char* fa_status_string(int status);
 

@@ -36,6 +36,7 @@ class Workload:
     grad_seed: int | None = None   # seed of dO (backward workloads)
     oracle_heads: int | None = None  # heads the oracle checks (None = all)
     description: str = ""
+    H_kv: int | None = None  # K/V heads (None = H); H must be a multiple (shared K/V heads)
 
     @property
     def scale(self) -> float:
@@ -46,6 +47,10 @@ class Workload:
     @property
     def BH(self) -> int:
         return self.B * self.H
+
+    @property
+    def kv_heads(self) -> int:
+        return self.H if self.H_kv is None else self.H_kv
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
@@ -67,6 +72,9 @@ WORKLOADS: dict[str, Workload] = {
     # the same length with the local window on both sides (non-causal sliding-window attention)
     "swa": Workload("swa", 1, 16, 32768, 128, window=4096, seed=1006, grad_seed=2006, oracle_heads=2,
                     description="long-context two-sided window B1 H16 N32768 d128, |i-j| < 4096"),
+    # the causal LLM shape with 8 K/V heads for 32 query heads (grouped-query attention)
+    "gqa": Workload("gqa", 2, 32, 4096, 128, causal=True, std=0.5, seed=1007, grad_seed=2007, H_kv=8,
+                    description="causal B2 H32 (8 K/V heads) N4096 d128"),
 }
 
 
@@ -78,13 +86,12 @@ def _randn_bf16(gen: torch.Generator, shape, std: float) -> torch.Tensor:
 
 
 def make_inputs(wl: Workload, seed: int | None = None):
-    """Q, K, V as contiguous CPU bf16 tensors of shape [B, H, N, d]."""
+    """Q [B, H, N, d] and K, V [B, H_kv, N, d] as contiguous CPU bf16 tensors."""
     gen = torch.Generator(device="cpu")
     gen.manual_seed(wl.seed if seed is None else seed)
-    shape = (wl.B, wl.H, wl.N, wl.d)
-    q = _randn_bf16(gen, shape, wl.std)
-    k = _randn_bf16(gen, shape, wl.std)
-    v = _randn_bf16(gen, shape, wl.std)
+    q = _randn_bf16(gen, (wl.B, wl.H, wl.N, wl.d), wl.std)
+    k = _randn_bf16(gen, (wl.B, wl.kv_heads, wl.N, wl.d), wl.std)
+    v = _randn_bf16(gen, (wl.B, wl.kv_heads, wl.N, wl.d), wl.std)
     return q, k, v
 
 

@@ -102,3 +102,15 @@ def test_bwd_phases_rejects_bad_mask(lib, phases):
     ptrs = [A + 4096 * i for i in range(9)]
     st = _lib.fa_bwd_phases(*ptrs, 1, 2, 128, 64, 0.125, 0, 0, A + 65536, 1 << 30, phases, None)
     assert _lib.STATUS_NAMES[st] == "FA_ERR_PHASES"
+
+
+@pytest.mark.parametrize("H,H_kv", [(4, 0), (4, 3), (4, 8), (6, -2)])
+def test_shared_kv_head_counts_rejected(lib, H, H_kv):
+    """H must be a whole multiple of H_kv >= 1, in the forward and the backward."""
+    a = dict(GOOD, H=H)
+    ptrs = [A + 4096 * i for i in range(9)]
+    st = _lib.fa_fwd_gqa(*ptrs[:5], a["B"], H, H_kv, a["N"], a["d"], a["scale"], a["causal"], a["window"], None)
+    assert _lib.STATUS_NAMES[st] == "FA_ERR_SHAPE"
+    st = _lib.fa_bwd_gqa(*ptrs, a["B"], H, H_kv, a["N"], a["d"], a["scale"], a["causal"], a["window"],
+                         A + 65536, 1 << 30, 7, None)
+    assert _lib.STATUS_NAMES[st] == "FA_ERR_SHAPE"
