@@ -193,8 +193,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int n_i = i_end - i_begin;                         // query tiles per query head, >= 1
   const int n_it = n_i * prm.group;
   const int bh_q0 = (bh / prm.H_kv) * prm.H + (bh % prm.H_kv) * prm.group;   // first query head
-  auto q_tile = [&](int it) { return i_begin + it % n_i; };
-  auto q_head = [&](int it) { return bh_q0 + it / n_i; };
+  // (no division when every K/V head serves one query head)
+  auto q_tile = [&](int it) { return prm.group == 1 ? i_begin + it : i_begin + it % n_i; };
+  auto q_head = [&](int it) { return prm.group == 1 ? bh_q0 : bh_q0 + it / n_i; };
   volatile int* abort = &sm.abort;
   const uint64_t lim = prm.wait_limit_ns;
 

@@ -375,11 +375,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       return true;
     };
+    // a KV tile needs the mask when some key lies outside some row's band: below the band of the
+    // tile's last row, or above the band of its first row (or past N)
+    const int band_lo_max = prm.window > 0 ? qw0 + kBlockM - prm.window : 0;
+    const int band_hi_min = min(prm.N - 1, prm.causal ? qw0 : (prm.window > 0 ? qw0 + prm.window - 1 : prm.N - 1));
     for (int t = tb; t < te; ++t) {
       const int kv0 = t * kBlockN;
-      const bool need_mask = (kv0 + kBlockN > prm.N) || (prm.causal && kv0 + kBlockN - 1 > qw0) ||
-                             (prm.window > 0 && kv0 < qw0 + kBlockM - prm.window) ||
-                             (!prm.causal && prm.window > 0 && kv0 + kBlockN - 1 > qw0 + prm.window - 1);
+      const bool need_mask = kv0 < band_lo_max || kv0 + kBlockN - 1 > band_hi_min;
       ok = need_mask ? step(t, std::true_type{}) : step(t, std::false_type{});
       if (!ok) break;
     }
