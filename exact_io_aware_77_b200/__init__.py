@@ -9,6 +9,7 @@ streams only.
 
 from __future__ import annotations
 
+import ctypes
 import math
 
 from . import _lib
@@ -28,11 +29,12 @@ def _stream_handle(device) -> int:
 
 
 def _check_qkv(q, k, v, *rest):
-    """q (and o, dO in rest): [B, H, N, d]; k, v: [B, H_kv, N, d] with H a multiple of H_kv."""
+    """q (and o, dO in rest): [B, H, N, d]; k, v: [B, H_kv, N, d] with H a multiple of H_kv.
+    Any strides with a contiguous last dimension (the library checks their alignment)."""
     import torch
     for t in (q, k, v) + rest:
-        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.dim() == 4 and t.is_contiguous()):
-            raise ValueError("expected contiguous bf16 CUDA tensors of shape [B, H, N, d]")
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.dim() == 4 and t.stride(-1) == 1):
+            raise ValueError("expected bf16 CUDA tensors of shape [B, H, N, d] with contiguous d")
         if t.device != q.device:
             raise ValueError("device mismatch")
     if any(t.shape != q.shape for t in rest) or k.shape != v.shape:
@@ -61,7 +63,10 @@ def forward(q, k, v, scale: float | None = None, causal: bool = False, window: i
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr())
     mask = (scale, int(bool(causal)), int(window), _stream_handle(q.device))
-    if H_kv == H:
+    if not all(t.is_contiguous() for t in (q, k, v, out)):
+        st = _lib.strides_array((q, k, v, out))
+        _raise("fa_fwd_strided", _lib.fa_fwd_strided(*ptrs, B, H, H_kv, N, d, ctypes.addressof(st), *mask))
+    elif H_kv == H:
         _raise("fa_fwd", _lib.fa_fwd(*ptrs, B, H, N, d, *mask))
     else:
         _raise("fa_fwd_gqa", _lib.fa_fwd_gqa(*ptrs, B, H, H_kv, N, d, *mask))
@@ -91,6 +96,9 @@ def backward(q, k, v, o, lse, do, scale: float | None = None, causal: bool = Fal
     scale = default_scale(d) if scale is None else float(scale)
     if grads is None:
         grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+    for g, t in zip(grads, (q, k, v)):
+        if g.shape != t.shape or g.stride(-1) != 1 or g.dtype != torch.bfloat16 or g.device != q.device:
+            raise ValueError("grads must be bf16 CUDA tensors shaped like q, k, v with contiguous d")
     need = bwd_workspace_size(B, H, N, d)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
@@ -99,6 +107,13 @@ def backward(q, k, v, o, lse, do, scale: float | None = None, causal: bool = Fal
             dq.data_ptr(), dk.data_ptr(), dv.data_ptr())
     rest = (d, scale, int(bool(causal)), int(window), workspace.data_ptr(),
             workspace.numel() * workspace.element_size())
+    if not all(t.is_contiguous() for t in (q, k, v, o, do, dq, dk, dv)):
+        st = _lib.strides_array((q, k, v, o, do, dq, dk, dv))
+        _raise("fa_bwd_strided", _lib.fa_bwd_strided(*ptrs, B, H, H_kv, N, d, ctypes.addressof(st), scale,
+                                                     int(bool(causal)), int(window), workspace.data_ptr(),
+                                                     workspace.numel() * workspace.element_size(), int(phases),
+                                                     _stream_handle(q.device)))
+        return dq, dk, dv
     if H_kv != H:
         _raise("fa_bwd_gqa", _lib.fa_bwd_gqa(*ptrs, B, H, H_kv, N, *rest, int(phases), _stream_handle(q.device)))
         return dq, dk, dv

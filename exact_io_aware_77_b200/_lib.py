@@ -36,6 +36,9 @@ SIGNATURES = {
                                                                 _c_int, _c_void_p]),
     "fa_bwd_noalloc": (_c_int, [_c_void_p] * 9 + [_c_int] * 4 + [_c_float, _c_int, _c_int, _c_void_p]),
     "fa_fwd_gqa": (_c_int, [_c_void_p] * 5 + [_c_int] * 5 + [_c_float, _c_int, _c_int, _c_void_p]),
+    "fa_fwd_strided": (_c_int, [_c_void_p] * 5 + [_c_int] * 5 + [_c_void_p, _c_float, _c_int, _c_int, _c_void_p]),
+    "fa_bwd_strided": (_c_int, [_c_void_p] * 9 + [_c_int] * 5 + [_c_void_p, _c_float, _c_int, _c_int, _c_void_p,
+                                                                 _c_size_t, _c_int, _c_void_p]),
     "fa_bwd_gqa": (_c_int, [_c_void_p] * 9 + [_c_int] * 5 + [_c_float, _c_int, _c_int, _c_void_p, _c_size_t,
                                                              _c_int, _c_void_p]),
     "fa_status_string": (ctypes.c_char_p, [_c_int]),
@@ -121,6 +124,32 @@ def fa_bwd_gqa(q, k, v, o, lse, dO, dq, dk, dv, B, H, H_kv, N, d, scale, causal,
     """fa_bwd_phases with H_kv shared K/V heads; dk, dv are [B, H_kv, N, d]."""
     return _call("fa_bwd_gqa", q, k, v, o, lse, dO, dq, dk, dv, B, H, H_kv, N, d, scale, causal, window,
                  workspace, workspace_bytes, phases, stream)
+
+
+class FaStrides(ctypes.Structure):
+    """fa_strides: element strides (b, h, n) of a [B, heads, N, d] array with contiguous d."""
+    _fields_ = [("b", ctypes.c_longlong), ("h", ctypes.c_longlong), ("n", ctypes.c_longlong)]
+
+
+def strides_array(tensors):
+    """A ctypes array of FaStrides for [B, heads, N, d] tensors (kept alive by the caller)."""
+    arr = (FaStrides * len(tensors))()
+    for i, t in enumerate(tensors):
+        sb, sh, sn, _ = t.stride()
+        arr[i] = FaStrides(sb, sh, sn)
+    return arr
+
+
+def fa_fwd_strided(q, k, v, o, lse, B, H, H_kv, N, d, strides, scale, causal, window, stream) -> int:
+    """fa_fwd_gqa with per-array strides (``strides``: address of 4 fa_strides, or 0)."""
+    return _call("fa_fwd_strided", q, k, v, o, lse, B, H, H_kv, N, d, strides, scale, causal, window, stream)
+
+
+def fa_bwd_strided(q, k, v, o, lse, dO, dq, dk, dv, B, H, H_kv, N, d, strides, scale, causal, window, workspace,
+                   workspace_bytes, phases, stream) -> int:
+    """fa_bwd_gqa with per-array strides (``strides``: address of 8 fa_strides)."""
+    return _call("fa_bwd_strided", q, k, v, o, lse, dO, dq, dk, dv, B, H, H_kv, N, d, strides, scale, causal,
+                 window, workspace, workspace_bytes, phases, stream)
 
 
 def fa_status_string(status: int) -> str:

@@ -62,6 +62,7 @@ struct BwdParams {
   __nv_bfloat16* dv;      // [BH, N, D]
   int N, Np, BH, n_kv_tiles, causal, window;
   int H, H_kv, group;     // query heads, K/V heads per batch entry; group = H / H_kv
+  Strides dk_st, dv_st;   // element strides of dK and dV
   float scale_log2;       // scale * log2(e)
   float scale;
   unsigned long long wait_limit_ns;
@@ -112,7 +113,7 @@ __global__ void __launch_bounds__(256) fa_bwd_prep(const __nv_bfloat16* __restri
                                                    const __nv_bfloat16* __restrict__ dout,
                                                    const float* __restrict__ lse, float* __restrict__ lp,
                                                    float* __restrict__ dd, float* __restrict__ dq_acc, int N, int Np,
-                                                   long long total_rows) {
+                                                   int H, Strides o_st, Strides do_st, long long total_rows) {
   constexpr int G = D / 8;                      // threads per row
   const long long g = (long long)blockIdx.x * (256 / G) + threadIdx.x / G;
   const int c = threadIdx.x % G;
@@ -121,9 +122,9 @@ __global__ void __launch_bounds__(256) fa_bwd_prep(const __nv_bfloat16* __restri
   const int n = int(g % Np);
   float dot = 0.f;
   if (n < N) {
-    const size_t off = (size_t(bh) * N + n) * D + c * 8;
-    const uint4 a = *reinterpret_cast<const uint4*>(o + off);
-    const uint4 b = *reinterpret_cast<const uint4*>(dout + off);
+    const int b_idx = int(bh / H), h = int(bh % H);
+    const uint4 a = *reinterpret_cast<const uint4*>(o + o_st.at(b_idx, h, n) + c * 8);
+    const uint4 b = *reinterpret_cast<const uint4*>(dout + do_st.at(b_idx, h, n) + c * 8);
     const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
     const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b);
 #pragma unroll
@@ -149,7 +150,7 @@ __global__ void __launch_bounds__(256) fa_bwd_prep(const __nv_bfloat16* __restri
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_dq_final(const float* __restrict__ dq_acc,
                                                        __nv_bfloat16* __restrict__ dq, int N, int Np, float scale,
-                                                       long long total_rows) {
+                                                       int H, Strides dq_st, long long total_rows) {
   constexpr int G = D / 8;
   const long long g = (long long)blockIdx.x * (256 / G) + threadIdx.x / G;   // row of [BH, N]
   const int c = threadIdx.x % G;
@@ -163,7 +164,7 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_final(const float* __restrict__
   out.y = pack_bf16x2(a.z * scale, a.w * scale);
   out.z = pack_bf16x2(b.x * scale, b.y * scale);
   out.w = pack_bf16x2(b.z * scale, b.w * scale);
-  *reinterpret_cast<uint4*>(dq + size_t(g) * D + c * 8) = out;
+  *reinterpret_cast<uint4*>(dq + dq_st.at(int(bh / H), int(bh % H), n) + c * 8) = out;
 }
 
 // ----------------------------------------------------------------------------- main kernel
@@ -194,6 +195,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int n_it = n_i * prm.group;
   const int bh_q0 = (bh / prm.H_kv) * prm.H + (bh % prm.H_kv) * prm.group;   // first query head
   // (no division when every K/V head serves one query head)
+  const int b_idx = bh / prm.H_kv, h_kv = bh % prm.H_kv;   // batch entry and K/V head
   auto q_tile = [&](int it) { return prm.group == 1 ? i_begin + it : i_begin + it % n_i; };
   auto q_head = [&](int it) { return prm.group == 1 ? bh_q0 : bh_q0 + it / n_i; };
   volatile int* abort = &sm.abort;
@@ -243,8 +245,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint32_t kvb = smem_u32(&sm.kv_full);
       mbar_expect_tx(kvb, 2 * Smem::kTileBytes);
       for (int c = 0; c < Smem::kChunks; ++c) {
-        tma_load_3d(smem_u32(sm.k) + c * 16384, &tm_k, kvb, c * 64, kv0, bh);
-        tma_load_3d(smem_u32(sm.v) + c * 16384, &tm_v, kvb, c * 64, kv0, bh);
+        tma_load_rows(smem_u32(sm.k) + c * 16384, &tm_k, kvb, c * 64, kv0, h_kv, b_idx);
+        tma_load_rows(smem_u32(sm.v) + c * 16384, &tm_v, kvb, c * 64, kv0, h_kv, b_idx);
       }
       int issued = 0;
       // Q_i (with its L and D rows) through two stages; dO_i through one: its last reader,
@@ -260,7 +262,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t qb = smem_u32(&sm.q_full[qs]);
         mbar_expect_tx(qb, Smem::kTileBytes + 2 * kBwdRows * 4);
         for (int c = 0; c < Smem::kChunks; ++c)
-          tma_load_3d(smem_u32(sm.q[qs]) + c * 16384, &tm_q, qb, c * 64, q0, bq);
+          tma_load_rows(smem_u32(sm.q[qs]) + c * 16384, &tm_q, qb, c * 64, q0, bq - b_idx * prm.H, b_idx);
         const size_t row = size_t(bq) * prm.Np + q0;
         bulk_load(smem_u32(sm.lp[qs]), prm.lp + row, kBwdRows * 4, qb);
         bulk_load(smem_u32(sm.dd[qs]), prm.dd + row, kBwdRows * 4, qb);
@@ -269,7 +271,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t db = smem_u32(&sm.do_full);
         mbar_expect_tx(db, Smem::kTileBytes);
         for (int c = 0; c < Smem::kChunks; ++c)
-          tma_load_3d(smem_u32(sm.dout) + c * 16384, &tm_do, db, c * 64, q0, bq);
+          tma_load_rows(smem_u32(sm.dout) + c * 16384, &tm_do, db, c * 64, q0, bq - b_idx * prm.H, b_idx);
         issued_do = it + 1;
       }
       mbar_wait_drain(kvb, 0, lim);
@@ -517,8 +519,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (ok && __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.mma_final), 0, abort, lim))) {
       tc_fence_after();
       const bool in_range = key < prm.N;
-      const size_t row_off = (size_t(bh) * prm.N + (in_range ? key : 0)) * D;
-      __nv_bfloat16* dst_row = (hq == 0 ? prm.dk : prm.dv) + row_off;
+      const int krow = in_range ? key : 0;
+      __nv_bfloat16* dst_row = hq == 0 ? prm.dk + prm.dk_st.at(b_idx, h_kv, krow)
+                                       : prm.dv + prm.dv_st.at(b_idx, h_kv, krow);
       const float mul = hq == 0 ? prm.scale : 1.f;
       const uint32_t col0 = hq == 0 ? kTdK : kTdV;
 #pragma unroll

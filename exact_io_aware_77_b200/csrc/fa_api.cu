@@ -38,18 +38,30 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [BH, rows, d] bf16 viewed as a 3-D tensor (d, rows, BH); box = 64 columns x box_rows rows
-// of one head, 128-byte swizzled.  Rows past the end of a head read as zero.
-bool make_map_bf16(CUtensorMap* map, const void* base, int d, int rows, int bh, int box_rows) {
+// A bf16 [B, heads, rows, d] array with element strides st (d contiguous) viewed as the 4-D
+// tensor (d, rows, heads, B); box = 64 columns x box_rows rows of one head, 128-byte swizzled.
+// Rows past the end of a head read as zero.
+bool make_map_bf16(CUtensorMap* map, const void* base, int d, int rows, int heads, int B, Strides st,
+                   int box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
-  cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(rows), cuuint64_t(bh)};
-  cuuint64_t strides[2] = {cuuint64_t(d) * 2, cuuint64_t(d) * 2 * cuuint64_t(rows)};
-  cuuint32_t box[3] = {64, cuuint32_t(box_rows), 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+  cuuint64_t dims[4] = {cuuint64_t(d), cuuint64_t(rows), cuuint64_t(heads), cuuint64_t(B)};
+  cuuint64_t strides[3] = {cuuint64_t(st.n) * 2, cuuint64_t(st.h) * 2, cuuint64_t(st.b) * 2};
+  cuuint32_t box[4] = {64, cuuint32_t(box_rows), 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// strides of a contiguous [B, heads, N, d] array
+Strides packed(int heads, int N, int d) {
+  return Strides{(long long)heads * N * d, (long long)N * d, (long long)d};
+}
+
+// every stride a positive multiple of 8 elements (16 bytes: TMA and the vector stores)
+bool strides_ok(const Strides& s) {
+  return s.b > 0 && s.h > 0 && s.n > 0 && s.b % 8 == 0 && s.h % 8 == 0 && s.n % 8 == 0;
 }
 
 // ---------------------------------------------------------------- validation
@@ -94,11 +106,11 @@ int set_smem(Kernel k, int bytes) {
 
 template <int D>
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv, int N,
-               float scale, int causal, int window, cudaStream_t stream) {
-  const int BH = B * H, BH_kv = B * H_kv;
+               const Strides* st, float scale, int causal, int window, cudaStream_t stream) {
+  const int BH = B * H;
   CUtensorMap tq, tk, tv;
-  if (!make_map_bf16(&tq, q, D, N, BH, kBlockM) || !make_map_bf16(&tk, k, D, N, BH_kv, kBlockN) ||
-      !make_map_bf16(&tv, v, D, N, BH_kv, kBlockN))
+  if (!make_map_bf16(&tq, q, D, N, H, B, st[0], kBlockM) || !make_map_bf16(&tk, k, D, N, H_kv, B, st[1], kBlockN) ||
+      !make_map_bf16(&tv, v, D, N, H_kv, B, st[2], kBlockN))
     return FA_ERR_CUDA;
   FwdParams prm;
   prm.o = static_cast<__nv_bfloat16*>(o);
@@ -107,6 +119,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   prm.BH = BH;
   prm.H = H;
   prm.group = H / H_kv;
+  prm.o_st = st[3];
   prm.n_pairs = ((N + kBlockM - 1) / kBlockM + kQTiles - 1) / kQTiles;
   prm.causal = causal;
   prm.window = window > N ? N : window;   // a band of N or more keys is no band at all
@@ -131,8 +144,9 @@ size_t bwd_workspace_bytes(long long BH, int N, int d) {
 
 template <int D>
 int launch_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
-               void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, float scale, int causal, int window,
-               void* ws, cudaStream_t stream, int phases = kBwdAllPhases) {
+               void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, const Strides* st, float scale,
+               int causal, int window, void* ws, cudaStream_t stream, int phases = kBwdAllPhases) {
+  // st: q, k, v, o, dO, dq, dk, dv
   const int BH = B * H, BH_kv = B * H_kv;
   const long long Np = padded_rows(N);
   float* lp = static_cast<float*>(ws);
@@ -144,13 +158,13 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
     const long long blocks = (rows + (256 / G) - 1) / (256 / G);
     fa_bwd_prep<D><<<unsigned(blocks), 256, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, lp, dd, dq_acc, N,
-        int(Np), rows);
+        int(Np), H, st[3], st[4], rows);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   if (phases & kBwdPhaseMain) {
   CUtensorMap tq, tk, tv, tdo;
-  if (!make_map_bf16(&tq, q, D, N, BH, kBwdRows) || !make_map_bf16(&tk, k, D, N, BH_kv, kBwdKeys) ||
-      !make_map_bf16(&tv, v, D, N, BH_kv, kBwdKeys) || !make_map_bf16(&tdo, dout, D, N, BH, kBwdRows))
+  if (!make_map_bf16(&tq, q, D, N, H, B, st[0], kBwdRows) || !make_map_bf16(&tk, k, D, N, H_kv, B, st[1], kBwdKeys) ||
+      !make_map_bf16(&tv, v, D, N, H_kv, B, st[2], kBwdKeys) || !make_map_bf16(&tdo, dout, D, N, H, B, st[4], kBwdRows))
     return FA_ERR_CUDA;
   BwdParams prm;
   prm.lp = lp;
@@ -164,6 +178,8 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   prm.H = H;
   prm.H_kv = H_kv;
   prm.group = H / H_kv;
+  prm.dk_st = st[6];
+  prm.dv_st = st[7];
   prm.n_kv_tiles = (N + kBwdKeys - 1) / kBwdKeys;
   prm.causal = causal;
   prm.window = window > N ? N : window;   // a band of N or more keys is no band at all
@@ -181,7 +197,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
     const long long rows = (long long)BH * N;
     const long long blocks = (rows + (256 / G) - 1) / (256 / G);
     fa_bwd_dq_final<D><<<unsigned(blocks), 256, 0, stream>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), N, int(Np),
-                                                             scale, rows);
+                                                             scale, H, st[5], rows);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   return FA_OK;
@@ -231,8 +247,9 @@ using namespace fa;
 extern "C" {
 
 static int bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
-                    void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, int d, float scale, int causal,
-                    int window, void* workspace, size_t workspace_bytes, int phases, void* stream);
+                    void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, int d, const fa_strides* strides,
+                    float scale, int causal, int window, void* workspace, size_t workspace_bytes, int phases,
+                    void* stream);
 
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
            float scale, int causal, int window, void* stream) {
@@ -241,16 +258,28 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
 
 int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv, int N,
                int d, float scale, int causal, int window, void* stream) {
+  return fa_fwd_strided(q, k, v, o, lse, B, H, H_kv, N, d, nullptr, scale, causal, window, stream);
+}
+
+int fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv, int N,
+                   int d, const fa_strides* strides, float scale, int causal, int window, void* stream) {
   if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
   int st = check_problem(B, H, N, d, scale, causal, window);
   if (st == FA_OK) st = check_kv_heads(H, H_kv);
   if (st != FA_OK) return st;
+  // q, k, v, o: the caller's strides, or the packed [B, heads, N, d] ones
+  Strides s4[4] = {packed(H, N, d), packed(H_kv, N, d), packed(H_kv, N, d), packed(H, N, d)};
+  if (strides)
+    for (int i = 0; i < 4; ++i) {
+      s4[i] = Strides{strides[i].b, strides[i].h, strides[i].n};
+      if (!strides_ok(s4[i])) return FA_ERR_ALIGN;
+    }
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
     return FA_ERR_ALIGN;
   if ((st = check_device()) != FA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return d == 64 ? launch_fwd<64>(q, k, v, o, lse, B, H, H_kv, N, scale, causal, window, s)
-                 : launch_fwd<128>(q, k, v, o, lse, B, H, H_kv, N, scale, causal, window, s);
+  return d == 64 ? launch_fwd<64>(q, k, v, o, lse, B, H, H_kv, N, s4, scale, causal, window, s)
+                 : launch_fwd<128>(q, k, v, o, lse, B, H, H_kv, N, s4, scale, causal, window, s);
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
@@ -268,25 +297,43 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
 int fa_bwd_phases(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
                   void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal, int window,
                   void* workspace, size_t workspace_bytes, int phases, void* stream) {
-  return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, B, H, H, N, d, scale, causal, window, workspace,
+  return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, B, H, H, N, d, nullptr, scale, causal, window, workspace,
                   workspace_bytes, phases, stream);
 }
 
 int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
                void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, int d, float scale, int causal,
                int window, void* workspace, size_t workspace_bytes, int phases, void* stream) {
-  return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, d, scale, causal, window, workspace,
+  return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, d, nullptr, scale, causal, window, workspace,
+                  workspace_bytes, phases, stream);
+}
+
+int fa_bwd_strided(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                   void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, int d, const fa_strides* strides,
+                   float scale, int causal, int window, void* workspace, size_t workspace_bytes, int phases,
+                   void* stream) {
+  if (!strides) return FA_ERR_NULL;
+  return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, d, strides, scale, causal, window, workspace,
                   workspace_bytes, phases, stream);
 }
 
 static int bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
-                    void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, int d, float scale, int causal,
-                    int window, void* workspace, size_t workspace_bytes, int phases, void* stream) {
+                    void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, int d, const fa_strides* strides,
+                    float scale, int causal, int window, void* workspace, size_t workspace_bytes, int phases,
+                    void* stream) {
   if (phases < 1 || phases > kBwdAllPhases) return FA_ERR_PHASES;
   if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FA_ERR_NULL;
   int st = check_problem(B, H, N, d, scale, causal, window);
   if (st == FA_OK) st = check_kv_heads(H, H_kv);
   if (st != FA_OK) return st;
+  // q, k, v, o, dO, dq, dk, dv: the caller's strides, or the packed ones
+  Strides s8[8] = {packed(H, N, d),    packed(H_kv, N, d), packed(H_kv, N, d), packed(H, N, d),
+                   packed(H, N, d),    packed(H, N, d),    packed(H_kv, N, d), packed(H_kv, N, d)};
+  if (strides)
+    for (int i = 0; i < 8; ++i) {
+      s8[i] = Strides{strides[i].b, strides[i].h, strides[i].n};
+      if (!strides_ok(s8[i])) return FA_ERR_ALIGN;
+    }
   const long long BH = (long long)B * H;
   if (BH * ((N + kBwdKeys - 1) / kBwdKeys) > 0x7fffffffLL || BH * padded_rows(N) > 0x7fffffffLL) return FA_ERR_SHAPE;
   if (!workspace || workspace_bytes < bwd_workspace_bytes(BH, N, d)) return FA_ERR_WORKSPACE;
@@ -295,9 +342,9 @@ static int bwd_impl(const void* q, const void* k, const void* v, const void* o, 
     return FA_ERR_ALIGN;
   if ((st = check_device()) != FA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return d == 64 ? launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, scale, causal, window,
+  return d == 64 ? launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, s8, scale, causal, window,
                                   workspace, s, phases)
-                 : launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, scale, causal, window,
+                 : launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, s8, scale, causal, window,
                                    workspace, s, phases);
 }
 
@@ -363,8 +410,10 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
   // every byte of the scratch the kernels read is rewritten first by fa_bwd_prep (D, L and a
   // zeroed dQ accumulator), so what an earlier call left there does not leak in
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return d == 64 ? launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H, N, scale, causal, window, ws, s)
-                 : launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H, N, scale, causal, window, ws, s);
+  const Strides s8[8] = {packed(H, N, d), packed(H, N, d), packed(H, N, d), packed(H, N, d),
+                         packed(H, N, d), packed(H, N, d), packed(H, N, d), packed(H, N, d)};
+  return d == 64 ? launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H, N, s8, scale, causal, window, ws, s)
+                 : launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H, N, s8, scale, causal, window, ws, s);
 }
 
 }  // extern "C"

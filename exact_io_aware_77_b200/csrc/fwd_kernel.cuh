@@ -51,12 +51,13 @@ constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only when m
 constexpr int kEmuPairs = FA_FWD_EMU_PAIRS;   // of every 16 exponential pairs, this many use the FMA pipe
 
 struct FwdParams {
-  __nv_bfloat16* o;   // [BH, N, D]
+  __nv_bfloat16* o;   // [B, H, N, D] with strides o_st
   float* lse;         // [BH, N]
   int N;
   int BH;             // query heads, B * H
   int H;              // query heads per batch entry
   int group;          // query heads per K/V head (H / H_kv)
+  Strides o_st;       // element strides of O
   int n_pairs;        // ceil(ceil(N / 128) / 2)
   int causal;
   int window;
@@ -105,8 +106,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const int lane = threadIdx.x & 31;
   // head-major order keeps a head's K/V hot in L2; longest causal pairs first within a head
   const int bh = int(blockIdx.x / prm.n_pairs);
-  // K/V head this query head reads: heads share K/V in contiguous groups of prm.group
-  const int bh_kv = (bh / prm.H) * (prm.H / prm.group) + (bh % prm.H) / prm.group;
+  // batch entry, query head, and the K/V head it reads (heads share K/V in contiguous groups)
+  const int b_idx = bh / prm.H, h_q = bh % prm.H, h_kv = h_q / prm.group;
   const int pair = prm.n_pairs - 1 - int(blockIdx.x % prm.n_pairs);
   const int q0 = pair * (kQTiles * kBlockM);
   int b0, e0, b1, e1;
@@ -155,7 +156,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_expect_tx(qb, kQTiles * Smem::kTileBytes);
       for (int w = 0; w < kQTiles; ++w)
         for (int c = 0; c < Smem::kChunks; ++c)
-          tma_load_3d(smem_u32(sm.q[w]) + c * 16384, &tm_q, qb, c * 64, q0 + w * kBlockM, bh);
+          tma_load_rows(smem_u32(sm.q[w]) + c * 16384, &tm_q, qb, c * 64, q0 + w * kBlockM, h_q, b_idx);
       int issued = 0;   // loads issued: K_t is load 2(t - t_begin), V_t the next one
       const int n_loads = 2 * (t_end - t_begin);
       for (int L = 0; L < n_loads; ++L) {
@@ -166,7 +167,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const CUtensorMap* map = (L & 1) ? &tm_v : &tm_k;
         mbar_expect_tx(fb, Smem::kTileBytes);
         for (int c = 0; c < Smem::kChunks; ++c)
-          tma_load_3d(smem_u32(sm.kv[slot]) + c * 16384, map, fb, c * 64, kv0, bh_kv);
+          tma_load_rows(smem_u32(sm.kv[slot]) + c * 16384, map, fb, c * 64, kv0, h_kv, b_idx);
         issued = L + 1;
       }
       // let every copy this CTA started land before the CTA may exit
@@ -389,7 +390,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       tc_fence_after();
       const float inv_l = 1.f / l;
       const bool in_range = qi < prm.N;
-      __nv_bfloat16* orow = prm.o + (size_t(bh) * prm.N + (in_range ? qi : 0)) * D;
+      __nv_bfloat16* orow = prm.o + prm.o_st.at(b_idx, h_q, in_range ? qi : 0);
 #pragma unroll
       for (int ch = 0; ch < D / 32; ++ch) {
         uint32_t r[32];

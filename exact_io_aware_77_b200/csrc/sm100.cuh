@@ -88,14 +88,22 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, u
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
-// 3-D tiled load (x = innermost element index, y = row, z = head) into shared
-// memory, completing `bytes` of the transaction count on `bar`.
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y,
-                                            int z) {
+// Element strides of one [B, heads, N, d] array whose d elements are contiguous.
+struct Strides {
+  long long b, h, n;
+  __host__ __device__ long long at(int b_, int h_, int n_) const {
+    return (long long)b_ * b + (long long)h_ * h + (long long)n_ * n;
+  }
+};
+
+// 4-D tiled load of one head's rows (tensor (d, N, heads, B): x = element of d, y = row,
+// head, batch) into shared memory, completing its bytes of the transaction count on `bar`.
+__device__ __forceinline__ void tma_load_rows(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int row,
+                                              int head, int batch) {
   asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(row), "r"(head), "r"(batch)
       : "memory");
 }
 

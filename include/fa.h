@@ -116,6 +116,16 @@ FA_EXPORT int fa_bwd_phases(const void* q, const void* k, const void* v, const v
                             void* stream);
 
 /*
+ * Element strides of one bf16 array of logical shape [B, heads, N, d] whose d elements are
+ * contiguous: element (b, h, n, c) is at b * b_stride + h * h_stride + n * n_stride + c.  The
+ * packed layout [B, heads, N, d] is {heads*N*d, N*d, d}; [B, N, heads, d] (sequence-major) is
+ * {N*heads*d, d, heads*d}.
+ */
+typedef struct fa_strides {
+  long long b, h, n;
+} fa_strides;
+
+/*
  * Shared K/V heads (multi-query and grouped-query attention).  The FlashAttention (NL) page
  * lists Multi-Query Attention among what FlashAttention-2 supports ("Evolutie en verdere
  * ontwikkelingen"); here H query heads read H_kv K/V heads (H a multiple of H_kv; H_kv = 1 is
@@ -133,6 +143,23 @@ FA_EXPORT int fa_bwd_gqa(const void* q, const void* k, const void* v, const void
                          const void* dO, void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, int d,
                          float scale, int causal, int window, void* workspace, size_t workspace_bytes,
                          int phases, void* stream);
+
+/*
+ * fa_fwd_gqa / fa_bwd_gqa on arrays with arbitrary strides (for instance the sequence-major
+ * [B, N, H, d] layout of many frameworks) instead of packed ones.  `strides` (host memory)
+ * holds one fa_strides per array: q, k, v, o for the forward (4 entries, or NULL for packed
+ * arrays); q, k, v, o, dO, dq, dk, dv for the backward (8 entries, not NULL).  Every stride must
+ * be a positive multiple of 8 elements (FA_ERR_ALIGN otherwise); strides that make an output
+ * overlap itself are the caller's error.  lse stays packed fp32 [B, H, N].  The pages print no
+ * layout: the strides only say where the same [B, heads, N, d] elements live.
+ */
+FA_EXPORT int fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                             int H_kv, int N, int d, const fa_strides* strides, float scale, int causal, int window,
+                             void* stream);
+FA_EXPORT int fa_bwd_strided(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                             const void* dO, void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, int d,
+                             const fa_strides* strides, float scale, int causal, int window, void* workspace,
+                             size_t workspace_bytes, int phases, void* stream);
 
 /* Human-readable name of a status code (static string, never NULL). */
 FA_EXPORT const char* fa_status_string(int status);

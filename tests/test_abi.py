@@ -114,3 +114,23 @@ def test_shared_kv_head_counts_rejected(lib, H, H_kv):
     st = _lib.fa_bwd_gqa(*ptrs, a["B"], H, H_kv, a["N"], a["d"], a["scale"], a["causal"], a["window"],
                          A + 65536, 1 << 30, 7, None)
     assert _lib.STATUS_NAMES[st] == "FA_ERR_SHAPE"
+
+
+def test_strided_entry_points_validate_strides(lib):
+    """Strides must be positive multiples of 8 elements; the backward needs its strides."""
+    good = [_lib.FaStrides(2 * 128 * 64, 128 * 64, 64) for _ in range(8)]
+    ptrs = [A + 4096 * i for i in range(9)]
+    a = dict(GOOD)
+    for bad in (_lib.FaStrides(2 * 128 * 64, 128 * 64, 60), _lib.FaStrides(0, 128 * 64, 64),
+                _lib.FaStrides(-64, 128 * 64, 64)):
+        arr = (_lib.FaStrides * 8)(*good)
+        arr[1] = bad
+        st = _lib.fa_fwd_strided(*ptrs[:5], a["B"], a["H"], a["H"], a["N"], a["d"], ctypes.addressof(arr),
+                                 a["scale"], a["causal"], a["window"], None)
+        assert _lib.STATUS_NAMES[st] == "FA_ERR_ALIGN"
+        st = _lib.fa_bwd_strided(*ptrs, a["B"], a["H"], a["H"], a["N"], a["d"], ctypes.addressof(arr), a["scale"],
+                                 a["causal"], a["window"], A + 65536, 1 << 30, 7, None)
+        assert _lib.STATUS_NAMES[st] == "FA_ERR_ALIGN"
+    st = _lib.fa_bwd_strided(*ptrs, a["B"], a["H"], a["H"], a["N"], a["d"], None, a["scale"], a["causal"],
+                             a["window"], A + 65536, 1 << 30, 7, None)
+    assert _lib.STATUS_NAMES[st] == "FA_ERR_NULL"
