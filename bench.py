@@ -437,12 +437,12 @@ def measure_e2e(fa, torch, wl, dev, stream, q_h, k_h, v_h, do_h, has_bwd, steps,
 # the causal B2 H32 N4096 d128 workload, keyed by kernel, with the SHA-1 of the kernel's sources
 # when the counters were taken (profiles/ holds the summaries).  A changed source reports null.
 NCU_TRAFFIC = {
-    "fa_fwd_kernel<128>": {"bytes": 250811648,
-                           "sources": {"fwd_kernel.cuh": "d88e1c82f25fa87714e5197793ec2b1e6aaba0fc",
-                                       "sm100.cuh": "f5bfef53a203d01b5f2fa38e4a691ac48c3cc963"}},
-    "fa_bwd_kernel<128>": {"bytes": 629637376,
-                           "sources": {"bwd_kernel.cuh": "ec7f1612959af91065d856c081bf03dd0ae0bb95",
-                                       "sm100.cuh": "f5bfef53a203d01b5f2fa38e4a691ac48c3cc963"}},
+    "fa_fwd_kernel<128>": {"bytes": 251356416,
+                           "sources": {"fwd_kernel.cuh": "35b94dbef8d8bf21170a8812fab6ac84911c902b",
+                                       "sm100.cuh": "765aea2ea7410d534e289cfea85ff6d2b3b159c9"}},
+    "fa_bwd_kernel<128>": {"bytes": 628199424,
+                           "sources": {"bwd_kernel.cuh": "a16249a9909c16bc8d6b854ecf39824e9ae17b7a",
+                                       "sm100.cuh": "765aea2ea7410d534e289cfea85ff6d2b3b159c9"}},
 }
 
 
