@@ -1,0 +1,23 @@
+"""bench.py's FLOP counts: the closed-form pair counts of banded masks agree with the oracle's
+brute-force count, and the unbanded convention is 4 B H N^2 d, halved when causal."""
+
+import pytest
+
+import bench
+from oracle import attention as orc
+
+
+@pytest.mark.parametrize("n", [1, 7, 128, 300])
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("window", [1, 3, 64, 500])
+def test_band_pairs_match_oracle(n, causal, window):
+    assert bench.band_pairs(n, causal, window) == orc.allowed_pairs(n, causal, window)
+
+
+def test_flop_conventions():
+    assert bench.fwd_flops(2, 32, 4096, 128, True) == 4.0 * 2 * 32 * 4096 ** 2 * 128 / 2
+    assert bench.fwd_flops(4, 16, 2048, 64, False) == 4.0 * 4 * 16 * 2048 ** 2 * 64
+    assert bench.bwd_flops(2, 32, 4096, 128, True) == 2.5 * bench.fwd_flops(2, 32, 4096, 128, True)
+    # the long-context shape: 4 d per kept pair, not the causal-halved square
+    pairs = orc.allowed_pairs(32768, True, 4096)
+    assert bench.fwd_flops(1, 16, 32768, 128, True, 4096) == 4.0 * 16 * 128 * pairs
