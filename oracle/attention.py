@@ -45,6 +45,14 @@ H_kv K/V heads for H query heads (H a multiple of H_kv; H_kv = 1 is MQA): query 
 h reads K/V head h // (H / H_kv), so each K/V head serves a contiguous group of query
 heads, and its gradient is the sum over that group.
 
+Few new rows over many keys (a generation step).  The pages name attention engines
+for LLM inference that work on the key/value cache during streaming generation
+(FlashAttention (NL), "Gespecialiseerde oplossingen": FlashInfer; its reference
+list adds FlashDecoding++).  Reading: N_q query rows attend N_k >= N_q keys, and
+query row i stands at position N_k - N_q + i of the key sequence (the new rows are
+the last N_q positions, after the cached ones), so the causal and window masks
+above apply to that position.  With N_q = N_k this is the self-attention above.
+
 Arithmetic is numpy float64 with ``@`` (BLAS DGEMM) as the only library step.
 Parity of every function here is pinned by tests/test_oracle.py.
 """
@@ -64,6 +72,7 @@ __all__ = [
     "kv_head_of",
     "attention_forward_shared_kv",
     "attention_backward_shared_kv",
+    "attention_forward_decode",
 ]
 
 
@@ -257,6 +266,28 @@ def attention_backward_shared_kv(q, k, v, do, scale: float, causal: bool = False
     dk = dk.reshape(dk.shape[:-3] + group + dk.shape[-2:]).sum(axis=-3)
     dv = dv.reshape(dv.shape[:-3] + group + dv.shape[-2:]).sum(axis=-3)
     return dq, dk, dv
+
+
+def _decode_row_start(n_q: int, n_k: int) -> int:
+    """Position, among the n_k keys, of the first of n_q new query rows: they are the last n_q."""
+    return n_k - n_q
+
+
+def attention_forward_decode(q, k, v, scale: float, causal: bool = False, window: int = 0):
+    """Forward of N_q new query rows over N_k >= N_q keys: q [..., H, N_q, d];
+    k, v [..., H_kv, N_k, d] (shared K/V heads as above).
+
+    Query row i stands at key position N_k - N_q + i; the masks apply there.
+    Returns (O [..., H, N_q, d], L [..., H, N_q]).
+    """
+    q, k, v = _as64(q), _as64(k), _as64(v)
+    n_q, n_k = q.shape[-2], k.shape[-2]
+    if n_q > n_k:
+        raise ValueError("more query rows than keys")
+    idx = kv_head_of(q.shape[-3], k.shape[-3])
+    start = _decode_row_start(n_q, n_k)
+    return _per_head(lambda a, b, c: _head_forward(a, b, c, scale, causal, window, start)[:2],
+                     q, k[..., idx, :, :], v[..., idx, :, :])
 
 
 def allowed_pairs(n: int, causal: bool, window: int) -> int:

@@ -390,6 +390,71 @@ def shared_kv_finite_differences(orc):
             assert np.linalg.norm(fd - g) / np.linalg.norm(fd) < 1e-6, (which, causal, window)
 
 
+def _decode_torch_mask(n_q, n_k, causal, window):
+    """Boolean [n_q, n_k] mask of the generation-step reading: row i sits at key position
+    n_k - n_q + i (written here with torch ops, apart from the oracle's mask code)."""
+    import torch
+    pos = torch.arange(n_k - n_q, n_k)[:, None]
+    j = torch.arange(n_k)[None, :]
+    ok = torch.ones(n_q, n_k, dtype=torch.bool)
+    if causal:
+        ok &= j <= pos
+    if window:
+        ok &= (j - pos).abs() <= window - 1 if not causal else j >= pos - window + 1
+    return ok
+
+
+def decode_library(orc):
+    """Few new rows over more keys: O agrees with torch scaled_dot_product_attention
+    (float64, enable_gqa, boolean mask) and L with torch.logsumexp of the masked scores, to
+    1e-12, for every mask, with 1, 2 or 4 K/V heads for 4 query heads."""
+    import torch
+    import torch.nn.functional as F
+    r = _rng(31)
+    for n_q, n_k in ((1, 9), (3, 9), (7, 12), (12, 12)):
+        for h_kv in (1, 2, 4):
+            q = r.standard_normal((2, 4, n_q, 6))
+            k, v = (r.standard_normal((2, h_kv, n_k, 6)) for _ in range(2))
+            for causal, window in MASKS:
+                ok = _decode_torch_mask(n_q, n_k, causal, window)
+                tq, tk, tv = (torch.tensor(x, dtype=torch.float64) for x in (q, k, v))
+                o_ref = F.scaled_dot_product_attention(tq, tk, tv, attn_mask=ok, scale=0.45, enable_gqa=True)
+                rep = tk.repeat_interleave(4 // h_kv, dim=1)
+                s = torch.where(ok, 0.45 * tq @ rep.transpose(-1, -2), torch.tensor(-math.inf, dtype=torch.float64))
+                l_ref = torch.logsumexp(s, dim=-1)
+                o, lse = orc.attention_forward_decode(q, k, v, 0.45, causal, window)
+                assert o.shape == q.shape and lse.shape == q.shape[:-1]
+                assert np.max(np.abs(o - o_ref.numpy())) < 1e-12, (n_q, n_k, h_kv, causal, window)
+                assert np.max(np.abs(lse - l_ref.numpy())) < 1e-12, (n_q, n_k, h_kv, causal, window)
+
+
+def decode_scale_zero(orc):
+    """scale = 0 over N_k keys: L_i = ln(#keys allowed at position N_k - N_q + i) and O_i the
+    mean of those v_j, for every mask."""
+    r = _rng(32)
+    n_q, n_k = 4, 11
+    q = r.standard_normal((1, n_q, 3))
+    k, v = (r.standard_normal((1, n_k, 3)) for _ in range(2))
+    for causal, window in MASKS:
+        o, lse = orc.attention_forward_decode(q, k, v, 0.0, causal, window)
+        for i in range(n_q):
+            lo, hi = _band(n_k - n_q + i, n_k, causal, window)
+            assert abs(lse[0, i] - math.log(hi - lo + 1)) < 1e-12, (causal, window, i)
+            assert np.max(np.abs(o[0, i] - v[0, lo:hi + 1].mean(axis=0))) < 1e-12
+
+
+def decode_last_rows_of_self_attention(orc):
+    """The N_q new rows equal the last N_q rows of the self-attention over all N_k positions."""
+    r = _rng(33)
+    q_full, k, v = (r.standard_normal((2, 10, 4)) for _ in range(3))
+    for n_q in (1, 4, 10):
+        for causal, window in MASKS:
+            o_full, l_full = orc.attention_forward(q_full, k, v, 0.6, causal, window)
+            o, lse = orc.attention_forward_decode(q_full[:, None, -n_q:], k[:, None], v[:, None], 0.6, causal, window)
+            assert np.max(np.abs(o[:, 0] - o_full[:, -n_q:])) < 1e-12
+            assert np.max(np.abs(lse[:, 0] - l_full[:, -n_q:])) < 1e-12
+
+
 def rejects_bad_masks(orc):
     """A negative window is rejected, with or without causal."""
     q, k, v = _qkv(21, n=4, d=2, lead=())
@@ -406,5 +471,6 @@ PINS = {f.__name__: f for f in (
     window_covering_is_causal, window_edge, scale_zero, key_shift, key_permutation,
     large_scores, golden_examples, library_forward, library_backward, finite_differences,
     delta_identity, row_blocks_match, pair_count, two_sided_window, shared_kv_library,
-    shared_kv_finite_differences, rejects_bad_masks,
+    shared_kv_finite_differences, decode_library, decode_scale_zero, decode_last_rows_of_self_attention,
+    rejects_bad_masks,
 )}

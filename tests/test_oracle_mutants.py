@@ -129,6 +129,8 @@ def _backward_shared_kv_first_only(q, k, v, do, scale, causal=False, window=0):
 
 
 MUTANTS = {
+    "decode_rows_first": ("_decode_row_start", lambda n_q, n_k: 0),
+    "decode_rows_one_early": ("_decode_row_start", lambda n_q, n_k: max(0, n_k - n_q - 1)),
     "scores_transposed": ("_scores", _scores_transposed),
     "scale_dropped": ("_scores", _scores_no_scale),
     "causal_excludes_diagonal": ("_rows_mask", _rows_mask_causal_strict),
