@@ -41,7 +41,7 @@ WORKLOAD = "causal"          # forward workload; the backward uses the same shap
 GRAD_WORKLOAD = "bwd"
 # --workload choices: the forward workload and the one whose dO seed the backward uses
 BENCH_WORKLOADS = {"causal": ("causal", "bwd"), "long": ("long", "long"), "swa": ("swa", "swa"),
-                   "gqa": ("gqa", "gqa")}
+                   "gqa": ("gqa", "gqa"), "decode": ("decode", "decode")}
 FLUSH_BYTES = 256 << 20      # > 126 MB L2
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -60,7 +60,8 @@ def parse_args():
     ap.add_argument("--workload", choices=sorted(BENCH_WORKLOADS), default="causal",
                     help="causal: B2 H32 N4096 d128 (the default line); gqa: the same with 8 K/V heads; "
                          "long / swa: N32768 with a one- / two-sided window of 4096, FLOPs counted over "
-                         "the pairs the band keeps")
+                         "the pairs the band keeps; decode: one new row per query head over 32768 "
+                         "cached keys (B8, 64 query heads on 8 K/V heads), forward only, HBM-bound")
     return ap.parse_args()
 
 
@@ -83,6 +84,41 @@ def fwd_flops(B, H, N, d, causal, window=0) -> float:
 
 def bwd_flops(B, H, N, d, causal, window=0) -> float:
     return 2.5 * fwd_flops(B, H, N, d, causal, window)
+
+
+def decode_band(pos, n_k, causal, window):
+    """Closed interval of keys a query at key position pos may attend (the mask readings)."""
+    lo = max(0, pos - window + 1) if window > 0 else 0
+    if causal:
+        hi = pos
+    elif window > 0:
+        hi = min(n_k - 1, pos + window - 1)
+    else:
+        hi = n_k - 1
+    return lo, hi
+
+
+def decode_pairs(n_q, n_k, causal, window) -> int:
+    """(query, key) pairs kept when n_q new rows stand at the last n_q of n_k key positions."""
+    total = 0
+    for i in range(n_q):
+        lo, hi = decode_band(n_k - n_q + i, n_k, causal, window)
+        total += hi - lo + 1
+    return total
+
+
+def decode_flops(B, H, n_q, n_k, d, causal, window=0) -> float:
+    """4 d per kept (query, key) pair: Q K^T and P V, two flops per multiply-add."""
+    return 4.0 * B * H * d * decode_pairs(n_q, n_k, causal, window)
+
+
+def decode_bytes(B, H, H_kv, n_q, n_k, d, causal, window=0) -> int:
+    """Algorithmic HBM bytes of a decode forward: read Q (bf16) and, once, the K and V rows
+    of the keys any new row may attend; write O (bf16) and L (fp32)."""
+    lo, _ = decode_band(n_k - n_q, n_k, causal, window)
+    _, hi = decode_band(n_k - 1, n_k, causal, window)
+    keys = hi - lo + 1
+    return 2 * B * H * n_q * d * 2 + 2 * B * H_kv * keys * d * 2 + B * H * n_q * 4
 
 
 def max_over_ranks(values, device=None):
@@ -462,6 +498,168 @@ def load_traffic(kernel: str):
     return entry["bytes"]
 
 
+# ----------------------------------------------------------------------------- decode arm
+_INPUT_CACHE = {}
+
+
+def decode_oracle_sample(seconds: float, max_heads: int | None = None):
+    """Time the fp64 oracle's decode forward head by head (batch entry 0) on the decode
+    workload.  Returns (flops credited, seconds, heads, cores)."""
+    from oracle import attention as orc
+    from synthetic import WORKLOADS, make_inputs
+    wl = WORKLOADS["decode"]
+    if "decode" not in _INPUT_CACHE:
+        _INPUT_CACHE["decode"] = make_inputs(wl)
+    q, k, v = _INPUT_CACHE["decode"]
+    g = wl.H // wl.kv_heads
+    per_head = decode_flops(1, 1, wl.q_rows, wl.N, wl.d, wl.causal, wl.window)
+    t0 = time.perf_counter()
+    heads = 0
+    while True:
+        h = heads % wl.H
+        orc.attention_forward_decode(q[0:1, h:h + 1], k[0:1, h // g:h // g + 1], v[0:1, h // g:h // g + 1],
+                                     wl.scale, wl.causal, wl.window)
+        heads += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or (max_heads is not None and heads >= max_heads):
+            break
+    return per_head * heads, el, heads, blas_threads()
+
+
+def decode_workload_text(wl) -> str:
+    return (f"decode forward: B={wl.B} H={wl.H} (K/V heads {wl.kv_heads}) N_q={wl.q_rows} new row(s) at "
+            f"the last positions of N_k={wl.N} keys, d={wl.d} {'causal' if wl.causal else 'no mask'}"
+            f"{f' window {wl.window}' if wl.window else ''}, inputs N(0,1)*{wl.std:g} bf16 seeded")
+
+
+def run_decode(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=300))
+
+    import exact_io_aware_77_b200 as fa
+    fa.load()
+    from synthetic import WORKLOADS, make_inputs
+    wl = WORKLOADS["decode"]
+    B, H, Hkv, Nq, Nk, d = wl.B, wl.H, wl.kv_heads, wl.q_rows, wl.N, wl.d
+    q_h, k_h, v_h = make_inputs(wl)
+    q, k, v = (x.to(dev) for x in (q_h, k_h, v_h))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=dev)
+    need = fa.decode_workspace_size(B, H, Hkv, Nq, Nk, d, wl.causal, wl.window)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    launches = 2 if need else 1                  # split kernel, then the split merge
+    flops = decode_flops(B, H, Nq, Nk, d, wl.causal, wl.window)
+    nbytes = decode_bytes(B, H, Hkv, Nq, Nk, d, wl.causal, wl.window)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        fa.decode(q, k, v, wl.scale, wl.causal, wl.window, out=o, lse=lse, workspace=ws)
+        if ev:
+            ev[1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    st = fa.check_status(dev)
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {fa.STATUS_NAMES.get(st, st)}")
+    sampler = ClockSampler(gpu_id_for(local))
+    sampler.start()
+    time.sleep(0.3)
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    wall0 = time.time()
+    for i in range(args.steps):
+        step(events[i])                           # K and V (1.07 GB) exceed L2: no flush needed
+    torch.cuda.synchronize(dev)
+    wall1 = time.time()
+    if world > 1:
+        dist.barrier()
+    sampler.mark(wall0, wall1)
+    time.sleep(0.25)
+    sampler.stop()
+    st = fa.check_status(dev)
+    if st != 0:
+        raise RuntimeError(f"device status after timing: {fa.STATUS_NAMES.get(st, st)}")
+    total = max_over_ranks([sum(e[0].elapsed_time(e[1]) for e in events)], dev)[0]
+    ms = total / args.steps
+    value = job_throughput(world, flops, ms)
+
+    e2e = None
+    if not args.no_e2e:
+        pin = [x.pin_memory() for x in (q_h, k_h, v_h)]
+        o_h = torch.empty_like(pin[0]).pin_memory()
+        l_h = torch.empty((B, H, Nq), dtype=torch.float32).pin_memory()
+        qe, ke, ve = (torch.empty_like(x, device=dev) for x in pin)
+
+        def one():
+            for dst, src in zip((qe, ke, ve), pin):
+                dst.copy_(src, non_blocking=True)
+            fa.decode(qe, ke, ve, wl.scale, wl.causal, wl.window, out=o, lse=lse, workspace=ws)
+            o_h.copy_(o, non_blocking=True)
+            l_h.copy_(lse, non_blocking=True)
+
+        one()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(1, min(args.e2e_steps, 3))
+        e0.record(stream)
+        for _ in range(n_e2e):
+            one()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_e2e = max_over_ranks([e0.elapsed_time(e1) / n_e2e], dev)[0]
+        e2e = {"value": round(job_throughput(world, flops, ms_e2e), 4), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in pin),
+               "d2h_bytes_per_step": o_h.numel() * 2 + l_h.numel() * 4, "ms_per_step": round(ms_e2e, 3)}
+
+    peaks, peak_kind = load_peaks()
+    achieved = nbytes / (ms * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "kernel": "fa_decode_kernel<128>+fa_decode_merge_kernel<128>",
+                "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json)" if peak_kind == "measured"
+                else "fallback 6.65 TB/s",
+                "algorithmic_bytes": nbytes, "traffic": None}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        f, secs, heads, cores = decode_oracle_sample(args.cpu_seconds)
+        cpu = {"value": round(f / secs / 1e12, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+               "sample": f"{heads} query heads (batch entry 0) of the decode workload through the fp64 "
+                         f"oracle, {secs:.1f} s, credited each head's FLOPs"}
+    line = {
+        "metric": "attention fwd/bwd TFLOP/s at 1 B200; % of dense BF16 tensor peak",
+        "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": decode_workload_text(wl), "global_batch": B * world, "seq_len": Nk,
+                   "parallelism": f"replicas{world}",
+                   "l2": "not flushed: the K and V read each step (1.07 GB) exceed the 126 MB L2"},
+        "hbm_gbs": round(achieved, 1),
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": args.steps * launches,
+        "clocks": sampler.summary(),
+    }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 # ----------------------------------------------------------------------------- reference arm
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
@@ -469,6 +667,8 @@ def run_reference(args):
         return
     from synthetic import WORKLOADS
     wl = WORKLOADS[WORKLOAD]
+    if WORKLOAD == "decode":
+        return run_decode_reference(args, wl)
     import exact_io_aware_77_b200 as fa_pkg   # only to learn whether the path has a backward
     with_bwd = hasattr(fa_pkg, "backward")
     times, flops = [], []
@@ -497,6 +697,32 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_decode_reference(args, wl):
+    times, flops = [], []
+    cores = blas_threads()
+    for i in range(args.warmup + args.steps):
+        f, secs, _, cores = decode_oracle_sample(0.0, max_heads=1)
+        if i >= args.warmup:
+            times.append(secs)
+            flops.append(f)
+    secs = sum(times)
+    value = sum(flops) / secs / 1e12
+    line = {
+        "metric": "attention fwd/bwd TFLOP/s at 1 B200; % of dense BF16 tensor peak",
+        "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * secs / args.steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": decode_workload_text(wl) + " (one-head sample per step)",
+                   "global_batch": wl.B, "seq_len": wl.N, "parallelism": "cpu"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": "each step: query head 0 of batch entry 0 of the decode workload through "
+                                   "the fp64 oracle, credited that head's FLOPs"},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
 def workload_text(wl, with_bwd: bool) -> str:
     if wl.window:
         band = (f"{'causal' if wl.causal else 'two-sided'} window {wl.window}, FLOPs over the "
@@ -515,6 +741,8 @@ def main():
     WORKLOAD, GRAD_WORKLOAD = BENCH_WORKLOADS[args.workload]
     if args.impl == "reference":
         run_reference(args)
+    elif WORKLOAD == "decode":
+        run_decode(args)
     else:
         run_ours(args)
 

@@ -15,7 +15,7 @@ import math
 from . import _lib
 from ._lib import FAError, STATUS, STATUS_NAMES, load
 
-__all__ = ["forward", "backward", "bwd_workspace_size", "check_status", "FAError", "STATUS", "STATUS_NAMES", "load", "default_scale"]
+__all__ = ["forward", "backward", "decode", "decode_workspace_size", "bwd_workspace_size", "check_status", "FAError", "STATUS", "STATUS_NAMES", "load", "default_scale"]
 
 
 def default_scale(d: int) -> float:
@@ -123,6 +123,56 @@ def backward(q, k, v, o, lse, do, scale: float | None = None, causal: bool = Fal
     else:
         _raise("fa_bwd_phases", _lib.fa_bwd_phases(*args, int(phases), _stream_handle(q.device)))
     return dq, dk, dv
+
+
+def decode_workspace_size(B: int, H: int, H_kv: int, N_q: int, N_k: int, d: int, causal: bool = False,
+                          window: int = 0) -> int:
+    """Bytes of scratch device memory decode() needs (0 when the keys fit one split)."""
+    if not (1 <= N_q <= N_k and B >= 1 and H_kv >= 1 and H % H_kv == 0 and d in (64, 128) and window >= 0):
+        raise ValueError("invalid shape")
+    return _lib.fa_decode_workspace_size(B, H, H_kv, N_q, N_k, d, int(bool(causal)), int(window))
+
+
+def decode(q, k, v, scale: float | None = None, causal: bool = False, window: int = 0,
+           out=None, lse=None, workspace=None):
+    """O, L for N_q new query rows over N_k >= N_q keys (a generation step over a K/V cache).
+
+    q: bf16 [B, H, N_q, d]; k, v: bf16 [B, H_kv, N_k, d]; query row i stands at key position
+    N_k - N_q + i, where the causal and window masks apply.  Returns O bf16 [B, H, N_q, d] and
+    L fp32 [B, H, N_q].  Any strides with a contiguous last dimension.
+    """
+    import torch
+    for t in (q, k, v):
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.dim() == 4 and t.stride(-1) == 1):
+            raise ValueError("expected bf16 CUDA tensors of shape [B, heads, N, d] with contiguous d")
+        if t.device != q.device:
+            raise ValueError("device mismatch")
+    B, H, N_q, d = q.shape
+    if k.shape != v.shape or k.shape[0] != B or k.shape[3] != d:
+        raise ValueError("k and v must be [B, H_kv, N_k, d]")
+    H_kv, N_k = int(k.shape[1]), int(k.shape[2])
+    scale = default_scale(d) if scale is None else float(scale)
+    need = decode_workspace_size(B, H, H_kv, N_q, N_k, d, causal, window)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N_q), dtype=torch.float32, device=q.device)
+    if out.shape != q.shape or out.stride(-1) != 1 or out.dtype != torch.bfloat16 or out.device != q.device:
+        raise ValueError("out must be a bf16 tensor shaped like q with contiguous d")
+    if not (lse.dtype == torch.float32 and lse.is_contiguous() and lse.numel() == B * H * N_q and lse.device == q.device):
+        raise ValueError("lse must be a contiguous fp32 tensor of B*H*N_q elements")
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = workspace.data_ptr() if workspace is not None else 0
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = None
+    if not all(t.is_contiguous() for t in (q, k, v, out)):
+        st = _lib.strides_array((q, k, v, out))
+    _raise("fa_fwd_decode", _lib.fa_fwd_decode(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, H, H_kv, N_q, N_k, d,
+        ctypes.addressof(st) if st is not None else 0, scale, int(bool(causal)), int(window), ws_ptr, ws_bytes,
+        _stream_handle(q.device)))
+    return out, lse
 
 
 def check_status(device=None) -> int:

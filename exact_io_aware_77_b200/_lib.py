@@ -41,6 +41,9 @@ SIGNATURES = {
                                                                  _c_size_t, _c_int, _c_void_p]),
     "fa_bwd_gqa": (_c_int, [_c_void_p] * 9 + [_c_int] * 5 + [_c_float, _c_int, _c_int, _c_void_p, _c_size_t,
                                                              _c_int, _c_void_p]),
+    "fa_decode_workspace_size": (_c_size_t, [_c_int] * 8),
+    "fa_fwd_decode": (_c_int, [_c_void_p] * 5 + [_c_int] * 6 + [_c_void_p, _c_float, _c_int, _c_int, _c_void_p,
+                                                                _c_size_t, _c_void_p]),
     "fa_status_string": (ctypes.c_char_p, [_c_int]),
     "fa_check_status": (_c_int, [_c_void_p]),
     "fa_set_wait_limit_ns": (None, [_c_ull]),
@@ -150,6 +153,17 @@ def fa_bwd_strided(q, k, v, o, lse, dO, dq, dk, dv, B, H, H_kv, N, d, strides, s
     """fa_bwd_gqa with per-array strides (``strides``: address of 8 fa_strides)."""
     return _call("fa_bwd_strided", q, k, v, o, lse, dO, dq, dk, dv, B, H, H_kv, N, d, strides, scale, causal,
                  window, workspace, workspace_bytes, phases, stream)
+
+
+def fa_decode_workspace_size(B, H, H_kv, N_q, N_k, d, causal, window) -> int:
+    return _call("fa_decode_workspace_size", B, H, H_kv, N_q, N_k, d, causal, window)
+
+
+def fa_fwd_decode(q, k, v, o, lse, B, H, H_kv, N_q, N_k, d, strides, scale, causal, window, workspace,
+                  workspace_bytes, stream) -> int:
+    """Forward of N_q new query rows (the last N_q key positions) over N_k keys."""
+    return _call("fa_fwd_decode", q, k, v, o, lse, B, H, H_kv, N_q, N_k, d, strides, scale, causal, window,
+                 workspace, workspace_bytes, stream)
 
 
 def fa_status_string(status: int) -> str:

@@ -18,7 +18,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libfa_b200.so")
 SOURCES = ["fa_api.cu"]
-DEPS = ["fa_api.cu", "sm100.cuh", "fwd_kernel.cuh", "bwd_kernel.cuh"]
+DEPS = ["fa_api.cu", "sm100.cuh", "fwd_kernel.cuh", "bwd_kernel.cuh", "decode_ops.cuh",
+        "decode_kernel.cuh"]
 
 
 def nvcc_path() -> str:

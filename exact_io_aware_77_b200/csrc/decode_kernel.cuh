@@ -1,0 +1,397 @@
+// Split-key forward for a few new query rows over a long key sequence (a generation step
+// over a key/value cache).
+//
+// Query row i stands at key position N_k - N_q + i, and the causal and window masks apply
+// there.  The rows that read one K/V head (its group of query heads times the N_q new
+// positions, "rows" in all) are cut into blocks of 16, the M of an m16n8k16 warp MMA, so one
+// pass over the head's keys serves all of them.  The keys are cut into chunks ("splits"),
+// one CTA per (split, row block, K/V head).  Each of a CTA's four warps streams its own
+// 16-key steps through a private three-stage cp.async ring and keeps its own running max m,
+// sum l and unnormalised output; the CTA merges its warps, and when there is more than one
+// split a second kernel merges the splits by their logsumexps:
+//   L = M + ln sum_s exp(L_s - M),  O = sum_s exp(L_s - L) O_s   (M = max_s L_s).
+// Every split's O_s is already normalised by its own l; a split with no allowed key has
+// L_s = -inf and weight 0.  The work is bound by reading K and V from HBM once.
+#pragma once
+
+#include <climits>
+#include <cstdint>
+
+#include "sm100.cuh"
+
+namespace fa {
+
+constexpr int kDecWarps = 4;
+constexpr int kDecThreads = 32 * kDecWarps;
+constexpr int kDecRows = 16;        // query rows per CTA: the M of the MMA
+constexpr int kDecKeys = 16;        // keys per warp step
+constexpr int kDecStages = 3;       // depth of each warp's copy ring
+constexpr int kDecMergeWarps = 8;   // warps (one output row each) per CTA of the split merge
+constexpr int kDecSlots = 148 * 2;  // CTAs resident at once on a B200 (148 SMs, two CTAs each)
+constexpr int kDecCtaOverheadKeys = 128;   // a CTA's fixed cost (Q load, ring fill, merge), in keys
+
+template <int D>
+struct DecLayout {
+  // one K or V row in shared memory, padded by 16 bytes so that the eight rows an 8x8
+  // matrix load reads start in eight different 16-byte bank groups
+  static constexpr int kRowBytes = 2 * D + 16;
+  static constexpr int kTileBytes = kDecKeys * kRowBytes;
+  static constexpr int kStageBytes = 2 * kTileBytes;   // K rows, then V rows
+  static constexpr int kWarpBytes = kDecStages * kStageBytes;
+  static constexpr int kRingBytes = kDecWarps * kWarpBytes;
+  // after the key loop the rings hold each warp's O [16][D], m [16] and l [16] (fp32)
+  static constexpr int kMergeFloats = kDecRows * D + 2 * kDecRows;
+  static constexpr int kMergeBytes = kDecWarps * kMergeFloats * 4;
+  static constexpr int kSmemBytes = kRingBytes > kMergeBytes ? kRingBytes : kMergeBytes;
+};
+
+struct DecParams {
+  const __nv_bfloat16* q;   // [B, H, N_q, d]
+  const __nv_bfloat16* k;   // [B, H_kv, N_k, d]
+  const __nv_bfloat16* v;
+  __nv_bfloat16* o;         // [B, H, N_q, d]
+  float* lse;               // [B, H, N_q] contiguous
+  float* o_part;            // [n_splits][total_rows][d]; only when n_splits > 1
+  float* l_part;            // [n_splits][total_rows]
+  Strides q_st, k_st, v_st, o_st;
+  long long total_rows;     // B * H * N_q
+  int H, H_kv, group, Nq, Nk;
+  int rows, row_blocks;     // rows per K/V head (group * N_q), blocks of 16 of them
+  int n_splits, chunk, key_begin;   // split s covers keys [key_begin + s chunk, + chunk)
+  int causal, window;
+  float scale_log2;         // scale * log2(e)
+};
+
+// Closed interval [lo, hi] of the keys a query at position pos may attend.
+__host__ __device__ inline void dec_band(int pos, int Nk, int causal, int window, int& lo, int& hi) {
+  if (causal) {
+    hi = pos;
+    lo = window > 0 ? pos - window + 1 : 0;
+  } else if (window > 0) {
+    lo = pos - window + 1;
+    hi = pos + window - 1;
+  } else {
+    lo = 0;
+    hi = Nk - 1;
+  }
+  if (lo < 0) lo = 0;
+  if (hi > Nk - 1) hi = Nk - 1;
+}
+
+// How a decode problem is cut: a pure function of the shapes, so that the workspace size
+// can be asked before the call.  window must already be clamped to N_k.
+struct DecPlan {
+  int rows, row_blocks, n_splits, chunk, key_begin;
+  long long total_rows, ctas;
+  size_t ws_bytes;
+};
+
+inline DecPlan dec_plan(int B, int H, int H_kv, int Nq, int Nk, int d, int causal, int window) {
+  DecPlan pl;
+  pl.rows = (H / H_kv) * Nq;
+  pl.row_blocks = (pl.rows + kDecRows - 1) / kDecRows;
+  pl.total_rows = (long long)B * H * Nq;
+  // keys any row may attend: the bands move right with the position, so they run from the
+  // first row's lowest key to the last row's highest
+  int lo_first, hi_first, lo_last, hi_last;
+  dec_band(Nk - Nq, Nk, causal, window, lo_first, hi_first);
+  dec_band(Nk - 1, Nk, causal, window, lo_last, hi_last);
+  pl.key_begin = lo_first & ~(kDecKeys - 1);
+  const int steps = (hi_last + 1 - pl.key_begin + kDecKeys - 1) / kDecKeys;
+  const long long base = (long long)B * H_kv * pl.row_blocks;
+  // pick the split count that minimises (waves of resident CTAs) x (keys per CTA + its fixed
+  // cost); at least two steps per warp in a split
+  int max_splits = steps / (2 * kDecWarps);
+  if (max_splits < 1) max_splits = 1;
+  if (max_splits > 512) max_splits = 512;
+  long long best_cost = -1;
+  int best_steps = steps;
+  for (int ns = 1; ns <= max_splits; ++ns) {
+    const int per = (steps + ns - 1) / ns;
+    const int used = (steps + per - 1) / per;
+    const long long waves = (base * used + kDecSlots - 1) / kDecSlots;
+    const long long cost = waves * ((long long)per * kDecKeys + kDecCtaOverheadKeys);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best_steps = per;
+    }
+  }
+  pl.chunk = best_steps * kDecKeys;
+  pl.n_splits = (steps + best_steps - 1) / best_steps;
+  pl.ctas = base * pl.n_splits;
+  pl.ws_bytes = pl.n_splits > 1 ? size_t(pl.n_splits) * size_t(pl.total_rows) * size_t(d + 1) * 4 : 0;
+  return pl;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kDecThreads, 2) fa_decode_kernel(const DecParams p) {
+  using Lay = DecLayout<D>;
+  constexpr int KS = D / 16;   // k-steps of S = Q K^T
+  constexpr int NT = D / 8;    // 8-column n-tiles of O
+  constexpr float kLn2 = 0.6931471805599453f;
+  unsigned char* smem = dec_dyn_smem();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;   // MMA fragment row group and column pair
+
+  int bid = blockIdx.x;
+  const int rb = bid % p.row_blocks;
+  bid /= p.row_blocks;
+  const int split = bid % p.n_splits;
+  bid /= p.n_splits;
+  const int hkv = bid % p.H_kv, b = bid / p.H_kv;
+  const int row0 = rb * kDecRows;
+  const int pos0 = p.Nk - p.Nq;   // key position of query row 0
+
+  // bands of the block's rows: the union bounds the keys to visit, the intersection says
+  // which 16-key steps need no mask
+  int lo_min = INT_MAX, hi_max = -1, lo_max = 0, hi_min = INT_MAX;
+  for (int lr = 0; lr < kDecRows && row0 + lr < p.rows; ++lr) {
+    int lo, hi;
+    dec_band(pos0 + (row0 + lr) % p.Nq, p.Nk, p.causal, p.window, lo, hi);
+    lo_min = min(lo_min, lo);
+    hi_max = max(hi_max, hi);
+    lo_max = max(lo_max, lo);
+    hi_min = min(hi_min, hi);
+  }
+
+  // this lane's rows g and g + 8 of the block (rows past the end stay unmasked, read zero Q
+  // and are never written)
+  int band_lo[2], band_hi[2];
+  const __nv_bfloat16* qrow[2];
+  for (int hf = 0; hf < 2; ++hf) {
+    const int r = row0 + g + 8 * hf;
+    if (r < p.rows) {
+      const int hq = hkv * p.group + r / p.Nq, i = r % p.Nq;
+      dec_band(pos0 + i, p.Nk, p.causal, p.window, band_lo[hf], band_hi[hf]);
+      qrow[hf] = p.q + p.q_st.at(b, hq, i);
+    } else {
+      band_lo[hf] = INT_MIN;
+      band_hi[hf] = INT_MAX;
+      qrow[hf] = nullptr;
+    }
+  }
+  // Q as the A operand of every k-step: rows g, g + 8; columns 2t, 2t + 1 (+ 8)
+  uint32_t qa[KS][4];
+#pragma unroll
+  for (int kk = 0; kk < KS; ++kk) {
+    const int c = 16 * kk + 2 * t;
+    qa[kk][0] = qrow[0] ? ld_global_u32(qrow[0] + c) : 0u;
+    qa[kk][1] = qrow[1] ? ld_global_u32(qrow[1] + c) : 0u;
+    qa[kk][2] = qrow[0] ? ld_global_u32(qrow[0] + c + 8) : 0u;
+    qa[kk][3] = qrow[1] ? ld_global_u32(qrow[1] + c + 8) : 0u;
+  }
+
+  // this CTA's keys, in 16-key steps dealt round-robin to the warps
+  const int k_begin = p.key_begin + split * p.chunk;
+  const int k_end = min(p.Nk, k_begin + p.chunk);
+  const int kb = max(k_begin, lo_min), ke = min(k_end - 1, hi_max);
+  const int s0 = kb & ~(kDecKeys - 1);
+  const int n_steps = kb <= ke ? (ke - s0) / kDecKeys + 1 : 0;
+  const int my_steps = n_steps > warp ? (n_steps - warp + kDecWarps - 1) / kDecWarps : 0;
+
+  unsigned char* ring = smem + warp * Lay::kWarpBytes;
+  auto issue = [&](int it) {
+    const int key0 = s0 + kDecKeys * (warp + kDecWarps * it);
+    unsigned char* stage = ring + (it % kDecStages) * Lay::kStageBytes;
+    constexpr int kPieces = D / 8;   // 16-byte pieces per row
+#pragma unroll
+    for (int x = 0; x < kDecKeys * kPieces / 32; ++x) {
+      const int c = lane + 32 * x;
+      const int row = c / kPieces, col = c % kPieces;
+      const int key = key0 + row;
+      const bool in = key < p.Nk;
+      const int src_key = in ? key : 0;
+      cp_async_16(stage + row * Lay::kRowBytes + col * 16, p.k + p.k_st.at(b, hkv, src_key) + col * 8, in ? 16 : 0);
+      cp_async_16(stage + Lay::kTileBytes + row * Lay::kRowBytes + col * 16,
+                  p.v + p.v_st.at(b, hkv, src_key) + col * 8, in ? 16 : 0);
+    }
+  };
+
+  float acc[NT][4];
+#pragma unroll
+  for (int j = 0; j < NT; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+
+#pragma unroll
+  for (int it = 0; it < kDecStages - 1; ++it) {
+    if (it < my_steps) issue(it);
+    cp_async_commit();
+  }
+  for (int it = 0; it < my_steps; ++it) {
+    cp_async_wait<kDecStages - 2>();   // step it has landed (this lane's pieces)
+    __syncwarp();                      // ... and every lane's; all lanes are past step it - 1
+    const unsigned char* ks = ring + (it % kDecStages) * Lay::kStageBytes;
+    const unsigned char* vs = ks + Lay::kTileBytes;
+    const int key0 = s0 + kDecKeys * (warp + kDecWarps * it);
+
+    // S = Q K^T for 16 keys: n-tiles of keys 0-7 and 8-15
+    float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+    for (int kk = 0; kk < KS; ++kk) {
+      uint32_t kf[4];   // matrices: keys 0-7 | 8-15  x  columns 16kk + 0-7 | 8-15
+      ldmatrix_x4(kf, ks + (((lane >> 4) << 3) + (lane & 7)) * Lay::kRowBytes + (16 * kk + ((lane >> 3) & 1) * 8) * 2);
+      mma_16816(s[0], qa[kk], kf[0], kf[1]);
+      mma_16816(s[1], qa[kk], kf[2], kf[3]);
+    }
+    // scale into the log2 domain; mask keys outside a row's band (and past N_k)
+    const bool need_mask = key0 < lo_max || key0 + kDecKeys - 1 > hi_min;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        s[nt][c] *= p.scale_log2;
+        if (need_mask) {
+          const int key = key0 + 8 * nt + 2 * t + (c & 1);
+          if (key < band_lo[c >> 1] || key > band_hi[c >> 1]) s[nt][c] = -INFINITY;
+        }
+      }
+    // online softmax per row: the four lanes of a row group share it
+    float alpha[2];
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      float mx = fmaxf(fmaxf(s[0][2 * hf], s[0][2 * hf + 1]), fmaxf(s[1][2 * hf], s[1][2 * hf + 1]));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      const float m_new = fmaxf(m_run[hf], mx);
+      const float m_use = m_new == -INFINITY ? 0.f : m_new;   // a row with no key yet stays at 0
+      alpha[hf] = ex2_approx(m_run[hf] - m_use);
+      m_run[hf] = m_new;
+      float sum = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          s[nt][2 * hf + e] = ex2_approx(s[nt][2 * hf + e] - m_use);
+          sum += s[nt][2 * hf + e];
+        }
+      l_run[hf] = l_run[hf] * alpha[hf] + sum;   // this lane's share; summed over the group at the end
+    }
+    // O = alpha O + P V; P (bf16) is the A operand straight from the S fragments
+    const uint32_t pa[4] = {pack_bf16x2(s[0][0], s[0][1]), pack_bf16x2(s[0][2], s[0][3]),
+                            pack_bf16x2(s[1][0], s[1][1]), pack_bf16x2(s[1][2], s[1][3])};
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      acc[j][0] *= alpha[0];
+      acc[j][1] *= alpha[0];
+      acc[j][2] *= alpha[1];
+      acc[j][3] *= alpha[1];
+    }
+#pragma unroll
+    for (int j = 0; j < D / 16; ++j) {
+      uint32_t vf[4];   // transposed matrices: keys 0-7 | 8-15  x  columns 16j + 0-7 | 8-15
+      ldmatrix_x4_trans(vf, vs + (((lane >> 3) & 1) * 8 + (lane & 7)) * Lay::kRowBytes + (16 * j + (lane >> 4) * 8) * 2);
+      mma_16816(acc[2 * j], pa, vf[0], vf[1]);
+      mma_16816(acc[2 * j + 1], pa, vf[2], vf[3]);
+    }
+    if (it + kDecStages - 1 < my_steps) issue(it + kDecStages - 1);
+    cp_async_commit();
+  }
+  cp_async_wait<0>();
+#pragma unroll
+  for (int hf = 0; hf < 2; ++hf) {
+    l_run[hf] += __shfl_xor_sync(0xffffffffu, l_run[hf], 1);
+    l_run[hf] += __shfl_xor_sync(0xffffffffu, l_run[hf], 2);
+  }
+
+  // merge the four warps through shared memory (the rings are free once all warps are here)
+  __syncthreads();
+  float* mw = reinterpret_cast<float*>(smem) + warp * Lay::kMergeFloats;
+#pragma unroll
+  for (int j = 0; j < NT; ++j) {
+    *reinterpret_cast<float2*>(mw + g * D + 8 * j + 2 * t) = make_float2(acc[j][0], acc[j][1]);
+    *reinterpret_cast<float2*>(mw + (g + 8) * D + 8 * j + 2 * t) = make_float2(acc[j][2], acc[j][3]);
+  }
+  if (t == 0) {
+    mw[kDecRows * D + g] = m_run[0];
+    mw[kDecRows * D + g + 8] = m_run[1];
+    mw[kDecRows * D + kDecRows + g] = l_run[0];
+    mw[kDecRows * D + kDecRows + g + 8] = l_run[1];
+  }
+  __syncthreads();
+
+  constexpr int kPairs = D / 2;                    // column pairs per row
+  constexpr int kRowSets = kDecThreads / kPairs;   // rows handled side by side
+  const int cp = threadIdx.x % kPairs;
+  const float* all = reinterpret_cast<const float*>(smem);
+  for (int lr = threadIdx.x / kPairs; lr < kDecRows; lr += kRowSets) {
+    const int r = row0 + lr;
+    if (r >= p.rows) break;
+    float mx = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kDecWarps; ++w) mx = fmaxf(mx, all[w * Lay::kMergeFloats + kDecRows * D + lr]);
+    float l = 0.f, o0 = 0.f, o1 = 0.f;
+    if (mx != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kDecWarps; ++w) {
+        const float* src = all + w * Lay::kMergeFloats;
+        const float wt = ex2_approx(src[kDecRows * D + lr] - mx);
+        l += wt * src[kDecRows * D + kDecRows + lr];
+        o0 += wt * src[lr * D + 2 * cp];
+        o1 += wt * src[lr * D + 2 * cp + 1];
+      }
+    }
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    const float lse = l > 0.f ? (mx + lg2_approx(l)) * kLn2 : -INFINITY;
+    const int hq = hkv * p.group + r / p.Nq, i = r % p.Nq;
+    const long long grow = ((long long)b * p.H + hq) * p.Nq + i;
+    if (p.n_splits == 1) {
+      *reinterpret_cast<uint32_t*>(p.o + p.o_st.at(b, hq, i) + 2 * cp) = pack_bf16x2(o0 * inv, o1 * inv);
+      if (cp == 0) p.lse[grow] = lse;
+    } else {
+      const long long prow = (long long)split * p.total_rows + grow;
+      *reinterpret_cast<float2*>(p.o_part + prow * D + 2 * cp) = make_float2(o0 * inv, o1 * inv);
+      if (cp == 0) p.l_part[prow] = lse;
+    }
+  }
+}
+
+// Merge the splits of every output row: one warp per row, D / 32 columns per lane.
+template <int D>
+__global__ void __launch_bounds__(32 * kDecMergeWarps) fa_decode_merge_kernel(const DecParams p) {
+  constexpr float kLn2 = 0.6931471805599453f, kLog2e = 1.4426950408889634f;
+  constexpr int C = D / 32;
+  const long long grow = (long long)blockIdx.x * kDecMergeWarps + (threadIdx.x >> 5);
+  if (grow >= p.total_rows) return;
+  const int lane = threadIdx.x & 31;
+  float mx = -INFINITY;
+  for (int s = 0; s < p.n_splits; ++s) mx = fmaxf(mx, p.l_part[(long long)s * p.total_rows + grow]);
+  float acc[C];
+#pragma unroll
+  for (int c = 0; c < C; ++c) acc[c] = 0.f;
+  float sum = 0.f;
+  if (mx != -INFINITY) {
+    for (int s = 0; s < p.n_splits; ++s) {
+      const long long prow = (long long)s * p.total_rows + grow;
+      const float wt = ex2_approx((p.l_part[prow] - mx) * kLog2e);
+      sum += wt;
+      const float* src = p.o_part + prow * D + lane * C;
+      if constexpr (C == 4) {
+        const float4 x = *reinterpret_cast<const float4*>(src);
+        acc[0] += wt * x.x;
+        acc[1] += wt * x.y;
+        acc[2] += wt * x.z;
+        acc[3] += wt * x.w;
+      } else {
+        const float2 x = *reinterpret_cast<const float2*>(src);
+        acc[0] += wt * x.x;
+        acc[1] += wt * x.y;
+      }
+    }
+  }
+  const float inv = sum > 0.f ? 1.f / sum : 0.f;
+  const int i = int(grow % p.Nq);
+  const long long bh = grow / p.Nq;
+  const int b = int(bh / p.H), hq = int(bh % p.H);
+  __nv_bfloat16* dst = p.o + p.o_st.at(b, hq, i) + lane * C;
+  if constexpr (C == 4) {
+    uint2 w;
+    w.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+    w.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+    *reinterpret_cast<uint2*>(dst) = w;
+  } else {
+    *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+  }
+  if (lane == 0) p.lse[grow] = sum > 0.f ? mx + lg2_approx(sum) * kLn2 : -INFINITY;
+}
+
+}  // namespace fa

@@ -1,0 +1,61 @@
+// Device primitives of the split-key decode kernel: 16-byte asynchronous copies from
+// global into shared memory (zero-filling rows past the end of the keys), 8x8 matrix loads
+// from shared memory into warp MMA operand registers, and the m16n8k16 bf16 warp MMA with
+// fp32 accumulators.  These are warp-level instructions: the decode kernel's rows are too
+// few (16) for a tcgen05 MMA tile, and its time goes to reading K and V from HBM.
+#pragma once
+
+#include <cstdint>
+
+namespace fa {
+
+// The kernel's dynamic shared memory.
+__device__ __forceinline__ unsigned char* dec_dyn_smem() {
+  extern __shared__ __align__(128) unsigned char dec_smem_raw[];
+  return dec_smem_raw;
+}
+
+// Copy 16 bytes from global to shared memory, bypassing L1.  src_bytes = 0 reads nothing
+// and writes 16 zero bytes.
+__device__ __forceinline__ void cp_async_16(void* dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Wait until at most N of this thread's committed copy groups are still in flight.
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Four 8x8 b16 matrices; lane l gives the address of row l % 8 of matrix l / 8, and receives
+// in r[m] the pair (row l / 4, columns 2 (l % 4) and 2 (l % 4) + 1) of matrix m.
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], const void* row) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(row))
+               : "memory");
+}
+// The same, transposed: r[m] holds (rows 2 (l % 4) and 2 (l % 4) + 1, column l / 4) of matrix m.
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], const void* row) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(row))
+               : "memory");
+}
+
+// d += a b for a 16x16 bf16 A (row-major fragment), a 16x8 bf16 B (column fragment) and a
+// 16x8 fp32 accumulator, over one warp.
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t ld_global_u32(const void* p) {
+  return *reinterpret_cast<const uint32_t*>(p);
+}
+
+}  // namespace fa

@@ -13,6 +13,8 @@
 
 #include "fwd_kernel.cuh"
 #include "bwd_kernel.cuh"
+#include "decode_ops.cuh"
+#include "decode_kernel.cuh"
 
 namespace fa {
 namespace {
@@ -203,6 +205,63 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   return FA_OK;
 }
 
+// ---------------------------------------------------------------- decode (few rows, many keys)
+// Validates a decode problem and returns its plan (window clamped to N_k first).
+int check_decode(int B, int H, int H_kv, int Nq, int Nk, int d, float scale, int causal, int window, DecPlan* pl) {
+  if (B < 1 || H < 1 || H_kv < 1 || Nq < 1 || Nk < 1 || Nq > Nk) return FA_ERR_SHAPE;
+  if (check_kv_heads(H, H_kv) != FA_OK) return FA_ERR_SHAPE;
+  if (d != 64 && d != 128) return FA_ERR_HEADDIM;
+  if (!(causal == 0 || causal == 1) || window < 0) return FA_ERR_MASK;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_SCALE;
+  const long long rows = (long long)(H / H_kv) * Nq;
+  if (rows > 0x7fffffffLL - kDecRows || (long long)B * H * Nq > 0x7fffffffLL) return FA_ERR_SHAPE;
+  *pl = dec_plan(B, H, H_kv, Nq, Nk, d, causal, window > Nk ? Nk : window);
+  if (pl->ctas > 0x7fffffffLL) return FA_ERR_SHAPE;
+  return FA_OK;
+}
+
+template <int D>
+int launch_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv, int Nq,
+                  int Nk, const Strides* st, float scale, int causal, int window, void* ws, const DecPlan& pl,
+                  cudaStream_t stream) {
+  DecParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.o_part = static_cast<float*>(ws);
+  p.l_part = pl.n_splits > 1 ? p.o_part + size_t(pl.n_splits) * size_t(pl.total_rows) * D : nullptr;
+  p.q_st = st[0];
+  p.k_st = st[1];
+  p.v_st = st[2];
+  p.o_st = st[3];
+  p.total_rows = pl.total_rows;
+  p.H = H;
+  p.H_kv = H_kv;
+  p.group = H / H_kv;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.rows = pl.rows;
+  p.row_blocks = pl.row_blocks;
+  p.n_splits = pl.n_splits;
+  p.chunk = pl.chunk;
+  p.key_begin = pl.key_begin;
+  p.causal = causal;
+  p.window = window > Nk ? Nk : window;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  constexpr int smem = DecLayout<D>::kSmemBytes;
+  if (set_smem(fa_decode_kernel<D>, smem) != FA_OK) return FA_ERR_CUDA;
+  fa_decode_kernel<D><<<unsigned(pl.ctas), kDecThreads, smem, stream>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  if (pl.n_splits > 1) {
+    const long long blocks = (pl.total_rows + kDecMergeWarps - 1) / kDecMergeWarps;
+    fa_decode_merge_kernel<D><<<unsigned(blocks), 32 * kDecMergeWarps, 0, stream>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
+
 // ---------------------------------------------------------------- backward without caller memory
 // Built-in scratch for fa_bwd_noalloc.  It lives in the module's global memory, so every GPU
 // that loads this library holds these 64 MiB until the process exits.  Host code must not
@@ -348,15 +407,45 @@ static int bwd_impl(const void* q, const void* k, const void* v, const void* o, 
                                    workspace, s, phases);
 }
 
+size_t fa_decode_workspace_size(int B, int H, int H_kv, int N_q, int N_k, int d, int causal, int window) {
+  DecPlan pl;
+  if (check_decode(B, H, H_kv, N_q, N_k, d, 1.f, causal, window, &pl) != FA_OK) return 0;
+  return pl.ws_bytes;
+}
+
+int fa_fwd_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv, int N_q,
+                  int N_k, int d, const fa_strides* strides, float scale, int causal, int window, void* workspace,
+                  size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
+  DecPlan pl;
+  int st = check_decode(B, H, H_kv, N_q, N_k, d, scale, causal, window, &pl);
+  if (st != FA_OK) return st;
+  Strides s4[4] = {packed(H, N_q, d), packed(H_kv, N_k, d), packed(H_kv, N_k, d), packed(H, N_q, d)};
+  if (strides)
+    for (int i = 0; i < 4; ++i) {
+      s4[i] = Strides{strides[i].b, strides[i].h, strides[i].n};
+      if (!strides_ok(s4[i])) return FA_ERR_ALIGN;
+    }
+  if (pl.ws_bytes > 0 && (!workspace || workspace_bytes < pl.ws_bytes)) return FA_ERR_WORKSPACE;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
+      !aligned(workspace, 16))
+    return FA_ERR_ALIGN;
+  if ((st = check_device()) != FA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_decode<64>(q, k, v, o, lse, B, H, H_kv, N_q, N_k, s4, scale, causal, window, workspace, pl, s)
+                 : launch_decode<128>(q, k, v, o, lse, B, H, H_kv, N_q, N_k, s4, scale, causal, window, workspace, pl,
+                                      s);
+}
+
 const char* fa_status_string(int status) {
   switch (status) {
     case FA_OK: return "ok";
     case FA_ERR_NULL: return "null pointer";
-    case FA_ERR_SHAPE: return "bad shape (B, H, N must be >= 1 and within launch limits)";
+    case FA_ERR_SHAPE: return "bad shape (sizes >= 1, H a multiple of H_kv, N_q <= N_k, within launch limits)";
     case FA_ERR_HEADDIM: return "unsupported head dimension (64 or 128)";
     case FA_ERR_ALIGN: return "misaligned pointer (bf16 arrays 16 B, L 4 B)";
     case FA_ERR_MASK: return "bad mask (causal must be 0 or 1, window >= 0)";
-    case FA_ERR_WORKSPACE: return "backward workspace missing or too small";
+    case FA_ERR_WORKSPACE: return "workspace missing or too small";
     case FA_ERR_CUDA: return "CUDA runtime or launch error";
     case FA_ERR_DEVICE: return "device is not compute capability 10.0 (B200)";
     case FA_ERR_TIMEOUT: return "a kernel-side wait timed out";

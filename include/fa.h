@@ -57,11 +57,11 @@ extern "C" {
 typedef enum {
   FA_OK = 0,
   FA_ERR_NULL = 1,       /* a required pointer is NULL */
-  FA_ERR_SHAPE = 2,      /* B, H or N < 1, or the problem exceeds the launch limits */
+  FA_ERR_SHAPE = 2,      /* a size < 1, H not a multiple of H_kv, N_q > N_k, or beyond the launch limits */
   FA_ERR_HEADDIM = 3,    /* d is not 64 or 128 */
   FA_ERR_ALIGN = 4,      /* a bf16 array is not 16-byte aligned, or L not 4-byte aligned */
   FA_ERR_MASK = 5,       /* causal not 0/1, or window < 0 */
-  FA_ERR_WORKSPACE = 6,  /* backward workspace missing or smaller than fa_bwd_workspace_size */
+  FA_ERR_WORKSPACE = 6,  /* workspace missing or smaller than fa_bwd_ / fa_decode_workspace_size */
   FA_ERR_CUDA = 7,       /* a CUDA runtime call or kernel launch failed */
   FA_ERR_DEVICE = 8,     /* the current device is not compute capability 10.0 */
   FA_ERR_TIMEOUT = 9,    /* a kernel-side wait ran out of time (reported by fa_check_status) */
@@ -160,6 +160,34 @@ FA_EXPORT int fa_bwd_strided(const void* q, const void* k, const void* v, const 
                              const void* dO, void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, int d,
                              const fa_strides* strides, float scale, int causal, int window, void* workspace,
                              size_t workspace_bytes, int phases, void* stream);
+
+/*
+ * Forward of a few new query rows over a longer key sequence: a generation step over a
+ * key/value cache.  The FlashAttention (NL) page names engines for LLM inference that work on
+ * the key/value cache during streaming generation ("Gespecialiseerde oplossingen": FlashInfer;
+ * its references add FlashDecoding++); it prints no interface.  Reading: the N_q query rows are
+ * the last N_q of the N_k key positions, so query row i stands at position N_k - N_q + i and
+ * the masks of fa_fwd apply there (causal: keys j <= N_k - N_q + i; with a window W also
+ * j >= N_k - N_q + i - W + 1; a window without causal keeps |j - (N_k - N_q + i)| <= W - 1).
+ * N_q = N_k is the self-attention of fa_fwd_gqa.
+ *
+ *   q, o   bf16 [B, H, N_q, d];  k, v  bf16 [B, H_kv, N_k, d]  (H a multiple of H_kv; query
+ *          head h reads K/V head h / (H / H_kv));  lse  fp32 [B, H, N_q], packed.
+ *   strides  NULL for packed arrays, else 4 fa_strides (q, k, v, o) as for fa_fwd_strided.
+ *   workspace  device memory of at least fa_decode_workspace_size(...) bytes, 16-byte aligned,
+ *          owned by the caller; it holds the per-split partial results (fp32).  When that size
+ *          is 0 (the keys fit one split) workspace may be NULL.
+ *
+ * The keys are cut into splits that run on separate CTAs; a second kernel merges the splits'
+ * partial outputs by their logsumexps.  How the problem is cut depends only on the arguments
+ * of fa_decode_workspace_size, which returns 0 for an invalid problem.  Errors, scale, streams
+ * and ownership are as for fa_fwd; FA_ERR_SHAPE also when N_q > N_k, FA_ERR_WORKSPACE when the
+ * workspace is missing or short.
+ */
+FA_EXPORT size_t fa_decode_workspace_size(int B, int H, int H_kv, int N_q, int N_k, int d, int causal, int window);
+FA_EXPORT int fa_fwd_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv,
+                            int N_q, int N_k, int d, const fa_strides* strides, float scale, int causal, int window,
+                            void* workspace, size_t workspace_bytes, void* stream);
 
 /* Human-readable name of a status code (static string, never NULL). */
 FA_EXPORT const char* fa_status_string(int status);

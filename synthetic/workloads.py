@@ -37,6 +37,7 @@ class Workload:
     oracle_heads: int | None = None  # heads the oracle checks (None = all)
     description: str = ""
     H_kv: int | None = None  # K/V heads (None = H); H must be a multiple (shared K/V heads)
+    Nq: int | None = None    # query rows (None = N); fewer rows than keys: the last Nq positions
 
     @property
     def scale(self) -> float:
@@ -51,6 +52,10 @@ class Workload:
     @property
     def kv_heads(self) -> int:
         return self.H if self.H_kv is None else self.H_kv
+
+    @property
+    def q_rows(self) -> int:
+        return self.N if self.Nq is None else self.Nq
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
@@ -75,6 +80,10 @@ WORKLOADS: dict[str, Workload] = {
     # the causal LLM shape with 8 K/V heads for 32 query heads (grouped-query attention)
     "gqa": Workload("gqa", 2, 32, 4096, 128, causal=True, std=0.5, seed=1007, grad_seed=2007, H_kv=8,
                     description="causal B2 H32 (8 K/V heads) N4096 d128"),
+    # one generation step over a key/value cache: one new row per query head, 64 query heads
+    # on 8 K/V heads (a 70B-class grouped-query layout), 32768 cached positions
+    "decode": Workload("decode", 8, 64, 32768, 128, causal=True, seed=1008, H_kv=8, Nq=1,
+                       description="decode B8 H64 (8 K/V heads) N_q 1 over N_k 32768 d128 causal"),
 }
 
 
@@ -86,10 +95,10 @@ def _randn_bf16(gen: torch.Generator, shape, std: float) -> torch.Tensor:
 
 
 def make_inputs(wl: Workload, seed: int | None = None):
-    """Q [B, H, N, d] and K, V [B, H_kv, N, d] as contiguous CPU bf16 tensors."""
+    """Q [B, H, Nq, d] and K, V [B, H_kv, N, d] as contiguous CPU bf16 tensors."""
     gen = torch.Generator(device="cpu")
     gen.manual_seed(wl.seed if seed is None else seed)
-    q = _randn_bf16(gen, (wl.B, wl.H, wl.N, wl.d), wl.std)
+    q = _randn_bf16(gen, (wl.B, wl.H, wl.q_rows, wl.d), wl.std)
     k = _randn_bf16(gen, (wl.B, wl.kv_heads, wl.N, wl.d), wl.std)
     v = _randn_bf16(gen, (wl.B, wl.kv_heads, wl.N, wl.d), wl.std)
     return q, k, v

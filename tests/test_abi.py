@@ -134,3 +134,56 @@ def test_strided_entry_points_validate_strides(lib):
     st = _lib.fa_bwd_strided(*ptrs, a["B"], a["H"], a["H"], a["N"], a["d"], None, a["scale"], a["causal"],
                              a["window"], A + 65536, 1 << 30, 7, None)
     assert _lib.STATUS_NAMES[st] == "FA_ERR_NULL"
+
+
+def _dec(ws_bytes=1 << 30, **kw):
+    a = dict(B=1, H=8, H_kv=2, N_q=1, N_k=4096, d=128, scale=0.125, causal=1, window=0)
+    ptrs = kw.pop("ptrs", [A + 4096 * i for i in range(5)])
+    ws = kw.pop("ws", A + 65536)
+    st = kw.pop("strides", None)
+    a.update(kw)
+    return _lib.fa_fwd_decode(*ptrs, a["B"], a["H"], a["H_kv"], a["N_q"], a["N_k"], a["d"], st, a["scale"],
+                              a["causal"], a["window"], ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(ptrs=[0] + [A] * 4), "FA_ERR_NULL"),
+    (dict(ptrs=[A] * 4 + [0]), "FA_ERR_NULL"),
+    (dict(N_q=0), "FA_ERR_SHAPE"),
+    (dict(N_q=4097), "FA_ERR_SHAPE"),
+    (dict(H_kv=3), "FA_ERR_SHAPE"),
+    (dict(B=0), "FA_ERR_SHAPE"),
+    (dict(d=96), "FA_ERR_HEADDIM"),
+    (dict(window=-1), "FA_ERR_MASK"),
+    (dict(causal=2), "FA_ERR_MASK"),
+    (dict(scale=0.0), "FA_ERR_SCALE"),
+    (dict(ws=0), "FA_ERR_WORKSPACE"),
+    (dict(ws_bytes=100), "FA_ERR_WORKSPACE"),
+    (dict(ws=A + 8), "FA_ERR_ALIGN"),
+    (dict(ptrs=[A + 8] + [A] * 4), "FA_ERR_ALIGN"),
+    (dict(ptrs=[A] * 4 + [A + 2]), "FA_ERR_ALIGN"),
+])
+def test_decode_rejects_bad_arguments(lib, kw, code):
+    assert _lib.STATUS_NAMES[_dec(**kw)] == code
+
+
+def test_decode_rejects_bad_strides(lib):
+    arr = (_lib.FaStrides * 4)(*[_lib.FaStrides(8 * 4096 * 128, 4096 * 128, 128) for _ in range(4)])
+    arr[2] = _lib.FaStrides(8 * 4096 * 128, 4096 * 128, 100)
+    assert _lib.STATUS_NAMES[_dec(strides=ctypes.addressof(arr))] == "FA_ERR_ALIGN"
+
+
+def test_decode_workspace_size(lib):
+    """0 for an invalid problem and for keys that fit one split; otherwise whole splits of
+    B*H*N_q rows of (d + 1) fp32 values each, at most 512 of them."""
+    size = _lib.fa_decode_workspace_size
+    assert size(1, 8, 3, 1, 100, 128, 1, 0) == 0          # H not a multiple of H_kv
+    assert size(1, 8, 2, 5, 4, 128, 1, 0) == 0            # N_q > N_k
+    assert size(1, 8, 2, 1, 200, 128, 1, 0) == 0          # 13 key steps: one split
+    for B, H, H_kv, N_q, N_k, d, causal, window in ((8, 64, 8, 1, 32768, 128, 1, 0), (2, 16, 2, 1, 3000, 128, 1, 0),
+                                                    (1, 8, 1, 4, 2049, 64, 0, 0), (1, 4, 4, 2, 1 << 20, 64, 0, 0)):
+        n = size(B, H, H_kv, N_q, N_k, d, causal, window)
+        per_split = B * H * N_q * (d + 1) * 4
+        assert n > 0 and n % per_split == 0 and 2 <= n // per_split <= 512, (n, per_split)
+    # a causal window leaves only the last keys to visit: the same as the keys alone
+    assert size(1, 8, 2, 1, 32768, 128, 1, 1000) == size(1, 8, 2, 1, 1000, 128, 1, 0)

@@ -21,3 +21,19 @@ def test_flop_conventions():
     # the long-context shape: 4 d per kept pair, not the causal-halved square
     pairs = orc.allowed_pairs(32768, True, 4096)
     assert bench.fwd_flops(1, 16, 32768, 128, True, 4096) == 4.0 * 16 * 128 * pairs
+
+
+@pytest.mark.parametrize("n_q,n_k", [(1, 1), (1, 300), (3, 40), (17, 17), (5, 777)])
+@pytest.mark.parametrize("causal,window", [(False, 0), (True, 0), (True, 1), (True, 30), (False, 4), (False, 100)])
+def test_decode_pairs_match_oracle_mask(n_q, n_k, causal, window):
+    """Decode rows stand at the last n_q key positions: the kept pairs are the oracle mask's."""
+    assert bench.decode_pairs(n_q, n_k, causal, window) == int(
+        orc.allowed_mask(n_q, n_k, causal, window, n_k - n_q).sum())
+
+
+def test_decode_bytes():
+    # the decode workload: one row per query head, every cached key read once
+    b = bench.decode_bytes(8, 64, 8, 1, 32768, 128, True)
+    assert b == 2 * 8 * 64 * 128 * 2 + 2 * 8 * 8 * 32768 * 128 * 2 + 8 * 64 * 4
+    # a causal window reads only the keys the window keeps
+    assert bench.decode_bytes(1, 1, 1, 1, 10000, 64, True, 100) == 2 * 64 * 2 + 2 * 100 * 64 * 2 + 4
