@@ -470,7 +470,7 @@ def measure_e2e(fa, torch, wl, dev, stream, q_h, k_h, v_h, do_h, has_bwd, steps,
 
 
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu capture of
-# the causal B2 H32 N4096 d128 workload, keyed by kernel, with the SHA-1 of the kernel's sources
+# the workload the bench line times (the causal B2 H32 N4096 d128 one, or the decode one), keyed by kernel, with the SHA-1 of the kernel's sources
 # when the counters were taken (profiles/ holds the summaries).  A changed source reports null.
 NCU_TRAFFIC = {
     "fa_fwd_kernel<128>": {"bytes": 251356416,
@@ -479,6 +479,12 @@ NCU_TRAFFIC = {
     "fa_bwd_kernel<128>": {"bytes": 628199424,
                            "sources": {"bwd_kernel.cuh": "a16249a9909c16bc8d6b854ecf39824e9ae17b7a",
                                        "sm100.cuh": "765aea2ea7410d534e289cfea85ff6d2b3b159c9"}},
+    # the decode workload (B8 H64 with 8 K/V heads, N_q 1, N_k 32768): both kernels of one step
+    "fa_decode_kernel<128>+fa_decode_merge_kernel<128>": {
+        "bytes": 1083981824,
+        "sources": {"decode_kernel.cuh": "37262a272745d1c2ddd9eb7bd89f5f55d265e07b",
+                    "decode_ops.cuh": "71a63f81cb1eccd17e2d315ab066de5238a9c0a4",
+                    "sm100.cuh": "765aea2ea7410d534e289cfea85ff6d2b3b159c9"}},
 }
 
 
@@ -631,7 +637,8 @@ def run_decode(args):
                 "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json)" if peak_kind == "measured"
                 else "fallback 6.65 TB/s",
-                "algorithmic_bytes": nbytes, "traffic": None}
+                "algorithmic_bytes": nbytes,
+                "traffic": load_traffic("fa_decode_kernel<128>+fa_decode_merge_kernel<128>")}
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         f, secs, heads, cores = decode_oracle_sample(args.cpu_seconds)

@@ -3,12 +3,14 @@
 Shapes are per head ``[B, H, N, d]`` (d fastest).  Values are iid N(0, 1)
 (times ``std``) drawn in fp32 from a CPU ``torch.Generator`` and rounded to
 bf16 (round-to-nearest-even), in the order Q, K, V; the output gradient dO of
-the backward workload comes from a second seed.  The five workloads follow the
+the backward workload comes from a second seed.  The workloads follow the
 shapes the FlashAttention pages discuss: a tiny smoke case, a GPT-2-like
 sequence length (FlashAttention (NL), "Empirische resultaten": GPT-2 at 1K),
 a causal LLM shape, its backward with recomputation (memory-optimized flash
-attention page, "How it works") and a long-context sliding-window case
-(sparse-attention glossary, "Abgrenzung": sliding-window attention).
+attention page, "How it works"), long-context sliding-window cases
+(sparse-attention glossary, "Abgrenzung": sliding-window attention), shared
+K/V heads, and one generation step over a key/value cache (FlashAttention (NL),
+"Gespecialiseerde oplossingen"), where Q has Nq rows and K, V have N.
 
 Nothing in this module computes attention.
 """

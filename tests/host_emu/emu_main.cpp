@@ -1,0 +1,92 @@
+// TEST INFRASTRUCTURE ONLY: runs the decode kernels of decode_kernel.cuh on the host through
+// the SIMT emulation of emu.h, with the launch parameters fa_fwd_decode derives.
+// usage: emu_main B H Hkv Nq Nk d causal window scale  sq(3) sk(3) sv(3) so(3)  nq nk nv no  prefix
+#include "emu.h"
+#include "decode_kernel.cuh"
+
+#include <fstream>
+#include <string>
+
+using namespace fa;
+
+template <class T>
+std::vector<T> read_file(const std::string& path, size_t n) {
+  std::vector<T> v(n);
+  std::ifstream f(path, std::ios::binary);
+  f.read(reinterpret_cast<char*>(v.data()), n * sizeof(T));
+  if (!f) { std::fprintf(stderr, "short read %s\n", path.c_str()); std::exit(2); }
+  return v;
+}
+template <class T>
+void write_file(const std::string& path, const std::vector<T>& v) {
+  std::ofstream f(path, std::ios::binary);
+  f.write(reinterpret_cast<const char*>(v.data()), v.size() * sizeof(T));
+}
+
+int main(int argc, char** argv) {
+  if (argc != 1 + 9 + 12 + 4 + 1) { std::fprintf(stderr, "bad args\n"); return 2; }
+  int a = 1;
+  const int B = atoi(argv[a++]), H = atoi(argv[a++]), Hkv = atoi(argv[a++]), Nq = atoi(argv[a++]),
+            Nk = atoi(argv[a++]), d = atoi(argv[a++]), causal = atoi(argv[a++]), window = atoi(argv[a++]);
+  const float scale = float(atof(argv[a++]));
+  Strides st[4];
+  for (int i = 0; i < 4; ++i) {
+    st[i].b = atoll(argv[a++]);
+    st[i].h = atoll(argv[a++]);
+    st[i].n = atoll(argv[a++]);
+  }
+  size_t n[4];
+  for (int i = 0; i < 4; ++i) n[i] = size_t(atoll(argv[a++]));
+  const std::string prefix = argv[a++];
+  auto q = read_file<uint16_t>(prefix + ".q", n[0]);
+  auto k = read_file<uint16_t>(prefix + ".k", n[1]);
+  auto v = read_file<uint16_t>(prefix + ".v", n[2]);
+  std::vector<uint16_t> o(n[3], 0x7fc0);   // NaN: rows the kernels fail to write show up
+  std::vector<float> lse(size_t(B) * H * Nq, NAN);
+
+  const int win = window > Nk ? Nk : window;
+  const DecPlan pl = dec_plan(B, H, Hkv, Nq, Nk, d, causal, win);
+  std::vector<float> ws(pl.ws_bytes / 4 + 1, NAN);
+  DecParams p;
+  p.q = reinterpret_cast<const __nv_bfloat16*>(q.data());
+  p.k = reinterpret_cast<const __nv_bfloat16*>(k.data());
+  p.v = reinterpret_cast<const __nv_bfloat16*>(v.data());
+  p.o = reinterpret_cast<__nv_bfloat16*>(o.data());
+  p.lse = lse.data();
+  p.o_part = pl.ws_bytes ? ws.data() : nullptr;
+  p.l_part = pl.n_splits > 1 ? p.o_part + size_t(pl.n_splits) * size_t(pl.total_rows) * d : nullptr;
+  p.q_st = st[0];
+  p.k_st = st[1];
+  p.v_st = st[2];
+  p.o_st = st[3];
+  p.total_rows = pl.total_rows;
+  p.H = H;
+  p.H_kv = Hkv;
+  p.group = H / Hkv;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.rows = pl.rows;
+  p.row_blocks = pl.row_blocks;
+  p.n_splits = pl.n_splits;
+  p.chunk = pl.chunk;
+  p.key_begin = pl.key_begin;
+  p.causal = causal;
+  p.window = win;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  std::printf("plan rows=%d row_blocks=%d n_splits=%d chunk=%d key_begin=%d ctas=%lld ws=%zu\n", pl.rows,
+              pl.row_blocks, pl.n_splits, pl.chunk, pl.key_begin, pl.ctas, pl.ws_bytes);
+  if (d == 64) {
+    emu_launch(unsigned(pl.ctas), kDecThreads, DecLayout<64>::kSmemBytes, [&] { fa_decode_kernel<64>(p); });
+    if (pl.n_splits > 1)
+      emu_launch(unsigned((pl.total_rows + kDecMergeWarps - 1) / kDecMergeWarps), 32 * kDecMergeWarps, 0,
+                 [&] { fa_decode_merge_kernel<64>(p); });
+  } else {
+    emu_launch(unsigned(pl.ctas), kDecThreads, DecLayout<128>::kSmemBytes, [&] { fa_decode_kernel<128>(p); });
+    if (pl.n_splits > 1)
+      emu_launch(unsigned((pl.total_rows + kDecMergeWarps - 1) / kDecMergeWarps), 32 * kDecMergeWarps, 0,
+                 [&] { fa_decode_merge_kernel<128>(p); });
+  }
+  write_file(prefix + ".o", o);
+  write_file(prefix + ".lse", lse);
+  return 0;
+}
