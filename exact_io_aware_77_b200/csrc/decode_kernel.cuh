@@ -345,38 +345,51 @@ __global__ void __launch_bounds__(kDecThreads, 2) fa_decode_kernel(const DecPara
   }
 }
 
-// Merge the splits of every output row: one warp per row, D / 32 columns per lane.
+// Merge the splits of every output row: one warp per row, D / 32 columns per lane.  The
+// lanes first read up to 32 splits' L_s at once (lane s holds split s); the O_s loads of
+// eight splits are then in flight together, so the row costs a few memory latencies rather
+// than one per split.
 template <int D>
 __global__ void __launch_bounds__(32 * kDecMergeWarps) fa_decode_merge_kernel(const DecParams p) {
   constexpr float kLn2 = 0.6931471805599453f, kLog2e = 1.4426950408889634f;
   constexpr int C = D / 32;
   const long long grow = (long long)blockIdx.x * kDecMergeWarps + (threadIdx.x >> 5);
-  if (grow >= p.total_rows) return;
+  if (grow >= p.total_rows) return;   // whole warps leave together
   const int lane = threadIdx.x & 31;
   float mx = -INFINITY;
-  for (int s = 0; s < p.n_splits; ++s) mx = fmaxf(mx, p.l_part[(long long)s * p.total_rows + grow]);
+  for (int s0 = 0; s0 < p.n_splits; s0 += 32)
+    if (s0 + lane < p.n_splits) mx = fmaxf(mx, p.l_part[(long long)(s0 + lane) * p.total_rows + grow]);
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
   float acc[C];
 #pragma unroll
   for (int c = 0; c < C; ++c) acc[c] = 0.f;
   float sum = 0.f;
   if (mx != -INFINITY) {
-    for (int s = 0; s < p.n_splits; ++s) {
-      const long long prow = (long long)s * p.total_rows + grow;
-      const float wt = ex2_approx((p.l_part[prow] - mx) * kLog2e);
+    for (int s0 = 0; s0 < p.n_splits; s0 += 32) {
+      const int s = s0 + lane;
+      const float wt = s < p.n_splits ? ex2_approx((p.l_part[(long long)s * p.total_rows + grow] - mx) * kLog2e) : 0.f;
       sum += wt;
-      const float* src = p.o_part + prow * D + lane * C;
-      if constexpr (C == 4) {
-        const float4 x = *reinterpret_cast<const float4*>(src);
-        acc[0] += wt * x.x;
-        acc[1] += wt * x.y;
-        acc[2] += wt * x.z;
-        acc[3] += wt * x.w;
-      } else {
-        const float2 x = *reinterpret_cast<const float2*>(src);
-        acc[0] += wt * x.x;
-        acc[1] += wt * x.y;
+      const int cnt = min(32, p.n_splits - s0);
+#pragma unroll 8
+      for (int j = 0; j < cnt; ++j) {
+        const float w = __shfl_sync(0xffffffffu, wt, j);
+        const float* src = p.o_part + ((long long)(s0 + j) * p.total_rows + grow) * D + lane * C;
+        if constexpr (C == 4) {
+          const float4 x = *reinterpret_cast<const float4*>(src);
+          acc[0] += w * x.x;
+          acc[1] += w * x.y;
+          acc[2] += w * x.z;
+          acc[3] += w * x.w;
+        } else {
+          const float2 x = *reinterpret_cast<const float2*>(src);
+          acc[0] += w * x.x;
+          acc[1] += w * x.y;
+        }
       }
     }
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, m);
   }
   const float inv = sum > 0.f ? 1.f / sum : 0.f;
   const int i = int(grow % p.Nq);

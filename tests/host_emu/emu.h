@@ -59,6 +59,17 @@ inline float __shfl_xor_sync(unsigned, float v, int m) {
   return r;
 }
 
+inline float __shfl_sync(unsigned, float v, int src) {
+  WarpCtx& w = my_warp();
+  int l = lane_id();
+  std::memcpy(&w.xch[l][0], &v, 4);
+  w.bar->arrive_and_wait();
+  float r;
+  std::memcpy(&r, &w.xch[src & 31][0], 4);
+  w.bar->arrive_and_wait();
+  return r;
+}
+
 template <class F>
 void emu_launch(unsigned grid, unsigned block, size_t smem_bytes, F call) {
   for (unsigned bx = 0; bx < grid; ++bx) {

@@ -94,6 +94,7 @@ CASES = [
     (1, 2, 2, 37, 37, 128, False, 5),
     (1, 3, 3, 2, 40, 64, True, 1000),
     (1, 2, 2, 64, 4096, 128, True, 300),    # splits that some rows see no key of
+    (1, 2, 1, 1, 8192, 64, True, 0),        # 64 splits: the merge reads them 32 at a time
 ]
 
 
