@@ -45,6 +45,28 @@ def _check_qkv(q, k, v, *rest):
     return int(k.shape[1])
 
 
+def _check_like(t, ref, what: str) -> None:
+    """t must be a bf16 tensor shaped like ref, on ref's device, with contiguous d."""
+    import torch
+    if not (t.dtype == torch.bfloat16 and t.shape == ref.shape and t.dim() == 4 and t.stride(-1) == 1
+            and t.device == ref.device):
+        raise ValueError(f"{what} must be a bf16 tensor shaped like {tuple(ref.shape)} on {ref.device} "
+                         "with contiguous d")
+
+
+def _check_lse(lse, ref, rows: int) -> None:
+    import torch
+    if not (lse.dtype == torch.float32 and lse.is_contiguous() and lse.numel() == rows and lse.device == ref.device):
+        raise ValueError(f"lse must be a contiguous fp32 tensor of {rows} elements on {ref.device}")
+
+
+def _check_workspace(ws, ref) -> None:
+    """Caller scratch must be a contiguous tensor on ref's device; its size and alignment are
+    the library's to check (FA_ERR_WORKSPACE, FA_ERR_ALIGN)."""
+    if not (ws.device == ref.device and ws.is_contiguous()):
+        raise ValueError(f"workspace must be a contiguous tensor on {ref.device}")
+
+
 def _raise(name, st):
     if st != _lib.FA_OK:
         raise FAError(name, st)
@@ -61,6 +83,8 @@ def forward(q, k, v, scale: float | None = None, causal: bool = False, window: i
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    _check_like(out, q, "out")
+    _check_lse(lse, q, B * H * N)
     ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr())
     mask = (scale, int(bool(causal)), int(window), _stream_handle(q.device))
     if not all(t.is_contiguous() for t in (q, k, v, out)):
@@ -91,17 +115,16 @@ def backward(q, k, v, o, lse, do, scale: float | None = None, causal: bool = Fal
     import torch
     H_kv = _check_qkv(q, k, v, o, do)
     B, H, N, d = q.shape
-    if not (lse.is_cuda and lse.dtype == torch.float32 and lse.is_contiguous() and lse.numel() == B * H * N):
-        raise ValueError("lse must be a contiguous fp32 CUDA tensor of B*H*N elements")
+    _check_lse(lse, q, B * H * N)
     scale = default_scale(d) if scale is None else float(scale)
     if grads is None:
         grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
-    for g, t in zip(grads, (q, k, v)):
-        if g.shape != t.shape or g.stride(-1) != 1 or g.dtype != torch.bfloat16 or g.device != q.device:
-            raise ValueError("grads must be bf16 CUDA tensors shaped like q, k, v with contiguous d")
+    for g, t, name in zip(grads, (q, k, v), ("dq", "dk", "dv")):
+        _check_like(g, t, name)
     need = bwd_workspace_size(B, H, N, d)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _check_workspace(workspace, q)
     dq, dk, dv = grads
     ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
             dq.data_ptr(), dk.data_ptr(), dv.data_ptr())
@@ -157,12 +180,12 @@ def decode(q, k, v, scale: float | None = None, causal: bool = False, window: in
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, N_q), dtype=torch.float32, device=q.device)
-    if out.shape != q.shape or out.stride(-1) != 1 or out.dtype != torch.bfloat16 or out.device != q.device:
-        raise ValueError("out must be a bf16 tensor shaped like q with contiguous d")
-    if not (lse.dtype == torch.float32 and lse.is_contiguous() and lse.numel() == B * H * N_q and lse.device == q.device):
-        raise ValueError("lse must be a contiguous fp32 tensor of B*H*N_q elements")
+    _check_like(out, q, "out")
+    _check_lse(lse, q, B * H * N_q)
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if workspace is not None:
+        _check_workspace(workspace, q)
     ws_ptr = workspace.data_ptr() if workspace is not None else 0
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     st = None
