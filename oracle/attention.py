@@ -53,6 +53,13 @@ query row i stands at position N_k - N_q + i of the key sequence (the new rows a
 the last N_q positions, after the cached ones), so the causal and window masks
 above apply to that position.  With N_q = N_k this is the self-attention above.
 
+FP8 keys and values.  The pages say that FlashAttention-3 supports FP8 (FlashAttention (NL),
+"Evolutie en verdere ontwikkelingen", FlashAttention-3), without a format.  Reading: the
+E4M3 format of that paper's FP8 path -- 1 sign bit, 4 exponent bits with bias 7, 3 mantissa
+bits, exponent field 0 for subnormals, no infinities, S.1111.111 the only NaN -- with one
+scale per tensor: K = s_k * E4M3(K8), V = s_v * E4M3(V8).  The attention is then the
+definition above on those dequantised values, in fp64.
+
 Arithmetic is numpy float64 with ``@`` (BLAS DGEMM) as the only library step.
 Parity of every function here is pinned by tests/test_oracle.py.
 """
@@ -73,6 +80,8 @@ __all__ = [
     "attention_forward_shared_kv",
     "attention_backward_shared_kv",
     "attention_forward_decode",
+    "e4m3_to_float",
+    "attention_forward_decode_fp8kv",
 ]
 
 
@@ -288,6 +297,29 @@ def attention_forward_decode(q, k, v, scale: float, causal: bool = False, window
     start = _decode_row_start(n_q, n_k)
     return _per_head(lambda a, b, c: _head_forward(a, b, c, scale, causal, window, start)[:2],
                      q, k[..., idx, :, :], v[..., idx, :, :])
+
+
+def e4m3_to_float(codes) -> np.ndarray:
+    """fp64 values of FP8 E4M3 codes (uint8): (-1)^s 2^(e-7) (1 + m/8) for exponent fields
+    e = 1..15, (-1)^s 2^-6 (m/8) for e = 0, NaN for e = 15 with m = 7."""
+    c = np.asarray(codes).astype(np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, (m / 8.0) * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    mag = np.where((e == 15) & (c & 0x7 == 7), np.nan, mag)
+    return sign * mag
+
+
+def attention_forward_decode_fp8kv(q, k8, v8, k_scale: float, v_scale: float, scale: float,
+                                   causal: bool = False, window: int = 0):
+    """attention_forward_decode with K = k_scale E4M3(k8) and V = v_scale E4M3(v8): q [..., H, N_q, d];
+    k8, v8 uint8 codes [..., H_kv, N_k, d]."""
+    if hasattr(k8, "detach"):
+        k8, v8 = (x.detach().cpu().numpy() for x in (k8, v8))
+    k = float(k_scale) * e4m3_to_float(k8)
+    v = float(v_scale) * e4m3_to_float(v8)
+    return attention_forward_decode(q, k, v, scale, causal, window)
 
 
 def allowed_pairs(n: int, causal: bool, window: int) -> int:

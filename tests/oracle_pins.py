@@ -455,6 +455,47 @@ def decode_last_rows_of_self_attention(orc):
             assert np.max(np.abs(lse[:, 0] - l_full[:, -n_q:])) < 1e-12
 
 
+def e4m3_decoding(orc):
+    """Every one of the 256 E4M3 codes decodes as torch's float8_e4m3fn does, and hand-worked
+    codes give their values: 0x38 = 1, 0x3C = 1.5, 0xB8 = -1, 0x7E = 448 (largest), 0x08 = 2^-6
+    (smallest normal), 0x07 = 7 * 2^-9, 0x01 = 2^-9 (smallest subnormal), 0x80 = -0, 0x7F NaN."""
+    import torch
+    codes = np.arange(256, dtype=np.uint8)
+    mine = orc.e4m3_to_float(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(mine), nan) and nan.sum() == 2
+    assert np.array_equal(mine[~nan], ref[~nan])
+    worked = {0x38: 1.0, 0x3C: 1.5, 0xB8: -1.0, 0x7E: 448.0, 0x08: 2.0 ** -6, 0x07: 7 * 2.0 ** -9,
+              0x01: 2.0 ** -9, 0x00: 0.0}
+    for code, val in worked.items():
+        assert orc.e4m3_to_float(np.array([code], dtype=np.uint8))[0] == val, hex(code)
+    neg0 = orc.e4m3_to_float(np.array([0x80], dtype=np.uint8))[0]
+    assert neg0 == 0.0 and math.copysign(1.0, neg0) < 0
+    assert np.isnan(orc.e4m3_to_float(np.array([0x7F, 0xFF], dtype=np.uint8))).all()
+
+
+def fp8kv_decode(orc):
+    """The FP8 K/V forward equals the plain decode forward on K and V dequantised by torch
+    (float8_e4m3fn times the scale); doubling s_k while halving the softmax scale changes
+    nothing; O is linear in s_v and L does not depend on it."""
+    import torch
+    r = _rng(34)
+    q = r.standard_normal((2, 4, 3, 8))
+    k8, v8 = (r.integers(0, 256, size=(2, 2, 20, 8)).astype(np.uint8) for _ in range(2))
+    for a in (k8, v8):   # no NaN codes in the cache
+        a[(a & 0x7F) == 0x7F] = 0x38
+    dq = lambda c: torch.from_numpy(c).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    for causal, window in MASKS:
+        o, lse = orc.attention_forward_decode_fp8kv(q, k8, v8, 0.05, 0.7, 0.3, causal, window)
+        o_ref, l_ref = orc.attention_forward_decode(q, 0.05 * dq(k8), 0.7 * dq(v8), 0.3, causal, window)
+        assert np.max(np.abs(o - o_ref)) < 1e-12 and np.max(np.abs(lse - l_ref)) < 1e-12
+        o2, l2 = orc.attention_forward_decode_fp8kv(q, k8, v8, 0.1, 0.7, 0.15, causal, window)
+        assert np.max(np.abs(o2 - o)) < 1e-12 and np.max(np.abs(l2 - lse)) < 1e-12
+        o3, l3 = orc.attention_forward_decode_fp8kv(q, k8, v8, 0.05, 1.4, 0.3, causal, window)
+        assert np.max(np.abs(o3 - 2 * o)) < 1e-12 and np.max(np.abs(l3 - lse)) < 1e-12
+
+
 def rejects_bad_masks(orc):
     """A negative window is rejected, with or without causal."""
     q, k, v = _qkv(21, n=4, d=2, lead=())
@@ -472,5 +513,5 @@ PINS = {f.__name__: f for f in (
     large_scores, golden_examples, library_forward, library_backward, finite_differences,
     delta_identity, row_blocks_match, pair_count, two_sided_window, shared_kv_library,
     shared_kv_finite_differences, decode_library, decode_scale_zero, decode_last_rows_of_self_attention,
-    rejects_bad_masks,
+    e4m3_decoding, fp8kv_decode, rejects_bad_masks,
 )}

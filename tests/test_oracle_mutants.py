@@ -128,7 +128,33 @@ def _backward_shared_kv_first_only(q, k, v, do, scale, causal=False, window=0):
     return dq, dk[..., ::g, :, :], dv[..., ::g, :, :]
 
 
+def _e4m3_bias_8(codes):
+    c = np.asarray(codes).astype(np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, (m / 8.0) * 2.0 ** -7, (1.0 + m / 8.0) * np.exp2(e - 8.0))
+    return sign * np.where((e == 15) & (c & 0x7 == 7), np.nan, mag)
+
+
+def _e4m3_no_subnormals(codes):
+    c = np.asarray(codes).astype(np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = (1.0 + m / 8.0) * np.exp2(e - 7.0)
+    return sign * np.where((e == 15) & (c & 0x7 == 7), np.nan, mag)
+
+
+def _fp8kv_v_scale_dropped(q, k8, v8, k_scale, v_scale, scale, causal=False, window=0):
+    return orc.attention_forward_decode(q, k_scale * orc.e4m3_to_float(k8), orc.e4m3_to_float(v8), scale, causal,
+                                        window)
+
+
 MUTANTS = {
+    "e4m3_bias_8": ("e4m3_to_float", _e4m3_bias_8),
+    "e4m3_no_subnormals": ("e4m3_to_float", _e4m3_no_subnormals),
+    "fp8kv_v_scale_dropped": ("attention_forward_decode_fp8kv", _fp8kv_v_scale_dropped),
     "decode_rows_first": ("_decode_row_start", lambda n_q, n_k: 0),
     "decode_rows_one_early": ("_decode_row_start", lambda n_q, n_k: max(0, n_k - n_q - 1)),
     "scores_transposed": ("_scores", _scores_transposed),
