@@ -41,7 +41,7 @@ WORKLOAD = "causal"          # forward workload; the backward uses the same shap
 GRAD_WORKLOAD = "bwd"
 # --workload choices: the forward workload and the one whose dO seed the backward uses
 BENCH_WORKLOADS = {"causal": ("causal", "bwd"), "long": ("long", "long"), "swa": ("swa", "swa"),
-                   "gqa": ("gqa", "gqa"), "decode": ("decode", "decode")}
+                   "gqa": ("gqa", "gqa"), "decode": ("decode", "decode"), "decode_fp8": ("decode", "decode")}
 FLUSH_BYTES = 256 << 20      # > 126 MB L2
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -61,7 +61,8 @@ def parse_args():
                     help="causal: B2 H32 N4096 d128 (the default line); gqa: the same with 8 K/V heads; "
                          "long / swa: N32768 with a one- / two-sided window of 4096, FLOPs counted over "
                          "the pairs the band keeps; decode: one new row per query head over 32768 "
-                         "cached keys (B8, 64 query heads on 8 K/V heads), forward only, HBM-bound")
+                         "cached keys (B8, 64 query heads on 8 K/V heads), forward only, HBM-bound; "
+                         "decode_fp8: the same over an E4M3 K/V cache with per-tensor scales")
     return ap.parse_args()
 
 
@@ -112,13 +113,14 @@ def decode_flops(B, H, n_q, n_k, d, causal, window=0) -> float:
     return 4.0 * B * H * d * decode_pairs(n_q, n_k, causal, window)
 
 
-def decode_bytes(B, H, H_kv, n_q, n_k, d, causal, window=0) -> int:
+def decode_bytes(B, H, H_kv, n_q, n_k, d, causal, window=0, kv_elem_bytes=2) -> int:
     """Algorithmic HBM bytes of a decode forward: read Q (bf16) and, once, the K and V rows
-    of the keys any new row may attend; write O (bf16) and L (fp32)."""
+    of the keys any new row may attend (kv_elem_bytes each: 2 for bf16, 1 for E4M3); write O
+    (bf16) and L (fp32)."""
     lo, _ = decode_band(n_k - n_q, n_k, causal, window)
     _, hi = decode_band(n_k - 1, n_k, causal, window)
     keys = hi - lo + 1
-    return 2 * B * H * n_q * d * 2 + 2 * B * H_kv * keys * d * 2 + B * H * n_q * 4
+    return 2 * B * H * n_q * d * 2 + 2 * B * H_kv * keys * d * kv_elem_bytes + B * H * n_q * 4
 
 
 def max_over_ranks(values, device=None):
@@ -480,7 +482,7 @@ NCU_TRAFFIC = {
                            "sources": {"bwd_kernel.cuh": "a16249a9909c16bc8d6b854ecf39824e9ae17b7a",
                                        "sm100.cuh": "765aea2ea7410d534e289cfea85ff6d2b3b159c9"}},
     # the decode workload (B8 H64 with 8 K/V heads, N_q 1, N_k 32768): both kernels of one step
-    "fa_decode_kernel<128>+fa_decode_merge_kernel<128>": {
+    "fa_decode_kernel<128,false>+fa_decode_merge_kernel<128>": {
         "bytes": 1083981824,
         "sources": {"decode_kernel.cuh": "37262a272745d1c2ddd9eb7bd89f5f55d265e07b",
                     "decode_ops.cuh": "71a63f81cb1eccd17e2d315ab066de5238a9c0a4",
@@ -508,23 +510,31 @@ def load_traffic(kernel: str):
 _INPUT_CACHE = {}
 
 
-def decode_oracle_sample(seconds: float, max_heads: int | None = None):
+def decode_oracle_sample(seconds: float, max_heads: int | None = None, fp8: bool = False):
     """Time the fp64 oracle's decode forward head by head (batch entry 0) on the decode
-    workload.  Returns (flops credited, seconds, heads, cores)."""
+    workload (fp8: over its E4M3 K/V cache).  Returns (flops credited, seconds, heads, cores)."""
     from oracle import attention as orc
-    from synthetic import WORKLOADS, make_inputs
+    from synthetic import WORKLOADS, make_inputs, make_inputs_fp8kv
     wl = WORKLOADS["decode"]
-    if "decode" not in _INPUT_CACHE:
-        _INPUT_CACHE["decode"] = make_inputs(wl)
-    q, k, v = _INPUT_CACHE["decode"]
+    key = "decode_fp8" if fp8 else "decode"
+    if key not in _INPUT_CACHE:
+        _INPUT_CACHE[key] = make_inputs_fp8kv(wl) if fp8 else make_inputs(wl)
+    if fp8:
+        q, k8, v8, s_k, s_v = _INPUT_CACHE[key]
+    else:
+        q, k, v = _INPUT_CACHE[key]
     g = wl.H // wl.kv_heads
     per_head = decode_flops(1, 1, wl.q_rows, wl.N, wl.d, wl.causal, wl.window)
     t0 = time.perf_counter()
     heads = 0
     while True:
         h = heads % wl.H
-        orc.attention_forward_decode(q[0:1, h:h + 1], k[0:1, h // g:h // g + 1], v[0:1, h // g:h // g + 1],
-                                     wl.scale, wl.causal, wl.window)
+        kv = slice(h // g, h // g + 1)
+        if fp8:
+            orc.attention_forward_decode_fp8kv(q[0:1, h:h + 1], k8[0:1, kv], v8[0:1, kv], s_k, s_v, wl.scale,
+                                               wl.causal, wl.window)
+        else:
+            orc.attention_forward_decode(q[0:1, h:h + 1], k[0:1, kv], v[0:1, kv], wl.scale, wl.causal, wl.window)
         heads += 1
         el = time.perf_counter() - t0
         if el >= seconds or (max_heads is not None and heads >= max_heads):
@@ -532,13 +542,14 @@ def decode_oracle_sample(seconds: float, max_heads: int | None = None):
     return per_head * heads, el, heads, blas_threads()
 
 
-def decode_workload_text(wl) -> str:
+def decode_workload_text(wl, fp8: bool = False) -> str:
+    kv = ("K and V as E4M3 codes with per-tensor scales (max|x|/448)" if fp8 else "bf16")
     return (f"decode forward: B={wl.B} H={wl.H} (K/V heads {wl.kv_heads}) N_q={wl.q_rows} new row(s) at "
             f"the last positions of N_k={wl.N} keys, d={wl.d} {'causal' if wl.causal else 'no mask'}"
-            f"{f' window {wl.window}' if wl.window else ''}, inputs N(0,1)*{wl.std:g} bf16 seeded")
+            f"{f' window {wl.window}' if wl.window else ''}, inputs N(0,1)*{wl.std:g} bf16 seeded, K/V {kv}")
 
 
-def run_decode(args):
+def run_decode(args, fp8: bool = False):
     import torch
     import torch.distributed as dist
 
@@ -552,10 +563,14 @@ def run_decode(args):
 
     import exact_io_aware_77_b200 as fa
     fa.load()
-    from synthetic import WORKLOADS, make_inputs
+    from synthetic import WORKLOADS, make_inputs, make_inputs_fp8kv
     wl = WORKLOADS["decode"]
     B, H, Hkv, Nq, Nk, d = wl.B, wl.H, wl.kv_heads, wl.q_rows, wl.N, wl.d
-    q_h, k_h, v_h = make_inputs(wl)
+    s_k = s_v = 1.0
+    if fp8:
+        q_h, k_h, v_h, s_k, s_v = make_inputs_fp8kv(wl)
+    else:
+        q_h, k_h, v_h = make_inputs(wl)
     q, k, v = (x.to(dev) for x in (q_h, k_h, v_h))
     o = torch.empty_like(q)
     lse = torch.empty((B, H, Nq), dtype=torch.float32, device=dev)
@@ -563,13 +578,19 @@ def run_decode(args):
     ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
     launches = 2 if need else 1                  # split kernel, then the split merge
     flops = decode_flops(B, H, Nq, Nk, d, wl.causal, wl.window)
-    nbytes = decode_bytes(B, H, Hkv, Nq, Nk, d, wl.causal, wl.window)
+    nbytes = decode_bytes(B, H, Hkv, Nq, Nk, d, wl.causal, wl.window, kv_elem_bytes=1 if fp8 else 2)
     stream = torch.cuda.current_stream(dev)
+
+    def run(qq, kk, vv):
+        if fp8:
+            fa.decode_fp8kv(qq, kk, vv, s_k, s_v, wl.scale, wl.causal, wl.window, out=o, lse=lse, workspace=ws)
+        else:
+            fa.decode(qq, kk, vv, wl.scale, wl.causal, wl.window, out=o, lse=lse, workspace=ws)
 
     def step(ev=None):
         if ev:
             ev[0].record(stream)
-        fa.decode(q, k, v, wl.scale, wl.causal, wl.window, out=o, lse=lse, workspace=ws)
+        run(q, k, v)
         if ev:
             ev[1].record(stream)
 
@@ -587,7 +608,7 @@ def run_decode(args):
     torch.cuda.synchronize(dev)
     wall0 = time.time()
     for i in range(args.steps):
-        step(events[i])                           # K and V (1.07 GB) exceed L2: no flush needed
+        step(events[i])                           # K and V (1.07 GB, or 0.54 GB as E4M3) exceed L2
     torch.cuda.synchronize(dev)
     wall1 = time.time()
     if world > 1:
@@ -612,7 +633,7 @@ def run_decode(args):
         def one():
             for dst, src in zip((qe, ke, ve), pin):
                 dst.copy_(src, non_blocking=True)
-            fa.decode(qe, ke, ve, wl.scale, wl.causal, wl.window, out=o, lse=lse, workspace=ws)
+            run(qe, ke, ve)
             o_h.copy_(o, non_blocking=True)
             l_h.copy_(lse, non_blocking=True)
 
@@ -632,16 +653,17 @@ def run_decode(args):
 
     peaks, peak_kind = load_peaks()
     achieved = nbytes / (ms * 1e-3) / 1e9
-    roofline = {"bound": "hbm", "kernel": "fa_decode_kernel<128>+fa_decode_merge_kernel<128>",
+    roofline_kernel = f"fa_decode_kernel<128,{'true' if fp8 else 'false'}>+fa_decode_merge_kernel<128>"
+    roofline = {"bound": "hbm", "kernel": roofline_kernel,
                 "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json)" if peak_kind == "measured"
                 else "fallback 6.65 TB/s",
                 "algorithmic_bytes": nbytes,
-                "traffic": load_traffic("fa_decode_kernel<128>+fa_decode_merge_kernel<128>")}
+                "traffic": load_traffic(roofline_kernel)}
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        f, secs, heads, cores = decode_oracle_sample(args.cpu_seconds)
+        f, secs, heads, cores = decode_oracle_sample(args.cpu_seconds, fp8=fp8)
         cpu = {"value": round(f / secs / 1e12, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                "sample": f"{heads} query heads (batch entry 0) of the decode workload through the fp64 "
                          f"oracle, {secs:.1f} s, credited each head's FLOPs"}
@@ -650,9 +672,9 @@ def run_decode(args):
         "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": decode_workload_text(wl), "global_batch": B * world, "seq_len": Nk,
+        "config": {"workload": decode_workload_text(wl, fp8), "global_batch": B * world, "seq_len": Nk,
                    "parallelism": f"replicas{world}",
-                   "l2": "not flushed: the K and V read each step (1.07 GB) exceed the 126 MB L2"},
+                   "l2": "not flushed: the K and V read each step (1.07 GB bf16, 0.54 GB E4M3) exceed the 126 MB L2"},
         "hbm_gbs": round(achieved, 1),
         "roofline": roofline,
         "cpu_baseline": cpu,
@@ -675,7 +697,7 @@ def run_reference(args):
     from synthetic import WORKLOADS
     wl = WORKLOADS[WORKLOAD]
     if WORKLOAD == "decode":
-        return run_decode_reference(args, wl)
+        return run_decode_reference(args, wl, fp8=args.workload == "decode_fp8")
     import exact_io_aware_77_b200 as fa_pkg   # only to learn whether the path has a backward
     with_bwd = hasattr(fa_pkg, "backward")
     times, flops = [], []
@@ -704,11 +726,11 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
-def run_decode_reference(args, wl):
+def run_decode_reference(args, wl, fp8: bool = False):
     times, flops = [], []
     cores = blas_threads()
     for i in range(args.warmup + args.steps):
-        f, secs, _, cores = decode_oracle_sample(0.0, max_heads=1)
+        f, secs, _, cores = decode_oracle_sample(0.0, max_heads=1, fp8=fp8)
         if i >= args.warmup:
             times.append(secs)
             flops.append(f)
@@ -720,7 +742,7 @@ def run_decode_reference(args, wl):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * secs / args.steps, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "impl": "reference",
-        "config": {"workload": decode_workload_text(wl) + " (one-head sample per step)",
+        "config": {"workload": decode_workload_text(wl, fp8) + " (one-head sample per step)",
                    "global_batch": wl.B, "seq_len": wl.N, "parallelism": "cpu"},
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                          "sample": "each step: query head 0 of batch entry 0 of the decode workload through "
@@ -749,7 +771,7 @@ def main():
     if args.impl == "reference":
         run_reference(args)
     elif WORKLOAD == "decode":
-        run_decode(args)
+        run_decode(args, fp8=args.workload == "decode_fp8")
     else:
         run_ours(args)
 

@@ -15,7 +15,7 @@ import math
 from . import _lib
 from ._lib import FAError, STATUS, STATUS_NAMES, load
 
-__all__ = ["forward", "backward", "decode", "decode_workspace_size", "bwd_workspace_size", "check_status", "FAError", "STATUS", "STATUS_NAMES", "load", "default_scale"]
+__all__ = ["forward", "backward", "decode", "decode_fp8kv", "decode_workspace_size", "bwd_workspace_size", "check_status", "FAError", "STATUS", "STATUS_NAMES", "load", "default_scale"]
 
 
 def default_scale(d: int) -> float:
@@ -195,6 +195,48 @@ def decode(q, k, v, scale: float | None = None, causal: bool = False, window: in
         q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, H, H_kv, N_q, N_k, d,
         ctypes.addressof(st) if st is not None else 0, scale, int(bool(causal)), int(window), ws_ptr, ws_bytes,
         _stream_handle(q.device)))
+    return out, lse
+
+
+def decode_fp8kv(q, k8, v8, k_scale: float, v_scale: float, scale: float | None = None, causal: bool = False,
+                 window: int = 0, out=None, lse=None, workspace=None):
+    """decode() over an FP8 key/value cache: K = k_scale * E4M3(k8), V = v_scale * E4M3(v8).
+
+    k8, v8: [B, H_kv, N_k, d] E4M3 codes (torch.uint8 or torch.float8_e4m3fn), strides in
+    multiples of 16 elements; q bf16 [B, H, N_q, d].  Returns O bf16 and L fp32 as decode().
+    """
+    import torch
+    k8, v8 = (x.view(torch.uint8) if x.dtype == torch.float8_e4m3fn else x for x in (k8, v8))
+    if not (q.is_cuda and q.dtype == torch.bfloat16 and q.dim() == 4 and q.stride(-1) == 1):
+        raise ValueError("q must be a bf16 CUDA tensor [B, H, N_q, d] with contiguous d")
+    for t in (k8, v8):
+        if not (t.dtype == torch.uint8 and t.dim() == 4 and t.stride(-1) == 1 and t.device == q.device):
+            raise ValueError("k8 and v8 must be E4M3 code tensors [B, H_kv, N_k, d] on q's device, d contiguous")
+    B, H, N_q, d = q.shape
+    if k8.shape != v8.shape or k8.shape[0] != B or k8.shape[3] != d:
+        raise ValueError("k8 and v8 must be [B, H_kv, N_k, d]")
+    H_kv, N_k = int(k8.shape[1]), int(k8.shape[2])
+    scale = default_scale(d) if scale is None else float(scale)
+    need = decode_workspace_size(B, H, H_kv, N_q, N_k, d, causal, window)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N_q), dtype=torch.float32, device=q.device)
+    _check_like(out, q, "out")
+    _check_lse(lse, q, B * H * N_q)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if workspace is not None:
+        _check_workspace(workspace, q)
+    ws_ptr = workspace.data_ptr() if workspace is not None else 0
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = None
+    if not all(t.is_contiguous() for t in (q, k8, v8, out)):
+        st = _lib.strides_array((q, k8, v8, out))
+    _raise("fa_fwd_decode_fp8kv", _lib.fa_fwd_decode_fp8kv(
+        q.data_ptr(), k8.data_ptr(), v8.data_ptr(), float(k_scale), float(v_scale), out.data_ptr(), lse.data_ptr(),
+        B, H, H_kv, N_q, N_k, d, ctypes.addressof(st) if st is not None else 0, scale, int(bool(causal)),
+        int(window), ws_ptr, ws_bytes, _stream_handle(q.device)))
     return out, lse
 
 

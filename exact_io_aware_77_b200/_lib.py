@@ -44,6 +44,8 @@ SIGNATURES = {
     "fa_decode_workspace_size": (_c_size_t, [_c_int] * 8),
     "fa_fwd_decode": (_c_int, [_c_void_p] * 5 + [_c_int] * 6 + [_c_void_p, _c_float, _c_int, _c_int, _c_void_p,
                                                                 _c_size_t, _c_void_p]),
+    "fa_fwd_decode_fp8kv": (_c_int, [_c_void_p] * 3 + [_c_float, _c_float] + [_c_void_p] * 2 + [_c_int] * 6 +
+                            [_c_void_p, _c_float, _c_int, _c_int, _c_void_p, _c_size_t, _c_void_p]),
     "fa_status_string": (ctypes.c_char_p, [_c_int]),
     "fa_check_status": (_c_int, [_c_void_p]),
     "fa_set_wait_limit_ns": (None, [_c_ull]),
@@ -164,6 +166,13 @@ def fa_fwd_decode(q, k, v, o, lse, B, H, H_kv, N_q, N_k, d, strides, scale, caus
     """Forward of N_q new query rows (the last N_q key positions) over N_k keys."""
     return _call("fa_fwd_decode", q, k, v, o, lse, B, H, H_kv, N_q, N_k, d, strides, scale, causal, window,
                  workspace, workspace_bytes, stream)
+
+
+def fa_fwd_decode_fp8kv(q, k8, v8, k_scale, v_scale, o, lse, B, H, H_kv, N_q, N_k, d, strides, scale, causal,
+                        window, workspace, workspace_bytes, stream) -> int:
+    """fa_fwd_decode over E4M3 K/V codes with per-tensor scales."""
+    return _call("fa_fwd_decode_fp8kv", q, k8, v8, k_scale, v_scale, o, lse, B, H, H_kv, N_q, N_k, d, strides, scale,
+                 causal, window, workspace, workspace_bytes, stream)
 
 
 def fa_status_string(status: int) -> str:

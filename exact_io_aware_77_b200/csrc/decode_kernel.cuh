@@ -12,6 +12,12 @@
 //   L = M + ln sum_s exp(L_s - M),  O = sum_s exp(L_s - L) O_s   (M = max_s L_s).
 // Every split's O_s is already normalised by its own l; a split with no allowed key has
 // L_s = -inf and weight 0.  The work is bound by reading K and V from HBM once.
+//
+// With an FP8 K/V cache (kFp8) K and V arrive as E4M3 codes with one scale per tensor
+// (K = s_k K8, V = s_v V8).  The ring then holds the raw codes; before each step the warp
+// converts its 16 keys to f16 (exactly: every E4M3 value is an f16 value) into one tile laid
+// out as the bf16 stages are, and the MMAs run on f16 operands (Q rounded to f16, clamped to
+// its finite range).  s_k is folded into the softmax scale and s_v into the final division.
 #pragma once
 
 #include <climits>
@@ -30,14 +36,18 @@ constexpr int kDecMergeWarps = 8;   // warps (one output row each) per CTA of th
 constexpr int kDecSlots = 148 * 2;  // CTAs resident at once on a B200 (148 SMs, two CTAs each)
 constexpr int kDecCtaOverheadKeys = 128;   // a CTA's fixed cost (Q load, ring fill, merge), in keys
 
-template <int D>
+template <int D, bool kFp8 = false>
 struct DecLayout {
-  // one K or V row in shared memory, padded by 16 bytes so that the eight rows an 8x8
-  // matrix load reads start in eight different 16-byte bank groups
+  // one K or V row (16-bit values) in shared memory, padded by 16 bytes so that the eight rows
+  // an 8x8 matrix load reads start in eight different 16-byte bank groups
   static constexpr int kRowBytes = 2 * D + 16;
   static constexpr int kTileBytes = kDecKeys * kRowBytes;
-  static constexpr int kStageBytes = 2 * kTileBytes;   // K rows, then V rows
-  static constexpr int kWarpBytes = kDecStages * kStageBytes;
+  // bf16: the ring stages are the tiles the MMAs read.  FP8: the stages hold the raw E4M3
+  // rows (D bytes each), and one converted f16 K, V tile pair follows the ring.
+  static constexpr int kRawTileBytes = kDecKeys * D;
+  static constexpr int kStageBytes = kFp8 ? 2 * kRawTileBytes : 2 * kTileBytes;   // K rows, then V rows
+  static constexpr int kConvBytes = kFp8 ? 2 * kTileBytes : 0;
+  static constexpr int kWarpBytes = kDecStages * kStageBytes + kConvBytes;
   static constexpr int kRingBytes = kDecWarps * kWarpBytes;
   // after the key loop the rings hold each warp's O [16][D], m [16] and l [16] (fp32)
   static constexpr int kMergeFloats = kDecRows * D + 2 * kDecRows;
@@ -49,6 +59,9 @@ struct DecParams {
   const __nv_bfloat16* q;   // [B, H, N_q, d]
   const __nv_bfloat16* k;   // [B, H_kv, N_k, d]
   const __nv_bfloat16* v;
+  const unsigned char* k8;  // FP8 K/V cache: E4M3 codes [B, H_kv, N_k, d] (else unused)
+  const unsigned char* v8;
+  float v_scale;            // FP8: s_v (s_k is in scale_log2)
   __nv_bfloat16* o;         // [B, H, N_q, d]
   float* lse;               // [B, H, N_q] contiguous
   float* o_part;            // [n_splits][total_rows][d]; only when n_splits > 1
@@ -123,9 +136,25 @@ inline DecPlan dec_plan(int B, int H, int H_kv, int Nq, int Nk, int d, int causa
   return pl;
 }
 
-template <int D>
+// The MMA and the P packing in the operand type: bf16, or f16 for the FP8 K/V path.
+template <bool kF16>
+__device__ __forceinline__ void dec_mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  if constexpr (kF16)
+    mma_16816_f16(d, a, b0, b1);
+  else
+    mma_16816(d, a, b0, b1);
+}
+template <bool kF16>
+__device__ __forceinline__ uint32_t dec_pack(float lo, float hi) {
+  if constexpr (kF16)
+    return pack_f16x2(lo, hi);
+  else
+    return pack_bf16x2(lo, hi);
+}
+
+template <int D, bool kFp8>
 __global__ void __launch_bounds__(kDecThreads, 2) fa_decode_kernel(const DecParams p) {
-  using Lay = DecLayout<D>;
+  using Lay = DecLayout<D, kFp8>;
   constexpr int KS = D / 16;   // k-steps of S = Q K^T
   constexpr int NT = D / 8;    // 8-column n-tiles of O
   constexpr float kLn2 = 0.6931471805599453f;
@@ -171,14 +200,22 @@ __global__ void __launch_bounds__(kDecThreads, 2) fa_decode_kernel(const DecPara
     }
   }
   // Q as the A operand of every k-step: rows g, g + 8; columns 2t, 2t + 1 (+ 8)
+  auto qword = [&](const __nv_bfloat16* row, int c) -> uint32_t {
+    if (!row) return 0u;
+    const uint32_t w = ld_global_u32(row + c);
+    if constexpr (kFp8)
+      return bf16x2_to_f16x2_sat(w);
+    else
+      return w;
+  };
   uint32_t qa[KS][4];
 #pragma unroll
   for (int kk = 0; kk < KS; ++kk) {
     const int c = 16 * kk + 2 * t;
-    qa[kk][0] = qrow[0] ? ld_global_u32(qrow[0] + c) : 0u;
-    qa[kk][1] = qrow[1] ? ld_global_u32(qrow[1] + c) : 0u;
-    qa[kk][2] = qrow[0] ? ld_global_u32(qrow[0] + c + 8) : 0u;
-    qa[kk][3] = qrow[1] ? ld_global_u32(qrow[1] + c + 8) : 0u;
+    qa[kk][0] = qword(qrow[0], c);
+    qa[kk][1] = qword(qrow[1], c);
+    qa[kk][2] = qword(qrow[0], c + 8);
+    qa[kk][3] = qword(qrow[1], c + 8);
   }
 
   // this CTA's keys, in 16-key steps dealt round-robin to the warps
@@ -193,17 +230,33 @@ __global__ void __launch_bounds__(kDecThreads, 2) fa_decode_kernel(const DecPara
   auto issue = [&](int it) {
     const int key0 = s0 + kDecKeys * (warp + kDecWarps * it);
     unsigned char* stage = ring + (it % kDecStages) * Lay::kStageBytes;
-    constexpr int kPieces = D / 8;   // 16-byte pieces per row
+    if constexpr (kFp8) {
+      constexpr int kPieces = D / 16;   // 16-byte pieces per raw E4M3 row
 #pragma unroll
-    for (int x = 0; x < kDecKeys * kPieces / 32; ++x) {
-      const int c = lane + 32 * x;
-      const int row = c / kPieces, col = c % kPieces;
-      const int key = key0 + row;
-      const bool in = key < p.Nk;
-      const int src_key = in ? key : 0;
-      cp_async_16(stage + row * Lay::kRowBytes + col * 16, p.k + p.k_st.at(b, hkv, src_key) + col * 8, in ? 16 : 0);
-      cp_async_16(stage + Lay::kTileBytes + row * Lay::kRowBytes + col * 16,
-                  p.v + p.v_st.at(b, hkv, src_key) + col * 8, in ? 16 : 0);
+      for (int x = 0; x < kDecKeys * kPieces / 32; ++x) {
+        const int c = lane + 32 * x;
+        const int row = c / kPieces, col = c % kPieces;
+        const int key = key0 + row;
+        const bool in = key < p.Nk;
+        const int src_key = in ? key : 0;
+        cp_async_16(stage + row * D + col * 16, p.k8 + p.k_st.at(b, hkv, src_key) + col * 16, in ? 16 : 0);
+        cp_async_16(stage + Lay::kRawTileBytes + row * D + col * 16, p.v8 + p.v_st.at(b, hkv, src_key) + col * 16,
+                    in ? 16 : 0);
+      }
+    } else {
+      constexpr int kPieces = D / 8;   // 16-byte pieces per row
+#pragma unroll
+      for (int x = 0; x < kDecKeys * kPieces / 32; ++x) {
+        const int c = lane + 32 * x;
+        const int row = c / kPieces, col = c % kPieces;
+        const int key = key0 + row;
+        const bool in = key < p.Nk;
+        const int src_key = in ? key : 0;
+        cp_async_16(stage + row * Lay::kRowBytes + col * 16, p.k + p.k_st.at(b, hkv, src_key) + col * 8,
+                    in ? 16 : 0);
+        cp_async_16(stage + Lay::kTileBytes + row * Lay::kRowBytes + col * 16,
+                    p.v + p.v_st.at(b, hkv, src_key) + col * 8, in ? 16 : 0);
+      }
     }
   };
 
@@ -221,6 +274,33 @@ __global__ void __launch_bounds__(kDecThreads, 2) fa_decode_kernel(const DecPara
     cp_async_wait<kDecStages - 2>();   // step it has landed (this lane's pieces)
     __syncwarp();                      // ... and every lane's; all lanes are past step it - 1
     const unsigned char* ks = ring + (it % kDecStages) * Lay::kStageBytes;
+    if constexpr (kFp8) {
+      // E4M3 -> f16 into the converted tiles: 16 codes (one 16-byte piece) per lane at a time
+      constexpr int kPieces = D / 16;
+      constexpr int kPerTensor = kDecKeys * kPieces;
+      unsigned char* conv = ring + kDecStages * Lay::kStageBytes;
+#pragma unroll
+      for (int x = 0; x < 2 * kPerTensor / 32; ++x) {
+        const int c = lane + 32 * x;
+        const int tensor = c / kPerTensor, rem = c % kPerTensor;
+        const int row = rem / kPieces, col = rem % kPieces;
+        const uint4 w = *reinterpret_cast<const uint4*>(ks + tensor * Lay::kRawTileBytes + row * D + col * 16);
+        uint4 lo, hi;
+        lo.x = e4m3x2_to_f16x2(w.x);
+        lo.y = e4m3x2_to_f16x2(w.x >> 16);
+        lo.z = e4m3x2_to_f16x2(w.y);
+        lo.w = e4m3x2_to_f16x2(w.y >> 16);
+        hi.x = e4m3x2_to_f16x2(w.z);
+        hi.y = e4m3x2_to_f16x2(w.z >> 16);
+        hi.z = e4m3x2_to_f16x2(w.w);
+        hi.w = e4m3x2_to_f16x2(w.w >> 16);
+        unsigned char* dst = conv + tensor * Lay::kTileBytes + row * Lay::kRowBytes + col * 32;
+        *reinterpret_cast<uint4*>(dst) = lo;
+        *reinterpret_cast<uint4*>(dst + 16) = hi;
+      }
+      __syncwarp();   // the converted tiles are complete for every lane
+      ks = conv;
+    }
     const unsigned char* vs = ks + Lay::kTileBytes;
     const int key0 = s0 + kDecKeys * (warp + kDecWarps * it);
 
@@ -230,8 +310,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) fa_decode_kernel(const DecPara
     for (int kk = 0; kk < KS; ++kk) {
       uint32_t kf[4];   // matrices: keys 0-7 | 8-15  x  columns 16kk + 0-7 | 8-15
       ldmatrix_x4(kf, ks + (((lane >> 4) << 3) + (lane & 7)) * Lay::kRowBytes + (16 * kk + ((lane >> 3) & 1) * 8) * 2);
-      mma_16816(s[0], qa[kk], kf[0], kf[1]);
-      mma_16816(s[1], qa[kk], kf[2], kf[3]);
+      dec_mma<kFp8>(s[0], qa[kk], kf[0], kf[1]);
+      dec_mma<kFp8>(s[1], qa[kk], kf[2], kf[3]);
     }
     // scale into the log2 domain; mask keys outside a row's band (and past N_k)
     const bool need_mask = key0 < lo_max || key0 + kDecKeys - 1 > hi_min;
@@ -266,9 +346,9 @@ __global__ void __launch_bounds__(kDecThreads, 2) fa_decode_kernel(const DecPara
         }
       l_run[hf] = l_run[hf] * alpha[hf] + sum;   // this lane's share; summed over the group at the end
     }
-    // O = alpha O + P V; P (bf16) is the A operand straight from the S fragments
-    const uint32_t pa[4] = {pack_bf16x2(s[0][0], s[0][1]), pack_bf16x2(s[0][2], s[0][3]),
-                            pack_bf16x2(s[1][0], s[1][1]), pack_bf16x2(s[1][2], s[1][3])};
+    // O = alpha O + P V; P (bf16, or f16) is the A operand straight from the S fragments
+    const uint32_t pa[4] = {dec_pack<kFp8>(s[0][0], s[0][1]), dec_pack<kFp8>(s[0][2], s[0][3]),
+                            dec_pack<kFp8>(s[1][0], s[1][1]), dec_pack<kFp8>(s[1][2], s[1][3])};
 #pragma unroll
     for (int j = 0; j < NT; ++j) {
       acc[j][0] *= alpha[0];
@@ -280,8 +360,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) fa_decode_kernel(const DecPara
     for (int j = 0; j < D / 16; ++j) {
       uint32_t vf[4];   // transposed matrices: keys 0-7 | 8-15  x  columns 16j + 0-7 | 8-15
       ldmatrix_x4_trans(vf, vs + (((lane >> 3) & 1) * 8 + (lane & 7)) * Lay::kRowBytes + (16 * j + (lane >> 4) * 8) * 2);
-      mma_16816(acc[2 * j], pa, vf[0], vf[1]);
-      mma_16816(acc[2 * j + 1], pa, vf[2], vf[3]);
+      dec_mma<kFp8>(acc[2 * j], pa, vf[0], vf[1]);
+      dec_mma<kFp8>(acc[2 * j + 1], pa, vf[2], vf[3]);
     }
     if (it + kDecStages - 1 < my_steps) issue(it + kDecStages - 1);
     cp_async_commit();
@@ -330,7 +410,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) fa_decode_kernel(const DecPara
         o1 += wt * src[lr * D + 2 * cp + 1];
       }
     }
-    const float inv = l > 0.f ? 1.f / l : 0.f;
+    float inv = l > 0.f ? 1.f / l : 0.f;
+    if constexpr (kFp8) inv *= p.v_scale;   // V = s_v V8
     const float lse = l > 0.f ? (mx + lg2_approx(l)) * kLn2 : -INFINITY;
     const int hq = hkv * p.group + r / p.Nq, i = r % p.Nq;
     const long long grow = ((long long)b * p.H + hq) * p.Nq + i;

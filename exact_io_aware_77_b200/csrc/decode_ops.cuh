@@ -6,6 +6,8 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 namespace fa {
 
@@ -52,6 +54,35 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
       "{%0, %1, %2, %3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// The same MMA on f16 operands (the FP8 K/V path: e4m3 converts to f16 exactly).
+__device__ __forceinline__ void mma_16816_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Two fp32 values as f16x2 (round to nearest even; lo in the low half).
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Two E4M3 codes (lo in the low byte) as f16x2; the conversion is exact.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two_codes & 0xffffu), __NV_E4M3);
+  return uint32_t(h.x) | (uint32_t(h.y) << 16);
+}
+
+// A bf16x2 word as f16x2, each value clamped to the finite f16 range first.
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2_sat(uint32_t w) {
+  constexpr float kMax = 65504.f;
+  const float lo = fminf(fmaxf(__uint_as_float(w << 16), -kMax), kMax);
+  const float hi = fminf(fmaxf(__uint_as_float(w & 0xffff0000u), -kMax), kMax);
+  return pack_f16x2(lo, hi);
 }
 
 __device__ __forceinline__ uint32_t ld_global_u32(const void* p) {

@@ -220,14 +220,18 @@ int check_decode(int B, int H, int H_kv, int Nq, int Nk, int d, float scale, int
   return FA_OK;
 }
 
-template <int D>
+// k, v: bf16 arrays, or (kFp8) E4M3 codes with K = k_scale K8, V = v_scale V8.
+template <int D, bool kFp8>
 int launch_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv, int Nq,
                   int Nk, const Strides* st, float scale, int causal, int window, void* ws, const DecPlan& pl,
-                  cudaStream_t stream) {
+                  cudaStream_t stream, float k_scale = 1.f, float v_scale = 1.f) {
   DecParams p;
   p.q = static_cast<const __nv_bfloat16*>(q);
-  p.k = static_cast<const __nv_bfloat16*>(k);
-  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.k = kFp8 ? nullptr : static_cast<const __nv_bfloat16*>(k);
+  p.v = kFp8 ? nullptr : static_cast<const __nv_bfloat16*>(v);
+  p.k8 = kFp8 ? static_cast<const unsigned char*>(k) : nullptr;
+  p.v8 = kFp8 ? static_cast<const unsigned char*>(v) : nullptr;
+  p.v_scale = v_scale;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.o_part = static_cast<float*>(ws);
@@ -249,10 +253,10 @@ int launch_decode(const void* q, const void* k, const void* v, void* o, float* l
   p.key_begin = pl.key_begin;
   p.causal = causal;
   p.window = window > Nk ? Nk : window;
-  p.scale_log2 = scale * 1.4426950408889634f;
-  constexpr int smem = DecLayout<D>::kSmemBytes;
-  if (set_smem(fa_decode_kernel<D>, smem) != FA_OK) return FA_ERR_CUDA;
-  fa_decode_kernel<D><<<unsigned(pl.ctas), kDecThreads, smem, stream>>>(p);
+  p.scale_log2 = scale * k_scale * 1.4426950408889634f;
+  constexpr int smem = DecLayout<D, kFp8>::kSmemBytes;
+  if (set_smem(fa_decode_kernel<D, kFp8>, smem) != FA_OK) return FA_ERR_CUDA;
+  fa_decode_kernel<D, kFp8><<<unsigned(pl.ctas), kDecThreads, smem, stream>>>(p);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   if (pl.n_splits > 1) {
     const long long blocks = (pl.total_rows + kDecMergeWarps - 1) / kDecMergeWarps;
@@ -432,9 +436,39 @@ int fa_fwd_decode(const void* q, const void* k, const void* v, void* o, float* l
     return FA_ERR_ALIGN;
   if ((st = check_device()) != FA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return d == 64 ? launch_decode<64>(q, k, v, o, lse, B, H, H_kv, N_q, N_k, s4, scale, causal, window, workspace, pl, s)
-                 : launch_decode<128>(q, k, v, o, lse, B, H, H_kv, N_q, N_k, s4, scale, causal, window, workspace, pl,
-                                      s);
+  return d == 64
+             ? launch_decode<64, false>(q, k, v, o, lse, B, H, H_kv, N_q, N_k, s4, scale, causal, window, workspace, pl, s)
+             : launch_decode<128, false>(q, k, v, o, lse, B, H, H_kv, N_q, N_k, s4, scale, causal, window, workspace, pl,
+                                         s);
+}
+
+int fa_fwd_decode_fp8kv(const void* q, const void* k8, const void* v8, float k_scale, float v_scale, void* o,
+                        float* lse, int B, int H, int H_kv, int N_q, int N_k, int d, const fa_strides* strides,
+                        float scale, int causal, int window, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !k8 || !v8 || !o || !lse) return FA_ERR_NULL;
+  DecPlan pl;
+  int st = check_decode(B, H, H_kv, N_q, N_k, d, scale, causal, window, &pl);
+  if (st != FA_OK) return st;
+  if (!std::isfinite(k_scale) || !(k_scale > 0.f) || !std::isfinite(v_scale) || !(v_scale > 0.f))
+    return FA_ERR_SCALE;
+  Strides s4[4] = {packed(H, N_q, d), packed(H_kv, N_k, d), packed(H_kv, N_k, d), packed(H, N_q, d)};
+  if (strides)
+    for (int i = 0; i < 4; ++i) {
+      s4[i] = Strides{strides[i].b, strides[i].h, strides[i].n};
+      if (!strides_ok(s4[i])) return FA_ERR_ALIGN;
+      // the code arrays are read in 16-byte pieces: 16 one-byte elements
+      if ((i == 1 || i == 2) && (s4[i].b % 16 || s4[i].h % 16 || s4[i].n % 16)) return FA_ERR_ALIGN;
+    }
+  if (pl.ws_bytes > 0 && (!workspace || workspace_bytes < pl.ws_bytes)) return FA_ERR_WORKSPACE;
+  if (!aligned(q, 16) || !aligned(k8, 16) || !aligned(v8, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
+      !aligned(workspace, 16))
+    return FA_ERR_ALIGN;
+  if ((st = check_device()) != FA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_decode<64, true>(q, k8, v8, o, lse, B, H, H_kv, N_q, N_k, s4, scale, causal, window,
+                                           workspace, pl, s, k_scale, v_scale)
+                 : launch_decode<128, true>(q, k8, v8, o, lse, B, H, H_kv, N_q, N_k, s4, scale, causal, window,
+                                            workspace, pl, s, k_scale, v_scale);
 }
 
 const char* fa_status_string(int status) {

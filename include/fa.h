@@ -189,6 +189,28 @@ FA_EXPORT int fa_fwd_decode(const void* q, const void* k, const void* v, void* o
                             int N_q, int N_k, int d, const fa_strides* strides, float scale, int causal, int window,
                             void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * fa_fwd_decode over an FP8 key/value cache.  The FlashAttention (NL) page says FlashAttention-3
+ * supports FP8 ("Evolutie en verdere ontwikkelingen"), without a format; the reading is that
+ * paper's E4M3 with one scale per tensor: K = k_scale * E4M3(k8), V = v_scale * E4M3(v8), where
+ * E4M3 has 1 sign, 4 exponent (bias 7) and 3 mantissa bits, subnormals, no infinities, and
+ * S.1111.111 as NaN (NaN codes give NaN results).
+ *
+ *   k8, v8   E4M3 codes, one byte each, [B, H_kv, N_k, d]; with `strides`, their strides count
+ *            bytes and must be multiples of 16.
+ *   k_scale, v_scale  finite and > 0 (FA_ERR_SCALE otherwise).
+ *   everything else as for fa_fwd_decode (q, o bf16; lse fp32; the same workspace size,
+ *   fa_decode_workspace_size).
+ *
+ * The kernels convert the codes to f16, which is exact, and run the products with f16 operands:
+ * Q is rounded to f16 after clamping to +-65504, and P enters P V as f16.  k_scale multiplies
+ * the softmax scale; v_scale multiplies O before it is rounded to bf16.
+ */
+FA_EXPORT int fa_fwd_decode_fp8kv(const void* q, const void* k8, const void* v8, float k_scale, float v_scale,
+                                  void* o, float* lse, int B, int H, int H_kv, int N_q, int N_k, int d,
+                                  const fa_strides* strides, float scale, int causal, int window, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 FA_EXPORT const char* fa_status_string(int status);
 

@@ -106,6 +106,24 @@ def make_inputs(wl: Workload, seed: int | None = None):
     return q, k, v
 
 
+def quantize_e4m3(x: torch.Tensor):
+    """Per-tensor E4M3 codes of x: scale = max|x| / 448 (the largest E4M3 value), codes =
+    x / scale rounded to nearest even by torch's float8_e4m3fn conversion, as uint8.
+    Returns (codes, scale)."""
+    amax = float(x.float().abs().max())
+    scale = amax / 448.0 if amax > 0 else 1.0
+    codes = (x.float() / scale).to(torch.float8_e4m3fn).view(torch.uint8)
+    return codes.contiguous(), scale
+
+
+def make_inputs_fp8kv(wl: Workload, seed: int | None = None):
+    """make_inputs with K and V quantised to E4M3 per tensor: (Q bf16, K8, V8, s_k, s_v)."""
+    q, k, v = make_inputs(wl, seed)
+    k8, s_k = quantize_e4m3(k)
+    v8, s_v = quantize_e4m3(v)
+    return q, k8, v8, s_k, s_v
+
+
 def make_grad_output(wl: Workload, seed: int | None = None) -> torch.Tensor:
     """dO as a contiguous CPU bf16 tensor [B, H, N, d], N(0, 1) from the grad seed."""
     s = seed if seed is not None else (wl.grad_seed if wl.grad_seed is not None else wl.seed + 1000)

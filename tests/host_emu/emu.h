@@ -30,6 +30,7 @@ inline thread_local dim3s threadIdx, blockIdx;
 struct float2 { float x, y; };
 struct float4 { float x, y, z, w; };
 struct uint2 { uint32_t x, y; };
+struct uint4 { uint32_t x, y, z, w; };
 inline float2 make_float2(float a, float b) { return {a, b}; }
 struct __nv_bfloat16 { uint16_t x; };
 

@@ -1,6 +1,7 @@
 // TEST INFRASTRUCTURE ONLY: runs the decode kernels of decode_kernel.cuh on the host through
 // the SIMT emulation of emu.h, with the launch parameters fa_fwd_decode derives.
 // usage: emu_main B H Hkv Nq Nk d causal window scale  sq(3) sk(3) sv(3) so(3)  nq nk nv no  prefix
+//                 [k_scale v_scale]   (with the scales: prefix.k / prefix.v hold E4M3 codes, one byte each)
 #include "emu.h"
 #include "decode_kernel.cuh"
 
@@ -24,7 +25,9 @@ void write_file(const std::string& path, const std::vector<T>& v) {
 }
 
 int main(int argc, char** argv) {
-  if (argc != 1 + 9 + 12 + 4 + 1) { std::fprintf(stderr, "bad args\n"); return 2; }
+  const int base_args = 1 + 9 + 12 + 4 + 1;
+  if (argc != base_args && argc != base_args + 2) { std::fprintf(stderr, "bad args\n"); return 2; }
+  const bool fp8 = argc == base_args + 2;
   int a = 1;
   const int B = atoi(argv[a++]), H = atoi(argv[a++]), Hkv = atoi(argv[a++]), Nq = atoi(argv[a++]),
             Nk = atoi(argv[a++]), d = atoi(argv[a++]), causal = atoi(argv[a++]), window = atoi(argv[a++]);
@@ -38,9 +41,17 @@ int main(int argc, char** argv) {
   size_t n[4];
   for (int i = 0; i < 4; ++i) n[i] = size_t(atoll(argv[a++]));
   const std::string prefix = argv[a++];
+  const float k_scale = fp8 ? float(atof(argv[a++])) : 1.f, v_scale = fp8 ? float(atof(argv[a++])) : 1.f;
   auto q = read_file<uint16_t>(prefix + ".q", n[0]);
-  auto k = read_file<uint16_t>(prefix + ".k", n[1]);
-  auto v = read_file<uint16_t>(prefix + ".v", n[2]);
+  std::vector<uint16_t> k, v;
+  std::vector<uint8_t> k8, v8;
+  if (fp8) {
+    k8 = read_file<uint8_t>(prefix + ".k", n[1]);
+    v8 = read_file<uint8_t>(prefix + ".v", n[2]);
+  } else {
+    k = read_file<uint16_t>(prefix + ".k", n[1]);
+    v = read_file<uint16_t>(prefix + ".v", n[2]);
+  }
   std::vector<uint16_t> o(n[3], 0x7fc0);   // NaN: rows the kernels fail to write show up
   std::vector<float> lse(size_t(B) * H * Nq, NAN);
 
@@ -49,8 +60,11 @@ int main(int argc, char** argv) {
   std::vector<float> ws(pl.ws_bytes / 4 + 1, NAN);
   DecParams p;
   p.q = reinterpret_cast<const __nv_bfloat16*>(q.data());
-  p.k = reinterpret_cast<const __nv_bfloat16*>(k.data());
-  p.v = reinterpret_cast<const __nv_bfloat16*>(v.data());
+  p.k = fp8 ? nullptr : reinterpret_cast<const __nv_bfloat16*>(k.data());
+  p.v = fp8 ? nullptr : reinterpret_cast<const __nv_bfloat16*>(v.data());
+  p.k8 = fp8 ? k8.data() : nullptr;
+  p.v8 = fp8 ? v8.data() : nullptr;
+  p.v_scale = v_scale;
   p.o = reinterpret_cast<__nv_bfloat16*>(o.data());
   p.lse = lse.data();
   p.o_part = pl.ws_bytes ? ws.data() : nullptr;
@@ -72,16 +86,27 @@ int main(int argc, char** argv) {
   p.key_begin = pl.key_begin;
   p.causal = causal;
   p.window = win;
-  p.scale_log2 = scale * 1.4426950408889634f;
+  p.scale_log2 = scale * k_scale * 1.4426950408889634f;
   std::printf("plan rows=%d row_blocks=%d n_splits=%d chunk=%d key_begin=%d ctas=%lld ws=%zu\n", pl.rows,
               pl.row_blocks, pl.n_splits, pl.chunk, pl.key_begin, pl.ctas, pl.ws_bytes);
-  if (d == 64) {
-    emu_launch(unsigned(pl.ctas), kDecThreads, DecLayout<64>::kSmemBytes, [&] { fa_decode_kernel<64>(p); });
+  if (fp8 && d == 64) {
+    emu_launch(unsigned(pl.ctas), kDecThreads, DecLayout<64, true>::kSmemBytes, [&] { fa_decode_kernel<64, true>(p); });
+    if (pl.n_splits > 1)
+      emu_launch(unsigned((pl.total_rows + kDecMergeWarps - 1) / kDecMergeWarps), 32 * kDecMergeWarps, 0,
+                 [&] { fa_decode_merge_kernel<64>(p); });
+  } else if (fp8) {
+    emu_launch(unsigned(pl.ctas), kDecThreads, DecLayout<128, true>::kSmemBytes,
+               [&] { fa_decode_kernel<128, true>(p); });
+    if (pl.n_splits > 1)
+      emu_launch(unsigned((pl.total_rows + kDecMergeWarps - 1) / kDecMergeWarps), 32 * kDecMergeWarps, 0,
+                 [&] { fa_decode_merge_kernel<128>(p); });
+  } else if (d == 64) {
+    emu_launch(unsigned(pl.ctas), kDecThreads, DecLayout<64>::kSmemBytes, [&] { fa_decode_kernel<64, false>(p); });
     if (pl.n_splits > 1)
       emu_launch(unsigned((pl.total_rows + kDecMergeWarps - 1) / kDecMergeWarps), 32 * kDecMergeWarps, 0,
                  [&] { fa_decode_merge_kernel<64>(p); });
   } else {
-    emu_launch(unsigned(pl.ctas), kDecThreads, DecLayout<128>::kSmemBytes, [&] { fa_decode_kernel<128>(p); });
+    emu_launch(unsigned(pl.ctas), kDecThreads, DecLayout<128>::kSmemBytes, [&] { fa_decode_kernel<128, false>(p); });
     if (pl.n_splits > 1)
       emu_launch(unsigned((pl.total_rows + kDecMergeWarps - 1) / kDecMergeWarps), 32 * kDecMergeWarps, 0,
                  [&] { fa_decode_merge_kernel<128>(p); });

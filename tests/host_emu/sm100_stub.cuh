@@ -3,7 +3,8 @@
 // name sm100.cuh.  ldmatrix and mma.sync are emulated from the fragment layouts the PTX ISA
 // documents (m8n8 b16 matrices; m16n8k16 row.col bf16 with fp32 accumulators); cp.async is a
 // synchronous copy (zero-fill when the source size is 0); ex2 / lg2 are std::exp2 / std::log2;
-// bf16 rounding is round-to-nearest-even.
+// bf16 and f16 rounding is round-to-nearest-even (f16 with subnormals and overflow to
+// infinity); E4M3 codes decode by the format's definition (they are all f16 values).
 #pragma once
 #include "emu.h"
 
@@ -28,6 +29,48 @@ inline float bf2f(uint16_t h) {
   return f;
 }
 inline uint32_t pack_bf16x2(float lo, float hi) { return uint32_t(f2bf(lo)) | (uint32_t(f2bf(hi)) << 16); }
+inline uint16_t f2h(float f) {
+  uint32_t x;
+  std::memcpy(&x, &f, 4);
+  const uint32_t sign = (x >> 16) & 0x8000u, ax = x & 0x7fffffffu;
+  if (ax >= 0x7f800000u) return uint16_t(sign | (ax > 0x7f800000u ? 0x7e00u : 0x7c00u));
+  if (ax >= 0x477ff000u) return uint16_t(sign | 0x7c00u);   // >= 65520 rounds to infinity
+  if (ax < 0x38800000u) {                                    // below 2^-14: subnormal
+    float v;
+    std::memcpy(&v, &ax, 4);
+    return uint16_t(sign | uint32_t(std::nearbyint(v * 16777216.0f)));
+  }
+  const uint32_t m = ax & 0x7fffffu;
+  uint32_t h = (((ax >> 23) - 112u) << 10) | (m >> 13);
+  const uint32_t rem = m & 0x1fffu;
+  if (rem > 0x1000u || (rem == 0x1000u && (h & 1u))) h += 1;
+  return uint16_t(sign | h);
+}
+inline float h2f(uint16_t h) {
+  const int e = (h >> 10) & 0x1f, m = h & 0x3ff;
+  float v;
+  if (e == 0) v = std::ldexp(float(m), -24);
+  else if (e == 31) v = m ? NAN : INFINITY;
+  else v = std::ldexp(float(1024 + m), e - 25);
+  return (h & 0x8000) ? -v : v;
+}
+inline float e4m3_to_f(uint8_t c) {
+  const int e = (c >> 3) & 0xf, m = c & 7;
+  float v;
+  if (e == 0) v = std::ldexp(float(m), -9);
+  else if (e == 15 && m == 7) v = NAN;
+  else v = std::ldexp(float(8 + m), e - 10);
+  return (c & 0x80) ? -v : v;
+}
+inline uint32_t pack_f16x2(float lo, float hi) { return uint32_t(f2h(lo)) | (uint32_t(f2h(hi)) << 16); }
+inline uint32_t e4m3x2_to_f16x2(uint32_t two) {
+  return uint32_t(f2h(e4m3_to_f(uint8_t(two & 0xff)))) | (uint32_t(f2h(e4m3_to_f(uint8_t((two >> 8) & 0xff)))) << 16);
+}
+inline uint32_t bf16x2_to_f16x2_sat(uint32_t w) {
+  const float lo = std::fmin(std::fmax(bf2f(uint16_t(w & 0xffff)), -65504.f), 65504.f);
+  const float hi = std::fmin(std::fmax(bf2f(uint16_t(w >> 16)), -65504.f), 65504.f);
+  return pack_f16x2(lo, hi);
+}
 inline unsigned char* dec_dyn_smem() { return g_blk->smem; }
 inline void cp_async_16(void* dst, const void* src, int n) {
   if (n == 16) std::memcpy(dst, src, 16);
@@ -73,7 +116,8 @@ inline void ldmatrix_x4_trans(uint32_t (&r)[4], const void* row) {
   }
   w.bar->arrive_and_wait();
 }
-inline void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+template <class Dec>
+inline void mma_emu(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1, Dec dec) {
   WarpCtx& w = my_warp();
   int l = lane_id();
   for (int i = 0; i < 4; ++i) w.xch[l][i] = a[i];
@@ -85,8 +129,8 @@ inline void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32
   for (int L = 0; L < 32; ++L) {
     const int g = L >> 2, t = L & 3;
     const uint32_t* x = w.xch[L];
-    auto lo = [](uint32_t v) { return bf2f(uint16_t(v & 0xffff)); };
-    auto hi = [](uint32_t v) { return bf2f(uint16_t(v >> 16)); };
+    auto lo = [&](uint32_t v) { return dec(uint16_t(v & 0xffff)); };
+    auto hi = [&](uint32_t v) { return dec(uint16_t(v >> 16)); };
     A[g][2 * t] = lo(x[0]); A[g][2 * t + 1] = hi(x[0]);
     A[g + 8][2 * t] = lo(x[1]); A[g + 8][2 * t + 1] = hi(x[1]);
     A[g][2 * t + 8] = lo(x[2]); A[g][2 * t + 9] = hi(x[2]);
@@ -106,5 +150,11 @@ inline void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32
     d[i] = s;
   }
   w.bar->arrive_and_wait();
+}
+inline void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  mma_emu(d, a, b0, b1, [](uint16_t h) { return bf2f(h); });
+}
+inline void mma_16816_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  mma_emu(d, a, b0, b1, [](uint16_t h) { return h2f(h); });
 }
 }  // namespace fa

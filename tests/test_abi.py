@@ -187,3 +187,40 @@ def test_decode_workspace_size(lib):
         assert n > 0 and n % per_split == 0 and 2 <= n // per_split <= 512, (n, per_split)
     # a causal window leaves only the last keys to visit: the same as the keys alone
     assert size(1, 8, 2, 1, 32768, 128, 1, 1000) == size(1, 8, 2, 1, 1000, 128, 1, 0)
+
+
+def _dec8(ws_bytes=1 << 30, **kw):
+    a = dict(B=1, H=8, H_kv=2, N_q=1, N_k=4096, d=128, scale=0.125, causal=1, window=0, k_scale=0.01, v_scale=0.02)
+    ptrs = kw.pop("ptrs", [A + 4096 * i for i in range(5)])
+    ws = kw.pop("ws", A + 65536)
+    st = kw.pop("strides", None)
+    a.update(kw)
+    return _lib.fa_fwd_decode_fp8kv(ptrs[0], ptrs[1], ptrs[2], a["k_scale"], a["v_scale"], ptrs[3], ptrs[4], a["B"],
+                                    a["H"], a["H_kv"], a["N_q"], a["N_k"], a["d"], st, a["scale"], a["causal"],
+                                    a["window"], ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(ptrs=[A, 0, A, A, A]), "FA_ERR_NULL"),
+    (dict(N_q=4097), "FA_ERR_SHAPE"),
+    (dict(H_kv=3), "FA_ERR_SHAPE"),
+    (dict(d=256), "FA_ERR_HEADDIM"),
+    (dict(window=-2), "FA_ERR_MASK"),
+    (dict(k_scale=0.0), "FA_ERR_SCALE"),
+    (dict(v_scale=-1.0), "FA_ERR_SCALE"),
+    (dict(k_scale=float("inf")), "FA_ERR_SCALE"),
+    (dict(v_scale=float("nan")), "FA_ERR_SCALE"),
+    (dict(ws=0), "FA_ERR_WORKSPACE"),
+    (dict(ptrs=[A, A + 8, A, A, A]), "FA_ERR_ALIGN"),
+    (dict(ptrs=[A, A, A + 1, A, A]), "FA_ERR_ALIGN"),
+])
+def test_decode_fp8kv_rejects_bad_arguments(lib, kw, code):
+    assert _lib.STATUS_NAMES[_dec8(**kw)] == code
+
+
+def test_decode_fp8kv_code_strides_are_16_byte_multiples(lib):
+    """The E4M3 arrays are read in 16-byte pieces: a stride of 8 codes is refused, 16 is not."""
+    good = [_lib.FaStrides(8 * 4096 * 128, 4096 * 128, 128) for _ in range(4)]
+    arr = (_lib.FaStrides * 4)(*good)
+    arr[1] = _lib.FaStrides(2 * 4096 * 136, 4096 * 136, 136)      # K rows padded by 8 codes
+    assert _lib.STATUS_NAMES[_dec8(strides=ctypes.addressof(arr))] == "FA_ERR_ALIGN"

@@ -35,5 +35,8 @@ def test_decode_bytes():
     # the decode workload: one row per query head, every cached key read once
     b = bench.decode_bytes(8, 64, 8, 1, 32768, 128, True)
     assert b == 2 * 8 * 64 * 128 * 2 + 2 * 8 * 8 * 32768 * 128 * 2 + 8 * 64 * 4
+    # an E4M3 cache halves the K and V bytes
+    assert bench.decode_bytes(8, 64, 8, 1, 32768, 128, True, kv_elem_bytes=1) == \
+        2 * 8 * 64 * 128 * 2 + 2 * 8 * 8 * 32768 * 128 + 8 * 64 * 4
     # a causal window reads only the keys the window keeps
     assert bench.decode_bytes(1, 1, 1, 1, 10000, 64, True, 100) == 2 * 64 * 2 + 2 * 100 * 64 * 2 + 4

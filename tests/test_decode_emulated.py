@@ -20,7 +20,7 @@ import pytest
 import torch
 
 from oracle import attention as orc
-from synthetic import Workload, make_inputs
+from synthetic import Workload, make_inputs, make_inputs_fp8kv
 from tests.parity import O_MAX_ABS, O_MEAN_ABS, L_MAX_ABS
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -50,8 +50,11 @@ def _bits(t):
     return t.contiguous().view(torch.int16).numpy().view(np.uint16)
 
 
-def _run(exe, wl, seq_major=False):
-    q, k, v = make_inputs(wl)
+def _run(exe, wl, seq_major=False, fp8=False):
+    if fp8:
+        q, k, v, s_k, s_v = make_inputs_fp8kv(wl)
+    else:
+        q, k, v = make_inputs(wl)
     B, H, Nq, d = q.shape
     Hkv, Nk = k.shape[1], k.shape[2]
     if seq_major:   # [B, N, heads, d] storage seen as [B, heads, N, d]
@@ -66,16 +69,21 @@ def _run(exe, wl, seq_major=False):
     with tempfile.TemporaryDirectory() as tmp:
         pre = os.path.join(tmp, "x")
         for name, t in zip("qkv", store):
-            _bits(t).tofile(pre + "." + name)
+            (t.contiguous().numpy() if t.dtype == torch.uint8 else _bits(t)).tofile(pre + "." + name)
         args = [B, H, Hkv, Nq, Nk, d, int(wl.causal), wl.window, repr(wl.scale)] + strides + \
                [t.numel() for t in store] + [o_store.numel(), pre]
+        if fp8:
+            args += [repr(s_k), repr(s_v)]
         r = subprocess.run([exe] + [str(a) for a in args], capture_output=True, text=True, timeout=600)
         assert r.returncode == 0, r.stdout + r.stderr[-4000:]
         o_bits = np.fromfile(pre + ".o", dtype=np.uint16)
         lse = np.fromfile(pre + ".lse", dtype=np.float32).reshape(B, H, Nq)
     o = torch.from_numpy(o_bits.view(np.int16).copy()).view(torch.bfloat16).reshape(o_store.shape)
     o = (o.transpose(1, 2) if seq_major else o).double().numpy()
-    o_ref, l_ref = orc.attention_forward_decode(q, k, v, wl.scale, wl.causal, wl.window)
+    if fp8:
+        o_ref, l_ref = orc.attention_forward_decode_fp8kv(q, k, v, s_k, s_v, wl.scale, wl.causal, wl.window)
+    else:
+        o_ref, l_ref = orc.attention_forward_decode(q, k, v, wl.scale, wl.causal, wl.window)
     assert np.isfinite(o).all() and np.isfinite(lse).all(), "a row was not written"
     err = np.abs(o - o_ref)
     assert err.max() <= O_MAX_ABS and err.mean() <= O_MEAN_ABS, (err.max(), err.mean())
@@ -103,6 +111,22 @@ def test_decode_kernel_emulated(emu_binary, B, H, H_kv, N_q, N_k, d, causal, win
     wl = Workload("decode_emu", B, H, N_k, d, causal, window, seed=71 + N_k + N_q, H_kv=H_kv, Nq=N_q)
     out = _run(emu_binary, wl)
     assert out.startswith("plan ")
+
+
+FP8_CASES = [
+    (1, 4, 1, 1, 300, 128, True, 0),
+    (2, 8, 2, 3, 1000, 128, True, 0),
+    (1, 4, 4, 20, 20, 64, True, 0),
+    (1, 2, 1, 5, 777, 64, False, 50),
+    (1, 2, 2, 64, 4096, 128, True, 300),
+]
+
+
+@pytest.mark.parametrize("B,H,H_kv,N_q,N_k,d,causal,window", FP8_CASES)
+def test_decode_fp8kv_kernel_emulated(emu_binary, B, H, H_kv, N_q, N_k, d, causal, window):
+    """The FP8 K/V path (E4M3 codes, per-tensor scales) against the oracle on the dequantised cache."""
+    wl = Workload("decode_fp8_emu", B, H, N_k, d, causal, window, seed=81 + N_k + N_q, H_kv=H_kv, Nq=N_q)
+    _run(emu_binary, wl, fp8=True)
 
 
 def test_decode_kernel_emulated_strided(emu_binary):
