@@ -151,7 +151,7 @@ def backward(q, k, v, o, lse, do, scale: float | None = None, causal: bool = Fal
 def decode_workspace_size(B: int, H: int, H_kv: int, N_q: int, N_k: int, d: int, causal: bool = False,
                           window: int = 0) -> int:
     """Bytes of scratch device memory decode() needs (0 when the keys fit one split)."""
-    if not (1 <= N_q <= N_k and B >= 1 and H_kv >= 1 and H % H_kv == 0 and d in (64, 128) and window >= 0):
+    if not (1 <= N_q <= N_k and B >= 1 and H_kv >= 1 and H % H_kv == 0 and d in (64, 128, 256) and window >= 0):
         raise ValueError("invalid shape")
     return _lib.fa_decode_workspace_size(B, H, H_kv, N_q, N_k, d, int(bool(causal)), int(window))
 

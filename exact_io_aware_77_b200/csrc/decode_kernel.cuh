@@ -33,7 +33,8 @@ constexpr int kDecRows = 16;        // query rows per CTA: the M of the MMA
 constexpr int kDecKeys = 16;        // keys per warp step
 constexpr int kDecStages = 3;       // depth of each warp's copy ring
 constexpr int kDecMergeWarps = 8;   // warps (one output row each) per CTA of the split merge
-constexpr int kDecSlots = 148 * 2;  // CTAs resident at once on a B200 (148 SMs, two CTAs each)
+// CTAs resident at once on a B200 (148 SMs): two per SM, one at d = 256 (its rings take 198 KB)
+__host__ __device__ constexpr int dec_slots(int d) { return d == 256 ? 148 : 148 * 2; }
 constexpr int kDecCtaOverheadKeys = 128;   // a CTA's fixed cost (Q load, ring fill, merge), in keys
 
 template <int D, bool kFp8 = false>
@@ -53,6 +54,7 @@ struct DecLayout {
   static constexpr int kMergeFloats = kDecRows * D + 2 * kDecRows;
   static constexpr int kMergeBytes = kDecWarps * kMergeFloats * 4;
   static constexpr int kSmemBytes = kRingBytes > kMergeBytes ? kRingBytes : kMergeBytes;
+  static_assert(kSmemBytes <= 232448, "decode shared memory exceeds 227 KB");
 };
 
 struct DecParams {
@@ -122,7 +124,7 @@ inline DecPlan dec_plan(int B, int H, int H_kv, int Nq, int Nk, int d, int causa
   for (int ns = 1; ns <= max_splits; ++ns) {
     const int per = (steps + ns - 1) / ns;
     const int used = (steps + per - 1) / per;
-    const long long waves = (base * used + kDecSlots - 1) / kDecSlots;
+    const long long waves = (base * used + dec_slots(d) - 1) / dec_slots(d);
     const long long cost = waves * ((long long)per * kDecKeys + kDecCtaOverheadKeys);
     if (best_cost < 0 || cost < best_cost) {
       best_cost = cost;
@@ -426,7 +428,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) fa_decode_kernel(const DecPara
   }
 }
 
-// Merge the splits of every output row: one warp per row, D / 32 columns per lane.  The
+// Merge the splits of every output row: one warp per row, D / 32 (2, 4 or 8) columns per lane.  The
 // lanes first read up to 32 splits' L_s at once (lane s holds split s); the O_s loads of
 // eight splits are then in flight together, so the row costs a few memory latencies rather
 // than one per split.
@@ -456,12 +458,15 @@ __global__ void __launch_bounds__(32 * kDecMergeWarps) fa_decode_merge_kernel(co
       for (int j = 0; j < cnt; ++j) {
         const float w = __shfl_sync(0xffffffffu, wt, j);
         const float* src = p.o_part + ((long long)(s0 + j) * p.total_rows + grow) * D + lane * C;
-        if constexpr (C == 4) {
-          const float4 x = *reinterpret_cast<const float4*>(src);
-          acc[0] += w * x.x;
-          acc[1] += w * x.y;
-          acc[2] += w * x.z;
-          acc[3] += w * x.w;
+        if constexpr (C % 4 == 0) {
+#pragma unroll
+          for (int c = 0; c < C; c += 4) {
+            const float4 x = *reinterpret_cast<const float4*>(src + c);
+            acc[c] += w * x.x;
+            acc[c + 1] += w * x.y;
+            acc[c + 2] += w * x.z;
+            acc[c + 3] += w * x.w;
+          }
         } else {
           const float2 x = *reinterpret_cast<const float2*>(src);
           acc[0] += w * x.x;
@@ -477,11 +482,14 @@ __global__ void __launch_bounds__(32 * kDecMergeWarps) fa_decode_merge_kernel(co
   const long long bh = grow / p.Nq;
   const int b = int(bh / p.H), hq = int(bh % p.H);
   __nv_bfloat16* dst = p.o + p.o_st.at(b, hq, i) + lane * C;
-  if constexpr (C == 4) {
-    uint2 w;
-    w.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
-    w.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
-    *reinterpret_cast<uint2*>(dst) = w;
+  if constexpr (C % 4 == 0) {
+#pragma unroll
+    for (int c = 0; c < C; c += 4) {
+      uint2 w;
+      w.x = pack_bf16x2(acc[c] * inv, acc[c + 1] * inv);
+      w.y = pack_bf16x2(acc[c + 2] * inv, acc[c + 3] * inv);
+      *reinterpret_cast<uint2*>(dst + c) = w;
+    }
   } else {
     *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
   }

@@ -210,7 +210,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
 int check_decode(int B, int H, int H_kv, int Nq, int Nk, int d, float scale, int causal, int window, DecPlan* pl) {
   if (B < 1 || H < 1 || H_kv < 1 || Nq < 1 || Nk < 1 || Nq > Nk) return FA_ERR_SHAPE;
   if (check_kv_heads(H, H_kv) != FA_OK) return FA_ERR_SHAPE;
-  if (d != 64 && d != 128) return FA_ERR_HEADDIM;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_HEADDIM;
   if (!(causal == 0 || causal == 1) || window < 0) return FA_ERR_MASK;
   if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_SCALE;
   const long long rows = (long long)(H / H_kv) * Nq;
@@ -436,10 +436,11 @@ int fa_fwd_decode(const void* q, const void* k, const void* v, void* o, float* l
     return FA_ERR_ALIGN;
   if ((st = check_device()) != FA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return d == 64
-             ? launch_decode<64, false>(q, k, v, o, lse, B, H, H_kv, N_q, N_k, s4, scale, causal, window, workspace, pl, s)
-             : launch_decode<128, false>(q, k, v, o, lse, B, H, H_kv, N_q, N_k, s4, scale, causal, window, workspace, pl,
-                                         s);
+  switch (d) {
+    case 64: return launch_decode<64, false>(q, k, v, o, lse, B, H, H_kv, N_q, N_k, s4, scale, causal, window, workspace, pl, s);
+    case 128: return launch_decode<128, false>(q, k, v, o, lse, B, H, H_kv, N_q, N_k, s4, scale, causal, window, workspace, pl, s);
+    default: return launch_decode<256, false>(q, k, v, o, lse, B, H, H_kv, N_q, N_k, s4, scale, causal, window, workspace, pl, s);
+  }
 }
 
 int fa_fwd_decode_fp8kv(const void* q, const void* k8, const void* v8, float k_scale, float v_scale, void* o,
@@ -465,10 +466,11 @@ int fa_fwd_decode_fp8kv(const void* q, const void* k8, const void* v8, float k_s
     return FA_ERR_ALIGN;
   if ((st = check_device()) != FA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return d == 64 ? launch_decode<64, true>(q, k8, v8, o, lse, B, H, H_kv, N_q, N_k, s4, scale, causal, window,
-                                           workspace, pl, s, k_scale, v_scale)
-                 : launch_decode<128, true>(q, k8, v8, o, lse, B, H, H_kv, N_q, N_k, s4, scale, causal, window,
-                                            workspace, pl, s, k_scale, v_scale);
+  switch (d) {
+    case 64: return launch_decode<64, true>(q, k8, v8, o, lse, B, H, H_kv, N_q, N_k, s4, scale, causal, window, workspace, pl, s, k_scale, v_scale);
+    case 128: return launch_decode<128, true>(q, k8, v8, o, lse, B, H, H_kv, N_q, N_k, s4, scale, causal, window, workspace, pl, s, k_scale, v_scale);
+    default: return launch_decode<256, true>(q, k8, v8, o, lse, B, H, H_kv, N_q, N_k, s4, scale, causal, window, workspace, pl, s, k_scale, v_scale);
+  }
 }
 
 const char* fa_status_string(int status) {

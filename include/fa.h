@@ -174,6 +174,7 @@ FA_EXPORT int fa_bwd_strided(const void* q, const void* k, const void* v, const 
  *   q, o   bf16 [B, H, N_q, d];  k, v  bf16 [B, H_kv, N_k, d]  (H a multiple of H_kv; query
  *          head h reads K/V head h / (H / H_kv));  lse  fp32 [B, H, N_q], packed.
  *   strides  NULL for packed arrays, else 4 fa_strides (q, k, v, o) as for fa_fwd_strided.
+ *   d      64, 128 or 256 (the decode entry points take head dimension 256; fa_fwd / fa_bwd do not).
  *   workspace  device memory of at least fa_decode_workspace_size(...) bytes, 16-byte aligned,
  *          owned by the caller; it holds the per-split partial results (fp32).  When that size
  *          is 0 (the keys fit one split) workspace may be NULL.

@@ -89,7 +89,15 @@ int main(int argc, char** argv) {
   p.scale_log2 = scale * k_scale * 1.4426950408889634f;
   std::printf("plan rows=%d row_blocks=%d n_splits=%d chunk=%d key_begin=%d ctas=%lld ws=%zu\n", pl.rows,
               pl.row_blocks, pl.n_splits, pl.chunk, pl.key_begin, pl.ctas, pl.ws_bytes);
-  if (fp8 && d == 64) {
+  if (d == 256) {
+    if (fp8)
+      emu_launch(unsigned(pl.ctas), kDecThreads, DecLayout<256, true>::kSmemBytes, [&] { fa_decode_kernel<256, true>(p); });
+    else
+      emu_launch(unsigned(pl.ctas), kDecThreads, DecLayout<256>::kSmemBytes, [&] { fa_decode_kernel<256, false>(p); });
+    if (pl.n_splits > 1)
+      emu_launch(unsigned((pl.total_rows + kDecMergeWarps - 1) / kDecMergeWarps), 32 * kDecMergeWarps, 0,
+                 [&] { fa_decode_merge_kernel<256>(p); });
+  } else if (fp8 && d == 64) {
     emu_launch(unsigned(pl.ctas), kDecThreads, DecLayout<64, true>::kSmemBytes, [&] { fa_decode_kernel<64, true>(p); });
     if (pl.n_splits > 1)
       emu_launch(unsigned((pl.total_rows + kDecMergeWarps - 1) / kDecMergeWarps), 32 * kDecMergeWarps, 0,

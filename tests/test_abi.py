@@ -185,6 +185,9 @@ def test_decode_workspace_size(lib):
         n = size(B, H, H_kv, N_q, N_k, d, causal, window)
         per_split = B * H * N_q * (d + 1) * 4
         assert n > 0 and n % per_split == 0 and 2 <= n // per_split <= 512, (n, per_split)
+    # head dimension 256 is a decode shape too (one resident CTA per SM: fewer slots, same rule)
+    n = size(8, 64, 8, 1, 32768, 256, 1, 0)
+    assert n > 0 and n % (8 * 64 * 257 * 4) == 0
     # a causal window leaves only the last keys to visit: the same as the keys alone
     assert size(1, 8, 2, 1, 32768, 128, 1, 1000) == size(1, 8, 2, 1, 1000, 128, 1, 0)
 
@@ -204,7 +207,8 @@ def _dec8(ws_bytes=1 << 30, **kw):
     (dict(ptrs=[A, 0, A, A, A]), "FA_ERR_NULL"),
     (dict(N_q=4097), "FA_ERR_SHAPE"),
     (dict(H_kv=3), "FA_ERR_SHAPE"),
-    (dict(d=256), "FA_ERR_HEADDIM"),
+    (dict(d=96), "FA_ERR_HEADDIM"),
+    (dict(d=512), "FA_ERR_HEADDIM"),
     (dict(window=-2), "FA_ERR_MASK"),
     (dict(k_scale=0.0), "FA_ERR_SCALE"),
     (dict(v_scale=-1.0), "FA_ERR_SCALE"),

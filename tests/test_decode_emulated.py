@@ -103,6 +103,8 @@ CASES = [
     (1, 3, 3, 2, 40, 64, True, 1000),
     (1, 2, 2, 64, 4096, 128, True, 300),    # splits that some rows see no key of
     (1, 2, 1, 1, 8192, 64, True, 0),        # 64 splits: the merge reads them 32 at a time
+    (1, 4, 1, 2, 700, 256, True, 0),        # head dimension 256, split merge with 8 columns per lane
+    (1, 2, 2, 9, 100, 256, False, 20),
 ]
 
 
@@ -119,6 +121,7 @@ FP8_CASES = [
     (1, 4, 4, 20, 20, 64, True, 0),
     (1, 2, 1, 5, 777, 64, False, 50),
     (1, 2, 2, 64, 4096, 128, True, 300),
+    (1, 4, 1, 2, 700, 256, True, 0),
 ]
 
 
