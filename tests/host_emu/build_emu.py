@@ -1,0 +1,58 @@
+"""TEST INFRASTRUCTURE ONLY: assemble and compile a host-emulation binary for one kernel header.
+
+The kernel header is copied next to sm100_stub.cuh (as sm100.cuh), emu.h and the harness, with
+sm100_extracted.inc: the pure helpers cut from the real sm100.cuh (descriptor encoders and the
+FMA-pipe exponential), so that the emulation restates no encoding of the library's own.
+"""
+
+from __future__ import annotations
+
+import os
+import re
+import shutil
+import subprocess
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+CSRC = os.path.join(os.path.dirname(os.path.dirname(HERE)), "exact_io_aware_77_b200", "csrc")
+PURE_HELPERS = ("idesc_bf16_f32", "sw128_desc", "desc_advance", "exp2_poly_x2")
+
+
+def extract(src: str, name: str) -> str:
+    """The full definition (signature line through its closing brace) of function `name`."""
+    m = re.search(r"^[^\n]*\b" + re.escape(name) + r"\s*\(", src, re.M)
+    if m is None:
+        raise RuntimeError(f"{name} not found in sm100.cuh")
+    i = src.index("{", m.end())
+    depth = 0
+    for j in range(i, len(src)):
+        if src[j] == "{":
+            depth += 1
+        elif src[j] == "}":
+            depth -= 1
+            if depth == 0:
+                return src[m.start():j + 1] + "\n"
+    raise RuntimeError(f"unbalanced braces in {name}")
+
+
+def build(out_dir: str, kernel_header: str, harness: str, exe_name: str, defines=()) -> str:
+    gxx = shutil.which("g++")
+    if gxx is None:
+        raise FileNotFoundError("g++")
+    with open(os.path.join(CSRC, "sm100.cuh")) as f:
+        real = f.read()
+    with open(os.path.join(out_dir, "sm100_extracted.inc"), "w") as f:
+        f.write("// cut from sm100.cuh by tests/host_emu/build_emu.py\n")
+        for name in PURE_HELPERS:
+            f.write(extract(real, name))
+    shutil.copy(os.path.join(CSRC, kernel_header), os.path.join(out_dir, kernel_header))
+    shutil.copy(os.path.join(HERE, "sm100_stub.cuh"), os.path.join(out_dir, "sm100.cuh"))
+    shutil.copy(os.path.join(HERE, "emu.h"), os.path.join(out_dir, "emu.h"))
+    shutil.copy(os.path.join(HERE, harness), os.path.join(out_dir, harness))
+    exe = os.path.join(out_dir, exe_name)
+    cmd = [gxx, "-std=c++20", "-O1", "-g", "-fsanitize=address,undefined", "-fno-sanitize-recover=all",
+           "-fno-omit-frame-pointer", "-pthread"] + [f"-D{d}" for d in defines] + \
+          ["-x", "c++", os.path.join(out_dir, harness), "-o", exe]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    if r.returncode != 0:
+        raise RuntimeError("host emulation does not compile:\n" + r.stderr[-6000:])
+    return exe

@@ -1,0 +1,86 @@
+// TEST INFRASTRUCTURE ONLY: runs fa_fwd_kernel<EMU_D> of fwd_kernel.cuh on the host through the
+// emulation of emu.h / sm100_stub.cuh, with the tensor maps and parameters fa_fwd_gqa derives
+// for packed [B, heads, N, d] arrays.
+// usage: emu_fwd_main B H Hkv N causal window scale prefix   (prefix.q/.k/.v bf16; writes .o, .lse)
+#include "emu.h"
+#include "fwd_kernel.cuh"
+
+#include <fstream>
+#include <string>
+
+#ifndef EMU_D
+#define EMU_D 128
+#endif
+
+namespace fa {
+// the kernel's dynamic shared memory: exactly one (1024-byte aligned) FwdSmem, so AddressSanitizer
+// sees any access past it
+alignas(1024) uint8_t smem_raw[sizeof(FwdSmem<EMU_D>)];
+}  // namespace fa
+
+using namespace fa;
+
+template <class T>
+std::vector<T> read_file(const std::string& path, size_t n) {
+  std::vector<T> v(n);
+  std::ifstream f(path, std::ios::binary);
+  f.read(reinterpret_cast<char*>(v.data()), n * sizeof(T));
+  if (!f) { std::fprintf(stderr, "short read %s\n", path.c_str()); std::exit(2); }
+  return v;
+}
+template <class T>
+void write_file(const std::string& path, const std::vector<T>& v) {
+  std::ofstream f(path, std::ios::binary);
+  f.write(reinterpret_cast<const char*>(v.data()), v.size() * sizeof(T));
+}
+
+CUtensorMap make_map(const uint16_t* base, int d, int rows, int heads, int B, int box_rows) {
+  CUtensorMap m;
+  m.base = reinterpret_cast<const unsigned char*>(base);
+  m.dims[0] = uint64_t(d);
+  m.dims[1] = uint64_t(rows);
+  m.dims[2] = uint64_t(heads);
+  m.dims[3] = uint64_t(B);
+  m.strides[0] = uint64_t(d) * 2;
+  m.strides[1] = uint64_t(rows) * d * 2;
+  m.strides[2] = uint64_t(heads) * rows * d * 2;
+  m.box_x = 64;
+  m.box_rows = uint32_t(box_rows);
+  return m;
+}
+
+int main(int argc, char** argv) {
+  if (argc != 9) { std::fprintf(stderr, "bad args\n"); return 2; }
+  const int B = atoi(argv[1]), H = atoi(argv[2]), Hkv = atoi(argv[3]), N = atoi(argv[4]), causal = atoi(argv[5]),
+            window = atoi(argv[6]);
+  const float scale = float(atof(argv[7]));
+  const std::string prefix = argv[8];
+  constexpr int D = EMU_D;
+  auto q = read_file<uint16_t>(prefix + ".q", size_t(B) * H * N * D);
+  auto k = read_file<uint16_t>(prefix + ".k", size_t(B) * Hkv * N * D);
+  auto v = read_file<uint16_t>(prefix + ".v", size_t(B) * Hkv * N * D);
+  std::vector<uint16_t> o(size_t(B) * H * N * D, 0x7fc0);
+  std::vector<float> lse(size_t(B) * H * N, NAN);
+  const CUtensorMap tq = make_map(q.data(), D, N, H, B, kBlockM), tk = make_map(k.data(), D, N, Hkv, B, kBlockN),
+                    tv = make_map(v.data(), D, N, Hkv, B, kBlockN);
+  FwdParams prm;
+  prm.o = reinterpret_cast<__nv_bfloat16*>(o.data());
+  prm.lse = lse.data();
+  prm.N = N;
+  prm.BH = B * H;
+  prm.H = H;
+  prm.group = H / Hkv;
+  prm.o_st = Strides{(long long)H * N * D, (long long)N * D, (long long)D};
+  prm.n_pairs = ((N + kBlockM - 1) / kBlockM + kQTiles - 1) / kQTiles;
+  prm.causal = causal;
+  prm.window = window > N ? N : window;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.wait_limit_ns = 60ull * 1000000000ull;
+  const unsigned grid = unsigned(prm.n_pairs) * unsigned(B * H);
+  std::printf("grid %u smem %zu\n", grid, sizeof(FwdSmem<D>));
+  emu_launch(grid, kFwdThreads, sizeof(FwdSmem<D>), [&] { fa_fwd_kernel<D>(tq, tk, tv, prm); }, fa::smem_raw);
+  if (g_status != 0) { std::fprintf(stderr, "device status %d\n", g_status); return 3; }
+  write_file(prefix + ".o", o);
+  write_file(prefix + ".lse", lse);
+  return 0;
+}

@@ -1,6 +1,21 @@
-// TEST INFRASTRUCTURE ONLY: host stand-ins for the device helpers the decode kernel takes from
-// sm100.cuh and decode_ops.cuh.  The test copies this file next to decode_kernel.cuh under the
-// name sm100.cuh.  ldmatrix and mma.sync are emulated from the fragment layouts the PTX ISA
+// TEST INFRASTRUCTURE ONLY: host stand-ins for the device helpers the decode and forward
+// kernels take from sm100.cuh and decode_ops.cuh.  The tests copy this file next to the kernel
+// under the name sm100.cuh, with sm100_extracted.inc: the pure helpers (descriptor encoders,
+// the FMA-pipe exponential) cut from the real sm100.cuh, so their encodings are not restated.
+//
+// tcgen05, TMA and mbarriers are emulated from their documented behaviour:
+//   mbarrier    phases with an arrival count and a transaction-byte count; try_wait.parity(P)
+//               succeeds once the phase of parity P has completed.
+//   TMA         a 4-D tiled load of a 64-element x rows box, zero outside the tensor, written
+//               with the 128-byte swizzle (16-byte chunk c of a 128-byte row r lands at chunk
+//               c ^ (r % 8) of its 1024-byte atom), completing its bytes on the barrier.
+//   TMEM        128 lanes x 512 32-bit columns; address = lane << 16 | column; a warp's
+//               32x32b loads and stores reach only the lane quadrant 32 (warp % 4).
+//   MMA         kind::f16 bf16 x bf16 -> fp32, M = 128, K = 16, N from the instruction
+//               descriptor; operands read through SW128 shared-memory descriptors (K-major:
+//               8-row atoms SBO apart; MN-major: 64 MN-contiguous elements per row, 8-k atoms
+//               SBO apart, the next 64 MN elements LBO apart) or A from TMEM (bf16 pairs);
+//               executed when issued, so a commit arrives at once.  ldmatrix and mma.sync are emulated from the fragment layouts the PTX ISA
 // documents (m8n8 b16 matrices; m16n8k16 row.col bf16 with fp32 accumulators); cp.async is a
 // synchronous copy (zero-fill when the source size is 0); ex2 / lg2 are std::exp2 / std::log2;
 // bf16 and f16 rounding is round-to-nearest-even (f16 with subnormals and overflow to
@@ -157,4 +172,239 @@ inline void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32
 inline void mma_16816_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   mma_emu(d, a, b0, b1, [](uint16_t h) { return h2f(h); });
 }
+// ------------------------------------------------------------ shared memory addresses
+inline uint32_t smem_u32(const void* p) {
+  const long long off = static_cast<const unsigned char*>(p) - g_blk->smem;
+  if (off < 0 || size_t(off) >= g_blk->smem_bytes) { std::fprintf(stderr, "smem_u32 outside shared memory\n"); std::abort(); }
+  return uint32_t(off);
+}
+inline unsigned char* smem_at(uint32_t a, size_t bytes) {
+  if (size_t(a) + bytes > g_blk->smem_bytes) { std::fprintf(stderr, "shared access past the end: %u\n", a); std::abort(); }
+  return g_blk->smem + a;
+}
+inline uint64_t global_timer_ns() {
+  return uint64_t(std::chrono::duration_cast<std::chrono::nanoseconds>(
+                      std::chrono::steady_clock::now().time_since_epoch()).count());
+}
+inline int g_status = 0;
+constexpr int FA_DEVICE_TIMEOUT = 1;
+
+// ------------------------------------------------------------ mbarriers
+inline BarState& bar_state(uint32_t bar) {
+  auto it = g_blk->bars->find(bar);
+  if (it == g_blk->bars->end()) { std::fprintf(stderr, "mbarrier %u used before init\n", bar); std::abort(); }
+  return it->second;
+}
+inline void bar_flip_if_done(BarState& b) {
+  if (b.pending == 0 && b.tx == 0) {
+    b.phase ^= 1u;
+    b.pending = b.expected;
+  }
+}
+inline void mbar_init(uint32_t bar, uint32_t count) {
+  std::lock_guard<std::mutex> lk(*g_blk->mu);
+  (*g_blk->bars)[bar] = BarState{count, count, 0, 0};
+}
+inline void fence_mbar_init() {}
+inline void mbar_arrive(uint32_t bar) {
+  std::lock_guard<std::mutex> lk(*g_blk->mu);
+  BarState& b = bar_state(bar);
+  if (b.pending == 0) { std::fprintf(stderr, "mbarrier %u: too many arrivals\n", bar); std::abort(); }
+  b.pending -= 1;
+  bar_flip_if_done(b);
+}
+inline void mbar_expect_tx(uint32_t bar, uint32_t bytes) {   // arrive.expect_tx
+  std::lock_guard<std::mutex> lk(*g_blk->mu);
+  BarState& b = bar_state(bar);
+  if (b.pending == 0) { std::fprintf(stderr, "mbarrier %u: too many arrivals\n", bar); std::abort(); }
+  b.tx += bytes;
+  b.pending -= 1;
+  bar_flip_if_done(b);
+}
+inline void bar_complete_tx(uint32_t bar, uint32_t bytes) {
+  std::lock_guard<std::mutex> lk(*g_blk->mu);
+  BarState& b = bar_state(bar);
+  b.tx -= bytes;
+  bar_flip_if_done(b);
+}
+inline bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  std::lock_guard<std::mutex> lk(*g_blk->mu);
+  return bar_state(bar).phase != (parity & 1u);
+}
+inline bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort, uint64_t limit_ns) {
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (global_timer_ns() - t0 > limit_ns) {
+      *abort = 1;
+      atomicOr(&g_status, FA_DEVICE_TIMEOUT);
+      return false;
+    }
+    std::this_thread::yield();
+  }
+}
+inline bool mbar_wait_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  int never = 0;
+  return mbar_wait(bar, parity, &never, limit_ns);
+}
+
+// ------------------------------------------------------------ TMA
+struct CUtensorMap {
+  const unsigned char* base;
+  uint64_t dims[4];      // d, rows, heads, batch (elements)
+  uint64_t strides[3];   // bytes: rows, heads, batch
+  uint32_t box_x, box_rows;
+};
+inline void tma_prefetch_desc(const CUtensorMap*) {}
+inline uint32_t sw128(uint32_t addr) { return addr ^ (((addr >> 7) & 7u) << 4); }
+inline void tma_load_rows(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int row, int head, int batch) {
+  if (x % 8) { std::fprintf(stderr, "TMA x coordinate not 16-byte aligned\n"); std::abort(); }
+  if (map->box_x != 64) { std::fprintf(stderr, "TMA box is not 64 elements wide\n"); std::abort(); }
+  for (uint32_t r = 0; r < map->box_rows; ++r)
+    for (uint32_t c = 0; c < map->box_x; ++c) {
+      const long long gx = (long long)x + c, gr = (long long)row + r;
+      uint16_t val = 0;
+      if (gx >= 0 && gr >= 0 && head >= 0 && batch >= 0 && uint64_t(gx) < map->dims[0] &&
+          uint64_t(gr) < map->dims[1] && uint64_t(head) < map->dims[2] && uint64_t(batch) < map->dims[3])
+        std::memcpy(&val, map->base + uint64_t(batch) * map->strides[2] + uint64_t(head) * map->strides[1] +
+                              uint64_t(gr) * map->strides[0] + uint64_t(gx) * 2, 2);
+      std::memcpy(smem_at(sw128(dst + r * 128 + c * 2), 2), &val, 2);
+    }
+  bar_complete_tx(bar, map->box_x * map->box_rows * 2);
+}
+
+// ------------------------------------------------------------ tensor memory
+inline uint32_t& tmem_cell(uint32_t lane, uint32_t col) {
+  if (lane >= 128 || col >= 512) { std::fprintf(stderr, "TMEM access out of range (%u, %u)\n", lane, col); std::abort(); }
+  return g_blk->tmem[lane * 512 + col];
+}
+inline void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+  if (ncols < 32 || ncols > 512 || (ncols & (ncols - 1))) { std::fprintf(stderr, "bad TMEM allocation\n"); std::abort(); }
+  if (lane_id() == 0) {
+    const uint32_t base = 0;
+    std::memcpy(smem_at(dst_smem, 4), &base, 4);
+  }
+  __syncwarp();
+}
+inline void tmem_relinquish() {}
+inline void tmem_dealloc(uint32_t, uint32_t) {}
+inline void tc_fence_before() {}
+inline void tc_fence_after() {}
+inline void fence_proxy_async_smem() {}
+// the lane quadrant a warp may access: lanes 32 (warp % 4) .. + 31
+inline uint32_t tmem_row(uint32_t taddr) {
+  const uint32_t base = taddr >> 16, warp = threadIdx.x >> 5;
+  if (base != 32u * (warp % 4u)) { std::fprintf(stderr, "TMEM lane base %u outside warp %u's quadrant\n", base, warp); std::abort(); }
+  return base + uint32_t(lane_id());
+}
+template <int N>
+inline void tmem_ld_n(uint32_t taddr, uint32_t* r) {
+  const uint32_t row = tmem_row(taddr), col = taddr & 0xffffu;
+  std::lock_guard<std::mutex> lk(*g_blk->mu);
+  for (int i = 0; i < N; ++i) r[i] = tmem_cell(row, col + i);
+}
+template <int N>
+inline void tmem_st_n(uint32_t taddr, const uint32_t* r) {
+  const uint32_t row = tmem_row(taddr), col = taddr & 0xffffu;
+  std::lock_guard<std::mutex> lk(*g_blk->mu);
+  for (int i = 0; i < N; ++i) tmem_cell(row, col + i) = r[i];
+}
+inline void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) { tmem_ld_n<32>(taddr, r); }
+inline void tmem_ld32_async(uint32_t taddr, uint32_t* r) { tmem_ld_n<32>(taddr, r); }
+inline void tmem_ld_wait() {}
+template <int N>
+inline void reg_fence(uint32_t*) {}
+inline void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) { tmem_st_n<32>(taddr, r); }
+inline void tmem_st16(uint32_t taddr, const uint32_t* r) { tmem_st_n<16>(taddr, r); }
+inline void tmem_st_wait() {}
+
+// bf16 element (i along M or N, k along K) of a 128-byte-swizzled shared-memory operand
+inline float sw128_operand(uint64_t desc, bool mn_major, uint32_t i, uint32_t k) {
+  if ((desc >> 61) != 2u) { std::fprintf(stderr, "descriptor layout is not the 128-byte swizzle\n"); std::abort(); }
+  const uint32_t start = uint32_t(desc & 0x3fffu) << 4, lbo = uint32_t((desc >> 16) & 0x3fffu) << 4,
+                 sbo = uint32_t((desc >> 32) & 0x3fffu) << 4;
+  const uint32_t addr = mn_major ? start + (i / 64) * lbo + (k / 8) * sbo + (k % 8) * 128 + (i % 64) * 2
+                                 : start + (i / 8) * sbo + (i % 8) * 128 + k * 2;
+  uint16_t h;
+  std::memcpy(&h, smem_at(sw128(addr), 2), 2);
+  return bf2f(h);
+}
+// D (+)= A B^T with A 128 x 16 (shared memory, or TMEM when a_tmem_addr != ~0u), B N x 16
+inline void mma_exec(uint32_t d_tmem, uint64_t a_desc, uint32_t a_tmem_addr, uint64_t b_desc, uint32_t idesc,
+                     uint32_t accumulate) {
+  if (((idesc >> 4) & 3u) != 1u || ((idesc >> 7) & 7u) != 1u || ((idesc >> 10) & 7u) != 1u) {
+    std::fprintf(stderr, "instruction descriptor is not bf16 x bf16 -> f32\n");
+    std::abort();
+  }
+  const uint32_t M = ((idesc >> 24) & 0x1fu) << 4, N = ((idesc >> 17) & 0x3fu) << 3;
+  const bool a_mn = (idesc >> 15) & 1u, b_mn = (idesc >> 16) & 1u;
+  if (M != 128 || N < 8 || N > 256 || N % 16) { std::fprintf(stderr, "unsupported MMA shape\n"); std::abort(); }
+  std::lock_guard<std::mutex> lk(*g_blk->mu);
+  static thread_local std::vector<float> A, B;
+  A.assign(128 * 16, 0.f);
+  B.assign(N * 16, 0.f);
+  for (uint32_t m = 0; m < 128; ++m)
+    for (uint32_t k = 0; k < 16; ++k) {
+      if (a_tmem_addr != ~0u) {
+        const uint32_t w = tmem_cell((a_tmem_addr >> 16) + m, (a_tmem_addr & 0xffffu) + k / 2);
+        A[m * 16 + k] = bf2f(uint16_t((k & 1) ? (w >> 16) : (w & 0xffffu)));
+      } else {
+        A[m * 16 + k] = sw128_operand(a_desc, a_mn, m, k);
+      }
+    }
+  for (uint32_t n = 0; n < N; ++n)
+    for (uint32_t k = 0; k < 16; ++k) B[n * 16 + k] = sw128_operand(b_desc, b_mn, n, k);
+  const uint32_t lane0 = d_tmem >> 16, col0 = d_tmem & 0xffffu;
+  for (uint32_t m = 0; m < 128; ++m)
+    for (uint32_t n = 0; n < N; ++n) {
+      uint32_t& cell = tmem_cell(lane0 + m, col0 + n);
+      float acc = accumulate ? __uint_as_float(cell) : 0.f;
+      for (uint32_t k = 0; k < 16; ++k) acc += A[m * 16 + k] * B[n * 16 + k];
+      cell = __float_as_uint(acc);
+    }
+}
+inline void mma_bf16_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) { mma_exec(d, a, ~0u, b, idesc, acc); }
+inline void mma_bf16_ts(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc, uint32_t acc) { mma_exec(d, 0, a, b, idesc, acc); }
+inline void mma_commit(uint32_t bar) { mbar_arrive(bar); }
+// warp-uniform forms: one elected lane issues
+inline void mma_bf16_ss_w(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  if (lane_id() == 0) mma_bf16_ss(d, a, b, idesc, acc);
+}
+inline void mma_bf16_ts_w(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  if (lane_id() == 0) mma_bf16_ts(d, a, b, idesc, acc);
+}
+inline void mma_commit_w(uint32_t bar) {
+  if (lane_id() == 0) mma_commit(bar);
+}
+
+// ------------------------------------------------------------ packed fp32 pairs, max
+inline uint64_t f2(float lo, float hi) { return uint64_t(__float_as_uint(lo)) | (uint64_t(__float_as_uint(hi)) << 32); }
+inline void f2_split(uint64_t v, float& lo, float& hi) {
+  lo = __uint_as_float(uint32_t(v));
+  hi = __uint_as_float(uint32_t(v >> 32));
+}
+inline uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  float a0, a1, b0, b1, c0, c1;
+  f2_split(a, a0, a1);
+  f2_split(b, b0, b1);
+  f2_split(c, c0, c1);
+  return f2(std::fma(a0, b0, c0), std::fma(a1, b1, c1));
+}
+inline uint64_t f2_mul(uint64_t a, uint64_t b) {
+  float a0, a1, b0, b1;
+  f2_split(a, a0, a1);
+  f2_split(b, b0, b1);
+  return f2(a0 * b0, a1 * b1);
+}
+inline uint64_t f2_add(uint64_t a, uint64_t b) {
+  float a0, a1, b0, b1;
+  f2_split(a, a0, a1);
+  f2_split(b, b0, b1);
+  return f2(a0 + b0, a1 + b1);
+}
+inline float max3f(float a, float b, float c) { return std::fmax(std::fmax(a, b), c); }
+
+#include "sm100_extracted.inc"
+
 }  // namespace fa

@@ -11,7 +11,6 @@ and merges without a GPU; the fragment layouts themselves are checked only on th
 """
 
 import os
-import shutil
 import subprocess
 import tempfile
 
@@ -29,21 +28,11 @@ CSRC = os.path.join(os.path.dirname(HERE), "exact_io_aware_77_b200", "csrc")
 
 @pytest.fixture(scope="module")
 def emu_binary(tmp_path_factory):
-    gxx = shutil.which("g++")
-    if gxx is None:
+    from tests.host_emu.build_emu import build
+    try:
+        return build(str(tmp_path_factory.mktemp("host_emu")), "decode_kernel.cuh", "emu_main.cpp", "emu_main")
+    except FileNotFoundError:
         pytest.skip("g++ not available")
-    d = tmp_path_factory.mktemp("host_emu")
-    shutil.copy(os.path.join(CSRC, "decode_kernel.cuh"), d / "decode_kernel.cuh")
-    shutil.copy(os.path.join(HERE, "host_emu", "sm100_stub.cuh"), d / "sm100.cuh")
-    shutil.copy(os.path.join(HERE, "host_emu", "emu.h"), d / "emu.h")
-    shutil.copy(os.path.join(HERE, "host_emu", "emu_main.cpp"), d / "emu_main.cpp")
-    exe = d / "emu_main"
-    r = subprocess.run([gxx, "-std=c++20", "-O1", "-g", "-fsanitize=address,undefined", "-fno-sanitize-recover=all",
-                        "-fno-omit-frame-pointer", "-pthread", "-x", "c++", str(d / "emu_main.cpp"), "-o", str(exe)],
-                       capture_output=True, text=True)
-    if r.returncode != 0:
-        pytest.fail("host emulation does not compile:\n" + r.stderr[-4000:])
-    return str(exe)
 
 
 def _bits(t):

@@ -1,0 +1,72 @@
+"""The tcgen05 forward kernel's own CUDA source, run on the CPU under an emulation of its
+primitives, vs the oracle.
+
+Test infrastructure only.  tests/host_emu/sm100_stub.cuh restates the documented behaviour of
+the sm_100a primitives fwd_kernel.cuh uses -- mbarrier phases and transaction counts, 4-D TMA
+tile loads with the 128-byte swizzle and zero fill, TMEM (128 lanes x 512 columns, one lane
+quadrant per warp), and kind::f16 MMAs that read their operands through the shared-memory
+descriptors (K-major and MN-major 128-byte-swizzled layouts) or from TMEM -- with one host
+thread per CUDA thread.  The pure helpers (descriptor encoders, the FMA-pipe exponential) are
+cut from the real sm100.cuh, not restated.  Compiled with AddressSanitizer and
+UndefinedBehaviorSanitizer: an access outside shared memory, TMEM or a tensor aborts the run,
+as does an mbarrier misuse or a TMEM access outside the warp's lane quadrant.  Outputs start as
+NaN.  What this cannot show is timing and the hardware's own reading of the descriptors; the
+GPU parity tests (tests/test_fwd_parity.py) are the check of those.
+"""
+
+import os
+import tempfile
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention as orc
+from synthetic import Workload, make_inputs
+from tests.parity import L_MAX_ABS, O_MAX_ABS, O_MEAN_ABS
+
+
+@pytest.fixture(scope="module")
+def emu_fwd(tmp_path_factory):
+    from tests.host_emu.build_emu import build
+    d = str(tmp_path_factory.mktemp("host_emu_fwd"))
+    try:
+        return {D: build(d, "fwd_kernel.cuh", "emu_fwd_main.cpp", f"emu_fwd_{D}", defines=(f"EMU_D={D}",))
+                for D in (64, 128)}
+    except FileNotFoundError:
+        pytest.skip("g++ not available")
+
+
+CASES = [
+    # B, H, H_kv, N, d, causal, window
+    (1, 1, 1, 128, 128, True, 0),       # one tile pair, second tile past N
+    (1, 2, 2, 300, 128, True, 0),       # ragged: two CTA pairs, partial last tile
+    (1, 2, 2, 300, 128, False, 0),
+    (1, 2, 1, 520, 128, True, 100),     # causal window, shared K/V head
+    (1, 4, 2, 400, 128, False, 50),     # two-sided window
+    (1, 2, 2, 700, 64, False, 0),
+    (2, 2, 1, 257, 64, True, 3),        # multi-query, narrow window, ragged
+    (1, 1, 1, 1000, 64, True, 1),       # window 1: O = V
+]
+
+
+@pytest.mark.parametrize("B,H,H_kv,N,d,causal,window", CASES)
+def test_fwd_kernel_emulated(emu_fwd, B, H, H_kv, N, d, causal, window):
+    import subprocess
+    wl = Workload("fwd_emu", B, H, N, d, causal, window, seed=91 + N + H_kv, H_kv=H_kv)
+    q, k, v = make_inputs(wl)
+    with tempfile.TemporaryDirectory() as tmp:
+        pre = os.path.join(tmp, "x")
+        for name, t in zip("qkv", (q, k, v)):
+            t.contiguous().view(torch.int16).numpy().tofile(pre + "." + name)
+        r = subprocess.run([emu_fwd[d], str(B), str(H), str(H_kv), str(N), str(int(causal)), str(window),
+                            repr(wl.scale), pre], capture_output=True, text=True, timeout=900)
+        assert r.returncode == 0, r.stdout[-1000:] + r.stderr[-4000:]
+        o = np.fromfile(pre + ".o", dtype=np.uint16)
+        lse = np.fromfile(pre + ".lse", dtype=np.float32).reshape(B, H, N)
+    o = torch.from_numpy(o.view(np.int16).copy()).view(torch.bfloat16).reshape(q.shape).double().numpy()
+    o_ref, l_ref = orc.attention_forward_shared_kv(q, k, v, wl.scale, causal, window)
+    assert np.isfinite(o).all() and np.isfinite(lse).all(), "a row was not written"
+    err = np.abs(o - o_ref)
+    assert err.max() <= O_MAX_ABS and err.mean() <= O_MEAN_ABS, (err.max(), err.mean())
+    assert np.abs(lse - l_ref).max() <= L_MAX_ABS
