@@ -12,6 +12,7 @@
 #include "../../include/fa.h"
 
 #include "fwd_kernel.cuh"
+#include "fwd256_kernel.cuh"
 #include "bwd_kernel.cuh"
 #include "decode_ops.cuh"
 #include "decode_kernel.cuh"
@@ -91,7 +92,7 @@ int check_problem(int B, int H, int N, int d, float scale, int causal, int windo
   const long long bh = (long long)B * H;
   const long long tiles = (N + kBlockM - 1) / kBlockM;
   if (bh > 0x7fffffffLL || bh * tiles > 0x7fffffffLL) return FA_ERR_SHAPE;
-  if (d != 64 && d != 128) return FA_ERR_HEADDIM;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_HEADDIM;   // 256: forward only (checked by the callers)
   if (!(causal == 0 || causal == 1) || window < 0) return FA_ERR_MASK;
   if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_SCALE;
   return FA_OK;
@@ -132,6 +133,35 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   if (set_smem(fa_fwd_kernel<D>, smem) != FA_OK) return FA_ERR_CUDA;
   const unsigned grid = unsigned(prm.n_pairs) * unsigned(BH);
   fa_fwd_kernel<D><<<grid, kFwdThreads, smem, stream>>>(tq, tk, tv, prm);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// head dimension 256: one 128-row query tile per CTA, 64-key K/V tiles (fwd256_kernel.cuh)
+int launch_fwd256(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv, int N,
+                  const Strides* st, float scale, int causal, int window, cudaStream_t stream) {
+  const int BH = B * H;
+  CUtensorMap tq, tk, tv;
+  if (!make_map_bf16(&tq, q, kD256, N, H, B, st[0], k256BlockM) ||
+      !make_map_bf16(&tk, k, kD256, N, H_kv, B, st[1], k256BlockN) ||
+      !make_map_bf16(&tv, v, kD256, N, H_kv, B, st[2], k256BlockN))
+    return FA_ERR_CUDA;
+  FwdParams prm;
+  prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.lse = lse;
+  prm.N = N;
+  prm.BH = BH;
+  prm.H = H;
+  prm.group = H / H_kv;
+  prm.o_st = st[3];
+  prm.n_pairs = (N + k256BlockM - 1) / k256BlockM;   // query tiles per head
+  prm.causal = causal;
+  prm.window = window > N ? N : window;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.wait_limit_ns = g_wait_limit_ns;
+  static_assert(sizeof(Fwd256Smem) + 1024 <= 232448, "d = 256 forward shared memory exceeds 227 KB");
+  const int smem = int(sizeof(Fwd256Smem)) + 1024;
+  if (set_smem(fa_fwd256_kernel, smem) != FA_OK) return FA_ERR_CUDA;
+  fa_fwd256_kernel<<<unsigned(prm.n_pairs) * unsigned(BH), k256Threads, smem, stream>>>(tq, tk, tv, prm);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -341,12 +371,15 @@ int fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* 
     return FA_ERR_ALIGN;
   if ((st = check_device()) != FA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return d == 64 ? launch_fwd<64>(q, k, v, o, lse, B, H, H_kv, N, s4, scale, causal, window, s)
-                 : launch_fwd<128>(q, k, v, o, lse, B, H, H_kv, N, s4, scale, causal, window, s);
+  switch (d) {
+    case 64: return launch_fwd<64>(q, k, v, o, lse, B, H, H_kv, N, s4, scale, causal, window, s);
+    case 128: return launch_fwd<128>(q, k, v, o, lse, B, H, H_kv, N, s4, scale, causal, window, s);
+    default: return launch_fwd256(q, k, v, o, lse, B, H, H_kv, N, s4, scale, causal, window, s);
+  }
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
-  if (check_problem(B, H, N, d, 1.f, 0, 0) != FA_OK) return 0;
+  if (d == 256 || check_problem(B, H, N, d, 1.f, 0, 0) != FA_OK) return 0;
   return bwd_workspace_bytes((long long)B * H, N, d);
 }
 
@@ -387,6 +420,7 @@ static int bwd_impl(const void* q, const void* k, const void* v, const void* o, 
   if (phases < 1 || phases > kBwdAllPhases) return FA_ERR_PHASES;
   if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FA_ERR_NULL;
   int st = check_problem(B, H, N, d, scale, causal, window);
+  if (st == FA_OK && d == 256) st = FA_ERR_HEADDIM;   // the backward has no d = 256 kernel
   if (st == FA_OK) st = check_kv_heads(H, H_kv);
   if (st != FA_OK) return st;
   // q, k, v, o, dO, dq, dk, dv: the caller's strides, or the packed ones
@@ -478,7 +512,7 @@ const char* fa_status_string(int status) {
     case FA_OK: return "ok";
     case FA_ERR_NULL: return "null pointer";
     case FA_ERR_SHAPE: return "bad shape (sizes >= 1, H a multiple of H_kv, N_q <= N_k, within launch limits)";
-    case FA_ERR_HEADDIM: return "unsupported head dimension (64 or 128)";
+    case FA_ERR_HEADDIM: return "unsupported head dimension (64 or 128; 256 for the forward and decode)";
     case FA_ERR_ALIGN: return "misaligned pointer (bf16 arrays 16 B, L 4 B)";
     case FA_ERR_MASK: return "bad mask (causal must be 0 or 1, window >= 0)";
     case FA_ERR_WORKSPACE: return "workspace missing or too small";
@@ -520,6 +554,7 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
                    void* stream) {
   if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FA_ERR_NULL;
   int st = check_problem(B, H, N, d, scale, causal, window);
+  if (st == FA_OK && d == 256) st = FA_ERR_HEADDIM;
   if (st != FA_OK) return st;
   const long long BH = (long long)B * H;
   if (BH * ((N + kBwdKeys - 1) / kBwdKeys) > 0x7fffffffLL || BH * padded_rows(N) > 0x7fffffffLL) return FA_ERR_SHAPE;

@@ -34,7 +34,9 @@ def extract(src: str, name: str) -> str:
     raise RuntimeError(f"unbalanced braces in {name}")
 
 
-def build(out_dir: str, kernel_header: str, harness: str, exe_name: str, defines=()) -> str:
+def build(out_dir: str, kernel_header, harness: str, exe_name: str, defines=()) -> str:
+    """kernel_header: one header name, or a list (a kernel header and the headers it includes)."""
+    headers = [kernel_header] if isinstance(kernel_header, str) else list(kernel_header)
     gxx = shutil.which("g++")
     if gxx is None:
         raise FileNotFoundError("g++")
@@ -44,7 +46,8 @@ def build(out_dir: str, kernel_header: str, harness: str, exe_name: str, defines
         f.write("// cut from sm100.cuh by tests/host_emu/build_emu.py\n")
         for name in PURE_HELPERS:
             f.write(extract(real, name))
-    shutil.copy(os.path.join(CSRC, kernel_header), os.path.join(out_dir, kernel_header))
+    for h in headers:
+        shutil.copy(os.path.join(CSRC, h), os.path.join(out_dir, h))
     shutil.copy(os.path.join(HERE, "sm100_stub.cuh"), os.path.join(out_dir, "sm100.cuh"))
     shutil.copy(os.path.join(HERE, "emu.h"), os.path.join(out_dir, "emu.h"))
     shutil.copy(os.path.join(HERE, harness), os.path.join(out_dir, harness))

@@ -1,9 +1,15 @@
-// TEST INFRASTRUCTURE ONLY: runs fa_fwd_kernel<EMU_D> of fwd_kernel.cuh on the host through the
-// emulation of emu.h / sm100_stub.cuh, with the tensor maps and parameters fa_fwd_gqa derives
-// for packed [B, heads, N, d] arrays.
+// TEST INFRASTRUCTURE ONLY: runs fa_fwd_kernel<EMU_D> of fwd_kernel.cuh (or, with EMU_FWD256,
+// fa_fwd256_kernel of fwd256_kernel.cuh) on the host through the emulation of emu.h /
+// sm100_stub.cuh, with the tensor maps and parameters the library derives for packed
+// [B, heads, N, d] arrays.
 // usage: emu_fwd_main B H Hkv N causal window scale prefix   (prefix.q/.k/.v bf16; writes .o, .lse)
 #include "emu.h"
+#ifdef EMU_FWD256
+#include "fwd256_kernel.cuh"
+#define EMU_D 256
+#else
 #include "fwd_kernel.cuh"
+#endif
 
 #include <fstream>
 #include <string>
@@ -15,7 +21,11 @@
 namespace fa {
 // the kernel's dynamic shared memory: exactly one (1024-byte aligned) FwdSmem, so AddressSanitizer
 // sees any access past it
+#ifdef EMU_FWD256
+alignas(1024) uint8_t smem_raw[sizeof(Fwd256Smem)];
+#else
 alignas(1024) uint8_t smem_raw[sizeof(FwdSmem<EMU_D>)];
+#endif
 }  // namespace fa
 
 using namespace fa;
@@ -61,8 +71,13 @@ int main(int argc, char** argv) {
   auto v = read_file<uint16_t>(prefix + ".v", size_t(B) * Hkv * N * D);
   std::vector<uint16_t> o(size_t(B) * H * N * D, 0x7fc0);
   std::vector<float> lse(size_t(B) * H * N, NAN);
-  const CUtensorMap tq = make_map(q.data(), D, N, H, B, kBlockM), tk = make_map(k.data(), D, N, Hkv, B, kBlockN),
-                    tv = make_map(v.data(), D, N, Hkv, B, kBlockN);
+#ifdef EMU_FWD256
+  constexpr int box_q = k256BlockM, box_kv = k256BlockN;
+#else
+  constexpr int box_q = kBlockM, box_kv = kBlockN;
+#endif
+  const CUtensorMap tq = make_map(q.data(), D, N, H, B, box_q), tk = make_map(k.data(), D, N, Hkv, B, box_kv),
+                    tv = make_map(v.data(), D, N, Hkv, B, box_kv);
   FwdParams prm;
   prm.o = reinterpret_cast<__nv_bfloat16*>(o.data());
   prm.lse = lse.data();
@@ -71,14 +86,22 @@ int main(int argc, char** argv) {
   prm.H = H;
   prm.group = H / Hkv;
   prm.o_st = Strides{(long long)H * N * D, (long long)N * D, (long long)D};
+#ifdef EMU_FWD256
+  prm.n_pairs = (N + k256BlockM - 1) / k256BlockM;   // query tiles per head
+#else
   prm.n_pairs = ((N + kBlockM - 1) / kBlockM + kQTiles - 1) / kQTiles;
+#endif
   prm.causal = causal;
   prm.window = window > N ? N : window;
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.wait_limit_ns = 60ull * 1000000000ull;
   const unsigned grid = unsigned(prm.n_pairs) * unsigned(B * H);
-  std::printf("grid %u smem %zu\n", grid, sizeof(FwdSmem<D>));
-  emu_launch(grid, kFwdThreads, sizeof(FwdSmem<D>), [&] { fa_fwd_kernel<D>(tq, tk, tv, prm); }, fa::smem_raw);
+  std::printf("grid %u smem %zu\n", grid, sizeof(fa::smem_raw));
+#ifdef EMU_FWD256
+  emu_launch(grid, k256Threads, sizeof(fa::smem_raw), [&] { fa_fwd256_kernel(tq, tk, tv, prm); }, fa::smem_raw);
+#else
+  emu_launch(grid, kFwdThreads, sizeof(fa::smem_raw), [&] { fa_fwd_kernel<D>(tq, tk, tv, prm); }, fa::smem_raw);
+#endif
   if (g_status != 0) { std::fprintf(stderr, "device status %d\n", g_status); return 3; }
   write_file(prefix + ".o", o);
   write_file(prefix + ".lse", lse);

@@ -49,7 +49,7 @@ def _fwd(**kw):
     (dict(N=0), "FA_ERR_SHAPE"),
     (dict(B=1 << 20, H=1 << 20), "FA_ERR_SHAPE"),
     (dict(d=96), "FA_ERR_HEADDIM"),
-    (dict(d=256), "FA_ERR_HEADDIM"),
+    (dict(d=512), "FA_ERR_HEADDIM"),
     (dict(window=-1, causal=1), "FA_ERR_MASK"),
     (dict(causal=2), "FA_ERR_MASK"),
     (dict(scale=0.0), "FA_ERR_SCALE"),
@@ -228,3 +228,15 @@ def test_decode_fp8kv_code_strides_are_16_byte_multiples(lib):
     arr = (_lib.FaStrides * 4)(*good)
     arr[1] = _lib.FaStrides(2 * 4096 * 136, 4096 * 136, 136)      # K rows padded by 8 codes
     assert _lib.STATUS_NAMES[_dec8(strides=ctypes.addressof(arr))] == "FA_ERR_ALIGN"
+
+
+def test_head_dim_256_is_forward_only(lib):
+    """The forward and decode take d = 256; the backward, its workspace size and the no-alloc
+    backward refuse it."""
+    assert _lib.fa_bwd_workspace_size(1, 2, 128, 256) == 0
+    assert _lib.STATUS_NAMES[_bwd(d=256)] == "FA_ERR_HEADDIM"
+    ptrs = [A + 4096 * i for i in range(9)]
+    st = _lib.fa_bwd_noalloc(*ptrs, 1, 2, 128, 256, 0.125, 0, 0, None)
+    assert _lib.STATUS_NAMES[st] == "FA_ERR_HEADDIM"
+    st = _lib.fa_bwd_gqa(*ptrs, 1, 2, 1, 128, 256, 0.125, 0, 0, A + 65536, 1 << 30, 7, None)
+    assert _lib.STATUS_NAMES[st] == "FA_ERR_HEADDIM"

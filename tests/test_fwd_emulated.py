@@ -1,5 +1,6 @@
-"""The tcgen05 forward kernel's own CUDA source, run on the CPU under an emulation of its
-primitives, vs the oracle.
+"""The tcgen05 forward kernels' own CUDA source (fa_fwd_kernel at d = 64 and 128,
+fa_fwd256_kernel at d = 256), run on the CPU under an emulation of their primitives, vs the
+oracle.
 
 Test infrastructure only.  tests/host_emu/sm100_stub.cuh restates the documented behaviour of
 the sm_100a primitives fwd_kernel.cuh uses -- mbarrier phases and transaction counts, 4-D TMA
@@ -31,8 +32,11 @@ def emu_fwd(tmp_path_factory):
     from tests.host_emu.build_emu import build
     d = str(tmp_path_factory.mktemp("host_emu_fwd"))
     try:
-        return {D: build(d, "fwd_kernel.cuh", "emu_fwd_main.cpp", f"emu_fwd_{D}", defines=(f"EMU_D={D}",))
+        exes = {D: build(d, "fwd_kernel.cuh", "emu_fwd_main.cpp", f"emu_fwd_{D}", defines=(f"EMU_D={D}",))
                 for D in (64, 128)}
+        exes[256] = build(d, ["fwd256_kernel.cuh", "fwd_kernel.cuh"], "emu_fwd_main.cpp", "emu_fwd_256",
+                          defines=("EMU_FWD256",))
+        return exes
     except FileNotFoundError:
         pytest.skip("g++ not available")
 
@@ -47,6 +51,13 @@ CASES = [
     (1, 2, 2, 700, 64, False, 0),
     (2, 2, 1, 257, 64, True, 3),        # multi-query, narrow window, ragged
     (1, 1, 1, 1000, 64, True, 1),       # window 1: O = V
+    # head dimension 256 (fa_fwd256_kernel: one query tile per CTA, 64-key K/V tiles)
+    (1, 1, 1, 128, 256, True, 0),
+    (1, 2, 2, 300, 256, True, 0),
+    (1, 2, 2, 300, 256, False, 0),
+    (1, 2, 1, 520, 256, True, 100),
+    (1, 4, 2, 400, 256, False, 50),
+    (2, 2, 1, 257, 256, True, 3),
 ]
 
 
