@@ -34,6 +34,16 @@ def extract(src: str, name: str) -> str:
     raise RuntimeError(f"unbalanced braces in {name}")
 
 
+# Inline asm that a kernel header itself holds, replaced in the emulation's copy (only) by a
+# call to the stub's stand-in.  The library's sources are not changed.
+PATCHES = {
+    "bwd_kernel.cuh": [
+        (r'asm volatile\("cp\.async\.bulk\.shared::cluster\.global\.mbarrier::complete_tx::bytes.*?: "memory"\);',
+         "emu_bulk_load(dst, src, bytes, bar);"),
+    ],
+}
+
+
 def build(out_dir: str, kernel_header, harness: str, exe_name: str, defines=()) -> str:
     """kernel_header: one header name, or a list (a kernel header and the headers it includes)."""
     headers = [kernel_header] if isinstance(kernel_header, str) else list(kernel_header)
@@ -47,7 +57,14 @@ def build(out_dir: str, kernel_header, harness: str, exe_name: str, defines=()) 
         for name in PURE_HELPERS:
             f.write(extract(real, name))
     for h in headers:
-        shutil.copy(os.path.join(CSRC, h), os.path.join(out_dir, h))
+        with open(os.path.join(CSRC, h)) as f:
+            text = f.read()
+        for pattern, repl in PATCHES.get(h, []):
+            text, n = re.subn(pattern, repl, text, flags=re.S)
+            if n != 1:
+                raise RuntimeError(f"patch for {h} matched {n} times")
+        with open(os.path.join(out_dir, h), "w") as f:
+            f.write(text)
     shutil.copy(os.path.join(HERE, "sm100_stub.cuh"), os.path.join(out_dir, "sm100.cuh"))
     shutil.copy(os.path.join(HERE, "emu.h"), os.path.join(out_dir, "emu.h"))
     shutil.copy(os.path.join(HERE, harness), os.path.join(out_dir, harness))

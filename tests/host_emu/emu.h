@@ -28,6 +28,7 @@
 #define __noinline__
 #define __grid_constant__
 #define __shared__
+#define __align__(x) __attribute__((aligned(x)))
 using std::max;
 using std::min;
 
@@ -35,6 +36,7 @@ struct dim3s { unsigned x = 0, y = 0, z = 0; };
 inline thread_local dim3s threadIdx, blockIdx;
 struct float2 { float x, y; };
 struct float4 { float x, y, z, w; };
+inline float4 make_float4(float a, float b, float c, float d) { return {a, b, c, d}; }
 struct uint2 { uint32_t x, y; };
 struct uint4 { uint32_t x, y, z, w; };
 inline float2 make_float2(float a, float b) { return {a, b}; }
@@ -87,6 +89,11 @@ inline float __shfl_xor_sync(unsigned, float v, int m) {
   return r;
 }
 
+// width-limited xor shuffle: the partner is lane ^ m inside the lane's segment of `width`
+inline float __shfl_xor_sync(unsigned mask, float v, int m, int width) {
+  if (m >= width) { std::fprintf(stderr, "shuffle mask leaves its segment\n"); std::abort(); }
+  return __shfl_xor_sync(mask, v, m);
+}
 inline int __all_sync(unsigned, int pred) {
   WarpCtx& w = my_warp();
   int l = lane_id();

@@ -21,6 +21,7 @@
 // bf16 and f16 rounding is round-to-nearest-even (f16 with subnormals and overflow to
 // infinity); E4M3 codes decode by the format's definition (they are all f16 values).
 #pragma once
+#include <atomic>
 #include "emu.h"
 
 namespace fa {
@@ -44,6 +45,8 @@ inline float bf2f(uint16_t h) {
   return f;
 }
 inline uint32_t pack_bf16x2(float lo, float hi) { return uint32_t(f2bf(lo)) | (uint32_t(f2bf(hi)) << 16); }
+struct __nv_bfloat162 { uint16_t x, y; };
+inline float2 __bfloat1622float2(__nv_bfloat162 h) { return {bf2f(h.x), bf2f(h.y)}; }
 inline uint16_t f2h(float f) {
   uint32_t x;
   std::memcpy(&x, &f, 4);
@@ -376,6 +379,32 @@ inline void mma_bf16_ts_w(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc, ui
 }
 inline void mma_commit_w(uint32_t bar) {
   if (lane_id() == 0) mma_commit(bar);
+}
+
+// ------------------------------------------------------------ shared vectors, bulk copies, reductions
+inline uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  std::memcpy(&v, smem_at(addr, 16), 16);
+  return v;
+}
+inline void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  const uint4 v{a, b, c, d};
+  std::memcpy(smem_at(addr, 16), &v, 16);
+}
+// the untiled bulk copy global -> shared, completing its bytes on the barrier
+inline void emu_bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  if (dst % 16 || bytes % 16 || reinterpret_cast<uintptr_t>(src) % 16) {
+    std::fprintf(stderr, "bulk copy not 16-byte aligned\n");
+    std::abort();
+  }
+  std::memcpy(smem_at(dst, bytes), src, bytes);
+  bar_complete_tx(bar, bytes);
+}
+// red.global.add.v4.f32: four fp32 adds done atomically at the target
+inline void red_add_v4(float* addr, uint4 v) {
+  if (reinterpret_cast<uintptr_t>(addr) % 16) { std::fprintf(stderr, "vector reduction not 16-byte aligned\n"); std::abort(); }
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  for (int i = 0; i < 4; ++i) std::atomic_ref<float>(addr[i]).fetch_add(__uint_as_float(w[i]));
 }
 
 // ------------------------------------------------------------ packed fp32 pairs, max
