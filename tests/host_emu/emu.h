@@ -13,6 +13,7 @@
 #include <cstdio>
 #include <cstring>
 #include <chrono>
+#include <functional>
 #include <memory>
 #include <mutex>
 #include <thread>
@@ -64,6 +65,11 @@ struct BarState {
   uint32_t expected = 0, pending = 0, phase = 0;
   long long tx = 0;
 };
+// an asynchronous operation (TMA or bulk copy, MMA) not yet performed
+struct PendingOp {
+  uint32_t bar;                    // copies: the barrier that tracks them
+  std::function<void()> run;
+};
 struct BlockCtx {
   std::barrier<>* bar;
   unsigned char* smem;
@@ -72,6 +78,8 @@ struct BlockCtx {
   std::mutex* mu;                                    // guards bars
   std::unordered_map<uint32_t, BarState>* bars;
   uint32_t* tmem;                                    // 128 lanes x 512 columns
+  std::vector<PendingOp>* copies;                    // TMA / bulk copies issued, not yet landed
+  std::vector<PendingOp>* mmas;                      // MMAs issued, not yet executed (in order)
 };
 inline thread_local BlockCtx* g_blk = nullptr;
 inline int lane_id() { return threadIdx.x & 31; }
@@ -137,6 +145,7 @@ void emu_launch(unsigned grid, unsigned block, size_t smem_bytes, F call, unsign
     std::mutex mu;
     std::unordered_map<uint32_t, BarState> bars;
     std::vector<uint32_t> tmem(128 * 512, 0x7fc07fc0u);
+    std::vector<PendingOp> copies, mmas;
     std::barrier<> bar(block);
     std::vector<WarpCtx> warps(block / 32);
     std::vector<std::unique_ptr<std::barrier<>>> wb;
@@ -144,7 +153,7 @@ void emu_launch(unsigned grid, unsigned block, size_t smem_bytes, F call, unsign
       wb.emplace_back(new std::barrier<>(32));
       w.bar = wb.back().get();
     }
-    BlockCtx ctx{&bar, smem, &warps, smem_bytes, &mu, &bars, tmem.data()};
+    BlockCtx ctx{&bar, smem, &warps, smem_bytes, &mu, &bars, tmem.data(), &copies, &mmas};
     std::vector<std::thread> th;
     th.reserve(block);
     for (unsigned tx = 0; tx < block; ++tx)

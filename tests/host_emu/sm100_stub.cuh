@@ -15,7 +15,12 @@
 //               descriptor; operands read through SW128 shared-memory descriptors (K-major:
 //               8-row atoms SBO apart; MN-major: 64 MN-contiguous elements per row, 8-k atoms
 //               SBO apart, the next 64 MN elements LBO apart) or A from TMEM (bf16 pairs);
-//               executed when issued, so a commit arrives at once.  ldmatrix and mma.sync are emulated from the fragment layouts the PTX ISA
+//               queued when issued and executed, in issue order, at the issuing thread's
+//               next tcgen05.commit (a legal schedule: the hardware runs them asynchronously,
+//               in order, and the commit's barrier tracks their completion).
+// TMA and bulk copies likewise land only when some thread tests the barrier that tracks them,
+// so a consumer that reads shared memory or TMEM without waiting on the right barrier sees
+// stale (NaN-filled) data.  ldmatrix and mma.sync are emulated from the fragment layouts the PTX ISA
 // documents (m8n8 b16 matrices; m16n8k16 row.col bf16 with fp32 accumulators); cp.async is a
 // synchronous copy (zero-fill when the source size is 0); ex2 / lg2 are std::exp2 / std::log2;
 // bf16 and f16 rounding is round-to-nearest-even (f16 with subnormals and overflow to
@@ -230,7 +235,9 @@ inline void bar_complete_tx(uint32_t bar, uint32_t bytes) {
   b.tx -= bytes;
   bar_flip_if_done(b);
 }
+inline void land_copies(uint32_t bar);
 inline bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  land_copies(bar);
   std::lock_guard<std::mutex> lk(*g_blk->mu);
   return bar_state(bar).phase != (parity & 1u);
 }
@@ -261,9 +268,43 @@ struct CUtensorMap {
 };
 inline void tma_prefetch_desc(const CUtensorMap*) {}
 inline uint32_t sw128(uint32_t addr) { return addr ^ (((addr >> 7) & 7u) << 4); }
+// performs the copies issued so far that `bar` tracks (each completes its bytes on it)
+inline void land_copies(uint32_t bar) {
+  std::vector<std::function<void()>> todo;
+  {
+    std::lock_guard<std::mutex> lk(*g_blk->mu);
+    auto& q = *g_blk->copies;
+    for (auto it = q.begin(); it != q.end();) {
+      if (it->bar == bar) {
+        todo.push_back(std::move(it->run));
+        it = q.erase(it);
+      } else {
+        ++it;
+      }
+    }
+  }
+  for (auto& f : todo) f();
+}
+inline void queue_copy(uint32_t bar, std::function<void()> f) {
+  std::lock_guard<std::mutex> lk(*g_blk->mu);
+  g_blk->copies->push_back(PendingOp{bar, std::move(f)});
+}
+inline void tma_copy_now(uint32_t dst, CUtensorMap map, uint32_t bar, int x, int row, int head, int batch);
 inline void tma_load_rows(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int row, int head, int batch) {
   if (x % 8) { std::fprintf(stderr, "TMA x coordinate not 16-byte aligned\n"); std::abort(); }
   if (map->box_x != 64) { std::fprintf(stderr, "TMA box is not 64 elements wide\n"); std::abort(); }
+  smem_at(dst, size_t(map->box_rows) * 128);   // the destination must lie in shared memory
+  const CUtensorMap m = *map;
+  BlockCtx* blk = g_blk;
+  queue_copy(bar, [=] {
+    BlockCtx* saved = g_blk;
+    g_blk = blk;
+    tma_copy_now(dst, m, bar, x, row, head, batch);
+    g_blk = saved;
+  });
+}
+inline void tma_copy_now(uint32_t dst, CUtensorMap mm, uint32_t bar, int x, int row, int head, int batch) {
+  const CUtensorMap* map = &mm;
   for (uint32_t r = 0; r < map->box_rows; ++r)
     for (uint32_t c = 0; c < map->box_x; ++c) {
       const long long gx = (long long)x + c, gr = (long long)row + r;
@@ -367,9 +408,26 @@ inline void mma_exec(uint32_t d_tmem, uint64_t a_desc, uint32_t a_tmem_addr, uin
       cell = __float_as_uint(acc);
     }
 }
-inline void mma_bf16_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) { mma_exec(d, a, ~0u, b, idesc, acc); }
-inline void mma_bf16_ts(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc, uint32_t acc) { mma_exec(d, 0, a, b, idesc, acc); }
-inline void mma_commit(uint32_t bar) { mbar_arrive(bar); }
+inline void queue_mma(std::function<void()> f) {
+  std::lock_guard<std::mutex> lk(*g_blk->mu);
+  g_blk->mmas->push_back(PendingOp{0, std::move(f)});
+}
+inline void mma_bf16_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  queue_mma([=] { mma_exec(d, a, ~0u, b, idesc, acc); });
+}
+inline void mma_bf16_ts(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  queue_mma([=] { mma_exec(d, 0, a, b, idesc, acc); });
+}
+// the MMAs issued so far complete, in order, then the barrier sees one arrival
+inline void mma_commit(uint32_t bar) {
+  std::vector<PendingOp> todo;
+  {
+    std::lock_guard<std::mutex> lk(*g_blk->mu);
+    todo.swap(*g_blk->mmas);
+  }
+  for (auto& op : todo) op.run();
+  mbar_arrive(bar);
+}
 // warp-uniform forms: one elected lane issues
 inline void mma_bf16_ss_w(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
   if (lane_id() == 0) mma_bf16_ss(d, a, b, idesc, acc);
@@ -397,8 +455,11 @@ inline void emu_bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_
     std::fprintf(stderr, "bulk copy not 16-byte aligned\n");
     std::abort();
   }
-  std::memcpy(smem_at(dst, bytes), src, bytes);
-  bar_complete_tx(bar, bytes);
+  smem_at(dst, bytes);
+  queue_copy(bar, [=] {
+    std::memcpy(smem_at(dst, bytes), src, bytes);
+    bar_complete_tx(bar, bytes);
+  });
 }
 // red.global.add.v4.f32: four fp32 adds done atomically at the target
 inline void red_add_v4(float* addr, uint4 v) {
