@@ -76,7 +76,7 @@ def forward(q, k, v, scale: float | None = None, causal: bool = False, window: i
             out=None, lse=None):
     """O, L = attention(Q, K, V); O bf16 [B,H,N,d], L fp32 [B,H,N] (natural-log logsumexp).
 
-    d is 64, 128 or 256 (backward() takes 64 and 128 only)."""
+    d is 64, 128 or 256."""
     import torch
     H_kv = _check_qkv(q, k, v)
     B, H, N, d = q.shape

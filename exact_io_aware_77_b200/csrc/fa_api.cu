@@ -14,6 +14,7 @@
 #include "fwd_kernel.cuh"
 #include "fwd256_kernel.cuh"
 #include "bwd_kernel.cuh"
+#include "bwd256_kernel.cuh"
 #include "decode_ops.cuh"
 #include "decode_kernel.cuh"
 
@@ -92,7 +93,7 @@ int check_problem(int B, int H, int N, int d, float scale, int causal, int windo
   const long long bh = (long long)B * H;
   const long long tiles = (N + kBlockM - 1) / kBlockM;
   if (bh > 0x7fffffffLL || bh * tiles > 0x7fffffffLL) return FA_ERR_SHAPE;
-  if (d != 64 && d != 128 && d != 256) return FA_ERR_HEADDIM;   // 256: forward only (checked by the callers)
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_HEADDIM;
   if (!(causal == 0 || causal == 1) || window < 0) return FA_ERR_MASK;
   if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_SCALE;
   return FA_OK;
@@ -195,8 +196,9 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   }
   if (phases & kBwdPhaseMain) {
   CUtensorMap tq, tk, tv, tdo;
-  if (!make_map_bf16(&tq, q, D, N, H, B, st[0], kBwdRows) || !make_map_bf16(&tk, k, D, N, H_kv, B, st[1], kBwdKeys) ||
-      !make_map_bf16(&tv, v, D, N, H_kv, B, st[2], kBwdKeys) || !make_map_bf16(&tdo, dout, D, N, H, B, st[4], kBwdRows))
+  constexpr int box_keys = D == 256 ? kB256Keys : kBwdKeys;
+  if (!make_map_bf16(&tq, q, D, N, H, B, st[0], kBwdRows) || !make_map_bf16(&tk, k, D, N, H_kv, B, st[1], box_keys) ||
+      !make_map_bf16(&tv, v, D, N, H_kv, B, st[2], box_keys) || !make_map_bf16(&tdo, dout, D, N, H, B, st[4], kBwdRows))
     return FA_ERR_CUDA;
   BwdParams prm;
   prm.lp = lp;
@@ -218,11 +220,21 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.scale = scale;
   prm.wait_limit_ns = g_wait_limit_ns;
-  static_assert(sizeof(BwdSmem<D>) <= 232448, "backward shared memory exceeds 227 KB");
-  const int smem = int(sizeof(BwdSmem<D>));   // the kernel checks that the base is 1 KB aligned
-  if (set_smem(fa_bwd_kernel<D>, smem) != FA_OK) return FA_ERR_CUDA;
-  // one CTA per (K/V head, key tile)
-  fa_bwd_kernel<D><<<unsigned(prm.n_kv_tiles) * unsigned(BH_kv), kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, prm);
+  if constexpr (D == 256) {
+    // one CTA per (K/V head, 64-key tile, head-dim half): bwd256_kernel.cuh
+    prm.n_kv_tiles = (N + kB256Keys - 1) / kB256Keys;
+    static_assert(sizeof(Bwd256Smem) <= 232448, "d = 256 backward shared memory exceeds 227 KB");
+    const int smem = int(sizeof(Bwd256Smem));
+    if (set_smem(fa_bwd256_kernel, smem) != FA_OK) return FA_ERR_CUDA;
+    fa_bwd256_kernel<<<unsigned(prm.n_kv_tiles) * unsigned(BH_kv) * 2u, kB256Threads, smem, stream>>>(tq, tk, tv, tdo,
+                                                                                                         prm);
+  } else {
+    static_assert(sizeof(BwdSmem<D>) <= 232448, "backward shared memory exceeds 227 KB");
+    const int smem = int(sizeof(BwdSmem<D>));   // the kernel checks that the base is 1 KB aligned
+    if (set_smem(fa_bwd_kernel<D>, smem) != FA_OK) return FA_ERR_CUDA;
+    // one CTA per (K/V head, key tile)
+    fa_bwd_kernel<D><<<unsigned(prm.n_kv_tiles) * unsigned(BH_kv), kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, prm);
+  }
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   if (phases & kBwdPhaseFinal) {
@@ -379,7 +391,7 @@ int fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* 
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
-  if (d == 256 || check_problem(B, H, N, d, 1.f, 0, 0) != FA_OK) return 0;
+  if (check_problem(B, H, N, d, 1.f, 0, 0) != FA_OK) return 0;
   return bwd_workspace_bytes((long long)B * H, N, d);
 }
 
@@ -420,7 +432,6 @@ static int bwd_impl(const void* q, const void* k, const void* v, const void* o, 
   if (phases < 1 || phases > kBwdAllPhases) return FA_ERR_PHASES;
   if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FA_ERR_NULL;
   int st = check_problem(B, H, N, d, scale, causal, window);
-  if (st == FA_OK && d == 256) st = FA_ERR_HEADDIM;   // the backward has no d = 256 kernel
   if (st == FA_OK) st = check_kv_heads(H, H_kv);
   if (st != FA_OK) return st;
   // q, k, v, o, dO, dq, dk, dv: the caller's strides, or the packed ones
@@ -432,17 +443,20 @@ static int bwd_impl(const void* q, const void* k, const void* v, const void* o, 
       if (!strides_ok(s8[i])) return FA_ERR_ALIGN;
     }
   const long long BH = (long long)B * H;
-  if (BH * ((N + kBwdKeys - 1) / kBwdKeys) > 0x7fffffffLL || BH * padded_rows(N) > 0x7fffffffLL) return FA_ERR_SHAPE;
+  // grid: one CTA per 128-key tile (d = 256: per 64-key tile and head-dim half)
+  const long long bwd_ctas = d == 256 ? BH * ((N + kB256Keys - 1) / kB256Keys) * 2 : BH * ((N + kBwdKeys - 1) / kBwdKeys);
+  if (bwd_ctas > 0x7fffffffLL || BH * padded_rows(N) > 0x7fffffffLL) return FA_ERR_SHAPE;
   if (!workspace || workspace_bytes < bwd_workspace_bytes(BH, N, d)) return FA_ERR_WORKSPACE;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dout, 16) ||
       !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4) || !aligned(workspace, 16))
     return FA_ERR_ALIGN;
   if ((st = check_device()) != FA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return d == 64 ? launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, s8, scale, causal, window,
-                                  workspace, s, phases)
-                 : launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, s8, scale, causal, window,
-                                   workspace, s, phases);
+  switch (d) {
+    case 64: return launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, s8, scale, causal, window, workspace, s, phases);
+    case 128: return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, s8, scale, causal, window, workspace, s, phases);
+    default: return launch_bwd<256>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, s8, scale, causal, window, workspace, s, phases);
+  }
 }
 
 size_t fa_decode_workspace_size(int B, int H, int H_kv, int N_q, int N_k, int d, int causal, int window) {
@@ -512,7 +526,7 @@ const char* fa_status_string(int status) {
     case FA_OK: return "ok";
     case FA_ERR_NULL: return "null pointer";
     case FA_ERR_SHAPE: return "bad shape (sizes >= 1, H a multiple of H_kv, N_q <= N_k, within launch limits)";
-    case FA_ERR_HEADDIM: return "unsupported head dimension (64 or 128; 256 for the forward and decode)";
+    case FA_ERR_HEADDIM: return "unsupported head dimension (64, 128 or 256)";
     case FA_ERR_ALIGN: return "misaligned pointer (bf16 arrays 16 B, L 4 B)";
     case FA_ERR_MASK: return "bad mask (causal must be 0 or 1, window >= 0)";
     case FA_ERR_WORKSPACE: return "workspace missing or too small";
@@ -554,10 +568,11 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
                    void* stream) {
   if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FA_ERR_NULL;
   int st = check_problem(B, H, N, d, scale, causal, window);
-  if (st == FA_OK && d == 256) st = FA_ERR_HEADDIM;
   if (st != FA_OK) return st;
   const long long BH = (long long)B * H;
-  if (BH * ((N + kBwdKeys - 1) / kBwdKeys) > 0x7fffffffLL || BH * padded_rows(N) > 0x7fffffffLL) return FA_ERR_SHAPE;
+  // grid: one CTA per 128-key tile (d = 256: per 64-key tile and head-dim half)
+  const long long bwd_ctas = d == 256 ? BH * ((N + kB256Keys - 1) / kB256Keys) * 2 : BH * ((N + kBwdKeys - 1) / kBwdKeys);
+  if (bwd_ctas > 0x7fffffffLL || BH * padded_rows(N) > 0x7fffffffLL) return FA_ERR_SHAPE;
   if (bwd_workspace_bytes(BH, N, d) > kNoAllocScratchBytes) return FA_ERR_NOALLOC_LIMIT;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dout, 16) ||
       !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4))
@@ -572,8 +587,11 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const Strides s8[8] = {packed(H, N, d), packed(H, N, d), packed(H, N, d), packed(H, N, d),
                          packed(H, N, d), packed(H, N, d), packed(H, N, d), packed(H, N, d)};
-  return d == 64 ? launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H, N, s8, scale, causal, window, ws, s)
-                 : launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H, N, s8, scale, causal, window, ws, s);
+  switch (d) {
+    case 64: return launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H, N, s8, scale, causal, window, ws, s);
+    case 128: return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H, N, s8, scale, causal, window, ws, s);
+    default: return launch_bwd<256>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H, N, s8, scale, causal, window, ws, s);
+  }
 }
 
 }  // extern "C"

@@ -58,7 +58,7 @@ typedef enum {
   FA_OK = 0,
   FA_ERR_NULL = 1,       /* a required pointer is NULL */
   FA_ERR_SHAPE = 2,      /* a size < 1, H not a multiple of H_kv, N_q > N_k, or beyond the launch limits */
-  FA_ERR_HEADDIM = 3,    /* d is not 64 or 128 (or 256, where the forward and decode take it) */
+  FA_ERR_HEADDIM = 3,    /* d is not 64, 128 or 256 */
   FA_ERR_ALIGN = 4,      /* a bf16 array is not 16-byte aligned, or L not 4-byte aligned */
   FA_ERR_MASK = 5,       /* causal not 0/1, or window < 0 */
   FA_ERR_WORKSPACE = 6,  /* workspace missing or smaller than fa_bwd_ / fa_decode_workspace_size */
@@ -84,8 +84,7 @@ FA_EXPORT int fa_fwd(const void* q, const void* k, const void* v, void* o, float
 /*
  * Bytes of device workspace fa_bwd needs: 4 * B*H * Np * (d + 2) with Np = N rounded up to
  * a multiple of 128 (per row: D, L in log2 units, and a d-wide fp32 dQ accumulator).
- * Returns 0 when the shape itself is invalid (d = 256 included: the backward does not take it).
- * O(N * d): no N x N buffer.
+ * Returns 0 when the shape itself is invalid.  O(N * d): no N x N buffer.
  */
 FA_EXPORT size_t fa_bwd_workspace_size(int B, int H, int N, int d);
 
@@ -96,7 +95,9 @@ FA_EXPORT size_t fa_bwd_workspace_size(int B, int H, int N, int d);
  * `workspace` (device, caller-owned, 16-byte aligned, at least fa_bwd_workspace_size bytes)
  * is scratch: it is overwritten and may be reused once the call's work has completed on
  * `stream`.  Three kernels are enqueued: D = rowsum(dO o O) with a cleared accumulator, the
- * fused recompute kernel, and the dQ scaling.  d must be 64 or 128 (FA_ERR_HEADDIM for 256).
+ * fused recompute kernel, and the dQ scaling.  d must be 64, 128 or 256; d = 256 runs a kernel of
+ * its own (one CTA per 64-key tile and head-dim half), checked in a host emulation of its
+ * primitives but not yet run on a B200.
  */
 FA_EXPORT int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
                      void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal, int window,

@@ -4,7 +4,12 @@
 // usage: emu_bwd_main B H Hkv N causal window scale prefix
 //   reads prefix.q .k .v .o .do (bf16) and .lse (fp32); writes prefix.dq .dk .dv (bf16)
 #include "emu.h"
+#ifdef EMU_BWD256
+#include "bwd256_kernel.cuh"
+#define EMU_D 256
+#else
 #include "bwd_kernel.cuh"
+#endif
 
 #include <fstream>
 #include <string>
@@ -14,7 +19,11 @@
 #endif
 
 namespace fa {
+#ifdef EMU_BWD256
+alignas(1024) uint8_t smem_raw[sizeof(Bwd256Smem)];
+#else
 alignas(1024) uint8_t smem_raw[sizeof(BwdSmem<EMU_D>)];
+#endif
 }  // namespace fa
 
 using namespace fa;
@@ -77,8 +86,13 @@ int main(int argc, char** argv) {
     fa_bwd_prep<D>(reinterpret_cast<const __nv_bfloat16*>(o.data()), reinterpret_cast<const __nv_bfloat16*>(dout.data()),
                    lse.data(), lp, dd, dq_acc, N, Np, H, st_q, st_q, prep_rows);
   });
-  const CUtensorMap tq = make_map(q.data(), D, N, H, B, kBwdRows), tk = make_map(k.data(), D, N, Hkv, B, kBwdKeys),
-                    tv = make_map(v.data(), D, N, Hkv, B, kBwdKeys), tdo = make_map(dout.data(), D, N, H, B, kBwdRows);
+#ifdef EMU_BWD256
+  constexpr int box_keys = kB256Keys;
+#else
+  constexpr int box_keys = kBwdKeys;
+#endif
+  const CUtensorMap tq = make_map(q.data(), D, N, H, B, kBwdRows), tk = make_map(k.data(), D, N, Hkv, B, box_keys),
+                    tv = make_map(v.data(), D, N, Hkv, B, box_keys), tdo = make_map(dout.data(), D, N, H, B, kBwdRows);
   BwdParams prm;
   prm.lp = lp;
   prm.dd = dd;
@@ -93,14 +107,19 @@ int main(int argc, char** argv) {
   prm.group = H / Hkv;
   prm.dk_st = st_kv;
   prm.dv_st = st_kv;
-  prm.n_kv_tiles = (N + kBwdKeys - 1) / kBwdKeys;
+  prm.n_kv_tiles = (N + box_keys - 1) / box_keys;
   prm.causal = causal;
   prm.window = window > N ? N : window;
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.scale = scale;
   prm.wait_limit_ns = 60ull * 1000000000ull;
+#ifdef EMU_BWD256
+  emu_launch(unsigned(prm.n_kv_tiles) * unsigned(BH_kv) * 2u, kB256Threads, sizeof(fa::smem_raw),
+             [&] { fa_bwd256_kernel(tq, tk, tv, tdo, prm); }, fa::smem_raw);
+#else
   emu_launch(unsigned(prm.n_kv_tiles) * unsigned(BH_kv), kBwdThreads, sizeof(fa::smem_raw),
              [&] { fa_bwd_kernel<D>(tq, tk, tv, tdo, prm); }, fa::smem_raw);
+#endif
   if (g_status != 0) { std::fprintf(stderr, "device status %d\n", g_status); return 3; }
   const long long rows = (long long)BH * N;
   emu_launch(unsigned((rows + (256 / G) - 1) / (256 / G)), 256, 0, [&] {

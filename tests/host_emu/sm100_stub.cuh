@@ -51,6 +51,7 @@ inline float bf2f(uint16_t h) {
 }
 inline uint32_t pack_bf16x2(float lo, float hi) { return uint32_t(f2bf(lo)) | (uint32_t(f2bf(hi)) << 16); }
 struct __nv_bfloat162 { uint16_t x, y; };
+inline __nv_bfloat16 __float2bfloat16_rn(float f) { return __nv_bfloat16{f2bf(f)}; }
 inline float2 __bfloat1622float2(__nv_bfloat162 h) { return {bf2f(h.x), bf2f(h.y)}; }
 inline uint16_t f2h(float f) {
   uint32_t x;

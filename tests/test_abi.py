@@ -230,13 +230,8 @@ def test_decode_fp8kv_code_strides_are_16_byte_multiples(lib):
     assert _lib.STATUS_NAMES[_dec8(strides=ctypes.addressof(arr))] == "FA_ERR_ALIGN"
 
 
-def test_head_dim_256_is_forward_only(lib):
-    """The forward and decode take d = 256; the backward, its workspace size and the no-alloc
-    backward refuse it."""
-    assert _lib.fa_bwd_workspace_size(1, 2, 128, 256) == 0
-    assert _lib.STATUS_NAMES[_bwd(d=256)] == "FA_ERR_HEADDIM"
-    ptrs = [A + 4096 * i for i in range(9)]
-    st = _lib.fa_bwd_noalloc(*ptrs, 1, 2, 128, 256, 0.125, 0, 0, None)
-    assert _lib.STATUS_NAMES[st] == "FA_ERR_HEADDIM"
-    st = _lib.fa_bwd_gqa(*ptrs, 1, 2, 1, 128, 256, 0.125, 0, 0, A + 65536, 1 << 30, 7, None)
-    assert _lib.STATUS_NAMES[st] == "FA_ERR_HEADDIM"
+def test_head_dim_256_workspace(lib):
+    """d = 256 has a backward too (bwd256_kernel.cuh): the same workspace formula."""
+    for B, H, N in ((1, 2, 128), (2, 4, 300)):
+        np_ = (N + 127) // 128 * 128
+        assert _lib.fa_bwd_workspace_size(B, H, N, 256) == 4 * B * H * np_ * (256 + 2)

@@ -1,5 +1,6 @@
-"""The backward kernels' own CUDA source (fa_bwd_prep, fa_bwd_kernel<D>, fa_bwd_dq_final), run on
-the CPU under the emulation of tests/host_emu/, vs the oracle's gradients.
+"""The backward kernels' own CUDA source (fa_bwd_prep, fa_bwd_kernel<D> at d = 64/128,
+fa_bwd256_kernel at d = 256, fa_bwd_dq_final), run on the CPU under the emulation of
+tests/host_emu/, vs the oracle's gradients.
 
 Test infrastructure only (see tests/test_fwd_emulated.py for what the emulation restates).
 The one inline-asm helper bwd_kernel.cuh holds itself (the untiled bulk copy) is replaced, in
@@ -26,8 +27,11 @@ def emu_bwd(tmp_path_factory):
     from tests.host_emu.build_emu import build
     d = str(tmp_path_factory.mktemp("host_emu_bwd"))
     try:
-        return {D: build(d, "bwd_kernel.cuh", "emu_bwd_main.cpp", f"emu_bwd_{D}", defines=(f"EMU_D={D}",))
+        exes = {D: build(d, "bwd_kernel.cuh", "emu_bwd_main.cpp", f"emu_bwd_{D}", defines=(f"EMU_D={D}",))
                 for D in (64, 128)}
+        exes[256] = build(d, ["bwd256_kernel.cuh", "bwd_kernel.cuh"], "emu_bwd_main.cpp", "emu_bwd_256",
+                          defines=("EMU_BWD256",))
+        return exes
     except FileNotFoundError:
         pytest.skip("g++ not available")
 
@@ -38,6 +42,10 @@ CASES = [
     (1, 4, 2, 400, 128, False, 50),    # two-sided window, two query heads per K/V head
     (2, 2, 1, 257, 64, True, 3),       # multi-query, narrow causal window
     (1, 1, 1, 600, 64, True, 1),       # window 1: dQ = dK = 0, dV = dO
+    # head dimension 256 (fa_bwd256_kernel: 64-key tiles, one CTA per head-dim half)
+    (1, 1, 1, 128, 256, True, 0),
+    (1, 1, 1, 300, 256, True, 1),
+    (1, 2, 2, 300, 256, False, 0),
 ]
 
 
