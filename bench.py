@@ -41,7 +41,8 @@ WORKLOAD = "causal"          # forward workload; the backward uses the same shap
 GRAD_WORKLOAD = "bwd"
 # --workload choices: the forward workload and the one whose dO seed the backward uses
 BENCH_WORKLOADS = {"causal": ("causal", "bwd"), "long": ("long", "long"), "swa": ("swa", "swa"),
-                   "gqa": ("gqa", "gqa"), "decode": ("decode", "decode"), "decode_fp8": ("decode", "decode")}
+                   "gqa": ("gqa", "gqa"), "decode": ("decode", "decode"), "decode_fp8": ("decode", "decode"),
+                   "d256": ("d256", "d256")}
 FLUSH_BYTES = 256 << 20      # > 126 MB L2
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -62,7 +63,8 @@ def parse_args():
                          "long / swa: N32768 with a one- / two-sided window of 4096, FLOPs counted over "
                          "the pairs the band keeps; decode: one new row per query head over 32768 "
                          "cached keys (B8, 64 query heads on 8 K/V heads), forward only, HBM-bound; "
-                         "decode_fp8: the same over an E4M3 K/V cache with per-tensor scales")
+                         "decode_fp8: the same over an E4M3 K/V cache with per-tensor scales; "
+                         "d256: B2 H16 N4096 head dimension 256, causal, forward+backward")
     return ap.parse_args()
 
 
@@ -121,6 +123,13 @@ def decode_bytes(B, H, H_kv, n_q, n_k, d, causal, window=0, kv_elem_bytes=2) -> 
     _, hi = decode_band(n_k - 1, n_k, causal, window)
     keys = hi - lo + 1
     return 2 * B * H * n_q * d * 2 + 2 * B * H_kv * keys * d * kv_elem_bytes + B * H * n_q * 4
+
+
+def kernel_names(d: int):
+    """(forward kernel, backward main kernel) names for head dimension d."""
+    if d == 256:
+        return "fa_fwd256_kernel", "fa_bwd256_kernel"
+    return f"fa_fwd_kernel<{d}>", f"fa_bwd_kernel<{d}>"
 
 
 def max_over_ranks(values, device=None):
@@ -376,9 +385,9 @@ def run_ours(args):
     main_ms_avg = main_total / args.steps
     if has_bwd and main_ms_avg > fwd_ms_avg:
         # the backward's conventional FLOPs are all tensor work of the recompute kernel
-        dom, dom_flops, dom_ms = "fa_bwd_kernel<128>", f_bwd, main_ms_avg
+        dom, dom_flops, dom_ms = kernel_names(d)[1], f_bwd, main_ms_avg
     else:
-        dom, dom_flops, dom_ms = "fa_fwd_kernel<128>", f_fwd, fwd_ms_avg
+        dom, dom_flops, dom_ms = kernel_names(d)[0], f_fwd, fwd_ms_avg
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 1),
                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
@@ -414,9 +423,9 @@ def run_ours(args):
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": args.steps * (1 + (3 if has_bwd else 0)),
-        "kernel_ms": {"fa_fwd_kernel<128>": round(fwd_ms_avg, 4),
-                      "fa_bwd_prep+fa_bwd_kernel+fa_bwd_dq_final": round(bwd_ms_avg, 4),
-                      "fa_bwd_kernel<128>": round(main_ms_avg, 4)} if has_bwd else None,
+        "kernel_ms": {kernel_names(d)[0]: round(fwd_ms_avg, 4),
+                      "fa_bwd_prep+" + kernel_names(d)[1] + "+fa_bwd_dq_final": round(bwd_ms_avg, 4),
+                      kernel_names(d)[1]: round(main_ms_avg, 4)} if has_bwd else None,
         "clocks": clocks,
     }
     if has_bwd:

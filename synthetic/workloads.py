@@ -82,6 +82,9 @@ WORKLOADS: dict[str, Workload] = {
     # the causal LLM shape with 8 K/V heads for 32 query heads (grouped-query attention)
     "gqa": Workload("gqa", 2, 32, 4096, 128, causal=True, std=0.5, seed=1007, grad_seed=2007, H_kv=8,
                     description="causal B2 H32 (8 K/V heads) N4096 d128"),
+    # head dimension 256 (the pages list it among what FlashAttention-2 supports)
+    "d256": Workload("d256", 2, 16, 4096, 256, causal=True, std=0.5, seed=1010, grad_seed=2010,
+                     description="causal B2 H16 N4096 d256"),
     # one generation step over a key/value cache: one new row per query head, 64 query heads
     # on 8 K/V heads (a 70B-class grouped-query layout), 32768 cached positions
     "decode": Workload("decode", 8, 64, 32768, 128, causal=True, seed=1008, H_kv=8, Nq=1,

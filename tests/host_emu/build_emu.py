@@ -76,3 +76,17 @@ def build(out_dir: str, kernel_header, harness: str, exe_name: str, defines=()) 
     if r.returncode != 0:
         raise RuntimeError("host emulation does not compile:\n" + r.stderr[-6000:])
     return exe
+
+
+def build_many(out_dir: str, jobs) -> dict:
+    """Build several emulation binaries at once: jobs = {key: (kernel_header(s), harness, exe_name,
+    defines)}; returns {key: path}.  The g++ runs overlap (they are independent processes)."""
+    from concurrent.futures import ThreadPoolExecutor
+    # each build gets its own directory, so the copies the builds write never collide
+    with ThreadPoolExecutor(max_workers=min(4, len(jobs))) as pool:
+        futures = {}
+        for i, (key, (hdr, harness, exe, defines)) in enumerate(jobs.items()):
+            sub = os.path.join(out_dir, f"b{i}")
+            os.makedirs(sub, exist_ok=True)
+            futures[key] = pool.submit(build, sub, hdr, harness, exe, defines)
+        return {key: f.result() for key, f in futures.items()}

@@ -24,14 +24,14 @@ from tests.parity import GRAD_REL_L2, rel_l2
 
 @pytest.fixture(scope="module")
 def emu_bwd(tmp_path_factory):
-    from tests.host_emu.build_emu import build
+    from tests.host_emu.build_emu import build_many
     d = str(tmp_path_factory.mktemp("host_emu_bwd"))
     try:
-        exes = {D: build(d, "bwd_kernel.cuh", "emu_bwd_main.cpp", f"emu_bwd_{D}", defines=(f"EMU_D={D}",))
-                for D in (64, 128)}
-        exes[256] = build(d, ["bwd256_kernel.cuh", "bwd_kernel.cuh"], "emu_bwd_main.cpp", "emu_bwd_256",
-                          defines=("EMU_BWD256",))
-        return exes
+        return build_many(d, {
+            64: ("bwd_kernel.cuh", "emu_bwd_main.cpp", "emu_bwd_64", ("EMU_D=64",)),
+            128: ("bwd_kernel.cuh", "emu_bwd_main.cpp", "emu_bwd_128", ("EMU_D=128",)),
+            256: (["bwd256_kernel.cuh", "bwd_kernel.cuh"], "emu_bwd_main.cpp", "emu_bwd_256", ("EMU_BWD256",)),
+        })
     except FileNotFoundError:
         pytest.skip("g++ not available")
 

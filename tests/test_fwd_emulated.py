@@ -29,14 +29,14 @@ from tests.parity import L_MAX_ABS, O_MAX_ABS, O_MEAN_ABS
 
 @pytest.fixture(scope="module")
 def emu_fwd(tmp_path_factory):
-    from tests.host_emu.build_emu import build
+    from tests.host_emu.build_emu import build_many
     d = str(tmp_path_factory.mktemp("host_emu_fwd"))
     try:
-        exes = {D: build(d, "fwd_kernel.cuh", "emu_fwd_main.cpp", f"emu_fwd_{D}", defines=(f"EMU_D={D}",))
-                for D in (64, 128)}
-        exes[256] = build(d, ["fwd256_kernel.cuh", "fwd_kernel.cuh"], "emu_fwd_main.cpp", "emu_fwd_256",
-                          defines=("EMU_FWD256",))
-        return exes
+        return build_many(d, {
+            64: ("fwd_kernel.cuh", "emu_fwd_main.cpp", "emu_fwd_64", ("EMU_D=64",)),
+            128: ("fwd_kernel.cuh", "emu_fwd_main.cpp", "emu_fwd_128", ("EMU_D=128",)),
+            256: (["fwd256_kernel.cuh", "fwd_kernel.cuh"], "emu_fwd_main.cpp", "emu_fwd_256", ("EMU_FWD256",)),
+        })
     except FileNotFoundError:
         pytest.skip("g++ not available")
 
