@@ -6,17 +6,22 @@
 // leave no room for a ring next to two Q tiles.  Here:
 //   one CTA per 128-row query tile of one head (192 threads);
 //   K/V tiles of 64 keys (32 KB), four of them in the shared-memory ring next to Q (64 KB);
-//   TMEM: S [0, 64) (P over its first 32 columns as bf16 pairs), O [256, 512).
+//   TMEM: two S buffers, S_0 [0, 64) and S_1 [64, 128) (P over the first 32 columns of its S
+//   as bf16 pairs), O [256, 512).  Tile j uses S_(j % 2).
 //   warp 4      TMA producer and TMEM owner: Q once, then K_j, V_j through the ring.
-//   warp 5      MMA issuer: S(j) = Q K_j^T (16 k-steps, N = 64), then after the softmax
-//               O += P(j) V_j (4 k-steps of 16 keys, N = 256), with S(j+1) issued right behind
-//               it: MMAs from one thread run in order, so S(j+1) overwrites P(j) only after
-//               PV(j) has read it.
+//   warp 5      MMA issuer, per tile j: S(j+1) = Q K_{j+1}^T into the other buffer first
+//               (16 k-steps, N = 64), so that it runs while the softmax works on S(j); then,
+//               once P(j) is in TMEM, O += P(j) V_j (4 k-steps of 16 keys, N = 256).  MMAs from
+//               one thread run in order, so S(j+1) overwrites S_(j+1 % 2) only after PV(j-1) has
+//               read the P that was there.
 //   warps 0-3   softmax: thread t owns row t (TMEM lane t), as in fa_fwd_kernel: running max
 //               (updated lazily, O rescaled only when it grows by more than 2^8), running sum,
-//               P = 2^(S c - m) to bf16 into TMEM, and at the end O / l and L.
-// With one query tile per CTA the tensor pipe waits for each tile's softmax (no ping-pong
-// between two tiles); the products per tile are twice those at d = 128.
+//               P = 2^(S c - m) to bf16 into TMEM, and at the end O / l and L.  Since S(j+1)
+//               is issued before PV(j), S(j+1) completing no longer implies PV(j) completed: a
+//               tile that rescales O first waits for the previous PV (pv_done).
+// With one query tile per CTA the two S buffers take the place of fa_fwd_kernel's ping-pong
+// between two query tiles: the tensor pipe computes S(j+1) during softmax(j) and PV(j) during
+// softmax(j+1).
 #pragma once
 
 #include <type_traits>
@@ -42,7 +47,7 @@ struct Fwd256Smem {
   alignas(1024) uint8_t kv[k256Slots][kTileBytes];
   alignas(8) uint64_t q_full;
   uint64_t slot_full[k256Slots], slot_empty[k256Slots];
-  uint64_t s_full, p_full, o_final, mma_drain;
+  uint64_t s_full[2], p_full[2], pv_done, o_final, mma_drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -83,8 +88,11 @@ __global__ void __launch_bounds__(k256Threads, 1)
       mbar_init(smem_u32(&sm.slot_full[s]), 1);
       mbar_init(smem_u32(&sm.slot_empty[s]), 1);
     }
-    mbar_init(smem_u32(&sm.s_full), 1);
-    mbar_init(smem_u32(&sm.p_full), k256BlockM);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&sm.s_full[b]), 1);
+      mbar_init(smem_u32(&sm.p_full[b]), k256BlockM);
+    }
+    mbar_init(smem_u32(&sm.pv_done), 1);
     mbar_init(smem_u32(&sm.o_final), 1);
     mbar_init(smem_u32(&sm.mma_drain), 1);
     fence_mbar_init();
@@ -140,23 +148,23 @@ __global__ void __launch_bounds__(k256Threads, 1)
     // one 8 KB chunk further (LBO), 8 keys per 1024-byte atom (SBO)
     const uint64_t dv0 = sw128_desc(smem_u32(sm.kv[0]), Smem::kKvChunk, 1024);
     int pv_count = 0;
-    auto issue_s = [&](uint32_t slot) {
+    auto issue_s = [&](uint32_t slot, int buf) {
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         // 16-element k-steps are 32 bytes apart inside a 128-byte row; 64-element chunks are
         // separate 16 KB (Q) or 8 KB (K) blocks
         const uint32_t qoff = (kk >> 2) * Smem::kQChunk + (kk & 3) * 32;
         const uint32_t koff = slot * Smem::kTileBytes + (kk >> 2) * Smem::kKvChunk + (kk & 3) * 32;
-        mma_bf16_ss_w(tmem, desc_advance(dq, qoff), desc_advance(dk0, koff), idesc_s, kk > 0);
+        mma_bf16_ss_w(tmem + 64 * buf, desc_advance(dq, qoff), desc_advance(dk0, koff), idesc_s, kk > 0);
       }
-      mma_commit_w(smem_u32(&sm.s_full));
+      mma_commit_w(smem_u32(&sm.s_full[buf]));
     };
-    auto issue_pv = [&](uint32_t slot) {
+    auto issue_pv = [&](uint32_t slot, int buf) {
       const uint64_t dv = desc_advance(dv0, slot * Smem::kTileBytes);
       const uint32_t acc = pv_count > 0;
 #pragma unroll
       for (int kk = 0; kk < k256BlockN / 16; ++kk)
-        mma_bf16_ts_w(tmem + 256, tmem + kk * 8, desc_advance(dv, kk * 2048), idesc_o, kk > 0 ? 1u : acc);
+        mma_bf16_ts_w(tmem + 256, tmem + 64 * buf + kk * 8, desc_advance(dv, kk * 2048), idesc_o, kk > 0 ? 1u : acc);
       ++pv_count;
     };
     bool ok = t_end > t_begin && wait(smem_u32(&sm.q_full), 0);
@@ -164,23 +172,26 @@ __global__ void __launch_bounds__(k256Threads, 1)
       ok = wait(smem_u32(&sm.slot_full[0]), 0);
       if (ok) {
         tc_fence_after();
-        issue_s(0);
+        issue_s(0, 0);
         mma_commit_w(smem_u32(&sm.slot_empty[0]));
       }
     }
     for (int t = t_begin; ok && t < t_end; ++t) {
-      const int Lv = 2 * (t - t_begin) + 1;   // V of tile t
-      const int Lk = Lv + 1;                  // K of tile t + 1
-      const bool has_next = t + 1 < t_end;
-      if (!wait(smem_u32(&sm.slot_full[Lv % k256Slots]), (Lv / k256Slots) & 1)) break;
-      if (has_next && !wait(smem_u32(&sm.slot_full[Lk % k256Slots]), (Lk / k256Slots) & 1)) break;
-      if (!wait(smem_u32(&sm.p_full), pv_count & 1)) break;
-      tc_fence_after();
-      issue_pv(Lv % k256Slots);
-      if (has_next) {
-        issue_s(Lk % k256Slots);
+      const int k = t - t_begin;
+      const int Lv = 2 * k + 1;   // V of tile t
+      const int Lk = Lv + 1;      // K of tile t + 1
+      if (t + 1 < t_end) {
+        // S of the next tile into the other buffer, ahead of this tile's PV
+        if (!wait(smem_u32(&sm.slot_full[Lk % k256Slots]), (Lk / k256Slots) & 1)) break;
+        tc_fence_after();
+        issue_s(Lk % k256Slots, (k + 1) & 1);
         mma_commit_w(smem_u32(&sm.slot_empty[Lk % k256Slots]));
       }
+      if (!wait(smem_u32(&sm.slot_full[Lv % k256Slots]), (Lv / k256Slots) & 1)) break;
+      if (!wait(smem_u32(&sm.p_full[k & 1]), (k >> 1) & 1)) break;
+      tc_fence_after();
+      issue_pv(Lv % k256Slots, k & 1);
+      mma_commit_w(smem_u32(&sm.pv_done));
       mma_commit_w(smem_u32(&sm.slot_empty[Lv % k256Slots]));
     }
     mma_commit_w(smem_u32(&sm.o_final));
@@ -191,7 +202,6 @@ __global__ void __launch_bounds__(k256Threads, 1)
     const int row = threadIdx.x;   // == TMEM lane
     const int qi = q0 + row;
     const uint32_t lane_base = uint32_t(warp * 32) << 16;
-    const uint32_t s_col = tmem + lane_base;
     const uint32_t o_col = tmem + lane_base + 256;
     const float c = prm.scale_log2;
     bool ok = true;
@@ -200,7 +210,9 @@ __global__ void __launch_bounds__(k256Threads, 1)
     auto step = [&](const int t, auto masked) -> bool {
       const int k = t - t_begin;
       const int kv0 = t * k256BlockN;
-      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.s_full), k & 1, abort, lim))) return false;
+      const int buf = k & 1;
+      const uint32_t s_col = tmem + lane_base + 64 * buf;
+      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.s_full[buf]), (k >> 1) & 1, abort, lim))) return false;
       tc_fence_after();
       float sv[k256BlockN];
       {
@@ -277,7 +289,10 @@ __global__ void __launch_bounds__(k256Threads, 1)
       l = l * alpha + sum;
       m = m_new;
       if (k > 0 && __any_sync(0xffffffffu, grow)) {
-        // PV of the previous tile completed before this S did (in-order MMAs): O is stable
+        // S(k) was issued before PV(k-1), so wait for PV(k-1) before touching O (S(k) completing
+        // does imply PV(k-2) completed, so the phase of parity (k-1) & 1 is the right one)
+        if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.pv_done), (k - 1) & 1, abort, lim))) return false;
+        tc_fence_after();
 #pragma unroll
         for (int ch = 0; ch < D / 32; ++ch) {
           uint32_t r[32];
@@ -289,7 +304,7 @@ __global__ void __launch_bounds__(k256Threads, 1)
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(smem_u32(&sm.p_full));
+      mbar_arrive(smem_u32(&sm.p_full[buf]));
       return true;
     };
     const int band_lo_max = prm.window > 0 ? q0 + k256BlockM - prm.window : 0;

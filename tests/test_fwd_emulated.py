@@ -81,3 +81,36 @@ def test_fwd_kernel_emulated(emu_fwd, B, H, H_kv, N, d, causal, window):
     err = np.abs(o - o_ref)
     assert err.max() <= O_MAX_ABS and err.mean() <= O_MEAN_ABS, (err.max(), err.mean())
     assert np.abs(lse - l_ref).max() <= L_MAX_ABS
+
+
+@pytest.mark.parametrize("d", [128, 256])
+def test_fwd_kernel_emulated_late_rescales(emu_fwd, d):
+    """Keys that score ever higher along the sequence make many rows' maxima grow by more than
+    2^8 after their first key tile, so the lazy rescale of O runs at later tiles (with the d = 256
+    kernel's two S buffers it must first wait for the previous P V product)."""
+    import subprocess
+    N = 400
+    g = torch.Generator().manual_seed(97)
+    q, k, v = (torch.randn(1, 1, N, d, generator=g) for _ in range(3))
+    qdir = q.mean(dim=2, keepdim=True)
+    k = k + torch.linspace(0, 6.0, N).view(1, 1, N, 1) * qdir / qdir.norm() * 40.0
+    q, k, v = (x.to(torch.bfloat16) for x in (q, k, v))
+    scale = 1.0 / d ** 0.5
+    s = scale * (q.double() @ k.double().transpose(-1, -2))[0, 0].numpy()
+    late = sum((s[i, :i + 1].max() - s[i, :min(64, i + 1)].max()) / np.log(2) > 8 for i in range(64, N))
+    assert late > 100, late   # the case does exercise late rescales
+    with tempfile.TemporaryDirectory() as tmp:
+        pre = os.path.join(tmp, "x")
+        for name, t in zip("qkv", (q, k, v)):
+            t.contiguous().view(torch.int16).numpy().tofile(pre + "." + name)
+        r = subprocess.run([emu_fwd[d], "1", "1", "1", str(N), "1", "0", repr(scale), pre],
+                           capture_output=True, text=True, timeout=900)
+        assert r.returncode == 0, r.stderr[-4000:]
+        o = np.fromfile(pre + ".o", dtype=np.uint16)
+        lse = np.fromfile(pre + ".lse", dtype=np.float32).reshape(1, 1, N)
+    o = torch.from_numpy(o.view(np.int16).copy()).view(torch.bfloat16).reshape(q.shape).double().numpy()
+    o_ref, l_ref = orc.attention_forward(q, k, v, scale, True, 0)
+    assert np.isfinite(o).all()
+    err = np.abs(o - o_ref)
+    assert err.max() <= O_MAX_ABS and err.mean() <= O_MEAN_ABS, (err.max(), err.mean())
+    assert np.abs(lse - l_ref).max() <= L_MAX_ABS
