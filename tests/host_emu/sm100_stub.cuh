@@ -21,8 +21,8 @@
 // TMA and bulk copies likewise land only when some thread tests the barrier that tracks them,
 // so a consumer that reads shared memory or TMEM without waiting on the right barrier sees
 // stale (NaN-filled) data.  ldmatrix and mma.sync are emulated from the fragment layouts the PTX ISA
-// documents (m8n8 b16 matrices; m16n8k16 row.col bf16 with fp32 accumulators); cp.async is a
-// synchronous copy (zero-fill when the source size is 0); ex2 / lg2 are std::exp2 / std::log2;
+// documents (m8n8 b16 matrices; m16n8k16 row.col bf16 with fp32 accumulators); cp.async
+// copies land at the issuing thread's wait_group (zero-fill when the source size is 0); ex2 / lg2 are std::exp2 / std::log2;
 // bf16 and f16 rounding is round-to-nearest-even (f16 with subnormals and overflow to
 // infinity); E4M3 codes decode by the format's definition (they are all f16 values).
 #pragma once
@@ -96,13 +96,32 @@ inline uint32_t bf16x2_to_f16x2_sat(uint32_t w) {
   return pack_f16x2(lo, hi);
 }
 inline unsigned char* dec_dyn_smem() { return g_blk->smem; }
+// cp.async: a thread's copies are grouped by its commits and land only at its own
+// cp.async.wait_group, oldest groups first (copies not yet committed are not waited for)
+struct CpAsyncState {
+  std::vector<std::function<void()>> open;
+  std::vector<std::vector<std::function<void()>>> committed;
+};
+inline thread_local CpAsyncState t_cp;
 inline void cp_async_16(void* dst, const void* src, int n) {
-  if (n == 16) std::memcpy(dst, src, 16);
-  else if (n == 0) std::memset(dst, 0, 16);
-  else { std::fprintf(stderr, "bad cp.async size %d\n", n); std::abort(); }
+  if (n != 16 && n != 0) { std::fprintf(stderr, "bad cp.async size %d\n", n); std::abort(); }
+  if (reinterpret_cast<uintptr_t>(dst) % 16) { std::fprintf(stderr, "cp.async destination not 16-byte aligned\n"); std::abort(); }
+  t_cp.open.push_back([=] {
+    if (n == 16) std::memcpy(dst, src, 16);
+    else std::memset(dst, 0, 16);
+  });
 }
-inline void cp_async_commit() {}
-template <int N> inline void cp_async_wait() {}
+inline void cp_async_commit() {
+  t_cp.committed.push_back(std::move(t_cp.open));
+  t_cp.open.clear();
+}
+template <int N>
+inline void cp_async_wait() {
+  while (t_cp.committed.size() > size_t(N)) {
+    for (auto& f : t_cp.committed.front()) f();
+    t_cp.committed.erase(t_cp.committed.begin());
+  }
+}
 inline uint32_t ld_global_u32(const void* p) {
   if (reinterpret_cast<uintptr_t>(p) % 4) { std::fprintf(stderr, "misaligned u32 load\n"); std::abort(); }
   uint32_t v;
