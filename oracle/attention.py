@@ -82,6 +82,7 @@ __all__ = [
     "attention_forward_decode",
     "e4m3_to_float",
     "attention_forward_decode_fp8kv",
+    "attention_forward_fp8",
 ]
 
 
@@ -320,6 +321,18 @@ def attention_forward_decode_fp8kv(q, k8, v8, k_scale: float, v_scale: float, sc
     k = float(k_scale) * e4m3_to_float(k8)
     v = float(v_scale) * e4m3_to_float(v8)
     return attention_forward_decode(q, k, v, scale, causal, window)
+
+
+def attention_forward_fp8(q8, k8, vt8, q_scale: float, k_scale: float, v_scale: float, scale: float,
+                          causal: bool = False, window: int = 0):
+    """The forward on E4M3 codes with one scale per tensor: Q = q_scale E4M3(q8) [..., H, N, d],
+    K = k_scale E4M3(k8) [..., H_kv, N, d], and V = v_scale E4M3(vt8) given transposed,
+    vt8 [..., H_kv, d, N]."""
+    q8, k8, vt8 = (x.detach().cpu().numpy() if hasattr(x, "detach") else np.asarray(x) for x in (q8, k8, vt8))
+    q = float(q_scale) * e4m3_to_float(q8)
+    k = float(k_scale) * e4m3_to_float(k8)
+    v = float(v_scale) * np.swapaxes(e4m3_to_float(vt8), -1, -2)
+    return attention_forward_shared_kv(q, k, v, scale, causal, window)
 
 
 def allowed_pairs(n: int, causal: bool, window: int) -> int:

@@ -127,6 +127,16 @@ def make_inputs_fp8kv(wl: Workload, seed: int | None = None):
     return q, k8, v8, s_k, s_v
 
 
+def make_inputs_fp8(wl: Workload, seed: int | None = None):
+    """make_inputs with Q, K and V quantised to E4M3 per tensor, V returned transposed
+    ([B, H_kv, d, N], contiguous): (Q8, K8, V8^T, s_q, s_k, s_v)."""
+    q, k, v = make_inputs(wl, seed)
+    q8, s_q = quantize_e4m3(q)
+    k8, s_k = quantize_e4m3(k)
+    v8, s_v = quantize_e4m3(v)
+    return q8, k8, v8.transpose(-1, -2).contiguous(), s_q, s_k, s_v
+
+
 def make_grad_output(wl: Workload, seed: int | None = None) -> torch.Tensor:
     """dO as a contiguous CPU bf16 tensor [B, H, N, d], N(0, 1) from the grad seed."""
     s = seed if seed is not None else (wl.grad_seed if wl.grad_seed is not None else wl.seed + 1000)

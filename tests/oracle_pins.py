@@ -496,6 +496,29 @@ def fp8kv_decode(orc):
         assert np.max(np.abs(o3 - 2 * o)) < 1e-12 and np.max(np.abs(l3 - lse)) < 1e-12
 
 
+def fp8_forward(orc):
+    """The FP8 forward (V given transposed) equals the plain forward on torch-dequantised Q, K and
+    V^T transposed back; doubling s_q while halving s_k changes nothing; O is linear in s_v."""
+    import torch
+    r = _rng(35)
+    dq = lambda c: torch.from_numpy(c).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    q8 = r.integers(0, 256, size=(1, 4, 9, 6)).astype(np.uint8)
+    k8 = r.integers(0, 256, size=(1, 2, 9, 6)).astype(np.uint8)
+    vt8 = r.integers(0, 256, size=(1, 2, 6, 9)).astype(np.uint8)
+    for a in (q8, k8, vt8):
+        a[(a & 0x7F) == 0x7F] = 0x38
+    for causal, window in MASKS:
+        o, lse = orc.attention_forward_fp8(q8, k8, vt8, 0.02, 0.05, 0.7, 0.3, causal, window)
+        ref = orc.attention_forward_shared_kv(0.02 * dq(q8), 0.05 * dq(k8), 0.7 * np.swapaxes(dq(vt8), -1, -2), 0.3,
+                                              causal, window)
+        assert o.shape == q8.shape
+        assert np.max(np.abs(o - ref[0])) < 1e-12 and np.max(np.abs(lse - ref[1])) < 1e-12
+        o2, l2 = orc.attention_forward_fp8(q8, k8, vt8, 0.04, 0.025, 0.7, 0.3, causal, window)
+        assert np.max(np.abs(o2 - o)) < 1e-12 and np.max(np.abs(l2 - lse)) < 1e-12
+        o3, l3 = orc.attention_forward_fp8(q8, k8, vt8, 0.02, 0.05, 1.4, 0.3, causal, window)
+        assert np.max(np.abs(o3 - 2 * o)) < 1e-12 and np.max(np.abs(l3 - lse)) < 1e-12
+
+
 def rejects_bad_masks(orc):
     """A negative window is rejected, with or without causal."""
     q, k, v = _qkv(21, n=4, d=2, lead=())
@@ -513,5 +536,5 @@ PINS = {f.__name__: f for f in (
     large_scores, golden_examples, library_forward, library_backward, finite_differences,
     delta_identity, row_blocks_match, pair_count, two_sided_window, shared_kv_library,
     shared_kv_finite_differences, decode_library, decode_scale_zero, decode_last_rows_of_self_attention,
-    e4m3_decoding, fp8kv_decode, rejects_bad_masks,
+    e4m3_decoding, fp8kv_decode, fp8_forward, rejects_bad_masks,
 )}

@@ -151,7 +151,15 @@ def _fp8kv_v_scale_dropped(q, k8, v8, k_scale, v_scale, scale, causal=False, win
                                         window)
 
 
+def _fp8_v_not_transposed(q8, k8, vt8, q_scale, k_scale, v_scale, scale, causal=False, window=0):
+    q = q_scale * orc.e4m3_to_float(q8)
+    k = k_scale * orc.e4m3_to_float(k8)
+    v = v_scale * orc.e4m3_to_float(vt8).reshape(k.shape)   # the codes read as [N, d], not transposed
+    return orc.attention_forward_shared_kv(q, k, v, scale, causal, window)
+
+
 MUTANTS = {
+    "fp8_v_not_transposed": ("attention_forward_fp8", _fp8_v_not_transposed),
     "e4m3_bias_8": ("e4m3_to_float", _e4m3_bias_8),
     "e4m3_no_subnormals": ("e4m3_to_float", _e4m3_no_subnormals),
     "fp8kv_v_scale_dropped": ("attention_forward_decode_fp8kv", _fp8kv_v_scale_dropped),
