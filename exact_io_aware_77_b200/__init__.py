@@ -15,7 +15,7 @@ import math
 from . import _lib
 from ._lib import FAError, STATUS, STATUS_NAMES, load
 
-__all__ = ["forward", "backward", "decode", "decode_fp8kv", "decode_workspace_size", "bwd_workspace_size", "check_status", "FAError", "STATUS", "STATUS_NAMES", "load", "default_scale"]
+__all__ = ["forward", "forward_fp8", "backward", "decode", "decode_fp8kv", "decode_workspace_size", "bwd_workspace_size", "check_status", "FAError", "STATUS", "STATUS_NAMES", "load", "default_scale"]
 
 
 def default_scale(d: int) -> float:
@@ -96,6 +96,38 @@ def forward(q, k, v, scale: float | None = None, causal: bool = False, window: i
         _raise("fa_fwd", _lib.fa_fwd(*ptrs, B, H, N, d, *mask))
     else:
         _raise("fa_fwd_gqa", _lib.fa_fwd_gqa(*ptrs, B, H, H_kv, N, d, *mask))
+    return out, lse
+
+
+def forward_fp8(q8, k8, vt8, q_scale: float, k_scale: float, v_scale: float, scale: float | None = None,
+                causal: bool = False, window: int = 0, out=None, lse=None):
+    """O, L of attention on E4M3 inputs: Q = q_scale E4M3(q8), K = k_scale E4M3(k8),
+    V = v_scale E4M3(vt8)^T.
+
+    q8 [B, H, N, 128], k8 [B, H_kv, N, 128], vt8 [B, H_kv, 128, N]: contiguous CUDA tensors of
+    torch.uint8 or torch.float8_e4m3fn codes; N a multiple of 16.  Returns O bf16 [B, H, N, 128] and
+    L fp32 [B, H, N].
+    """
+    import torch
+    q8, k8, vt8 = (x.view(torch.uint8) if x.dtype == torch.float8_e4m3fn else x for x in (q8, k8, vt8))
+    for t in (q8, k8, vt8):
+        if not (t.is_cuda and t.dtype == torch.uint8 and t.dim() == 4 and t.is_contiguous() and t.device == q8.device):
+            raise ValueError("q8, k8, vt8 must be contiguous E4M3 code tensors on one CUDA device")
+    B, H, N, d = q8.shape
+    H_kv = int(k8.shape[1])
+    if k8.shape != (B, H_kv, N, d) or vt8.shape != (B, H_kv, d, N):
+        raise ValueError("k8 must be [B, H_kv, N, d] and vt8 [B, H_kv, d, N]")
+    scale = default_scale(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q8.device)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q8.device)
+    if not (out.shape == (B, H, N, d) and out.dtype == torch.bfloat16 and out.is_contiguous() and out.device == q8.device):
+        raise ValueError("out must be a contiguous bf16 tensor [B, H, N, d] on q8's device")
+    _check_lse(lse, q8, B * H * N)
+    _raise("fa_fwd_fp8", _lib.fa_fwd_fp8(q8.data_ptr(), k8.data_ptr(), vt8.data_ptr(), float(q_scale), float(k_scale),
+                                         float(v_scale), out.data_ptr(), lse.data_ptr(), B, H, H_kv, N, d, scale,
+                                         int(bool(causal)), int(window), _stream_handle(q8.device)))
     return out, lse
 
 

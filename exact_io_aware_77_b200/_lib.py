@@ -46,6 +46,8 @@ SIGNATURES = {
                                                                 _c_size_t, _c_void_p]),
     "fa_fwd_decode_fp8kv": (_c_int, [_c_void_p] * 3 + [_c_float, _c_float] + [_c_void_p] * 2 + [_c_int] * 6 +
                             [_c_void_p, _c_float, _c_int, _c_int, _c_void_p, _c_size_t, _c_void_p]),
+    "fa_fwd_fp8": (_c_int, [_c_void_p] * 3 + [_c_float] * 3 + [_c_void_p] * 2 + [_c_int] * 5 +
+                   [_c_float, _c_int, _c_int, _c_void_p]),
     "fa_status_string": (ctypes.c_char_p, [_c_int]),
     "fa_check_status": (_c_int, [_c_void_p]),
     "fa_set_wait_limit_ns": (None, [_c_ull]),
@@ -173,6 +175,13 @@ def fa_fwd_decode_fp8kv(q, k8, v8, k_scale, v_scale, o, lse, B, H, H_kv, N_q, N_
     """fa_fwd_decode over E4M3 K/V codes with per-tensor scales."""
     return _call("fa_fwd_decode_fp8kv", q, k8, v8, k_scale, v_scale, o, lse, B, H, H_kv, N_q, N_k, d, strides, scale,
                  causal, window, workspace, workspace_bytes, stream)
+
+
+def fa_fwd_fp8(q8, k8, vt8, q_scale, k_scale, v_scale, o, lse, B, H, H_kv, N, d, scale, causal, window,
+               stream) -> int:
+    """The forward on E4M3 Q, K and transposed V with per-tensor scales."""
+    return _call("fa_fwd_fp8", q8, k8, vt8, q_scale, k_scale, v_scale, o, lse, B, H, H_kv, N, d, scale, causal,
+                 window, stream)
 
 
 def fa_status_string(status: int) -> str:

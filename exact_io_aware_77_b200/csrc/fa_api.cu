@@ -13,6 +13,8 @@
 
 #include "fwd_kernel.cuh"
 #include "fwd256_kernel.cuh"
+#include "fp8_ops.cuh"
+#include "fwd_fp8_kernel.cuh"
 #include "bwd_kernel.cuh"
 #include "bwd256_kernel.cuh"
 #include "decode_ops.cuh"
@@ -54,6 +56,20 @@ bool make_map_bf16(CUtensorMap* map, const void* base, int d, int rows, int head
   cuuint32_t box[4] = {64, cuuint32_t(box_rows), 1, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// A one-byte (E4M3 code) packed array [B, heads, rows, x] as the 4-D tensor (x, rows, heads, B),
+// box = 128 x 128, 128-byte swizzled; outside the tensor reads as zero.
+bool make_map_u8(CUtensorMap* map, const void* base, int x, int rows, int heads, int B) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {cuuint64_t(x), cuuint64_t(rows), cuuint64_t(heads), cuuint64_t(B)};
+  cuuint64_t strides[3] = {cuuint64_t(x), cuuint64_t(x) * rows, cuuint64_t(x) * rows * heads};
+  cuuint32_t box[4] = {128, 128, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -163,6 +179,33 @@ int launch_fwd256(const void* q, const void* k, const void* v, void* o, float* l
   const int smem = int(sizeof(Fwd256Smem)) + 1024;
   if (set_smem(fa_fwd256_kernel, smem) != FA_OK) return FA_ERR_CUDA;
   fa_fwd256_kernel<<<unsigned(prm.n_pairs) * unsigned(BH), k256Threads, smem, stream>>>(tq, tk, tv, prm);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// FP8 forward: q8, k8 [B, heads, N, 128] and vt8 [B, H_kv, 128, N] E4M3 codes, packed
+int launch_fwd_fp8(const void* q8, const void* k8, const void* vt8, float q_scale, float k_scale, float v_scale,
+                   void* o, float* lse, int B, int H, int H_kv, int N, float scale, int causal, int window,
+                   cudaStream_t stream) {
+  CUtensorMap tq, tk, tvt;
+  if (!make_map_u8(&tq, q8, kF8D, N, H, B) || !make_map_u8(&tk, k8, kF8D, N, H_kv, B) ||
+      !make_map_u8(&tvt, vt8, N, kF8D, H_kv, B))
+    return FA_ERR_CUDA;
+  FwdParams prm;
+  prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.lse = lse;
+  prm.N = N;
+  prm.BH = B * H;
+  prm.H = H;
+  prm.group = H / H_kv;
+  prm.o_st = packed(H, N, kF8D);
+  prm.n_pairs = ((N + kBlockM - 1) / kBlockM + kQTiles - 1) / kQTiles;
+  prm.causal = causal;
+  prm.window = window > N ? N : window;
+  prm.scale_log2 = scale * q_scale * k_scale * 1.4426950408889634f;
+  prm.wait_limit_ns = g_wait_limit_ns;
+  const int smem = int(sizeof(FwdFp8Smem)) + 1024;
+  if (set_smem(fa_fwd_fp8_kernel, smem) != FA_OK) return FA_ERR_CUDA;
+  fa_fwd_fp8_kernel<<<unsigned(prm.n_pairs) * unsigned(prm.BH), kFwdThreads, smem, stream>>>(tq, tk, tvt, prm, v_scale);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -457,6 +500,23 @@ static int bwd_impl(const void* q, const void* k, const void* v, const void* o, 
     case 128: return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, s8, scale, causal, window, workspace, s, phases);
     default: return launch_bwd<256>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, s8, scale, causal, window, workspace, s, phases);
   }
+}
+
+int fa_fwd_fp8(const void* q8, const void* k8, const void* vt8, float q_scale, float k_scale, float v_scale, void* o,
+               float* lse, int B, int H, int H_kv, int N, int d, float scale, int causal, int window, void* stream) {
+  if (!q8 || !k8 || !vt8 || !o || !lse) return FA_ERR_NULL;
+  int st = check_problem(B, H, N, d, scale, causal, window);
+  if (st == FA_OK) st = check_kv_heads(H, H_kv);
+  if (st != FA_OK) return st;
+  if (d != kF8D) return FA_ERR_HEADDIM;
+  if (N % 16) return FA_ERR_SHAPE;   // rows of the transposed V are N bytes: 16-byte multiples
+  for (float sc : {q_scale, k_scale, v_scale})
+    if (!std::isfinite(sc) || !(sc > 0.f)) return FA_ERR_SCALE;
+  if (!aligned(q8, 16) || !aligned(k8, 16) || !aligned(vt8, 16) || !aligned(o, 16) || !aligned(lse, 4))
+    return FA_ERR_ALIGN;
+  if ((st = check_device()) != FA_OK) return st;
+  return launch_fwd_fp8(q8, k8, vt8, q_scale, k_scale, v_scale, o, lse, B, H, H_kv, N, scale, causal, window,
+                        static_cast<cudaStream_t>(stream));
 }
 
 size_t fa_decode_workspace_size(int B, int H, int H_kv, int N_q, int N_k, int d, int causal, int window) {

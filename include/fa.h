@@ -216,6 +216,28 @@ FA_EXPORT int fa_fwd_decode_fp8kv(const void* q, const void* k8, const void* v8,
                                   const fa_strides* strides, float scale, int causal, int window, void* workspace,
                                   size_t workspace_bytes, void* stream);
 
+/*
+ * Forward on FP8 (E4M3) Q, K and V with one scale per tensor: Q = q_scale * E4M3(q8),
+ * K = k_scale * E4M3(k8), V = v_scale * E4M3(vt8)^T; the FP8 forward the FlashAttention (NL)
+ * page attributes to FlashAttention-3 ("Evolutie en verdere ontwikkelingen").  E4M3 as for
+ * fa_fwd_decode_fp8kv.  Both products run on the tensor cores' 8-bit path (E4M3 x E4M3 -> fp32);
+ * P is rounded to E4M3 before P V (O carries that rounding: relative 2^-4 per weight).
+ *
+ *   q8     E4M3 codes [B, H, N, d], packed;  k8  [B, H_kv, N, d], packed.
+ *   vt8    V transposed: E4M3 codes [B, H_kv, d, N], packed (N contiguous), so that both operands
+ *          of the 8-bit P V product are K-major.
+ *   o, lse bf16 [B, H, N, d] and fp32 [B, H, N], packed.
+ *   d must be 128 (FA_ERR_HEADDIM otherwise); N a multiple of 16 (FA_ERR_SHAPE); the scales
+ *   finite and > 0 (FA_ERR_SCALE).  Masks, scale, errors and streams as for fa_fwd_gqa.
+ *
+ * The kernel has been checked against the reference only in a host emulation of its
+ * primitives, not yet on a B200; the 8-bit instruction descriptor (type code 0 for E4M3) is the
+ * documented encoding, still to be confirmed on the hardware.
+ */
+FA_EXPORT int fa_fwd_fp8(const void* q8, const void* k8, const void* vt8, float q_scale, float k_scale, float v_scale,
+                         void* o, float* lse, int B, int H, int H_kv, int N, int d, float scale, int causal, int window,
+                         void* stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 FA_EXPORT const char* fa_status_string(int status);
 

@@ -15,6 +15,8 @@ import subprocess
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(os.path.dirname(os.path.dirname(HERE)), "exact_io_aware_77_b200", "csrc")
 PURE_HELPERS = ("idesc_bf16_f32", "sw128_desc", "desc_advance", "exp2_poly_x2")
+# headers whose every function the stub itself provides: the emulation gets an empty file
+STUBBED_HEADERS = ("fp8_ops.cuh", "decode_ops.cuh")
 
 
 def extract(src: str, name: str) -> str:
@@ -66,6 +68,9 @@ def build(out_dir: str, kernel_header, harness: str, exe_name: str, defines=()) 
         with open(os.path.join(out_dir, h), "w") as f:
             f.write(text)
     shutil.copy(os.path.join(HERE, "sm100_stub.cuh"), os.path.join(out_dir, "sm100.cuh"))
+    for h in STUBBED_HEADERS:
+        with open(os.path.join(out_dir, h), "w") as f:
+            f.write("// provided by the host emulation's sm100.cuh\n#pragma once\n")
     shutil.copy(os.path.join(HERE, "emu.h"), os.path.join(out_dir, "emu.h"))
     shutil.copy(os.path.join(HERE, harness), os.path.join(out_dir, harness))
     exe = os.path.join(out_dir, exe_name)

@@ -7,6 +7,9 @@
 #ifdef EMU_FWD256
 #include "fwd256_kernel.cuh"
 #define EMU_D 256
+#elif defined(EMU_FWD_FP8)
+#include "fwd_fp8_kernel.cuh"
+#define EMU_D 128
 #else
 #include "fwd_kernel.cuh"
 #endif
@@ -23,6 +26,8 @@ namespace fa {
 // sees any access past it
 #ifdef EMU_FWD256
 alignas(1024) uint8_t smem_raw[sizeof(Fwd256Smem)];
+#elif defined(EMU_FWD_FP8)
+alignas(1024) uint8_t smem_raw[sizeof(FwdFp8Smem)];
 #else
 alignas(1024) uint8_t smem_raw[sizeof(FwdSmem<EMU_D>)];
 #endif
@@ -59,6 +64,60 @@ CUtensorMap make_map(const uint16_t* base, int d, int rows, int heads, int B, in
   return m;
 }
 
+#ifdef EMU_FWD_FP8
+// E4M3 code arrays: q8, k8 [B, heads, N, 128]; vt8 [B, H_kv, 128, N]
+// usage: emu_fwd_fp8 B H Hkv N causal window scale prefix s_q s_k s_v
+int main(int argc, char** argv) {
+  if (argc != 12) { std::fprintf(stderr, "bad args\n"); return 2; }
+  const int B = atoi(argv[1]), H = atoi(argv[2]), Hkv = atoi(argv[3]), N = atoi(argv[4]), causal = atoi(argv[5]),
+            window = atoi(argv[6]);
+  const float scale = float(atof(argv[7]));
+  const std::string prefix = argv[8];
+  const float s_q = float(atof(argv[9])), s_k = float(atof(argv[10])), s_v = float(atof(argv[11]));
+  constexpr int D = 128;
+  auto q = read_file<uint8_t>(prefix + ".q", size_t(B) * H * N * D);
+  auto k = read_file<uint8_t>(prefix + ".k", size_t(B) * Hkv * N * D);
+  auto vt = read_file<uint8_t>(prefix + ".v", size_t(B) * Hkv * D * N);
+  std::vector<uint16_t> o(size_t(B) * H * N * D, 0x7fc0);
+  std::vector<float> lse(size_t(B) * H * N, NAN);
+  auto map8 = [](const uint8_t* base, uint64_t x, uint64_t rows, uint64_t heads, uint64_t b) {
+    CUtensorMap m;
+    m.base = base;
+    m.dims[0] = x;
+    m.dims[1] = rows;
+    m.dims[2] = heads;
+    m.dims[3] = b;
+    m.strides[0] = x;
+    m.strides[1] = rows * x;
+    m.strides[2] = heads * rows * x;
+    m.box_x = 128;
+    m.box_rows = 128;
+    m.esize = 1;
+    return m;
+  };
+  const CUtensorMap tq = map8(q.data(), D, N, H, B), tk = map8(k.data(), D, N, Hkv, B),
+                    tvt = map8(vt.data(), N, D, Hkv, B);
+  FwdParams prm;
+  prm.o = reinterpret_cast<__nv_bfloat16*>(o.data());
+  prm.lse = lse.data();
+  prm.N = N;
+  prm.BH = B * H;
+  prm.H = H;
+  prm.group = H / Hkv;
+  prm.o_st = Strides{(long long)H * N * D, (long long)N * D, (long long)D};
+  prm.n_pairs = ((N + kBlockM - 1) / kBlockM + kQTiles - 1) / kQTiles;
+  prm.causal = causal;
+  prm.window = window > N ? N : window;
+  prm.scale_log2 = scale * s_q * s_k * 1.4426950408889634f;
+  prm.wait_limit_ns = 60ull * 1000000000ull;
+  const unsigned grid = unsigned(prm.n_pairs) * unsigned(B * H);
+  emu_launch(grid, kFwdThreads, sizeof(fa::smem_raw), [&] { fa_fwd_fp8_kernel(tq, tk, tvt, prm, s_v); }, fa::smem_raw);
+  if (g_status != 0) { std::fprintf(stderr, "device status %d\n", g_status); return 3; }
+  write_file(prefix + ".o", o);
+  write_file(prefix + ".lse", lse);
+  return 0;
+}
+#else
 int main(int argc, char** argv) {
   if (argc != 9) { std::fprintf(stderr, "bad args\n"); return 2; }
   const int B = atoi(argv[1]), H = atoi(argv[2]), Hkv = atoi(argv[3]), N = atoi(argv[4]), causal = atoi(argv[5]),
@@ -107,3 +166,4 @@ int main(int argc, char** argv) {
   write_file(prefix + ".lse", lse);
   return 0;
 }
+#endif

@@ -282,9 +282,10 @@ inline bool mbar_wait_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
 // ------------------------------------------------------------ TMA
 struct CUtensorMap {
   const unsigned char* base;
-  uint64_t dims[4];      // d, rows, heads, batch (elements)
+  uint64_t dims[4];      // x (contiguous), rows, heads, batch (elements)
   uint64_t strides[3];   // bytes: rows, heads, batch
   uint32_t box_x, box_rows;
+  uint32_t esize = 2;    // bytes per element; box_x * esize is the 128-byte swizzle row
 };
 inline void tma_prefetch_desc(const CUtensorMap*) {}
 inline uint32_t sw128(uint32_t addr) { return addr ^ (((addr >> 7) & 7u) << 4); }
@@ -311,8 +312,8 @@ inline void queue_copy(uint32_t bar, std::function<void()> f) {
 }
 inline void tma_copy_now(uint32_t dst, CUtensorMap map, uint32_t bar, int x, int row, int head, int batch);
 inline void tma_load_rows(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int row, int head, int batch) {
-  if (x % 8) { std::fprintf(stderr, "TMA x coordinate not 16-byte aligned\n"); std::abort(); }
-  if (map->box_x != 64) { std::fprintf(stderr, "TMA box is not 64 elements wide\n"); std::abort(); }
+  if ((x * int(map->esize)) % 16) { std::fprintf(stderr, "TMA x coordinate not 16-byte aligned\n"); std::abort(); }
+  if (map->box_x * map->esize != 128) { std::fprintf(stderr, "TMA box row is not 128 bytes\n"); std::abort(); }
   smem_at(dst, size_t(map->box_rows) * 128);   // the destination must lie in shared memory
   const CUtensorMap m = *map;
   BlockCtx* blk = g_blk;
@@ -328,14 +329,15 @@ inline void tma_copy_now(uint32_t dst, CUtensorMap mm, uint32_t bar, int x, int 
   for (uint32_t r = 0; r < map->box_rows; ++r)
     for (uint32_t c = 0; c < map->box_x; ++c) {
       const long long gx = (long long)x + c, gr = (long long)row + r;
+      const uint32_t es = map->esize;
       uint16_t val = 0;
       if (gx >= 0 && gr >= 0 && head >= 0 && batch >= 0 && uint64_t(gx) < map->dims[0] &&
           uint64_t(gr) < map->dims[1] && uint64_t(head) < map->dims[2] && uint64_t(batch) < map->dims[3])
         std::memcpy(&val, map->base + uint64_t(batch) * map->strides[2] + uint64_t(head) * map->strides[1] +
-                              uint64_t(gr) * map->strides[0] + uint64_t(gx) * 2, 2);
-      std::memcpy(smem_at(sw128(dst + r * 128 + c * 2), 2), &val, 2);
+                              uint64_t(gr) * map->strides[0] + uint64_t(gx) * es, es);
+      std::memcpy(smem_at(sw128(dst + r * 128 + c * es), es), &val, es);
     }
-  bar_complete_tx(bar, map->box_x * map->box_rows * 2);
+  bar_complete_tx(bar, map->box_x * map->box_rows * map->esize);
 }
 
 // ------------------------------------------------------------ tensor memory
@@ -432,6 +434,37 @@ inline void queue_mma(std::function<void()> f) {
   std::lock_guard<std::mutex> lk(*g_blk->mu);
   g_blk->mmas->push_back(PendingOp{0, std::move(f)});
 }
+// kind::f8f6f4 with E4M3 A and B (type code 0), fp32 D, M = 128, K = 32: byte elements of
+// K-major 128-byte-swizzled shared-memory operands
+inline float sw128_operand_u8(uint64_t desc, uint32_t i, uint32_t k) {
+  if ((desc >> 61) != 2u) { std::fprintf(stderr, "descriptor layout is not the 128-byte swizzle\n"); std::abort(); }
+  const uint32_t start = uint32_t(desc & 0x3fffu) << 4, sbo = uint32_t((desc >> 32) & 0x3fffu) << 4;
+  const uint32_t addr = start + (i / 8) * sbo + (i % 8) * 128 + k;
+  return e4m3_to_f(*smem_at(sw128(addr), 1));
+}
+inline void mma_f8_exec(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
+  if (((idesc >> 4) & 3u) != 1u || ((idesc >> 7) & 7u) != 0u || ((idesc >> 10) & 7u) != 0u ||
+      ((idesc >> 15) & 3u) != 0u) {
+    std::fprintf(stderr, "instruction descriptor is not K-major E4M3 x E4M3 -> f32\n");
+    std::abort();
+  }
+  const uint32_t M = ((idesc >> 24) & 0x1fu) << 4, N = ((idesc >> 17) & 0x3fu) << 3;
+  if (M != 128 || N < 8 || N > 256 || N % 16) { std::fprintf(stderr, "unsupported MMA shape\n"); std::abort(); }
+  std::lock_guard<std::mutex> lk(*g_blk->mu);
+  std::vector<float> A(128 * 32), B(N * 32);
+  for (uint32_t m = 0; m < 128; ++m)
+    for (uint32_t k = 0; k < 32; ++k) A[m * 32 + k] = sw128_operand_u8(a_desc, m, k);
+  for (uint32_t n = 0; n < N; ++n)
+    for (uint32_t k = 0; k < 32; ++k) B[n * 32 + k] = sw128_operand_u8(b_desc, n, k);
+  const uint32_t lane0 = d_tmem >> 16, col0 = d_tmem & 0xffffu;
+  for (uint32_t m = 0; m < 128; ++m)
+    for (uint32_t n = 0; n < N; ++n) {
+      uint32_t& cell = tmem_cell(lane0 + m, col0 + n);
+      float acc = accumulate ? __uint_as_float(cell) : 0.f;
+      for (uint32_t k = 0; k < 32; ++k) acc += A[m * 32 + k] * B[n * 32 + k];
+      cell = __float_as_uint(acc);
+    }
+}
 inline void mma_bf16_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
   queue_mma([=] { mma_exec(d, a, ~0u, b, idesc, acc); });
 }
@@ -458,6 +491,26 @@ inline void mma_bf16_ts_w(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc, ui
 inline void mma_commit_w(uint32_t bar) {
   if (lane_id() == 0) mma_commit(bar);
 }
+inline void mma_e4m3_ss_w(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  if (lane_id() == 0) queue_mma([=] { mma_f8_exec(d, a, b, idesc, acc); });
+}
+// two fp32 values as E4M3 codes (round to nearest even, saturating to +-448; lo in the low byte)
+inline uint8_t f2e4m3(float f) {
+  if (std::isnan(f)) return 0x7f;
+  const uint8_t sign = std::signbit(f) ? 0x80 : 0;
+  float a = std::fabs(f);
+  if (a >= 448.f) return sign | 0x7e;
+  // find the nearest representable magnitude by search over the 127 finite codes (exact and simple)
+  uint8_t best = 0;
+  float bd = INFINITY;
+  for (int c = 0; c <= 0x7e; ++c) {
+    const float v = e4m3_to_f(uint8_t(c));
+    const float dd = std::fabs(v - a);
+    if (dd < bd || (dd == bd && (c & 1) == 0 && (best & 1) == 1)) { bd = dd; best = uint8_t(c); }
+  }
+  return sign | best;
+}
+inline uint32_t f32x2_to_e4m3x2(float lo, float hi) { return uint32_t(f2e4m3(lo)) | (uint32_t(f2e4m3(hi)) << 8); }
 
 // ------------------------------------------------------------ shared vectors, bulk copies, reductions
 inline uint4 ld_shared_v4(uint32_t addr) {

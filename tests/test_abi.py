@@ -235,3 +235,27 @@ def test_head_dim_256_workspace(lib):
     for B, H, N in ((1, 2, 128), (2, 4, 300)):
         np_ = (N + 127) // 128 * 128
         assert _lib.fa_bwd_workspace_size(B, H, N, 256) == 4 * B * H * np_ * (256 + 2)
+
+
+def _f8(**kw):
+    a = dict(B=1, H=2, H_kv=2, N=256, d=128, scale=0.125, causal=1, window=0, qs=0.01, ks=0.01, vs=0.01)
+    ptrs = kw.pop("ptrs", [A + 4096 * i for i in range(5)])
+    a.update(kw)
+    return _lib.fa_fwd_fp8(ptrs[0], ptrs[1], ptrs[2], a["qs"], a["ks"], a["vs"], ptrs[3], ptrs[4], a["B"], a["H"],
+                           a["H_kv"], a["N"], a["d"], a["scale"], a["causal"], a["window"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(ptrs=[0] + [A] * 4), "FA_ERR_NULL"),
+    (dict(d=64), "FA_ERR_HEADDIM"),
+    (dict(d=256), "FA_ERR_HEADDIM"),
+    (dict(N=250), "FA_ERR_SHAPE"),
+    (dict(H_kv=3), "FA_ERR_SHAPE"),
+    (dict(qs=0.0), "FA_ERR_SCALE"),
+    (dict(ks=float("inf")), "FA_ERR_SCALE"),
+    (dict(vs=-1.0), "FA_ERR_SCALE"),
+    (dict(window=-1), "FA_ERR_MASK"),
+    (dict(ptrs=[A, A + 8, A, A, A]), "FA_ERR_ALIGN"),
+])
+def test_fwd_fp8_rejects_bad_arguments(lib, kw, code):
+    assert _lib.STATUS_NAMES[_f8(**kw)] == code

@@ -23,7 +23,7 @@ import pytest
 import torch
 
 from oracle import attention as orc
-from synthetic import Workload, make_inputs
+from synthetic import Workload, make_inputs, make_inputs_fp8
 from tests.parity import L_MAX_ABS, O_MAX_ABS, O_MEAN_ABS
 
 
@@ -36,6 +36,7 @@ def emu_fwd(tmp_path_factory):
             64: ("fwd_kernel.cuh", "emu_fwd_main.cpp", "emu_fwd_64", ("EMU_D=64",)),
             128: ("fwd_kernel.cuh", "emu_fwd_main.cpp", "emu_fwd_128", ("EMU_D=128",)),
             256: (["fwd256_kernel.cuh", "fwd_kernel.cuh"], "emu_fwd_main.cpp", "emu_fwd_256", ("EMU_FWD256",)),
+            "fp8": (["fwd_fp8_kernel.cuh", "fwd_kernel.cuh"], "emu_fwd_main.cpp", "emu_fwd_fp8", ("EMU_FWD_FP8",)),
         })
     except FileNotFoundError:
         pytest.skip("g++ not available")
@@ -114,3 +115,57 @@ def test_fwd_kernel_emulated_late_rescales(emu_fwd, d):
     err = np.abs(o - o_ref)
     assert err.max() <= O_MAX_ABS and err.mean() <= O_MEAN_ABS, (err.max(), err.mean())
     assert np.abs(lse - l_ref).max() <= L_MAX_ABS
+
+
+FP8_CASES = [
+    # B, H, H_kv, N, causal, window (d = 128; N a multiple of 16 for the transposed V)
+    (1, 2, 2, 256, True, 0),
+    (1, 2, 1, 400, True, 0),
+    (1, 2, 2, 304, False, 0),
+    (1, 4, 2, 512, True, 100),
+    (2, 2, 1, 144, False, 40),
+]
+
+
+@pytest.mark.parametrize("B,H,H_kv,N,causal,window", FP8_CASES)
+def test_fwd_fp8_kernel_emulated(emu_fwd, B, H, H_kv, N, causal, window):
+    """The FP8 forward (E4M3 Q, K, V^T with per-tensor scales) against the oracle on the
+    dequantised values.  Tolerance, derived: the kernel rounds each P to E4M3 before P V
+    (relative error <= 2^-4 for normal values, absolute <= 2^-10 below E4M3's normal range) while l
+    sums the exact P, so with w_j = exp(s_j - max s) over the allowed keys,
+    |dO_c| <= sum_j max(2^-4 w_j, 2^-10) |V_jc| / sum_j w_j; plus bf16 rounding of O (2^-8 |O|) and
+    1e-3 for the fp32 exponentials and sums.  L uses the exact P: the usual 1e-3."""
+    import subprocess
+    d = 128
+    wl = Workload("fwd_fp8_emu", B, H, N, d, causal, window, seed=99 + N + H_kv, H_kv=H_kv)
+    q8, k8, vt8, s_q, s_k, s_v = make_inputs_fp8(wl)
+    with tempfile.TemporaryDirectory() as tmp:
+        pre = os.path.join(tmp, "x")
+        for name, t in zip("qkv", (q8, k8, vt8)):
+            t.contiguous().numpy().tofile(pre + "." + name)
+        r = subprocess.run([emu_fwd["fp8"], str(B), str(H), str(H_kv), str(N), str(int(causal)), str(window),
+                            repr(wl.scale), pre, repr(s_q), repr(s_k), repr(s_v)],
+                           capture_output=True, text=True, timeout=900)
+        assert r.returncode == 0, r.stderr[-4000:]
+        o = np.fromfile(pre + ".o", dtype=np.uint16)
+        lse = np.fromfile(pre + ".lse", dtype=np.float32).reshape(B, H, N)
+    o = torch.from_numpy(o.view(np.int16).copy()).view(torch.bfloat16).reshape(B, H, N, d).double().numpy()
+    o_ref, l_ref = orc.attention_forward_fp8(q8, k8, vt8, s_q, s_k, s_v, wl.scale, causal, window)
+    assert np.isfinite(o).all()
+    assert np.abs(lse - l_ref).max() <= L_MAX_ABS
+    # the bound, from the dequantised inputs in fp64
+    q = s_q * orc.e4m3_to_float(q8.numpy())
+    k = s_k * orc.e4m3_to_float(k8.numpy())
+    v = s_v * np.swapaxes(orc.e4m3_to_float(vt8.numpy()), -1, -2)
+    g = H // H_kv
+    ok = orc.allowed_mask(N, N, causal, window)
+    for b in range(B):
+        for h in range(H):
+            sc = wl.scale * (q[b, h] @ k[b, h // g].T)
+            sc = np.where(ok, sc, -np.inf)
+            w = np.exp(sc - sc.max(axis=1, keepdims=True))
+            per = np.where(ok, np.maximum(2.0 ** -4 * w, 2.0 ** -10), 0.0)
+            bound = (per @ np.abs(v[b, h // g])) / w.sum(axis=1, keepdims=True)
+            bound += 2.0 ** -8 * np.abs(o_ref[b, h]) + 1e-3
+            err = np.abs(o[b, h] - o_ref[b, h])
+            assert np.all(err <= bound), (b, h, float((err - bound).max()))
