@@ -42,7 +42,7 @@ GRAD_WORKLOAD = "bwd"
 # --workload choices: the forward workload and the one whose dO seed the backward uses
 BENCH_WORKLOADS = {"causal": ("causal", "bwd"), "long": ("long", "long"), "swa": ("swa", "swa"),
                    "gqa": ("gqa", "gqa"), "decode": ("decode", "decode"), "decode_fp8": ("decode", "decode"),
-                   "d256": ("d256", "d256")}
+                   "d256": ("d256", "d256"), "fp8": ("causal", "bwd")}
 FLUSH_BYTES = 256 << 20      # > 126 MB L2
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -64,7 +64,8 @@ def parse_args():
                          "the pairs the band keeps; decode: one new row per query head over 32768 "
                          "cached keys (B8, 64 query heads on 8 K/V heads), forward only, HBM-bound; "
                          "decode_fp8: the same over an E4M3 K/V cache with per-tensor scales; "
-                         "d256: B2 H16 N4096 head dimension 256, causal, forward+backward")
+                         "d256: B2 H16 N4096 head dimension 256, causal, forward+backward; "
+                         "fp8: the causal shape's forward on E4M3 Q, K, V (V transposed)")
     return ap.parse_args()
 
 
@@ -698,6 +699,151 @@ def run_decode(args, fp8: bool = False):
         print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------- FP8 forward arm
+FP8_OVER_BF16 = 2.0   # nominal dense E4M3 / bf16 tensor throughput of a B200 (4.5 / 2.25 PFLOP/s)
+
+
+def fp8_oracle_sample(seconds: float, max_heads: int | None = None):
+    """Time the oracle's FP8 forward head by head on the causal workload's E4M3 inputs.
+    Returns (flops credited, seconds, heads, cores)."""
+    from oracle import attention as orc
+    from synthetic import WORKLOADS, make_inputs_fp8
+    wl = WORKLOADS["causal"]
+    if "fp8" not in _INPUT_CACHE:
+        _INPUT_CACHE["fp8"] = make_inputs_fp8(wl.with_(B=1, H=4))
+    q8, k8, vt8, s_q, s_k, s_v = _INPUT_CACHE["fp8"]
+    per_head = fwd_flops(1, 1, wl.N, wl.d, wl.causal, wl.window)
+    t0 = time.perf_counter()
+    heads = 0
+    while True:
+        h = heads % 4
+        orc.attention_forward_fp8(q8[:, h:h + 1], k8[:, h:h + 1], vt8[:, h:h + 1], s_q, s_k, s_v, wl.scale,
+                                  wl.causal, wl.window)
+        heads += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or (max_heads is not None and heads >= max_heads):
+            break
+    return per_head * heads, el, heads, blas_threads()
+
+
+def run_fp8(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=300))
+    import exact_io_aware_77_b200 as fa
+    fa.load()
+    from synthetic import WORKLOADS, make_inputs_fp8
+    wl = WORKLOADS["causal"]
+    B, H, N, d = wl.B, wl.H, wl.N, wl.d
+    q8_h, k8_h, vt8_h, s_q, s_k, s_v = make_inputs_fp8(wl)
+    q8, k8, vt8 = (x.to(dev) for x in (q8_h, k8_h, vt8_h))
+    o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flops = fwd_flops(B, H, N, d, wl.causal, wl.window)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        fa.forward_fp8(q8, k8, vt8, s_q, s_k, s_v, wl.scale, wl.causal, wl.window, out=o, lse=lse)
+        if ev:
+            ev[1].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    st = fa.check_status(dev)
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {fa.STATUS_NAMES.get(st, st)}")
+    sampler = ClockSampler(gpu_id_for(local))
+    sampler.start()
+    time.sleep(0.3)
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    wall0 = time.time()
+    for i in range(args.steps):
+        flush.zero_()
+        step(events[i])
+    torch.cuda.synchronize(dev)
+    wall1 = time.time()
+    if world > 1:
+        dist.barrier()
+    sampler.mark(wall0, wall1)
+    time.sleep(0.25)
+    sampler.stop()
+    st = fa.check_status(dev)
+    if st != 0:
+        raise RuntimeError(f"device status after timing: {fa.STATUS_NAMES.get(st, st)}")
+    total = max_over_ranks([sum(e[0].elapsed_time(e[1]) for e in events)], dev)[0]
+    ms = total / args.steps
+    value = job_throughput(world, flops, ms)
+    e2e = None
+    if not args.no_e2e:
+        pin = [x.pin_memory() for x in (q8_h, k8_h, vt8_h)]
+        o_h = torch.empty((B, H, N, d), dtype=torch.bfloat16).pin_memory()
+        l_h = torch.empty((B, H, N), dtype=torch.float32).pin_memory()
+        dq, dk, dvt = (torch.empty_like(x, device=dev) for x in pin)
+
+        def one():
+            for dst, src in zip((dq, dk, dvt), pin):
+                dst.copy_(src, non_blocking=True)
+            fa.forward_fp8(dq, dk, dvt, s_q, s_k, s_v, wl.scale, wl.causal, wl.window, out=o, lse=lse)
+            o_h.copy_(o, non_blocking=True)
+            l_h.copy_(lse, non_blocking=True)
+
+        one()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(1, args.e2e_steps)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            one()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_e2e = max_over_ranks([e0.elapsed_time(e1) / n_e2e], dev)[0]
+        e2e = {"value": round(job_throughput(world, flops, ms_e2e), 3), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": sum(x.numel() for x in pin),
+               "d2h_bytes_per_step": o_h.numel() * 2 + l_h.numel() * 4, "ms_per_step": round(ms_e2e, 3)}
+    peaks, peak_kind = load_peaks()
+    peak = peaks["bf16_tflops"] * FP8_OVER_BF16
+    roofline = {"bound": "tensor", "kernel": "fa_fwd_fp8_kernel", "achieved": round(value / world, 1),
+                "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(value / world / peak, 4),
+                "peak_source": f"{peak_kind} burst bf16 (MEASURED_PEAKS.json) x {FP8_OVER_BF16:g}, the nominal "
+                               f"E4M3/bf16 ratio", "traffic": None}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        f, secs, heads, cores = fp8_oracle_sample(args.cpu_seconds)
+        cpu = {"value": round(f / secs / 1e12, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+               "sample": f"{heads} heads of the causal shape's E4M3 inputs through the fp64 oracle, {secs:.1f} s"}
+    line = {
+        "metric": "attention fwd/bwd TFLOP/s at 1 B200; % of dense BF16 tensor peak",
+        "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3", "data": "synthetic",
+        "config": {"workload": f"FP8 forward: B={B} H={H} N={N} d={d} causal, E4M3 Q, K, V^T with per-tensor "
+                               f"scales from N(0,1)*{wl.std:g} inputs",
+                   "global_batch": B * world, "seq_len": N, "parallelism": f"replicas{world}",
+                   "l2": "flushed (256 MB write) between timed steps, outside the events"},
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps,
+        "clocks": sampler.summary(),
+    }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 # ----------------------------------------------------------------------------- reference arm
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
@@ -707,6 +853,8 @@ def run_reference(args):
     wl = WORKLOADS[WORKLOAD]
     if WORKLOAD == "decode":
         return run_decode_reference(args, wl, fp8=args.workload == "decode_fp8")
+    if args.workload == "fp8":
+        return run_fp8_reference(args, wl)
     import exact_io_aware_77_b200 as fa_pkg   # only to learn whether the path has a backward
     with_bwd = hasattr(fa_pkg, "backward")
     times, flops = [], []
@@ -761,6 +909,30 @@ def run_decode_reference(args, wl, fp8: bool = False):
     print(json.dumps(line), flush=True)
 
 
+def run_fp8_reference(args, wl):
+    times, flops = [], []
+    cores = blas_threads()
+    for i in range(args.warmup + args.steps):
+        f, secs, _, cores = fp8_oracle_sample(0.0, max_heads=1)
+        if i >= args.warmup:
+            times.append(secs)
+            flops.append(f)
+    secs = sum(times)
+    value = sum(flops) / secs / 1e12
+    print(json.dumps({
+        "metric": "attention fwd/bwd TFLOP/s at 1 B200; % of dense BF16 tensor peak",
+        "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * secs / args.steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "impl": "reference",
+        "config": {"workload": f"FP8 forward of the causal shape (B={wl.B} H={wl.H} N={wl.N} d={wl.d}), one head "
+                               f"per step", "global_batch": wl.B, "seq_len": wl.N, "parallelism": "cpu"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": "each step: one head of the E4M3 inputs through the fp64 oracle"},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
 def workload_text(wl, with_bwd: bool) -> str:
     if wl.window:
         band = (f"{'causal' if wl.causal else 'two-sided'} window {wl.window}, FLOPs over the "
@@ -781,6 +953,8 @@ def main():
         run_reference(args)
     elif WORKLOAD == "decode":
         run_decode(args, fp8=args.workload == "decode_fp8")
+    elif args.workload == "fp8":
+        run_fp8(args)
     else:
         run_ours(args)
 

@@ -57,3 +57,24 @@ def assert_grads_close(grads_gpu, grads_ref, what=""):
         errs[name] = rel_l2(gg, r)
         assert errs[name] <= GRAD_REL_L2, (what, errs)
     return errs
+
+
+def fp8_o_bound(q, k, v, scale, causal, window, o_ref):
+    """Per-element bound on |O - O_ref| for the FP8 forward, derived from its arithmetic: P is
+    rounded to E4M3 before P V (relative error <= 2^-4 for normal values, absolute <= 2^-10 below
+    E4M3's normal range) while l sums the exact P, so with w_j = exp(s_j - max s) over the allowed
+    keys, |dO_c| <= sum_j max(2^-4 w_j, 2^-10) |V_jc| / sum_j w_j; plus the bf16 rounding of O
+    (2^-8 |O|) and 1e-3 for the fp32 exponentials and sums.  q [B, H, N, d], k and v [B, H_kv, N, d]
+    (dequantised, fp64)."""
+    from oracle import attention as orc
+    B, H, N, _ = q.shape
+    g = H // k.shape[1]
+    ok = orc.allowed_mask(N, N, causal, window)
+    bound = np.empty_like(o_ref)
+    for b in range(B):
+        for h in range(H):
+            sc = np.where(ok, scale * (q[b, h] @ k[b, h // g].T), -np.inf)
+            w = np.exp(sc - sc.max(axis=1, keepdims=True))
+            per = np.where(ok, np.maximum(2.0 ** -4 * w, 2.0 ** -10), 0.0)
+            bound[b, h] = (per @ np.abs(v[b, h // g])) / w.sum(axis=1, keepdims=True)
+    return bound + 2.0 ** -8 * np.abs(o_ref) + 1e-3

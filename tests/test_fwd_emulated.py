@@ -24,7 +24,7 @@ import torch
 
 from oracle import attention as orc
 from synthetic import Workload, make_inputs, make_inputs_fp8
-from tests.parity import L_MAX_ABS, O_MAX_ABS, O_MEAN_ABS
+from tests.parity import L_MAX_ABS, O_MAX_ABS, O_MEAN_ABS, fp8_o_bound
 
 
 @pytest.fixture(scope="module")
@@ -153,19 +153,8 @@ def test_fwd_fp8_kernel_emulated(emu_fwd, B, H, H_kv, N, causal, window):
     o_ref, l_ref = orc.attention_forward_fp8(q8, k8, vt8, s_q, s_k, s_v, wl.scale, causal, window)
     assert np.isfinite(o).all()
     assert np.abs(lse - l_ref).max() <= L_MAX_ABS
-    # the bound, from the dequantised inputs in fp64
     q = s_q * orc.e4m3_to_float(q8.numpy())
     k = s_k * orc.e4m3_to_float(k8.numpy())
     v = s_v * np.swapaxes(orc.e4m3_to_float(vt8.numpy()), -1, -2)
-    g = H // H_kv
-    ok = orc.allowed_mask(N, N, causal, window)
-    for b in range(B):
-        for h in range(H):
-            sc = wl.scale * (q[b, h] @ k[b, h // g].T)
-            sc = np.where(ok, sc, -np.inf)
-            w = np.exp(sc - sc.max(axis=1, keepdims=True))
-            per = np.where(ok, np.maximum(2.0 ** -4 * w, 2.0 ** -10), 0.0)
-            bound = (per @ np.abs(v[b, h // g])) / w.sum(axis=1, keepdims=True)
-            bound += 2.0 ** -8 * np.abs(o_ref[b, h]) + 1e-3
-            err = np.abs(o[b, h] - o_ref[b, h])
-            assert np.all(err <= bound), (b, h, float((err - bound).max()))
+    bound = fp8_o_bound(q, k, v, wl.scale, causal, window, o_ref)
+    assert np.all(np.abs(o - o_ref) <= bound), float((np.abs(o - o_ref) - bound).max())
