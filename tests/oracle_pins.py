@@ -201,6 +201,19 @@ def golden_examples(orc):
             assert np.max(np.abs(dv - np.array(b["dV"]))) < 1e-12
 
 
+def golden_decode_examples(orc):
+    """Hand-derived decode examples (tests/golden/decode/*.json): new rows at the last key
+    positions, every mask kind, reproduce to 1e-12."""
+    for path in sorted((GOLDEN / "decode").glob("*.json")):
+        g = json.loads(path.read_text())
+        k, v = np.array(g["k"])[None, None], np.array(g["v"])[None, None]
+        for case in g["cases"]:
+            q = np.ones((1, 1, case["n_q"], 1))
+            o, lse = orc.attention_forward_decode(q, k, v, g["scale"], case["causal"], case["window"])
+            assert np.max(np.abs(o[0, 0] - np.array(case["O"]))) < 1e-12, (path.name, case)
+            assert np.max(np.abs(lse[0, 0] - np.array(case["L"]))) < 1e-12, (path.name, case)
+
+
 def _torch_reference(q, k, v, scale, causal, window):
     import torch
     import torch.nn.functional as F
@@ -536,5 +549,5 @@ PINS = {f.__name__: f for f in (
     large_scores, golden_examples, library_forward, library_backward, finite_differences,
     delta_identity, row_blocks_match, pair_count, two_sided_window, shared_kv_library,
     shared_kv_finite_differences, decode_library, decode_scale_zero, decode_last_rows_of_self_attention,
-    e4m3_decoding, fp8kv_decode, fp8_forward, rejects_bad_masks,
+    e4m3_decoding, fp8kv_decode, fp8_forward, golden_decode_examples, rejects_bad_masks,
 )}
