@@ -6,19 +6,23 @@ import os
 import subprocess
 import sys
 
+import pytest
+
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def _run(env_extra):
+def _run(env_extra, workload=None):
     env = dict(os.environ, **env_extra)
+    extra = ["--workload", workload] if workload else []
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
-                          "--warmup", "0"], capture_output=True, text=True, env=env, cwd=ROOT, timeout=600)
+                          "--warmup", "0"] + extra, capture_output=True, text=True, env=env, cwd=ROOT, timeout=600)
     assert out.returncode == 0, out.stderr[-2000:]
     return out.stdout
 
 
-def test_reference_arm_line():
-    lines = [l for l in _run({}).splitlines() if l.strip()]
+@pytest.mark.parametrize("workload", [None, "decode", "decode_fp8", "fp8", "d256"])
+def test_reference_arm_line(workload):
+    lines = [l for l in _run({}, workload).splitlines() if l.strip()]
     assert len(lines) == 1
     rec = json.loads(lines[0])
     for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
