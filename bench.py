@@ -58,6 +58,9 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--persistent-fwd", action="store_true",
+                    help="d 64 / 128 workloads: run the forward on the persistent grid (one CTA per SM "
+                         "looping over the work items) instead of one CTA per item")
     ap.add_argument("--workload", choices=sorted(BENCH_WORKLOADS), default="causal",
                     help="causal: B2 H32 N4096 d128 (the default line); gqa: the same with 8 K/V heads; "
                          "long / swa: N32768 with a one- / two-sided window of 4096, FLOPs counted over "
@@ -126,11 +129,11 @@ def decode_bytes(B, H, H_kv, n_q, n_k, d, causal, window=0, kv_elem_bytes=2) -> 
     return 2 * B * H * n_q * d * 2 + 2 * B * H_kv * keys * d * kv_elem_bytes + B * H * n_q * 4
 
 
-def kernel_names(d: int):
+def kernel_names(d: int, persistent: bool = False):
     """(forward kernel, backward main kernel) names for head dimension d."""
     if d == 256:
         return "fa_fwd256_kernel", "fa_bwd256_kernel"
-    return f"fa_fwd_kernel<{d}>", f"fa_bwd_kernel<{d}>"
+    return f"fa_fwd_{'persist_' if persistent else ''}kernel<{d}>", f"fa_bwd_kernel<{d}>"
 
 
 def max_over_ranks(values, device=None):
@@ -303,6 +306,10 @@ def run_ours(args):
 
     wl = WORKLOADS[WORKLOAD]
     B, H, N, d = wl.B, wl.H, wl.N, wl.d
+    persistent = bool(args.persistent_fwd)
+    if persistent and d == 256:
+        raise SystemExit("--persistent-fwd: the persistent forward covers d 64 and 128")
+    names = kernel_names(d, persistent)
     has_bwd = hasattr(fa, "backward")
     q_h, k_h, v_h = make_inputs(wl)
     do_h = make_grad_output(WORKLOADS[GRAD_WORKLOAD])
@@ -324,7 +331,7 @@ def run_ours(args):
         # kernel, the dominant one, has events of its own
         if ev:
             ev[0].record(stream)
-        fa.forward(q, k, v, wl.scale, wl.causal, wl.window, out=o, lse=lse)
+        fa.forward(q, k, v, wl.scale, wl.causal, wl.window, out=o, lse=lse, persistent=persistent)
         if ev:
             ev[1].record(stream)
         if has_bwd:
@@ -378,7 +385,7 @@ def run_ours(args):
     e2e = None
     if not args.no_e2e:
         e2e = measure_e2e(fa, torch, wl, dev, stream, q_h, k_h, v_h, do_h, has_bwd, args.e2e_steps,
-                          f_fwd + f_bwd, world)
+                          f_fwd + f_bwd, world, persistent)
 
     peaks, peak_kind = load_peaks()
     fwd_ms_avg = fwd_total / args.steps
@@ -386,9 +393,9 @@ def run_ours(args):
     main_ms_avg = main_total / args.steps
     if has_bwd and main_ms_avg > fwd_ms_avg:
         # the backward's conventional FLOPs are all tensor work of the recompute kernel
-        dom, dom_flops, dom_ms = kernel_names(d)[1], f_bwd, main_ms_avg
+        dom, dom_flops, dom_ms = names[1], f_bwd, main_ms_avg
     else:
-        dom, dom_flops, dom_ms = kernel_names(d)[0], f_fwd, fwd_ms_avg
+        dom, dom_flops, dom_ms = names[0], f_fwd, fwd_ms_avg
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 1),
                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
@@ -415,7 +422,8 @@ def run_ours(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": workload_text(wl, has_bwd),
                    "global_batch": B * world, "seq_len": N, "parallelism": f"replicas{world}",
-                   "l2": "flushed (256 MB write) between timed steps, outside the events"},
+                   "l2": "flushed (256 MB write) between timed steps, outside the events",
+                   "fwd_grid": "persistent, one CTA per SM" if persistent else "one CTA per work item"},
         "fwd_tflops": round(job_throughput(world, f_fwd, fwd_ms_avg), 2),
         "fwd_ms": round(fwd_ms_avg, 4),
         "pct_of_measured_peak": round(100 * value / world / peaks["bf16_tflops"], 2),
@@ -424,9 +432,9 @@ def run_ours(args):
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": args.steps * (1 + (3 if has_bwd else 0)),
-        "kernel_ms": {kernel_names(d)[0]: round(fwd_ms_avg, 4),
-                      "fa_bwd_prep+" + kernel_names(d)[1] + "+fa_bwd_dq_final": round(bwd_ms_avg, 4),
-                      kernel_names(d)[1]: round(main_ms_avg, 4)} if has_bwd else None,
+        "kernel_ms": {names[0]: round(fwd_ms_avg, 4),
+                      "fa_bwd_prep+" + names[1] + "+fa_bwd_dq_final": round(bwd_ms_avg, 4),
+                      names[1]: round(main_ms_avg, 4)} if has_bwd else None,
         "clocks": clocks,
     }
     if has_bwd:
@@ -439,7 +447,8 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
 
 
-def measure_e2e(fa, torch, wl, dev, stream, q_h, k_h, v_h, do_h, has_bwd, steps, flops, world):
+def measure_e2e(fa, torch, wl, dev, stream, q_h, k_h, v_h, do_h, has_bwd, steps, flops, world,
+                persistent=False):
     pin = [x.pin_memory() for x in (q_h, k_h, v_h, do_h if has_bwd else q_h[:0])]
     q, k, v = (torch.empty_like(x, device=dev) for x in pin[:3])
     do = torch.empty_like(pin[3], device=dev) if has_bwd else None
@@ -458,7 +467,7 @@ def measure_e2e(fa, torch, wl, dev, stream, q_h, k_h, v_h, do_h, has_bwd, steps,
     def one():
         for dst, src in zip((q, k, v) + ((do,) if has_bwd else ()), pin):
             dst.copy_(src, non_blocking=True)
-        fa.forward(q, k, v, wl.scale, wl.causal, wl.window, out=o, lse=lse)
+        fa.forward(q, k, v, wl.scale, wl.causal, wl.window, out=o, lse=lse, persistent=persistent)
         if has_bwd:
             fa.backward(q, k, v, o, lse, do, wl.scale, wl.causal, wl.window, grads=grads, workspace=ws)
         o_h.copy_(o, non_blocking=True)

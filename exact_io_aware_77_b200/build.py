@@ -18,8 +18,11 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libfa_b200.so")
 SOURCES = ["fa_api.cu"]
-DEPS = ["fa_api.cu", "sm100.cuh", "fwd_kernel.cuh", "bwd_kernel.cuh", "decode_ops.cuh",
-        "decode_kernel.cuh"]
+
+
+def _deps() -> list[str]:
+    """fa_api.cu and every kernel header it may include."""
+    return sorted(f for f in os.listdir(CSRC) if f.endswith((".cu", ".cuh")))
 
 
 def nvcc_path() -> str:
@@ -33,7 +36,7 @@ def _stale() -> bool:
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
-    files = [os.path.join(CSRC, f) for f in DEPS] + [os.path.join(ROOT, "include", "fa.h"), __file__]
+    files = [os.path.join(CSRC, f) for f in _deps()] + [os.path.join(ROOT, "include", "fa.h"), __file__]
     return any(os.path.exists(f) and os.path.getmtime(f) > t for f in files)
 
 

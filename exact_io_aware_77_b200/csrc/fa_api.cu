@@ -12,6 +12,7 @@
 #include "../../include/fa.h"
 
 #include "fwd_kernel.cuh"
+#include "fwd_persist_kernel.cuh"
 #include "fwd256_kernel.cuh"
 #include "fp8_ops.cuh"
 #include "fwd_fp8_kernel.cuh"
@@ -124,32 +125,69 @@ int set_smem(Kernel k, int bytes) {
                                                                                                      : FA_ERR_CUDA;
 }
 
+// tensor maps and parameters of the d = 64 / 128 forward (fwd_kernel.cuh), shared by its two launches
+template <int D>
+bool fwd_setup(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv, int N,
+               const Strides* st, float scale, int causal, int window, CUtensorMap* tq, CUtensorMap* tk,
+               CUtensorMap* tv, FwdParams* prm) {
+  if (!make_map_bf16(tq, q, D, N, H, B, st[0], kBlockM) || !make_map_bf16(tk, k, D, N, H_kv, B, st[1], kBlockN) ||
+      !make_map_bf16(tv, v, D, N, H_kv, B, st[2], kBlockN))
+    return false;
+  prm->o = static_cast<__nv_bfloat16*>(o);
+  prm->lse = lse;
+  prm->N = N;
+  prm->BH = B * H;
+  prm->H = H;
+  prm->group = H / H_kv;
+  prm->o_st = st[3];
+  prm->n_pairs = ((N + kBlockM - 1) / kBlockM + kQTiles - 1) / kQTiles;
+  prm->causal = causal;
+  prm->window = window > N ? N : window;   // a band of N or more keys is no band at all
+  prm->scale_log2 = scale * 1.4426950408889634f;
+  prm->wait_limit_ns = g_wait_limit_ns;
+  return true;
+}
+
+// at least 120 KB of shared memory so that one CTA (and its 512 TMEM columns) owns the SM
+constexpr int fwd_smem_bytes(int struct_bytes) {
+  return struct_bytes + 1024 > 120 * 1024 ? struct_bytes + 1024 : 120 * 1024;
+}
+
 template <int D>
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv, int N,
                const Strides* st, float scale, int causal, int window, cudaStream_t stream) {
-  const int BH = B * H;
   CUtensorMap tq, tk, tv;
-  if (!make_map_bf16(&tq, q, D, N, H, B, st[0], kBlockM) || !make_map_bf16(&tk, k, D, N, H_kv, B, st[1], kBlockN) ||
-      !make_map_bf16(&tv, v, D, N, H_kv, B, st[2], kBlockN))
-    return FA_ERR_CUDA;
   FwdParams prm;
-  prm.o = static_cast<__nv_bfloat16*>(o);
-  prm.lse = lse;
-  prm.N = N;
-  prm.BH = BH;
-  prm.H = H;
-  prm.group = H / H_kv;
-  prm.o_st = st[3];
-  prm.n_pairs = ((N + kBlockM - 1) / kBlockM + kQTiles - 1) / kQTiles;
-  prm.causal = causal;
-  prm.window = window > N ? N : window;   // a band of N or more keys is no band at all
-  prm.scale_log2 = scale * 1.4426950408889634f;
-  prm.wait_limit_ns = g_wait_limit_ns;
-  // at least 120 KB so that one CTA (and its 512 TMEM columns) owns the SM
-  const int smem = int(sizeof(FwdSmem<D>)) + 1024 > 120 * 1024 ? int(sizeof(FwdSmem<D>)) + 1024 : 120 * 1024;
+  if (!fwd_setup<D>(q, k, v, o, lse, B, H, H_kv, N, st, scale, causal, window, &tq, &tk, &tv, &prm))
+    return FA_ERR_CUDA;
+  const int smem = fwd_smem_bytes(int(sizeof(FwdSmem<D>)));
   if (set_smem(fa_fwd_kernel<D>, smem) != FA_OK) return FA_ERR_CUDA;
-  const unsigned grid = unsigned(prm.n_pairs) * unsigned(BH);
+  const unsigned grid = unsigned(prm.n_pairs) * unsigned(prm.BH);
   fa_fwd_kernel<D><<<grid, kFwdThreads, smem, stream>>>(tq, tk, tv, prm);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// the persistent form (fwd_persist_kernel.cuh): `ctas` CTAs, or one per SM when ctas is 0, each
+// looping over the work items blockIdx.x, blockIdx.x + gridDim.x, ...
+template <int D>
+int launch_fwd_persist(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv,
+                       int N, const Strides* st, float scale, int causal, int window, int ctas,
+                       cudaStream_t stream) {
+  CUtensorMap tq, tk, tv;
+  FwdParams prm;
+  if (!fwd_setup<D>(q, k, v, o, lse, B, H, H_kv, N, st, scale, causal, window, &tq, &tk, &tv, &prm))
+    return FA_ERR_CUDA;
+  if (ctas == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&ctas, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return FA_ERR_CUDA;
+  }
+  const long long n_items = (long long)prm.n_pairs * prm.BH;
+  const unsigned grid = unsigned(ctas < n_items ? ctas : n_items);
+  const int smem = fwd_smem_bytes(int(sizeof(FwdPersistSmem<D>)));
+  if (set_smem(fa_fwd_persist_kernel<D>, smem) != FA_OK) return FA_ERR_CUDA;
+  fa_fwd_persist_kernel<D><<<grid, kFwdThreads, smem, stream>>>(tq, tk, tv, prm);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -431,6 +469,29 @@ int fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* 
     case 128: return launch_fwd<128>(q, k, v, o, lse, B, H, H_kv, N, s4, scale, causal, window, s);
     default: return launch_fwd256(q, k, v, o, lse, B, H, H_kv, N, s4, scale, causal, window, s);
   }
+}
+
+int fa_fwd_persistent(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv,
+                      int N, int d, const fa_strides* strides, float scale, int causal, int window, int ctas,
+                      void* stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
+  int st = check_problem(B, H, N, d, scale, causal, window);
+  if (st == FA_OK) st = check_kv_heads(H, H_kv);
+  if (st == FA_OK && d == 256) st = FA_ERR_HEADDIM;
+  if (st == FA_OK && ctas < 0) st = FA_ERR_SHAPE;
+  if (st != FA_OK) return st;
+  Strides s4[4] = {packed(H, N, d), packed(H_kv, N, d), packed(H_kv, N, d), packed(H, N, d)};
+  if (strides)
+    for (int i = 0; i < 4; ++i) {
+      s4[i] = Strides{strides[i].b, strides[i].h, strides[i].n};
+      if (!strides_ok(s4[i])) return FA_ERR_ALIGN;
+    }
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+    return FA_ERR_ALIGN;
+  if ((st = check_device()) != FA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_fwd_persist<64>(q, k, v, o, lse, B, H, H_kv, N, s4, scale, causal, window, ctas, s)
+                 : launch_fwd_persist<128>(q, k, v, o, lse, B, H, H_kv, N, s4, scale, causal, window, ctas, s);
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {

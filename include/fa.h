@@ -166,6 +166,20 @@ FA_EXPORT int fa_bwd_strided(const void* q, const void* k, const void* v, const 
                              size_t workspace_bytes, int phases, void* stream);
 
 /*
+ * fa_fwd_strided computed by a persistent grid: `ctas` CTAs (0: one per SM of the current
+ * device), each looping over the forward's work items (pairs of 128-row query tiles of one
+ * head), so that one item's Q load and first S = Q K^T overlap the previous item's output
+ * write.  The computation is the tiled forward of the FlashAttention (EN) page ("Algorithm"):
+ * the same tiles, online softmax and logsumexp as fa_fwd_strided, whose results it returns to
+ * within rounding (the per-tile arithmetic is the same; only the order in which a CTA meets
+ * the tiles differs).  d is 64 or 128 (FA_ERR_HEADDIM otherwise); ctas < 0 gives FA_ERR_SHAPE.
+ * Arguments, strides, errors, streams and ownership are otherwise as for fa_fwd_strided.
+ */
+FA_EXPORT int fa_fwd_persistent(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                                int H_kv, int N, int d, const fa_strides* strides, float scale, int causal,
+                                int window, int ctas, void* stream);
+
+/*
  * Forward of a few new query rows over a longer key sequence: a generation step over a
  * key/value cache.  The FlashAttention (NL) page names engines for LLM inference that work on
  * the key/value cache during streaming generation ("Gespecialiseerde oplossingen": FlashInfer;

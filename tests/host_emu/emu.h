@@ -35,6 +35,7 @@ using std::min;
 
 struct dim3s { unsigned x = 0, y = 0, z = 0; };
 inline thread_local dim3s threadIdx, blockIdx;
+inline dim3s gridDim, blockDim;   // set by emu_launch for the whole grid
 struct float2 { float x, y; };
 struct float4 { float x, y, z, w; };
 inline float4 make_float4(float a, float b, float c, float d) { return {a, b, c, d}; }
@@ -138,6 +139,8 @@ inline float __shfl_sync(unsigned, float v, int src) {
 // buffer of exactly smem_bytes.
 template <class F>
 void emu_launch(unsigned grid, unsigned block, size_t smem_bytes, F call, unsigned char* external_smem = nullptr) {
+  gridDim = dim3s{grid, 1, 1};
+  blockDim = dim3s{block, 1, 1};
   for (unsigned bx = 0; bx < grid; ++bx) {
     std::vector<unsigned char> own(external_smem ? 1 : (smem_bytes ? smem_bytes : 1), 0xFF);   // NaN-filled
     unsigned char* smem = external_smem ? external_smem : own.data();

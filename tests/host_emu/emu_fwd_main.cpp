@@ -10,6 +10,8 @@
 #elif defined(EMU_FWD_FP8)
 #include "fwd_fp8_kernel.cuh"
 #define EMU_D 128
+#elif defined(EMU_FWD_PERSIST)
+#include "fwd_persist_kernel.cuh"
 #else
 #include "fwd_kernel.cuh"
 #endif
@@ -28,6 +30,8 @@ namespace fa {
 alignas(1024) uint8_t smem_raw[sizeof(Fwd256Smem)];
 #elif defined(EMU_FWD_FP8)
 alignas(1024) uint8_t smem_raw[sizeof(FwdFp8Smem)];
+#elif defined(EMU_FWD_PERSIST)
+alignas(1024) uint8_t smem_raw[sizeof(FwdPersistSmem<EMU_D>)];
 #else
 alignas(1024) uint8_t smem_raw[sizeof(FwdSmem<EMU_D>)];
 #endif
@@ -118,8 +122,13 @@ int main(int argc, char** argv) {
   return 0;
 }
 #else
+// usage (persistent form): ... prefix grid   (grid = the number of persistent CTAs)
 int main(int argc, char** argv) {
+#ifdef EMU_FWD_PERSIST
+  if (argc != 10) { std::fprintf(stderr, "bad args\n"); return 2; }
+#else
   if (argc != 9) { std::fprintf(stderr, "bad args\n"); return 2; }
+#endif
   const int B = atoi(argv[1]), H = atoi(argv[2]), Hkv = atoi(argv[3]), N = atoi(argv[4]), causal = atoi(argv[5]),
             window = atoi(argv[6]);
   const float scale = float(atof(argv[7]));
@@ -154,9 +163,16 @@ int main(int argc, char** argv) {
   prm.window = window > N ? N : window;
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.wait_limit_ns = 60ull * 1000000000ull;
+#ifdef EMU_FWD_PERSIST
+  const unsigned n_items = unsigned(prm.n_pairs) * unsigned(B * H);
+  const unsigned grid = std::min(n_items, unsigned(atoi(argv[9])));
+#else
   const unsigned grid = unsigned(prm.n_pairs) * unsigned(B * H);
+#endif
   std::printf("grid %u smem %zu\n", grid, sizeof(fa::smem_raw));
-#ifdef EMU_FWD256
+#ifdef EMU_FWD_PERSIST
+  emu_launch(grid, kFwdThreads, sizeof(fa::smem_raw), [&] { fa_fwd_persist_kernel<D>(tq, tk, tv, prm); }, fa::smem_raw);
+#elif defined(EMU_FWD256)
   emu_launch(grid, k256Threads, sizeof(fa::smem_raw), [&] { fa_fwd256_kernel(tq, tk, tv, prm); }, fa::smem_raw);
 #else
   emu_launch(grid, kFwdThreads, sizeof(fa::smem_raw), [&] { fa_fwd_kernel<D>(tq, tk, tv, prm); }, fa::smem_raw);

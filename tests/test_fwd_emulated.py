@@ -37,6 +37,10 @@ def emu_fwd(tmp_path_factory):
             128: ("fwd_kernel.cuh", "emu_fwd_main.cpp", "emu_fwd_128", ("EMU_D=128",)),
             256: (["fwd256_kernel.cuh", "fwd_kernel.cuh"], "emu_fwd_main.cpp", "emu_fwd_256", ("EMU_FWD256",)),
             "fp8": (["fwd_fp8_kernel.cuh", "fwd_kernel.cuh"], "emu_fwd_main.cpp", "emu_fwd_fp8", ("EMU_FWD_FP8",)),
+            "persist64": (["fwd_persist_kernel.cuh", "fwd_kernel.cuh"], "emu_fwd_main.cpp", "emu_fwd_persist_64",
+                          ("EMU_FWD_PERSIST", "EMU_D=64")),
+            "persist128": (["fwd_persist_kernel.cuh", "fwd_kernel.cuh"], "emu_fwd_main.cpp", "emu_fwd_persist_128",
+                           ("EMU_FWD_PERSIST", "EMU_D=128")),
         })
     except FileNotFoundError:
         pytest.skip("g++ not available")
@@ -64,6 +68,29 @@ CASES = [
 
 @pytest.mark.parametrize("B,H,H_kv,N,d,causal,window", CASES)
 def test_fwd_kernel_emulated(emu_fwd, B, H, H_kv, N, d, causal, window):
+    _check_fwd_emulated(emu_fwd[d], [], B, H, H_kv, N, d, causal, window)
+
+
+PERSIST_CASES = [
+    # B, H, H_kv, N, d, causal, window, CTAs.  Few CTAs, so that each runs several work items
+    # and every barrier goes through phases across items; causal pairs whose second query tile
+    # lies past N (no keys for it in that item) take the o_free handshake without any P V.
+    (1, 2, 2, 300, 128, True, 0, 1),
+    (2, 2, 1, 600, 128, False, 0, 3),
+    (1, 4, 2, 520, 128, True, 100, 2),
+    (1, 2, 2, 400, 128, False, 50, 3),
+    (2, 2, 1, 257, 64, True, 3, 2),
+    (1, 1, 1, 1000, 64, True, 1, 3),
+]
+
+
+@pytest.mark.parametrize("B,H,H_kv,N,d,causal,window,ctas", PERSIST_CASES)
+def test_fwd_persistent_kernel_emulated(emu_fwd, B, H, H_kv, N, d, causal, window, ctas):
+    """fa_fwd_persist_kernel (the persistent grid: each CTA loops over work items) vs the oracle."""
+    _check_fwd_emulated(emu_fwd[f"persist{d}"], [str(ctas)], B, H, H_kv, N, d, causal, window)
+
+
+def _check_fwd_emulated(exe, extra, B, H, H_kv, N, d, causal, window):
     import subprocess
     wl = Workload("fwd_emu", B, H, N, d, causal, window, seed=91 + N + H_kv, H_kv=H_kv)
     q, k, v = make_inputs(wl)
@@ -71,8 +98,8 @@ def test_fwd_kernel_emulated(emu_fwd, B, H, H_kv, N, d, causal, window):
         pre = os.path.join(tmp, "x")
         for name, t in zip("qkv", (q, k, v)):
             t.contiguous().view(torch.int16).numpy().tofile(pre + "." + name)
-        r = subprocess.run([emu_fwd[d], str(B), str(H), str(H_kv), str(N), str(int(causal)), str(window),
-                            repr(wl.scale), pre], capture_output=True, text=True, timeout=900)
+        r = subprocess.run([exe, str(B), str(H), str(H_kv), str(N), str(int(causal)), str(window),
+                            repr(wl.scale), pre] + extra, capture_output=True, text=True, timeout=900)
         assert r.returncode == 0, r.stdout[-1000:] + r.stderr[-4000:]
         o = np.fromfile(pre + ".o", dtype=np.uint16)
         lse = np.fromfile(pre + ".lse", dtype=np.float32).reshape(B, H, N)

@@ -2,8 +2,8 @@
 
 Marked gpu_pending, not gpu: the B200 runs of the verified suite (-m gpu) do not select these
 until a first GPU run has confirmed them (python -m pytest tests -m gpu_pending).  They cover the
-head-dimension-256 forward and backward, the FP8 (E4M3) forward, and the decode kernels over an
-E4M3 K/V cache and at d = 256, with the tolerances of the other parity tests (the FP8 forward's
+head-dimension-256 forward and backward, the FP8 (E4M3) forward, the decode kernels over an
+E4M3 K/V cache and at d = 256, and the persistent form of the d = 64 / 128 forward, with the tolerances of the other parity tests (the FP8 forward's
 derived per-element bound from tests/parity.py).
 """
 
@@ -42,6 +42,43 @@ def test_d256_forward_and_backward(fa, B, H, H_kv, N, causal, window):
     assert_forward_close(o.cpu(), lse.cpu(), o_ref, l_ref, (B, H, H_kv, N, causal, window))
     refs = orc.attention_backward_shared_kv(q, k, v, do, wl.scale, causal, window)
     assert_grads_close([dq.cpu(), dk.cpu(), dv.cpu()], refs, (B, H, H_kv, N, causal, window))
+
+
+@pytest.mark.parametrize("B,H,H_kv,N,d,causal,window,ctas", [
+    (1, 2, 2, 300, 128, True, 0, 1), (2, 2, 1, 600, 128, False, 0, 3), (1, 4, 2, 520, 128, True, 100, 0),
+    (2, 2, 1, 257, 64, True, 3, 2), (1, 3, 3, 1000, 64, False, 0, 0), (1, 1, 1, 1, 128, True, 0, 0)])
+def test_persistent_forward(fa, B, H, H_kv, N, d, causal, window, ctas):
+    """The persistent grid against the oracle, and bit for bit against the one-item-per-CTA
+    forward: every tile meets the same arithmetic in the same order."""
+    wl = Workload("persist_pending", B, H, N, d, causal, window, seed=141 + N, H_kv=H_kv)
+    q, k, v = make_inputs(wl)
+    qd, kd, vd = (x.cuda() for x in (q, k, v))
+    o, lse = fa.forward(qd, kd, vd, wl.scale, causal, window, persistent=True, ctas=ctas)
+    o1, lse1 = fa.forward(qd, kd, vd, wl.scale, causal, window)
+    assert fa.check_status() == 0
+    o_ref, l_ref = orc.attention_forward_shared_kv(q, k, v, wl.scale, causal, window)
+    assert_forward_close(o.cpu(), lse.cpu(), o_ref, l_ref, (B, H, H_kv, N, d, causal, window, ctas))
+    assert torch.equal(o, o1) and torch.equal(lse, lse1)
+
+
+def test_persistent_forward_full_size(fa):
+    """The causal B2 H32 N4096 d128 workload: the persistent grid (one CTA per SM, several
+    items each) equals the one-item-per-CTA forward bit for bit; sampled rows against the oracle."""
+    from synthetic import WORKLOADS
+    wl = WORKLOADS["causal"]
+    q, k, v = make_inputs(wl)
+    qd, kd, vd = (x.cuda() for x in (q, k, v))
+    o, lse = fa.forward(qd, kd, vd, wl.scale, wl.causal, wl.window, persistent=True)
+    o1, lse1 = fa.forward(qd, kd, vd, wl.scale, wl.causal, wl.window)
+    assert fa.check_status() == 0
+    assert torch.equal(o, o1) and torch.equal(lse, lse1)
+    b, h = 1, 17
+    rows = [0, 127, 128, 2049, wl.N - 1]
+    o_ref, l_ref = orc.attention_forward(q[b:b + 1, h:h + 1], k[b:b + 1, h:h + 1], v[b:b + 1, h:h + 1], wl.scale,
+                                         wl.causal, wl.window)
+    got = to64(o[b, h, rows])
+    assert np.abs(got - o_ref[0, 0, rows]).max() <= 2e-2
+    assert np.abs(to64(lse[b, h, rows]) - l_ref[0, 0, rows]).max() <= L_MAX_ABS
 
 
 @pytest.mark.parametrize("B,H,H_kv,N,causal,window", [
