@@ -61,6 +61,8 @@ def parse_args():
     ap.add_argument("--persistent-fwd", action="store_true",
                     help="d 64 / 128 workloads: run the forward on the persistent grid (one CTA per SM "
                          "looping over the work items) instead of one CTA per item")
+    ap.add_argument("--fwd-schedule", choices=["balanced", "head_major"], default="balanced",
+                    help="item order of the persistent forward")
     ap.add_argument("--workload", choices=sorted(BENCH_WORKLOADS), default="causal",
                     help="causal: B2 H32 N4096 d128 (the default line); gqa: the same with 8 K/V heads; "
                          "long / swa: N32768 with a one- / two-sided window of 4096, FLOPs counted over "
@@ -331,7 +333,8 @@ def run_ours(args):
         # kernel, the dominant one, has events of its own
         if ev:
             ev[0].record(stream)
-        fa.forward(q, k, v, wl.scale, wl.causal, wl.window, out=o, lse=lse, persistent=persistent)
+        fa.forward(q, k, v, wl.scale, wl.causal, wl.window, out=o, lse=lse, persistent=persistent,
+                   schedule=args.fwd_schedule)
         if ev:
             ev[1].record(stream)
         if has_bwd:
@@ -385,7 +388,7 @@ def run_ours(args):
     e2e = None
     if not args.no_e2e:
         e2e = measure_e2e(fa, torch, wl, dev, stream, q_h, k_h, v_h, do_h, has_bwd, args.e2e_steps,
-                          f_fwd + f_bwd, world, persistent)
+                          f_fwd + f_bwd, world, persistent, args.fwd_schedule)
 
     peaks, peak_kind = load_peaks()
     fwd_ms_avg = fwd_total / args.steps
@@ -423,7 +426,8 @@ def run_ours(args):
         "config": {"workload": workload_text(wl, has_bwd),
                    "global_batch": B * world, "seq_len": N, "parallelism": f"replicas{world}",
                    "l2": "flushed (256 MB write) between timed steps, outside the events",
-                   "fwd_grid": "persistent, one CTA per SM" if persistent else "one CTA per work item"},
+                   "fwd_grid": f"persistent, one CTA per SM, {args.fwd_schedule} item order" if persistent
+                   else "one CTA per work item"},
         "fwd_tflops": round(job_throughput(world, f_fwd, fwd_ms_avg), 2),
         "fwd_ms": round(fwd_ms_avg, 4),
         "pct_of_measured_peak": round(100 * value / world / peaks["bf16_tflops"], 2),
@@ -448,7 +452,7 @@ def run_ours(args):
 
 
 def measure_e2e(fa, torch, wl, dev, stream, q_h, k_h, v_h, do_h, has_bwd, steps, flops, world,
-                persistent=False):
+                persistent=False, schedule="balanced"):
     pin = [x.pin_memory() for x in (q_h, k_h, v_h, do_h if has_bwd else q_h[:0])]
     q, k, v = (torch.empty_like(x, device=dev) for x in pin[:3])
     do = torch.empty_like(pin[3], device=dev) if has_bwd else None
@@ -467,7 +471,8 @@ def measure_e2e(fa, torch, wl, dev, stream, q_h, k_h, v_h, do_h, has_bwd, steps,
     def one():
         for dst, src in zip((q, k, v) + ((do,) if has_bwd else ()), pin):
             dst.copy_(src, non_blocking=True)
-        fa.forward(q, k, v, wl.scale, wl.causal, wl.window, out=o, lse=lse, persistent=persistent)
+        fa.forward(q, k, v, wl.scale, wl.causal, wl.window, out=o, lse=lse, persistent=persistent,
+                   schedule=schedule)
         if has_bwd:
             fa.backward(q, k, v, o, lse, do, wl.scale, wl.causal, wl.window, grads=grads, workspace=ws)
         o_h.copy_(o, non_blocking=True)

@@ -72,12 +72,17 @@ def _raise(name, st):
         raise FAError(name, st)
 
 
+_SCHEDULES = {"balanced": _lib.FA_SCHED_BALANCED, "head_major": _lib.FA_SCHED_HEAD_MAJOR}
+
+
 def forward(q, k, v, scale: float | None = None, causal: bool = False, window: int = 0,
-            out=None, lse=None, persistent: bool = False, ctas: int = 0):
+            out=None, lse=None, persistent: bool = False, ctas: int = 0, schedule: str = "balanced"):
     """O, L = attention(Q, K, V); O bf16 [B,H,N,d], L fp32 [B,H,N] (natural-log logsumexp).
 
     d is 64, 128 or 256.  ``persistent`` (d 64 or 128) runs the same tiles on a persistent grid
-    of ``ctas`` CTAs (0: one per SM) that loop over the work items."""
+    of ``ctas`` CTAs (0: one per SM) that loop over the work items, taken in the ``schedule``
+    "balanced" (longest first over all heads when a mask makes the costs differ) or
+    "head_major" order."""
     import torch
     H_kv = _check_qkv(q, k, v)
     B, H, N, d = q.shape
@@ -91,11 +96,13 @@ def forward(q, k, v, scale: float | None = None, causal: bool = False, window: i
     ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr())
     mask = (scale, int(bool(causal)), int(window), _stream_handle(q.device))
     if persistent:
+        if schedule not in _SCHEDULES:
+            raise ValueError(f"schedule must be one of {sorted(_SCHEDULES)}")
         st = None if all(t.is_contiguous() for t in (q, k, v, out)) else _lib.strides_array((q, k, v, out))
         _raise("fa_fwd_persistent", _lib.fa_fwd_persistent(*ptrs, B, H, H_kv, N, d,
                                                            ctypes.addressof(st) if st is not None else 0,
                                                            scale, int(bool(causal)), int(window), int(ctas),
-                                                           _stream_handle(q.device)))
+                                                           _SCHEDULES[schedule], _stream_handle(q.device)))
     elif not all(t.is_contiguous() for t in (q, k, v, out)):
         st = _lib.strides_array((q, k, v, out))
         _raise("fa_fwd_strided", _lib.fa_fwd_strided(*ptrs, B, H, H_kv, N, d, ctypes.addressof(st), *mask))

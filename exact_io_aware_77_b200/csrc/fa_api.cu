@@ -168,10 +168,10 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
 }
 
 // the persistent form (fwd_persist_kernel.cuh): `ctas` CTAs, or one per SM when ctas is 0, each
-// looping over the work items blockIdx.x, blockIdx.x + gridDim.x, ...
+// taking its items round by round from the item order (snake-dealt)
 template <int D>
 int launch_fwd_persist(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv,
-                       int N, const Strides* st, float scale, int causal, int window, int ctas,
+                       int N, const Strides* st, float scale, int causal, int window, int ctas, int schedule,
                        cudaStream_t stream) {
   CUtensorMap tq, tk, tv;
   FwdParams prm;
@@ -185,9 +185,13 @@ int launch_fwd_persist(const void* q, const void* k, const void* v, void* o, flo
   }
   const long long n_items = (long long)prm.n_pairs * prm.BH;
   const unsigned grid = unsigned(ctas < n_items ? ctas : n_items);
+  // an item's cost grows with its query position under a causal mask, and is lower for the first
+  // pairs of a band: then longest first over all heads; with every item alike, head-major
+  const bool costs_vary = causal || (prm.window > 0 && prm.window < N);
+  const int order = schedule == FA_SCHED_BALANCED && costs_vary ? kOrderPairMajor : kOrderHeadMajor;
   const int smem = fwd_smem_bytes(int(sizeof(FwdPersistSmem<D>)));
   if (set_smem(fa_fwd_persist_kernel<D>, smem) != FA_OK) return FA_ERR_CUDA;
-  fa_fwd_persist_kernel<D><<<grid, kFwdThreads, smem, stream>>>(tq, tk, tv, prm);
+  fa_fwd_persist_kernel<D><<<grid, kFwdThreads, smem, stream>>>(tq, tk, tv, prm, order);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -473,12 +477,13 @@ int fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* 
 
 int fa_fwd_persistent(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv,
                       int N, int d, const fa_strides* strides, float scale, int causal, int window, int ctas,
-                      void* stream) {
+                      int schedule, void* stream) {
   if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
   int st = check_problem(B, H, N, d, scale, causal, window);
   if (st == FA_OK) st = check_kv_heads(H, H_kv);
   if (st == FA_OK && d == 256) st = FA_ERR_HEADDIM;
-  if (st == FA_OK && ctas < 0) st = FA_ERR_SHAPE;
+  if (st == FA_OK && (ctas < 0 || (schedule != FA_SCHED_BALANCED && schedule != FA_SCHED_HEAD_MAJOR)))
+    st = FA_ERR_SHAPE;
   if (st != FA_OK) return st;
   Strides s4[4] = {packed(H, N, d), packed(H_kv, N, d), packed(H_kv, N, d), packed(H, N, d)};
   if (strides)
@@ -490,8 +495,9 @@ int fa_fwd_persistent(const void* q, const void* k, const void* v, void* o, floa
     return FA_ERR_ALIGN;
   if ((st = check_device()) != FA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return d == 64 ? launch_fwd_persist<64>(q, k, v, o, lse, B, H, H_kv, N, s4, scale, causal, window, ctas, s)
-                 : launch_fwd_persist<128>(q, k, v, o, lse, B, H, H_kv, N, s4, scale, causal, window, ctas, s);
+  return d == 64
+             ? launch_fwd_persist<64>(q, k, v, o, lse, B, H, H_kv, N, s4, scale, causal, window, ctas, schedule, s)
+             : launch_fwd_persist<128>(q, k, v, o, lse, B, H, H_kv, N, s4, scale, causal, window, ctas, schedule, s);
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {

@@ -37,18 +37,35 @@ struct FwdPersistSmem {
   int abort;
 };
 
-// The work item `item` (of prm.n_pairs * prm.BH, head-major, longest causal pairs first within a
-// head): its head, first query row and the K/V tile ranges of its two query tiles.
+// Orders of the work items (pairs of query tiles of one head).  Head-major keeps the items that
+// run at the same time on few heads (their K/V stay in L2); pair-major puts the longest items of
+// every head first, so that items come in decreasing cost when the mask makes the cost grow
+// with the query position (causal, or a band whose first pairs are short).
+enum : int { kOrderHeadMajor = 0, kOrderPairMajor = 1 };
+
+// The r-th item of this CTA, as a position in the item order, or -1 when it has no r-th item.
+// Rounds of gridDim.x items are dealt out in a snake (round 0 to CTAs 0, 1, ..., round 1 to
+// CTAs G-1, G-2, ...), so that in a cost-decreasing order a CTA that took a costly item in one
+// round takes a cheap one in the next.  Positions grow with r, so the first -1 ends the list.
+__device__ __forceinline__ int persist_item(int n_items, int r) {
+  const long long g = gridDim.x;
+  const long long pos = (long long)r * g + ((r & 1) ? g - 1 - blockIdx.x : blockIdx.x);
+  return pos < n_items ? int(pos) : -1;
+}
+
+// The item at position `pos` of `order`: its head, first query row and the K/V tile ranges of
+// its two query tiles.  Within a head, the longest (last) pair comes first.
 struct FwdItem {
   int bh, b_idx, h_q, h_kv, q0, b0, e0, b1, e1, t_begin, t_end;
 };
-__device__ __forceinline__ FwdItem fwd_item(const FwdParams& prm, int item) {
+__device__ __forceinline__ FwdItem fwd_item(const FwdParams& prm, int order, int pos) {
   FwdItem it;
-  it.bh = item / prm.n_pairs;
+  const int rank = order == kOrderPairMajor ? pos / prm.BH : pos % prm.n_pairs;   // 0 = the longest pair
+  it.bh = order == kOrderPairMajor ? pos % prm.BH : pos / prm.n_pairs;
   it.b_idx = it.bh / prm.H;
   it.h_q = it.bh % prm.H;
   it.h_kv = it.h_q / prm.group;
-  const int pair = prm.n_pairs - 1 - item % prm.n_pairs;
+  const int pair = prm.n_pairs - 1 - rank;
   it.q0 = pair * (kQTiles * kBlockM);
   kv_tile_range(it.q0, prm.N, prm.causal, prm.window, it.b0, it.e0);
   kv_tile_range(it.q0 + kBlockM, prm.N, prm.causal, prm.window, it.b1, it.e1);
@@ -61,7 +78,7 @@ __device__ __forceinline__ FwdItem fwd_item(const FwdParams& prm, int item) {
 template <int D>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_persist_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                          const __grid_constant__ CUtensorMap tm_v, const FwdParams prm) {
+                          const __grid_constant__ CUtensorMap tm_v, const FwdParams prm, const int order) {
   using Smem = FwdPersistSmem<D>;
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -110,8 +127,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       int L_run = 0;   // loads issued over the whole run: load L uses slot L % kSlots
       int n_local = 0;
       bool ok = true;
-      for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x, ++n_local) {
-        const FwdItem w_it = fwd_item(prm, item);
+      for (int pos; ok && (pos = persist_item(n_items, n_local)) >= 0; ++n_local) {
+        const FwdItem w_it = fwd_item(prm, order, pos);
         // the previous item's S products have read Q
         if (n_local > 0 && !mbar_wait(smem_u32(&sm.q_empty), (n_local - 1) & 1, abort, lim)) break;
         mbar_expect_tx(qb, kQTiles * Smem::kTileBytes);
@@ -153,8 +170,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     int L_run = 0;
     int n_local = 0;
     bool ok = true;
-    for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x, ++n_local) {
-      const FwdItem w_it = fwd_item(prm, item);
+    for (int pos; ok && (pos = persist_item(n_items, n_local)) >= 0; ++n_local) {
+      const FwdItem w_it = fwd_item(prm, order, pos);
       const int bw[2] = {w_it.b0, w_it.b1}, ew[2] = {w_it.e0, w_it.e1};
       auto active = [&](int w, int t) { return t >= bw[w] && t < ew[w]; };
       int pv_item[2] = {0, 0};   // this item's P V products per tile (the first overwrites O)
@@ -244,8 +261,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     int s_run = 0;   // S tiles of this query tile consumed over the run (s_full parity)
     int n_local = 0;
     bool ok = true;
-    for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x, ++n_local) {
-      const FwdItem w_it = fwd_item(prm, item);
+    for (int pos; ok && (pos = persist_item(n_items, n_local)) >= 0; ++n_local) {
+      const FwdItem w_it = fwd_item(prm, order, pos);
       const int qw0 = w_it.q0 + w * kBlockM;
       const int qi = qw0 + row;
       const int tb = w == 0 ? w_it.b0 : w_it.b1;

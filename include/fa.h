@@ -170,14 +170,24 @@ FA_EXPORT int fa_bwd_strided(const void* q, const void* k, const void* v, const 
  * device), each looping over the forward's work items (pairs of 128-row query tiles of one
  * head), so that one item's Q load and first S = Q K^T overlap the previous item's output
  * write.  The computation is the tiled forward of the FlashAttention (EN) page ("Algorithm"):
- * the same tiles, online softmax and logsumexp as fa_fwd_strided, whose results it returns to
- * within rounding (the per-tile arithmetic is the same; only the order in which a CTA meets
- * the tiles differs).  d is 64 or 128 (FA_ERR_HEADDIM otherwise); ctas < 0 gives FA_ERR_SHAPE.
- * Arguments, strides, errors, streams and ownership are otherwise as for fa_fwd_strided.
+ * the same tiles, online softmax and logsumexp as fa_fwd_strided, whose results it returns bit
+ * for bit (the per-tile arithmetic and its order within a tile are the same; only which CTA
+ * takes which tile differs).
+ *
+ *   schedule  FA_SCHED_BALANCED: with a causal or banded mask (item costs differ) the items go
+ *             longest first over all heads, dealt to the CTAs round by round in a snake
+ *             (0, 1, ..., G-1, then G-1, ..., 0), which evens out the CTAs' total work; with no
+ *             mask, head-major.  FA_SCHED_HEAD_MAJOR: head-major, longest first within a head,
+ *             snake-dealt the same way.
+ *   d         64 or 128 (FA_ERR_HEADDIM otherwise).
+ *
+ * ctas < 0 or another schedule gives FA_ERR_SHAPE.  Arguments, strides, errors, streams and
+ * ownership are otherwise as for fa_fwd_strided.
  */
+enum { FA_SCHED_BALANCED = 0, FA_SCHED_HEAD_MAJOR = 1 };
 FA_EXPORT int fa_fwd_persistent(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                                 int H_kv, int N, int d, const fa_strides* strides, float scale, int causal,
-                                int window, int ctas, void* stream);
+                                int window, int ctas, int schedule, void* stream);
 
 /*
  * Forward of a few new query rows over a longer key sequence: a generation step over a

@@ -122,10 +122,11 @@ int main(int argc, char** argv) {
   return 0;
 }
 #else
-// usage (persistent form): ... prefix grid   (grid = the number of persistent CTAs)
+// usage (persistent form): ... prefix grid order   (grid: the number of persistent CTAs; order:
+// 0 head-major, 1 pair-major item order)
 int main(int argc, char** argv) {
 #ifdef EMU_FWD_PERSIST
-  if (argc != 10) { std::fprintf(stderr, "bad args\n"); return 2; }
+  if (argc != 11) { std::fprintf(stderr, "bad args\n"); return 2; }
 #else
   if (argc != 9) { std::fprintf(stderr, "bad args\n"); return 2; }
 #endif
@@ -166,12 +167,13 @@ int main(int argc, char** argv) {
 #ifdef EMU_FWD_PERSIST
   const unsigned n_items = unsigned(prm.n_pairs) * unsigned(B * H);
   const unsigned grid = std::min(n_items, unsigned(atoi(argv[9])));
+  const int order = atoi(argv[10]);
 #else
   const unsigned grid = unsigned(prm.n_pairs) * unsigned(B * H);
 #endif
   std::printf("grid %u smem %zu\n", grid, sizeof(fa::smem_raw));
 #ifdef EMU_FWD_PERSIST
-  emu_launch(grid, kFwdThreads, sizeof(fa::smem_raw), [&] { fa_fwd_persist_kernel<D>(tq, tk, tv, prm); }, fa::smem_raw);
+  emu_launch(grid, kFwdThreads, sizeof(fa::smem_raw), [&] { fa_fwd_persist_kernel<D>(tq, tk, tv, prm, order); }, fa::smem_raw);
 #elif defined(EMU_FWD256)
   emu_launch(grid, k256Threads, sizeof(fa::smem_raw), [&] { fa_fwd256_kernel(tq, tk, tv, prm); }, fa::smem_raw);
 #else

@@ -142,6 +142,8 @@ def test_strided_entry_points_validate_strides(lib):
     (dict(N=0), "FA_ERR_SHAPE"),
     (dict(H_kv=3), "FA_ERR_SHAPE"),
     (dict(ctas=-1), "FA_ERR_SHAPE"),
+    (dict(schedule=2), "FA_ERR_SHAPE"),
+    (dict(schedule=-1), "FA_ERR_SHAPE"),
     (dict(d=256), "FA_ERR_HEADDIM"),
     (dict(d=96), "FA_ERR_HEADDIM"),
     (dict(causal=2), "FA_ERR_MASK"),
@@ -150,8 +152,8 @@ def test_strided_entry_points_validate_strides(lib):
     (dict(bad_stride=True), "FA_ERR_ALIGN"),
 ])
 def test_persistent_fwd_rejects_bad_arguments(lib, kw, code):
-    """fa_fwd_persistent: fa_fwd_strided's checks, d 64 or 128 only, ctas >= 0."""
-    a = dict(GOOD, H_kv=GOOD["H"], ctas=0)
+    """fa_fwd_persistent: fa_fwd_strided's checks, d 64 or 128 only, ctas >= 0, a known schedule."""
+    a = dict(GOOD, H_kv=GOOD["H"], ctas=0, schedule=_lib.FA_SCHED_BALANCED)
     ptrs = kw.pop("ptrs", [A + 4096 * i for i in range(5)])
     bad_stride = kw.pop("bad_stride", False)
     a.update(kw)
@@ -161,7 +163,7 @@ def test_persistent_fwd_rejects_bad_arguments(lib, kw, code):
         arr[3] = _lib.FaStrides(2 * 128 * 64, 128 * 64, 12)
     st = _lib.fa_fwd_persistent(*ptrs, a["B"], a["H"], a["H_kv"], a["N"], a["d"],
                                 ctypes.addressof(arr) if arr is not None else None, a["scale"], a["causal"],
-                                a["window"], a["ctas"], None)
+                                a["window"], a["ctas"], a["schedule"], None)
     assert _lib.STATUS_NAMES[st] == code
 
 

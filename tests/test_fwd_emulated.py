@@ -72,22 +72,25 @@ def test_fwd_kernel_emulated(emu_fwd, B, H, H_kv, N, d, causal, window):
 
 
 PERSIST_CASES = [
-    # B, H, H_kv, N, d, causal, window, CTAs.  Few CTAs, so that each runs several work items
-    # and every barrier goes through phases across items; causal pairs whose second query tile
-    # lies past N (no keys for it in that item) take the o_free handshake without any P V.
-    (1, 2, 2, 300, 128, True, 0, 1),
-    (2, 2, 1, 600, 128, False, 0, 3),
-    (1, 4, 2, 520, 128, True, 100, 2),
-    (1, 2, 2, 400, 128, False, 50, 3),
-    (2, 2, 1, 257, 64, True, 3, 2),
-    (1, 1, 1, 1000, 64, True, 1, 3),
+    # B, H, H_kv, N, d, causal, window, CTAs, item order (0 head-major, 1 pair-major).  Few CTAs,
+    # so that each runs several work items (dealt in a snake) and every barrier goes through
+    # phases across items; causal pairs whose second query tile lies past N (no keys for it in
+    # that item) take the o_free handshake without any P V.
+    (1, 2, 2, 300, 128, True, 0, 1, 0),
+    (1, 2, 2, 300, 128, True, 0, 2, 1),
+    (2, 2, 1, 600, 128, False, 0, 3, 0),
+    (1, 4, 2, 520, 128, True, 100, 2, 1),
+    (1, 2, 2, 400, 128, False, 50, 3, 1),
+    (2, 2, 1, 257, 64, True, 3, 2, 0),
+    (1, 1, 1, 1000, 64, True, 1, 3, 1),
+    (2, 3, 3, 700, 64, True, 0, 5, 1),
 ]
 
 
-@pytest.mark.parametrize("B,H,H_kv,N,d,causal,window,ctas", PERSIST_CASES)
-def test_fwd_persistent_kernel_emulated(emu_fwd, B, H, H_kv, N, d, causal, window, ctas):
+@pytest.mark.parametrize("B,H,H_kv,N,d,causal,window,ctas,order", PERSIST_CASES)
+def test_fwd_persistent_kernel_emulated(emu_fwd, B, H, H_kv, N, d, causal, window, ctas, order):
     """fa_fwd_persist_kernel (the persistent grid: each CTA loops over work items) vs the oracle."""
-    _check_fwd_emulated(emu_fwd[f"persist{d}"], [str(ctas)], B, H, H_kv, N, d, causal, window)
+    _check_fwd_emulated(emu_fwd[f"persist{d}"], [str(ctas), str(order)], B, H, H_kv, N, d, causal, window)
 
 
 def _check_fwd_emulated(exe, extra, B, H, H_kv, N, d, causal, window):

@@ -44,16 +44,18 @@ def test_d256_forward_and_backward(fa, B, H, H_kv, N, causal, window):
     assert_grads_close([dq.cpu(), dk.cpu(), dv.cpu()], refs, (B, H, H_kv, N, causal, window))
 
 
-@pytest.mark.parametrize("B,H,H_kv,N,d,causal,window,ctas", [
-    (1, 2, 2, 300, 128, True, 0, 1), (2, 2, 1, 600, 128, False, 0, 3), (1, 4, 2, 520, 128, True, 100, 0),
-    (2, 2, 1, 257, 64, True, 3, 2), (1, 3, 3, 1000, 64, False, 0, 0), (1, 1, 1, 1, 128, True, 0, 0)])
-def test_persistent_forward(fa, B, H, H_kv, N, d, causal, window, ctas):
+@pytest.mark.parametrize("B,H,H_kv,N,d,causal,window,ctas,schedule", [
+    (1, 2, 2, 300, 128, True, 0, 1, "balanced"), (1, 2, 2, 300, 128, True, 0, 2, "head_major"),
+    (2, 2, 1, 600, 128, False, 0, 3, "balanced"), (1, 4, 2, 520, 128, True, 100, 0, "balanced"),
+    (2, 2, 1, 257, 64, True, 3, 2, "head_major"), (1, 3, 3, 1000, 64, False, 0, 0, "balanced"),
+    (2, 3, 3, 700, 64, True, 0, 5, "balanced"), (1, 1, 1, 1, 128, True, 0, 0, "balanced")])
+def test_persistent_forward(fa, B, H, H_kv, N, d, causal, window, ctas, schedule):
     """The persistent grid against the oracle, and bit for bit against the one-item-per-CTA
     forward: every tile meets the same arithmetic in the same order."""
     wl = Workload("persist_pending", B, H, N, d, causal, window, seed=141 + N, H_kv=H_kv)
     q, k, v = make_inputs(wl)
     qd, kd, vd = (x.cuda() for x in (q, k, v))
-    o, lse = fa.forward(qd, kd, vd, wl.scale, causal, window, persistent=True, ctas=ctas)
+    o, lse = fa.forward(qd, kd, vd, wl.scale, causal, window, persistent=True, ctas=ctas, schedule=schedule)
     o1, lse1 = fa.forward(qd, kd, vd, wl.scale, causal, window)
     assert fa.check_status() == 0
     o_ref, l_ref = orc.attention_forward_shared_kv(q, k, v, wl.scale, causal, window)
@@ -61,14 +63,15 @@ def test_persistent_forward(fa, B, H, H_kv, N, d, causal, window, ctas):
     assert torch.equal(o, o1) and torch.equal(lse, lse1)
 
 
-def test_persistent_forward_full_size(fa):
+@pytest.mark.parametrize("schedule", ["balanced", "head_major"])
+def test_persistent_forward_full_size(fa, schedule):
     """The causal B2 H32 N4096 d128 workload: the persistent grid (one CTA per SM, several
     items each) equals the one-item-per-CTA forward bit for bit; sampled rows against the oracle."""
     from synthetic import WORKLOADS
     wl = WORKLOADS["causal"]
     q, k, v = make_inputs(wl)
     qd, kd, vd = (x.cuda() for x in (q, k, v))
-    o, lse = fa.forward(qd, kd, vd, wl.scale, wl.causal, wl.window, persistent=True)
+    o, lse = fa.forward(qd, kd, vd, wl.scale, wl.causal, wl.window, persistent=True, schedule=schedule)
     o1, lse1 = fa.forward(qd, kd, vd, wl.scale, wl.causal, wl.window)
     assert fa.check_status() == 0
     assert torch.equal(o, o1) and torch.equal(lse, lse1)
