@@ -84,6 +84,8 @@ def forward(q, k, v, scale: float | None = None, causal: bool = False, window: i
     "balanced" (longest first over all heads when a mask makes the costs differ) or
     "head_major" order."""
     import torch
+    if persistent and schedule not in _SCHEDULES:
+        raise ValueError(f"schedule must be one of {sorted(_SCHEDULES)}")
     H_kv = _check_qkv(q, k, v)
     B, H, N, d = q.shape
     scale = default_scale(d) if scale is None else float(scale)
@@ -96,8 +98,6 @@ def forward(q, k, v, scale: float | None = None, causal: bool = False, window: i
     ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr())
     mask = (scale, int(bool(causal)), int(window), _stream_handle(q.device))
     if persistent:
-        if schedule not in _SCHEDULES:
-            raise ValueError(f"schedule must be one of {sorted(_SCHEDULES)}")
         st = None if all(t.is_contiguous() for t in (q, k, v, out)) else _lib.strides_array((q, k, v, out))
         _raise("fa_fwd_persistent", _lib.fa_fwd_persistent(*ptrs, B, H, H_kv, N, d,
                                                            ctypes.addressof(st) if st is not None else 0,
