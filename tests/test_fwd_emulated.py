@@ -84,6 +84,8 @@ PERSIST_CASES = [
     (2, 2, 1, 257, 64, True, 3, 2, 0),
     (1, 1, 1, 1000, 64, True, 1, 3, 1),
     (2, 3, 3, 700, 64, True, 0, 5, 1),
+    (1, 1, 1, 1, 128, True, 0, 1, 1),        # N = 1: one row, the pair's second tile empty
+    (1, 2, 1, 129, 64, False, 0, 1, 1),      # one row past a tile, one CTA for both heads
 ]
 
 

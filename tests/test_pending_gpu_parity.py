@@ -63,6 +63,22 @@ def test_persistent_forward(fa, B, H, H_kv, N, d, causal, window, ctas, schedule
     assert torch.equal(o, o1) and torch.equal(lse, lse1)
 
 
+def test_persistent_forward_strided(fa):
+    """Sequence-major [B, N, H, d] arrays (strided views): the persistent grid equals the
+    one-item-per-CTA forward on the same views bit for bit, and the oracle within tolerance."""
+    B, H, H_kv, N, d = 2, 4, 2, 333, 128
+    wl = Workload("persist_strided", B, H, N, d, True, 0, seed=151, H_kv=H_kv)
+    q, k, v = make_inputs(wl)
+    qs, ks, vs = (x.transpose(1, 2).contiguous().cuda().transpose(1, 2) for x in (q, k, v))
+    out = torch.empty(B, N, H, d, dtype=torch.bfloat16, device="cuda").transpose(1, 2)
+    o, lse = fa.forward(qs, ks, vs, wl.scale, True, 0, out=out, persistent=True, ctas=7)
+    o1, lse1 = fa.forward(qs, ks, vs, wl.scale, True, 0)
+    assert fa.check_status() == 0
+    assert torch.equal(o, o1) and torch.equal(lse, lse1)
+    o_ref, l_ref = orc.attention_forward_shared_kv(q, k, v, wl.scale, True, 0)
+    assert_forward_close(o.cpu(), lse.cpu(), o_ref, l_ref, "strided persistent")
+
+
 @pytest.mark.parametrize("schedule", ["balanced", "head_major"])
 def test_persistent_forward_full_size(fa, schedule):
     """The causal B2 H32 N4096 d128 workload: the persistent grid (one CTA per SM, several
