@@ -163,6 +163,9 @@ __global__ void __launch_bounds__(kDecThreads, 2) fa_decode_kernel(const DecPara
   unsigned char* smem = dec_dyn_smem();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;   // MMA fragment row group and column pair
+  // the merge grid may be scheduled once every CTA of this one has started: its CTAs then wait
+  // (grid_dep_wait) on SMs this grid's last wave frees, instead of a launch after it
+  grid_dep_launch_dependents();
 
   int bid = blockIdx.x;
   const int rb = bid % p.row_blocks;
@@ -436,6 +439,7 @@ template <int D>
 __global__ void __launch_bounds__(32 * kDecMergeWarps) fa_decode_merge_kernel(const DecParams p) {
   constexpr float kLn2 = 0.6931471805599453f, kLog2e = 1.4426950408889634f;
   constexpr int C = D / 32;
+  grid_dep_wait();   // the splits' partial results are complete and visible
   const long long grow = (long long)blockIdx.x * kDecMergeWarps + (threadIdx.x >> 5);
   if (grow >= p.total_rows) return;   // whole warps leave together
   const int lane = threadIdx.x & 31;

@@ -89,4 +89,12 @@ __device__ __forceinline__ uint32_t ld_global_u32(const void* p) {
   return *reinterpret_cast<const uint32_t*>(p);
 }
 
+// Programmatic dependent launch.  A grid launched with programmatic stream serialization may be
+// scheduled before the previous grid on its stream has finished: grid_dep_wait blocks until that
+// grid has completed and its memory operations are visible to this one (at once when the grid was
+// launched without the attribute).  grid_dep_launch_dependents lets the next grid be scheduled as
+// soon as every CTA of this grid has issued it or exited.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
+
 }  // namespace fa

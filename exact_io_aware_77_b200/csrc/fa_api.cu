@@ -387,7 +387,19 @@ int launch_decode(const void* q, const void* k, const void* v, void* o, float* l
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   if (pl.n_splits > 1) {
     const long long blocks = (pl.total_rows + kDecMergeWarps - 1) / kDecMergeWarps;
-    fa_decode_merge_kernel<D><<<unsigned(blocks), 32 * kDecMergeWarps, 0, stream>>>(p);
+    // programmatic dependent launch: the merge grid is scheduled under the split grid's last
+    // wave and waits for its results in the kernel (grid_dep_wait)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(blocks));
+    cfg.blockDim = dim3(32 * kDecMergeWarps);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, fa_decode_merge_kernel<D>, p) != cudaSuccess) return FA_ERR_CUDA;
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   return FA_OK;

@@ -122,6 +122,10 @@ inline void cp_async_wait() {
     t_cp.committed.erase(t_cp.committed.begin());
   }
 }
+// programmatic dependent launch: the emulation runs grids one after another, so both are no-ops
+inline void grid_dep_wait() {}
+inline void grid_dep_launch_dependents() {}
+
 inline uint32_t ld_global_u32(const void* p) {
   if (reinterpret_cast<uintptr_t>(p) % 4) { std::fprintf(stderr, "misaligned u32 load\n"); std::abort(); }
   uint32_t v;
