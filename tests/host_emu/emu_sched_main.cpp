@@ -1,0 +1,95 @@
+// TEST INFRASTRUCTURE ONLY: the persistent forward's work-item schedule (persist_item and fwd_item
+// of fwd_persist_kernel.cuh, compiled from the kernel's own source) evaluated on the host for
+// many shapes, grid sizes and both item orders.
+//
+// For each case it checks that the CTAs' item lists together hold every (head, query-tile pair)
+// exactly once, that a CTA's list ends at its first -1 (no later round yields an item), and that
+// every item's K/V tile ranges are the ones kv_tile_range gives its two query tiles.  It prints
+// one line per case: BH N causal window order grid, the largest CTA load and the mean load, in
+// K/V tile steps plus one per item.
+// usage: emu_sched_main   (exit 1 at the first violation)
+#include "emu.h"
+#include "fwd_persist_kernel.cuh"
+
+#include <algorithm>
+#include <cstdio>
+#include <vector>
+
+using namespace fa;
+
+int main() {
+  struct Shape {
+    int BH, N, causal, window;
+  };
+  const Shape shapes[] = {{1, 1, 1, 0},       {1, 128, 0, 0},     {1, 300, 1, 0},        {3, 700, 1, 0},
+                          {4, 520, 1, 100},   {4, 400, 0, 50},    {5, 1000, 1, 1},       {2, 257, 0, 0},
+                          {64, 4096, 1, 0},   {64, 4096, 0, 0},   {16, 32768, 1, 4096},  {16, 32768, 0, 4096},
+                          {128, 1024, 1, 0},  {7, 3000, 1, 600}};
+  const unsigned grids[] = {1, 2, 3, 5, 7, 64, 148, 1000};
+  for (const Shape& sh : shapes) {
+    FwdParams prm{};
+    prm.N = sh.N;
+    prm.BH = sh.BH;
+    prm.H = sh.BH;
+    prm.group = 1;
+    prm.causal = sh.causal;
+    prm.window = std::min(sh.window, sh.N);
+    prm.n_pairs = ((sh.N + kBlockM - 1) / kBlockM + kQTiles - 1) / kQTiles;
+    const int n_items = prm.n_pairs * prm.BH;
+    for (int order : {int(kOrderHeadMajor), int(kOrderPairMajor)}) {
+      for (unsigned G : grids) {
+        const unsigned g = std::min<unsigned>(G, unsigned(n_items));   // the launch's clamp
+        gridDim = dim3s{g, 1, 1};
+        std::vector<int> seen(n_items, 0);
+        long long max_load = 0, total = 0;
+        for (unsigned cta = 0; cta < g; ++cta) {
+          blockIdx = dim3s{cta, 0, 0};
+          long long load = 0;
+          int r = 0;
+          for (;; ++r) {
+            const int pos = persist_item(n_items, r);
+            if (pos < 0) break;
+            if (pos >= n_items) {
+              std::printf("FAIL position %d out of range\n", pos);
+              return 1;
+            }
+            const FwdItem it = fwd_item(prm, order, pos);
+            const int pair = it.q0 / (kQTiles * kBlockM);
+            if (it.bh < 0 || it.bh >= prm.BH || pair < 0 || pair >= prm.n_pairs ||
+                it.q0 != pair * kQTiles * kBlockM || it.b_idx != it.bh / prm.H || it.h_q != it.bh % prm.H) {
+              std::printf("FAIL bad item at position %d\n", pos);
+              return 1;
+            }
+            int b0, e0, b1, e1;
+            kv_tile_range(it.q0, prm.N, prm.causal, prm.window, b0, e0);
+            kv_tile_range(it.q0 + kBlockM, prm.N, prm.causal, prm.window, b1, e1);
+            if (e1 == 0) b1 = e1 = b0;
+            if (it.b0 != b0 || it.e0 != e0 || it.b1 != b1 || it.e1 != e1 || it.t_begin != b0 ||
+                it.t_end != std::max(e0, e1)) {
+              std::printf("FAIL tile ranges of item (%d, %d)\n", it.bh, pair);
+              return 1;
+            }
+            ++seen[it.bh * prm.n_pairs + pair];
+            load += (it.t_end - it.t_begin) + 1;
+          }
+          for (int rr = r + 1; rr < r + 4; ++rr)
+            if (persist_item(n_items, rr) >= 0) {
+              std::printf("FAIL CTA %u has an item after its list ended\n", cta);
+              return 1;
+            }
+          max_load = std::max(max_load, load);
+          total += load;
+        }
+        for (int i = 0; i < n_items; ++i)
+          if (seen[i] != 1) {
+            std::printf("FAIL item %d taken %d times (BH %d N %d order %d grid %u)\n", i, seen[i], sh.BH, sh.N,
+                        order, g);
+            return 1;
+          }
+        std::printf("%d %d %d %d %d %u %lld %.3f\n", sh.BH, sh.N, sh.causal, sh.window, order, g, max_load,
+                    double(total) / g);
+      }
+    }
+  }
+  return 0;
+}

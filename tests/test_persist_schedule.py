@@ -1,0 +1,44 @@
+"""The persistent forward's work-item schedule, compiled from fwd_persist_kernel.cuh and run on
+the host (tests/host_emu/emu_sched_main.cpp): every (head, query-tile pair) goes to exactly one
+CTA for every shape, grid size and item order tried, with the tile ranges of kv_tile_range; and
+on the causal and banded workloads the balanced (pair-major) order brings the largest CTA load
+within a few percent of the mean.  CPU only."""
+
+import subprocess
+
+import pytest
+
+
+@pytest.fixture(scope="module")
+def sched_rows(tmp_path_factory):
+    from tests.host_emu.build_emu import build
+    d = str(tmp_path_factory.mktemp("host_emu_sched"))
+    try:
+        exe = build(d, ["fwd_persist_kernel.cuh", "fwd_kernel.cuh"], "emu_sched_main.cpp", "emu_sched")
+    except FileNotFoundError:
+        pytest.skip("g++ not available")
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-2000:]
+    lines = [l for l in r.stdout.split("\n") if l.strip()]
+    assert len(lines) == 14 * 2 * 8   # shapes x item orders x grid sizes, one line each
+    rows = {}
+    for line in lines:
+        if line.strip():
+            BH, N, causal, window, order, g, max_load, mean = line.split()
+            rows[(int(BH), int(N), int(causal), int(window), int(order), int(g))] = (int(max_load), float(mean))
+    return rows
+
+
+def test_every_item_once(sched_rows):
+    """The harness exits non-zero on any item taken twice or never, and prints a line per case."""
+    assert (64, 4096, 1, 0, 1, 148) in sched_rows and (1, 1, 1, 0, 0, 1) in sched_rows
+
+
+@pytest.mark.parametrize("shape", [(64, 4096, 1, 0), (16, 32768, 1, 4096), (16, 32768, 0, 4096)])
+def test_balanced_order_evens_the_loads(sched_rows, shape):
+    """148 CTAs: causal B2 H32 N4096, and N 32768 with a one- and a two-sided window of 4096."""
+    head_max, mean = sched_rows[shape + (0, 148)]
+    pair_max, mean2 = sched_rows[shape + (1, 148)]
+    assert mean == mean2
+    assert pair_max <= 1.03 * mean, (pair_max, mean)
+    assert pair_max < head_max
