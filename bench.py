@@ -63,6 +63,10 @@ def parse_args():
                          "looping over the work items) instead of one CTA per item")
     ap.add_argument("--fwd-schedule", choices=["balanced", "head_major"], default="balanced",
                     help="item order of the persistent forward")
+    ap.add_argument("--persistent-bwd", action="store_true",
+                    help="d 64 / 128 workloads: run the backward's recompute kernel on the persistent grid")
+    ap.add_argument("--bwd-schedule", choices=["balanced", "head_major"], default="balanced",
+                    help="item order of the persistent backward")
     ap.add_argument("--workload", choices=sorted(BENCH_WORKLOADS), default="causal",
                     help="causal: B2 H32 N4096 d128 (the default line); gqa: the same with 8 K/V heads; "
                          "long / swa: N32768 with a one- / two-sided window of 4096, FLOPs counted over "
@@ -131,11 +135,12 @@ def decode_bytes(B, H, H_kv, n_q, n_k, d, causal, window=0, kv_elem_bytes=2) -> 
     return 2 * B * H * n_q * d * 2 + 2 * B * H_kv * keys * d * kv_elem_bytes + B * H * n_q * 4
 
 
-def kernel_names(d: int, persistent: bool = False):
+def kernel_names(d: int, persistent: bool = False, persistent_bwd: bool = False):
     """(forward kernel, backward main kernel) names for head dimension d."""
     if d == 256:
         return "fa_fwd256_kernel", "fa_bwd256_kernel"
-    return f"fa_fwd_{'persist_' if persistent else ''}kernel<{d}>", f"fa_bwd_kernel<{d}>"
+    return (f"fa_fwd_{'persist_' if persistent else ''}kernel<{d}>",
+            f"fa_bwd_{'persist_' if persistent_bwd else ''}kernel<{d}>")
 
 
 def max_over_ranks(values, device=None):
@@ -309,9 +314,11 @@ def run_ours(args):
     wl = WORKLOADS[WORKLOAD]
     B, H, N, d = wl.B, wl.H, wl.N, wl.d
     persistent = bool(args.persistent_fwd)
-    if persistent and d == 256:
-        raise SystemExit("--persistent-fwd: the persistent forward covers d 64 and 128")
-    names = kernel_names(d, persistent)
+    persistent_bwd = bool(args.persistent_bwd)
+    if (persistent or persistent_bwd) and d == 256:
+        raise SystemExit("--persistent-fwd / --persistent-bwd: the persistent kernels cover d 64 and 128")
+    names = kernel_names(d, persistent, persistent_bwd)
+    bwd_opts = {"persistent": persistent_bwd, "schedule": args.bwd_schedule}
     has_bwd = hasattr(fa, "backward")
     q_h, k_h, v_h = make_inputs(wl)
     do_h = make_grad_output(WORKLOADS[GRAD_WORKLOAD])
@@ -340,7 +347,7 @@ def run_ours(args):
         if has_bwd:
             for i, ph in enumerate((1, 2, 4)):
                 fa.backward(q, k, v, o, lse, do, wl.scale, wl.causal, wl.window, grads=grads, workspace=ws,
-                            phases=ph)
+                            phases=ph, **bwd_opts)
                 if ev:
                     ev[2 + i].record(stream)
 
@@ -388,7 +395,7 @@ def run_ours(args):
     e2e = None
     if not args.no_e2e:
         e2e = measure_e2e(fa, torch, wl, dev, stream, q_h, k_h, v_h, do_h, has_bwd, args.e2e_steps,
-                          f_fwd + f_bwd, world, persistent, args.fwd_schedule)
+                          f_fwd + f_bwd, world, persistent, args.fwd_schedule, bwd_opts)
 
     peaks, peak_kind = load_peaks()
     fwd_ms_avg = fwd_total / args.steps
@@ -427,6 +434,8 @@ def run_ours(args):
                    "global_batch": B * world, "seq_len": N, "parallelism": f"replicas{world}",
                    "l2": "flushed (256 MB write) between timed steps, outside the events",
                    "fwd_grid": f"persistent, one CTA per SM, {args.fwd_schedule} item order" if persistent
+                   else "one CTA per work item",
+                   "bwd_grid": f"persistent, one CTA per SM, {args.bwd_schedule} item order" if persistent_bwd
                    else "one CTA per work item"},
         "fwd_tflops": round(job_throughput(world, f_fwd, fwd_ms_avg), 2),
         "fwd_ms": round(fwd_ms_avg, 4),
@@ -452,7 +461,7 @@ def run_ours(args):
 
 
 def measure_e2e(fa, torch, wl, dev, stream, q_h, k_h, v_h, do_h, has_bwd, steps, flops, world,
-                persistent=False, schedule="balanced"):
+                persistent=False, schedule="balanced", bwd_opts=None):
     """The step through the public API with its host copies inside the timed region: every step
     copies its inputs from pinned host memory to the device and its results (O, L and, with the
     backward, dQ, dK, dV) back to pinned host memory.
@@ -490,7 +499,7 @@ def measure_e2e(fa, torch, wl, dev, stream, q_h, k_h, v_h, do_h, has_bwd, steps,
                    schedule=schedule)
         if has_bwd:
             fa.backward(q, k, v, outs[0], outs[1], ins[3], wl.scale, wl.causal, wl.window,
-                        grads=tuple(outs[2:5]), workspace=ws)
+                        grads=tuple(outs[2:5]), workspace=ws, **(bwd_opts or {}))
 
     def copy_out(outs):
         for h, t in zip((o_h, l_h) + grads_h, outs):

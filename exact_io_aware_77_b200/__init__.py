@@ -154,13 +154,18 @@ def bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
 
 
 def backward(q, k, v, o, lse, do, scale: float | None = None, causal: bool = False, window: int = 0,
-             grads=None, workspace=None, phases: int = 7):
+             grads=None, workspace=None, phases: int = 7, persistent: bool = False, ctas: int = 0,
+             schedule: str = "balanced"):
     """dQ (like q), dK, dV (like k) of sum(O o dO), recomputing P from the forward's L.
 
     ``phases`` selects the steps of the backward (1 preprocess, 2 recompute kernel, 4 dQ
     finalise); running 1, 2, 4 in turn with the same workspace equals the default 7.
+    ``persistent`` (d 64 or 128) runs the recompute kernel on a persistent grid of ``ctas`` CTAs
+    (0: one per SM) that loop over the (K/V head, key tile) items in the ``schedule`` order.
     """
     import torch
+    if persistent and schedule not in _SCHEDULES:
+        raise ValueError(f"schedule must be one of {sorted(_SCHEDULES)}")
     H_kv = _check_qkv(q, k, v, o, do)
     B, H, N, d = q.shape
     _check_lse(lse, q, B * H * N)
@@ -176,6 +181,15 @@ def backward(q, k, v, o, lse, do, scale: float | None = None, causal: bool = Fal
     dq, dk, dv = grads
     ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
             dq.data_ptr(), dk.data_ptr(), dv.data_ptr())
+    if persistent:
+        st = None
+        if not all(t.is_contiguous() for t in (q, k, v, o, do, dq, dk, dv)):
+            st = _lib.strides_array((q, k, v, o, do, dq, dk, dv))
+        _raise("fa_bwd_persistent", _lib.fa_bwd_persistent(
+            *ptrs, B, H, H_kv, N, d, ctypes.addressof(st) if st is not None else 0, scale, int(bool(causal)),
+            int(window), workspace.data_ptr(), workspace.numel() * workspace.element_size(), int(phases), int(ctas),
+            _SCHEDULES[schedule], _stream_handle(q.device)))
+        return dq, dk, dv
     rest = (d, scale, int(bool(causal)), int(window), workspace.data_ptr(),
             workspace.numel() * workspace.element_size())
     if not all(t.is_contiguous() for t in (q, k, v, o, do, dq, dk, dv)):

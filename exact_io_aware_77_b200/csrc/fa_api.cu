@@ -17,6 +17,7 @@
 #include "fp8_ops.cuh"
 #include "fwd_fp8_kernel.cuh"
 #include "bwd_kernel.cuh"
+#include "bwd_persist_kernel.cuh"
 #include "bwd256_kernel.cuh"
 #include "decode_ops.cuh"
 #include "decode_kernel.cuh"
@@ -263,7 +264,8 @@ size_t bwd_workspace_bytes(long long BH, int N, int d) {
 template <int D>
 int launch_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
                void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, const Strides* st, float scale,
-               int causal, int window, void* ws, cudaStream_t stream, int phases = kBwdAllPhases) {
+               int causal, int window, void* ws, cudaStream_t stream, int phases = kBwdAllPhases,
+               int persist_ctas = -1, int schedule = FA_SCHED_BALANCED) {
   // st: q, k, v, o, dO, dq, dk, dv
   const int BH = B * H, BH_kv = B * H_kv;
   const long long Np = padded_rows(N);
@@ -313,6 +315,25 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
     if (set_smem(fa_bwd256_kernel, smem) != FA_OK) return FA_ERR_CUDA;
     fa_bwd256_kernel<<<unsigned(prm.n_kv_tiles) * unsigned(BH_kv) * 2u, kB256Threads, smem, stream>>>(tq, tk, tv, tdo,
                                                                                                          prm);
+  } else if (persist_ctas >= 0) {
+    // the persistent form (bwd_persist_kernel.cuh): persist_ctas CTAs, or one per SM when 0
+    int ctas = persist_ctas;
+    if (ctas == 0) {
+      int dev = 0;
+      if (cudaGetDevice(&dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&ctas, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return FA_ERR_CUDA;
+    }
+    const long long n_items = (long long)prm.n_kv_tiles * BH_kv;
+    const unsigned grid = unsigned(ctas < n_items ? ctas : n_items);
+    // a key tile's cost falls with its position under a causal mask and at a band's edges:
+    // then key-tile-major from tile 0 over all heads; with every item alike, head-major
+    const bool costs_vary = causal || (prm.window > 0 && prm.window < N);
+    const int order = schedule == FA_SCHED_BALANCED && costs_vary ? kOrderPairMajor : kOrderHeadMajor;
+    static_assert(sizeof(BwdPersistSmem<D>) <= 232448, "persistent backward shared memory exceeds 227 KB");
+    const int smem = int(sizeof(BwdPersistSmem<D>));
+    if (set_smem(fa_bwd_persist_kernel<D>, smem) != FA_OK) return FA_ERR_CUDA;
+    fa_bwd_persist_kernel<D><<<grid, kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, prm, order);
   } else {
     static_assert(sizeof(BwdSmem<D>) <= 232448, "backward shared memory exceeds 227 KB");
     const int smem = int(sizeof(BwdSmem<D>));   // the kernel checks that the base is 1 KB aligned
@@ -451,7 +472,7 @@ extern "C" {
 static int bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
                     void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, int d, const fa_strides* strides,
                     float scale, int causal, int window, void* workspace, size_t workspace_bytes, int phases,
-                    void* stream);
+                    void* stream, int persist_ctas = -1, int schedule = FA_SCHED_BALANCED);
 
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
            float scale, int causal, int window, void* stream) {
@@ -550,7 +571,7 @@ int fa_bwd_strided(const void* q, const void* k, const void* v, const void* o, c
 static int bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
                     void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, int d, const fa_strides* strides,
                     float scale, int causal, int window, void* workspace, size_t workspace_bytes, int phases,
-                    void* stream) {
+                    void* stream, int persist_ctas, int schedule) {
   if (phases < 1 || phases > kBwdAllPhases) return FA_ERR_PHASES;
   if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FA_ERR_NULL;
   int st = check_problem(B, H, N, d, scale, causal, window);
@@ -575,10 +596,20 @@ static int bwd_impl(const void* q, const void* k, const void* v, const void* o, 
   if ((st = check_device()) != FA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (d) {
-    case 64: return launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, s8, scale, causal, window, workspace, s, phases);
-    case 128: return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, s8, scale, causal, window, workspace, s, phases);
+    case 64: return launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, s8, scale, causal, window, workspace, s, phases, persist_ctas, schedule);
+    case 128: return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, s8, scale, causal, window, workspace, s, phases, persist_ctas, schedule);
     default: return launch_bwd<256>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, s8, scale, causal, window, workspace, s, phases);
   }
+}
+
+int fa_bwd_persistent(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                      void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, int d, const fa_strides* strides,
+                      float scale, int causal, int window, void* workspace, size_t workspace_bytes, int phases,
+                      int ctas, int schedule, void* stream) {
+  if (ctas < 0 || (schedule != FA_SCHED_BALANCED && schedule != FA_SCHED_HEAD_MAJOR)) return FA_ERR_SHAPE;
+  if (d == 256 && check_problem(B, H, N, d, scale, causal, window) == FA_OK) return FA_ERR_HEADDIM;
+  return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, d, strides, scale, causal, window, workspace,
+                  workspace_bytes, phases, stream, ctas, schedule);
 }
 
 int fa_fwd_fp8(const void* q8, const void* k8, const void* vt8, float q_scale, float k_scale, float v_scale, void* o,

@@ -20,6 +20,7 @@
 #include <type_traits>
 
 #include "fwd_kernel.cuh"
+#include "persist_sched.cuh"
 
 namespace fa {
 
@@ -36,22 +37,6 @@ struct FwdPersistSmem {
   uint32_t tmem_base;
   int abort;
 };
-
-// Orders of the work items (pairs of query tiles of one head).  Head-major keeps the items that
-// run at the same time on few heads (their K/V stay in L2); pair-major puts the longest items of
-// every head first, so that items come in decreasing cost when the mask makes the cost grow
-// with the query position (causal, or a band whose first pairs are short).
-enum : int { kOrderHeadMajor = 0, kOrderPairMajor = 1 };
-
-// The r-th item of this CTA, as a position in the item order, or -1 when it has no r-th item.
-// Rounds of gridDim.x items are dealt out in a snake (round 0 to CTAs 0, 1, ..., round 1 to
-// CTAs G-1, G-2, ...), so that in a cost-decreasing order a CTA that took a costly item in one
-// round takes a cheap one in the next.  Positions grow with r, so the first -1 ends the list.
-__device__ __forceinline__ int persist_item(int n_items, int r) {
-  const long long g = gridDim.x;
-  const long long pos = (long long)r * g + ((r & 1) ? g - 1 - blockIdx.x : blockIdx.x);
-  return pos < n_items ? int(pos) : -1;
-}
 
 // The item at position `pos` of `order`: its head, first query row and the K/V tile ranges of
 // its two query tiles.  Within a head, the longest (last) pair comes first.

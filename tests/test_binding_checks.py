@@ -54,3 +54,5 @@ def test_persistent_schedule_name_checked_first():
         fa.forward(q, q, q, persistent=True, schedule="pair_major")
     with pytest.raises(ValueError, match="bf16 CUDA tensors"):   # a known name passes on to the tensor checks
         fa.forward(q, q, q, persistent=True, schedule="head_major")
+    with pytest.raises(ValueError, match="schedule"):
+        fa.backward(q, q, q, q, None, q, persistent=True, schedule="cost")

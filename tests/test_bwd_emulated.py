@@ -31,6 +31,10 @@ def emu_bwd(tmp_path_factory):
             64: ("bwd_kernel.cuh", "emu_bwd_main.cpp", "emu_bwd_64", ("EMU_D=64",)),
             128: ("bwd_kernel.cuh", "emu_bwd_main.cpp", "emu_bwd_128", ("EMU_D=128",)),
             256: (["bwd256_kernel.cuh", "bwd_kernel.cuh"], "emu_bwd_main.cpp", "emu_bwd_256", ("EMU_BWD256",)),
+            "persist64": (["bwd_persist_kernel.cuh", "bwd_kernel.cuh", "persist_sched.cuh"], "emu_bwd_main.cpp",
+                          "emu_bwd_persist_64", ("EMU_BWD_PERSIST", "EMU_D=64")),
+            "persist128": (["bwd_persist_kernel.cuh", "bwd_kernel.cuh", "persist_sched.cuh"], "emu_bwd_main.cpp",
+                           "emu_bwd_persist_128", ("EMU_BWD_PERSIST", "EMU_D=128")),
         })
     except FileNotFoundError:
         pytest.skip("g++ not available")
@@ -55,6 +59,29 @@ def _bits(t):
 
 @pytest.mark.parametrize("B,H,H_kv,N,d,causal,window", CASES)
 def test_bwd_kernels_emulated(emu_bwd, B, H, H_kv, N, d, causal, window):
+    _check_bwd_emulated(emu_bwd[d], [], B, H, H_kv, N, d, causal, window)
+
+
+PERSIST_CASES = [
+    # B, H, H_kv, N, d, causal, window, CTAs, item order (0 head-major, 1 cost-major).  Few CTAs,
+    # so that each runs several (K/V head, key tile) items and every ring and barrier goes through
+    # phases across items.
+    (1, 2, 2, 300, 128, True, 0, 1, 0),
+    (1, 2, 2, 300, 128, True, 0, 2, 1),
+    (1, 4, 2, 400, 128, False, 50, 3, 1),
+    (2, 2, 1, 257, 64, True, 3, 2, 0),
+    (1, 1, 1, 600, 64, True, 1, 3, 1),
+    (2, 2, 2, 520, 64, True, 0, 5, 1),
+]
+
+
+@pytest.mark.parametrize("B,H,H_kv,N,d,causal,window,ctas,order", PERSIST_CASES)
+def test_bwd_persistent_kernel_emulated(emu_bwd, B, H, H_kv, N, d, causal, window, ctas, order):
+    """fa_bwd_persist_kernel (each CTA loops over work items) with the same prep and dQ finalise."""
+    _check_bwd_emulated(emu_bwd[f"persist{d}"], [str(ctas), str(order)], B, H, H_kv, N, d, causal, window)
+
+
+def _check_bwd_emulated(exe, extra, B, H, H_kv, N, d, causal, window):
     wl = Workload("bwd_emu", B, H, N, d, causal, window, seed=95 + N + H_kv, H_kv=H_kv)
     q, k, v = make_inputs(wl)
     do = make_grad_output(wl)
@@ -64,8 +91,8 @@ def test_bwd_kernels_emulated(emu_bwd, B, H, H_kv, N, d, causal, window):
         for name, t in (("q", q), ("k", k), ("v", v), ("o", torch.from_numpy(o_ref).to(torch.bfloat16)), ("do", do)):
             _bits(t).tofile(pre + "." + name)
         l_ref.astype(np.float32).tofile(pre + ".lse")
-        r = subprocess.run([emu_bwd[d], str(B), str(H), str(H_kv), str(N), str(int(causal)), str(window),
-                            repr(wl.scale), pre], capture_output=True, text=True, timeout=1800)
+        r = subprocess.run([exe, str(B), str(H), str(H_kv), str(N), str(int(causal)), str(window),
+                            repr(wl.scale), pre] + extra, capture_output=True, text=True, timeout=1800)
         assert r.returncode == 0, r.stdout[-1000:] + r.stderr[-4000:]
         outs = [torch.from_numpy(np.fromfile(pre + "." + n, dtype=np.int16)).view(torch.bfloat16).double().numpy()
                 for n in ("dq", "dk", "dv")]

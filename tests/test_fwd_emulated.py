@@ -37,9 +37,9 @@ def emu_fwd(tmp_path_factory):
             128: ("fwd_kernel.cuh", "emu_fwd_main.cpp", "emu_fwd_128", ("EMU_D=128",)),
             256: (["fwd256_kernel.cuh", "fwd_kernel.cuh"], "emu_fwd_main.cpp", "emu_fwd_256", ("EMU_FWD256",)),
             "fp8": (["fwd_fp8_kernel.cuh", "fwd_kernel.cuh"], "emu_fwd_main.cpp", "emu_fwd_fp8", ("EMU_FWD_FP8",)),
-            "persist64": (["fwd_persist_kernel.cuh", "fwd_kernel.cuh"], "emu_fwd_main.cpp", "emu_fwd_persist_64",
+            "persist64": (["fwd_persist_kernel.cuh", "fwd_kernel.cuh", "persist_sched.cuh"], "emu_fwd_main.cpp", "emu_fwd_persist_64",
                           ("EMU_FWD_PERSIST", "EMU_D=64")),
-            "persist128": (["fwd_persist_kernel.cuh", "fwd_kernel.cuh"], "emu_fwd_main.cpp", "emu_fwd_persist_128",
+            "persist128": (["fwd_persist_kernel.cuh", "fwd_kernel.cuh", "persist_sched.cuh"], "emu_fwd_main.cpp", "emu_fwd_persist_128",
                            ("EMU_FWD_PERSIST", "EMU_D=128")),
         })
     except FileNotFoundError:

@@ -79,6 +79,29 @@ def test_persistent_forward_strided(fa):
     assert_forward_close(o.cpu(), lse.cpu(), o_ref, l_ref, "strided persistent")
 
 
+@pytest.mark.parametrize("B,H,H_kv,N,d,causal,window,ctas,schedule", [
+    (1, 2, 2, 300, 128, True, 0, 1, "balanced"), (1, 4, 2, 400, 128, False, 50, 3, "balanced"),
+    (2, 2, 1, 257, 64, True, 3, 2, "head_major"), (2, 2, 2, 520, 64, True, 0, 0, "balanced"),
+    (1, 2, 2, 1000, 128, False, 0, 0, "head_major")])
+def test_persistent_backward(fa, B, H, H_kv, N, d, causal, window, ctas, schedule):
+    """The persistent recompute kernel against the oracle; dK and dV bit for bit against the
+    one-item-per-CTA kernel (each is summed inside one CTA), dQ to rounding (its fp32 reductions
+    arrive in hardware order in both)."""
+    wl = Workload("persist_bwd_pending", B, H, N, d, causal, window, seed=161 + N, H_kv=H_kv)
+    q, k, v = make_inputs(wl)
+    do = make_grad_output(wl)
+    qd, kd, vd, dod = (x.cuda() for x in (q, k, v, do))
+    o, lse = fa.forward(qd, kd, vd, wl.scale, causal, window)
+    dq, dk, dv = fa.backward(qd, kd, vd, o, lse, dod, wl.scale, causal, window, persistent=True, ctas=ctas,
+                             schedule=schedule)
+    dq1, dk1, dv1 = fa.backward(qd, kd, vd, o, lse, dod, wl.scale, causal, window)
+    assert fa.check_status() == 0
+    assert torch.equal(dk, dk1) and torch.equal(dv, dv1)
+    assert (dq.float() - dq1.float()).abs().max().item() <= 1e-2 * max(dq1.float().abs().max().item(), 1e-3)
+    refs = orc.attention_backward_shared_kv(q, k, v, do, wl.scale, causal, window)
+    assert_grads_close([dq.cpu(), dk.cpu(), dv.cpu()], refs, (B, H, H_kv, N, d, causal, window, ctas, schedule))
+
+
 @pytest.mark.parametrize("schedule", ["balanced", "head_major"])
 def test_persistent_forward_full_size(fa, schedule):
     """The causal B2 H32 N4096 d128 workload: the persistent grid (one CTA per SM, several

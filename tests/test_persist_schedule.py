@@ -14,7 +14,7 @@ def sched_rows(tmp_path_factory):
     from tests.host_emu.build_emu import build
     d = str(tmp_path_factory.mktemp("host_emu_sched"))
     try:
-        exe = build(d, ["fwd_persist_kernel.cuh", "fwd_kernel.cuh"], "emu_sched_main.cpp", "emu_sched")
+        exe = build(d, ["fwd_persist_kernel.cuh", "fwd_kernel.cuh", "persist_sched.cuh"], "emu_sched_main.cpp", "emu_sched")
     except FileNotFoundError:
         pytest.skip("g++ not available")
     r = subprocess.run([exe], capture_output=True, text=True, timeout=600)
