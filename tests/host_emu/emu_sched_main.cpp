@@ -1,15 +1,18 @@
-// TEST INFRASTRUCTURE ONLY: the persistent forward's work-item schedule (persist_item and fwd_item
-// of fwd_persist_kernel.cuh, compiled from the kernel's own source) evaluated on the host for
-// many shapes, grid sizes and both item orders.
+// TEST INFRASTRUCTURE ONLY: the persistent kernels' work-item schedules (persist_item, and
+// fwd_item of fwd_persist_kernel.cuh / bwd_item of bwd_persist_kernel.cuh, compiled from the
+// kernels' own source) evaluated on the host for many shapes, grid sizes and both item orders.
 //
 // For each case it checks that the CTAs' item lists together hold every (head, query-tile pair)
 // exactly once, that a CTA's list ends at its first -1 (no later round yields an item), and that
 // every item's K/V tile ranges are the ones kv_tile_range gives its two query tiles.  It prints
 // one line per case: BH N causal window order grid, the largest CTA load and the mean load, in
-// K/V tile steps plus one per item.
+// K/V tile steps plus one per item.  Then the same coverage check for the backward's items
+// (K/V head, key tile) with q_tile_range's query tiles, for 1, 2 and 4 query heads per K/V
+// head, printing "bwd" lines with the loads in query iterations plus one per item.
 // usage: emu_sched_main   (exit 1 at the first violation)
 #include "emu.h"
 #include "fwd_persist_kernel.cuh"
+#include "bwd_persist_kernel.cuh"
 
 #include <algorithm>
 #include <cstdio>
@@ -88,6 +91,61 @@ int main() {
           }
         std::printf("%d %d %d %d %d %u %lld %.3f\n", sh.BH, sh.N, sh.causal, sh.window, order, g, max_load,
                     double(total) / g);
+      }
+    }
+  }
+  // the backward: BH here counts query heads; the items are (K/V head, key tile)
+  for (const Shape& sh : shapes) {
+    for (int group : {1, 2, 4}) {
+      if (sh.BH % group) continue;
+      BwdParams prm{};
+      prm.N = sh.N;
+      prm.BH = sh.BH;
+      prm.H = sh.BH;   // one batch entry
+      prm.H_kv = sh.BH / group;
+      prm.group = group;
+      prm.causal = sh.causal;
+      prm.window = std::min(sh.window, sh.N);
+      prm.n_kv_tiles = (sh.N + kBwdKeys - 1) / kBwdKeys;
+      const int n_items = prm.n_kv_tiles * prm.H_kv;
+      for (int order : {int(kOrderHeadMajor), int(kOrderPairMajor)}) {
+        for (unsigned G : grids) {
+          const unsigned g = std::min<unsigned>(G, unsigned(n_items));
+          gridDim = dim3s{g, 1, 1};
+          std::vector<int> seen(n_items, 0);
+          long long max_load = 0, total = 0;
+          for (unsigned cta = 0; cta < g; ++cta) {
+            blockIdx = dim3s{cta, 0, 0};
+            long long load = 0;
+            for (int r = 0;; ++r) {
+              const int pos = persist_item(n_items, r);
+              if (pos < 0) break;
+              const BwdItem it = bwd_item(prm, order, pos);
+              const int tile = it.kv0 / kBwdKeys;
+              int ib, ie;
+              q_tile_range(it.kv0, prm.N, prm.causal, prm.window, ib, ie);
+              if (it.b_idx != 0 || it.h_kv < 0 || it.h_kv >= prm.H_kv || tile < 0 || tile >= prm.n_kv_tiles ||
+                  it.kv0 != tile * kBwdKeys || it.i_begin != ib || it.n_i != ie - ib || it.n_i < 1 ||
+                  it.n_it != it.n_i * group || it.bh_q0 != it.h_kv * group ||
+                  bwd_q_head(it, group, it.n_it - 1) != it.bh_q0 + group - 1 ||
+                  bwd_q_tile(it, group, it.n_it - 1) != ie - 1) {
+                std::printf("FAIL bwd item at position %d\n", pos);
+                return 1;
+              }
+              ++seen[it.h_kv * prm.n_kv_tiles + tile];
+              load += it.n_it + 1;
+            }
+            max_load = std::max(max_load, load);
+            total += load;
+          }
+          for (int i = 0; i < n_items; ++i)
+            if (seen[i] != 1) {
+              std::printf("FAIL bwd item %d taken %d times\n", i, seen[i]);
+              return 1;
+            }
+          std::printf("bwd %d %d %d %d %d %d %u %lld %.3f\n", sh.BH, group, sh.N, sh.causal, sh.window, order, g,
+                      max_load, double(total) / g);
+        }
       }
     }
   }

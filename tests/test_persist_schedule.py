@@ -1,8 +1,9 @@
-"""The persistent forward's work-item schedule, compiled from fwd_persist_kernel.cuh and run on
-the host (tests/host_emu/emu_sched_main.cpp): every (head, query-tile pair) goes to exactly one
-CTA for every shape, grid size and item order tried, with the tile ranges of kv_tile_range; and
-on the causal and banded workloads the balanced (pair-major) order brings the largest CTA load
-within a few percent of the mean.  CPU only."""
+"""The persistent kernels' work-item schedules, compiled from fwd_persist_kernel.cuh and
+bwd_persist_kernel.cuh and run on the host (tests/host_emu/emu_sched_main.cpp): every forward item
+(head, query-tile pair) and every backward item (K/V head, key tile) goes to exactly one CTA for
+every shape, grid size and item order tried, with the tile ranges of kv_tile_range / q_tile_range;
+and on the causal and banded workloads the balanced order brings the largest CTA load within a
+few percent of the mean.  CPU only."""
 
 import subprocess
 
@@ -14,18 +15,25 @@ def sched_rows(tmp_path_factory):
     from tests.host_emu.build_emu import build
     d = str(tmp_path_factory.mktemp("host_emu_sched"))
     try:
-        exe = build(d, ["fwd_persist_kernel.cuh", "fwd_kernel.cuh", "persist_sched.cuh"], "emu_sched_main.cpp", "emu_sched")
+        exe = build(d, ["fwd_persist_kernel.cuh", "fwd_kernel.cuh", "persist_sched.cuh", "bwd_persist_kernel.cuh",
+                        "bwd_kernel.cuh"], "emu_sched_main.cpp", "emu_sched")
     except FileNotFoundError:
         pytest.skip("g++ not available")
     r = subprocess.run([exe], capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-2000:]
     lines = [l for l in r.stdout.split("\n") if l.strip()]
-    assert len(lines) == 14 * 2 * 8   # shapes x item orders x grid sizes, one line each
+    fwd = [l for l in lines if not l.startswith("bwd")]
+    bwd = [l for l in lines if l.startswith("bwd")]
+    assert len(fwd) == 14 * 2 * 8   # shapes x item orders x grid sizes, one line each
+    assert len(bwd) >= 14 * 2 * 8   # and per query heads per K/V head that divide the heads
     rows = {}
-    for line in lines:
-        if line.strip():
-            BH, N, causal, window, order, g, max_load, mean = line.split()
-            rows[(int(BH), int(N), int(causal), int(window), int(order), int(g))] = (int(max_load), float(mean))
+    for line in fwd:
+        BH, N, causal, window, order, g, max_load, mean = line.split()
+        rows[(int(BH), int(N), int(causal), int(window), int(order), int(g))] = (int(max_load), float(mean))
+    for line in bwd:
+        _, BH, group, N, causal, window, order, g, max_load, mean = line.split()
+        rows[("bwd", int(BH), int(group), int(N), int(causal), int(window), int(order), int(g))] = (int(max_load),
+                                                                                                   float(mean))
     return rows
 
 
@@ -42,3 +50,14 @@ def test_balanced_order_evens_the_loads(sched_rows, shape):
     assert mean == mean2
     assert pair_max <= 1.03 * mean, (pair_max, mean)
     assert pair_max < head_max
+
+
+@pytest.mark.parametrize("group,slack", [(1, 1.03), (4, 1.06)])
+def test_backward_balanced_order(sched_rows, group, slack):
+    """Causal B2 H32 N4096 (64 query heads), with 1 or 4 query heads per K/V head, 148 CTAs: the
+    balanced (key-tile-major) order's largest load is within 3 % of the mean, or 6 % with 4 query
+    heads per K/V head, whose 512 items (up to 129 load units each) are too coarse for less."""
+    head_max, mean = sched_rows[("bwd", 64, group, 4096, 1, 0, 0, 148)]
+    bal_max, _ = sched_rows[("bwd", 64, group, 4096, 1, 0, 1, 148)]
+    assert bal_max <= slack * mean, (bal_max, mean)
+    assert bal_max <= head_max
