@@ -116,11 +116,12 @@ def _check_fwd_emulated(exe, extra, B, H, H_kv, N, d, causal, window):
     assert np.abs(lse - l_ref).max() <= L_MAX_ABS
 
 
-@pytest.mark.parametrize("d", [128, 256])
-def test_fwd_kernel_emulated_late_rescales(emu_fwd, d):
+@pytest.mark.parametrize("d,persistent", [(128, False), (256, False), (128, True)])
+def test_fwd_kernel_emulated_late_rescales(emu_fwd, d, persistent):
     """Keys that score ever higher along the sequence make many rows' maxima grow by more than
     2^8 after their first key tile, so the lazy rescale of O runs at later tiles (with the d = 256
-    kernel's two S buffers it must first wait for the previous P V product)."""
+    kernel's two S buffers it must first wait for the previous P V product; the persistent
+    kernel runs both work items on one CTA, in the pair-major order)."""
     import subprocess
     N = 400
     g = torch.Generator().manual_seed(97)
@@ -136,7 +137,8 @@ def test_fwd_kernel_emulated_late_rescales(emu_fwd, d):
         pre = os.path.join(tmp, "x")
         for name, t in zip("qkv", (q, k, v)):
             t.contiguous().view(torch.int16).numpy().tofile(pre + "." + name)
-        r = subprocess.run([emu_fwd[d], "1", "1", "1", str(N), "1", "0", repr(scale), pre],
+        exe, extra = (emu_fwd["persist128"], ["1", "1"]) if persistent else (emu_fwd[d], [])
+        r = subprocess.run([exe, "1", "1", "1", str(N), "1", "0", repr(scale), pre] + extra,
                            capture_output=True, text=True, timeout=900)
         assert r.returncode == 0, r.stderr[-4000:]
         o = np.fromfile(pre + ".o", dtype=np.uint16)
