@@ -106,6 +106,11 @@ inline thread_local CpAsyncState t_cp;
 inline void cp_async_16(void* dst, const void* src, int n) {
   if (n != 16 && n != 0) { std::fprintf(stderr, "bad cp.async size %d\n", n); std::abort(); }
   if (reinterpret_cast<uintptr_t>(dst) % 16) { std::fprintf(stderr, "cp.async destination not 16-byte aligned\n"); std::abort(); }
+#ifdef EMU_EAGER_COPIES
+  if (n == 16) std::memcpy(dst, src, 16);
+  else std::memset(dst, 0, 16);
+  return;
+#endif
   t_cp.open.push_back([=] {
     if (n == 16) std::memcpy(dst, src, 16);
     else std::memset(dst, 0, 16);
@@ -310,7 +315,15 @@ inline void land_copies(uint32_t bar) {
   }
   for (auto& f : todo) f();
 }
+// By default a copy lands only when its barrier is tested (late: a consumer that skips its wait
+// reads stale data).  Built with EMU_EAGER_COPIES it lands at issue instead (early: a producer
+// that skips its wait for the consumers' release overwrites data they still need).  Both are
+// schedules the hardware may take.
 inline void queue_copy(uint32_t bar, std::function<void()> f) {
+#ifdef EMU_EAGER_COPIES
+  f();
+  return;
+#endif
   std::lock_guard<std::mutex> lk(*g_blk->mu);
   g_blk->copies->push_back(PendingOp{bar, std::move(f)});
 }

@@ -35,6 +35,8 @@ def emu_bwd(tmp_path_factory):
                           "emu_bwd_persist_64", ("EMU_BWD_PERSIST", "EMU_D=64")),
             "persist128": (["bwd_persist_kernel.cuh", "bwd_kernel.cuh", "persist_sched.cuh"], "emu_bwd_main.cpp",
                            "emu_bwd_persist_128", ("EMU_BWD_PERSIST", "EMU_D=128")),
+            "persist128_eager": (["bwd_persist_kernel.cuh", "bwd_kernel.cuh", "persist_sched.cuh"], "emu_bwd_main.cpp",
+                                 "emu_bwd_persist_128_eager", ("EMU_BWD_PERSIST", "EMU_D=128", "EMU_EAGER_COPIES")),
         })
     except FileNotFoundError:
         pytest.skip("g++ not available")
@@ -79,6 +81,14 @@ PERSIST_CASES = [
 def test_bwd_persistent_kernel_emulated(emu_bwd, B, H, H_kv, N, d, causal, window, ctas, order):
     """fa_bwd_persist_kernel (each CTA loops over work items) with the same prep and dQ finalise."""
     _check_bwd_emulated(emu_bwd[f"persist{d}"], [str(ctas), str(order)], B, H, H_kv, N, d, causal, window)
+
+
+@pytest.mark.parametrize("B,H,H_kv,N,causal,window,ctas,order", [
+    (1, 2, 2, 300, True, 0, 1, 0), (1, 4, 2, 400, False, 50, 3, 1)])
+def test_bwd_persistent_kernel_emulated_eager_copies(emu_bwd, B, H, H_kv, N, causal, window, ctas, order):
+    """The persistent backward with copies that land as soon as they are issued: a K/V, Q or dO
+    load before the MMAs released the buffer would overwrite operands still to be read."""
+    _check_bwd_emulated(emu_bwd["persist128_eager"], [str(ctas), str(order)], B, H, H_kv, N, 128, causal, window)
 
 
 def _check_bwd_emulated(exe, extra, B, H, H_kv, N, d, causal, window):

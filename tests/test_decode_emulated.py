@@ -27,6 +27,16 @@ CSRC = os.path.join(os.path.dirname(HERE), "exact_io_aware_77_b200", "csrc")
 
 
 @pytest.fixture(scope="module")
+def emu_binary_eager(tmp_path_factory):
+    from tests.host_emu.build_emu import build
+    try:
+        return build(str(tmp_path_factory.mktemp("host_emu_eager")), "decode_kernel.cuh", "emu_main.cpp",
+                     "emu_main_eager", defines=("EMU_EAGER_COPIES",))
+    except FileNotFoundError:
+        pytest.skip("g++ not available")
+
+
+@pytest.fixture(scope="module")
 def emu_binary(tmp_path_factory):
     from tests.host_emu.build_emu import build
     try:
@@ -124,3 +134,12 @@ def test_decode_fp8kv_kernel_emulated(emu_binary, B, H, H_kv, N_q, N_k, d, causa
 def test_decode_kernel_emulated_strided(emu_binary):
     wl = Workload("decode_emu_strided", 2, 4, 500, 128, True, 0, seed=72, H_kv=2, Nq=3)
     _run(emu_binary, wl, seq_major=True)
+
+
+@pytest.mark.parametrize("B,H,H_kv,N_q,N_k,d,causal,window", [
+    (2, 8, 2, 3, 1000, 128, True, 0), (1, 2, 1, 5, 777, 64, False, 50), (1, 4, 1, 2, 700, 256, True, 0)])
+def test_decode_kernel_emulated_eager_copies(emu_binary_eager, B, H, H_kv, N_q, N_k, d, causal, window):
+    """cp.async copies that land as soon as they are issued: a lane refilling a ring stage that
+    another lane of its warp still reads would overwrite those keys."""
+    wl = Workload("decode_emu", B, H, N_k, d, causal, window, seed=71 + N_k + N_q, H_kv=H_kv, Nq=N_q)
+    _run(emu_binary_eager, wl)

@@ -41,6 +41,8 @@ def emu_fwd(tmp_path_factory):
                           ("EMU_FWD_PERSIST", "EMU_D=64")),
             "persist128": (["fwd_persist_kernel.cuh", "fwd_kernel.cuh", "persist_sched.cuh"], "emu_fwd_main.cpp", "emu_fwd_persist_128",
                            ("EMU_FWD_PERSIST", "EMU_D=128")),
+            "persist128_eager": (["fwd_persist_kernel.cuh", "fwd_kernel.cuh", "persist_sched.cuh"], "emu_fwd_main.cpp",
+                                 "emu_fwd_persist_128_eager", ("EMU_FWD_PERSIST", "EMU_D=128", "EMU_EAGER_COPIES")),
         })
     except FileNotFoundError:
         pytest.skip("g++ not available")
@@ -93,6 +95,15 @@ PERSIST_CASES = [
 def test_fwd_persistent_kernel_emulated(emu_fwd, B, H, H_kv, N, d, causal, window, ctas, order):
     """fa_fwd_persist_kernel (the persistent grid: each CTA loops over work items) vs the oracle."""
     _check_fwd_emulated(emu_fwd[f"persist{d}"], [str(ctas), str(order)], B, H, H_kv, N, d, causal, window)
+
+
+@pytest.mark.parametrize("B,H,H_kv,N,causal,window,ctas,order", [
+    (1, 2, 2, 300, True, 0, 1, 1), (2, 2, 1, 600, False, 0, 3, 0), (1, 4, 2, 520, True, 100, 2, 1)])
+def test_fwd_persistent_kernel_emulated_eager_copies(emu_fwd, B, H, H_kv, N, causal, window, ctas, order):
+    """The persistent forward with TMA copies that land as soon as they are issued (the other legal
+    extreme to landing when waited for): a load into a ring slot or the Q buffer before its
+    consumers released it would overwrite data still to be read."""
+    _check_fwd_emulated(emu_fwd["persist128_eager"], [str(ctas), str(order)], B, H, H_kv, N, 128, causal, window)
 
 
 def _check_fwd_emulated(exe, extra, B, H, H_kv, N, d, causal, window):
