@@ -447,7 +447,14 @@ inline void mma_exec(uint32_t d_tmem, uint64_t a_desc, uint32_t a_tmem_addr, uin
       cell = __float_as_uint(acc);
     }
 }
+// By default an MMA runs at its issuing thread's next commit.  Built with EMU_EAGER_MMA it runs
+// at issue instead, the other legal extreme: an MMA issued before its operands are ready (a P
+// in TMEM, a tile in shared memory) then reads them too early.
 inline void queue_mma(std::function<void()> f) {
+#ifdef EMU_EAGER_MMA
+  f();
+  return;
+#endif
   std::lock_guard<std::mutex> lk(*g_blk->mu);
   g_blk->mmas->push_back(PendingOp{0, std::move(f)});
 }

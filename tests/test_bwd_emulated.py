@@ -37,6 +37,9 @@ def emu_bwd(tmp_path_factory):
                            "emu_bwd_persist_128", ("EMU_BWD_PERSIST", "EMU_D=128")),
             "persist128_eager": (["bwd_persist_kernel.cuh", "bwd_kernel.cuh", "persist_sched.cuh"], "emu_bwd_main.cpp",
                                  "emu_bwd_persist_128_eager", ("EMU_BWD_PERSIST", "EMU_D=128", "EMU_EAGER_COPIES")),
+            "persist128_eager_mma": (["bwd_persist_kernel.cuh", "bwd_kernel.cuh", "persist_sched.cuh"],
+                                     "emu_bwd_main.cpp", "emu_bwd_persist_128_eager_mma",
+                                     ("EMU_BWD_PERSIST", "EMU_D=128", "EMU_EAGER_MMA")),
         })
     except FileNotFoundError:
         pytest.skip("g++ not available")
@@ -89,6 +92,12 @@ def test_bwd_persistent_kernel_emulated_eager_copies(emu_bwd, B, H, H_kv, N, cau
     """The persistent backward with copies that land as soon as they are issued: a K/V, Q or dO
     load before the MMAs released the buffer would overwrite operands still to be read."""
     _check_bwd_emulated(emu_bwd["persist128_eager"], [str(ctas), str(order)], B, H, H_kv, N, 128, causal, window)
+
+
+def test_bwd_persistent_kernel_emulated_eager_mma(emu_bwd):
+    """The persistent backward with MMAs that run as soon as they are issued: a dV, dK or dQ
+    product issued before P^T or dS^T is in place reads it too early."""
+    _check_bwd_emulated(emu_bwd["persist128_eager_mma"], ["2", "1"], 1, 4, 2, 400, 128, False, 50)
 
 
 def _check_bwd_emulated(exe, extra, B, H, H_kv, N, d, causal, window):

@@ -43,6 +43,11 @@ def emu_fwd(tmp_path_factory):
                            ("EMU_FWD_PERSIST", "EMU_D=128")),
             "persist128_eager": (["fwd_persist_kernel.cuh", "fwd_kernel.cuh", "persist_sched.cuh"], "emu_fwd_main.cpp",
                                  "emu_fwd_persist_128_eager", ("EMU_FWD_PERSIST", "EMU_D=128", "EMU_EAGER_COPIES")),
+            "persist128_eager_mma": (["fwd_persist_kernel.cuh", "fwd_kernel.cuh", "persist_sched.cuh"],
+                                     "emu_fwd_main.cpp", "emu_fwd_persist_128_eager_mma",
+                                     ("EMU_FWD_PERSIST", "EMU_D=128", "EMU_EAGER_MMA")),
+            "256_eager_mma": (["fwd256_kernel.cuh", "fwd_kernel.cuh"], "emu_fwd_main.cpp", "emu_fwd_256_eager_mma",
+                              ("EMU_FWD256", "EMU_EAGER_MMA")),
         })
     except FileNotFoundError:
         pytest.skip("g++ not available")
@@ -104,6 +109,18 @@ def test_fwd_persistent_kernel_emulated_eager_copies(emu_fwd, B, H, H_kv, N, cau
     extreme to landing when waited for): a load into a ring slot or the Q buffer before its
     consumers released it would overwrite data still to be read."""
     _check_fwd_emulated(emu_fwd["persist128_eager"], [str(ctas), str(order)], B, H, H_kv, N, 128, causal, window)
+
+
+@pytest.mark.parametrize("kind,B,H,H_kv,N,d,causal,window,extra", [
+    ("persist128_eager_mma", 1, 2, 2, 300, 128, True, 0, ["1", "1"]),
+    ("persist128_eager_mma", 2, 2, 1, 600, 128, False, 0, ["3", "0"]),
+    ("256_eager_mma", 1, 2, 2, 300, 256, True, 0, []),
+    ("256_eager_mma", 1, 4, 2, 400, 256, False, 50, [])])
+def test_fwd_kernel_emulated_eager_mma(emu_fwd, kind, B, H, H_kv, N, d, causal, window, extra):
+    """MMAs that run as soon as they are issued (the other legal extreme to running at the next
+    commit): a product issued before its operands are ready (P in TMEM, a K/V tile) reads them
+    too early."""
+    _check_fwd_emulated(emu_fwd[kind], extra, B, H, H_kv, N, d, causal, window)
 
 
 def _check_fwd_emulated(exe, extra, B, H, H_kv, N, d, causal, window):
