@@ -87,7 +87,7 @@ def test_bwd_persistent_kernel_emulated(emu_bwd, B, H, H_kv, N, d, causal, windo
 
 
 @pytest.mark.parametrize("B,H,H_kv,N,causal,window,ctas,order", [
-    (1, 2, 2, 300, True, 0, 1, 0), (1, 4, 2, 400, False, 50, 3, 1)])
+    (1, 2, 2, 300, True, 0, 1, 0), (1, 4, 2, 200, False, 50, 3, 1)])
 def test_bwd_persistent_kernel_emulated_eager_copies(emu_bwd, B, H, H_kv, N, causal, window, ctas, order):
     """The persistent backward with copies that land as soon as they are issued: a K/V, Q or dO
     load before the MMAs released the buffer would overwrite operands still to be read."""
@@ -97,7 +97,7 @@ def test_bwd_persistent_kernel_emulated_eager_copies(emu_bwd, B, H, H_kv, N, cau
 def test_bwd_persistent_kernel_emulated_eager_mma(emu_bwd):
     """The persistent backward with MMAs that run as soon as they are issued: a dV, dK or dQ
     product issued before P^T or dS^T is in place reads it too early."""
-    _check_bwd_emulated(emu_bwd["persist128_eager_mma"], ["2", "1"], 1, 4, 2, 400, 128, False, 50)
+    _check_bwd_emulated(emu_bwd["persist128_eager_mma"], ["2", "1"], 1, 4, 2, 200, 128, False, 50)
 
 
 def _check_bwd_emulated(exe, extra, B, H, H_kv, N, d, causal, window):
