@@ -143,3 +143,9 @@ def test_decode_kernel_emulated_eager_copies(emu_binary_eager, B, H, H_kv, N_q, 
     another lane of its warp still reads would overwrite those keys."""
     wl = Workload("decode_emu", B, H, N_k, d, causal, window, seed=71 + N_k + N_q, H_kv=H_kv, Nq=N_q)
     _run(emu_binary_eager, wl)
+
+
+def test_decode_fp8kv_kernel_emulated_eager_copies(emu_binary_eager):
+    """The FP8 K/V path (raw E4M3 ring, converted tiles) with cp.async copies landing at issue."""
+    wl = Workload("decode_fp8_emu", 2, 8, 1000, 128, True, 0, seed=81 + 1000 + 3, H_kv=2, Nq=3)
+    _run(emu_binary_eager, wl, fp8=True)

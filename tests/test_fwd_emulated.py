@@ -48,6 +48,8 @@ def emu_fwd(tmp_path_factory):
                                      ("EMU_FWD_PERSIST", "EMU_D=128", "EMU_EAGER_MMA")),
             "256_eager_mma": (["fwd256_kernel.cuh", "fwd_kernel.cuh"], "emu_fwd_main.cpp", "emu_fwd_256_eager_mma",
                               ("EMU_FWD256", "EMU_EAGER_MMA")),
+            "fp8_eager_mma": (["fwd_fp8_kernel.cuh", "fwd_kernel.cuh"], "emu_fwd_main.cpp", "emu_fwd_fp8_eager_mma",
+                              ("EMU_FWD_FP8", "EMU_EAGER_MMA")),
         })
     except FileNotFoundError:
         pytest.skip("g++ not available")
@@ -220,3 +222,9 @@ def test_fwd_fp8_kernel_emulated(emu_fwd, B, H, H_kv, N, causal, window):
     v = s_v * np.swapaxes(orc.e4m3_to_float(vt8.numpy()), -1, -2)
     bound = fp8_o_bound(q, k, v, wl.scale, causal, window, o_ref)
     assert np.all(np.abs(o - o_ref) <= bound), float((np.abs(o - o_ref) - bound).max())
+
+
+def test_fwd_fp8_kernel_emulated_eager_mma(emu_fwd):
+    """The FP8 forward with MMAs that run as soon as they are issued: a P V product issued before
+    the softmax warps staged P8 in shared memory would read it too early."""
+    test_fwd_fp8_kernel_emulated({"fp8": emu_fwd["fp8_eager_mma"]}, 1, 4, 2, 512, True, 100)
