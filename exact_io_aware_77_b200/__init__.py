@@ -79,7 +79,7 @@ def forward(q, k, v, scale: float | None = None, causal: bool = False, window: i
             out=None, lse=None, persistent: bool = False, ctas: int = 0, schedule: str = "balanced"):
     """O, L = attention(Q, K, V); O bf16 [B,H,N,d], L fp32 [B,H,N] (natural-log logsumexp).
 
-    d is 64, 128 or 256.  ``persistent`` (d 64 or 128) runs the same tiles on a persistent grid
+    d is 64, 128 or 256.  ``persistent`` runs the same tiles on a persistent grid
     of ``ctas`` CTAs (0: one per SM) that loop over the work items, taken in the ``schedule``
     "balanced" (longest first over all heads when a mask makes the costs differ) or
     "head_major" order."""

@@ -161,7 +161,7 @@ FA_SCHED_BALANCED, FA_SCHED_HEAD_MAJOR = 0, 1
 
 def fa_fwd_persistent(q, k, v, o, lse, B, H, H_kv, N, d, strides, scale, causal, window, ctas, schedule,
                       stream) -> int:
-    """fa_fwd_strided on a persistent grid of ``ctas`` CTAs (0: one per SM); d 64 or 128;
+    """fa_fwd_strided on a persistent grid of ``ctas`` CTAs (0: one per SM); d 64, 128 or 256;
     ``schedule`` FA_SCHED_BALANCED or FA_SCHED_HEAD_MAJOR."""
     return _call("fa_fwd_persistent", q, k, v, o, lse, B, H, H_kv, N, d, strides, scale, causal, window, ctas,
                  schedule, stream)

@@ -14,6 +14,7 @@
 #include "fwd_kernel.cuh"
 #include "fwd_persist_kernel.cuh"
 #include "fwd256_kernel.cuh"
+#include "fwd256_persist_kernel.cuh"
 #include "fp8_ops.cuh"
 #include "fwd_fp8_kernel.cuh"
 #include "bwd_kernel.cuh"
@@ -222,6 +223,45 @@ int launch_fwd256(const void* q, const void* k, const void* v, void* o, float* l
   const int smem = int(sizeof(Fwd256Smem)) + 1024;
   if (set_smem(fa_fwd256_kernel, smem) != FA_OK) return FA_ERR_CUDA;
   fa_fwd256_kernel<<<unsigned(prm.n_pairs) * unsigned(BH), k256Threads, smem, stream>>>(tq, tk, tv, prm);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// head dimension 256 on the persistent grid (fwd256_persist_kernel.cuh)
+int launch_fwd256_persist(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv,
+                          int N, const Strides* st, float scale, int causal, int window, int ctas, int schedule,
+                          cudaStream_t stream) {
+  CUtensorMap tq, tk, tv;
+  if (!make_map_bf16(&tq, q, kD256, N, H, B, st[0], k256BlockM) ||
+      !make_map_bf16(&tk, k, kD256, N, H_kv, B, st[1], k256BlockN) ||
+      !make_map_bf16(&tv, v, kD256, N, H_kv, B, st[2], k256BlockN))
+    return FA_ERR_CUDA;
+  FwdParams prm;
+  prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.lse = lse;
+  prm.N = N;
+  prm.BH = B * H;
+  prm.H = H;
+  prm.group = H / H_kv;
+  prm.o_st = st[3];
+  prm.n_pairs = (N + k256BlockM - 1) / k256BlockM;   // query tiles per head
+  prm.causal = causal;
+  prm.window = window > N ? N : window;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.wait_limit_ns = g_wait_limit_ns;
+  if (ctas == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&ctas, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return FA_ERR_CUDA;
+  }
+  const long long n_items = (long long)prm.n_pairs * prm.BH;
+  const unsigned grid = unsigned(ctas < n_items ? ctas : n_items);
+  const bool costs_vary = causal || (prm.window > 0 && prm.window < N);
+  const int order = schedule == FA_SCHED_BALANCED && costs_vary ? kOrderPairMajor : kOrderHeadMajor;
+  static_assert(sizeof(Fwd256PersistSmem) + 1024 <= 232448, "d = 256 persistent forward shared memory exceeds 227 KB");
+  const int smem = int(sizeof(Fwd256PersistSmem)) + 1024;
+  if (set_smem(fa_fwd256_persist_kernel, smem) != FA_OK) return FA_ERR_CUDA;
+  fa_fwd256_persist_kernel<<<grid, k256Threads, smem, stream>>>(tq, tk, tv, prm, order);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -514,7 +554,6 @@ int fa_fwd_persistent(const void* q, const void* k, const void* v, void* o, floa
   if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
   int st = check_problem(B, H, N, d, scale, causal, window);
   if (st == FA_OK) st = check_kv_heads(H, H_kv);
-  if (st == FA_OK && d == 256) st = FA_ERR_HEADDIM;
   if (st == FA_OK && (ctas < 0 || (schedule != FA_SCHED_BALANCED && schedule != FA_SCHED_HEAD_MAJOR)))
     st = FA_ERR_SHAPE;
   if (st != FA_OK) return st;
@@ -528,9 +567,11 @@ int fa_fwd_persistent(const void* q, const void* k, const void* v, void* o, floa
     return FA_ERR_ALIGN;
   if ((st = check_device()) != FA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return d == 64
-             ? launch_fwd_persist<64>(q, k, v, o, lse, B, H, H_kv, N, s4, scale, causal, window, ctas, schedule, s)
-             : launch_fwd_persist<128>(q, k, v, o, lse, B, H, H_kv, N, s4, scale, causal, window, ctas, schedule, s);
+  switch (d) {
+    case 64: return launch_fwd_persist<64>(q, k, v, o, lse, B, H, H_kv, N, s4, scale, causal, window, ctas, schedule, s);
+    case 128: return launch_fwd_persist<128>(q, k, v, o, lse, B, H, H_kv, N, s4, scale, causal, window, ctas, schedule, s);
+    default: return launch_fwd256_persist(q, k, v, o, lse, B, H, H_kv, N, s4, scale, causal, window, ctas, schedule, s);
+  }
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {

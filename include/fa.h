@@ -172,14 +172,15 @@ FA_EXPORT int fa_bwd_strided(const void* q, const void* k, const void* v, const 
  * write.  The computation is the tiled forward of the FlashAttention (EN) page ("Algorithm"):
  * the same tiles, online softmax and logsumexp as fa_fwd_strided, whose results it returns bit
  * for bit (the per-tile arithmetic and its order within a tile are the same; only which CTA
- * takes which tile differs).
+ * takes which tile differs).  At d = 256 the items are single 128-row query tiles, as in
+ * fa_fwd_strided's d = 256 kernel.
  *
  *   schedule  FA_SCHED_BALANCED: with a causal or banded mask (item costs differ) the items go
  *             longest first over all heads, dealt to the CTAs round by round in a snake
  *             (0, 1, ..., G-1, then G-1, ..., 0), which evens out the CTAs' total work; with no
  *             mask, head-major.  FA_SCHED_HEAD_MAJOR: head-major, longest first within a head,
  *             snake-dealt the same way.
- *   d         64 or 128 (FA_ERR_HEADDIM otherwise).
+ *   d         64, 128 or 256.
  *
  * ctas < 0 or another schedule gives FA_ERR_SHAPE.  Arguments, strides, errors, streams and
  * ownership are otherwise as for fa_fwd_strided.

@@ -4,7 +4,10 @@
 // [B, heads, N, d] arrays.
 // usage: emu_fwd_main B H Hkv N causal window scale prefix   (prefix.q/.k/.v bf16; writes .o, .lse)
 #include "emu.h"
-#ifdef EMU_FWD256
+#ifdef EMU_FWD256_PERSIST
+#include "fwd256_persist_kernel.cuh"
+#define EMU_D 256
+#elif defined(EMU_FWD256)
 #include "fwd256_kernel.cuh"
 #define EMU_D 256
 #elif defined(EMU_FWD_FP8)
@@ -26,7 +29,9 @@
 namespace fa {
 // the kernel's dynamic shared memory: exactly one (1024-byte aligned) FwdSmem, so AddressSanitizer
 // sees any access past it
-#ifdef EMU_FWD256
+#ifdef EMU_FWD256_PERSIST
+alignas(1024) uint8_t smem_raw[sizeof(Fwd256PersistSmem)];
+#elif defined(EMU_FWD256)
 alignas(1024) uint8_t smem_raw[sizeof(Fwd256Smem)];
 #elif defined(EMU_FWD_FP8)
 alignas(1024) uint8_t smem_raw[sizeof(FwdFp8Smem)];
@@ -124,8 +129,9 @@ int main(int argc, char** argv) {
 #else
 // usage (persistent form): ... prefix grid order   (grid: the number of persistent CTAs; order:
 // 0 head-major, 1 pair-major item order)
+// (EMU_FWD256_PERSIST, the d = 256 persistent form, is built together with EMU_FWD256)
 int main(int argc, char** argv) {
-#ifdef EMU_FWD_PERSIST
+#if defined(EMU_FWD_PERSIST) || defined(EMU_FWD256_PERSIST)
   if (argc != 11) { std::fprintf(stderr, "bad args\n"); return 2; }
 #else
   if (argc != 9) { std::fprintf(stderr, "bad args\n"); return 2; }
@@ -164,7 +170,7 @@ int main(int argc, char** argv) {
   prm.window = window > N ? N : window;
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.wait_limit_ns = 60ull * 1000000000ull;
-#ifdef EMU_FWD_PERSIST
+#if defined(EMU_FWD_PERSIST) || defined(EMU_FWD256_PERSIST)
   const unsigned n_items = unsigned(prm.n_pairs) * unsigned(B * H);
   const unsigned grid = std::min(n_items, unsigned(atoi(argv[9])));
   const int order = atoi(argv[10]);
@@ -174,6 +180,9 @@ int main(int argc, char** argv) {
   std::printf("grid %u smem %zu\n", grid, sizeof(fa::smem_raw));
 #ifdef EMU_FWD_PERSIST
   emu_launch(grid, kFwdThreads, sizeof(fa::smem_raw), [&] { fa_fwd_persist_kernel<D>(tq, tk, tv, prm, order); }, fa::smem_raw);
+#elif defined(EMU_FWD256_PERSIST)
+  emu_launch(grid, k256Threads, sizeof(fa::smem_raw), [&] { fa_fwd256_persist_kernel(tq, tk, tv, prm, order); },
+             fa::smem_raw);
 #elif defined(EMU_FWD256)
   emu_launch(grid, k256Threads, sizeof(fa::smem_raw), [&] { fa_fwd256_kernel(tq, tk, tv, prm); }, fa::smem_raw);
 #else

@@ -144,7 +144,6 @@ def test_strided_entry_points_validate_strides(lib):
     (dict(ctas=-1), "FA_ERR_SHAPE"),
     (dict(schedule=2), "FA_ERR_SHAPE"),
     (dict(schedule=-1), "FA_ERR_SHAPE"),
-    (dict(d=256), "FA_ERR_HEADDIM"),
     (dict(d=96), "FA_ERR_HEADDIM"),
     (dict(causal=2), "FA_ERR_MASK"),
     (dict(scale=float("nan")), "FA_ERR_SCALE"),
@@ -152,7 +151,7 @@ def test_strided_entry_points_validate_strides(lib):
     (dict(bad_stride=True), "FA_ERR_ALIGN"),
 ])
 def test_persistent_fwd_rejects_bad_arguments(lib, kw, code):
-    """fa_fwd_persistent: fa_fwd_strided's checks, d 64 or 128 only, ctas >= 0, a known schedule."""
+    """fa_fwd_persistent: fa_fwd_strided's checks, ctas >= 0, a known schedule."""
     a = dict(GOOD, H_kv=GOOD["H"], ctas=0, schedule=_lib.FA_SCHED_BALANCED)
     ptrs = kw.pop("ptrs", [A + 4096 * i for i in range(5)])
     bad_stride = kw.pop("bad_stride", False)

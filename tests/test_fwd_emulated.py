@@ -41,6 +41,8 @@ def emu_fwd(tmp_path_factory):
                           ("EMU_FWD_PERSIST", "EMU_D=64")),
             "persist128": (["fwd_persist_kernel.cuh", "fwd_kernel.cuh", "persist_sched.cuh"], "emu_fwd_main.cpp", "emu_fwd_persist_128",
                            ("EMU_FWD_PERSIST", "EMU_D=128")),
+            "persist256": (["fwd256_persist_kernel.cuh", "fwd256_kernel.cuh", "fwd_kernel.cuh", "persist_sched.cuh"],
+                           "emu_fwd_main.cpp", "emu_fwd_persist_256", ("EMU_FWD256", "EMU_FWD256_PERSIST")),
             "persist128_eager": (["fwd_persist_kernel.cuh", "fwd_kernel.cuh", "persist_sched.cuh"], "emu_fwd_main.cpp",
                                  "emu_fwd_persist_128_eager", ("EMU_FWD_PERSIST", "EMU_D=128", "EMU_EAGER_COPIES")),
             "persist128_eager_mma": (["fwd_persist_kernel.cuh", "fwd_kernel.cuh", "persist_sched.cuh"],
@@ -95,6 +97,11 @@ PERSIST_CASES = [
     (2, 3, 3, 700, 64, True, 0, 5, 1),
     (1, 1, 1, 1, 128, True, 0, 1, 1),        # N = 1: one row, the pair's second tile empty
     (1, 2, 1, 129, 64, False, 0, 1, 1),      # one row past a tile, one CTA for both heads
+    # head dimension 256 (fa_fwd256_persist_kernel: items are single query tiles)
+    (1, 2, 2, 300, 256, True, 0, 1, 1),
+    (1, 2, 1, 520, 256, True, 100, 3, 1),
+    (1, 4, 2, 400, 256, False, 50, 2, 1),
+    (2, 2, 1, 257, 256, True, 3, 3, 0),
 ]
 
 
@@ -146,7 +153,7 @@ def _check_fwd_emulated(exe, extra, B, H, H_kv, N, d, causal, window):
     assert np.abs(lse - l_ref).max() <= L_MAX_ABS
 
 
-@pytest.mark.parametrize("d,persistent", [(128, False), (256, False), (128, True)])
+@pytest.mark.parametrize("d,persistent", [(128, False), (256, False), (128, True), (256, True)])
 def test_fwd_kernel_emulated_late_rescales(emu_fwd, d, persistent):
     """Keys that score ever higher along the sequence make many rows' maxima grow by more than
     2^8 after their first key tile, so the lazy rescale of O runs at later tiles (with the d = 256
@@ -167,7 +174,7 @@ def test_fwd_kernel_emulated_late_rescales(emu_fwd, d, persistent):
         pre = os.path.join(tmp, "x")
         for name, t in zip("qkv", (q, k, v)):
             t.contiguous().view(torch.int16).numpy().tofile(pre + "." + name)
-        exe, extra = (emu_fwd["persist128"], ["1", "1"]) if persistent else (emu_fwd[d], [])
+        exe, extra = (emu_fwd[f"persist{d}"], ["1", "1"]) if persistent else (emu_fwd[d], [])
         r = subprocess.run([exe, "1", "1", "1", str(N), "1", "0", repr(scale), pre] + extra,
                            capture_output=True, text=True, timeout=900)
         assert r.returncode == 0, r.stderr[-4000:]

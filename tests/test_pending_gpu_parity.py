@@ -48,7 +48,9 @@ def test_d256_forward_and_backward(fa, B, H, H_kv, N, causal, window):
     (1, 2, 2, 300, 128, True, 0, 1, "balanced"), (1, 2, 2, 300, 128, True, 0, 2, "head_major"),
     (2, 2, 1, 600, 128, False, 0, 3, "balanced"), (1, 4, 2, 520, 128, True, 100, 0, "balanced"),
     (2, 2, 1, 257, 64, True, 3, 2, "head_major"), (1, 3, 3, 1000, 64, False, 0, 0, "balanced"),
-    (2, 3, 3, 700, 64, True, 0, 5, "balanced"), (1, 1, 1, 1, 128, True, 0, 0, "balanced")])
+    (2, 3, 3, 700, 64, True, 0, 5, "balanced"), (1, 1, 1, 1, 128, True, 0, 0, "balanced"),
+    (1, 2, 2, 300, 256, True, 0, 1, "balanced"), (1, 4, 2, 400, 256, False, 50, 0, "balanced"),
+    (2, 2, 1, 257, 256, True, 3, 3, "head_major")])
 def test_persistent_forward(fa, B, H, H_kv, N, d, causal, window, ctas, schedule):
     """The persistent grid against the oracle, and bit for bit against the one-item-per-CTA
     forward: every tile meets the same arithmetic in the same order."""
