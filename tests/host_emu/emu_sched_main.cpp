@@ -8,15 +8,23 @@
 // one line per case: BH N causal window order grid, the largest CTA load and the mean load, in
 // K/V tile steps plus one per item.  Then the same coverage check for the backward's items
 // (K/V head, key tile) with q_tile_range's query tiles, for 1, 2 and 4 query heads per K/V
-// head, printing "bwd" lines with the loads in query iterations plus one per item.
+// head, printing "bwd" lines with the loads in query iterations plus one per item; and for the
+// d = 256 forward's items (head, 128-row query tile) with kv_tile_range256's 64-key tiles,
+// printing "f256" lines.
 // usage: emu_sched_main   (exit 1 at the first violation)
 #include "emu.h"
 #include "fwd_persist_kernel.cuh"
 #include "bwd_persist_kernel.cuh"
+#include "fwd256_persist_kernel.cuh"
 
 #include <algorithm>
 #include <cstdio>
 #include <vector>
+
+namespace fa {
+// the shared memory the (never launched) d = 256 kernels refer to; this program only walks schedules
+alignas(1024) uint8_t smem_raw[1024];
+}  // namespace fa
 
 using namespace fa;
 
@@ -146,6 +154,54 @@ int main() {
           std::printf("bwd %d %d %d %d %d %d %u %lld %.3f\n", sh.BH, group, sh.N, sh.causal, sh.window, order, g,
                       max_load, double(total) / g);
         }
+      }
+    }
+  }
+  // the d = 256 forward: one 128-row query tile per item
+  for (const Shape& sh : shapes) {
+    FwdParams prm{};
+    prm.N = sh.N;
+    prm.BH = sh.BH;
+    prm.H = sh.BH;
+    prm.group = 1;
+    prm.causal = sh.causal;
+    prm.window = std::min(sh.window, sh.N);
+    prm.n_pairs = (sh.N + k256BlockM - 1) / k256BlockM;
+    const int n_items = prm.n_pairs * prm.BH;
+    for (int order : {int(kOrderHeadMajor), int(kOrderPairMajor)}) {
+      for (unsigned G : grids) {
+        const unsigned g = std::min<unsigned>(G, unsigned(n_items));
+        gridDim = dim3s{g, 1, 1};
+        std::vector<int> seen(n_items, 0);
+        long long max_load = 0, total = 0;
+        for (unsigned cta = 0; cta < g; ++cta) {
+          blockIdx = dim3s{cta, 0, 0};
+          long long load = 0;
+          for (int r = 0;; ++r) {
+            const int pos = persist_item(n_items, r);
+            if (pos < 0) break;
+            const Fwd256Item it = fwd256_item(prm, order, pos);
+            const int tile = it.q0 / k256BlockM;
+            int tb, te;
+            kv_tile_range256(it.q0, prm.N, prm.causal, prm.window, tb, te);
+            if (it.bh < 0 || it.bh >= prm.BH || tile < 0 || tile >= prm.n_pairs || it.q0 != tile * k256BlockM ||
+                it.t_begin != tb || it.t_end != te || te <= tb) {
+              std::printf("FAIL f256 item at position %d\n", pos);
+              return 1;
+            }
+            ++seen[it.bh * prm.n_pairs + tile];
+            load += (te - tb) + 1;
+          }
+          max_load = std::max(max_load, load);
+          total += load;
+        }
+        for (int i = 0; i < n_items; ++i)
+          if (seen[i] != 1) {
+            std::printf("FAIL f256 item %d taken %d times\n", i, seen[i]);
+            return 1;
+          }
+        std::printf("f256 %d %d %d %d %d %u %lld %.3f\n", sh.BH, sh.N, sh.causal, sh.window, order, g, max_load,
+                    double(total) / g);
       }
     }
   }

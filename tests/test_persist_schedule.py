@@ -16,20 +16,26 @@ def sched_rows(tmp_path_factory):
     d = str(tmp_path_factory.mktemp("host_emu_sched"))
     try:
         exe = build(d, ["fwd_persist_kernel.cuh", "fwd_kernel.cuh", "persist_sched.cuh", "bwd_persist_kernel.cuh",
-                        "bwd_kernel.cuh"], "emu_sched_main.cpp", "emu_sched")
+                        "bwd_kernel.cuh", "fwd256_persist_kernel.cuh", "fwd256_kernel.cuh"], "emu_sched_main.cpp",
+                    "emu_sched")
     except FileNotFoundError:
         pytest.skip("g++ not available")
     r = subprocess.run([exe], capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-2000:]
     lines = [l for l in r.stdout.split("\n") if l.strip()]
-    fwd = [l for l in lines if not l.startswith("bwd")]
+    fwd = [l for l in lines if not l.startswith(("bwd", "f256"))]
     bwd = [l for l in lines if l.startswith("bwd")]
+    f256 = [l for l in lines if l.startswith("f256")]
+    assert len(f256) == 14 * 2 * 8
     assert len(fwd) == 14 * 2 * 8   # shapes x item orders x grid sizes, one line each
     assert len(bwd) >= 14 * 2 * 8   # and per query heads per K/V head that divide the heads
     rows = {}
     for line in fwd:
         BH, N, causal, window, order, g, max_load, mean = line.split()
         rows[(int(BH), int(N), int(causal), int(window), int(order), int(g))] = (int(max_load), float(mean))
+    for line in f256:
+        _, BH, N, causal, window, order, g, max_load, mean = line.split()
+        rows[("f256", int(BH), int(N), int(causal), int(window), int(order), int(g))] = (int(max_load), float(mean))
     for line in bwd:
         _, BH, group, N, causal, window, order, g, max_load, mean = line.split()
         rows[("bwd", int(BH), int(group), int(N), int(causal), int(window), int(order), int(g))] = (int(max_load),
@@ -60,4 +66,13 @@ def test_backward_balanced_order(sched_rows, group, slack):
     head_max, mean = sched_rows[("bwd", 64, group, 4096, 1, 0, 0, 148)]
     bal_max, _ = sched_rows[("bwd", 64, group, 4096, 1, 0, 1, 148)]
     assert bal_max <= slack * mean, (bal_max, mean)
+    assert bal_max <= head_max
+
+
+def test_d256_forward_balanced_order(sched_rows):
+    """The d = 256 forward's items (one query tile each) at 148 CTAs on a causal N4096 shape with
+    64 heads: the balanced order's largest load is within 3 % of the mean."""
+    head_max, mean = sched_rows[("f256", 64, 4096, 1, 0, 0, 148)]
+    bal_max, _ = sched_rows[("f256", 64, 4096, 1, 0, 1, 148)]
+    assert bal_max <= 1.03 * mean, (bal_max, mean)
     assert bal_max <= head_max
