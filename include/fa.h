@@ -75,8 +75,7 @@ typedef enum {
  * Forward pass.  Writes O (bf16 [B,H,N,d]) and L (fp32 [B,H,N], natural-log logsumexp of
  * the masked, scaled scores of each query row).  Reads q, k, v (bf16 [B,H,N,d]).
  * d must be 64, 128 or 256.  Extra device memory: none beyond O and L.  d = 256 runs a kernel of
- * its own (one 128-row query tile per CTA, 64-key K/V tiles); it has been checked against the
- * reference in a host emulation of its primitives but not yet timed or run on a B200.
+ * its own (one 128-row query tile per CTA, 64-key K/V tiles).
  */
 FA_EXPORT int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
            float scale, int causal, int window, void* stream);
@@ -96,8 +95,7 @@ FA_EXPORT size_t fa_bwd_workspace_size(int B, int H, int N, int d);
  * is scratch: it is overwritten and may be reused once the call's work has completed on
  * `stream`.  Three kernels are enqueued: D = rowsum(dO o O) with a cleared accumulator, the
  * fused recompute kernel, and the dQ scaling.  d must be 64, 128 or 256; d = 256 runs a kernel of
- * its own (one CTA per 64-key tile and head-dim half), checked in a host emulation of its
- * primitives but not yet run on a B200.
+ * its own (one CTA per 64-key tile and head-dim half).
  */
 FA_EXPORT int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
                      void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal, int window,
@@ -278,9 +276,6 @@ FA_EXPORT int fa_fwd_decode_fp8kv(const void* q, const void* k8, const void* v8,
  *   d must be 128 (FA_ERR_HEADDIM otherwise); N a multiple of 16 (FA_ERR_SHAPE); the scales
  *   finite and > 0 (FA_ERR_SCALE).  Masks, scale, errors and streams as for fa_fwd_gqa.
  *
- * The kernel has been checked against the reference only in a host emulation of its
- * primitives, not yet on a B200; the 8-bit instruction descriptor (type code 0 for E4M3) is the
- * documented encoding, still to be confirmed on the hardware.
  */
 FA_EXPORT int fa_fwd_fp8(const void* q8, const void* k8, const void* vt8, float q_scale, float k_scale, float v_scale,
                          void* o, float* lse, int B, int H, int H_kv, int N, int d, float scale, int causal, int window,

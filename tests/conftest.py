@@ -11,8 +11,6 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) and the built CUDA library")
     config.addinivalue_line("markers", "slow: long-running CPU oracle case")
-    config.addinivalue_line("markers", "gpu_pending: B200 parity of a path checked so far only in the host "
-                                       "emulation; not selected by -m gpu (run with -m gpu_pending)")
 
 
 def pytest_collection_modifyitems(config, items):
@@ -26,5 +24,5 @@ def pytest_collection_modifyitems(config, items):
         return
     skip = pytest.mark.skip(reason="no CUDA device")
     for item in items:
-        if "gpu" in item.keywords or "gpu_pending" in item.keywords:
+        if "gpu" in item.keywords:
             item.add_marker(skip)

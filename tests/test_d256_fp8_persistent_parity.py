@@ -1,10 +1,7 @@
-"""B200 parity of the paths checked so far only in the host emulation.
-
-Marked gpu_pending, not gpu: the B200 runs of the verified suite (-m gpu) do not select these
-until a first GPU run has confirmed them (python -m pytest tests -m gpu_pending).  They cover the
-head-dimension-256 forward and backward, the FP8 (E4M3) forward, the decode kernels over an
-E4M3 K/V cache and at d = 256, and the persistent form of the d = 64 / 128 forward, with the tolerances of the other parity tests (the FP8 forward's
-derived per-element bound from tests/parity.py).
+"""B200 parity of the head-dimension-256 forward and backward, the FP8 (E4M3) forward, the decode
+kernels over an E4M3 K/V cache and at d = 256, and the persistent forward and backward, with the
+tolerances of the other parity tests (the FP8 forward's derived per-element bound from
+tests/parity.py).  The persistent kernels are also held bit for bit to the one-item-per-CTA ones.
 """
 
 import numpy as np
@@ -15,7 +12,7 @@ from oracle import attention as orc
 from synthetic import Workload, make_grad_output, make_inputs, make_inputs_fp8, make_inputs_fp8kv
 from tests.parity import assert_forward_close, assert_grads_close, fp8_o_bound, L_MAX_ABS, to64
 
-pytestmark = pytest.mark.gpu_pending
+pytestmark = pytest.mark.gpu
 
 
 @pytest.fixture(scope="module")
