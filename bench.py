@@ -42,7 +42,10 @@ GRAD_WORKLOAD = "bwd"
 # --workload choices: the forward workload and the one whose dO seed the backward uses
 BENCH_WORKLOADS = {"causal": ("causal", "bwd"), "long": ("long", "long"), "swa": ("swa", "swa"),
                    "gqa": ("gqa", "gqa"), "decode": ("decode", "decode"), "decode_fp8": ("decode", "decode"),
-                   "d256": ("d256", "d256"), "fp8": ("causal", "bwd")}
+                   "d256": ("d256", "d256"), "fp8": ("causal", "bwd"), "tiny": ("tiny", "tiny"),
+                   "gpt2": ("gpt2", "gpt2")}
+# workloads timed as a forward alone (the configurations that name only O and the logsumexp)
+FORWARD_ONLY = ("tiny", "gpt2")
 FLUSH_BYTES = 256 << 20      # > 126 MB L2
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -74,7 +77,9 @@ def parse_args():
                          "cached keys (B8, 64 query heads on 8 K/V heads), forward only, HBM-bound; "
                          "decode_fp8: the same over an E4M3 K/V cache with per-tensor scales; "
                          "d256: B2 H16 N4096 head dimension 256, causal, forward+backward; "
-                         "fp8: the causal shape's forward on E4M3 Q, K, V (V transposed)")
+                         "fp8: the causal shape's forward on E4M3 Q, K, V (V transposed); "
+                         "tiny: B1 H2 N128 d64 forward (launch/HBM-bound: reported against the HBM "
+                         "peak); gpt2: B4 H16 N2048 d64 non-causal forward")
     return ap.parse_args()
 
 
@@ -261,9 +266,10 @@ def oracle_sample(seconds: float, rows_per_block: int = 512, with_bwd: bool = Tr
     from synthetic import WORKLOADS, make_grad_output, make_inputs
     wl = WORKLOADS[WORKLOAD]
     sub = wl.with_(B=1, H=1, H_kv=None)
-    q, k, v = (x[0, 0] for x in make_inputs(sub))
-    do = make_grad_output(WORKLOADS[GRAD_WORKLOAD].with_(B=1, H=1, H_kv=None))[0, 0]
-    q, k, v, do = (x.double().numpy() for x in (q, k, v, do))
+    q, k, v = (x[0, 0].double().numpy() for x in make_inputs(sub))
+    do = None
+    if with_bwd:
+        do = make_grad_output(WORKLOADS[GRAD_WORKLOAD].with_(B=1, H=1, H_kv=None))[0, 0].double().numpy()
     per_row = fwd_flops(1, 1, wl.N, wl.d, wl.causal, wl.window) / wl.N
     if with_bwd:
         per_row += bwd_flops(1, 1, wl.N, wl.d, wl.causal, wl.window) / wl.N
@@ -945,6 +951,162 @@ def run_fp8(args):
         print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------- forward-only arm
+def fwd_hbm_bytes(wl) -> int:
+    """Algorithmic bytes of one forward: read Q, K, V once, write O (bf16) and L (fp32)."""
+    q_el = wl.B * wl.H * wl.q_rows * wl.d
+    kv_el = wl.B * wl.kv_heads * wl.N * wl.d
+    return 2 * (2 * q_el + 2 * kv_el) + 4 * wl.B * wl.H * wl.q_rows
+
+
+def run_forward_only(args):
+    """The forward alone (O and the logsumexp) on the tiny or the GPT-2-like workload.
+
+    tiny (B1 H2 N128 d64) is one CTA's work: launch latency and HBM bound, so its roofline is
+    the algorithmic bytes over the kernel time against the measured HBM copy bandwidth.  gpt2
+    (B4 H16 N2048 d64) is a dense contraction: TFLOP/s against the measured bf16 peak."""
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=300))
+    import exact_io_aware_77_b200 as fa
+    fa.load()
+    from synthetic import WORKLOADS, make_inputs
+    wl = WORKLOADS[WORKLOAD]
+    B, H, N, d = wl.B, wl.H, wl.N, wl.d
+    persistent = bool(args.persistent_fwd)
+    q_h, k_h, v_h = make_inputs(wl)
+    q, k, v = (x.to(dev) for x in (q_h, k_h, v_h))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flops = fwd_flops(B, H, N, d, wl.causal, wl.window)
+    nbytes = fwd_hbm_bytes(wl)
+    kname = kernel_names(d, persistent)[0]
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        fa.forward(q, k, v, wl.scale, wl.causal, wl.window, out=o, lse=lse, persistent=persistent,
+                   schedule=args.fwd_schedule)
+        if ev:
+            ev[1].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    st = fa.check_status(dev)
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {fa.STATUS_NAMES.get(st, st)}")
+    sampler = ClockSampler(gpu_id_for(local))
+    sampler.start()
+    time.sleep(0.3)
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    wall0 = time.time()
+    for i in range(args.steps):
+        flush.zero_()
+        step(events[i])
+    torch.cuda.synchronize(dev)
+    wall1 = time.time()
+    if world > 1:
+        dist.barrier()
+    sampler.mark(wall0, wall1)
+    time.sleep(0.25)
+    sampler.stop()
+    st = fa.check_status(dev)
+    if st != 0:
+        raise RuntimeError(f"device status after timing: {fa.STATUS_NAMES.get(st, st)}")
+    per_step = [e[0].elapsed_time(e[1]) for e in events]
+    total = max_over_ranks([sum(per_step)], dev)[0]
+    ms = total / args.steps
+    value = job_throughput(world, flops, ms)
+
+    e2e = None
+    if not args.no_e2e:
+        # through the public API with host buffers: pinned Q, K, V in, O and L out, every step
+        pin = [x.pin_memory() for x in (q_h, k_h, v_h)]
+        o_h = torch.empty_like(pin[0]).pin_memory()
+        l_h = torch.empty((B, H, N), dtype=torch.float32).pin_memory()
+        qd, kd, vd = (torch.empty_like(x, device=dev) for x in pin)
+
+        def one():
+            for dst, src in zip((qd, kd, vd), pin):
+                dst.copy_(src, non_blocking=True)
+            fa.forward(qd, kd, vd, wl.scale, wl.causal, wl.window, out=o, lse=lse, persistent=persistent,
+                       schedule=args.fwd_schedule)
+            o_h.copy_(o, non_blocking=True)
+            l_h.copy_(lse, non_blocking=True)
+
+        for _ in range(3):
+            one()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(1, args.e2e_steps)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            one()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_e2e = max_over_ranks([e0.elapsed_time(e1) / n_e2e], dev)[0]
+        e2e = {"value": round(job_throughput(world, flops, ms_e2e), 4), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in pin),
+               "d2h_bytes_per_step": o_h.numel() * 2 + l_h.numel() * 4, "ms_per_step": round(ms_e2e, 4),
+               "mode": "serial: copy in, forward, copy out on one stream"}
+
+    peaks, peak_kind = load_peaks()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    tflops = flops / (ms * 1e-3) / 1e12
+    if WORKLOAD == "tiny":
+        roofline = {"bound": "hbm", "kernel": kname, "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+                    "peak_source": f"{peak_kind} HBM copy (MEASURED_PEAKS.json)", "traffic": None,
+                    "bytes_per_launch": nbytes}
+    else:
+        roofline = {"bound": "tensor", "kernel": kname, "achieved": round(tflops, 1),
+                    "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                    "frac": round(tflops / peaks["bf16_tflops"], 4),
+                    "peak_source": f"{peak_kind} burst bf16 (MEASURED_PEAKS.json)", "traffic": None}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        f, secs, blocks, cores = oracle_sample(args.cpu_seconds, rows_per_block=min(512, N), with_bwd=False)
+        cpu = {"value": round(f / secs / 1e12, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+               "sample": f"{blocks} blocks of {min(512, N)} query rows of head 0 of the {wl.name} workload "
+                         f"(B{B} H{H} N{N} d{d}) through the fp64 oracle (fwd), {secs:.1f} s, credited "
+                         f"rows/N of a head's FLOPs"}
+    line = {
+        "metric": "attention fwd/bwd TFLOP/s at 1 B200; % of dense BF16 tensor peak",
+        "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": workload_text(wl, False), "global_batch": B * world, "seq_len": N,
+                   "parallelism": f"replicas{world}",
+                   "l2": "flushed (256 MB write) between timed steps, outside the events",
+                   "fwd_grid": f"persistent, one CTA per SM, {args.fwd_schedule} item order" if persistent
+                   else "one CTA per work item"},
+        "fwd_us": round(ms * 1e3, 2), "fwd_gbs": round(gbs, 1),
+        "pct_of_measured_peak": round(100 * tflops / peaks["bf16_tflops"], 2),
+        "pct_of_spec_peak_2250": round(100 * tflops / 2250.0, 2),
+        "pct_of_measured_hbm": round(100 * gbs / peaks["hbm_gbs"], 2),
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps,
+        "kernel_ms": {kname: round(ms, 5)}, "clocks": sampler.summary(),
+    }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 # ----------------------------------------------------------------------------- reference arm
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
@@ -957,16 +1119,16 @@ def run_reference(args):
     if args.workload == "fp8":
         return run_fp8_reference(args, wl)
     import exact_io_aware_77_b200 as fa_pkg   # only to learn whether the path has a backward
-    with_bwd = hasattr(fa_pkg, "backward")
+    with_bwd = hasattr(fa_pkg, "backward") and args.workload not in FORWARD_ONLY
     times, flops = [], []
     for i in range(args.warmup + args.steps):
-        f, s, _, cores = oracle_sample(0.0, rows_per_block=128, with_bwd=with_bwd, max_blocks=1)
+        f, s, _, cores = oracle_sample(0.0, rows_per_block=min(128, wl.N), with_bwd=with_bwd, max_blocks=1)
         if i >= args.warmup:
             times.append(s)
             flops.append(f)
     secs = sum(times)
     value = sum(flops) / secs / 1e12
-    sample = (f"each step: 128 query rows of head 0 of the {wl.name} workload (B{wl.B} H{wl.H} N{wl.N} "
+    sample = (f"each step: {min(128, wl.N)} query rows of head 0 of the {wl.name} workload (B{wl.B} H{wl.H} N{wl.N} "
               f"d{wl.d}) through the fp64 oracle ({'fwd+bwd' if with_bwd else 'fwd'}), credited rows/N "
               f"of a head's FLOPs")
     line = {
@@ -1040,7 +1202,8 @@ def workload_text(wl, with_bwd: bool) -> str:
                 f"{band_pairs(wl.N, wl.causal, wl.window)} kept pairs per head")
         kind = "long-context"
     else:
-        band, kind = ("causal" if wl.causal else "no mask"), "causal LLM shape"
+        kinds = {"tiny": "tiny", "gpt2": "GPT-2-like", "d256": "head dimension 256"}
+        band, kind = ("causal" if wl.causal else "no mask"), kinds.get(wl.name, "causal LLM shape")
     heads = f"H={wl.H}" + (f" (K/V heads {wl.kv_heads})" if wl.kv_heads != wl.H else "")
     return (f"{kind} {'forward+backward' if with_bwd else 'forward'}: B={wl.B} {heads} N={wl.N} "
             f"d={wl.d} {band}, inputs N(0,1)*{wl.std:g} bf16 seeded")
@@ -1056,6 +1219,8 @@ def main():
         run_decode(args, fp8=args.workload == "decode_fp8")
     elif args.workload == "fp8":
         run_fp8(args)
+    elif args.workload in FORWARD_ONLY:
+        run_forward_only(args)
     else:
         run_ours(args)
 

@@ -60,7 +60,8 @@ __device__ __forceinline__ void q_tile_range256(int kv0, int N, int causal, int 
   }
 }
 
-// One CTA per (K/V head, 64-key tile, head-dim half): blockIdx.x = (bh_kv * n_kv_tiles + tile) * 2 + c.
+// One CTA per (K/V head, 64-key tile, head-dim half): blockIdx.x = item * 2 + c, with the
+// (K/V head, tile) items in grid_item's chunked order.
 // prm.n_kv_tiles counts 64-key tiles here.
 __global__ void __launch_bounds__(kB256Threads, 1)
     fa_bwd256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -76,8 +77,8 @@ __global__ void __launch_bounds__(kB256Threads, 1)
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int dhalf = int(blockIdx.x & 1);   // head-dim half: columns 128 dhalf ..
-  const int tile = int((blockIdx.x >> 1) % prm.n_kv_tiles);
-  const int bh = int((blockIdx.x >> 1) / prm.n_kv_tiles);   // K/V head, b * H_kv + h_kv
+  int bh, tile;   // K/V head (b * H_kv + h_kv) and key tile
+  grid_item(int(blockIdx.x >> 1), prm.BH / prm.group, prm.n_kv_tiles, kBwdChunkHeads, bh, tile);
   const int b_idx = bh / prm.H_kv, h_kv = bh % prm.H_kv;
   const int bh_q0 = b_idx * prm.H + h_kv * prm.group;       // first query head of the group
   const int kv0 = tile * kB256Keys;

@@ -41,6 +41,7 @@
 
 #include <type_traits>
 
+#include "persist_sched.cuh"
 #include "sm100.cuh"
 
 namespace fa {
@@ -186,8 +187,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int lane = threadIdx.x & 31;
   // this CTA's K/V head; with shared K/V heads it runs the query tiles of every query head of
   // its group in turn (dK and dV accumulate over all of them)
-  const int bh = int(blockIdx.x / prm.n_kv_tiles);
-  const int kv_tile = int(blockIdx.x % prm.n_kv_tiles);
+  // chunks of K/V heads, key tile 0 (the longest under a causal mask) of every head first
+  int bh, kv_tile;
+  grid_item(int(blockIdx.x), prm.BH / prm.group, prm.n_kv_tiles, kBwdChunkHeads, bh, kv_tile);
   const int kv0 = kv_tile * kBwdKeys;
   int i_begin, i_end;
   q_tile_range(kv0, prm.N, prm.causal, prm.window, i_begin, i_end);

@@ -73,9 +73,10 @@ __global__ void __launch_bounds__(k256Threads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int n_tiles = prm.n_pairs;
-  const int bh = int(blockIdx.x / n_tiles);
+  int bh, rank;
+  grid_item(int(blockIdx.x), prm.BH, n_tiles, kFwdChunkHeads, bh, rank);
   const int b_idx = bh / prm.H, h_q = bh % prm.H, h_kv = h_q / prm.group;
-  const int q0 = (n_tiles - 1 - int(blockIdx.x % n_tiles)) * k256BlockM;   // longest causal tiles first
+  const int q0 = (n_tiles - 1 - rank) * k256BlockM;   // longest causal tiles of the chunk first
   int t_begin, t_end;
   kv_tile_range256(q0, prm.N, prm.causal, prm.window, t_begin, t_end);
   volatile int* abort = &sm.abort;

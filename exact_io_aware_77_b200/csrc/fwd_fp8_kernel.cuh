@@ -54,9 +54,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int bh = int(blockIdx.x / prm.n_pairs);
+  int bh, rank;
+  grid_item(int(blockIdx.x), prm.BH, prm.n_pairs, kFwdChunkHeads, bh, rank);
   const int b_idx = bh / prm.H, h_q = bh % prm.H, h_kv = h_q / prm.group;
-  const int pair = prm.n_pairs - 1 - int(blockIdx.x % prm.n_pairs);
+  const int pair = prm.n_pairs - 1 - rank;
   const int q0 = pair * (kQTiles * kBlockM);
   int b0, e0, b1, e1;
   kv_tile_range(q0, prm.N, prm.causal, prm.window, b0, e0);

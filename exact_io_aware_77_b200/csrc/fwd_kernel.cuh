@@ -32,6 +32,7 @@
 
 #include <type_traits>
 
+#include "persist_sched.cuh"
 #include "sm100.cuh"
 
 namespace fa {
@@ -104,11 +105,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // head-major order keeps a head's K/V hot in L2; longest causal pairs first within a head
-  const int bh = int(blockIdx.x / prm.n_pairs);
+  // chunks of heads (their K/V stay in L2), the longest causal pairs of a chunk first
+  int bh, rank;
+  grid_item(int(blockIdx.x), prm.BH, prm.n_pairs, kFwdChunkHeads, bh, rank);
   // batch entry, query head, and the K/V head it reads (heads share K/V in contiguous groups)
   const int b_idx = bh / prm.H, h_q = bh % prm.H, h_kv = h_q / prm.group;
-  const int pair = prm.n_pairs - 1 - int(blockIdx.x % prm.n_pairs);
+  const int pair = prm.n_pairs - 1 - rank;
   const int q0 = pair * (kQTiles * kBlockM);
   int b0, e0, b1, e1;
   kv_tile_range(q0, prm.N, prm.causal, prm.window, b0, e0);

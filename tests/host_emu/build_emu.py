@@ -49,6 +49,14 @@ PATCHES = {
 def build(out_dir: str, kernel_header, harness: str, exe_name: str, defines=()) -> str:
     """kernel_header: one header name, or a list (a kernel header and the headers it includes)."""
     headers = [kernel_header] if isinstance(kernel_header, str) else list(kernel_header)
+    # and every library header they include (sm100.cuh and the stubbed headers are the stub's)
+    i = 0
+    while i < len(headers):
+        with open(os.path.join(CSRC, headers[i])) as f:
+            for inc in re.findall(r'^#include "([^"/]+)"', f.read(), re.M):
+                if inc not in headers and inc != "sm100.cuh" and inc not in STUBBED_HEADERS:
+                    headers.append(inc)
+        i += 1
     gxx = shutil.which("g++")
     if gxx is None:
         raise FileNotFoundError("g++")

@@ -48,6 +48,10 @@ def emu_fwd(tmp_path_factory):
             "persist128_eager_mma": (["fwd_persist_kernel.cuh", "fwd_kernel.cuh", "persist_sched.cuh"],
                                      "emu_fwd_main.cpp", "emu_fwd_persist_128_eager_mma",
                                      ("EMU_FWD_PERSIST", "EMU_D=128", "EMU_EAGER_MMA")),
+            "128_eager": ("fwd_kernel.cuh", "emu_fwd_main.cpp", "emu_fwd_128_eager", ("EMU_D=128", "EMU_EAGER_COPIES")),
+            "128_eager_mma": ("fwd_kernel.cuh", "emu_fwd_main.cpp", "emu_fwd_128_eager_mma",
+                              ("EMU_D=128", "EMU_EAGER_MMA")),
+            "64_eager_mma": ("fwd_kernel.cuh", "emu_fwd_main.cpp", "emu_fwd_64_eager_mma", ("EMU_D=64", "EMU_EAGER_MMA")),
             "256_eager_mma": (["fwd256_kernel.cuh", "fwd_kernel.cuh"], "emu_fwd_main.cpp", "emu_fwd_256_eager_mma",
                               ("EMU_FWD256", "EMU_EAGER_MMA")),
             "fp8_eager_mma": (["fwd_fp8_kernel.cuh", "fwd_kernel.cuh"], "emu_fwd_main.cpp", "emu_fwd_fp8_eager_mma",
@@ -120,7 +124,19 @@ def test_fwd_persistent_kernel_emulated_eager_copies(emu_fwd, B, H, H_kv, N, cau
     _check_fwd_emulated(emu_fwd["persist128_eager"], [str(ctas), str(order)], B, H, H_kv, N, 128, causal, window)
 
 
+@pytest.mark.parametrize("B,H,H_kv,N,causal,window", [
+    (1, 2, 2, 300, True, 0), (2, 2, 1, 600, False, 0), (1, 4, 2, 520, True, 100), (1, 2, 2, 1000, False, 200)])
+def test_fwd_kernel_emulated_eager_copies(emu_fwd, B, H, H_kv, N, causal, window):
+    """fa_fwd_kernel with TMA copies that land as soon as they are issued: a load into a K/V ring
+    slot before the products reading its previous tile have completed would overwrite it."""
+    _check_fwd_emulated(emu_fwd["128_eager"], [], B, H, H_kv, N, 128, causal, window)
+
+
 @pytest.mark.parametrize("kind,B,H,H_kv,N,d,causal,window,extra", [
+    ("128_eager_mma", 1, 2, 2, 300, 128, True, 0, []),
+    ("128_eager_mma", 2, 2, 1, 600, 128, False, 0, []),
+    ("128_eager_mma", 1, 4, 2, 520, 128, True, 100, []),
+    ("64_eager_mma", 1, 2, 2, 1000, 64, False, 200, []),
     ("persist128_eager_mma", 1, 2, 2, 300, 128, True, 0, ["1", "1"]),
     ("persist128_eager_mma", 2, 2, 1, 600, 128, False, 0, ["3", "0"]),
     ("256_eager_mma", 1, 2, 2, 300, 256, True, 0, []),
