@@ -176,6 +176,36 @@ def load_peaks():
         return FALLBACK_PEAKS, "fallback"
 
 
+# A timed region at least this long runs at the clock the 1 kW power cap settles to; a shorter
+# one mostly at the boost clock.  The measured peaks come in both regimes.
+SUSTAINED_MS = 1000.0
+
+
+def regime_fields(roofline: dict, clocks: dict, timed_ms: float, kernel_ms: float, peaks: dict, scale: float = 1.0):
+    """Add to a tensor-bound roofline the regime of the timed region and the fraction of the other
+    regime's peak, and return the clock-normalised figures: the dominant kernel's time scaled to
+    the maximum SM clock (time x median MHz / max MHz) and its throughput at that time.  `scale`
+    converts the bf16 peaks to the kernel's own type (the FP8 arm)."""
+    regime = "sustained" if timed_ms >= SUSTAINED_MS else "burst"
+    burst, sustained = peaks["bf16_tflops"] * scale, peaks["bf16_tflops_sustained"] * scale
+    roofline["regime"] = regime
+    if regime == "sustained":
+        roofline["peak"] = round(sustained, 1)
+        roofline["frac"] = round(roofline["achieved"] / sustained, 4)
+        roofline["peak_source"] = roofline["peak_source"].replace("burst", "sustained")
+    roofline["timed_region_ms"] = round(timed_ms, 1)
+    roofline["frac_of_burst_peak"] = round(roofline["achieved"] / burst, 4)
+    roofline["frac_of_sustained_peak"] = round(roofline["achieved"] / sustained, 4)
+    mhz, mhz_max = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    if not mhz or not mhz_max:
+        return None
+    t_norm = kernel_ms * mhz / mhz_max
+    return {"sm_mhz_median": mhz, "sm_max_mhz": mhz_max, "samples_in_window": clocks.get("samples"),
+            "kernel": roofline["kernel"], "kernel_ms_at_max_clock": round(t_norm, 5),
+            "achieved_at_max_clock": round(roofline["achieved"] * kernel_ms / t_norm, 1),
+            "frac_at_max_clock": round(roofline["achieved"] * kernel_ms / t_norm / burst, 4)}
+
+
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
     """nvidia-smi samples (every 100 ms) of SM clock and throttle reasons."""
@@ -413,11 +443,14 @@ def run_ours(args):
     else:
         dom, dom_flops, dom_ms = names[0], f_fwd, fwd_ms_avg
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    # a long timed region runs under the power cap: its kernel is judged against the sustained peak
+    sustained = step_ms_total >= SUSTAINED_MS
+    peak = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
     roofline = {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 1),
-                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": round(achieved / peaks["bf16_tflops"], 4),
-                "peak_source": f"{peak_kind} burst bf16 (MEASURED_PEAKS.json)" if peak_kind == "measured"
-                else "fallback 1.59 PFLOP/s",
+                "peak": peak, "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4),
+                "peak_source": (f"{peak_kind} {'sustained' if sustained else 'burst'} bf16 (MEASURED_PEAKS.json)"
+                                if peak_kind == "measured" else "fallback (1.59 PFLOP/s burst, 1.4 sustained)"),
                 # the ncu counters were taken on the default causal workload only
                 "traffic": load_traffic(dom) if WORKLOAD == "causal" else None}
 
@@ -431,6 +464,7 @@ def run_ours(args):
                          f"head's FLOPs"}
 
     clocks = sampler.summary()
+    clock_norm = regime_fields(roofline, clocks, step_ms_total, dom_ms, peaks)
     line = {
         "metric": "attention fwd/bwd TFLOP/s at 1 B200; % of dense BF16 tensor peak",
         "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -455,6 +489,7 @@ def run_ours(args):
                       "fa_bwd_prep+" + names[1] + "+fa_bwd_dq_final": round(bwd_ms_avg, 4),
                       names[1]: round(main_ms_avg, 4)} if has_bwd else None,
         "clocks": clocks,
+        "clock_normalised": clock_norm,
     }
     if has_bwd:
         line["bwd_tflops"] = round(job_throughput(world, f_bwd, bwd_ms_avg), 2)
@@ -592,12 +627,14 @@ def measure_e2e(fa, torch, wl, dev, stream, q_h, k_h, v_h, do_h, has_bwd, steps,
 # the workload the bench line times (the causal B2 H32 N4096 d128 one, or the decode one), keyed by kernel, with the SHA-1 of the kernel's sources
 # when the counters were taken (profiles/ holds the summaries).  A changed source reports null.
 NCU_TRAFFIC = {
-    "fa_fwd_kernel<128>": {"bytes": 251356416,
-                           "sources": {"fwd_kernel.cuh": "35b94dbef8d8bf21170a8812fab6ac84911c902b",
-                                       "sm100.cuh": "765aea2ea7410d534e289cfea85ff6d2b3b159c9"}},
-    "fa_bwd_kernel<128>": {"bytes": 628199424,
-                           "sources": {"bwd_kernel.cuh": "a16249a9909c16bc8d6b854ecf39824e9ae17b7a",
-                                       "sm100.cuh": "765aea2ea7410d534e289cfea85ff6d2b3b159c9"}},
+    "fa_fwd_kernel<128>": {"bytes": 247744512,
+                           "sources": {"fwd_kernel.cuh": "e8641ce82d6dbdb61b9ba009f4929267d8e3e6ee",
+                                       "sm100.cuh": "2ad8f7efc3001a800d5f5280be5d66b6f64da97e",
+                                       "persist_sched.cuh": "64126a5757824c1f991611e9caf4a9229a7cb45c"}},
+    "fa_bwd_kernel<128>": {"bytes": 625011456,
+                           "sources": {"bwd_kernel.cuh": "74efb053dd65812bcd3bb44ae6532ddb950801ad",
+                                       "sm100.cuh": "2ad8f7efc3001a800d5f5280be5d66b6f64da97e",
+                                       "persist_sched.cuh": "64126a5757824c1f991611e9caf4a9229a7cb45c"}},
     # the decode workload (B8 H64 with 8 K/V heads, N_q 1, N_k 32768): both kernels of one step
     "fa_decode_kernel<128,false>+fa_decode_merge_kernel<128>": {
         "bytes": 1083981824,
@@ -927,6 +964,8 @@ def run_fp8(args):
                 "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(value / world / peak, 4),
                 "peak_source": f"{peak_kind} burst bf16 (MEASURED_PEAKS.json) x {FP8_OVER_BF16:g}, the nominal "
                                f"E4M3/bf16 ratio", "traffic": None}
+    clocks = sampler.summary()
+    clock_norm = regime_fields(roofline, clocks, total, ms, peaks, FP8_OVER_BF16)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         f, secs, heads, cores = fp8_oracle_sample(args.cpu_seconds)
@@ -942,7 +981,7 @@ def run_fp8(args):
                    "global_batch": B * world, "seq_len": N, "parallelism": f"replicas{world}",
                    "l2": "flushed (256 MB write) between timed steps, outside the events"},
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps,
-        "clocks": sampler.summary(),
+        "clocks": clocks, "clock_normalised": clock_norm,
     }
     if world > 1:
         dist.barrier()
@@ -1076,6 +1115,8 @@ def run_forward_only(args):
                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                     "frac": round(tflops / peaks["bf16_tflops"], 4),
                     "peak_source": f"{peak_kind} burst bf16 (MEASURED_PEAKS.json)", "traffic": None}
+    clocks = sampler.summary()
+    clock_norm = regime_fields(roofline, clocks, total, ms, peaks) if roofline["bound"] == "tensor" else None
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         f, secs, blocks, cores = oracle_sample(args.cpu_seconds, rows_per_block=min(512, N), with_bwd=False)
@@ -1098,7 +1139,7 @@ def run_forward_only(args):
         "pct_of_spec_peak_2250": round(100 * tflops / 2250.0, 2),
         "pct_of_measured_hbm": round(100 * gbs / peaks["hbm_gbs"], 2),
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps,
-        "kernel_ms": {kname: round(ms, 5)}, "clocks": sampler.summary(),
+        "kernel_ms": {kname: round(ms, 5)}, "clocks": clocks, "clock_normalised": clock_norm,
     }
     if world > 1:
         dist.barrier()

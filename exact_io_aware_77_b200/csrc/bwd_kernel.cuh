@@ -14,7 +14,7 @@
 //   fa_bwd_kernel    one CTA per 128-key tile of one head; loops over 128-row query tiles.
 //   fa_bwd_dq_final  dQ = scale * accumulator, rounded to bf16.
 //
-// fa_bwd_kernel roles (384 threads), every MMA 128 x 128 (narrower ones cost as much time):
+// fa_bwd_kernel roles (320 threads), every MMA 128 x 128 (narrower ones cost as much time):
 //   warp 8      TMA producer: K, V once; Q_i (+ its L and D rows) into a 2-stage ring, dO_i into
 //               one stage.
 //   warp 9      MMA issuer, per query tile i in the order
@@ -27,11 +27,11 @@
 //               w / 4 of each tile.  Phase A: P^T = exp2(S^T c - L) with the causal/window mask,
 //               stored to TMEM as bf16.  Phase B: dS^T = P^T o (dP^T - D) to TMEM (A of dK) and
 //               to shared memory (A of dQ).  Readout: its half of the dQ_i rows of its 32
-//               queries, from TMEM into its shared-memory staging slot, 32 columns at a time.
+//               queries, from TMEM into its shared-memory staging slot, 32 columns at a time,
+//               each block added into the fp32 accumulator by one TMA tensor reduction
+//               (cp.reduce.async.bulk.tensor .add), so that the adds leave the SM as whole
+//               128-byte lines and no warp waits for them.
 //               Order per tile: B(i), A(i+1), readout(i).  At the end: dK (half 0), dV (half 1).
-//   warps 10-11 reduction: read the staged dQ blocks back (so that each vector reduction
-//               covers whole 128-byte row segments) and add them into the fp32 accumulator
-//               with red.global.add.v4.f32, so that no compute warp waits on the reductions.
 // TMEM columns: dK [0,128), dV [128,256), S^T [256,384) with P^T in [256,288) and [320,352)
 // once read, dP^T [384,512) with dS^T in [384,416) and [448,480) once read, and dQ in
 // [384,512).  MMAs of one thread
@@ -49,7 +49,8 @@ namespace fa {
 constexpr int kBwdKeys = 128;    // keys per CTA
 constexpr int kBwdRows = 128;    // queries per iteration
 constexpr int kBwdQStages = 2;
-constexpr int kBwdThreads = 384;   // 8 compute warps, TMA, MMA, 2 reduction warps
+constexpr int kBwdThreads = 384;       // fa_bwd_persist_kernel: 8 compute warps, TMA, MMA, 2 reduction warps
+constexpr int kBwdMainThreads = 320;   // fa_bwd_kernel: 8 compute warps, TMA, MMA
 constexpr int kBwdWarpTma = 8;
 constexpr int kBwdWarpMma = 9;
 constexpr uint32_t kTdK = 0, kTdV = 128, kTS = 256, kTP = 256, kTdP = 384, kTdS = 384, kTdQ = 384;
@@ -79,12 +80,12 @@ struct BwdSmem {
   alignas(1024) uint8_t dout[kTileBytes];                  // one stage: see the producer
   alignas(1024) uint8_t ds[kBwdKeys * kBwdRows * 2];       // dS^T: [key][query], 64-query chunks
   alignas(1024) uint8_t stage[8][32 * 32 * 4];             // dQ staging: 32 rows x 32 fp32 per compute warp
+                                                           // (1 KB aligned: the 128-byte swizzle's atoms)
   alignas(16) float lp[kBwdQStages][kBwdRows];
   alignas(16) float dd[kBwdQStages][kBwdRows];
   alignas(8) uint64_t kv_full;
   uint64_t q_full[kBwdQStages], q_empty[kBwdQStages], do_full, do_empty;
   uint64_t s_full, dp_full, pa_full, ds_full, dq_full, dq_free, mma_final, mma_drain;
-  uint64_t st_full[8], st_free[8];   // dQ staging of each compute warp: filled / read back
   uint32_t tmem_base;
   int abort;
 };
@@ -169,11 +170,13 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_final(const float* __restrict__
 }
 
 // ----------------------------------------------------------------------------- main kernel
+// tm_dq: the fp32 accumulator [BH, Np, D] as the 4-D tensor (D, Np, BH, 1), 32 x 32 boxes with
+// the 128-byte swizzle (the layout of a compute warp's staging slot).
 template <int D>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kBwdMainThreads, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                  const BwdParams prm) {
+                  const __grid_constant__ CUtensorMap tm_dq, const BwdParams prm) {
   using Smem = BwdSmem<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // the layout fills almost all 227 KB, so no slack is left for realigning the base
@@ -220,10 +223,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(smem_u32(&sm.mma_drain), 1);
     mbar_init(smem_u32(&sm.do_full), 1);
     mbar_init(smem_u32(&sm.do_empty), 1);
-    for (int w = 0; w < 8; ++w) {
-      mbar_init(smem_u32(&sm.st_full[w]), 32);
-      mbar_init(smem_u32(&sm.st_free[w]), 32);
-    }
     fence_mbar_init();
   }
   if (warp == kBwdWarpTma && lane == 0) {
@@ -231,6 +230,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
     tma_prefetch_desc(&tm_do);
+    tma_prefetch_desc(&tm_dq);
   }
   if (warp == kBwdWarpMma) {
     tmem_alloc(smem_u32(&sm.tmem_base), 512);
@@ -473,10 +473,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       return true;
     };
     // dQ readout: my 32 query rows, head-dim columns D/2 hq ...  In passes of 32 columns the
-    // block goes from TMEM into my 4 KB staging slot; a reduction warp reads it back and issues
-    // the vector reductions, so this warp never waits on them.
+    // block goes from TMEM into my 4 KB staging slot, and lane 0 adds it into the accumulator
+    // with one TMA tensor reduction.  Before the slot is written again, lane 0 waits until the
+    // previous reduction has read it (it has had a whole pass, or a tile, to do so).
     const uint32_t stage = smem_u32(sm.stage[warp]);
-    int n_pass = 0;   // blocks staged so far: their parity is the slot barriers' phase
     auto readout = [&](int it) -> bool {
       if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.dq_full), it & 1, abort, lim))) return false;
       tc_fence_after();
@@ -487,17 +487,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       reg_fence<D / 2>(v);
       tc_fence_before();
       mbar_arrive(smem_u32(&sm.dq_free));
+      const int q_row = q_tile(it) * kBwdRows + quad * 32;   // my first query row of the tile
+      const int q_hd = q_head(it);
 #pragma unroll
-      for (int ps = 0; ps < D / 64; ++ps, ++n_pass) {
-        // the reduction warp has read the previous block out of the slot
-        if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.st_free[warp]), (n_pass & 1) ^ 1, abort, lim)))
-          return false;
-        // row `lane`, 16-byte chunk c at lane * 128 + (c ^ (lane & 7)) * 16
+      for (int ps = 0; ps < D / 64; ++ps) {
+        if (lane == 0) bulk_wait_group_read<0>();
+        __syncwarp();
+        // row `lane`, 16-byte chunk c at lane * 128 + (c ^ (lane & 7)) * 16: the 128-byte swizzle
 #pragma unroll
         for (int c16 = 0; c16 < 8; ++c16)
           st_shared_v4(stage + lane * 128 + ((c16 ^ (lane & 7)) << 4), v[32 * ps + 4 * c16],
                        v[32 * ps + 4 * c16 + 1], v[32 * ps + 4 * c16 + 2], v[32 * ps + 4 * c16 + 3]);
-        mbar_arrive(smem_u32(&sm.st_full[warp]));
+        fence_proxy_async_smem();   // the tensor reduction reads the slot through the async proxy
+        __syncwarp();
+        if (lane == 0) {
+          tma_reduce_add_rows(&tm_dq, stage, hq * (D / 2) + 32 * ps, q_row, q_hd, 0);
+          bulk_commit_group();
+        }
       }
       return true;
     };
@@ -541,43 +547,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       }
     }
-  }
-
-  if (warp >= 10) {
-    // ------------------------------------------------------------------ reduction warps
-    // Warp 10 serves compute warps 0-3, warp 11 warps 4-7, block by block in the order they
-    // stage them: read the block back so that each red.global.add.v4.f32 covers four whole
-    // 128-byte row segments of the fp32 accumulator, free the slot, then issue the reductions.
-    const int first = (warp - 10) * 4;
-    const int hq = first / 4;   // query half (= head-dim column half) of the warps served
-    for (int it = 0; it < n_it; ++it) {
-      for (int ps = 0; ps < D / 64; ++ps) {
-        const int n = it * (D / 64) + ps;
-        bool ok = true;
-        for (int qd = 0; qd < 4 && ok; ++qd) {
-          const int w = first + qd;
-          ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.st_full[w]), n & 1, abort, lim));
-          if (!ok) break;
-          const uint32_t slot = smem_u32(sm.stage[w]);
-          uint4 x[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int row = 4 * j + (lane >> 3), c = lane & 7;   // 8 lanes cover one 128-byte row
-            x[j] = ld_shared_v4(slot + row * 128 + ((c ^ (row & 7)) << 4));
-          }
-          mbar_arrive(smem_u32(&sm.st_free[w]));
-          const int q0 = q_tile(it) * kBwdRows + qd * 32;
-          float* acc = prm.dq_acc + (size_t(q_head(it)) * prm.Np + q0) * D + hq * (D / 2) + 32 * ps;
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int row = 4 * j + (lane >> 3), c = lane & 7;
-            red_add_v4(acc + size_t(row) * D + 4 * c, x[j]);
-          }
-        }
-        if (!ok) break;
-      }
-      if (*abort) break;
-    }
+    // every reduction this warp issued has finished (its slot read, its adds done) before the
+    // CTA's shared memory is released
+    if (lane == 0) bulk_wait_group<0>();
+    __syncwarp();
   }
 
   tc_fence_before();

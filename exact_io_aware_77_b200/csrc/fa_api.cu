@@ -77,6 +77,20 @@ bool make_map_u8(CUtensorMap* map, const void* base, int x, int rows, int heads,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The backward's fp32 dQ accumulator [BH, Np, d] as the 4-D tensor (d, Np, BH, 1) that its
+// tensor reductions add into: 32 x 32 boxes (128-byte rows), 128-byte swizzled.
+bool make_map_dq_acc(CUtensorMap* map, float* base, int d, long long Np, long long BH) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {cuuint64_t(d), cuuint64_t(Np), cuuint64_t(BH), 1};
+  cuuint64_t strides[3] = {cuuint64_t(d) * 4, cuuint64_t(Np) * d * 4, cuuint64_t(BH) * Np * d * 4};
+  cuuint32_t box[4] = {32, 32, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 // strides of a contiguous [B, heads, N, d] array
 Strides packed(int heads, int N, int d) {
   return Strides{(long long)heads * N * d, (long long)N * d, (long long)d};
@@ -377,9 +391,12 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   } else {
     static_assert(sizeof(BwdSmem<D>) <= 232448, "backward shared memory exceeds 227 KB");
     const int smem = int(sizeof(BwdSmem<D>));   // the kernel checks that the base is 1 KB aligned
+    CUtensorMap tdq;
+    if (!make_map_dq_acc(&tdq, dq_acc, D, Np, BH)) return FA_ERR_CUDA;
     if (set_smem(fa_bwd_kernel<D>, smem) != FA_OK) return FA_ERR_CUDA;
     // one CTA per (K/V head, key tile)
-    fa_bwd_kernel<D><<<unsigned(prm.n_kv_tiles) * unsigned(BH_kv), kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, prm);
+    fa_bwd_kernel<D><<<unsigned(prm.n_kv_tiles) * unsigned(BH_kv), kBwdMainThreads, smem, stream>>>(tq, tk, tv, tdo,
+                                                                                                   tdq, prm);
   }
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }

@@ -281,45 +281,70 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // the vote keeps every lane of the warp on the same path into the .sync.aligned TMEM ops
         if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.s_full[w]), k & 1, abort, lim))) return false;
         tc_fence_after();
-        float sv[kBlockN];
-        {
+        // Two passes over the S columns in TMEM: the row max from all 128, then the
+        // exponentials 32 columns at a time, each chunk reloaded (the next one's load in flight
+        // while this one is exponentiated).  Holding all 128 scores through the exponentials
+        // would leave too few of the 168 registers for the exponentials' temporaries.
+        // Allowed keys of this row form one range [lo, hi]; as columns of the tile, [a, b); the
+        // masked form applies it in both passes.
+        int a = 0, b = kBlockN;
+        if constexpr (decltype(masked)::value) {
+          const int hi = prm.causal ? min(qi, prm.N - 1)
+                                    : (prm.window > 0 ? min(qi + prm.window - 1, prm.N - 1) : prm.N - 1);
+          const int lo = prm.window > 0 ? qi - prm.window + 1 : 0;
+          a = lo - kv0;
+          b = hi - kv0 + 1;
+        }
+        // allowed columns 32 wd + j of the tile, as bits j
+        auto allowed_bits = [&](int wd) -> uint32_t {
+          const int aw = min(max(a - 32 * wd, 0), 32), bw = min(max(b - 32 * wd, 0), 32);
+          const uint32_t below_b = bw >= 32 ? 0xffffffffu : ((1u << bw) - 1u);
+          const uint32_t below_a = aw >= 32 ? 0xffffffffu : ((1u << aw) - 1u);
+          return below_b & ~below_a;
+        };
+        float mx;
+        if constexpr (!decltype(masked)::value) {
           uint32_t r[kBlockN];
 #pragma unroll
           for (int ch = 0; ch < kBlockN / 32; ++ch) tmem_ld32_async(s_col + ch * 32, r + ch * 32);
           tmem_ld_wait();
           reg_fence<kBlockN>(r);
+          // row max in 16 independent chains (one chain would be 127 dependent steps)
+          float mx16[16];
 #pragma unroll
-          for (int j = 0; j < kBlockN; ++j) sv[j] = __uint_as_float(r[j]);
-        }
-        if constexpr (decltype(masked)::value) {
-          // allowed keys of this row form one range [lo, hi]; as columns of the tile, [a, b)
-          const int hi = prm.causal ? min(qi, prm.N - 1)
-                                    : (prm.window > 0 ? min(qi + prm.window - 1, prm.N - 1) : prm.N - 1);
-          const int lo = prm.window > 0 ? qi - prm.window + 1 : 0;
-          const int a = lo - kv0, b = hi - kv0 + 1;
+          for (int i = 0; i < 16; ++i) mx16[i] = __uint_as_float(r[i]);
 #pragma unroll
-          for (int wd = 0; wd < kBlockN / 32; ++wd) {
-            const int aw = min(max(a - 32 * wd, 0), 32), bw = min(max(b - 32 * wd, 0), 32);
-            const uint32_t below_b = bw >= 32 ? 0xffffffffu : ((1u << bw) - 1u);
-            const uint32_t below_a = aw >= 32 ? 0xffffffffu : ((1u << aw) - 1u);
-            const uint32_t bits = below_b & ~below_a;   // allowed columns 32wd + j
+          for (int j = 16; j < kBlockN; j += 16)
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (!((bits >> j) & 1u)) sv[32 * wd + j] = -INFINITY;
+            for (int i = 0; i < 16; ++i) mx16[i] = fmaxf(mx16[i], __uint_as_float(r[j + i]));
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mx16[i] = fmaxf(mx16[i], mx16[i + 8]);
+          mx = max3f(max3f(mx16[0], mx16[1], mx16[2]), max3f(mx16[3], mx16[4], mx16[5]), fmaxf(mx16[6], mx16[7]));
+        } else {
+          // the masked form (diagonal and band-edge tiles) takes the max 64 columns at a time:
+          // its masking temporaries would not fit next to all 128 scores
+          float mx16[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) mx16[i] = -INFINITY;
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            uint32_t r[64];
+            tmem_ld32_async(s_col + half * 64, r);
+            tmem_ld32_async(s_col + half * 64 + 32, r + 32);
+            tmem_ld_wait();
+            reg_fence<64>(r);
+#pragma unroll
+            for (int wd = 0; wd < 2; ++wd) {
+              const uint32_t bits = allowed_bits(2 * half + wd);
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                mx16[j & 15] = fmaxf(mx16[j & 15], ((bits >> j) & 1u) ? __uint_as_float(r[32 * wd + j]) : -INFINITY);
+            }
           }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mx16[i] = fmaxf(mx16[i], mx16[i + 8]);
+          mx = max3f(max3f(mx16[0], mx16[1], mx16[2]), max3f(mx16[3], mx16[4], mx16[5]), fmaxf(mx16[6], mx16[7]));
         }
-        // row max in 16 independent chains (one chain would be 127 dependent steps)
-        float mx16[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) mx16[i] = sv[i];
-#pragma unroll
-        for (int j = 16; j < kBlockN; j += 16)
-#pragma unroll
-          for (int i = 0; i < 16; ++i) mx16[i] = fmaxf(mx16[i], sv[j + i]);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) mx16[i] = fmaxf(mx16[i], mx16[i + 8]);
-        const float mx = max3f(max3f(mx16[0], mx16[1], mx16[2]), max3f(mx16[3], mx16[4], mx16[5]),
-                               fmaxf(mx16[6], mx16[7]));
         const float m_cand = fmaxf(m, mx * c);
         const bool grow = m_cand > m + kRescaleThreshold;   // false while the row has no key
         const float m_new = grow ? m_cand : m;
@@ -329,13 +354,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // polynomial, the rest through MUFU ex2, so that neither unit limits the tile
         const uint64_t c2 = f2(c, c), nm2 = f2(-m_use, -m_use);
         uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+        // one chunk's exponentials: S columns 32 ch .. of `cur`, P into packed columns 16 ch ..
+        // (S columns already read), the sum into acc
+        auto exp_chunk = [&](int ch, const uint32_t* cur) {
+          float sv[32];
 #pragma unroll
-        for (int ch = 0; ch < kBlockN / 32; ++ch) {
+          for (int j = 0; j < 32; ++j) sv[j] = __uint_as_float(cur[j]);
+          if constexpr (decltype(masked)::value) {
+            const int aw = a - 32 * ch, bw = b - 32 * ch;   // allowed columns j of the chunk: [aw, bw)
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < aw || j >= bw) sv[j] = -INFINITY;
+          }
           uint32_t pk[16];
 #pragma unroll
           for (int jp = 0; jp < 16; ++jp) {
-            const int j = ch * 32 + 2 * jp;
-            const uint64_t x = f2_fma(f2(sv[j], sv[j + 1]), c2, nm2);
+            const uint64_t x = f2_fma(f2(sv[2 * jp], sv[2 * jp + 1]), c2, nm2);
             float p0, p1;
             if (jp < kEmuPairs) {
               exp2_poly_x2(x, p0, p1);
@@ -348,14 +382,31 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             acc[jp & 3] = f2_add(acc[jp & 3], f2(p0, p1));
             pk[jp] = pack_bf16x2(p0, p1);
           }
-          // P overwrites the S columns already read: keys 32ch.. -> packed columns 16ch..
           tmem_st16(s_col + ch * 16, pk);
+        };
+        {
+          // chunk ch + 1 loads while chunk ch is exponentiated
+          uint32_t ra[32], rb[32];
+          tmem_ld32_async(s_col, ra);
+          tmem_ld_wait();
+          reg_fence<32>(ra);
+#pragma unroll
+          for (int ch = 0; ch < kBlockN / 32; ++ch) {
+            uint32_t* cur = (ch & 1) ? rb : ra;
+            uint32_t* nxt = (ch & 1) ? ra : rb;
+            if (ch + 1 < kBlockN / 32) tmem_ld32_async(s_col + (ch + 1) * 32, nxt);
+            exp_chunk(ch, cur);
+            if (ch + 1 < kBlockN / 32) {
+              tmem_ld_wait();
+              reg_fence<32>(nxt);
+            }
+          }
         }
         float sum;
         {
-          const uint64_t a = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+          const uint64_t tot = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
           float lo, hi;
-          f2_split(a, lo, hi);
+          f2_split(tot, lo, hi);
           sum = lo + hi;
         }
         l = l * alpha + sum;

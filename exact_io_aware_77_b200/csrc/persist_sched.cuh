@@ -5,10 +5,12 @@
 namespace fa {
 
 // Heads per chunk of the one-item-per-CTA grids (grid_item): the forward's chunks are query
-// heads, the backward's K/V heads.  Large enough that the costliest items of a chunk fill the
-// 148 SMs' first wave; small enough that the chunk's K/V (forward) or Q, dO and dQ accumulator
-// (backward) stay well inside the 126 MB L2.
-constexpr int kFwdChunkHeads = 16;
+// heads, the backward's K/V heads.  Large enough that the costliest items of a chunk fill most
+// of the 148 SMs' first wave; small enough that the chunk's K/V (forward) or Q, dO and dQ
+// accumulator (backward) stay well inside the 126 MB L2.  Measured on a B200 (causal N4096 and
+// the N32768 causal band): 8 forward heads beat 16 and 32 by 1-1.5 %; 8 and 16 K/V heads tie
+// in the backward.
+constexpr int kFwdChunkHeads = 8;
 constexpr int kBwdChunkHeads = 8;
 
 // Item (head, pos) of CTA `blk` in a grid of n_heads * n_pos CTAs, where pos 0 is a head's

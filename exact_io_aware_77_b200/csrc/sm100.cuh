@@ -107,6 +107,30 @@ __device__ __forceinline__ void tma_load_rows(uint32_t dst, const CUtensorMap* m
       : "memory");
 }
 
+// 4-D tiled reduction: add the shared-memory box at `src` (laid out as a load of the same map
+// would leave it, 128-byte swizzle included) element-wise into global memory at the box's
+// coordinates; the element type and the add come from the map.  Tracked by this thread's bulk
+// async-groups: commit it with bulk_commit_group(); bulk_wait_group_read<N>() returns once at
+// most N of the thread's groups still read shared memory, bulk_wait_group<N>() once at most N
+// are unfinished.
+__device__ __forceinline__ void tma_reduce_add_rows(const CUtensorMap* map, uint32_t src, int x, int row, int head,
+                                                    int batch) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(src), "r"(x), "r"(row), "r"(head), "r"(batch)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void bulk_wait_group_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+template <int N>
+__device__ __forceinline__ void bulk_wait_group() {
+  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // ---------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)

@@ -134,6 +134,9 @@ inline float __shfl_sync(unsigned, float v, int src) {
   return r;
 }
 
+// checks the stub makes on every emulated thread as it ends (bulk operations it left in flight)
+inline void emu_thread_exit();
+
 // Runs the grid one CTA after another.  `external_smem` (for kernels that declare their own
 // extern shared array) is refilled with 0xFF before every CTA; otherwise each CTA gets a fresh
 // buffer of exactly smem_bytes.
@@ -165,6 +168,7 @@ void emu_launch(unsigned grid, unsigned block, size_t smem_bytes, F call, unsign
         blockIdx.x = bx;
         g_blk = &ctx;
         call();
+        emu_thread_exit();
       });
     for (auto& t : th) t.join();
   }

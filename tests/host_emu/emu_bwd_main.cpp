@@ -102,6 +102,19 @@ int main(int argc, char** argv) {
 #endif
   const CUtensorMap tq = make_map(q.data(), D, N, H, B, kBwdRows), tk = make_map(k.data(), D, N, Hkv, B, box_keys),
                     tv = make_map(v.data(), D, N, Hkv, B, box_keys), tdo = make_map(dout.data(), D, N, H, B, kBwdRows);
+  // the fp32 dQ accumulator [BH, Np, D] as (D, Np, BH, 1), 32 x 32 boxes
+  CUtensorMap tdq;
+  tdq.base = reinterpret_cast<const unsigned char*>(dq_acc);
+  tdq.dims[0] = uint64_t(D);
+  tdq.dims[1] = uint64_t(Np);
+  tdq.dims[2] = uint64_t(BH);
+  tdq.dims[3] = 1;
+  tdq.strides[0] = uint64_t(D) * 4;
+  tdq.strides[1] = uint64_t(Np) * D * 4;
+  tdq.strides[2] = uint64_t(BH) * Np * D * 4;
+  tdq.box_x = 32;
+  tdq.box_rows = 32;
+  tdq.esize = 4;
   BwdParams prm;
   prm.lp = lp;
   prm.dd = dd;
@@ -134,8 +147,8 @@ int main(int argc, char** argv) {
                fa::smem_raw);
   }
 #else
-  emu_launch(unsigned(prm.n_kv_tiles) * unsigned(BH_kv), kBwdThreads, sizeof(fa::smem_raw),
-             [&] { fa_bwd_kernel<D>(tq, tk, tv, tdo, prm); }, fa::smem_raw);
+  emu_launch(unsigned(prm.n_kv_tiles) * unsigned(BH_kv), kBwdMainThreads, sizeof(fa::smem_raw),
+             [&] { fa_bwd_kernel<D>(tq, tk, tv, tdo, tdq, prm); }, fa::smem_raw);
 #endif
   if (g_status != 0) { std::fprintf(stderr, "device status %d\n", g_status); return 3; }
   const long long rows = (long long)BH * N;

@@ -27,6 +27,8 @@
 // infinity); E4M3 codes decode by the format's definition (they are all f16 values).
 #pragma once
 #include <atomic>
+#include <deque>
+#include <functional>
 #include "emu.h"
 
 namespace fa {
@@ -357,6 +359,61 @@ inline void tma_copy_now(uint32_t dst, CUtensorMap mm, uint32_t bar, int x, int 
   bar_complete_tx(bar, map->box_x * map->box_rows * map->esize);
 }
 
+// cp.reduce.async.bulk.tensor .add (fp32): the reduction joins this thread's open bulk group;
+// a group's reductions run (read the shared-memory box, add atomically into the tensor) only
+// when a bulk wait retires the group -- late, so that a box rewritten before its wait shows up
+// as wrong sums.  Reductions still in flight when the thread ends abort the run.
+inline thread_local std::vector<std::function<void()>> t_bulk_open;
+inline thread_local std::deque<std::vector<std::function<void()>>> t_bulk_groups;
+inline void tma_reduce_add_rows(const CUtensorMap* map, uint32_t src, int x, int row, int head, int batch) {
+  if (map->esize != 4) { std::fprintf(stderr, "TMA reduce: only fp32 tensors are emulated\n"); std::abort(); }
+  if ((x * int(map->esize)) % 16) { std::fprintf(stderr, "TMA x coordinate not 16-byte aligned\n"); std::abort(); }
+  if (map->box_x * map->esize != 128) { std::fprintf(stderr, "TMA box row is not 128 bytes\n"); std::abort(); }
+  if (src % 128) { std::fprintf(stderr, "TMA reduce source not 128-byte aligned\n"); std::abort(); }
+  smem_at(src, size_t(map->box_rows) * 128);
+  const CUtensorMap m = *map;
+  BlockCtx* blk = g_blk;
+  t_bulk_open.push_back([=] {
+    BlockCtx* saved = g_blk;
+    g_blk = blk;
+    for (uint32_t r = 0; r < m.box_rows; ++r)
+      for (uint32_t c = 0; c < m.box_x; ++c) {
+        const long long gx = (long long)x + c, gr = (long long)row + r;
+        if (gx < 0 || gr < 0 || head < 0 || batch < 0 || uint64_t(gx) >= m.dims[0] || uint64_t(gr) >= m.dims[1] ||
+            uint64_t(head) >= m.dims[2] || uint64_t(batch) >= m.dims[3])
+          continue;   // outside the tensor: skipped
+        float val;
+        std::memcpy(&val, smem_at(sw128(src + r * 128 + c * 4), 4), 4);
+        float* dst = reinterpret_cast<float*>(const_cast<unsigned char*>(m.base) + uint64_t(batch) * m.strides[2] +
+                                              uint64_t(head) * m.strides[1] + uint64_t(gr) * m.strides[0] +
+                                              uint64_t(gx) * 4);
+        std::atomic_ref<float>(*dst).fetch_add(val);
+      }
+    g_blk = saved;
+  });
+}
+inline void bulk_commit_group() {
+  t_bulk_groups.push_back(std::move(t_bulk_open));
+  t_bulk_open.clear();
+}
+template <int N>
+inline void bulk_wait_group_read() {
+  while (t_bulk_groups.size() > size_t(N)) {
+    for (auto& f : t_bulk_groups.front()) f();
+    t_bulk_groups.pop_front();
+  }
+}
+template <int N>
+inline void bulk_wait_group() {
+  bulk_wait_group_read<N>();
+}
+inline void bulk_exit_check() {
+  if (!t_bulk_open.empty() || !t_bulk_groups.empty()) {
+    std::fprintf(stderr, "thread %u of CTA %u ends with bulk reductions in flight\n", threadIdx.x, blockIdx.x);
+    std::abort();
+  }
+}
+
 // ------------------------------------------------------------ tensor memory
 inline uint32_t& tmem_cell(uint32_t lane, uint32_t col) {
   if (lane >= 128 || col >= 512) { std::fprintf(stderr, "TMEM access out of range (%u, %u)\n", lane, col); std::abort(); }
@@ -595,3 +652,6 @@ inline float max3f(float a, float b, float c) { return std::fmax(std::fmax(a, b)
 #include "sm100_extracted.inc"
 
 }  // namespace fa
+
+// emu.h's end-of-thread hook
+inline void emu_thread_exit() { fa::bulk_exit_check(); }
