@@ -61,15 +61,6 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--persistent-fwd", action="store_true",
-                    help="run the forward on the persistent grid (one CTA per SM looping over the work "
-                         "items) instead of one CTA per item")
-    ap.add_argument("--fwd-schedule", choices=["balanced", "head_major"], default="balanced",
-                    help="item order of the persistent forward")
-    ap.add_argument("--persistent-bwd", action="store_true",
-                    help="d 64 / 128 workloads: run the backward's recompute kernel on the persistent grid")
-    ap.add_argument("--bwd-schedule", choices=["balanced", "head_major"], default="balanced",
-                    help="item order of the persistent backward")
     ap.add_argument("--workload", choices=sorted(BENCH_WORKLOADS), default="causal",
                     help="causal: B2 H32 N4096 d128 (the default line); gqa: the same with 8 K/V heads; "
                          "long / swa: N32768 with a one- / two-sided window of 4096, FLOPs counted over "
@@ -140,12 +131,11 @@ def decode_bytes(B, H, H_kv, n_q, n_k, d, causal, window=0, kv_elem_bytes=2) -> 
     return 2 * B * H * n_q * d * 2 + 2 * B * H_kv * keys * d * kv_elem_bytes + B * H * n_q * 4
 
 
-def kernel_names(d: int, persistent: bool = False, persistent_bwd: bool = False):
+def kernel_names(d: int):
     """(forward kernel, backward main kernel) names for head dimension d."""
     if d == 256:
-        return f"fa_fwd256_{'persist_' if persistent else ''}kernel", "fa_bwd256_kernel"
-    return (f"fa_fwd_{'persist_' if persistent else ''}kernel<{d}>",
-            f"fa_bwd_{'persist_' if persistent_bwd else ''}kernel<{d}>")
+        return "fa_fwd256_kernel", "fa_bwd256_kernel"
+    return f"fa_fwd_kernel<{d}>", f"fa_bwd_kernel<{d}>"
 
 
 def max_over_ranks(values, device=None):
@@ -349,12 +339,7 @@ def run_ours(args):
 
     wl = WORKLOADS[WORKLOAD]
     B, H, N, d = wl.B, wl.H, wl.N, wl.d
-    persistent = bool(args.persistent_fwd)
-    persistent_bwd = bool(args.persistent_bwd)
-    if persistent_bwd and d == 256:
-        raise SystemExit("--persistent-bwd: the persistent backward covers d 64 and 128")
-    names = kernel_names(d, persistent, persistent_bwd)
-    bwd_opts = {"persistent": persistent_bwd, "schedule": args.bwd_schedule}
+    names = kernel_names(d)
     has_bwd = hasattr(fa, "backward")
     q_h, k_h, v_h = make_inputs(wl)
     do_h = make_grad_output(WORKLOADS[GRAD_WORKLOAD])
@@ -376,14 +361,13 @@ def run_ours(args):
         # kernel, the dominant one, has events of its own
         if ev:
             ev[0].record(stream)
-        fa.forward(q, k, v, wl.scale, wl.causal, wl.window, out=o, lse=lse, persistent=persistent,
-                   schedule=args.fwd_schedule)
+        fa.forward(q, k, v, wl.scale, wl.causal, wl.window, out=o, lse=lse)
         if ev:
             ev[1].record(stream)
         if has_bwd:
             for i, ph in enumerate((1, 2, 4)):
                 fa.backward(q, k, v, o, lse, do, wl.scale, wl.causal, wl.window, grads=grads, workspace=ws,
-                            phases=ph, **bwd_opts)
+                            phases=ph)
                 if ev:
                     ev[2 + i].record(stream)
 
@@ -431,7 +415,7 @@ def run_ours(args):
     e2e = None
     if not args.no_e2e:
         e2e = measure_e2e(fa, torch, wl, dev, stream, q_h, k_h, v_h, do_h, has_bwd, args.e2e_steps,
-                          f_fwd + f_bwd, world, persistent, args.fwd_schedule, bwd_opts)
+                          f_fwd + f_bwd, world)
 
     peaks, peak_kind = load_peaks()
     fwd_ms_avg = fwd_total / args.steps
@@ -473,10 +457,7 @@ def run_ours(args):
         "config": {"workload": workload_text(wl, has_bwd),
                    "global_batch": B * world, "seq_len": N, "parallelism": f"replicas{world}",
                    "l2": "flushed (256 MB write) between timed steps, outside the events",
-                   "fwd_grid": f"persistent, one CTA per SM, {args.fwd_schedule} item order" if persistent
-                   else "one CTA per work item",
-                   "bwd_grid": f"persistent, one CTA per SM, {args.bwd_schedule} item order" if persistent_bwd
-                   else "one CTA per work item"},
+                   "grids": "one CTA per work item, heads in chunks, the costliest items of a chunk first"},
         "fwd_tflops": round(job_throughput(world, f_fwd, fwd_ms_avg), 2),
         "fwd_ms": round(fwd_ms_avg, 4),
         "pct_of_measured_peak": round(100 * value / world / peaks["bf16_tflops"], 2),
@@ -501,8 +482,7 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
 
 
-def measure_e2e(fa, torch, wl, dev, stream, q_h, k_h, v_h, do_h, has_bwd, steps, flops, world,
-                persistent=False, schedule="balanced", bwd_opts=None):
+def measure_e2e(fa, torch, wl, dev, stream, q_h, k_h, v_h, do_h, has_bwd, steps, flops, world):
     """The step through the public API with its host copies inside the timed region: every step
     copies its inputs from pinned host memory to the device and its results (O, L and, with the
     backward, dQ, dK, dV) back to pinned host memory.
@@ -536,11 +516,10 @@ def measure_e2e(fa, torch, wl, dev, stream, q_h, k_h, v_h, do_h, has_bwd, steps,
 
     def compute(ins, outs):
         q, k, v = ins[:3]
-        fa.forward(q, k, v, wl.scale, wl.causal, wl.window, out=outs[0], lse=outs[1], persistent=persistent,
-                   schedule=schedule)
+        fa.forward(q, k, v, wl.scale, wl.causal, wl.window, out=outs[0], lse=outs[1])
         if has_bwd:
             fa.backward(q, k, v, outs[0], outs[1], ins[3], wl.scale, wl.causal, wl.window,
-                        grads=tuple(outs[2:5]), workspace=ws, **(bwd_opts or {}))
+                        grads=tuple(outs[2:5]), workspace=ws)
 
     def copy_out(outs):
         for h, t in zip((o_h, l_h) + grads_h, outs):
@@ -630,11 +609,11 @@ NCU_TRAFFIC = {
     "fa_fwd_kernel<128>": {"bytes": 247744512,
                            "sources": {"fwd_kernel.cuh": "e8641ce82d6dbdb61b9ba009f4929267d8e3e6ee",
                                        "sm100.cuh": "2ad8f7efc3001a800d5f5280be5d66b6f64da97e",
-                                       "persist_sched.cuh": "64126a5757824c1f991611e9caf4a9229a7cb45c"}},
+                                       "grid_sched.cuh": "64126a5757824c1f991611e9caf4a9229a7cb45c"}},
     "fa_bwd_kernel<128>": {"bytes": 625011456,
                            "sources": {"bwd_kernel.cuh": "74efb053dd65812bcd3bb44ae6532ddb950801ad",
                                        "sm100.cuh": "2ad8f7efc3001a800d5f5280be5d66b6f64da97e",
-                                       "persist_sched.cuh": "64126a5757824c1f991611e9caf4a9229a7cb45c"}},
+                                       "grid_sched.cuh": "64126a5757824c1f991611e9caf4a9229a7cb45c"}},
     # the decode workload (B8 H64 with 8 K/V heads, N_q 1, N_k 32768): both kernels of one step
     "fa_decode_kernel<128,false>+fa_decode_merge_kernel<128>": {
         "bytes": 1083981824,
@@ -1019,7 +998,6 @@ def run_forward_only(args):
     from synthetic import WORKLOADS, make_inputs
     wl = WORKLOADS[WORKLOAD]
     B, H, N, d = wl.B, wl.H, wl.N, wl.d
-    persistent = bool(args.persistent_fwd)
     q_h, k_h, v_h = make_inputs(wl)
     q, k, v = (x.to(dev) for x in (q_h, k_h, v_h))
     o = torch.empty_like(q)
@@ -1028,13 +1006,12 @@ def run_forward_only(args):
     stream = torch.cuda.current_stream(dev)
     flops = fwd_flops(B, H, N, d, wl.causal, wl.window)
     nbytes = fwd_hbm_bytes(wl)
-    kname = kernel_names(d, persistent)[0]
+    kname = kernel_names(d)[0]
 
     def step(ev=None):
         if ev:
             ev[0].record(stream)
-        fa.forward(q, k, v, wl.scale, wl.causal, wl.window, out=o, lse=lse, persistent=persistent,
-                   schedule=args.fwd_schedule)
+        fa.forward(q, k, v, wl.scale, wl.causal, wl.window, out=o, lse=lse)
         if ev:
             ev[1].record(stream)
 
@@ -1081,8 +1058,7 @@ def run_forward_only(args):
         def one():
             for dst, src in zip((qd, kd, vd), pin):
                 dst.copy_(src, non_blocking=True)
-            fa.forward(qd, kd, vd, wl.scale, wl.causal, wl.window, out=o, lse=lse, persistent=persistent,
-                       schedule=args.fwd_schedule)
+            fa.forward(qd, kd, vd, wl.scale, wl.causal, wl.window, out=o, lse=lse)
             o_h.copy_(o, non_blocking=True)
             l_h.copy_(lse, non_blocking=True)
 
@@ -1131,9 +1107,7 @@ def run_forward_only(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": workload_text(wl, False), "global_batch": B * world, "seq_len": N,
                    "parallelism": f"replicas{world}",
-                   "l2": "flushed (256 MB write) between timed steps, outside the events",
-                   "fwd_grid": f"persistent, one CTA per SM, {args.fwd_schedule} item order" if persistent
-                   else "one CTA per work item"},
+                   "l2": "flushed (256 MB write) between timed steps, outside the events"},
         "fwd_us": round(ms * 1e3, 2), "fwd_gbs": round(gbs, 1),
         "pct_of_measured_peak": round(100 * tflops / peaks["bf16_tflops"], 2),
         "pct_of_spec_peak_2250": round(100 * tflops / 2250.0, 2),

@@ -72,20 +72,12 @@ def _raise(name, st):
         raise FAError(name, st)
 
 
-_SCHEDULES = {"balanced": _lib.FA_SCHED_BALANCED, "head_major": _lib.FA_SCHED_HEAD_MAJOR}
-
-
 def forward(q, k, v, scale: float | None = None, causal: bool = False, window: int = 0,
-            out=None, lse=None, persistent: bool = False, ctas: int = 0, schedule: str = "balanced"):
+            out=None, lse=None):
     """O, L = attention(Q, K, V); O bf16 [B,H,N,d], L fp32 [B,H,N] (natural-log logsumexp).
 
-    d is 64, 128 or 256.  ``persistent`` runs the same tiles on a persistent grid
-    of ``ctas`` CTAs (0: one per SM) that loop over the work items, taken in the ``schedule``
-    "balanced" (longest first over all heads when a mask makes the costs differ) or
-    "head_major" order."""
+    d is 64, 128 or 256."""
     import torch
-    if persistent and schedule not in _SCHEDULES:
-        raise ValueError(f"schedule must be one of {sorted(_SCHEDULES)}")
     H_kv = _check_qkv(q, k, v)
     B, H, N, d = q.shape
     scale = default_scale(d) if scale is None else float(scale)
@@ -97,13 +89,7 @@ def forward(q, k, v, scale: float | None = None, causal: bool = False, window: i
     _check_lse(lse, q, B * H * N)
     ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr())
     mask = (scale, int(bool(causal)), int(window), _stream_handle(q.device))
-    if persistent:
-        st = None if all(t.is_contiguous() for t in (q, k, v, out)) else _lib.strides_array((q, k, v, out))
-        _raise("fa_fwd_persistent", _lib.fa_fwd_persistent(*ptrs, B, H, H_kv, N, d,
-                                                           ctypes.addressof(st) if st is not None else 0,
-                                                           scale, int(bool(causal)), int(window), int(ctas),
-                                                           _SCHEDULES[schedule], _stream_handle(q.device)))
-    elif not all(t.is_contiguous() for t in (q, k, v, out)):
+    if not all(t.is_contiguous() for t in (q, k, v, out)):
         st = _lib.strides_array((q, k, v, out))
         _raise("fa_fwd_strided", _lib.fa_fwd_strided(*ptrs, B, H, H_kv, N, d, ctypes.addressof(st), *mask))
     elif H_kv == H:
@@ -154,18 +140,13 @@ def bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
 
 
 def backward(q, k, v, o, lse, do, scale: float | None = None, causal: bool = False, window: int = 0,
-             grads=None, workspace=None, phases: int = 7, persistent: bool = False, ctas: int = 0,
-             schedule: str = "balanced"):
+             grads=None, workspace=None, phases: int = 7):
     """dQ (like q), dK, dV (like k) of sum(O o dO), recomputing P from the forward's L.
 
     ``phases`` selects the steps of the backward (1 preprocess, 2 recompute kernel, 4 dQ
     finalise); running 1, 2, 4 in turn with the same workspace equals the default 7.
-    ``persistent`` (d 64 or 128) runs the recompute kernel on a persistent grid of ``ctas`` CTAs
-    (0: one per SM) that loop over the (K/V head, key tile) items in the ``schedule`` order.
     """
     import torch
-    if persistent and schedule not in _SCHEDULES:
-        raise ValueError(f"schedule must be one of {sorted(_SCHEDULES)}")
     H_kv = _check_qkv(q, k, v, o, do)
     B, H, N, d = q.shape
     _check_lse(lse, q, B * H * N)
@@ -181,15 +162,6 @@ def backward(q, k, v, o, lse, do, scale: float | None = None, causal: bool = Fal
     dq, dk, dv = grads
     ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
             dq.data_ptr(), dk.data_ptr(), dv.data_ptr())
-    if persistent:
-        st = None
-        if not all(t.is_contiguous() for t in (q, k, v, o, do, dq, dk, dv)):
-            st = _lib.strides_array((q, k, v, o, do, dq, dk, dv))
-        _raise("fa_bwd_persistent", _lib.fa_bwd_persistent(
-            *ptrs, B, H, H_kv, N, d, ctypes.addressof(st) if st is not None else 0, scale, int(bool(causal)),
-            int(window), workspace.data_ptr(), workspace.numel() * workspace.element_size(), int(phases), int(ctas),
-            _SCHEDULES[schedule], _stream_handle(q.device)))
-        return dq, dk, dv
     rest = (d, scale, int(bool(causal)), int(window), workspace.data_ptr(),
             workspace.numel() * workspace.element_size())
     if not all(t.is_contiguous() for t in (q, k, v, o, do, dq, dk, dv)):

@@ -37,10 +37,6 @@ SIGNATURES = {
     "fa_bwd_noalloc": (_c_int, [_c_void_p] * 9 + [_c_int] * 4 + [_c_float, _c_int, _c_int, _c_void_p]),
     "fa_fwd_gqa": (_c_int, [_c_void_p] * 5 + [_c_int] * 5 + [_c_float, _c_int, _c_int, _c_void_p]),
     "fa_fwd_strided": (_c_int, [_c_void_p] * 5 + [_c_int] * 5 + [_c_void_p, _c_float, _c_int, _c_int, _c_void_p]),
-    "fa_fwd_persistent": (_c_int, [_c_void_p] * 5 + [_c_int] * 5 + [_c_void_p, _c_float, _c_int, _c_int, _c_int,
-                                                                   _c_int, _c_void_p]),
-    "fa_bwd_persistent": (_c_int, [_c_void_p] * 9 + [_c_int] * 5 + [_c_void_p, _c_float, _c_int, _c_int, _c_void_p,
-                                                                    _c_size_t, _c_int, _c_int, _c_int, _c_void_p]),
     "fa_bwd_strided": (_c_int, [_c_void_p] * 9 + [_c_int] * 5 + [_c_void_p, _c_float, _c_int, _c_int, _c_void_p,
                                                                  _c_size_t, _c_int, _c_void_p]),
     "fa_bwd_gqa": (_c_int, [_c_void_p] * 9 + [_c_int] * 5 + [_c_float, _c_int, _c_int, _c_void_p, _c_size_t,
@@ -154,25 +150,6 @@ def strides_array(tensors):
 def fa_fwd_strided(q, k, v, o, lse, B, H, H_kv, N, d, strides, scale, causal, window, stream) -> int:
     """fa_fwd_gqa with per-array strides (``strides``: address of 4 fa_strides, or 0)."""
     return _call("fa_fwd_strided", q, k, v, o, lse, B, H, H_kv, N, d, strides, scale, causal, window, stream)
-
-
-FA_SCHED_BALANCED, FA_SCHED_HEAD_MAJOR = 0, 1
-
-
-def fa_fwd_persistent(q, k, v, o, lse, B, H, H_kv, N, d, strides, scale, causal, window, ctas, schedule,
-                      stream) -> int:
-    """fa_fwd_strided on a persistent grid of ``ctas`` CTAs (0: one per SM); d 64, 128 or 256;
-    ``schedule`` FA_SCHED_BALANCED or FA_SCHED_HEAD_MAJOR."""
-    return _call("fa_fwd_persistent", q, k, v, o, lse, B, H, H_kv, N, d, strides, scale, causal, window, ctas,
-                 schedule, stream)
-
-
-def fa_bwd_persistent(q, k, v, o, lse, dO, dq, dk, dv, B, H, H_kv, N, d, strides, scale, causal, window, workspace,
-                      workspace_bytes, phases, ctas, schedule, stream) -> int:
-    """fa_bwd_strided (``strides`` may be 0: packed) with its main phase on a persistent grid of
-    ``ctas`` CTAs (0: one per SM); d 64 or 128."""
-    return _call("fa_bwd_persistent", q, k, v, o, lse, dO, dq, dk, dv, B, H, H_kv, N, d, strides, scale, causal,
-                 window, workspace, workspace_bytes, phases, ctas, schedule, stream)
 
 
 def fa_bwd_strided(q, k, v, o, lse, dO, dq, dk, dv, B, H, H_kv, N, d, strides, scale, causal, window, workspace,

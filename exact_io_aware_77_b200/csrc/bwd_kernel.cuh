@@ -41,7 +41,7 @@
 
 #include <type_traits>
 
-#include "persist_sched.cuh"
+#include "grid_sched.cuh"
 #include "sm100.cuh"
 
 namespace fa {
@@ -49,8 +49,7 @@ namespace fa {
 constexpr int kBwdKeys = 128;    // keys per CTA
 constexpr int kBwdRows = 128;    // queries per iteration
 constexpr int kBwdQStages = 2;
-constexpr int kBwdThreads = 384;       // fa_bwd_persist_kernel: 8 compute warps, TMA, MMA, 2 reduction warps
-constexpr int kBwdMainThreads = 320;   // fa_bwd_kernel: 8 compute warps, TMA, MMA
+constexpr int kBwdThreads = 320;   // 8 compute warps, TMA, MMA
 constexpr int kBwdWarpTma = 8;
 constexpr int kBwdWarpMma = 9;
 constexpr uint32_t kTdK = 0, kTdV = 128, kTS = 256, kTP = 256, kTdP = 384, kTdS = 384, kTdQ = 384;
@@ -173,7 +172,7 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_final(const float* __restrict__
 // tm_dq: the fp32 accumulator [BH, Np, D] as the 4-D tensor (D, Np, BH, 1), 32 x 32 boxes with
 // the 128-byte swizzle (the layout of a compute warp's staging slot).
 template <int D>
-__global__ void __launch_bounds__(kBwdMainThreads, 1)
+__global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                   const __grid_constant__ CUtensorMap tm_dq, const BwdParams prm) {

@@ -12,13 +12,10 @@
 #include "../../include/fa.h"
 
 #include "fwd_kernel.cuh"
-#include "fwd_persist_kernel.cuh"
 #include "fwd256_kernel.cuh"
-#include "fwd256_persist_kernel.cuh"
 #include "fp8_ops.cuh"
 #include "fwd_fp8_kernel.cuh"
 #include "bwd_kernel.cuh"
-#include "bwd_persist_kernel.cuh"
 #include "bwd256_kernel.cuh"
 #include "decode_ops.cuh"
 #include "decode_kernel.cuh"
@@ -183,34 +180,6 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-// the persistent form (fwd_persist_kernel.cuh): `ctas` CTAs, or one per SM when ctas is 0, each
-// taking its items round by round from the item order (snake-dealt)
-template <int D>
-int launch_fwd_persist(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv,
-                       int N, const Strides* st, float scale, int causal, int window, int ctas, int schedule,
-                       cudaStream_t stream) {
-  CUtensorMap tq, tk, tv;
-  FwdParams prm;
-  if (!fwd_setup<D>(q, k, v, o, lse, B, H, H_kv, N, st, scale, causal, window, &tq, &tk, &tv, &prm))
-    return FA_ERR_CUDA;
-  if (ctas == 0) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&ctas, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      return FA_ERR_CUDA;
-  }
-  const long long n_items = (long long)prm.n_pairs * prm.BH;
-  const unsigned grid = unsigned(ctas < n_items ? ctas : n_items);
-  // an item's cost grows with its query position under a causal mask, and is lower for the first
-  // pairs of a band: then longest first over all heads; with every item alike, head-major
-  const bool costs_vary = causal || (prm.window > 0 && prm.window < N);
-  const int order = schedule == FA_SCHED_BALANCED && costs_vary ? kOrderPairMajor : kOrderHeadMajor;
-  const int smem = fwd_smem_bytes(int(sizeof(FwdPersistSmem<D>)));
-  if (set_smem(fa_fwd_persist_kernel<D>, smem) != FA_OK) return FA_ERR_CUDA;
-  fa_fwd_persist_kernel<D><<<grid, kFwdThreads, smem, stream>>>(tq, tk, tv, prm, order);
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
-}
-
 // head dimension 256: one 128-row query tile per CTA, 64-key K/V tiles (fwd256_kernel.cuh)
 int launch_fwd256(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv, int N,
                   const Strides* st, float scale, int causal, int window, cudaStream_t stream) {
@@ -237,45 +206,6 @@ int launch_fwd256(const void* q, const void* k, const void* v, void* o, float* l
   const int smem = int(sizeof(Fwd256Smem)) + 1024;
   if (set_smem(fa_fwd256_kernel, smem) != FA_OK) return FA_ERR_CUDA;
   fa_fwd256_kernel<<<unsigned(prm.n_pairs) * unsigned(BH), k256Threads, smem, stream>>>(tq, tk, tv, prm);
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
-}
-
-// head dimension 256 on the persistent grid (fwd256_persist_kernel.cuh)
-int launch_fwd256_persist(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv,
-                          int N, const Strides* st, float scale, int causal, int window, int ctas, int schedule,
-                          cudaStream_t stream) {
-  CUtensorMap tq, tk, tv;
-  if (!make_map_bf16(&tq, q, kD256, N, H, B, st[0], k256BlockM) ||
-      !make_map_bf16(&tk, k, kD256, N, H_kv, B, st[1], k256BlockN) ||
-      !make_map_bf16(&tv, v, kD256, N, H_kv, B, st[2], k256BlockN))
-    return FA_ERR_CUDA;
-  FwdParams prm;
-  prm.o = static_cast<__nv_bfloat16*>(o);
-  prm.lse = lse;
-  prm.N = N;
-  prm.BH = B * H;
-  prm.H = H;
-  prm.group = H / H_kv;
-  prm.o_st = st[3];
-  prm.n_pairs = (N + k256BlockM - 1) / k256BlockM;   // query tiles per head
-  prm.causal = causal;
-  prm.window = window > N ? N : window;
-  prm.scale_log2 = scale * 1.4426950408889634f;
-  prm.wait_limit_ns = g_wait_limit_ns;
-  if (ctas == 0) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&ctas, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      return FA_ERR_CUDA;
-  }
-  const long long n_items = (long long)prm.n_pairs * prm.BH;
-  const unsigned grid = unsigned(ctas < n_items ? ctas : n_items);
-  const bool costs_vary = causal || (prm.window > 0 && prm.window < N);
-  const int order = schedule == FA_SCHED_BALANCED && costs_vary ? kOrderPairMajor : kOrderHeadMajor;
-  static_assert(sizeof(Fwd256PersistSmem) + 1024 <= 232448, "d = 256 persistent forward shared memory exceeds 227 KB");
-  const int smem = int(sizeof(Fwd256PersistSmem)) + 1024;
-  if (set_smem(fa_fwd256_persist_kernel, smem) != FA_OK) return FA_ERR_CUDA;
-  fa_fwd256_persist_kernel<<<grid, k256Threads, smem, stream>>>(tq, tk, tv, prm, order);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -318,8 +248,7 @@ size_t bwd_workspace_bytes(long long BH, int N, int d) {
 template <int D>
 int launch_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
                void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, const Strides* st, float scale,
-               int causal, int window, void* ws, cudaStream_t stream, int phases = kBwdAllPhases,
-               int persist_ctas = -1, int schedule = FA_SCHED_BALANCED) {
+               int causal, int window, void* ws, cudaStream_t stream, int phases = kBwdAllPhases) {
   // st: q, k, v, o, dO, dq, dk, dv
   const int BH = B * H, BH_kv = B * H_kv;
   const long long Np = padded_rows(N);
@@ -369,25 +298,6 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
     if (set_smem(fa_bwd256_kernel, smem) != FA_OK) return FA_ERR_CUDA;
     fa_bwd256_kernel<<<unsigned(prm.n_kv_tiles) * unsigned(BH_kv) * 2u, kB256Threads, smem, stream>>>(tq, tk, tv, tdo,
                                                                                                          prm);
-  } else if (persist_ctas >= 0) {
-    // the persistent form (bwd_persist_kernel.cuh): persist_ctas CTAs, or one per SM when 0
-    int ctas = persist_ctas;
-    if (ctas == 0) {
-      int dev = 0;
-      if (cudaGetDevice(&dev) != cudaSuccess ||
-          cudaDeviceGetAttribute(&ctas, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return FA_ERR_CUDA;
-    }
-    const long long n_items = (long long)prm.n_kv_tiles * BH_kv;
-    const unsigned grid = unsigned(ctas < n_items ? ctas : n_items);
-    // a key tile's cost falls with its position under a causal mask and at a band's edges:
-    // then key-tile-major from tile 0 over all heads; with every item alike, head-major
-    const bool costs_vary = causal || (prm.window > 0 && prm.window < N);
-    const int order = schedule == FA_SCHED_BALANCED && costs_vary ? kOrderPairMajor : kOrderHeadMajor;
-    static_assert(sizeof(BwdPersistSmem<D>) <= 232448, "persistent backward shared memory exceeds 227 KB");
-    const int smem = int(sizeof(BwdPersistSmem<D>));
-    if (set_smem(fa_bwd_persist_kernel<D>, smem) != FA_OK) return FA_ERR_CUDA;
-    fa_bwd_persist_kernel<D><<<grid, kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, prm, order);
   } else {
     static_assert(sizeof(BwdSmem<D>) <= 232448, "backward shared memory exceeds 227 KB");
     const int smem = int(sizeof(BwdSmem<D>));   // the kernel checks that the base is 1 KB aligned
@@ -395,7 +305,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
     if (!make_map_dq_acc(&tdq, dq_acc, D, Np, BH)) return FA_ERR_CUDA;
     if (set_smem(fa_bwd_kernel<D>, smem) != FA_OK) return FA_ERR_CUDA;
     // one CTA per (K/V head, key tile)
-    fa_bwd_kernel<D><<<unsigned(prm.n_kv_tiles) * unsigned(BH_kv), kBwdMainThreads, smem, stream>>>(tq, tk, tv, tdo,
+    fa_bwd_kernel<D><<<unsigned(prm.n_kv_tiles) * unsigned(BH_kv), kBwdThreads, smem, stream>>>(tq, tk, tv, tdo,
                                                                                                    tdq, prm);
   }
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
@@ -529,7 +439,7 @@ extern "C" {
 static int bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
                     void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, int d, const fa_strides* strides,
                     float scale, int causal, int window, void* workspace, size_t workspace_bytes, int phases,
-                    void* stream, int persist_ctas = -1, int schedule = FA_SCHED_BALANCED);
+                    void* stream);
 
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
            float scale, int causal, int window, void* stream) {
@@ -562,32 +472,6 @@ int fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* 
     case 64: return launch_fwd<64>(q, k, v, o, lse, B, H, H_kv, N, s4, scale, causal, window, s);
     case 128: return launch_fwd<128>(q, k, v, o, lse, B, H, H_kv, N, s4, scale, causal, window, s);
     default: return launch_fwd256(q, k, v, o, lse, B, H, H_kv, N, s4, scale, causal, window, s);
-  }
-}
-
-int fa_fwd_persistent(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv,
-                      int N, int d, const fa_strides* strides, float scale, int causal, int window, int ctas,
-                      int schedule, void* stream) {
-  if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
-  int st = check_problem(B, H, N, d, scale, causal, window);
-  if (st == FA_OK) st = check_kv_heads(H, H_kv);
-  if (st == FA_OK && (ctas < 0 || (schedule != FA_SCHED_BALANCED && schedule != FA_SCHED_HEAD_MAJOR)))
-    st = FA_ERR_SHAPE;
-  if (st != FA_OK) return st;
-  Strides s4[4] = {packed(H, N, d), packed(H_kv, N, d), packed(H_kv, N, d), packed(H, N, d)};
-  if (strides)
-    for (int i = 0; i < 4; ++i) {
-      s4[i] = Strides{strides[i].b, strides[i].h, strides[i].n};
-      if (!strides_ok(s4[i])) return FA_ERR_ALIGN;
-    }
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
-    return FA_ERR_ALIGN;
-  if ((st = check_device()) != FA_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  switch (d) {
-    case 64: return launch_fwd_persist<64>(q, k, v, o, lse, B, H, H_kv, N, s4, scale, causal, window, ctas, schedule, s);
-    case 128: return launch_fwd_persist<128>(q, k, v, o, lse, B, H, H_kv, N, s4, scale, causal, window, ctas, schedule, s);
-    default: return launch_fwd256_persist(q, k, v, o, lse, B, H, H_kv, N, s4, scale, causal, window, ctas, schedule, s);
   }
 }
 
@@ -629,7 +513,7 @@ int fa_bwd_strided(const void* q, const void* k, const void* v, const void* o, c
 static int bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
                     void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, int d, const fa_strides* strides,
                     float scale, int causal, int window, void* workspace, size_t workspace_bytes, int phases,
-                    void* stream, int persist_ctas, int schedule) {
+                    void* stream) {
   if (phases < 1 || phases > kBwdAllPhases) return FA_ERR_PHASES;
   if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FA_ERR_NULL;
   int st = check_problem(B, H, N, d, scale, causal, window);
@@ -654,20 +538,10 @@ static int bwd_impl(const void* q, const void* k, const void* v, const void* o, 
   if ((st = check_device()) != FA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (d) {
-    case 64: return launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, s8, scale, causal, window, workspace, s, phases, persist_ctas, schedule);
-    case 128: return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, s8, scale, causal, window, workspace, s, phases, persist_ctas, schedule);
+    case 64: return launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, s8, scale, causal, window, workspace, s, phases);
+    case 128: return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, s8, scale, causal, window, workspace, s, phases);
     default: return launch_bwd<256>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, s8, scale, causal, window, workspace, s, phases);
   }
-}
-
-int fa_bwd_persistent(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
-                      void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, int d, const fa_strides* strides,
-                      float scale, int causal, int window, void* workspace, size_t workspace_bytes, int phases,
-                      int ctas, int schedule, void* stream) {
-  if (ctas < 0 || (schedule != FA_SCHED_BALANCED && schedule != FA_SCHED_HEAD_MAJOR)) return FA_ERR_SHAPE;
-  if (d == 256 && check_problem(B, H, N, d, scale, causal, window) == FA_OK) return FA_ERR_HEADDIM;
-  return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, d, strides, scale, causal, window, workspace,
-                  workspace_bytes, phases, stream, ctas, schedule);
 }
 
 int fa_fwd_fp8(const void* q8, const void* k8, const void* vt8, float q_scale, float k_scale, float v_scale, void* o,

@@ -32,7 +32,7 @@
 
 #include <type_traits>
 
-#include "persist_sched.cuh"
+#include "grid_sched.cuh"
 #include "sm100.cuh"
 
 namespace fa {

@@ -164,54 +164,6 @@ FA_EXPORT int fa_bwd_strided(const void* q, const void* k, const void* v, const 
                              size_t workspace_bytes, int phases, void* stream);
 
 /*
- * fa_fwd_strided computed by a persistent grid: `ctas` CTAs (0: one per SM of the current
- * device), each looping over the forward's work items (pairs of 128-row query tiles of one
- * head), so that one item's Q load and first S = Q K^T overlap the previous item's output
- * write.  The computation is the tiled forward of the FlashAttention (EN) page ("Algorithm"):
- * the same tiles, online softmax and logsumexp as fa_fwd_strided, whose results it returns bit
- * for bit (the per-tile arithmetic and its order within a tile are the same; only which CTA
- * takes which tile differs).  At d = 256 the items are single 128-row query tiles, as in
- * fa_fwd_strided's d = 256 kernel.
- *
- *   schedule  FA_SCHED_BALANCED: with a causal or banded mask (item costs differ) the items go
- *             longest first over all heads, dealt to the CTAs round by round in a snake
- *             (0, 1, ..., G-1, then G-1, ..., 0), which evens out the CTAs' total work; with no
- *             mask, head-major.  FA_SCHED_HEAD_MAJOR: head-major, longest first within a head,
- *             snake-dealt the same way.
- *   d         64, 128 or 256.
- *
- * ctas < 0 or another schedule gives FA_ERR_SHAPE.  Arguments, strides, errors, streams and
- * ownership are otherwise as for fa_fwd_strided.
- */
-enum { FA_SCHED_BALANCED = 0, FA_SCHED_HEAD_MAJOR = 1 };
-FA_EXPORT int fa_fwd_persistent(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-                                int H_kv, int N, int d, const fa_strides* strides, float scale, int causal,
-                                int window, int ctas, int schedule, void* stream);
-
-/*
- * fa_bwd_strided computed by a persistent grid in its main phase (`phases` as for
- * fa_bwd_phases: 1 preprocess, 2 the recompute kernel, 4 finalise dQ; 7 all): `ctas` CTAs (0: one
- * per SM of the current device) loop over the (K/V head, 128-key tile) work items, so that one
- * item's K/V load and first products overlap the previous item's dK/dV write.  The computation
- * is the recomputation of the FlashAttention (EN) page ("Algorithm"): the same tiles and
- * arithmetic as fa_bwd_strided, whose dK and dV it returns bit for bit (dQ sums the same fp32
- * partial products, in an order that may differ, so it agrees to rounding).
- *
- *   schedule  FA_SCHED_BALANCED: with a causal or banded mask the items go key-tile-major from
- *             tile 0 (the longest under a causal mask) over all heads, snake-dealt as in
- *             fa_fwd_persistent; with no mask, head-major.  FA_SCHED_HEAD_MAJOR: head-major.
- *   strides   NULL for packed arrays, else 8 fa_strides as for fa_bwd_strided.
- *   d         64 or 128 (FA_ERR_HEADDIM otherwise).
- *
- * ctas < 0 or another schedule gives FA_ERR_SHAPE.  Workspace, errors, streams and ownership
- * are otherwise as for fa_bwd_strided.
- */
-FA_EXPORT int fa_bwd_persistent(const void* q, const void* k, const void* v, const void* o, const float* lse,
-                                const void* dO, void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, int d,
-                                const fa_strides* strides, float scale, int causal, int window, void* workspace,
-                                size_t workspace_bytes, int phases, int ctas, int schedule, void* stream);
-
-/*
  * Forward of a few new query rows over a longer key sequence: a generation step over a
  * key/value cache.  The FlashAttention (NL) page names engines for LLM inference that work on
  * the key/value cache during streaming generation ("Gespecialiseerde oplossingen": FlashInfer;

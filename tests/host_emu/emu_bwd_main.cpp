@@ -7,8 +7,6 @@
 #ifdef EMU_BWD256
 #include "bwd256_kernel.cuh"
 #define EMU_D 256
-#elif defined(EMU_BWD_PERSIST)
-#include "bwd_persist_kernel.cuh"
 #else
 #include "bwd_kernel.cuh"
 #endif
@@ -23,8 +21,6 @@
 namespace fa {
 #ifdef EMU_BWD256
 alignas(1024) uint8_t smem_raw[sizeof(Bwd256Smem)];
-#elif defined(EMU_BWD_PERSIST)
-alignas(1024) uint8_t smem_raw[sizeof(BwdPersistSmem<EMU_D>)];
 #else
 alignas(1024) uint8_t smem_raw[sizeof(BwdSmem<EMU_D>)];
 #endif
@@ -62,12 +58,7 @@ CUtensorMap make_map(const uint16_t* base, int d, int rows, int heads, int B, in
 }
 
 int main(int argc, char** argv) {
-#ifdef EMU_BWD_PERSIST
-  // persistent form: ... prefix grid order   (grid: persistent CTAs; order: 0 head-major, 1 cost-major)
-  if (argc != 11) { std::fprintf(stderr, "bad args\n"); return 2; }
-#else
   if (argc != 9) { std::fprintf(stderr, "bad args\n"); return 2; }
-#endif
   const int B = atoi(argv[1]), H = atoi(argv[2]), Hkv = atoi(argv[3]), N = atoi(argv[4]), causal = atoi(argv[5]),
             window = atoi(argv[6]);
   const float scale = float(atof(argv[7]));
@@ -138,16 +129,8 @@ int main(int argc, char** argv) {
 #ifdef EMU_BWD256
   emu_launch(unsigned(prm.n_kv_tiles) * unsigned(BH_kv) * 2u, kB256Threads, sizeof(fa::smem_raw),
              [&] { fa_bwd256_kernel(tq, tk, tv, tdo, prm); }, fa::smem_raw);
-#elif defined(EMU_BWD_PERSIST)
-  {
-    const unsigned n_items = unsigned(prm.n_kv_tiles) * unsigned(BH_kv);
-    const unsigned grid = std::min(n_items, unsigned(atoi(argv[9])));
-    const int order = atoi(argv[10]);
-    emu_launch(grid, kBwdThreads, sizeof(fa::smem_raw), [&] { fa_bwd_persist_kernel<D>(tq, tk, tv, tdo, prm, order); },
-               fa::smem_raw);
-  }
 #else
-  emu_launch(unsigned(prm.n_kv_tiles) * unsigned(BH_kv), kBwdMainThreads, sizeof(fa::smem_raw),
+  emu_launch(unsigned(prm.n_kv_tiles) * unsigned(BH_kv), kBwdThreads, sizeof(fa::smem_raw),
              [&] { fa_bwd_kernel<D>(tq, tk, tv, tdo, tdq, prm); }, fa::smem_raw);
 #endif
   if (g_status != 0) { std::fprintf(stderr, "device status %d\n", g_status); return 3; }

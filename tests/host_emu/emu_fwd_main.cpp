@@ -4,17 +4,12 @@
 // [B, heads, N, d] arrays.
 // usage: emu_fwd_main B H Hkv N causal window scale prefix   (prefix.q/.k/.v bf16; writes .o, .lse)
 #include "emu.h"
-#ifdef EMU_FWD256_PERSIST
-#include "fwd256_persist_kernel.cuh"
-#define EMU_D 256
-#elif defined(EMU_FWD256)
+#if defined(EMU_FWD256)
 #include "fwd256_kernel.cuh"
 #define EMU_D 256
 #elif defined(EMU_FWD_FP8)
 #include "fwd_fp8_kernel.cuh"
 #define EMU_D 128
-#elif defined(EMU_FWD_PERSIST)
-#include "fwd_persist_kernel.cuh"
 #else
 #include "fwd_kernel.cuh"
 #endif
@@ -29,14 +24,10 @@
 namespace fa {
 // the kernel's dynamic shared memory: exactly one (1024-byte aligned) FwdSmem, so AddressSanitizer
 // sees any access past it
-#ifdef EMU_FWD256_PERSIST
-alignas(1024) uint8_t smem_raw[sizeof(Fwd256PersistSmem)];
-#elif defined(EMU_FWD256)
+#if defined(EMU_FWD256)
 alignas(1024) uint8_t smem_raw[sizeof(Fwd256Smem)];
 #elif defined(EMU_FWD_FP8)
 alignas(1024) uint8_t smem_raw[sizeof(FwdFp8Smem)];
-#elif defined(EMU_FWD_PERSIST)
-alignas(1024) uint8_t smem_raw[sizeof(FwdPersistSmem<EMU_D>)];
 #else
 alignas(1024) uint8_t smem_raw[sizeof(FwdSmem<EMU_D>)];
 #endif
@@ -127,15 +118,8 @@ int main(int argc, char** argv) {
   return 0;
 }
 #else
-// usage (persistent form): ... prefix grid order   (grid: the number of persistent CTAs; order:
-// 0 head-major, 1 pair-major item order)
-// (EMU_FWD256_PERSIST, the d = 256 persistent form, is built together with EMU_FWD256)
 int main(int argc, char** argv) {
-#if defined(EMU_FWD_PERSIST) || defined(EMU_FWD256_PERSIST)
-  if (argc != 11) { std::fprintf(stderr, "bad args\n"); return 2; }
-#else
   if (argc != 9) { std::fprintf(stderr, "bad args\n"); return 2; }
-#endif
   const int B = atoi(argv[1]), H = atoi(argv[2]), Hkv = atoi(argv[3]), N = atoi(argv[4]), causal = atoi(argv[5]),
             window = atoi(argv[6]);
   const float scale = float(atof(argv[7]));
@@ -170,20 +154,9 @@ int main(int argc, char** argv) {
   prm.window = window > N ? N : window;
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.wait_limit_ns = 60ull * 1000000000ull;
-#if defined(EMU_FWD_PERSIST) || defined(EMU_FWD256_PERSIST)
-  const unsigned n_items = unsigned(prm.n_pairs) * unsigned(B * H);
-  const unsigned grid = std::min(n_items, unsigned(atoi(argv[9])));
-  const int order = atoi(argv[10]);
-#else
   const unsigned grid = unsigned(prm.n_pairs) * unsigned(B * H);
-#endif
   std::printf("grid %u smem %zu\n", grid, sizeof(fa::smem_raw));
-#ifdef EMU_FWD_PERSIST
-  emu_launch(grid, kFwdThreads, sizeof(fa::smem_raw), [&] { fa_fwd_persist_kernel<D>(tq, tk, tv, prm, order); }, fa::smem_raw);
-#elif defined(EMU_FWD256_PERSIST)
-  emu_launch(grid, k256Threads, sizeof(fa::smem_raw), [&] { fa_fwd256_persist_kernel(tq, tk, tv, prm, order); },
-             fa::smem_raw);
-#elif defined(EMU_FWD256)
+#if defined(EMU_FWD256)
   emu_launch(grid, k256Threads, sizeof(fa::smem_raw), [&] { fa_fwd256_kernel(tq, tk, tv, prm); }, fa::smem_raw);
 #else
   emu_launch(grid, kFwdThreads, sizeof(fa::smem_raw), [&] { fa_fwd_kernel<D>(tq, tk, tv, prm); }, fa::smem_raw);

@@ -136,61 +136,6 @@ def test_strided_entry_points_validate_strides(lib):
     assert _lib.STATUS_NAMES[st] == "FA_ERR_NULL"
 
 
-@pytest.mark.parametrize("kw,code", [
-    (dict(ptrs=[0, A, A, A, A]), "FA_ERR_NULL"),
-    (dict(ptrs=[A, A, A, A, 0]), "FA_ERR_NULL"),
-    (dict(N=0), "FA_ERR_SHAPE"),
-    (dict(H_kv=3), "FA_ERR_SHAPE"),
-    (dict(ctas=-1), "FA_ERR_SHAPE"),
-    (dict(schedule=2), "FA_ERR_SHAPE"),
-    (dict(schedule=-1), "FA_ERR_SHAPE"),
-    (dict(d=96), "FA_ERR_HEADDIM"),
-    (dict(causal=2), "FA_ERR_MASK"),
-    (dict(scale=float("nan")), "FA_ERR_SCALE"),
-    (dict(ptrs=[A, A, A + 8, A, A]), "FA_ERR_ALIGN"),
-    (dict(bad_stride=True), "FA_ERR_ALIGN"),
-])
-def test_persistent_fwd_rejects_bad_arguments(lib, kw, code):
-    """fa_fwd_persistent: fa_fwd_strided's checks, ctas >= 0, a known schedule."""
-    a = dict(GOOD, H_kv=GOOD["H"], ctas=0, schedule=_lib.FA_SCHED_BALANCED)
-    ptrs = kw.pop("ptrs", [A + 4096 * i for i in range(5)])
-    bad_stride = kw.pop("bad_stride", False)
-    a.update(kw)
-    arr = None
-    if bad_stride:
-        arr = (_lib.FaStrides * 4)(*[_lib.FaStrides(2 * 128 * 64, 128 * 64, 64) for _ in range(4)])
-        arr[3] = _lib.FaStrides(2 * 128 * 64, 128 * 64, 12)
-    st = _lib.fa_fwd_persistent(*ptrs, a["B"], a["H"], a["H_kv"], a["N"], a["d"],
-                                ctypes.addressof(arr) if arr is not None else None, a["scale"], a["causal"],
-                                a["window"], a["ctas"], a["schedule"], None)
-    assert _lib.STATUS_NAMES[st] == code
-
-
-@pytest.mark.parametrize("kw,code", [
-    (dict(ptrs=[A] * 8 + [0]), "FA_ERR_NULL"),
-    (dict(N=0), "FA_ERR_SHAPE"),
-    (dict(H_kv=3), "FA_ERR_SHAPE"),
-    (dict(ctas=-2), "FA_ERR_SHAPE"),
-    (dict(schedule=5), "FA_ERR_SHAPE"),
-    (dict(d=256), "FA_ERR_HEADDIM"),
-    (dict(d=32), "FA_ERR_HEADDIM"),
-    (dict(phases=0), "FA_ERR_PHASES"),
-    (dict(window=-1), "FA_ERR_MASK"),
-    (dict(ws=0), "FA_ERR_WORKSPACE"),
-    (dict(ws_bytes=64), "FA_ERR_WORKSPACE"),
-    (dict(ptrs=[A] * 6 + [A + 4] + [A] * 2), "FA_ERR_ALIGN"),
-])
-def test_persistent_bwd_rejects_bad_arguments(lib, kw, code):
-    """fa_bwd_persistent: the backward's checks, d 64 or 128 only, ctas >= 0, a known schedule."""
-    a = dict(GOOD, H_kv=GOOD["H"], ctas=0, schedule=_lib.FA_SCHED_BALANCED, phases=7, ws=A + 65536,
-             ws_bytes=1 << 30)
-    ptrs = kw.pop("ptrs", [A + 4096 * i for i in range(9)])
-    a.update(kw)
-    st = _lib.fa_bwd_persistent(*ptrs, a["B"], a["H"], a["H_kv"], a["N"], a["d"], None, a["scale"], a["causal"],
-                                a["window"], a["ws"], a["ws_bytes"], a["phases"], a["ctas"], a["schedule"], None)
-    assert _lib.STATUS_NAMES[st] == code
-
-
 def _dec(ws_bytes=1 << 30, **kw):
     a = dict(B=1, H=8, H_kv=2, N_q=1, N_k=4096, d=128, scale=0.125, causal=1, window=0)
     ptrs = kw.pop("ptrs", [A + 4096 * i for i in range(5)])

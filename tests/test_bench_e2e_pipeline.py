@@ -135,7 +135,7 @@ class FakeFA:
         return 1 << 20
 
     @staticmethod
-    def forward(q, k, v, scale, causal, window, out=None, lse=None, persistent=False, schedule="balanced"):
+    def forward(q, k, v, scale, causal, window, out=None, lse=None):
         SIM.op("sm", FWD_MS, reads=[q, k, v], writes=[out, lse])
         return out, lse
 

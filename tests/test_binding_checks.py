@@ -46,13 +46,3 @@ def test_decode_workspace_size_argument_checks():
                  (0, 8, 2, 1, 10, 64)):
         with pytest.raises(ValueError):
             fa.decode_workspace_size(*args)
-
-
-def test_persistent_schedule_name_checked_first():
-    q = _q()
-    with pytest.raises(ValueError, match="schedule"):
-        fa.forward(q, q, q, persistent=True, schedule="pair_major")
-    with pytest.raises(ValueError, match="bf16 CUDA tensors"):   # a known name passes on to the tensor checks
-        fa.forward(q, q, q, persistent=True, schedule="head_major")
-    with pytest.raises(ValueError, match="schedule"):
-        fa.backward(q, q, q, q, None, q, persistent=True, schedule="cost")

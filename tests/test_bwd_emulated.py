@@ -31,15 +31,9 @@ def emu_bwd(tmp_path_factory):
             64: ("bwd_kernel.cuh", "emu_bwd_main.cpp", "emu_bwd_64", ("EMU_D=64",)),
             128: ("bwd_kernel.cuh", "emu_bwd_main.cpp", "emu_bwd_128", ("EMU_D=128",)),
             256: (["bwd256_kernel.cuh", "bwd_kernel.cuh"], "emu_bwd_main.cpp", "emu_bwd_256", ("EMU_BWD256",)),
-            "persist64": (["bwd_persist_kernel.cuh", "bwd_kernel.cuh", "persist_sched.cuh"], "emu_bwd_main.cpp",
-                          "emu_bwd_persist_64", ("EMU_BWD_PERSIST", "EMU_D=64")),
-            "persist128": (["bwd_persist_kernel.cuh", "bwd_kernel.cuh", "persist_sched.cuh"], "emu_bwd_main.cpp",
-                           "emu_bwd_persist_128", ("EMU_BWD_PERSIST", "EMU_D=128")),
-            "persist128_eager": (["bwd_persist_kernel.cuh", "bwd_kernel.cuh", "persist_sched.cuh"], "emu_bwd_main.cpp",
-                                 "emu_bwd_persist_128_eager", ("EMU_BWD_PERSIST", "EMU_D=128", "EMU_EAGER_COPIES")),
-            "persist128_eager_mma": (["bwd_persist_kernel.cuh", "bwd_kernel.cuh", "persist_sched.cuh"],
-                                     "emu_bwd_main.cpp", "emu_bwd_persist_128_eager_mma",
-                                     ("EMU_BWD_PERSIST", "EMU_D=128", "EMU_EAGER_MMA")),
+            "128_eager": ("bwd_kernel.cuh", "emu_bwd_main.cpp", "emu_bwd_128_eager", ("EMU_D=128", "EMU_EAGER_COPIES")),
+            "128_eager_mma": ("bwd_kernel.cuh", "emu_bwd_main.cpp", "emu_bwd_128_eager_mma",
+                              ("EMU_D=128", "EMU_EAGER_MMA")),
         })
     except FileNotFoundError:
         pytest.skip("g++ not available")
@@ -67,37 +61,18 @@ def test_bwd_kernels_emulated(emu_bwd, B, H, H_kv, N, d, causal, window):
     _check_bwd_emulated(emu_bwd[d], [], B, H, H_kv, N, d, causal, window)
 
 
-PERSIST_CASES = [
-    # B, H, H_kv, N, d, causal, window, CTAs, item order (0 head-major, 1 cost-major).  Few CTAs,
-    # so that each runs several (K/V head, key tile) items and every ring and barrier goes through
-    # phases across items.
-    (1, 2, 2, 300, 128, True, 0, 1, 0),
-    (1, 2, 2, 300, 128, True, 0, 2, 1),
-    (1, 4, 2, 400, 128, False, 50, 3, 1),
-    (2, 2, 1, 257, 64, True, 3, 2, 0),
-    (1, 1, 1, 600, 64, True, 1, 3, 1),
-    (2, 2, 2, 520, 64, True, 0, 5, 1),
-]
+@pytest.mark.parametrize("B,H,H_kv,N,causal,window", [(1, 2, 2, 300, True, 0), (1, 4, 2, 200, False, 50)])
+def test_bwd_kernel_emulated_eager_copies(emu_bwd, B, H, H_kv, N, causal, window):
+    """fa_bwd_kernel with copies that land as soon as they are issued: a Q, dO (or L, D) load
+    before the MMAs released the buffer would overwrite operands still to be read."""
+    _check_bwd_emulated(emu_bwd["128_eager"], [], B, H, H_kv, N, 128, causal, window)
 
 
-@pytest.mark.parametrize("B,H,H_kv,N,d,causal,window,ctas,order", PERSIST_CASES)
-def test_bwd_persistent_kernel_emulated(emu_bwd, B, H, H_kv, N, d, causal, window, ctas, order):
-    """fa_bwd_persist_kernel (each CTA loops over work items) with the same prep and dQ finalise."""
-    _check_bwd_emulated(emu_bwd[f"persist{d}"], [str(ctas), str(order)], B, H, H_kv, N, d, causal, window)
-
-
-@pytest.mark.parametrize("B,H,H_kv,N,causal,window,ctas,order", [
-    (1, 2, 2, 300, True, 0, 1, 0), (1, 4, 2, 200, False, 50, 3, 1)])
-def test_bwd_persistent_kernel_emulated_eager_copies(emu_bwd, B, H, H_kv, N, causal, window, ctas, order):
-    """The persistent backward with copies that land as soon as they are issued: a K/V, Q or dO
-    load before the MMAs released the buffer would overwrite operands still to be read."""
-    _check_bwd_emulated(emu_bwd["persist128_eager"], [str(ctas), str(order)], B, H, H_kv, N, 128, causal, window)
-
-
-def test_bwd_persistent_kernel_emulated_eager_mma(emu_bwd):
-    """The persistent backward with MMAs that run as soon as they are issued: a dV, dK or dQ
-    product issued before P^T or dS^T is in place reads it too early."""
-    _check_bwd_emulated(emu_bwd["persist128_eager_mma"], ["2", "1"], 1, 4, 2, 200, 128, False, 50)
+@pytest.mark.parametrize("B,H,H_kv,N,causal,window", [(1, 2, 2, 300, True, 0), (1, 4, 2, 200, False, 50)])
+def test_bwd_kernel_emulated_eager_mma(emu_bwd, B, H, H_kv, N, causal, window):
+    """fa_bwd_kernel with MMAs that run as soon as they are issued: a dV, dK or dQ product issued
+    before P^T or dS^T is in place reads it too early."""
+    _check_bwd_emulated(emu_bwd["128_eager_mma"], [], B, H, H_kv, N, 128, causal, window)
 
 
 def _check_bwd_emulated(exe, extra, B, H, H_kv, N, d, causal, window):

@@ -37,17 +37,6 @@ def emu_fwd(tmp_path_factory):
             128: ("fwd_kernel.cuh", "emu_fwd_main.cpp", "emu_fwd_128", ("EMU_D=128",)),
             256: (["fwd256_kernel.cuh", "fwd_kernel.cuh"], "emu_fwd_main.cpp", "emu_fwd_256", ("EMU_FWD256",)),
             "fp8": (["fwd_fp8_kernel.cuh", "fwd_kernel.cuh"], "emu_fwd_main.cpp", "emu_fwd_fp8", ("EMU_FWD_FP8",)),
-            "persist64": (["fwd_persist_kernel.cuh", "fwd_kernel.cuh", "persist_sched.cuh"], "emu_fwd_main.cpp", "emu_fwd_persist_64",
-                          ("EMU_FWD_PERSIST", "EMU_D=64")),
-            "persist128": (["fwd_persist_kernel.cuh", "fwd_kernel.cuh", "persist_sched.cuh"], "emu_fwd_main.cpp", "emu_fwd_persist_128",
-                           ("EMU_FWD_PERSIST", "EMU_D=128")),
-            "persist256": (["fwd256_persist_kernel.cuh", "fwd256_kernel.cuh", "fwd_kernel.cuh", "persist_sched.cuh"],
-                           "emu_fwd_main.cpp", "emu_fwd_persist_256", ("EMU_FWD256", "EMU_FWD256_PERSIST")),
-            "persist128_eager": (["fwd_persist_kernel.cuh", "fwd_kernel.cuh", "persist_sched.cuh"], "emu_fwd_main.cpp",
-                                 "emu_fwd_persist_128_eager", ("EMU_FWD_PERSIST", "EMU_D=128", "EMU_EAGER_COPIES")),
-            "persist128_eager_mma": (["fwd_persist_kernel.cuh", "fwd_kernel.cuh", "persist_sched.cuh"],
-                                     "emu_fwd_main.cpp", "emu_fwd_persist_128_eager_mma",
-                                     ("EMU_FWD_PERSIST", "EMU_D=128", "EMU_EAGER_MMA")),
             "128_eager": ("fwd_kernel.cuh", "emu_fwd_main.cpp", "emu_fwd_128_eager", ("EMU_D=128", "EMU_EAGER_COPIES")),
             "128_eager_mma": ("fwd_kernel.cuh", "emu_fwd_main.cpp", "emu_fwd_128_eager_mma",
                               ("EMU_D=128", "EMU_EAGER_MMA")),
@@ -86,44 +75,6 @@ def test_fwd_kernel_emulated(emu_fwd, B, H, H_kv, N, d, causal, window):
     _check_fwd_emulated(emu_fwd[d], [], B, H, H_kv, N, d, causal, window)
 
 
-PERSIST_CASES = [
-    # B, H, H_kv, N, d, causal, window, CTAs, item order (0 head-major, 1 pair-major).  Few CTAs,
-    # so that each runs several work items (dealt in a snake) and every barrier goes through
-    # phases across items; causal pairs whose second query tile lies past N (no keys for it in
-    # that item) take the o_free handshake without any P V.
-    (1, 2, 2, 300, 128, True, 0, 1, 0),
-    (1, 2, 2, 300, 128, True, 0, 2, 1),
-    (2, 2, 1, 600, 128, False, 0, 3, 0),
-    (1, 4, 2, 520, 128, True, 100, 2, 1),
-    (1, 2, 2, 400, 128, False, 50, 3, 1),
-    (2, 2, 1, 257, 64, True, 3, 2, 0),
-    (1, 1, 1, 1000, 64, True, 1, 3, 1),
-    (2, 3, 3, 700, 64, True, 0, 5, 1),
-    (1, 1, 1, 1, 128, True, 0, 1, 1),        # N = 1: one row, the pair's second tile empty
-    (1, 2, 1, 129, 64, False, 0, 1, 1),      # one row past a tile, one CTA for both heads
-    # head dimension 256 (fa_fwd256_persist_kernel: items are single query tiles)
-    (1, 2, 2, 300, 256, True, 0, 1, 1),
-    (1, 2, 1, 520, 256, True, 100, 3, 1),
-    (1, 4, 2, 400, 256, False, 50, 2, 1),
-    (2, 2, 1, 257, 256, True, 3, 3, 0),
-]
-
-
-@pytest.mark.parametrize("B,H,H_kv,N,d,causal,window,ctas,order", PERSIST_CASES)
-def test_fwd_persistent_kernel_emulated(emu_fwd, B, H, H_kv, N, d, causal, window, ctas, order):
-    """fa_fwd_persist_kernel (the persistent grid: each CTA loops over work items) vs the oracle."""
-    _check_fwd_emulated(emu_fwd[f"persist{d}"], [str(ctas), str(order)], B, H, H_kv, N, d, causal, window)
-
-
-@pytest.mark.parametrize("B,H,H_kv,N,causal,window,ctas,order", [
-    (1, 2, 2, 300, True, 0, 1, 1), (2, 2, 1, 600, False, 0, 3, 0), (1, 4, 2, 520, True, 100, 2, 1)])
-def test_fwd_persistent_kernel_emulated_eager_copies(emu_fwd, B, H, H_kv, N, causal, window, ctas, order):
-    """The persistent forward with TMA copies that land as soon as they are issued (the other legal
-    extreme to landing when waited for): a load into a ring slot or the Q buffer before its
-    consumers released it would overwrite data still to be read."""
-    _check_fwd_emulated(emu_fwd["persist128_eager"], [str(ctas), str(order)], B, H, H_kv, N, 128, causal, window)
-
-
 @pytest.mark.parametrize("B,H,H_kv,N,causal,window", [
     (1, 2, 2, 300, True, 0), (2, 2, 1, 600, False, 0), (1, 4, 2, 520, True, 100), (1, 2, 2, 1000, False, 200)])
 def test_fwd_kernel_emulated_eager_copies(emu_fwd, B, H, H_kv, N, causal, window):
@@ -137,8 +88,6 @@ def test_fwd_kernel_emulated_eager_copies(emu_fwd, B, H, H_kv, N, causal, window
     ("128_eager_mma", 2, 2, 1, 600, 128, False, 0, []),
     ("128_eager_mma", 1, 4, 2, 520, 128, True, 100, []),
     ("64_eager_mma", 1, 2, 2, 1000, 64, False, 200, []),
-    ("persist128_eager_mma", 1, 2, 2, 300, 128, True, 0, ["1", "1"]),
-    ("persist128_eager_mma", 2, 2, 1, 600, 128, False, 0, ["3", "0"]),
     ("256_eager_mma", 1, 2, 2, 300, 256, True, 0, []),
     ("256_eager_mma", 1, 4, 2, 400, 256, False, 50, [])])
 def test_fwd_kernel_emulated_eager_mma(emu_fwd, kind, B, H, H_kv, N, d, causal, window, extra):
@@ -169,12 +118,11 @@ def _check_fwd_emulated(exe, extra, B, H, H_kv, N, d, causal, window):
     assert np.abs(lse - l_ref).max() <= L_MAX_ABS
 
 
-@pytest.mark.parametrize("d,persistent", [(128, False), (256, False), (128, True), (256, True)])
-def test_fwd_kernel_emulated_late_rescales(emu_fwd, d, persistent):
+@pytest.mark.parametrize("d", [128, 256])
+def test_fwd_kernel_emulated_late_rescales(emu_fwd, d):
     """Keys that score ever higher along the sequence make many rows' maxima grow by more than
     2^8 after their first key tile, so the lazy rescale of O runs at later tiles (with the d = 256
-    kernel's two S buffers it must first wait for the previous P V product; the persistent
-    kernel runs both work items on one CTA, in the pair-major order)."""
+    kernel's two S buffers it must first wait for the previous P V product)."""
     import subprocess
     N = 400
     g = torch.Generator().manual_seed(97)
@@ -190,8 +138,7 @@ def test_fwd_kernel_emulated_late_rescales(emu_fwd, d, persistent):
         pre = os.path.join(tmp, "x")
         for name, t in zip("qkv", (q, k, v)):
             t.contiguous().view(torch.int16).numpy().tofile(pre + "." + name)
-        exe, extra = (emu_fwd[f"persist{d}"], ["1", "1"]) if persistent else (emu_fwd[d], [])
-        r = subprocess.run([exe, "1", "1", "1", str(N), "1", "0", repr(scale), pre] + extra,
+        r = subprocess.run([emu_fwd[d], "1", "1", "1", str(N), "1", "0", repr(scale), pre],
                            capture_output=True, text=True, timeout=900)
         assert r.returncode == 0, r.stderr[-4000:]
         o = np.fromfile(pre + ".o", dtype=np.uint16)
