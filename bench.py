@@ -616,10 +616,10 @@ NCU_TRAFFIC = {
                                        "grid_sched.cuh": "64126a5757824c1f991611e9caf4a9229a7cb45c"}},
     # the decode workload (B8 H64 with 8 K/V heads, N_q 1, N_k 32768): both kernels of one step
     "fa_decode_kernel<128,false>+fa_decode_merge_kernel<128>": {
-        "bytes": 1083981824,
-        "sources": {"decode_kernel.cuh": "37262a272745d1c2ddd9eb7bd89f5f55d265e07b",
-                    "decode_ops.cuh": "71a63f81cb1eccd17e2d315ab066de5238a9c0a4",
-                    "sm100.cuh": "765aea2ea7410d534e289cfea85ff6d2b3b159c9"}},
+        "bytes": 1081246720,
+        "sources": {"decode_kernel.cuh": "646085a87009b56663aaf2c8551717c0a3bfd77c",
+                    "decode_ops.cuh": "91d87da9815f4797f928aaebebba6d8d20d1d1c7",
+                    "sm100.cuh": "2ad8f7efc3001a800d5f5280be5d66b6f64da97e"}},
 }
 
 
