@@ -138,7 +138,7 @@ int set_smem(Kernel k, int bytes) {
                                                                                                      : FA_ERR_CUDA;
 }
 
-// tensor maps and parameters of the d = 64 / 128 forward (fwd_kernel.cuh), shared by its two launches
+// tensor maps and parameters of the d = 64 / 128 forward (fwd_kernel.cuh)
 template <int D>
 bool fwd_setup(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv, int N,
                const Strides* st, float scale, int causal, int window, CUtensorMap* tq, CUtensorMap* tk,
@@ -169,14 +169,15 @@ constexpr int fwd_smem_bytes(int struct_bytes) {
 template <int D>
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv, int N,
                const Strides* st, float scale, int causal, int window, cudaStream_t stream) {
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   FwdParams prm;
-  if (!fwd_setup<D>(q, k, v, o, lse, B, H, H_kv, N, st, scale, causal, window, &tq, &tk, &tv, &prm))
+  if (!fwd_setup<D>(q, k, v, o, lse, B, H, H_kv, N, st, scale, causal, window, &tq, &tk, &tv, &prm) ||
+      !make_map_bf16(&to, o, D, N, H, B, st[3], kBlockM))
     return FA_ERR_CUDA;
   const int smem = fwd_smem_bytes(int(sizeof(FwdSmem<D>)));
   if (set_smem(fa_fwd_kernel<D>, smem) != FA_OK) return FA_ERR_CUDA;
   const unsigned grid = unsigned(prm.n_pairs) * unsigned(prm.BH);
-  fa_fwd_kernel<D><<<grid, kFwdThreads, smem, stream>>>(tq, tk, tv, prm);
+  fa_fwd_kernel<D><<<grid, kFwdThreads, smem, stream>>>(tq, tk, tv, to, prm);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

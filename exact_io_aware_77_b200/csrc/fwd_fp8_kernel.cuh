@@ -208,43 +208,62 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const int kv0 = t * kBlockN;
       if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.s_full[w]), k & 1, abort, lim))) return false;
       tc_fence_after();
-      float sv[kBlockN];
-      {
+      // Two passes over the S columns in TMEM, as in fa_fwd_kernel: the row max from all 128,
+      // then the exponentials 32 columns at a time (the next chunk's load in flight), so that the
+      // exponentials' temporaries fit next to one chunk of scores rather than all 128.
+      int a = 0, b = kBlockN;   // allowed columns of this row in the tile: [a, b)
+      if constexpr (decltype(masked)::value) {
+        const int hi = prm.causal ? min(qi, prm.N - 1)
+                                  : (prm.window > 0 ? min(qi + prm.window - 1, prm.N - 1) : prm.N - 1);
+        const int lo = prm.window > 0 ? qi - prm.window + 1 : 0;
+        a = lo - kv0;
+        b = hi - kv0 + 1;
+      }
+      float mx;
+      if constexpr (!decltype(masked)::value) {
         uint32_t r[kBlockN];
 #pragma unroll
         for (int ch = 0; ch < kBlockN / 32; ++ch) tmem_ld32_async(s_col + ch * 32, r + ch * 32);
         tmem_ld_wait();
         reg_fence<kBlockN>(r);
+        float mx16[16];
 #pragma unroll
-        for (int j = 0; j < kBlockN; ++j) sv[j] = __uint_as_float(r[j]);
-      }
-      if constexpr (decltype(masked)::value) {
-        const int hi = prm.causal ? min(qi, prm.N - 1)
-                                  : (prm.window > 0 ? min(qi + prm.window - 1, prm.N - 1) : prm.N - 1);
-        const int lo = prm.window > 0 ? qi - prm.window + 1 : 0;
-        const int a = lo - kv0, b = hi - kv0 + 1;
+        for (int i = 0; i < 16; ++i) mx16[i] = __uint_as_float(r[i]);
 #pragma unroll
-        for (int wd = 0; wd < kBlockN / 32; ++wd) {
-          const int aw = min(max(a - 32 * wd, 0), 32), bw = min(max(b - 32 * wd, 0), 32);
-          const uint32_t below_b = bw >= 32 ? 0xffffffffu : ((1u << bw) - 1u);
-          const uint32_t below_a = aw >= 32 ? 0xffffffffu : ((1u << aw) - 1u);
-          const uint32_t bits = below_b & ~below_a;
+        for (int j = 16; j < kBlockN; j += 16)
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (!((bits >> j) & 1u)) sv[32 * wd + j] = -INFINITY;
+          for (int i = 0; i < 16; ++i) mx16[i] = fmaxf(mx16[i], __uint_as_float(r[j + i]));
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx16[i] = fmaxf(mx16[i], mx16[i + 8]);
+        mx = max3f(max3f(mx16[0], mx16[1], mx16[2]), max3f(mx16[3], mx16[4], mx16[5]), fmaxf(mx16[6], mx16[7]));
+      } else {
+        // the masked form takes the max 64 columns at a time (its masking temporaries would
+        // not fit next to all 128 scores)
+        float mx16[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) mx16[i] = -INFINITY;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t r[64];
+          tmem_ld32_async(s_col + half * 64, r);
+          tmem_ld32_async(s_col + half * 64 + 32, r + 32);
+          tmem_ld_wait();
+          reg_fence<64>(r);
+#pragma unroll
+          for (int wd = 0; wd < 2; ++wd) {
+            const int aw = min(max(a - 32 * (2 * half + wd), 0), 32), bw = min(max(b - 32 * (2 * half + wd), 0), 32);
+            const uint32_t below_b = bw >= 32 ? 0xffffffffu : ((1u << bw) - 1u);
+            const uint32_t below_a = aw >= 32 ? 0xffffffffu : ((1u << aw) - 1u);
+            const uint32_t bits = below_b & ~below_a;   // allowed columns 32 (2 half + wd) + j
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              mx16[j & 15] = fmaxf(mx16[j & 15], ((bits >> j) & 1u) ? __uint_as_float(r[32 * wd + j]) : -INFINITY);
+          }
         }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx16[i] = fmaxf(mx16[i], mx16[i + 8]);
+        mx = max3f(max3f(mx16[0], mx16[1], mx16[2]), max3f(mx16[3], mx16[4], mx16[5]), fmaxf(mx16[6], mx16[7]));
       }
-      float mx16[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) mx16[i] = sv[i];
-#pragma unroll
-      for (int j = 16; j < kBlockN; j += 16)
-#pragma unroll
-        for (int i = 0; i < 16; ++i) mx16[i] = fmaxf(mx16[i], sv[j + i]);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mx16[i] = fmaxf(mx16[i], mx16[i + 8]);
-      const float mx = max3f(max3f(mx16[0], mx16[1], mx16[2]), max3f(mx16[3], mx16[4], mx16[5]),
-                             fmaxf(mx16[6], mx16[7]));
       const float m_cand = fmaxf(m, mx * c);
       const bool grow = m_cand > m + kRescaleThreshold;
       const float m_new = grow ? m_cand : m;
@@ -252,32 +271,62 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
       const uint64_t c2 = f2(c, c), nm2 = f2(-m_use, -m_use);
       uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-      // P as E4M3 codes into this row of the P tile: 16-byte chunk j (keys 16j ..) at j ^ (row % 8)
+      // one 32-column chunk: P as E4M3 codes into this row of the P tile, 16-byte chunk j (keys
+      // 16 j ..) at j ^ (row % 8)
+      auto exp_chunk = [&](int ch, const uint32_t* cur) {
+        float sv[32];
 #pragma unroll
-      for (int ch = 0; ch < kBlockN / 16; ++ch) {
-        uint32_t words[4];
+        for (int j = 0; j < 32; ++j) sv[j] = __uint_as_float(cur[j]);
+        if constexpr (decltype(masked)::value) {
+          const int aw = a - 32 * ch, bw = b - 32 * ch;   // allowed columns j of the chunk: [aw, bw)
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          uint32_t codes = 0;
-#pragma unroll
-          for (int hp = 0; hp < 2; ++hp) {
-            const int j = ch * 16 + q4 * 4 + hp * 2;
-            const uint64_t x = f2_fma(f2(sv[j], sv[j + 1]), c2, nm2);
-            float p0, p1;
-            if (((j >> 1) & 15) < kEmuPairs) {
-              exp2_poly_x2(x, p0, p1);
-            } else {
-              float x0, x1;
-              f2_split(x, x0, x1);
-              p0 = ex2_approx(x0);
-              p1 = ex2_approx(x1);
-            }
-            acc[(j >> 1) & 3] = f2_add(acc[(j >> 1) & 3], f2(p0, p1));
-            codes |= f32x2_to_e4m3x2(p0, p1) << (16 * hp);
-          }
-          words[q4] = codes;
+          for (int j = 0; j < 32; ++j)
+            if (j < aw || j >= bw) sv[j] = -INFINITY;
         }
-        st_shared_v4(p_row + uint32_t((ch ^ (row & 7)) * 16), words[0], words[1], words[2], words[3]);
+#pragma unroll
+        for (int h16 = 0; h16 < 2; ++h16) {
+          uint32_t words[4];
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint32_t codes = 0;
+#pragma unroll
+            for (int hp = 0; hp < 2; ++hp) {
+              const int j = h16 * 16 + q4 * 4 + hp * 2;   // column in the chunk; pair jp = j / 2
+              const uint64_t x = f2_fma(f2(sv[j], sv[j + 1]), c2, nm2);
+              float p0, p1;
+              if ((j >> 1) < kEmuPairs) {
+                exp2_poly_x2(x, p0, p1);
+              } else {
+                float x0, x1;
+                f2_split(x, x0, x1);
+                p0 = ex2_approx(x0);
+                p1 = ex2_approx(x1);
+              }
+              acc[(j >> 1) & 3] = f2_add(acc[(j >> 1) & 3], f2(p0, p1));
+              codes |= f32x2_to_e4m3x2(p0, p1) << (16 * hp);
+            }
+            words[q4] = codes;
+          }
+          const int c16 = 2 * ch + h16;
+          st_shared_v4(p_row + uint32_t((c16 ^ (row & 7)) * 16), words[0], words[1], words[2], words[3]);
+        }
+      };
+      {
+        uint32_t ra[32], rb[32];
+        tmem_ld32_async(s_col, ra);
+        tmem_ld_wait();
+        reg_fence<32>(ra);
+#pragma unroll
+        for (int ch = 0; ch < kBlockN / 32; ++ch) {
+          uint32_t* cur = (ch & 1) ? rb : ra;
+          uint32_t* nxt = (ch & 1) ? ra : rb;
+          if (ch + 1 < kBlockN / 32) tmem_ld32_async(s_col + (ch + 1) * 32, nxt);
+          exp_chunk(ch, cur);
+          if (ch + 1 < kBlockN / 32) {
+            tmem_ld_wait();
+            reg_fence<32>(nxt);
+          }
+        }
       }
       float sum;
       {

@@ -75,6 +75,7 @@ struct FwdSmem {
   alignas(8) uint64_t q_full;
   uint64_t slot_full[kSlots], slot_empty[kSlots];
   uint64_t s_full[kQTiles], p_full[kQTiles], o_final[kQTiles];
+  uint64_t o_staged[kQTiles];   // a tile's 128 rows of O / l are in its Q buffer
   uint64_t mma_drain;
   uint32_t tmem_base;
   int abort;
@@ -98,7 +99,8 @@ __device__ __forceinline__ void kv_tile_range(int q0, int N, int causal, int win
 template <int D>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const FwdParams prm) {
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                  const FwdParams prm) {
   using Smem = FwdSmem<D>;
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -132,6 +134,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(smem_u32(&sm.s_full[w]), 1);
       mbar_init(smem_u32(&sm.p_full[w]), kBlockM);
       mbar_init(smem_u32(&sm.o_final[w]), 1);
+      mbar_init(smem_u32(&sm.o_staged[w]), kBlockM);
     }
     mbar_init(smem_u32(&sm.mma_drain), 1);
     fence_mbar_init();
@@ -141,6 +144,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_o);
     }
     __syncwarp();
     tmem_alloc(smem_u32(&sm.tmem_base), kTmemCols);
@@ -442,8 +446,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     if (ok && te > tb && __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.o_final[w]), 0, abort, lim))) {
       tc_fence_after();
       const float inv_l = 1.f / l;
-      const bool in_range = qi < prm.N;
-      __nv_bfloat16* orow = prm.o + prm.o_st.at(b_idx, h_q, in_range ? qi : 0);
+      // O / l as bf16, staged in this tile's Q buffer (every MMA has completed, so Q is read no
+      // more) in the layout a TMA load of the tile leaves there: 64-column chunks of 16 KB,
+      // 128-byte rows, 16-byte piece c of row r at c ^ (r % 8).  One thread then writes the tile
+      // with TMA tensor stores, which skip the rows past N.
+      const uint32_t stage = smem_u32(sm.q[w]);
 #pragma unroll
       for (int ch = 0; ch < D / 32; ++ch) {
         uint32_t r[32];
@@ -452,13 +459,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
         for (int j = 0; j < 16; ++j)
           wv[j] = pack_bf16x2(__uint_as_float(r[2 * j]) * inv_l, __uint_as_float(r[2 * j + 1]) * inv_l);
-        if (in_range) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+        const uint32_t row_addr = stage + (ch >> 1) * 16384 + row * 128;
 #pragma unroll
-          for (int j = 0; j < 4; ++j) dst[j] = make_uint4(wv[4 * j], wv[4 * j + 1], wv[4 * j + 2], wv[4 * j + 3]);
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t c16 = (ch & 1) * 4 + j;
+          st_shared_v4(row_addr + ((c16 ^ (row & 7)) << 4), wv[4 * j], wv[4 * j + 1], wv[4 * j + 2], wv[4 * j + 3]);
         }
       }
-      if (in_range) prm.lse[size_t(bh) * prm.N + qi] = (m + lg2_approx(l)) * 0.69314718055994531f;
+      fence_proxy_async_smem();   // the tensor store reads the rows through the async proxy
+      mbar_arrive(smem_u32(&sm.o_staged[w]));
+      if (qi < prm.N) prm.lse[size_t(bh) * prm.N + qi] = (m + lg2_approx(l)) * 0.69314718055994531f;
+      if (row == 0 && mbar_wait(smem_u32(&sm.o_staged[w]), 0, abort, lim)) {
+#pragma unroll
+        for (int c = 0; c < Smem::kChunks; ++c) tma_store_rows(&tm_o, stage + c * 16384, c * 64, qw0, h_q, b_idx);
+        bulk_commit_group();
+        bulk_wait_group<0>();   // the rows are read (and written) before the CTA's shared memory is released
+      }
     }
   }
 

@@ -121,6 +121,16 @@ __device__ __forceinline__ void tma_reduce_add_rows(const CUtensorMap* map, uint
       "r"(src), "r"(x), "r"(row), "r"(head), "r"(batch)
       : "memory");
 }
+// 4-D tiled store: the shared-memory box at `src` (laid out as a load of the same map would
+// leave it) into global memory at the box's coordinates; rows outside the tensor are skipped.
+// Tracked by this thread's bulk async-groups, as tma_reduce_add_rows.
+__device__ __forceinline__ void tma_store_rows(const CUtensorMap* map, uint32_t src, int x, int row, int head,
+                                               int batch) {
+  asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(x), "r"(row), "r"(head), "r"(batch)
+               : "memory");
+}
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void bulk_wait_group_read() {

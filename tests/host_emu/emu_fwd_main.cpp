@@ -159,7 +159,8 @@ int main(int argc, char** argv) {
 #if defined(EMU_FWD256)
   emu_launch(grid, k256Threads, sizeof(fa::smem_raw), [&] { fa_fwd256_kernel(tq, tk, tv, prm); }, fa::smem_raw);
 #else
-  emu_launch(grid, kFwdThreads, sizeof(fa::smem_raw), [&] { fa_fwd_kernel<D>(tq, tk, tv, prm); }, fa::smem_raw);
+  const CUtensorMap to = make_map(o.data(), D, N, H, B, box_q);
+  emu_launch(grid, kFwdThreads, sizeof(fa::smem_raw), [&] { fa_fwd_kernel<D>(tq, tk, tv, to, prm); }, fa::smem_raw);
 #endif
   if (g_status != 0) { std::fprintf(stderr, "device status %d\n", g_status); return 3; }
   write_file(prefix + ".o", o);

@@ -392,6 +392,31 @@ inline void tma_reduce_add_rows(const CUtensorMap* map, uint32_t src, int x, int
     g_blk = saved;
   });
 }
+// cp.async.bulk.tensor (shared -> global) tiled store: like the reduction above, it joins the
+// thread's open bulk group and runs (reads the box, writes the rows inside the tensor) only when
+// a bulk wait retires the group.
+inline void tma_store_rows(const CUtensorMap* map, uint32_t src, int x, int row, int head, int batch) {
+  if ((x * int(map->esize)) % 16) { std::fprintf(stderr, "TMA x coordinate not 16-byte aligned\n"); std::abort(); }
+  if (map->box_x * map->esize != 128) { std::fprintf(stderr, "TMA box row is not 128 bytes\n"); std::abort(); }
+  if (src % 128) { std::fprintf(stderr, "TMA store source not 128-byte aligned\n"); std::abort(); }
+  if (x < 0 || row < 0 || head < 0 || batch < 0) { std::fprintf(stderr, "TMA store at a negative coordinate\n"); std::abort(); }
+  smem_at(src, size_t(map->box_rows) * 128);
+  const CUtensorMap m = *map;
+  BlockCtx* blk = g_blk;
+  t_bulk_open.push_back([=] {
+    BlockCtx* saved = g_blk;
+    g_blk = blk;
+    for (uint32_t r = 0; r < m.box_rows; ++r)
+      for (uint32_t c = 0; c < m.box_x; ++c) {
+        const uint64_t gx = uint64_t(x) + c, gr = uint64_t(row) + r;
+        if (gx >= m.dims[0] || gr >= m.dims[1] || uint64_t(head) >= m.dims[2] || uint64_t(batch) >= m.dims[3]) continue;
+        std::memcpy(const_cast<unsigned char*>(m.base) + uint64_t(batch) * m.strides[2] + uint64_t(head) * m.strides[1] +
+                        gr * m.strides[0] + gx * m.esize,
+                    smem_at(sw128(src + r * 128 + c * m.esize), m.esize), m.esize);
+      }
+    g_blk = saved;
+  });
+}
 inline void bulk_commit_group() {
   t_bulk_groups.push_back(std::move(t_bulk_open));
   t_bulk_open.clear();
@@ -409,7 +434,7 @@ inline void bulk_wait_group() {
 }
 inline void bulk_exit_check() {
   if (!t_bulk_open.empty() || !t_bulk_groups.empty()) {
-    std::fprintf(stderr, "thread %u of CTA %u ends with bulk reductions in flight\n", threadIdx.x, blockIdx.x);
+    std::fprintf(stderr, "thread %u of CTA %u ends with bulk operations (tensor reductions or stores) in flight\n", threadIdx.x, blockIdx.x);
     std::abort();
   }
 }
