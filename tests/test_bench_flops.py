@@ -40,3 +40,30 @@ def test_decode_bytes():
         2 * 8 * 64 * 128 * 2 + 2 * 8 * 8 * 32768 * 128 + 8 * 64 * 4
     # a causal window reads only the keys the window keeps
     assert bench.decode_bytes(1, 1, 1, 1, 10000, 64, True, 100) == 2 * 64 * 2 + 2 * 100 * 64 * 2 + 4
+
+
+def _roof(achieved):
+    return {"bound": "tensor", "kernel": "k", "achieved": achieved, "peak": 1636.3, "unit": "TFLOP/s",
+            "frac": round(achieved / 1636.3, 4), "peak_source": "measured burst bf16 (MEASURED_PEAKS.json)"}
+
+
+def test_regime_fields_burst_and_sustained():
+    """A timed region under 1 s is judged against the burst peak, a longer one against the
+    sustained peak; both fractions and the clock-normalised kernel time are reported."""
+    peaks = {"bf16_tflops": 1636.3, "bf16_tflops_sustained": 1375.0}
+    clocks = {"sm_mhz": 1732.0, "sm_max_mhz": 1965.0, "samples": 13}
+    r = _roof(900.0)
+    cn = bench.regime_fields(r, clocks, 23.0, 0.3, peaks)
+    assert r["regime"] == "burst" and r["peak"] == 1636.3 and r["frac"] == round(900.0 / 1636.3, 4)
+    assert r["frac_of_sustained_peak"] == round(900.0 / 1375.0, 4)
+    assert cn["kernel_ms_at_max_clock"] == round(0.3 * 1732.0 / 1965.0, 5)
+    assert cn["achieved_at_max_clock"] == round(900.0 * 1965.0 / 1732.0, 1)
+    assert cn["samples_in_window"] == 13
+    r = _roof(900.0)
+    bench.regime_fields(r, clocks, 1230.0, 0.3, peaks)
+    assert r["regime"] == "sustained" and r["peak"] == 1375.0 and r["frac"] == round(900.0 / 1375.0, 4)
+    assert "sustained" in r["peak_source"]
+    # no clock samples: no clock-normalised figures, the regime still set
+    r = _roof(900.0)
+    assert bench.regime_fields(r, {"sm_mhz": None, "sm_max_mhz": None}, 10.0, 0.3, peaks) is None
+    assert r["regime"] == "burst"
