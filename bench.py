@@ -606,20 +606,20 @@ def measure_e2e(fa, torch, wl, dev, stream, q_h, k_h, v_h, do_h, has_bwd, steps,
 # the workload the bench line times (the causal B2 H32 N4096 d128 one, or the decode one), keyed by kernel, with the SHA-1 of the kernel's sources
 # when the counters were taken (profiles/ holds the summaries).  A changed source reports null.
 NCU_TRAFFIC = {
-    "fa_fwd_kernel<128>": {"bytes": 247744512,
-                           "sources": {"fwd_kernel.cuh": "e8641ce82d6dbdb61b9ba009f4929267d8e3e6ee",
-                                       "sm100.cuh": "2ad8f7efc3001a800d5f5280be5d66b6f64da97e",
-                                       "grid_sched.cuh": "64126a5757824c1f991611e9caf4a9229a7cb45c"}},
-    "fa_bwd_kernel<128>": {"bytes": 625011456,
-                           "sources": {"bwd_kernel.cuh": "74efb053dd65812bcd3bb44ae6532ddb950801ad",
-                                       "sm100.cuh": "2ad8f7efc3001a800d5f5280be5d66b6f64da97e",
-                                       "grid_sched.cuh": "64126a5757824c1f991611e9caf4a9229a7cb45c"}},
+    "fa_fwd_kernel<128>": {"bytes": 248753408,
+                           "sources": {"fwd_kernel.cuh": "f6bba43298dc9bfbf7d8590d67a3b7b0fe8aa3a7",
+                                       "sm100.cuh": "b39376276083f6773b526da3ba0d61e0d1b7673d",
+                                       "grid_sched.cuh": "d69cc1d77285fb320f5966be935efafc0d37f593"}},
+    "fa_bwd_kernel<128>": {"bytes": 623175680,
+                           "sources": {"bwd_kernel.cuh": "759b5ce5821fe90e981aca85c92c2ab7b4693723",
+                                       "sm100.cuh": "b39376276083f6773b526da3ba0d61e0d1b7673d",
+                                       "grid_sched.cuh": "d69cc1d77285fb320f5966be935efafc0d37f593"}},
     # the decode workload (B8 H64 with 8 K/V heads, N_q 1, N_k 32768): both kernels of one step
     "fa_decode_kernel<128,false>+fa_decode_merge_kernel<128>": {
-        "bytes": 1081246720,
+        "bytes": 1081105152,
         "sources": {"decode_kernel.cuh": "646085a87009b56663aaf2c8551717c0a3bfd77c",
                     "decode_ops.cuh": "91d87da9815f4797f928aaebebba6d8d20d1d1c7",
-                    "sm100.cuh": "2ad8f7efc3001a800d5f5280be5d66b6f64da97e"}},
+                    "sm100.cuh": "b39376276083f6773b526da3ba0d61e0d1b7673d"}},
 }
 
 
