@@ -3,20 +3,23 @@
 //
 // At d = 256 the dK and dV accumulators of a 128-key tile alone fill the 512 TMEM columns, and
 // full-width 128-key K and V tiles take 128 KB of shared memory.  Here each CTA owns a 64-key
-// tile of one K/V head and one half c of the head dimension (columns 128c .. 128c + 127), and
-// loops over the 128-row query tiles (of every query head that reads the K/V head):
+// tile of one K/V head and loops over the 128-row query tiles (of every query head that reads
+// the K/V head):
 //   S  = Q K^T,  dP = dO V^T             full d, M = 128 queries, N = 64 keys
 //   P  = exp2(S c - L log2 e) (masked),  dS = P o (dP - D)           compute warps
-//   dV^T_c += dO_c^T P,  dK^T_c += Q_c^T dS   M = 128 head-dim columns, N = 64 keys, K = 128
+//   dV^T_c += dO_c^T P,  dK^T_c += Q_c^T dS   for both head-dim halves c (columns 128c ..),
+//                                        M = 128 head-dim columns, N = 64 keys, K = 128
 //                                        queries: dO and Q as MN-major A operands (the same
 //                                        tiles the first products read K-major), P and dS
 //                                        staged in shared memory as MN-major B operands
 //   dQ_c = dS K_c                        M = 128 queries, N = 128, K = 64 keys; K_c MN-major;
-//                                        added into the fp32 accumulator with vector reductions
-// so S and dP are computed by both CTAs of a tile (1.4x the products of one full-width pass).
+//                                        one half after the other in the same 128 TMEM columns,
+//                                        each added into the fp32 accumulator with vector
+//                                        reductions before the next overwrites it.
 // Roles (192 threads): warps 0-3 compute (thread t of warp w owns TMEM lane 32w + t: a query
-// row of S, dP and dQ, and at the end a head-dim column of dV^T and dK^T), warp 4 TMA, warp 5
-// MMA.  TMEM columns: S [0, 64), dP [64, 128), dV^T [128, 192), dK^T [192, 256), dQ [256, 384).
+// row of S, dP and dQ, and at the end a head-dim column of each half of dV^T and dK^T), warp 4
+// TMA, warp 5 MMA.  TMEM columns: S [0, 64), dP [64, 128), dV^T_0 [128, 192), dV^T_1 [192, 256),
+// dK^T_0 [256, 320), dK^T_1 [320, 384), dQ_c [384, 512).
 // One stage of Q and dO: the next query tile loads once the MMAs of this one are done.
 #pragma once
 
@@ -31,7 +34,7 @@ constexpr int kB256Rows = 128;    // query rows per iteration
 constexpr int kB256Threads = 192;
 constexpr int kB256WarpTma = 4;
 constexpr int kB256WarpMma = 5;
-constexpr uint32_t kT256S = 0, kT256dP = 64, kT256dV = 128, kT256dK = 192, kT256dQ = 256;
+constexpr uint32_t kT256S = 0, kT256dP = 64, kT256dV = 128, kT256dK = 256, kT256dQ = 384;   // dV^T_c, dK^T_c at + 64c
 
 struct Bwd256Smem {
   static constexpr uint32_t kQChunk = kB256Rows * 128;   // 64 head-dim columns of 128 rows
@@ -60,8 +63,7 @@ __device__ __forceinline__ void q_tile_range256(int kv0, int N, int causal, int 
   }
 }
 
-// One CTA per (K/V head, 64-key tile, head-dim half): blockIdx.x = item * 2 + c, with the
-// (K/V head, tile) items in grid_item's chunked order.
+// One CTA per (K/V head, 64-key tile), in grid_item's chunked order.
 // prm.n_kv_tiles counts 64-key tiles here.
 __global__ void __launch_bounds__(kB256Threads, 1)
     fa_bwd256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -76,9 +78,8 @@ __global__ void __launch_bounds__(kB256Threads, 1)
   }
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int dhalf = int(blockIdx.x & 1);   // head-dim half: columns 128 dhalf ..
   int bh, tile;   // K/V head (b * H_kv + h_kv) and key tile
-  grid_item(int(blockIdx.x >> 1), prm.BH / prm.group, prm.n_kv_tiles, kBwdChunkHeads, bh, tile);
+  grid_item(int(blockIdx.x), prm.BH / prm.group, prm.n_kv_tiles, kBwdChunkHeads, bh, tile);
   const int b_idx = bh / prm.H_kv, h_kv = bh % prm.H_kv;
   const int bh_q0 = b_idx * prm.H + h_kv * prm.group;       // first query head of the group
   const int kv0 = tile * kB256Keys;
@@ -98,8 +99,8 @@ __global__ void __launch_bounds__(kB256Threads, 1)
     mbar_init(smem_u32(&sm.q_empty), 1);
     mbar_init(smem_u32(&sm.s_full), 1);
     mbar_init(smem_u32(&sm.p_full), kB256Rows);
-    mbar_init(smem_u32(&sm.dq_full), 1);
-    mbar_init(smem_u32(&sm.dq_free), kB256Rows);
+    mbar_init(smem_u32(&sm.dq_full), 1);      // completes twice per query tile (dQ_0, dQ_1)
+    mbar_init(smem_u32(&sm.dq_free), kB256Rows);   // likewise (each half read out)
     mbar_init(smem_u32(&sm.mma_final), 1);
     mbar_init(smem_u32(&sm.mma_drain), 1);
     fence_mbar_init();
@@ -161,11 +162,11 @@ __global__ void __launch_bounds__(kB256Threads, 1)
     const uint64_t dk_k = sw128_desc(smem_u32(sm.k), 16, 1024);
     const uint64_t dv_k = sw128_desc(smem_u32(sm.v), 16, 1024);
     const uint64_t dds_k = sw128_desc(smem_u32(sm.ds), 16, 1024);
-    // MN-major views of this CTA's head-dim half: 64 columns per 128-byte row, one row per
-    // query (or key), 8-row atoms 1024 bytes apart, the next 64 columns one chunk (LBO) further
-    const uint64_t dq_t = sw128_desc(smem_u32(sm.q) + 2 * dhalf * Smem::kQChunk, Smem::kQChunk, 1024);
-    const uint64_t ddo_t = sw128_desc(smem_u32(sm.dout) + 2 * dhalf * Smem::kQChunk, Smem::kQChunk, 1024);
-    const uint64_t dk_t = sw128_desc(smem_u32(sm.k) + 2 * dhalf * Smem::kKChunk, Smem::kKChunk, 1024);
+    // MN-major views of head-dim half c: 64 columns per 128-byte row, one row per query (or
+    // key), 8-row atoms 1024 bytes apart, the next 64 columns one chunk (LBO) further
+    auto dq_t = [&](int c) { return sw128_desc(smem_u32(sm.q) + 2 * c * Smem::kQChunk, Smem::kQChunk, 1024); };
+    auto ddo_t = [&](int c) { return sw128_desc(smem_u32(sm.dout) + 2 * c * Smem::kQChunk, Smem::kQChunk, 1024); };
+    auto dk_t = [&](int c) { return sw128_desc(smem_u32(sm.k) + 2 * c * Smem::kKChunk, Smem::kKChunk, 1024); };
     const uint64_t dp_t = sw128_desc(smem_u32(sm.p), Smem::kQChunk, 1024);
     const uint64_t dds_t = sw128_desc(smem_u32(sm.ds), Smem::kQChunk, 1024);
     bool ok = n_it > 0 && wait(smem_u32(&sm.kv_full), 0);
@@ -182,20 +183,38 @@ __global__ void __launch_bounds__(kB256Threads, 1)
       }
       mma_commit_w(smem_u32(&sm.s_full));
       if (!wait(smem_u32(&sm.p_full), it & 1)) break;
-      if (it > 0 && !wait(smem_u32(&sm.dq_free), (it - 1) & 1)) break;
       tc_fence_after();
-      // dV^T += dO_c^T P and dK^T += Q_c^T dS: 16 queries per k-step = 16 rows of 128 bytes
+      // dV^T_c += dO_c^T P and dK^T_c += Q_c^T dS for both halves: 16 queries per k-step = 16
+      // rows of 128 bytes
 #pragma unroll
-      for (int kk = 0; kk < kB256Rows / 16; ++kk) {
-        const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-        mma_bf16_ss_w(tmem + kT256dV, desc_advance(ddo_t, kk * 2048), desc_advance(dp_t, kk * 2048), idesc_t, acc);
-        mma_bf16_ss_w(tmem + kT256dK, desc_advance(dq_t, kk * 2048), desc_advance(dds_t, kk * 2048), idesc_t, acc);
+      for (int c = 0; c < 2; ++c) {
+        const uint64_t dot = ddo_t(c), qt = dq_t(c);
+#pragma unroll
+        for (int kk = 0; kk < kB256Rows / 16; ++kk) {
+          const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
+          mma_bf16_ss_w(tmem + kT256dV + 64 * c, desc_advance(dot, kk * 2048), desc_advance(dp_t, kk * 2048),
+                        idesc_t, acc);
+          mma_bf16_ss_w(tmem + kT256dK + 64 * c, desc_advance(qt, kk * 2048), desc_advance(dds_t, kk * 2048),
+                        idesc_t, acc);
+        }
       }
-      // dQ_c = dS K_c: 16 keys per k-step (32 bytes along dS's rows, 16 rows of K)
+      // dQ_c = dS K_c: 16 keys per k-step (32 bytes along dS's rows, 16 rows of K).  The two
+      // halves share the dQ columns: each waits until the previous one has been read out
+      // (dq_free completes twice per query tile: the readouts of dQ_0 and dQ_1)
 #pragma unroll
-      for (int kk = 0; kk < kB256Keys / 16; ++kk)
-        mma_bf16_ss_w(tmem + kT256dQ, desc_advance(dds_k, kk * 32), desc_advance(dk_t, kk * 2048), idesc_q, kk > 0);
-      mma_commit_w(smem_u32(&sm.dq_full));
+      for (int c = 0; c < 2; ++c) {
+        if ((it > 0 || c > 0) && !wait(smem_u32(&sm.dq_free), c == 0 ? 1u : 0u)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t kt = dk_t(c);
+#pragma unroll
+        for (int kk = 0; kk < kB256Keys / 16; ++kk)
+          mma_bf16_ss_w(tmem + kT256dQ, desc_advance(dds_k, kk * 32), desc_advance(kt, kk * 2048), idesc_q, kk > 0);
+        mma_commit_w(smem_u32(&sm.dq_full));
+      }
+      if (!ok) break;
       mma_commit_w(smem_u32(&sm.q_empty));
     }
     mma_commit_w(smem_u32(&sm.mma_final));
@@ -203,7 +222,7 @@ __global__ void __launch_bounds__(kB256Threads, 1)
     mbar_wait_drain(smem_u32(&sm.mma_drain), 0, lim);
   } else {
     // ------------------------------------------------------------------ compute warps
-    const int row = threadIdx.x;   // TMEM lane: a query row of S, dP, dQ; a head-dim column of dV^T, dK^T
+    const int row = threadIdx.x;   // TMEM lane: a query row of S, dP, dQ; head-dim column row (+ 128) of dV^T, dK^T
     const uint32_t lane_base = uint32_t(warp * 32) << 16;
     const float c = prm.scale_log2;
     bool ok = true;
@@ -257,44 +276,52 @@ __global__ void __launch_bounds__(kB256Threads, 1)
       fence_proxy_async_smem();   // the MMAs read P and dS through the async proxy
       tc_fence_before();
       mbar_arrive(smem_u32(&sm.p_full));
-      // dQ_c rows into the fp32 accumulator
-      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.dq_full), it & 1, abort, lim));
-      if (!ok) break;
-      tc_fence_after();
-      float* acc = prm.dq_acc + (size_t(hq) * prm.Np + qi) * D + dhalf * 128;
+      // dQ_0, then dQ_1 (the same TMEM columns, one after the other): this row's 128 columns of
+      // each into the fp32 accumulator
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t r[32];
-        tmem_ld32(tmem + lane_base + kT256dQ + ch * 32, r);
+      for (int c = 0; c < 2 && ok; ++c) {
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.dq_full), uint32_t(c), abort, lim));
+        if (!ok) break;
+        tc_fence_after();
+        float* acc = prm.dq_acc + (size_t(hq) * prm.Np + qi) * D + c * 128;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) red_add_v4(acc + ch * 32 + 4 * j, make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]));
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t r[32];
+          tmem_ld32(tmem + lane_base + kT256dQ + ch * 32, r);
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            red_add_v4(acc + ch * 32 + 4 * j, make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]));
+        }
+        tc_fence_before();
+        mbar_arrive(smem_u32(&sm.dq_free));
       }
-      tc_fence_before();
-      mbar_arrive(smem_u32(&sm.dq_free));
     }
-    // dV and dK of this tile's keys, head-dim column 128 * dhalf + row
+    // dV and dK of this tile's keys, head-dim columns row and 128 + row
     if (ok && __all_sync(0xffffffffu, n_it == 0 || mbar_wait(smem_u32(&sm.mma_final), 0, abort, lim))) {
       tc_fence_after();
-      uint32_t vr[kB256Keys], kr[kB256Keys];
-      if (n_it > 0) {
-        tmem_ld32_async(tmem + lane_base + kT256dV, vr);
-        tmem_ld32_async(tmem + lane_base + kT256dV + 32, vr + 32);
-        tmem_ld32_async(tmem + lane_base + kT256dK, kr);
-        tmem_ld32_async(tmem + lane_base + kT256dK + 32, kr + 32);
-        tmem_ld_wait();
-        reg_fence<kB256Keys>(vr);
-        reg_fence<kB256Keys>(kr);
-      } else {
 #pragma unroll
-        for (int j = 0; j < kB256Keys; ++j) vr[j] = kr[j] = 0u;
-      }
-      const int col = dhalf * 128 + row;
+      for (int c = 0; c < 2; ++c) {
+        uint32_t vr[kB256Keys], kr[kB256Keys];
+        if (n_it > 0) {
+          tmem_ld32_async(tmem + lane_base + kT256dV + 64 * c, vr);
+          tmem_ld32_async(tmem + lane_base + kT256dV + 64 * c + 32, vr + 32);
+          tmem_ld32_async(tmem + lane_base + kT256dK + 64 * c, kr);
+          tmem_ld32_async(tmem + lane_base + kT256dK + 64 * c + 32, kr + 32);
+          tmem_ld_wait();
+          reg_fence<kB256Keys>(vr);
+          reg_fence<kB256Keys>(kr);
+        } else {
 #pragma unroll
-      for (int j = 0; j < kB256Keys; ++j) {
-        const int key = kv0 + j;
-        if (key < prm.N) {
-          prm.dv[prm.dv_st.at(b_idx, h_kv, key) + col] = __float2bfloat16_rn(__uint_as_float(vr[j]));
-          prm.dk[prm.dk_st.at(b_idx, h_kv, key) + col] = __float2bfloat16_rn(__uint_as_float(kr[j]) * prm.scale);
+          for (int j = 0; j < kB256Keys; ++j) vr[j] = kr[j] = 0u;
+        }
+        const int col = c * 128 + row;
+#pragma unroll
+        for (int j = 0; j < kB256Keys; ++j) {
+          const int key = kv0 + j;
+          if (key < prm.N) {
+            prm.dv[prm.dv_st.at(b_idx, h_kv, key) + col] = __float2bfloat16_rn(__uint_as_float(vr[j]));
+            prm.dk[prm.dk_st.at(b_idx, h_kv, key) + col] = __float2bfloat16_rn(__uint_as_float(kr[j]) * prm.scale);
+          }
         }
       }
     }

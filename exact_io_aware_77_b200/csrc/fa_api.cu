@@ -292,12 +292,12 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   prm.scale = scale;
   prm.wait_limit_ns = g_wait_limit_ns;
   if constexpr (D == 256) {
-    // one CTA per (K/V head, 64-key tile, head-dim half): bwd256_kernel.cuh
+    // one CTA per (K/V head, 64-key tile): bwd256_kernel.cuh
     prm.n_kv_tiles = (N + kB256Keys - 1) / kB256Keys;
     static_assert(sizeof(Bwd256Smem) <= 232448, "d = 256 backward shared memory exceeds 227 KB");
     const int smem = int(sizeof(Bwd256Smem));
     if (set_smem(fa_bwd256_kernel, smem) != FA_OK) return FA_ERR_CUDA;
-    fa_bwd256_kernel<<<unsigned(prm.n_kv_tiles) * unsigned(BH_kv) * 2u, kB256Threads, smem, stream>>>(tq, tk, tv, tdo,
+    fa_bwd256_kernel<<<unsigned(prm.n_kv_tiles) * unsigned(BH_kv), kB256Threads, smem, stream>>>(tq, tk, tv, tdo,
                                                                                                          prm);
   } else {
     static_assert(sizeof(BwdSmem<D>) <= 232448, "backward shared memory exceeds 227 KB");
@@ -529,8 +529,8 @@ static int bwd_impl(const void* q, const void* k, const void* v, const void* o, 
       if (!strides_ok(s8[i])) return FA_ERR_ALIGN;
     }
   const long long BH = (long long)B * H;
-  // grid: one CTA per 128-key tile (d = 256: per 64-key tile and head-dim half)
-  const long long bwd_ctas = d == 256 ? BH * ((N + kB256Keys - 1) / kB256Keys) * 2 : BH * ((N + kBwdKeys - 1) / kBwdKeys);
+  // grid: one CTA per 128-key tile (d = 256: per 64-key tile)
+  const long long bwd_ctas = d == 256 ? BH * ((N + kB256Keys - 1) / kB256Keys) : BH * ((N + kBwdKeys - 1) / kBwdKeys);
   if (bwd_ctas > 0x7fffffffLL || BH * padded_rows(N) > 0x7fffffffLL) return FA_ERR_SHAPE;
   if (!workspace || workspace_bytes < bwd_workspace_bytes(BH, N, d)) return FA_ERR_WORKSPACE;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dout, 16) ||
@@ -673,8 +673,8 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
   int st = check_problem(B, H, N, d, scale, causal, window);
   if (st != FA_OK) return st;
   const long long BH = (long long)B * H;
-  // grid: one CTA per 128-key tile (d = 256: per 64-key tile and head-dim half)
-  const long long bwd_ctas = d == 256 ? BH * ((N + kB256Keys - 1) / kB256Keys) * 2 : BH * ((N + kBwdKeys - 1) / kBwdKeys);
+  // grid: one CTA per 128-key tile (d = 256: per 64-key tile)
+  const long long bwd_ctas = d == 256 ? BH * ((N + kB256Keys - 1) / kB256Keys) : BH * ((N + kBwdKeys - 1) / kBwdKeys);
   if (bwd_ctas > 0x7fffffffLL || BH * padded_rows(N) > 0x7fffffffLL) return FA_ERR_SHAPE;
   if (bwd_workspace_bytes(BH, N, d) > kNoAllocScratchBytes) return FA_ERR_NOALLOC_LIMIT;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dout, 16) ||

@@ -127,7 +127,7 @@ int main(int argc, char** argv) {
   prm.scale = scale;
   prm.wait_limit_ns = 60ull * 1000000000ull;
 #ifdef EMU_BWD256
-  emu_launch(unsigned(prm.n_kv_tiles) * unsigned(BH_kv) * 2u, kB256Threads, sizeof(fa::smem_raw),
+  emu_launch(unsigned(prm.n_kv_tiles) * unsigned(BH_kv), kB256Threads, sizeof(fa::smem_raw),
              [&] { fa_bwd256_kernel(tq, tk, tv, tdo, prm); }, fa::smem_raw);
 #else
   emu_launch(unsigned(prm.n_kv_tiles) * unsigned(BH_kv), kBwdThreads, sizeof(fa::smem_raw),

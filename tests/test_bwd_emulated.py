@@ -34,6 +34,10 @@ def emu_bwd(tmp_path_factory):
             "128_eager": ("bwd_kernel.cuh", "emu_bwd_main.cpp", "emu_bwd_128_eager", ("EMU_D=128", "EMU_EAGER_COPIES")),
             "128_eager_mma": ("bwd_kernel.cuh", "emu_bwd_main.cpp", "emu_bwd_128_eager_mma",
                               ("EMU_D=128", "EMU_EAGER_MMA")),
+            "256_eager_mma": (["bwd256_kernel.cuh", "bwd_kernel.cuh"], "emu_bwd_main.cpp", "emu_bwd_256_eager_mma",
+                              ("EMU_BWD256", "EMU_EAGER_MMA")),
+            "256_eager": (["bwd256_kernel.cuh", "bwd_kernel.cuh"], "emu_bwd_main.cpp", "emu_bwd_256_eager",
+                          ("EMU_BWD256", "EMU_EAGER_COPIES")),
         })
     except FileNotFoundError:
         pytest.skip("g++ not available")
@@ -73,6 +77,15 @@ def test_bwd_kernel_emulated_eager_mma(emu_bwd, B, H, H_kv, N, causal, window):
     """fa_bwd_kernel with MMAs that run as soon as they are issued: a dV, dK or dQ product issued
     before P^T or dS^T is in place reads it too early."""
     _check_bwd_emulated(emu_bwd["128_eager_mma"], [], B, H, H_kv, N, 128, causal, window)
+
+
+@pytest.mark.parametrize("kind", ["256_eager_mma", "256_eager"])
+@pytest.mark.parametrize("B,H,H_kv,N,causal,window", [(1, 2, 2, 300, True, 0), (1, 4, 2, 200, False, 50)])
+def test_bwd256_kernel_emulated_eager(emu_bwd, kind, B, H, H_kv, N, causal, window):
+    """fa_bwd256_kernel with MMAs that run at issue (the second dQ half must wait for the first
+    half's readout, since both use the same TMEM columns) and with copies that land at issue (a
+    Q or dO load before the MMAs of the previous query tile released the stage)."""
+    _check_bwd_emulated(emu_bwd[kind], [], B, H, H_kv, N, 256, causal, window)
 
 
 def _check_bwd_emulated(exe, extra, B, H, H_kv, N, d, causal, window):
