@@ -10,7 +10,8 @@
 // N x N score matrix never leaves the SM.
 //
 // sm_100a mapping: one CTA per pair of adjacent 128-row query tiles of one head, so every
-// K/V tile brought on chip serves 256 query rows.
+// K/V tile brought on chip serves 256 query rows; the grid takes heads in chunks, the longest
+// causal pairs of a chunk first (grid_item).
 //   warp 8      TMA producer (and TMEM owner): both Q tiles once, then K_j, V_j through a
 //               4-slot ring.
 //   warp 9      MMA issuer (one thread), in the order PV0(j), S0(j+1), PV1(j), S1(j+1), so
@@ -18,9 +19,11 @@
 //               runs (ping-pong).  S = Q K^T lands in TMEM; P is written back over the
 //               consumed S columns as bf16 and O += P V reads it from TMEM.
 //   warps 0-3   softmax of query tile 0, warps 4-7 of tile 1: thread t owns row t (TMEM
-//               lane t): tcgen05.ld of S, scale and mask, running max m and sum l,
+//               lane t): tcgen05.ld of S (twice: the row max, then the exponentials 32
+//               columns at a time), scale and mask, running max m and sum l,
 //               P = 2^(S c - m) packed to bf16 and stored to TMEM, and at the end O / l ->
-//               bf16 and L = (m + log2 l) ln 2.
+//               bf16 (written through the tile's Q buffer by TMA tensor stores) and
+//               L = (m + log2 l) ln 2.
 // The running max is updated lazily: O in TMEM is rescaled only when a row's max grows by
 // more than 2^8; otherwise the stale max keeps being used (P <= 256, exact after the final
 // division by l).  MMAs issued by one thread execute in order, so S(j) completing means
