@@ -116,7 +116,9 @@ __global__ void __launch_bounds__(256) fa_bwd_prep(const __nv_bfloat16* __restri
                                                    float* __restrict__ dd, float* __restrict__ dq_acc, int N, int Np,
                                                    int H, Strides o_st, Strides do_st, long long total_rows) {
   constexpr int G = D / 8;                      // threads per row
-  const long long g = (long long)blockIdx.x * (256 / G) + threadIdx.x / G;
+  // the last heads' rows first: the first heads' zeroed accumulator rows, which the main
+  // kernel's first chunk adds into, are then the most recently written (still in L2)
+  const long long g = (long long)(gridDim.x - 1 - blockIdx.x) * (256 / G) + threadIdx.x / G;
   const int c = threadIdx.x % G;
   if (g >= total_rows) return;
   const long long bh = g / Np;
@@ -153,7 +155,9 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_final(const float* __restrict__
                                                        __nv_bfloat16* __restrict__ dq, int N, int Np, float scale,
                                                        int H, Strides dq_st, long long total_rows) {
   constexpr int G = D / 8;
-  const long long g = (long long)blockIdx.x * (256 / G) + threadIdx.x / G;   // row of [BH, N]
+  // the last heads' rows first: the main kernel's last chunk added into them last, so they are
+  // the accumulator rows most likely still in L2
+  const long long g = (long long)(gridDim.x - 1 - blockIdx.x) * (256 / G) + threadIdx.x / G;   // row of [BH, N]
   const int c = threadIdx.x % G;
   if (g >= total_rows) return;
   const long long bh = g / N;

@@ -53,6 +53,16 @@ constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only when m
 #define FA_FWD_EMU_PAIRS 7
 #endif
 constexpr int kEmuPairs = FA_FWD_EMU_PAIRS;   // of every 16 exponential pairs, this many use the FMA pipe
+// fa_fwd_kernel's own split per head dimension: measured on a B200 (20-step causal / GPT-2-like
+// runs), 6 of 16 is best at d = 128 (0.2674 ms against 0.2691 at 7 and 0.2741 at 5) and 7 at
+// d = 64 (127.3 us against 128.2 at 6 and 135.3 at 8); the other forwards use kEmuPairs
+#ifdef FA_FWD_EMU_PAIRS_OVERRIDE
+template <int D>
+constexpr int kFwdEmuPairs = FA_FWD_EMU_PAIRS;
+#else
+template <int D>
+constexpr int kFwdEmuPairs = D == 64 ? 7 : 6;
+#endif
 
 struct FwdParams {
   __nv_bfloat16* o;   // [B, H, N, D] with strides o_st
@@ -357,7 +367,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const float m_new = grow ? m_cand : m;
         const float alpha = grow ? ex2_approx(m - m_new) : 1.f;   // 0 for the first keys of a row
         const float m_use = (m_new == -INFINITY) ? 0.f : m_new;   // a row with no key yet gives P = 0
-        // P = 2^(S c - m): in every 16 pairs the first kEmuPairs go through the FMA-pipe
+        // P = 2^(S c - m): in every 16 pairs the first kFwdEmuPairs<D> go through the FMA-pipe
         // polynomial, the rest through MUFU ex2, so that neither unit limits the tile
         const uint64_t c2 = f2(c, c), nm2 = f2(-m_use, -m_use);
         uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
@@ -378,7 +388,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           for (int jp = 0; jp < 16; ++jp) {
             const uint64_t x = f2_fma(f2(sv[2 * jp], sv[2 * jp + 1]), c2, nm2);
             float p0, p1;
-            if (jp < kEmuPairs) {
+            if (jp < kFwdEmuPairs<D>) {
               exp2_poly_x2(x, p0, p1);
             } else {
               float x0, x1;
