@@ -13,14 +13,21 @@
 //                                        tiles the first products read K-major), P and dS
 //                                        staged in shared memory as MN-major B operands
 //   dQ_c = dS K_c                        M = 128 queries, N = 128, K = 64 keys; K_c MN-major;
-//                                        one half after the other in the same 128 TMEM columns,
-//                                        each added into the fp32 accumulator with vector
-//                                        reductions before the next overwrites it.
+//                                        dQ_0 in its own columns, dQ_1 over those of S and dP
+//                                        (read by then), both right after dV^T and dK^T.
+// Each compute warp loads its 32 rows of dQ_c from TMEM at once (freeing the columns for the
+// next product), then stages them 32 columns at a time in 4 KB slots in the 128-byte swizzled
+// layout and adds each 32 x 32 block into the fp32 accumulator with one TMA tensor reduction
+// (whole 128-byte lines at the L2).  The slots are the warp's own 32 rows of the dS and P tiles,
+// in turn: both are free once dQ_1 is complete (every MMA that reads them came first).  The warp
+// writes those rows again (the next tile's P and dS) only after the reductions have read them.
 // Roles (192 threads): warps 0-3 compute (thread t of warp w owns TMEM lane 32w + t: a query
 // row of S, dP and dQ, and at the end a head-dim column of each half of dV^T and dK^T), warp 4
 // TMA, warp 5 MMA.  TMEM columns: S [0, 64), dP [64, 128), dV^T_0 [128, 192), dV^T_1 [192, 256),
-// dK^T_0 [256, 320), dK^T_1 [320, 384), dQ_c [384, 512).
-// One stage of Q and dO: the next query tile loads once the MMAs of this one are done.
+// dK^T_0 [256, 320), dK^T_1 [320, 384), dQ_0 [384, 512), dQ_1 [0, 128): the next tile's S and dP
+// wait until dQ_1 has been read out.
+// One stage of Q and dO: the next query tile loads once the dV and dK MMAs of this one are
+// done, while dQ is computed and read out.
 #pragma once
 
 #include <type_traits>
@@ -34,7 +41,8 @@ constexpr int kB256Rows = 128;    // query rows per iteration
 constexpr int kB256Threads = 192;
 constexpr int kB256WarpTma = 4;
 constexpr int kB256WarpMma = 5;
-constexpr uint32_t kT256S = 0, kT256dP = 64, kT256dV = 128, kT256dK = 256, kT256dQ = 384;   // dV^T_c, dK^T_c at + 64c
+constexpr uint32_t kT256S = 0, kT256dP = 64, kT256dV = 128, kT256dK = 256;   // dV^T_c, dK^T_c at + 64c
+constexpr uint32_t kT256dQ0 = 384, kT256dQ1 = 0;
 
 struct Bwd256Smem {
   static constexpr uint32_t kQChunk = kB256Rows * 128;   // 64 head-dim columns of 128 rows
@@ -47,7 +55,8 @@ struct Bwd256Smem {
   alignas(1024) uint8_t ds[kB256Rows * 128];   // dS [query][key]
   alignas(16) float lp[kB256Rows];
   alignas(16) float dd[kB256Rows];
-  alignas(8) uint64_t kv_full, q_full, q_empty, s_full, p_full, dq_full, dq_free, mma_final, mma_drain;
+  // q_empty: Q and dO read by this tile's last MMAs that use them (dV^T, dK^T)
+  alignas(8) uint64_t kv_full, q_full, q_empty, s_full, p_full, dq_full, dq_free0, dq_free1, mma_final, mma_drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -68,7 +77,7 @@ __device__ __forceinline__ void q_tile_range256(int kv0, int N, int causal, int 
 __global__ void __launch_bounds__(kB256Threads, 1)
     fa_bwd256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                     const BwdParams prm) {
+                     const __grid_constant__ CUtensorMap tm_dq, const BwdParams prm) {
   using Smem = Bwd256Smem;
   constexpr int D = 256;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -99,8 +108,9 @@ __global__ void __launch_bounds__(kB256Threads, 1)
     mbar_init(smem_u32(&sm.q_empty), 1);
     mbar_init(smem_u32(&sm.s_full), 1);
     mbar_init(smem_u32(&sm.p_full), kB256Rows);
-    mbar_init(smem_u32(&sm.dq_full), 1);      // completes twice per query tile (dQ_0, dQ_1)
-    mbar_init(smem_u32(&sm.dq_free), kB256Rows);   // likewise (each half read out)
+    mbar_init(smem_u32(&sm.dq_full), 1);            // dQ_0 and dQ_1 complete
+    mbar_init(smem_u32(&sm.dq_free0), kB256Rows);   // dQ_0 read out of TMEM
+    mbar_init(smem_u32(&sm.dq_free1), kB256Rows);   // dQ_1 read out of TMEM (S and dP may be written)
     mbar_init(smem_u32(&sm.mma_final), 1);
     mbar_init(smem_u32(&sm.mma_drain), 1);
     fence_mbar_init();
@@ -111,6 +121,7 @@ __global__ void __launch_bounds__(kB256Threads, 1)
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_do);
+      tma_prefetch_desc(&tm_dq);
     }
     __syncwarp();
     tmem_alloc(smem_u32(&sm.tmem_base), 512);
@@ -172,6 +183,7 @@ __global__ void __launch_bounds__(kB256Threads, 1)
     bool ok = n_it > 0 && wait(smem_u32(&sm.kv_full), 0);
     for (int it = 0; ok && it < n_it; ++it) {
       if (!wait(smem_u32(&sm.q_full), it & 1)) break;
+      if (it > 0 && !wait(smem_u32(&sm.dq_free1), (it - 1) & 1)) break;   // dQ_1 left S and dP's columns
       tc_fence_after();
       // S = Q K^T and dP = dO V^T over the full head dimension
 #pragma unroll
@@ -198,24 +210,20 @@ __global__ void __launch_bounds__(kB256Threads, 1)
                         idesc_t, acc);
         }
       }
-      // dQ_c = dS K_c: 16 keys per k-step (32 bytes along dS's rows, 16 rows of K).  The two
-      // halves share the dQ columns: each waits until the previous one has been read out
-      // (dq_free completes twice per query tile: the readouts of dQ_0 and dQ_1)
+      mma_commit_w(smem_u32(&sm.q_empty));   // the next Q and dO may load now
+      // dQ_c = dS K_c: 16 keys per k-step (32 bytes along dS's rows, 16 rows of K).  dQ_0 waits
+      // until the previous tile's dQ_0 has been read out of its columns
+      if (it > 0 && !wait(smem_u32(&sm.dq_free0), (it - 1) & 1)) break;
+      tc_fence_after();
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        if ((it > 0 || c > 0) && !wait(smem_u32(&sm.dq_free), c == 0 ? 1u : 0u)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
         const uint64_t kt = dk_t(c);
+        const uint32_t dst = c == 0 ? kT256dQ0 : kT256dQ1;
 #pragma unroll
         for (int kk = 0; kk < kB256Keys / 16; ++kk)
-          mma_bf16_ss_w(tmem + kT256dQ, desc_advance(dds_k, kk * 32), desc_advance(kt, kk * 2048), idesc_q, kk > 0);
-        mma_commit_w(smem_u32(&sm.dq_full));
+          mma_bf16_ss_w(tmem + dst, desc_advance(dds_k, kk * 32), desc_advance(kt, kk * 2048), idesc_q, kk > 0);
       }
-      if (!ok) break;
-      mma_commit_w(smem_u32(&sm.q_empty));
+      mma_commit_w(smem_u32(&sm.dq_full));
     }
     mma_commit_w(smem_u32(&sm.mma_final));
     mma_commit_w(smem_u32(&sm.mma_drain));
@@ -224,6 +232,8 @@ __global__ void __launch_bounds__(kB256Threads, 1)
     // ------------------------------------------------------------------ compute warps
     const int row = threadIdx.x;   // TMEM lane: a query row of S, dP, dQ; head-dim column row (+ 128) of dV^T, dK^T
     const uint32_t lane_base = uint32_t(warp * 32) << 16;
+    const uint32_t slot_p = smem_u32(sm.p) + uint32_t(warp) * 4096;    // my 32 rows of P and of dS:
+    const uint32_t slot_ds = smem_u32(sm.ds) + uint32_t(warp) * 4096;  // dQ staging slots
     const float c = prm.scale_log2;
     bool ok = true;
     for (int it = 0; ok && it < n_it; ++it) {
@@ -261,10 +271,12 @@ __global__ void __launch_bounds__(kB256Threads, 1)
         pk[j / 2] = pack_bf16x2(p2[0], p2[1]);
         dk2[j / 2] = pack_bf16x2(d2[0], d2[1]);
       }
-      // P and dS of the previous query tile must have been read by its MMAs
+      // P and dS of the previous query tile have been read by its MMAs: this warp saw its dQ
+      // complete, and the MMAs finish in issue order.  My rows of both must also have
+      // been read by the tensor reductions that staged dQ there.
       if (it > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.q_empty), (it - 1) & 1, abort, lim));
-        if (!ok) break;
+        if (lane == 0) bulk_wait_group_read<0>();
+        __syncwarp();
       }
       // row `row` of the P and dS tiles: 8 chunks of 16 bytes, chunk j at j ^ (row % 8)
 #pragma unroll
@@ -276,24 +288,42 @@ __global__ void __launch_bounds__(kB256Threads, 1)
       fence_proxy_async_smem();   // the MMAs read P and dS through the async proxy
       tc_fence_before();
       mbar_arrive(smem_u32(&sm.p_full));
-      // dQ_0, then dQ_1 (the same TMEM columns, one after the other): this row's 128 columns of
-      // each into the fp32 accumulator
+      // dQ_1 first (its columns are the next tile's S and dP), then dQ_0: my 32 rows into
+      // registers, then 32 columns a pass through the dS and P slots in turn into the
+      // accumulator rows q0 + 32 warp ..
+      const int q_row = q0 + warp * 32;
+      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.dq_full), it & 1, abort, lim));
+      if (!ok) break;
+      tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < 2 && ok; ++c) {
-        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.dq_full), uint32_t(c), abort, lim));
-        if (!ok) break;
-        tc_fence_after();
-        float* acc = prm.dq_acc + (size_t(hq) * prm.Np + qi) * D + c * 128;
+      for (int c = 1; c >= 0; --c) {
+        uint32_t r[128];
+        const uint32_t src = c == 0 ? kT256dQ0 : kT256dQ1;
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          uint32_t r[32];
-          tmem_ld32(tmem + lane_base + kT256dQ + ch * 32, r);
+        for (int ps = 0; ps < 4; ++ps) tmem_ld32_async(tmem + lane_base + src + ps * 32, r + 32 * ps);
+        tmem_ld_wait();
+        reg_fence<128>(r);
+        tc_fence_before();
+        mbar_arrive(smem_u32(c == 0 ? &sm.dq_free0 : &sm.dq_free1));   // the MMA warp may overwrite dQ_c
+#pragma unroll
+        for (int ps = 0; ps < 4; ++ps) {
+          // even passes through the dS rows, odd ones through the P rows, each after the read
+          // of the pass before the previous one
+          const uint32_t slot = (ps & 1) ? slot_p : slot_ds;
+          if (lane == 0) bulk_wait_group_read<1>();
+          __syncwarp();
+          // row `lane`, 16-byte chunk j at lane * 128 + (j ^ (lane & 7)) * 16
 #pragma unroll
           for (int j = 0; j < 8; ++j)
-            red_add_v4(acc + ch * 32 + 4 * j, make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]));
+            st_shared_v4(slot + lane * 128 + ((j ^ (lane & 7)) << 4), r[32 * ps + 4 * j], r[32 * ps + 4 * j + 1],
+                         r[32 * ps + 4 * j + 2], r[32 * ps + 4 * j + 3]);
+          fence_proxy_async_smem();   // the tensor reduction reads the slot through the async proxy
+          __syncwarp();
+          if (lane == 0) {
+            tma_reduce_add_rows(&tm_dq, slot, c * 128 + ps * 32, q_row, hq, 0);
+            bulk_commit_group();
+          }
         }
-        tc_fence_before();
-        mbar_arrive(smem_u32(&sm.dq_free));
       }
     }
     // dV and dK of this tile's keys, head-dim columns row and 128 + row
@@ -325,6 +355,10 @@ __global__ void __launch_bounds__(kB256Threads, 1)
         }
       }
     }
+    // every reduction this warp issued has finished (its slot read, its adds done) before the
+    // CTA's shared memory is released
+    if (lane == 0) bulk_wait_group<0>();
+    __syncwarp();
   }
 
   tc_fence_before();

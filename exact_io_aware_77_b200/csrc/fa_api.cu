@@ -296,9 +296,11 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
     prm.n_kv_tiles = (N + kB256Keys - 1) / kB256Keys;
     static_assert(sizeof(Bwd256Smem) <= 232448, "d = 256 backward shared memory exceeds 227 KB");
     const int smem = int(sizeof(Bwd256Smem));
+    CUtensorMap tdq;
+    if (!make_map_dq_acc(&tdq, dq_acc, D, Np, BH)) return FA_ERR_CUDA;
     if (set_smem(fa_bwd256_kernel, smem) != FA_OK) return FA_ERR_CUDA;
     fa_bwd256_kernel<<<unsigned(prm.n_kv_tiles) * unsigned(BH_kv), kB256Threads, smem, stream>>>(tq, tk, tv, tdo,
-                                                                                                         prm);
+                                                                                                         tdq, prm);
   } else {
     static_assert(sizeof(BwdSmem<D>) <= 232448, "backward shared memory exceeds 227 KB");
     const int smem = int(sizeof(BwdSmem<D>));   // the kernel checks that the base is 1 KB aligned

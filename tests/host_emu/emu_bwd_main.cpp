@@ -128,7 +128,7 @@ int main(int argc, char** argv) {
   prm.wait_limit_ns = 60ull * 1000000000ull;
 #ifdef EMU_BWD256
   emu_launch(unsigned(prm.n_kv_tiles) * unsigned(BH_kv), kB256Threads, sizeof(fa::smem_raw),
-             [&] { fa_bwd256_kernel(tq, tk, tv, tdo, prm); }, fa::smem_raw);
+             [&] { fa_bwd256_kernel(tq, tk, tv, tdo, tdq, prm); }, fa::smem_raw);
 #else
   emu_launch(unsigned(prm.n_kv_tiles) * unsigned(BH_kv), kBwdThreads, sizeof(fa::smem_raw),
              [&] { fa_bwd_kernel<D>(tq, tk, tv, tdo, tdq, prm); }, fa::smem_raw);

@@ -49,7 +49,7 @@ CASES = [
     (1, 4, 2, 400, 128, False, 50),    # two-sided window, two query heads per K/V head
     (2, 2, 1, 257, 64, True, 3),       # multi-query, narrow causal window
     (1, 1, 1, 600, 64, True, 1),       # window 1: dQ = dK = 0, dV = dO
-    # head dimension 256 (fa_bwd256_kernel: 64-key tiles, one CTA per head-dim half)
+    # head dimension 256 (fa_bwd256_kernel: one CTA per 64-key tile)
     (1, 1, 1, 128, 256, True, 0),
     (1, 1, 1, 300, 256, True, 1),
     (1, 2, 2, 300, 256, False, 0),
