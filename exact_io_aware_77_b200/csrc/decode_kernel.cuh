@@ -6,8 +6,9 @@
 // positions, "rows" in all) are cut into blocks of 16, the M of an m16n8k16 warp MMA, so one
 // pass over the head's keys serves all of them.  The keys are cut into chunks ("splits"),
 // one CTA per (split, row block, K/V head).  Each of a CTA's four warps streams its own
-// 16-key steps through a private three-stage cp.async ring and keeps its own running max m,
-// sum l and unnormalised output; the CTA merges its warps, and when there is more than one
+// 16-key steps through a private three-stage ring, filled by TMA tensor loads that its lane 0
+// issues and that complete on one mbarrier per stage, and keeps its own running max m, sum l
+// and unnormalised output; the CTA merges its warps, and when there is more than one
 // split a second kernel merges the splits by their logsumexps:
 //   L = M + ln sum_s exp(L_s - M),  O = sum_s exp(L_s - L) O_s   (M = max_s L_s).
 // Every split's O_s is already normalised by its own l; a split with no allowed key has
@@ -15,9 +16,9 @@
 //
 // With an FP8 K/V cache (kFp8) K and V arrive as E4M3 codes with one scale per tensor
 // (K = s_k K8, V = s_v V8).  The ring then holds the raw codes; before each step the warp
-// converts its 16 keys to f16 (exactly: every E4M3 value is an f16 value) into one tile laid
-// out as the bf16 stages are, and the MMAs run on f16 operands (Q rounded to f16, clamped to
-// its finite range).  s_k is folded into the softmax scale and s_v into the final division.
+// converts its 16 keys to f16 (exactly: every E4M3 value is an f16 value) into one padded
+// tile, and the MMAs run on f16 operands (Q rounded to f16, clamped to its finite range).
+// s_k is folded into the softmax scale and s_v into the final division.
 #pragma once
 
 #include <climits>
@@ -39,30 +40,41 @@ constexpr int kDecCtaOverheadKeys = 128;   // a CTA's fixed cost (Q load, ring f
 
 template <int D, bool kFp8 = false>
 struct DecLayout {
-  // one K or V row (16-bit values) in shared memory, padded by 16 bytes so that the eight rows
-  // an 8x8 matrix load reads start in eight different 16-byte bank groups
+  // A ring stage holds one step's K tile, then its V tile, as their TMA loads leave them: boxes
+  // of 16 key rows, 128-byte swizzled (16-byte piece c of row r at c ^ (r % 8)).  bf16: D / 64
+  // boxes of 64 elements a tile, read by the MMAs in place.  FP8: the raw E4M3 codes, D / 128
+  // boxes of 128 a tile (at d = 64 one unswizzled box of 64-byte rows), which the warp converts
+  // into the f16 K, V tile pair that follows its ring.
+  static constexpr int kBoxX = kFp8 && D >= 128 ? 128 : 64;   // elements of a box row
+  static constexpr bool kSwizzled = !kFp8 || D >= 128;
+  static constexpr int kBoxBytes = kDecKeys * kBoxX * (kFp8 ? 1 : 2);
+  static constexpr int kKvTileBytes = kDecKeys * D * (kFp8 ? 1 : 2);
+  static constexpr int kBoxes = kKvTileBytes / kBoxBytes;     // TMA loads per tile
+  static constexpr int kStageBytes = 2 * kKvTileBytes;        // K, then V
+  // a converted f16 row, padded by 16 bytes so that the eight rows an 8x8 matrix load reads
+  // start in eight different 16-byte bank groups
   static constexpr int kRowBytes = 2 * D + 16;
-  static constexpr int kTileBytes = kDecKeys * kRowBytes;
-  // bf16: the ring stages are the tiles the MMAs read.  FP8: the stages hold the raw E4M3
-  // rows (D bytes each), and one converted f16 K, V tile pair follows the ring.
-  static constexpr int kRawTileBytes = kDecKeys * D;
-  static constexpr int kStageBytes = kFp8 ? 2 * kRawTileBytes : 2 * kTileBytes;   // K rows, then V rows
-  static constexpr int kConvBytes = kFp8 ? 2 * kTileBytes : 0;
-  static constexpr int kWarpBytes = kDecStages * kStageBytes + kConvBytes;
+  static constexpr int kConvTileBytes = kDecKeys * kRowBytes;
+  static constexpr int kConvBytes = kFp8 ? 2 * kConvTileBytes : 0;
+  // each warp's ring starts on a 1 KB boundary (the swizzle's atom)
+  static constexpr int kWarpBytes = (kDecStages * kStageBytes + kConvBytes + 1023) / 1024 * 1024;
   static constexpr int kRingBytes = kDecWarps * kWarpBytes;
   // after the key loop the rings hold each warp's O [16][D], m [16] and l [16] (fp32)
   static constexpr int kMergeFloats = kDecRows * D + 2 * kDecRows;
   static constexpr int kMergeBytes = kDecWarps * kMergeFloats * 4;
-  static constexpr int kSmemBytes = kRingBytes > kMergeBytes ? kRingBytes : kMergeBytes;
+  static constexpr int kDataBytes = kRingBytes > kMergeBytes ? kRingBytes : kMergeBytes;
+  // then one mbarrier per (warp, stage) and one abort flag per warp
+  static constexpr int kBarOffset = kDataBytes;
+  static constexpr int kAbortOffset = kBarOffset + kDecWarps * kDecStages * 8;
+  // the dynamic shared memory is rounded up to 1 KB inside the kernel: 1 KB of slack
+  static constexpr int kSmemBytes = 1024 + kAbortOffset + kDecWarps * 4;
+  static_assert(kStageBytes % 1024 == 0 && kBoxBytes % 1024 == 0, "ring stages and boxes on 1 KB boundaries");
   static_assert(kSmemBytes <= 232448, "decode shared memory exceeds 227 KB");
 };
 
+// K and V ([B, H_kv, N_k, d], bf16 or E4M3 codes) reach the kernel as tensor maps.
 struct DecParams {
   const __nv_bfloat16* q;   // [B, H, N_q, d]
-  const __nv_bfloat16* k;   // [B, H_kv, N_k, d]
-  const __nv_bfloat16* v;
-  const unsigned char* k8;  // FP8 K/V cache: E4M3 codes [B, H_kv, N_k, d] (else unused)
-  const unsigned char* v8;
   float v_scale;            // FP8: s_v (s_k is in scale_log2)
   __nv_bfloat16* o;         // [B, H, N_q, d]
   float* lse;               // [B, H, N_q] contiguous
@@ -75,6 +87,7 @@ struct DecParams {
   int n_splits, chunk, key_begin;   // split s covers keys [key_begin + s chunk, + chunk)
   int causal, window;
   float scale_log2;         // scale * log2(e)
+  unsigned long long wait_limit_ns;   // bound on each wait for a ring stage
 };
 
 // Closed interval [lo, hi] of the keys a query at position pos may attend.
@@ -154,14 +167,45 @@ __device__ __forceinline__ uint32_t dec_pack(float lo, float hi) {
     return pack_bf16x2(lo, hi);
 }
 
+// Bounded wait for a ring stage, inline (no call in the key loop, whose registers would then
+// have to survive one): the same limit and status as mbar_wait.
+__device__ __forceinline__ bool dec_wait(uint32_t bar, uint32_t parity, volatile int* abort, uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t n = 1;; ++n) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((n & 63u) == 0 && (*abort || global_timer_ns() - t0 > limit_ns)) {
+      if (!*abort) atomicOr(&g_status, FA_DEVICE_TIMEOUT);
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
+// tm_k, tm_v: K and V (bf16, or the E4M3 codes) as the 4-D tensors (d, N_k, H_kv, B), boxes of
+// DecLayout::kBoxX elements x 16 keys.
 template <int D, bool kFp8>
-__global__ void __launch_bounds__(kDecThreads, 2) fa_decode_kernel(const DecParams p) {
+__global__ void __launch_bounds__(kDecThreads, 2)
+    fa_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                     const DecParams p) {
   using Lay = DecLayout<D, kFp8>;
   constexpr int KS = D / 16;   // k-steps of S = Q K^T
   constexpr int NT = D / 8;    // 8-column n-tiles of O
   constexpr float kLn2 = 0.6931471805599453f;
-  unsigned char* smem = dec_dyn_smem();
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(dec_dyn_smem()) + 1023) &
+                                                         ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBarOffset) + warp * kDecStages;   // my ring's
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + Lay::kAbortOffset) + warp;
+  if (lane == 0) {
+    *abort = 0;
+    for (int st = 0; st < kDecStages; ++st) mbar_init(smem_u32(&bars[st]), 1);
+    fence_mbar_init();
+    fence_proxy_async_smem();   // the ring's copies complete on these barriers through the async proxy
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  __syncwarp();
   const int g = lane >> 2, t = lane & 3;   // MMA fragment row group and column pair
   // the merge grid may be scheduled once every CTA of this one has started: its CTAs then wait
   // (grid_dep_wait) on SMs this grid's last wave frees, instead of a launch after it
@@ -232,37 +276,25 @@ __global__ void __launch_bounds__(kDecThreads, 2) fa_decode_kernel(const DecPara
   const int my_steps = n_steps > warp ? (n_steps - warp + kDecWarps - 1) / kDecWarps : 0;
 
   unsigned char* ring = smem + warp * Lay::kWarpBytes;
+  // lane 0: step it's K and V tiles into stage it % kDecStages; keys past N_k read as zero
   auto issue = [&](int it) {
     const int key0 = s0 + kDecKeys * (warp + kDecWarps * it);
-    unsigned char* stage = ring + (it % kDecStages) * Lay::kStageBytes;
-    if constexpr (kFp8) {
-      constexpr int kPieces = D / 16;   // 16-byte pieces per raw E4M3 row
+    const uint32_t stage = smem_u32(ring + (it % kDecStages) * Lay::kStageBytes);
+    const uint32_t bar = smem_u32(&bars[it % kDecStages]);
+    mbar_expect_tx(bar, Lay::kStageBytes);
 #pragma unroll
-      for (int x = 0; x < kDecKeys * kPieces / 32; ++x) {
-        const int c = lane + 32 * x;
-        const int row = c / kPieces, col = c % kPieces;
-        const int key = key0 + row;
-        const bool in = key < p.Nk;
-        const int src_key = in ? key : 0;
-        cp_async_16(stage + row * D + col * 16, p.k8 + p.k_st.at(b, hkv, src_key) + col * 16, in ? 16 : 0);
-        cp_async_16(stage + Lay::kRawTileBytes + row * D + col * 16, p.v8 + p.v_st.at(b, hkv, src_key) + col * 16,
-                    in ? 16 : 0);
-      }
-    } else {
-      constexpr int kPieces = D / 8;   // 16-byte pieces per row
-#pragma unroll
-      for (int x = 0; x < kDecKeys * kPieces / 32; ++x) {
-        const int c = lane + 32 * x;
-        const int row = c / kPieces, col = c % kPieces;
-        const int key = key0 + row;
-        const bool in = key < p.Nk;
-        const int src_key = in ? key : 0;
-        cp_async_16(stage + row * Lay::kRowBytes + col * 16, p.k + p.k_st.at(b, hkv, src_key) + col * 8,
-                    in ? 16 : 0);
-        cp_async_16(stage + Lay::kTileBytes + row * Lay::kRowBytes + col * 16,
-                    p.v + p.v_st.at(b, hkv, src_key) + col * 8, in ? 16 : 0);
-      }
+    for (int c = 0; c < Lay::kBoxes; ++c) {
+      tma_load_rows(stage + c * Lay::kBoxBytes, &tm_k, bar, c * Lay::kBoxX, key0, hkv, b);
+      tma_load_rows(stage + Lay::kKvTileBytes + c * Lay::kBoxBytes, &tm_v, bar, c * Lay::kBoxX, key0, hkv, b);
     }
+  };
+  // byte offset of the 16-byte piece holding elements col .. col + 7 of key row kr of a tile in a
+  // stage (128-byte swizzled boxes of 64 elements), or of a converted f16 tile (padded rows)
+  auto piece = [&](int kr, int col) -> int {
+    if constexpr (kFp8)
+      return kr * Lay::kRowBytes + col * 2;
+    else
+      return (col >> 6) * Lay::kBoxBytes + kr * 128 + ((((col & 63) >> 3) ^ (kr & 7)) << 4);
   };
 
   float acc[NT][4];
@@ -270,14 +302,20 @@ __global__ void __launch_bounds__(kDecThreads, 2) fa_decode_kernel(const DecPara
   for (int j = 0; j < NT; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
   float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
 
-#pragma unroll
-  for (int it = 0; it < kDecStages - 1; ++it) {
-    if (it < my_steps) issue(it);
-    cp_async_commit();
-  }
-  for (int it = 0; it < my_steps; ++it) {
-    cp_async_wait<kDecStages - 2>();   // step it has landed (this lane's pieces)
-    __syncwarp();                      // ... and every lane's; all lanes are past step it - 1
+  int issued = 0;   // lane 0's loads; every lane tracks the same count
+  if (lane == 0)
+    for (int it = 0; it < min(my_steps, kDecStages - 1); ++it) issue(it);
+  issued = min(my_steps, kDecStages - 1);
+  bool ok = true;
+  int it = 0;
+  for (; it < my_steps; ++it) {
+    // step it has landed; the vote also puts every lane past step it - 1, whose stage the next
+    // load (issued at the end of this step) overwrites
+    if (!__all_sync(0xffffffffu, dec_wait(smem_u32(&bars[it % kDecStages]), (it / kDecStages) & 1, abort,
+                                          p.wait_limit_ns))) {
+      ok = false;
+      break;
+    }
     const unsigned char* ks = ring + (it % kDecStages) * Lay::kStageBytes;
     if constexpr (kFp8) {
       // E4M3 -> f16 into the converted tiles: 16 codes (one 16-byte piece) per lane at a time
@@ -289,7 +327,9 @@ __global__ void __launch_bounds__(kDecThreads, 2) fa_decode_kernel(const DecPara
         const int c = lane + 32 * x;
         const int tensor = c / kPerTensor, rem = c % kPerTensor;
         const int row = rem / kPieces, col = rem % kPieces;
-        const uint4 w = *reinterpret_cast<const uint4*>(ks + tensor * Lay::kRawTileBytes + row * D + col * 16);
+        const int src = Lay::kSwizzled ? (col >> 3) * Lay::kBoxBytes + row * 128 + (((col & 7) ^ (row & 7)) << 4)
+                                       : row * D + col * 16;
+        const uint4 w = *reinterpret_cast<const uint4*>(ks + tensor * Lay::kKvTileBytes + src);
         uint4 lo, hi;
         lo.x = e4m3x2_to_f16x2(w.x);
         lo.y = e4m3x2_to_f16x2(w.x >> 16);
@@ -299,14 +339,14 @@ __global__ void __launch_bounds__(kDecThreads, 2) fa_decode_kernel(const DecPara
         hi.y = e4m3x2_to_f16x2(w.z >> 16);
         hi.z = e4m3x2_to_f16x2(w.w);
         hi.w = e4m3x2_to_f16x2(w.w >> 16);
-        unsigned char* dst = conv + tensor * Lay::kTileBytes + row * Lay::kRowBytes + col * 32;
+        unsigned char* dst = conv + tensor * Lay::kConvTileBytes + row * Lay::kRowBytes + col * 32;
         *reinterpret_cast<uint4*>(dst) = lo;
         *reinterpret_cast<uint4*>(dst + 16) = hi;
       }
       __syncwarp();   // the converted tiles are complete for every lane
       ks = conv;
     }
-    const unsigned char* vs = ks + Lay::kTileBytes;
+    const unsigned char* vs = ks + (kFp8 ? Lay::kConvTileBytes : Lay::kKvTileBytes);
     const int key0 = s0 + kDecKeys * (warp + kDecWarps * it);
 
     // S = Q K^T for 16 keys: n-tiles of keys 0-7 and 8-15
@@ -314,7 +354,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) fa_decode_kernel(const DecPara
 #pragma unroll
     for (int kk = 0; kk < KS; ++kk) {
       uint32_t kf[4];   // matrices: keys 0-7 | 8-15  x  columns 16kk + 0-7 | 8-15
-      ldmatrix_x4(kf, ks + (((lane >> 4) << 3) + (lane & 7)) * Lay::kRowBytes + (16 * kk + ((lane >> 3) & 1) * 8) * 2);
+      ldmatrix_x4(kf, ks + piece(((lane >> 4) << 3) + (lane & 7), 16 * kk + ((lane >> 3) & 1) * 8));
       dec_mma<kFp8>(s[0], qa[kk], kf[0], kf[1]);
       dec_mma<kFp8>(s[1], qa[kk], kf[2], kf[3]);
     }
@@ -364,14 +404,20 @@ __global__ void __launch_bounds__(kDecThreads, 2) fa_decode_kernel(const DecPara
 #pragma unroll
     for (int j = 0; j < D / 16; ++j) {
       uint32_t vf[4];   // transposed matrices: keys 0-7 | 8-15  x  columns 16j + 0-7 | 8-15
-      ldmatrix_x4_trans(vf, vs + (((lane >> 3) & 1) * 8 + (lane & 7)) * Lay::kRowBytes + (16 * j + (lane >> 4) * 8) * 2);
+      ldmatrix_x4_trans(vf, vs + piece(((lane >> 3) & 1) * 8 + (lane & 7), 16 * j + (lane >> 4) * 8));
       dec_mma<kFp8>(acc[2 * j], pa, vf[0], vf[1]);
       dec_mma<kFp8>(acc[2 * j + 1], pa, vf[2], vf[3]);
     }
-    if (it + kDecStages - 1 < my_steps) issue(it + kDecStages - 1);
-    cp_async_commit();
+    // the next load goes into stage it - 1's slot, which every lane has left (the vote above)
+    if (issued < my_steps) {
+      if (lane == 0) issue(issued);
+      ++issued;
+    }
   }
-  cp_async_wait<0>();
+  // after an abort, the loads still in flight land before the ring is reused or released
+  if (lane == 0)
+    for (int j = it; j < issued; ++j) mbar_wait_drain(smem_u32(&bars[j % kDecStages]), (j / kDecStages) & 1, p.wait_limit_ns);
+  __syncwarp();
 #pragma unroll
   for (int hf = 0; hf < 2; ++hf) {
     l_run[hf] += __shfl_xor_sync(0xffffffffu, l_run[hf], 1);

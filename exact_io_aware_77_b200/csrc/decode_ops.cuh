@@ -1,8 +1,7 @@
-// Device primitives of the split-key decode kernel: 16-byte asynchronous copies from
-// global into shared memory (zero-filling rows past the end of the keys), 8x8 matrix loads
-// from shared memory into warp MMA operand registers, and the m16n8k16 bf16 warp MMA with
-// fp32 accumulators.  These are warp-level instructions: the decode kernel's rows are too
-// few (16) for a tcgen05 MMA tile, and its time goes to reading K and V from HBM.
+// Device primitives of the split-key decode kernel: 8x8 matrix loads from shared memory into
+// warp MMA operand registers, and the m16n8k16 bf16 (or f16) warp MMA with fp32 accumulators.
+// These are warp-level instructions: the decode kernel's rows are too few (16) for a tcgen05
+// MMA tile, and its time goes to reading K and V from HBM.
 #pragma once
 
 #include <cstdint>
@@ -15,19 +14,6 @@ namespace fa {
 __device__ __forceinline__ unsigned char* dec_dyn_smem() {
   extern __shared__ __align__(128) unsigned char dec_smem_raw[];
   return dec_smem_raw;
-}
-
-// Copy 16 bytes from global to shared memory, bypassing L1.  src_bytes = 0 reads nothing
-// and writes 16 zero bytes.
-__device__ __forceinline__ void cp_async_16(void* dst, const void* src, int src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-// Wait until at most N of this thread's committed copy groups are still in flight.
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // Four 8x8 b16 matrices; lane l gives the address of row l % 8 of matrix l / 8, and receives

@@ -74,6 +74,21 @@ bool make_map_u8(CUtensorMap* map, const void* base, int x, int rows, int heads,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The decode kernel's E4M3 K or V cache [B, heads, rows, d] with element strides st as the 4-D
+// tensor (d, rows, heads, B): boxes of 16 rows x 128 codes, 128-byte swizzled, or at d = 64 of
+// 16 unswizzled 64-byte rows.  Rows past the end read as zero.
+bool make_map_dec_u8(CUtensorMap* map, const void* base, int d, int rows, int heads, int B, Strides st) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {cuuint64_t(d), cuuint64_t(rows), cuuint64_t(heads), cuuint64_t(B)};
+  cuuint64_t strides[3] = {cuuint64_t(st.n), cuuint64_t(st.h), cuuint64_t(st.b)};
+  cuuint32_t box[4] = {cuuint32_t(d >= 128 ? 128 : 64), cuuint32_t(kDecKeys), 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, d >= 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // The backward's fp32 dQ accumulator [BH, Np, d] as the 4-D tensor (d, Np, BH, 1) that its
 // tensor reductions add into: 32 x 32 boxes (128-byte rows), 128-byte swizzled.
 bool make_map_dq_acc(CUtensorMap* map, float* base, int d, long long Np, long long BH) {
@@ -345,10 +360,6 @@ int launch_decode(const void* q, const void* k, const void* v, void* o, float* l
                   cudaStream_t stream, float k_scale = 1.f, float v_scale = 1.f) {
   DecParams p;
   p.q = static_cast<const __nv_bfloat16*>(q);
-  p.k = kFp8 ? nullptr : static_cast<const __nv_bfloat16*>(k);
-  p.v = kFp8 ? nullptr : static_cast<const __nv_bfloat16*>(v);
-  p.k8 = kFp8 ? static_cast<const unsigned char*>(k) : nullptr;
-  p.v8 = kFp8 ? static_cast<const unsigned char*>(v) : nullptr;
   p.v_scale = v_scale;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
@@ -372,9 +383,15 @@ int launch_decode(const void* q, const void* k, const void* v, void* o, float* l
   p.causal = causal;
   p.window = window > Nk ? Nk : window;
   p.scale_log2 = scale * k_scale * 1.4426950408889634f;
+  p.wait_limit_ns = g_wait_limit_ns;
+  CUtensorMap tk, tv;
+  if (kFp8 ? !make_map_dec_u8(&tk, k, D, Nk, H_kv, B, st[1]) || !make_map_dec_u8(&tv, v, D, Nk, H_kv, B, st[2])
+           : !make_map_bf16(&tk, k, D, Nk, H_kv, B, st[1], kDecKeys) ||
+                 !make_map_bf16(&tv, v, D, Nk, H_kv, B, st[2], kDecKeys))
+    return FA_ERR_CUDA;
   constexpr int smem = DecLayout<D, kFp8>::kSmemBytes;
   if (set_smem(fa_decode_kernel<D, kFp8>, smem) != FA_OK) return FA_ERR_CUDA;
-  fa_decode_kernel<D, kFp8><<<unsigned(pl.ctas), kDecThreads, smem, stream>>>(p);
+  fa_decode_kernel<D, kFp8><<<unsigned(pl.ctas), kDecThreads, smem, stream>>>(tk, tv, p);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   if (pl.n_splits > 1) {
     const long long blocks = (pl.total_rows + kDecMergeWarps - 1) / kDecMergeWarps;

@@ -10,6 +10,10 @@
 
 using namespace fa;
 
+// the kernels' dynamic shared memory, on a 1 KB boundary as on the device (the swizzled ring
+// stages are placed relative to it)
+alignas(1024) static unsigned char dec_smem[232448];
+
 template <class T>
 std::vector<T> read_file(const std::string& path, size_t n) {
   std::vector<T> v(n);
@@ -60,10 +64,6 @@ int main(int argc, char** argv) {
   std::vector<float> ws(pl.ws_bytes / 4 + 1, NAN);
   DecParams p;
   p.q = reinterpret_cast<const __nv_bfloat16*>(q.data());
-  p.k = fp8 ? nullptr : reinterpret_cast<const __nv_bfloat16*>(k.data());
-  p.v = fp8 ? nullptr : reinterpret_cast<const __nv_bfloat16*>(v.data());
-  p.k8 = fp8 ? k8.data() : nullptr;
-  p.v8 = fp8 ? v8.data() : nullptr;
   p.v_scale = v_scale;
   p.o = reinterpret_cast<__nv_bfloat16*>(o.data());
   p.lse = lse.data();
@@ -87,34 +87,56 @@ int main(int argc, char** argv) {
   p.causal = causal;
   p.window = win;
   p.scale_log2 = scale * k_scale * 1.4426950408889634f;
+  p.wait_limit_ns = 2000000000ull;
+  // K and V as the tensor maps fa_fwd_decode encodes: (d, N_k, H_kv, B), 16-row boxes of 64 bf16
+  // or 128 codes (128-byte swizzled), at d = 64 with E4M3 codes 64 unswizzled
+  auto kv_map = [&](const void* base, const Strides& s) {
+    CUtensorMap m;
+    const uint32_t es = fp8 ? 1 : 2;
+    m.base = static_cast<const unsigned char*>(base);
+    m.dims[0] = uint64_t(d);
+    m.dims[1] = uint64_t(Nk);
+    m.dims[2] = uint64_t(Hkv);
+    m.dims[3] = uint64_t(B);
+    m.strides[0] = uint64_t(s.n) * es;
+    m.strides[1] = uint64_t(s.h) * es;
+    m.strides[2] = uint64_t(s.b) * es;
+    m.box_x = fp8 && d >= 128 ? 128 : 64;
+    m.box_rows = kDecKeys;
+    m.esize = es;
+    m.swizzle = fp8 && d < 128 ? 0 : 128;
+    return m;
+  };
+  const CUtensorMap tk = fp8 ? kv_map(k8.data(), st[1]) : kv_map(k.data(), st[1]);
+  const CUtensorMap tv = fp8 ? kv_map(v8.data(), st[2]) : kv_map(v.data(), st[2]);
   std::printf("plan rows=%d row_blocks=%d n_splits=%d chunk=%d key_begin=%d ctas=%lld ws=%zu\n", pl.rows,
               pl.row_blocks, pl.n_splits, pl.chunk, pl.key_begin, pl.ctas, pl.ws_bytes);
   if (d == 256) {
     if (fp8)
-      emu_launch(unsigned(pl.ctas), kDecThreads, DecLayout<256, true>::kSmemBytes, [&] { fa_decode_kernel<256, true>(p); });
+      emu_launch(unsigned(pl.ctas), kDecThreads, DecLayout<256, true>::kSmemBytes, [&] { fa_decode_kernel<256, true>(tk, tv, p); }, dec_smem);
     else
-      emu_launch(unsigned(pl.ctas), kDecThreads, DecLayout<256>::kSmemBytes, [&] { fa_decode_kernel<256, false>(p); });
+      emu_launch(unsigned(pl.ctas), kDecThreads, DecLayout<256>::kSmemBytes, [&] { fa_decode_kernel<256, false>(tk, tv, p); }, dec_smem);
     if (pl.n_splits > 1)
       emu_launch(unsigned((pl.total_rows + kDecMergeWarps - 1) / kDecMergeWarps), 32 * kDecMergeWarps, 0,
                  [&] { fa_decode_merge_kernel<256>(p); });
   } else if (fp8 && d == 64) {
-    emu_launch(unsigned(pl.ctas), kDecThreads, DecLayout<64, true>::kSmemBytes, [&] { fa_decode_kernel<64, true>(p); });
+    emu_launch(unsigned(pl.ctas), kDecThreads, DecLayout<64, true>::kSmemBytes, [&] { fa_decode_kernel<64, true>(tk, tv, p); }, dec_smem);
     if (pl.n_splits > 1)
       emu_launch(unsigned((pl.total_rows + kDecMergeWarps - 1) / kDecMergeWarps), 32 * kDecMergeWarps, 0,
                  [&] { fa_decode_merge_kernel<64>(p); });
   } else if (fp8) {
     emu_launch(unsigned(pl.ctas), kDecThreads, DecLayout<128, true>::kSmemBytes,
-               [&] { fa_decode_kernel<128, true>(p); });
+               [&] { fa_decode_kernel<128, true>(tk, tv, p); }, dec_smem);
     if (pl.n_splits > 1)
       emu_launch(unsigned((pl.total_rows + kDecMergeWarps - 1) / kDecMergeWarps), 32 * kDecMergeWarps, 0,
                  [&] { fa_decode_merge_kernel<128>(p); });
   } else if (d == 64) {
-    emu_launch(unsigned(pl.ctas), kDecThreads, DecLayout<64>::kSmemBytes, [&] { fa_decode_kernel<64, false>(p); });
+    emu_launch(unsigned(pl.ctas), kDecThreads, DecLayout<64>::kSmemBytes, [&] { fa_decode_kernel<64, false>(tk, tv, p); }, dec_smem);
     if (pl.n_splits > 1)
       emu_launch(unsigned((pl.total_rows + kDecMergeWarps - 1) / kDecMergeWarps), 32 * kDecMergeWarps, 0,
                  [&] { fa_decode_merge_kernel<64>(p); });
   } else {
-    emu_launch(unsigned(pl.ctas), kDecThreads, DecLayout<128>::kSmemBytes, [&] { fa_decode_kernel<128, false>(p); });
+    emu_launch(unsigned(pl.ctas), kDecThreads, DecLayout<128>::kSmemBytes, [&] { fa_decode_kernel<128, false>(tk, tv, p); }, dec_smem);
     if (pl.n_splits > 1)
       emu_launch(unsigned((pl.total_rows + kDecMergeWarps - 1) / kDecMergeWarps), 32 * kDecMergeWarps, 0,
                  [&] { fa_decode_merge_kernel<128>(p); });

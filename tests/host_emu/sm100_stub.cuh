@@ -21,8 +21,7 @@
 // TMA and bulk copies likewise land only when some thread tests the barrier that tracks them,
 // so a consumer that reads shared memory or TMEM without waiting on the right barrier sees
 // stale (NaN-filled) data.  ldmatrix and mma.sync are emulated from the fragment layouts the PTX ISA
-// documents (m8n8 b16 matrices; m16n8k16 row.col bf16 with fp32 accumulators); cp.async
-// copies land at the issuing thread's wait_group (zero-fill when the source size is 0); ex2 / lg2 are std::exp2 / std::log2;
+// documents (m8n8 b16 matrices; m16n8k16 row.col bf16 with fp32 accumulators); ex2 / lg2 are std::exp2 / std::log2;
 // bf16 and f16 rounding is round-to-nearest-even (f16 with subnormals and overflow to
 // infinity); E4M3 codes decode by the format's definition (they are all f16 values).
 #pragma once
@@ -98,37 +97,6 @@ inline uint32_t bf16x2_to_f16x2_sat(uint32_t w) {
   return pack_f16x2(lo, hi);
 }
 inline unsigned char* dec_dyn_smem() { return g_blk->smem; }
-// cp.async: a thread's copies are grouped by its commits and land only at its own
-// cp.async.wait_group, oldest groups first (copies not yet committed are not waited for)
-struct CpAsyncState {
-  std::vector<std::function<void()>> open;
-  std::vector<std::vector<std::function<void()>>> committed;
-};
-inline thread_local CpAsyncState t_cp;
-inline void cp_async_16(void* dst, const void* src, int n) {
-  if (n != 16 && n != 0) { std::fprintf(stderr, "bad cp.async size %d\n", n); std::abort(); }
-  if (reinterpret_cast<uintptr_t>(dst) % 16) { std::fprintf(stderr, "cp.async destination not 16-byte aligned\n"); std::abort(); }
-#ifdef EMU_EAGER_COPIES
-  if (n == 16) std::memcpy(dst, src, 16);
-  else std::memset(dst, 0, 16);
-  return;
-#endif
-  t_cp.open.push_back([=] {
-    if (n == 16) std::memcpy(dst, src, 16);
-    else std::memset(dst, 0, 16);
-  });
-}
-inline void cp_async_commit() {
-  t_cp.committed.push_back(std::move(t_cp.open));
-  t_cp.open.clear();
-}
-template <int N>
-inline void cp_async_wait() {
-  while (t_cp.committed.size() > size_t(N)) {
-    for (auto& f : t_cp.committed.front()) f();
-    t_cp.committed.erase(t_cp.committed.begin());
-  }
-}
 // programmatic dependent launch: the emulation runs grids one after another, so both are no-ops
 inline void grid_dep_wait() {}
 inline void grid_dep_launch_dependents() {}
@@ -296,7 +264,8 @@ struct CUtensorMap {
   uint64_t dims[4];      // x (contiguous), rows, heads, batch (elements)
   uint64_t strides[3];   // bytes: rows, heads, batch
   uint32_t box_x, box_rows;
-  uint32_t esize = 2;    // bytes per element; box_x * esize is the 128-byte swizzle row
+  uint32_t esize = 2;      // bytes per element; box_x * esize is the 128-byte swizzle row
+  uint32_t swizzle = 128;  // 128: the 128-byte swizzle; 0: plain rows of box_x * esize bytes
 };
 inline void tma_prefetch_desc(const CUtensorMap*) {}
 inline uint32_t sw128(uint32_t addr) { return addr ^ (((addr >> 7) & 7u) << 4); }
@@ -332,8 +301,13 @@ inline void queue_copy(uint32_t bar, std::function<void()> f) {
 inline void tma_copy_now(uint32_t dst, CUtensorMap map, uint32_t bar, int x, int row, int head, int batch);
 inline void tma_load_rows(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int row, int head, int batch) {
   if ((x * int(map->esize)) % 16) { std::fprintf(stderr, "TMA x coordinate not 16-byte aligned\n"); std::abort(); }
-  if (map->box_x * map->esize != 128) { std::fprintf(stderr, "TMA box row is not 128 bytes\n"); std::abort(); }
-  smem_at(dst, size_t(map->box_rows) * 128);   // the destination must lie in shared memory
+  const uint32_t row_bytes = map->box_x * map->esize;
+  if (map->swizzle == 128 ? row_bytes != 128 : (map->swizzle != 0 || row_bytes % 16 != 0)) {
+    std::fprintf(stderr, "TMA box row does not fit the swizzle mode\n");
+    std::abort();
+  }
+  if (dst % (map->swizzle == 128 ? 1024u : 16u)) { std::fprintf(stderr, "TMA destination misaligned\n"); std::abort(); }
+  smem_at(dst, size_t(map->box_rows) * row_bytes);   // the destination must lie in shared memory
   const CUtensorMap m = *map;
   BlockCtx* blk = g_blk;
   queue_copy(bar, [=] {
@@ -354,7 +328,8 @@ inline void tma_copy_now(uint32_t dst, CUtensorMap mm, uint32_t bar, int x, int 
           uint64_t(gr) < map->dims[1] && uint64_t(head) < map->dims[2] && uint64_t(batch) < map->dims[3])
         std::memcpy(&val, map->base + uint64_t(batch) * map->strides[2] + uint64_t(head) * map->strides[1] +
                               uint64_t(gr) * map->strides[0] + uint64_t(gx) * es, es);
-      std::memcpy(smem_at(sw128(dst + r * 128 + c * es), es), &val, es);
+      const uint32_t at = dst + r * map->box_x * es + c * es;
+      std::memcpy(smem_at(map->swizzle == 128 ? sw128(at) : at, es), &val, es);
     }
   bar_complete_tx(bar, map->box_x * map->box_rows * map->esize);
 }

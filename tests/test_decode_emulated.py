@@ -1,8 +1,8 @@
 """The decode kernels' own CUDA source, run on the CPU under a SIMT emulation, vs the oracle.
 
 Test infrastructure only.  tests/host_emu/ holds a host stand-in for the handful of device
-primitives decode_kernel.cuh uses (barriers, warp shuffles, cp.async, ldmatrix and the
-m16n8k16 MMA, emulated from their documented semantics).  The kernel source is compiled with
+primitives decode_kernel.cuh uses (barriers, warp shuffles, mbarriers, TMA tensor loads,
+ldmatrix and the m16n8k16 MMA, emulated from their documented semantics).  The kernel source is compiled with
 g++ under AddressSanitizer and UndefinedBehaviorSanitizer, so every global or shared-memory
 access outside its buffer aborts the run; outputs start as NaN, so a row the kernels fail to
 write fails the comparison.  This checks the kernels' index arithmetic, masks, split plan
@@ -139,13 +139,13 @@ def test_decode_kernel_emulated_strided(emu_binary):
 @pytest.mark.parametrize("B,H,H_kv,N_q,N_k,d,causal,window", [
     (2, 8, 2, 3, 1000, 128, True, 0), (1, 2, 1, 5, 777, 64, False, 50), (1, 4, 1, 2, 700, 256, True, 0)])
 def test_decode_kernel_emulated_eager_copies(emu_binary_eager, B, H, H_kv, N_q, N_k, d, causal, window):
-    """cp.async copies that land as soon as they are issued: a lane refilling a ring stage that
-    another lane of its warp still reads would overwrite those keys."""
+    """TMA copies that land as soon as they are issued: a load refilling a ring stage that a
+    lane of the warp still reads would overwrite those keys."""
     wl = Workload("decode_emu", B, H, N_k, d, causal, window, seed=71 + N_k + N_q, H_kv=H_kv, Nq=N_q)
     _run(emu_binary_eager, wl)
 
 
 def test_decode_fp8kv_kernel_emulated_eager_copies(emu_binary_eager):
-    """The FP8 K/V path (raw E4M3 ring, converted tiles) with cp.async copies landing at issue."""
+    """The FP8 K/V path (raw E4M3 ring, converted tiles) with TMA copies landing at issue."""
     wl = Workload("decode_fp8_emu", 2, 8, 1000, 128, True, 0, seed=81 + 1000 + 3, H_kv=2, Nq=3)
     _run(emu_binary_eager, wl, fp8=True)
