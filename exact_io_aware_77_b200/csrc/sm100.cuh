@@ -54,13 +54,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// The same test with an explicit bound on how long the thread may stay suspended in it: it
+// returns at the latest after about hint_ns, or when the phase completes.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait for the phase with the given parity to complete.  Returns false
-// (and raises *abort) if the CTA is aborting or the limit ran out.
+// (and raises *abort) if the CTA is aborting or the limit ran out.  The thread stays suspended
+// in each test for up to a microsecond rather than polling, so that a waiting warp (the TMA or
+// MMA issuer) leaves its SMSP's issue slots to the warps that share it.
 __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort,
                                             uint64_t limit_ns) {
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_suspend(bar, parity, 1000u)) return true;
     if ((it & 63u) == 0) {
       if (*abort) return false;
       if (global_timer_ns() - t0 > limit_ns) {
