@@ -427,7 +427,7 @@ def run_ours(args):
     else:
         dom, dom_flops, dom_ms = names[0], f_fwd, fwd_ms_avg
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12
-    # a long timed region runs under the power cap: its kernel is judged against the sustained peak
+    # a long timed region runs under the power cap: its kernel is compared with the sustained peak
     sustained = step_ms_total >= SUSTAINED_MS
     peak = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
     roofline = {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 1),

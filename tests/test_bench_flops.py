@@ -48,7 +48,7 @@ def _roof(achieved):
 
 
 def test_regime_fields_burst_and_sustained():
-    """A timed region under 1 s is judged against the burst peak, a longer one against the
+    """A timed region under 1 s is compared with the burst peak, a longer one with the
     sustained peak; both fractions and the clock-normalised kernel time are reported."""
     peaks = {"bf16_tflops": 1636.3, "bf16_tflops_sustained": 1375.0}
     clocks = {"sm_mhz": 1732.0, "sm_max_mhz": 1965.0, "samples": 13}
