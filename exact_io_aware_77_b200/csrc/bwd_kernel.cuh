@@ -550,9 +550,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       }
     }
-    // every reduction this warp issued has finished (its slot read, its adds done) before the
-    // CTA's shared memory is released
-    if (lane == 0) bulk_wait_group<0>();
+    // every reduction this warp issued has read its slot before the CTA's shared memory is
+    // released (the adds complete with the grid, before the finalise kernel runs)
+    if (lane == 0) bulk_wait_group_read<0>();
     __syncwarp();
   }
 

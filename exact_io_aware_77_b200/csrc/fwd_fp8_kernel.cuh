@@ -131,6 +131,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const int bw[2] = {b0, b1}, ew[2] = {e0, e1};
     auto active = [&](int w, int t) { return t >= bw[w] && t < ew[w]; };
     int pv_count[2] = {0, 0};
+    bool o_done[2] = {false, false};   // o_final committed (right after the tile's last P V)
     const uint64_t dq[2] = {sw128_desc(smem_u32(sm.q[0]), 16, 1024), sw128_desc(smem_u32(sm.q[1]), 16, 1024)};
     const uint64_t dp[2] = {sw128_desc(smem_u32(sm.p[0]), 16, 1024), sw128_desc(smem_u32(sm.p[1]), 16, 1024)};
     const uint64_t dkv0 = sw128_desc(smem_u32(sm.kv[0]), 16, 1024);
@@ -176,6 +177,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           }
           tc_fence_after();
           issue_pv(w, Lv % kSlots);
+          if (t + 1 == ew[w]) {
+            // the tile's O is final once this P V completes: its epilogue overlaps the other
+            // tile's last steps
+            mma_commit_w(smem_u32(&sm.o_final[w]));
+            o_done[w] = true;
+          }
         }
         if (has_next && active(w, t + 1)) issue_s(w, Lk % kSlots);
       }
@@ -184,7 +191,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mma_commit_w(smem_u32(&sm.slot_empty[Lv % kSlots]));
     }
 #pragma unroll
-    for (int w = 0; w < kQTiles; ++w) mma_commit_w(smem_u32(&sm.o_final[w]));
+    for (int w = 0; w < kQTiles; ++w)
+      if (!o_done[w]) mma_commit_w(smem_u32(&sm.o_final[w]));   // a tile without keys, or after an abort
     mma_commit_w(smem_u32(&sm.mma_drain));
     mbar_wait_drain(smem_u32(&sm.mma_drain), 0, lim);
   } else {

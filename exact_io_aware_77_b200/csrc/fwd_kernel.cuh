@@ -30,7 +30,9 @@
 // PV(j-1) of the same tile has completed: a rescale never races an MMA, and S(j+1) may be
 // issued right behind PV(j) although it overwrites the TMEM columns PV(j) reads P from.
 // TMEM columns: S0 [0,128), S1 [128,256), O0 [256, 256+D), O1 [384, 384+D); P_w occupies
-// the first 64 columns of S_w.
+// the first 64 columns of S_w.  A tile's O is final (o_final) right after its own last P V, so
+// its epilogue overlaps the other tile's last steps (under the causal mask the second tile
+// has one more key tile than the first).
 #pragma once
 
 #include <type_traits>
@@ -206,6 +208,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const int bw[2] = {b0, b1}, ew[2] = {e0, e1};
       auto active = [&](int w, int t) { return t >= bw[w] && t < ew[w]; };
       int pv_count[2] = {0, 0};
+      bool o_done[2] = {false, false};   // o_final committed (right after the tile's last P V)
       // descriptors are built once; each k-step only adds a constant to the start field
       const uint64_t dq[2] = {sw128_desc(smem_u32(sm.q[0]), 16, 1024), sw128_desc(smem_u32(sm.q[1]), 16, 1024)};
       const uint64_t dkv0 = sw128_desc(smem_u32(sm.kv[0]), 16, 1024);
@@ -260,6 +263,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             }
             tc_fence_after();
             issue_pv(w, Lv % kSlots);
+            if (t + 1 == ew[w]) {
+              // the tile's O is final once this P V completes: its softmax warps start the
+              // epilogue while the other tile's last steps run
+              mma_commit_w(smem_u32(&sm.o_final[w]));
+              o_done[w] = true;
+            }
           }
           if (has_next && active(w, t + 1)) issue_s(w, Lk % kSlots);
         }
@@ -268,7 +277,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         mma_commit_w(smem_u32(&sm.slot_empty[Lv % kSlots]));
       }
 #pragma unroll
-      for (int w = 0; w < kQTiles; ++w) mma_commit_w(smem_u32(&sm.o_final[w]));
+      for (int w = 0; w < kQTiles; ++w)
+        if (!o_done[w]) mma_commit_w(smem_u32(&sm.o_final[w]));   // a tile without keys, or after an abort
       // every MMA issued above completes before TMEM is released
       mma_commit_w(smem_u32(&sm.mma_drain));
       mbar_wait_drain(smem_u32(&sm.mma_drain), 0, lim);
@@ -486,7 +496,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
         for (int c = 0; c < Smem::kChunks; ++c) tma_store_rows(&tm_o, stage + c * 16384, c * 64, qw0, h_q, b_idx);
         bulk_commit_group();
-        bulk_wait_group<0>();   // the rows are read (and written) before the CTA's shared memory is released
+        // the rows are read before the CTA's shared memory is released (the writes to global
+        // memory complete with the grid)
+        bulk_wait_group_read<0>();
       }
     }
   }
