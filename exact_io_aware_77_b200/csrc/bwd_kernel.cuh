@@ -31,7 +31,8 @@
 //               each block added into the fp32 accumulator by one TMA tensor reduction
 //               (cp.reduce.async.bulk.tensor .add), so that the adds leave the SM as whole
 //               128-byte lines and no warp waits for them.
-//               Order per tile: B(i), A(i+1), readout(i).  At the end: dK (half 0), dV (half 1).
+//               Order per tile: B(i), A(i+1), readout(i).  At the end: dK (half 0), dV (half 1),
+//               staged in the idle Q buffers and written by TMA tensor stores.
 // TMEM columns: dK [0,128), dV [128,256), S^T [256,384) with P^T in [256,288) and [320,352)
 // once read, dP^T [384,512) with dS^T in [384,416) and [448,480) once read, and dQ in
 // [384,512).  MMAs of one thread
@@ -174,12 +175,14 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_final(const float* __restrict__
 
 // ----------------------------------------------------------------------------- main kernel
 // tm_dq: the fp32 accumulator [BH, Np, D] as the 4-D tensor (D, Np, BH, 1), 32 x 32 boxes with
-// the 128-byte swizzle (the layout of a compute warp's staging slot).
+// the 128-byte swizzle (the layout of a compute warp's staging slot).  tm_dk, tm_dv: dK and dV
+// as (D, N, H_kv, B), boxes of 64 columns x 32 rows (one compute warp's key rows).
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                  const __grid_constant__ CUtensorMap tm_dq, const BwdParams prm) {
+                  const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ CUtensorMap tm_dk,
+                  const __grid_constant__ CUtensorMap tm_dv, const BwdParams prm) {
   using Smem = BwdSmem<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // the layout fills almost all 227 KB, so no slack is left for realigning the base
@@ -234,6 +237,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     tma_prefetch_desc(&tm_v);
     tma_prefetch_desc(&tm_do);
     tma_prefetch_desc(&tm_dq);
+    tma_prefetch_desc(&tm_dk);
+    tma_prefetch_desc(&tm_dv);
   }
   if (warp == kBwdWarpMma) {
     tmem_alloc(smem_u32(&sm.tmem_base), 512);
@@ -526,15 +531,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (it + 1 < n_it && !run_a(it + 1)) { ok = false; break; }
       if (!readout(it)) { ok = false; break; }
     }
-    // epilogue: warps of query half 0 write dK = scale * acc, those of half 1 write dV = acc
+    // epilogue: warps of query half 0 write dK = scale * acc, those of half 1 write dV = acc.
+    // My 32 key rows, as bf16, go to the Q buffers (idle once every MMA has completed) in the
+    // layout of 32-row TMA boxes (64 columns of 128-byte swizzled rows each), and lane 0 writes
+    // them with TMA tensor stores, which skip the rows past N.
     if (ok && __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.mma_final), 0, abort, lim))) {
       tc_fence_after();
-      const bool in_range = key < prm.N;
-      const int krow = in_range ? key : 0;
-      __nv_bfloat16* dst_row = hq == 0 ? prm.dk + prm.dk_st.at(b_idx, h_kv, krow)
-                                       : prm.dv + prm.dv_st.at(b_idx, h_kv, krow);
       const float mul = hq == 0 ? prm.scale : 1.f;
       const uint32_t col0 = hq == 0 ? kTdK : kTdV;
+      const uint32_t out = smem_u32(sm.q[warp >> 2]) + uint32_t(warp & 3) * (D / 64) * 4096;
 #pragma unroll
       for (int ch = 0; ch < D / 32; ++ch) {
         uint32_t rr[32];
@@ -543,15 +548,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int j = 0; j < 16; ++j)
           w[j] = pack_bf16x2(__uint_as_float(rr[2 * j]) * mul, __uint_as_float(rr[2 * j + 1]) * mul);
-        if (in_range) {
-          uint4* dst = reinterpret_cast<uint4*>(dst_row + ch * 32);
+        // columns 32 ch .. : 16-byte pieces 4 (ch & 1) .. of row `lane` in box ch / 2
+        const uint32_t row = out + uint32_t(ch >> 1) * 4096 + uint32_t(lane) * 128;
 #pragma unroll
-          for (int j = 0; j < 4; ++j) dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
-        }
+        for (int j = 0; j < 4; ++j)
+          st_shared_v4(row + ((((ch & 1) * 4 + j) ^ (lane & 7)) << 4), w[4 * j], w[4 * j + 1], w[4 * j + 2],
+                       w[4 * j + 3]);
+      }
+      fence_proxy_async_smem();   // the tensor stores read the boxes through the async proxy
+      __syncwarp();
+      if (lane == 0) {
+#pragma unroll
+        for (int bx = 0; bx < D / 64; ++bx)
+          tma_store_rows(hq == 0 ? &tm_dk : &tm_dv, out + bx * 4096, bx * 64, kv0 + quad * 32, h_kv, b_idx);
+        bulk_commit_group();
       }
     }
-    // every reduction this warp issued has read its slot before the CTA's shared memory is
-    // released (the adds complete with the grid, before the finalise kernel runs)
+    // every reduction and store this warp issued has read its shared memory before the CTA's
+    // shared memory is released (the writes complete with the grid, before the finalise kernel)
     if (lane == 0) bulk_wait_group_read<0>();
     __syncwarp();
   }

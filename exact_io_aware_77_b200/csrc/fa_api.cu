@@ -319,12 +319,14 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   } else {
     static_assert(sizeof(BwdSmem<D>) <= 232448, "backward shared memory exceeds 227 KB");
     const int smem = int(sizeof(BwdSmem<D>));   // the kernel checks that the base is 1 KB aligned
-    CUtensorMap tdq;
-    if (!make_map_dq_acc(&tdq, dq_acc, D, Np, BH)) return FA_ERR_CUDA;
+    CUtensorMap tdq, tdk, tdv;
+    if (!make_map_dq_acc(&tdq, dq_acc, D, Np, BH) || !make_map_bf16(&tdk, dk, D, N, H_kv, B, st[6], 32) ||
+        !make_map_bf16(&tdv, dv, D, N, H_kv, B, st[7], 32))
+      return FA_ERR_CUDA;
     if (set_smem(fa_bwd_kernel<D>, smem) != FA_OK) return FA_ERR_CUDA;
     // one CTA per (K/V head, key tile)
     fa_bwd_kernel<D><<<unsigned(prm.n_kv_tiles) * unsigned(BH_kv), kBwdThreads, smem, stream>>>(tq, tk, tv, tdo,
-                                                                                                   tdq, prm);
+                                                                                                   tdq, tdk, tdv, prm);
   }
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }

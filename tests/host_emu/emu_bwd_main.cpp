@@ -106,6 +106,8 @@ int main(int argc, char** argv) {
   tdq.box_x = 32;
   tdq.box_rows = 32;
   tdq.esize = 4;
+  // dK and dV as (D, N, H_kv, B), 32-row boxes (the backward's TMA-store epilogue)
+  const CUtensorMap tdk = make_map(dk.data(), D, N, Hkv, B, 32), tdv = make_map(dv.data(), D, N, Hkv, B, 32);
   BwdParams prm;
   prm.lp = lp;
   prm.dd = dd;
@@ -131,7 +133,7 @@ int main(int argc, char** argv) {
              [&] { fa_bwd256_kernel(tq, tk, tv, tdo, tdq, prm); }, fa::smem_raw);
 #else
   emu_launch(unsigned(prm.n_kv_tiles) * unsigned(BH_kv), kBwdThreads, sizeof(fa::smem_raw),
-             [&] { fa_bwd_kernel<D>(tq, tk, tv, tdo, tdq, prm); }, fa::smem_raw);
+             [&] { fa_bwd_kernel<D>(tq, tk, tv, tdo, tdq, tdk, tdv, prm); }, fa::smem_raw);
 #endif
   if (g_status != 0) { std::fprintf(stderr, "device status %d\n", g_status); return 3; }
   const long long rows = (long long)BH * N;
