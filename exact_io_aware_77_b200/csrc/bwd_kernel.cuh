@@ -14,10 +14,10 @@
 //   fa_bwd_kernel    one CTA per 128-key tile of one head; loops over 128-row query tiles.
 //   fa_bwd_dq_final  dQ = scale * accumulator, rounded to bf16.
 //
-// fa_bwd_kernel roles (320 threads), every MMA 128 x 128 (narrower ones cost as much time):
-//   warp 8      TMA producer: K, V once; Q_i (+ its L and D rows) into a 2-stage ring, dO_i into
+// fa_bwd_kernel roles (512 threads), every MMA 128 x 128 (narrower ones cost as much time):
+//   warp 12     TMA producer: K, V once; Q_i (+ its L and D rows) into a 2-stage ring, dO_i into
 //               one stage.
-//   warp 9      MMA issuer, per query tile i in the order
+//   warp 13     MMA issuer, per query tile i in the order
 //                 dV += P_i^T dO_i, S_{i+1}^T = K Q_{i+1}^T, dK += dS_i^T Q_i, dQ_i = dS_i K,
 //                 dP_{i+1}^T = V dO_{i+1}^T
 //               (dV and dK read their A operand from TMEM), so that the exponentials of tile
@@ -26,18 +26,21 @@
 //   warps 0-7   two per TMEM lane quadrant; warp w owns lanes 32 (w % 4).. and the query half
 //               w / 4 of each tile.  Phase A: P^T = exp2(S^T c - L) with the causal/window mask,
 //               stored to TMEM as bf16.  Phase B: dS^T = P^T o (dP^T - D) to TMEM (A of dK) and
-//               to shared memory (A of dQ).  Readout: its half of the dQ_i rows of its 32
-//               queries, from TMEM into its shared-memory staging slot, 32 columns at a time,
-//               each block added into the fp32 accumulator by one TMA tensor reduction
-//               (cp.reduce.async.bulk.tensor .add), so that the adds leave the SM as whole
-//               128-byte lines and no warp waits for them.
-//               Order per tile: B(i), A(i+1), readout(i).  At the end: dK (half 0), dV (half 1),
-//               staged in the idle Q buffers and written by TMA tensor stores.
+//               to shared memory (A of dQ).  Order per tile: B(i), A(i+1).  At the end: dK
+//               (half 0), dV (half 1), staged in the idle Q buffers and written by TMA tensor
+//               stores.
+//   warps 8-11  dQ readout, one per TMEM lane quadrant: all D columns of its 32 query rows of
+//               dQ_i from TMEM as soon as the product completes, then 32 columns at a time
+//               through two shared-memory staging slots, each block added into the fp32
+//               accumulator by one TMA tensor reduction (cp.reduce.async.bulk.tensor .add), so
+//               that the adds leave the SM as whole 128-byte lines and no warp waits for them.
+//   warps 14-15 none (they complete the last warpgroup, whose registers go to the others:
+//               setmaxnreg moves them from the TMA/MMA warpgroup to the compute and readout ones).
 // TMEM columns: dK [0,128), dV [128,256), S^T [256,384) with P^T in [256,288) and [320,352)
 // once read, dP^T [384,512) with dS^T in [384,416) and [448,480) once read, and dQ in
 // [384,512).  MMAs of one thread
 // run in order, which makes each reuse safe: S_{i+1} is issued after dV_i read P_i, dQ_i after
-// dK_i read dS_i; only dP_{i+1} waits until the compute warps have read dQ_i out.
+// dK_i read dS_i; only dP_{i+1} waits until the readout warps have read dQ_i out.
 #pragma once
 
 #include <type_traits>
@@ -50,9 +53,25 @@ namespace fa {
 constexpr int kBwdKeys = 128;    // keys per CTA
 constexpr int kBwdRows = 128;    // queries per iteration
 constexpr int kBwdQStages = 2;
-constexpr int kBwdThreads = 320;   // 8 compute warps, TMA, MMA
-constexpr int kBwdWarpTma = 8;
-constexpr int kBwdWarpMma = 9;
+constexpr int kBwdThreads = 512;   // 8 compute warps, 4 dQ readout warps, TMA, MMA and 2 idle warps
+constexpr int kBwdWarpRead = 8;    // warps 8-11: the dQ readout, one per TMEM lane quadrant
+constexpr int kBwdWarpTma = 12;
+constexpr int kBwdWarpMma = 13;    // warps 14-15 complete the TMA/MMA warpgroup and do nothing
+// Registers per thread: 128 at launch (512 threads share the SM's 64K); the compute warpgroups
+// raise themselves to kBwdRegsCompute and the readout warpgroup to kBwdRegsRead out of what the
+// TMA/MMA warpgroup gives back by lowering itself to kBwdRegsOther.
+constexpr int kBwdLaunchRegs = 65536 / kBwdThreads;
+constexpr int kBwdRegsCompute = 160;
+constexpr int kBwdRegsRead = 88;
+constexpr int kBwdRegsOther = 4 * kBwdLaunchRegs - 2 * kBwdRegsCompute - kBwdRegsRead;
+static_assert(kBwdRegsOther >= 24 && kBwdRegsOther % 8 == 0 &&
+                  2 * kBwdRegsCompute + kBwdRegsRead + kBwdRegsOther <= 4 * kBwdLaunchRegs,
+              "the warpgroups' register budgets must fit in the launch share");
+// setmaxnreg.inc may only raise a warp's count and .dec only lower it: the compute warpgroups
+// raise, the readout and TMA/MMA warpgroups lower
+static_assert(kBwdRegsCompute >= kBwdLaunchRegs && kBwdRegsRead <= kBwdLaunchRegs &&
+                  kBwdRegsOther <= kBwdLaunchRegs,
+              "each warpgroup's budget moves in the direction of its setmaxnreg form");
 constexpr uint32_t kTdK = 0, kTdV = 128, kTS = 256, kTP = 256, kTdP = 384, kTdS = 384, kTdQ = 384;
 constexpr int FA_DEVICE_SMEM_ALIGN = 2;   // status bit: dynamic shared memory not 1 KB aligned
 
@@ -79,7 +98,7 @@ struct BwdSmem {
   alignas(1024) uint8_t q[kBwdQStages][kTileBytes];
   alignas(1024) uint8_t dout[kTileBytes];                  // one stage: see the producer
   alignas(1024) uint8_t ds[kBwdKeys * kBwdRows * 2];       // dS^T: [key][query], 64-query chunks
-  alignas(1024) uint8_t stage[8][32 * 32 * 4];             // dQ staging: 32 rows x 32 fp32 per compute warp
+  alignas(1024) uint8_t stage[8][32 * 32 * 4];             // dQ staging: 32 rows x 32 fp32, two per readout warp
                                                            // (1 KB aligned: the 128-byte swizzle's atoms)
   alignas(16) float lp[kBwdQStages][kBwdRows];
   alignas(16) float dd[kBwdQStages][kBwdRows];
@@ -224,7 +243,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(smem_u32(&sm.pa_full), 256);
     mbar_init(smem_u32(&sm.ds_full), 256);
     mbar_init(smem_u32(&sm.dq_full), 1);
-    mbar_init(smem_u32(&sm.dq_free), 256);
+    mbar_init(smem_u32(&sm.dq_free), 128);   // the four readout warps
     mbar_init(smem_u32(&sm.mma_final), 1);
     mbar_init(smem_u32(&sm.mma_drain), 1);
     mbar_init(smem_u32(&sm.do_full), 1);
@@ -249,6 +268,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
 
+  if (warp >= kBwdWarpTma) {
+  regs_lower<kBwdRegsOther>();
   if (warp == kBwdWarpTma) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -268,7 +289,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t ph = (it / kBwdQStages) & 1;
         const int q0 = q_tile(it) * kBwdRows;
         const int bq = q_head(it);
-        if (!mbar_wait(smem_u32(&sm.q_empty[qs]), ph ^ 1, abort, lim)) break;
+        if (!mbar_wait_inl(smem_u32(&sm.q_empty[qs]), ph ^ 1, abort, lim)) break;
         const uint32_t qb = smem_u32(&sm.q_full[qs]);
         mbar_expect_tx(qb, Smem::kTileBytes + 2 * kBwdRows * 4);
         for (int c = 0; c < Smem::kChunks; ++c)
@@ -277,24 +298,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         bulk_load(smem_u32(sm.lp[qs]), prm.lp + row, kBwdRows * 4, qb);
         bulk_load(smem_u32(sm.dd[qs]), prm.dd + row, kBwdRows * 4, qb);
         issued = it + 1;
-        if (!mbar_wait(smem_u32(&sm.do_empty), (it & 1) ^ 1, abort, lim)) break;
+        if (!mbar_wait_inl(smem_u32(&sm.do_empty), (it & 1) ^ 1, abort, lim)) break;
         const uint32_t db = smem_u32(&sm.do_full);
         mbar_expect_tx(db, Smem::kTileBytes);
         for (int c = 0; c < Smem::kChunks; ++c)
           tma_load_rows(smem_u32(sm.dout) + c * 16384, &tm_do, db, c * 64, q0, bq - b_idx * prm.H, b_idx);
         issued_do = it + 1;
       }
-      mbar_wait_drain(kvb, 0, lim);
+      mbar_wait_drain_inl(kvb, 0, lim);
       for (int it = max(0, issued - kBwdQStages); it < issued; ++it)
-        mbar_wait_drain(smem_u32(&sm.q_full[it % kBwdQStages]), (it / kBwdQStages) & 1, lim);
-      if (issued_do > 0) mbar_wait_drain(smem_u32(&sm.do_full), (issued_do - 1) & 1, lim);
+        mbar_wait_drain_inl(smem_u32(&sm.q_full[it % kBwdQStages]), (it / kBwdQStages) & 1, lim);
+      if (issued_do > 0) mbar_wait_drain_inl(smem_u32(&sm.do_full), (issued_do - 1) & 1, lim);
     }
   } else if (warp == kBwdWarpMma) {
     // ------------------------------------------------------------------ MMA issuer
     // the whole warp runs this loop (uniformly); each tcgen05 op is issued by one elected lane
     {
       auto wait = [&](uint32_t bar, uint32_t parity) {
-        return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, lim));
+        return __all_sync(0xffffffffu, mbar_wait_inl(bar, parity, abort, lim));
       };
       constexpr uint32_t idesc_t = idesc_bf16_f32(128, kBwdRows, false, false);   // S^T, dP^T
       constexpr uint32_t idesc_kv = idesc_bf16_f32(128, D, false, true);          // dV, dK (A in TMEM)
@@ -371,9 +392,62 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       mma_commit_w(smem_u32(&sm.mma_final));
       mma_commit_w(smem_u32(&sm.mma_drain));
-      mbar_wait_drain(smem_u32(&sm.mma_drain), 0, lim);
+      mbar_wait_drain_inl(smem_u32(&sm.mma_drain), 0, lim);
     }
-  } else if (warp < 8) {
+  }
+  } else if (warp >= kBwdWarpRead) {
+    regs_lower<kBwdRegsRead>();
+    // ------------------------------------------------------------------ dQ readout warps
+    // One warp per TMEM lane quadrant (query rows 32 q .. of a tile): its rows of dQ_i from TMEM
+    // into registers as soon as the product completes, then 32 columns at a time through its
+    // two 4 KB staging slots, in the 128-byte swizzled layout, into the fp32 accumulator, one
+    // TMA tensor reduction per block.
+    const int quad = warp & 3;
+    const uint32_t lane_base = uint32_t(quad * 32) << 16;
+    const uint32_t slot0 = smem_u32(sm.stage[2 * quad]), slot1 = smem_u32(sm.stage[2 * quad + 1]);
+    for (int it = 0; it < n_it; ++it) {
+      if (!__all_sync(0xffffffffu, mbar_wait_inl(smem_u32(&sm.dq_full), it & 1, abort, lim))) break;
+      tc_fence_after();
+      const int q_row = q_tile(it) * kBwdRows + quad * 32;   // my first query row of the tile
+      const int q_hd = q_head(it);
+      // 64 columns at a time (the registers the readout warpgroup has); the columns are free
+      // for dP_{i+1} once the last 64 are in registers
+#pragma unroll
+      for (int h = 0; h < D / 64; ++h) {
+        uint32_t v[64];
+        tmem_ld32_async(tmem + lane_base + kTdQ + h * 64, v);
+        tmem_ld32_async(tmem + lane_base + kTdQ + h * 64 + 32, v + 32);
+        tmem_ld_wait();
+        reg_fence<64>(v);
+        if (h == D / 64 - 1) {
+          tc_fence_before();
+          mbar_arrive(smem_u32(&sm.dq_free));
+        }
+#pragma unroll
+        for (int p2 = 0; p2 < 2; ++p2) {
+          const uint32_t slot = p2 ? slot1 : slot0;
+          if (lane == 0) bulk_wait_group_read<1>();   // the block before the previous one has left this slot
+          __syncwarp();
+          // row `lane`, 16-byte chunk c at lane * 128 + (c ^ (lane & 7)) * 16: the 128-byte swizzle
+#pragma unroll
+          for (int c16 = 0; c16 < 8; ++c16)
+            st_shared_v4(slot + lane * 128 + ((c16 ^ (lane & 7)) << 4), v[32 * p2 + 4 * c16],
+                         v[32 * p2 + 4 * c16 + 1], v[32 * p2 + 4 * c16 + 2], v[32 * p2 + 4 * c16 + 3]);
+          fence_proxy_async_smem();   // the tensor reduction reads the slot through the async proxy
+          __syncwarp();
+          if (lane == 0) {
+            tma_reduce_add_rows(&tm_dq, slot, 64 * h + 32 * p2, q_row, q_hd, 0);
+            bulk_commit_group();
+          }
+        }
+      }
+    }
+    // every reduction this warp issued has read its slot before the CTA's shared memory is
+    // released (the adds complete with the grid, before the finalise kernel runs)
+    if (lane == 0) bulk_wait_group_read<0>();
+    __syncwarp();
+  } else {
+    regs_raise<kBwdRegsCompute>();
     // ------------------------------------------------------------------ compute warps
     // Two warps per TMEM lane quadrant: warp w owns lanes 32 (w % 4) .. (keys for S^T, dP^T;
     // queries for dQ) and query half hq = w / 4 (queries 64 hq .. 64 hq + 63 of each tile).
@@ -385,7 +459,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const float c = prm.scale_log2;
     const uint32_t col_s = kTS + hq * 64;      // my S^T columns; P^T goes to the first 32 of them
     const uint32_t col_dp = kTdP + hq * 64;    // my dP^T columns; dS^T goes to the first 32 of them
-    const uint32_t col_dq = kTdQ + hq * (D / 2);
     const uint32_t ds_row = smem_u32(sm.ds) + hq * 16384 + r * 128;   // 64 queries = one 128-byte row
     const uint32_t sw = r & 7;
     uint32_t pk[32];                           // packed P^T of the current tile (phase A -> phase B)
@@ -398,8 +471,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     auto phase_a = [&](int it, auto masked) -> bool {
       const int qs = it % kBwdQStages;
       const int q0 = q_tile(it) * kBwdRows;
-      bool w_ok = mbar_wait(smem_u32(&sm.q_full[qs]), (it / kBwdQStages) & 1, abort, lim);
-      w_ok = w_ok && mbar_wait(smem_u32(&sm.s_full), it & 1, abort, lim);
+      bool w_ok = mbar_wait_inl(smem_u32(&sm.q_full[qs]), (it / kBwdQStages) & 1, abort, lim);
+      w_ok = w_ok && mbar_wait_inl(smem_u32(&sm.s_full), it & 1, abort, lim);
       if (!__all_sync(0xffffffffu, w_ok)) return false;
       tc_fence_after();
       uint32_t sr[64];
@@ -446,9 +519,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // phase B: dS^T = P^T o (dP^T - D) for my 64 queries -> TMEM (bf16) and shared memory
     auto phase_b = [&](int it) -> bool {
       const int qs = it % kBwdQStages;
-      // my rows of the dS buffer are free: the readout of the previous tile, earlier in this
-      // warp's program, waited for the dQ MMA that read them
-      const bool w_ok = mbar_wait(smem_u32(&sm.dp_full), it & 1, abort, lim);
+      // my rows of the dS buffer are free: dP of this tile completing means every earlier MMA
+      // has, the dQ product that read the previous tile's dS among them
+      const bool w_ok = mbar_wait_inl(smem_u32(&sm.dp_full), it & 1, abort, lim);
       if (!__all_sync(0xffffffffu, w_ok)) return false;
       tc_fence_after();
       uint32_t dr[64];
@@ -480,43 +553,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_arrive(smem_u32(&sm.ds_full));
       return true;
     };
-    // dQ readout: my 32 query rows, head-dim columns D/2 hq ...  In passes of 32 columns the
-    // block goes from TMEM into my 4 KB staging slot, and lane 0 adds it into the accumulator
-    // with one TMA tensor reduction.  Before the slot is written again, lane 0 waits until the
-    // previous reduction has read it (it has had a whole pass, or a tile, to do so).
-    const uint32_t stage = smem_u32(sm.stage[warp]);
-    auto readout = [&](int it) -> bool {
-      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.dq_full), it & 1, abort, lim))) return false;
-      tc_fence_after();
-      uint32_t v[D / 2];
-#pragma unroll
-      for (int ch = 0; ch < D / 64; ++ch) tmem_ld32_async(tmem + lane_base + col_dq + ch * 32, v + ch * 32);
-      tmem_ld_wait();
-      reg_fence<D / 2>(v);
-      tc_fence_before();
-      mbar_arrive(smem_u32(&sm.dq_free));
-      const int q_row = q_tile(it) * kBwdRows + quad * 32;   // my first query row of the tile
-      const int q_hd = q_head(it);
-#pragma unroll
-      for (int ps = 0; ps < D / 64; ++ps) {
-        if (lane == 0) bulk_wait_group_read<0>();
-        __syncwarp();
-        // row `lane`, 16-byte chunk c at lane * 128 + (c ^ (lane & 7)) * 16: the 128-byte swizzle
-#pragma unroll
-        for (int c16 = 0; c16 < 8; ++c16)
-          st_shared_v4(stage + lane * 128 + ((c16 ^ (lane & 7)) << 4), v[32 * ps + 4 * c16],
-                       v[32 * ps + 4 * c16 + 1], v[32 * ps + 4 * c16 + 2], v[32 * ps + 4 * c16 + 3]);
-        fence_proxy_async_smem();   // the tensor reduction reads the slot through the async proxy
-        __syncwarp();
-        if (lane == 0) {
-          tma_reduce_add_rows(&tm_dq, stage, hq * (D / 2) + 32 * ps, q_row, q_hd, 0);
-          bulk_commit_group();
-        }
-      }
-      return true;
-    };
-
-    // order: B(i), A(i+1), R(i): the dQ readout of tile i hides behind the exponentials of i+1
+    // order: B(i), A(i+1); the readout warps take dQ_i out of TMEM meanwhile
     // phase A masks only on the diagonal, the window's far edge and the tail key tile
     auto run_a = [&](int it) -> bool {
       const int qbase = q_tile(it) * kBwdRows + hq * 64;
@@ -529,13 +566,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int it = 0; ok && it < n_it; ++it) {
       if (!phase_b(it)) { ok = false; break; }
       if (it + 1 < n_it && !run_a(it + 1)) { ok = false; break; }
-      if (!readout(it)) { ok = false; break; }
     }
     // epilogue: warps of query half 0 write dK = scale * acc, those of half 1 write dV = acc.
     // My 32 key rows, as bf16, go to the Q buffers (idle once every MMA has completed) in the
     // layout of 32-row TMA boxes (64 columns of 128-byte swizzled rows each), and lane 0 writes
     // them with TMA tensor stores, which skip the rows past N.
-    if (ok && __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.mma_final), 0, abort, lim))) {
+    if (ok && __all_sync(0xffffffffu, mbar_wait_inl(smem_u32(&sm.mma_final), 0, abort, lim))) {
       tc_fence_after();
       const float mul = hq == 0 ? prm.scale : 1.f;
       const uint32_t col0 = hq == 0 ? kTdK : kTdV;

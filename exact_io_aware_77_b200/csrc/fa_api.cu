@@ -133,6 +133,22 @@ int check_device() {
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// A kernel that moves registers between its warpgroups (setmaxnreg) must be launched with at
+// least `regs` registers per thread: the raised budgets come out of the launch share, and a raise
+// the CTA cannot cover would wait forever.  Checked once per kernel and device.
+template <class Kernel>
+int check_launch_regs(Kernel k, int regs) {
+  static int cache[kMaxDevices] = {0};   // 0 unknown, 1 ok, 2 too few
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+  if (cache[dev] == 0) {
+    cudaFuncAttributes a;
+    if (cudaFuncGetAttributes(&a, k) != cudaSuccess) return FA_ERR_CUDA;
+    cache[dev] = a.numRegs >= regs ? 1 : 2;
+  }
+  return cache[dev] == 1 ? FA_OK : FA_ERR_INTERNAL;
+}
+
 int check_problem(int B, int H, int N, int d, float scale, int causal, int window) {
   if (B < 1 || H < 1 || N < 1) return FA_ERR_SHAPE;
   const long long bh = (long long)B * H;
@@ -324,6 +340,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
         !make_map_bf16(&tdv, dv, D, N, H_kv, B, st[7], 32))
       return FA_ERR_CUDA;
     if (set_smem(fa_bwd_kernel<D>, smem) != FA_OK) return FA_ERR_CUDA;
+    if (int rs = check_launch_regs(fa_bwd_kernel<D>, kBwdLaunchRegs); rs != FA_OK) return rs;
     // one CTA per (K/V head, key tile)
     fa_bwd_kernel<D><<<unsigned(prm.n_kv_tiles) * unsigned(BH_kv), kBwdThreads, smem, stream>>>(tq, tk, tv, tdo,
                                                                                                    tdq, tdk, tdv, prm);

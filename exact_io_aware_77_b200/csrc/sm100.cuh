@@ -92,6 +92,44 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   if (mbar_try_wait(bar, parity)) return true;
   return mbar_wait_slow(bar, parity, abort, limit_ns);
 }
+// The same wait with no call: a kernel that moves registers between its warpgroups (setmaxnreg)
+// cannot call a function from a region whose register budget differs from the function-wide one.
+__device__ __forceinline__ bool mbar_wait_inl(uint32_t bar, uint32_t parity, volatile int* abort,
+                                              uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait_suspend(bar, parity, 1000u)) return true;
+    if ((it & 63u) == 0) {
+      if (*abort) return false;
+      if (global_timer_ns() - t0 > limit_ns) {
+        *abort = 1;
+        atomicOr(&g_status, FA_DEVICE_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+__device__ __forceinline__ bool mbar_wait_drain_inl(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  int never = 0;
+  return mbar_wait_inl(bar, parity, &never, limit_ns);
+}
+
+// Move registers between the warpgroups of a CTA (setmaxnreg); every warp of a warpgroup makes
+// the same call.  regs_lower<N> returns the registers above N to the CTA's pool; regs_raise<N>
+// waits until the pool holds enough to grow to N, so the raised counts must fit in what the CTA
+// was launched with (threads x registers per thread), or it waits forever: the host checks the
+// kernel's register count before the first launch.
+template <uint32_t N>
+__device__ __forceinline__ void regs_lower() {
+  static_assert(N >= 24 && N <= 256 && N % 8 == 0, "setmaxnreg count");
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_raise() {
+  static_assert(N >= 24 && N <= 256 && N % 8 == 0, "setmaxnreg count");
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
 
 // Bounded wait that ignores the abort flag: used on the way out of a kernel to let copies
 // and MMAs already in flight land before shared or tensor memory is released.

@@ -257,6 +257,17 @@ inline bool mbar_wait_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
   int never = 0;
   return mbar_wait(bar, parity, &never, limit_ns);
 }
+// the inline forms the warpgroup-budget kernels use, and the budget moves (no effect on the host)
+inline bool mbar_wait_inl(uint32_t bar, uint32_t parity, volatile int* abort, uint64_t limit_ns) {
+  return mbar_wait(bar, parity, abort, limit_ns);
+}
+inline bool mbar_wait_drain_inl(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  return mbar_wait_drain(bar, parity, limit_ns);
+}
+template <uint32_t N>
+inline void regs_lower() {}
+template <uint32_t N>
+inline void regs_raise() {}
 
 // ------------------------------------------------------------ TMA
 struct CUtensorMap {
