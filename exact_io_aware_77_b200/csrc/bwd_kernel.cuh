@@ -61,7 +61,7 @@ constexpr int kBwdWarpMma = 13;    // warps 14-15 complete the TMA/MMA warpgroup
 // raise themselves to kBwdRegsCompute and the readout warpgroup to kBwdRegsRead out of what the
 // TMA/MMA warpgroup gives back by lowering itself to kBwdRegsOther.
 constexpr int kBwdLaunchRegs = 65536 / kBwdThreads;
-constexpr int kBwdRegsCompute = 160;
+constexpr int kBwdRegsCompute = 152;
 constexpr int kBwdRegsRead = 88;
 constexpr int kBwdRegsOther = 4 * kBwdLaunchRegs - 2 * kBwdRegsCompute - kBwdRegsRead;
 static_assert(kBwdRegsOther >= 24 && kBwdRegsOther % 8 == 0 &&
