@@ -606,20 +606,20 @@ def measure_e2e(fa, torch, wl, dev, stream, q_h, k_h, v_h, do_h, has_bwd, steps,
 # the workload the bench line times (the causal B2 H32 N4096 d128 one, or the decode one), keyed by kernel, with the SHA-1 of the kernel's sources
 # when the counters were taken (profiles/ holds the summaries).  A changed source reports null.
 NCU_TRAFFIC = {
-    "fa_fwd_kernel<128>": {"bytes": 249418240,
+    "fa_fwd_kernel<128>": {"bytes": 249242624,
                            "sources": {"fwd_kernel.cuh": "faf4e3c455010476279ab78331d6407948b04090",
-                                       "sm100.cuh": "b946d4acd10e4cd21e6f26dd3f8bd28a88214938",
+                                       "sm100.cuh": "d0155c807bbebb96a598c40bfe5826be5d752097",
                                        "grid_sched.cuh": "d69cc1d77285fb320f5966be935efafc0d37f593"}},
-    "fa_bwd_kernel<128>": {"bytes": 625575424,
-                           "sources": {"bwd_kernel.cuh": "6325a581d04ec87cf938a74f935012a499277631",
-                                       "sm100.cuh": "b946d4acd10e4cd21e6f26dd3f8bd28a88214938",
+    "fa_bwd_kernel<128>": {"bytes": 625636352,
+                           "sources": {"bwd_kernel.cuh": "6a4b8d5f32cf10f7fabb8e873f01767ce9f509a5",
+                                       "sm100.cuh": "d0155c807bbebb96a598c40bfe5826be5d752097",
                                        "grid_sched.cuh": "d69cc1d77285fb320f5966be935efafc0d37f593"}},
     # the decode workload (B8 H64 with 8 K/V heads, N_q 1, N_k 32768): both kernels of one step
     "fa_decode_kernel<128,false>+fa_decode_merge_kernel<128>": {
-        "bytes": 1081032960,
+        "bytes": 1080936960,
         "sources": {"decode_kernel.cuh": "0b0388b3ae07210bfe25fc0f560b02d870b7b25b",
                     "decode_ops.cuh": "ce1146b0eed95a0cdd62429f8d0ff970bb9bdcf5",
-                    "sm100.cuh": "b946d4acd10e4cd21e6f26dd3f8bd28a88214938"}},
+                    "sm100.cuh": "d0155c807bbebb96a598c40bfe5826be5d752097"}},
 }
 
 
