@@ -610,8 +610,8 @@ NCU_TRAFFIC = {
                            "sources": {"fwd_kernel.cuh": "faf4e3c455010476279ab78331d6407948b04090",
                                        "sm100.cuh": "d0155c807bbebb96a598c40bfe5826be5d752097",
                                        "grid_sched.cuh": "d69cc1d77285fb320f5966be935efafc0d37f593"}},
-    "fa_bwd_kernel<128>": {"bytes": 625636352,
-                           "sources": {"bwd_kernel.cuh": "6a4b8d5f32cf10f7fabb8e873f01767ce9f509a5",
+    "fa_bwd_kernel<128>": {"bytes": 625917696,
+                           "sources": {"bwd_kernel.cuh": "4ff5578c97f3b087315277901bd12f07653933dd",
                                        "sm100.cuh": "d0155c807bbebb96a598c40bfe5826be5d752097",
                                        "grid_sched.cuh": "d69cc1d77285fb320f5966be935efafc0d37f593"}},
     # the decode workload (B8 H64 with 8 K/V heads, N_q 1, N_k 32768): both kernels of one step

@@ -20,13 +20,16 @@
 //   warp 13     MMA issuer, per query tile i in the order
 //                 dV += P_i^T dO_i, S_{i+1}^T = K Q_{i+1}^T, dK += dS_i^T Q_i, dQ_i = dS_i K,
 //                 dP_{i+1}^T = V dO_{i+1}^T
-//               (dV and dK read their A operand from TMEM), so that the exponentials of tile
-//               i+1 run while dK_i and dQ_i are computed, and dS of tile i+1 while dV_{i+1}
-//               and S_{i+2} are.
+//               (dV and dK read their A operand from TMEM; dQ reads dS from shared memory), so
+//               that the exponentials of tile i+1 run while dK_i and dQ_i are computed, and dS
+//               of tile i+1 while dV_{i+1} and S_{i+2} are.  The kDkSmem form (shared K/V
+//               heads) swaps dK_i and dQ_i, dK reading dS from shared memory as well, so that
+//               the readout of dQ_i runs while dK_i is computed.
 //   warps 0-7   two per TMEM lane quadrant; warp w owns lanes 32 (w % 4).. and the query half
 //               w / 4 of each tile.  Phase A: P^T = exp2(S^T c - L) with the causal/window mask,
-//               stored to TMEM as bf16.  Phase B: dS^T = P^T o (dP^T - D) to TMEM (A of dK) and
-//               to shared memory (A of dQ).  Order per tile: B(i), A(i+1).  At the end: dK
+//               stored to TMEM as bf16.  Phase B: dS^T = P^T o (dP^T - D) to shared memory (A of
+//               dQ; and of dK in the kDkSmem form) and to TMEM (A of dK in the other form).
+//               Order per tile: B(i), A(i+1).  At the end: dK
 //               (half 0), dV (half 1), staged in the idle Q buffers and written by TMA tensor
 //               stores.
 //   warps 8-11  dQ readout, one per TMEM lane quadrant: all D columns of its 32 query rows of
@@ -37,10 +40,11 @@
 //   warps 14-15 none (they complete the last warpgroup, whose registers go to the others:
 //               setmaxnreg moves them from the TMA/MMA warpgroup to the compute and readout ones).
 // TMEM columns: dK [0,128), dV [128,256), S^T [256,384) with P^T in [256,288) and [320,352)
-// once read, dP^T [384,512) with dS^T in [384,416) and [448,480) once read, and dQ in
-// [384,512).  MMAs of one thread
-// run in order, which makes each reuse safe: S_{i+1} is issued after dV_i read P_i, dQ_i after
-// dK_i read dS_i; only dP_{i+1} waits until the readout warps have read dQ_i out.
+// once read, dP^T [384,512) with dS^T in [384,416) and [448,480) once read (TMEM form), and
+// dQ in [384,512).  MMAs of one thread run in order, which makes each reuse safe: S_{i+1} is
+// issued after dV_i read P_i, dQ_i after dK_i read dS_i^T (TMEM form) or after phase B read
+// dP_i^T; dP_{i+1} waits until the readout warps have read dQ_i out, and phase B of tile i+1
+// rewrites the dS buffer only once dP_{i+1}, and so dQ_i and dK_i before it, has completed.
 #pragma once
 
 #include <type_traits>
@@ -196,7 +200,12 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_final(const float* __restrict__
 // tm_dq: the fp32 accumulator [BH, Np, D] as the 4-D tensor (D, Np, BH, 1), 32 x 32 boxes with
 // the 128-byte swizzle (the layout of a compute warp's staging slot).  tm_dk, tm_dv: dK and dV
 // as (D, N, H_kv, B), boxes of 64 columns x 32 rows (one compute warp's key rows).
-template <int D>
+// kDkSmem: dK += dS^T Q_i reads dS from shared memory and is issued after dQ_i = dS_i K, so that
+// the readout of dQ_i runs under it; otherwise dK reads dS^T from TMEM (written there by phase B)
+// and is issued first.  The host takes the first form when K/V heads are shared: a CTA then
+// adds into the accumulators of every query head of its group, the L2 holds more of them at
+// once, and the readout is slower; with one query head per K/V head the second is faster.
+template <int D, bool kDkSmem>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -324,6 +333,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint64_t dv_kmaj = sw128_desc(smem_u32(sm.v), 16, 1024);
       const uint64_t dk_mn = sw128_desc(smem_u32(sm.k), 16384, 1024);
       const uint64_t dds_mn = sw128_desc(smem_u32(sm.ds), 16384, 1024);
+      // the dS buffer holds one 128-byte row of 64 queries per key: MN-major dS for dQ, K-major
+      // dS^T for dK
+      const uint64_t dds_kmaj = sw128_desc(smem_u32(sm.ds), 16, 1024);
+      constexpr uint32_t idesc_dk = idesc_bf16_f32(128, D, false, true);            // dK (A = dS^T)
       // X^T = M_tile N_i^T with both operands K-major over the head dim (S^T and dP^T)
       auto issue_t = [&](uint64_t a, const uint8_t* b_tile, uint32_t d_col) {
         const uint64_t b = sw128_desc(smem_u32(b_tile), 16, 1024);
@@ -333,9 +346,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           mma_bf16_ss_w(tmem + d_col, desc_advance(a, off), desc_advance(b, off), idesc_t, kk > 0);
         }
       };
-      // acc += A(TMEM, 128 x 128 queries) * B (MN-major Q_i or dO_i: 16 queries = 2 KB per k-step)
-      // A (P^T or dS^T) sits in TMEM as two 32-column halves, one per query half, at a_col and
-      // a_col + 64; each 16-query k-step takes 8 of those columns
+      // dV, dK += A(TMEM, 128 x 128 queries) * B (MN-major dO_i or Q_i: 16 queries = 2 KB per
+      // k-step); A (P^T or dS^T) sits in TMEM as two 32-column halves, one per query half, at
+      // a_col and a_col + 64; each 16-query k-step takes 8 of those columns
       auto issue_kv = [&](uint32_t a_col, const uint8_t* b_tile, uint32_t d_col, bool first) {
         const uint64_t b = sw128_desc(smem_u32(b_tile), 16384, 1024);
 #pragma unroll
@@ -370,16 +383,34 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           issue_t(dk_kmaj, sm.q[qn], kTS);
           mma_commit_w(smem_u32(&sm.s_full));
         }
-        // dK += dS^T Q_i, then dQ_i = dS_i K (A = dS^T from shared memory, MN-major over queries)
         if (!wait(smem_u32(&sm.ds_full), it & 1)) break;
-        tc_fence_after();
-        issue_kv(kTdS, sm.q[qs], kTdK, it == 0);
-        if (!wait(smem_u32(&sm.dq_free), (it & 1) ^ 1)) break;
-        tc_fence_after();
+        if constexpr (kDkSmem) {
+          // dQ_i = dS_i K first, so that its readout runs under dK += dS^T Q_i; both read dS
+          // from shared memory (dQ_i overwrites the dP^T columns, which phase B has read)
+          if (!wait(smem_u32(&sm.dq_free), (it & 1) ^ 1)) break;
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < kBwdKeys / 16; ++kk)
-          mma_bf16_ss_w(tmem + kTdQ, desc_advance(dds_mn, kk * 2048), desc_advance(dk_mn, kk * 2048), idesc_q, kk > 0);
-        mma_commit_w(smem_u32(&sm.dq_full));
+          for (int kk = 0; kk < kBwdKeys / 16; ++kk)
+            mma_bf16_ss_w(tmem + kTdQ, desc_advance(dds_mn, kk * 2048), desc_advance(dk_mn, kk * 2048), idesc_q,
+                          kk > 0);
+          mma_commit_w(smem_u32(&sm.dq_full));
+          const uint64_t bq = sw128_desc(smem_u32(sm.q[qs]), 16384, 1024);
+#pragma unroll
+          for (int kk = 0; kk < kBwdRows / 16; ++kk)
+            mma_bf16_ss_w(tmem + kTdK, desc_advance(dds_kmaj, (kk >> 2) * 16384 + (kk & 3) * 32),
+                          desc_advance(bq, kk * 2048), idesc_dk, (it == 0 && kk == 0) ? 0u : 1u);
+        } else {
+          // dK += dS^T Q_i with A = dS^T from TMEM, then dQ_i = dS_i K into the same columns
+          tc_fence_after();
+          issue_kv(kTdS, sm.q[qs], kTdK, it == 0);
+          if (!wait(smem_u32(&sm.dq_free), (it & 1) ^ 1)) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kBwdKeys / 16; ++kk)
+            mma_bf16_ss_w(tmem + kTdQ, desc_advance(dds_mn, kk * 2048), desc_advance(dk_mn, kk * 2048), idesc_q,
+                          kk > 0);
+          mma_commit_w(smem_u32(&sm.dq_full));
+        }
         mma_commit_w(smem_u32(&sm.q_empty[qs]));
         // dP^T of the next tile once dQ_i has been read out of the same columns
         if (has_next) {
@@ -458,7 +489,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t lane_base = uint32_t(quad * 32) << 16;
     const float c = prm.scale_log2;
     const uint32_t col_s = kTS + hq * 64;      // my S^T columns; P^T goes to the first 32 of them
-    const uint32_t col_dp = kTdP + hq * 64;    // my dP^T columns; dS^T goes to the first 32 of them
+    const uint32_t col_dp = kTdP + hq * 64;    // my dP^T columns
     const uint32_t ds_row = smem_u32(sm.ds) + hq * 16384 + r * 128;   // 64 queries = one 128-byte row
     const uint32_t sw = r & 7;
     uint32_t pk[32];                           // packed P^T of the current tile (phase A -> phase B)
@@ -516,11 +547,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_arrive(smem_u32(&sm.pa_full));
       return true;
     };
-    // phase B: dS^T = P^T o (dP^T - D) for my 64 queries -> TMEM (bf16) and shared memory
+    // phase B: dS^T = P^T o (dP^T - D) for my 64 queries -> shared memory and, unless dK reads
+    // it from there, TMEM (bf16)
     auto phase_b = [&](int it) -> bool {
       const int qs = it % kBwdQStages;
       // my rows of the dS buffer are free: dP of this tile completing means every earlier MMA
-      // has, the dQ product that read the previous tile's dS among them
+      // has, the products that read the previous tile's dS among them
       const bool w_ok = mbar_wait_inl(smem_u32(&sm.dp_full), it & 1, abort, lim);
       if (!__all_sync(0xffffffffu, w_ok)) return false;
       tc_fence_after();
@@ -542,12 +574,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         f2_split(f2_mul(t2, p2), s0, s1);
         pd[j2] = pack_bf16x2(s0, s1);
       }
-      tmem_st16(tmem + lane_base + col_dp, pd);
-      tmem_st16(tmem + lane_base + col_dp + 16, pd + 16);
+      if constexpr (!kDkSmem) {   // dS^T into my dP^T columns, the A operand of dK
+        tmem_st16(tmem + lane_base + col_dp, pd);
+        tmem_st16(tmem + lane_base + col_dp + 16, pd + 16);
+      }
 #pragma unroll
       for (int c16 = 0; c16 < 8; ++c16)
         st_shared_v4(ds_row + ((c16 ^ sw) << 4), pd[4 * c16], pd[4 * c16 + 1], pd[4 * c16 + 2], pd[4 * c16 + 3]);
-      tmem_st_wait();
+      if constexpr (!kDkSmem) tmem_st_wait();
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(smem_u32(&sm.ds_full));

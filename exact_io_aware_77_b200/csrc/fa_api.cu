@@ -136,14 +136,16 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 // A kernel that moves registers between its warpgroups (setmaxnreg) must be launched with at
 // least `regs` registers per thread: the raised budgets come out of the launch share, and a raise
 // the CTA cannot cover would wait forever.  Checked once per kernel and device.
-template <class Kernel>
-int check_launch_regs(Kernel k, int regs) {
+// (The kernel is a template argument, so that each kernel has its own cache: instantiations
+// share a function-pointer type.)
+template <auto Kernel>
+int check_launch_regs(int regs) {
   static int cache[kMaxDevices] = {0};   // 0 unknown, 1 ok, 2 too few
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
   if (cache[dev] == 0) {
     cudaFuncAttributes a;
-    if (cudaFuncGetAttributes(&a, k) != cudaSuccess) return FA_ERR_CUDA;
+    if (cudaFuncGetAttributes(&a, Kernel) != cudaSuccess) return FA_ERR_CUDA;
     cache[dev] = a.numRegs >= regs ? 1 : 2;
   }
   return cache[dev] == 1 ? FA_OK : FA_ERR_INTERNAL;
@@ -167,6 +169,16 @@ template <class Kernel>
 int set_smem(Kernel k, int bytes) {
   return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess ? FA_OK
                                                                                                      : FA_ERR_CUDA;
+}
+
+// launch a kernel that moves registers between its warpgroups, once its launch share is checked
+template <auto Kernel, class... Args>
+int launch_regs_checked(unsigned grid, unsigned threads, int smem, cudaStream_t stream, int regs,
+                        const Args&... args) {
+  if (set_smem(Kernel, smem) != FA_OK) return FA_ERR_CUDA;
+  if (int rs = check_launch_regs<Kernel>(regs); rs != FA_OK) return rs;
+  Kernel<<<grid, threads, smem, stream>>>(args...);
+  return FA_OK;
 }
 
 // tensor maps and parameters of the d = 64 / 128 forward (fwd_kernel.cuh)
@@ -339,11 +351,15 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
     if (!make_map_dq_acc(&tdq, dq_acc, D, Np, BH) || !make_map_bf16(&tdk, dk, D, N, H_kv, B, st[6], 32) ||
         !make_map_bf16(&tdv, dv, D, N, H_kv, B, st[7], 32))
       return FA_ERR_CUDA;
-    if (set_smem(fa_bwd_kernel<D>, smem) != FA_OK) return FA_ERR_CUDA;
-    if (int rs = check_launch_regs(fa_bwd_kernel<D>, kBwdLaunchRegs); rs != FA_OK) return rs;
-    // one CTA per (K/V head, key tile)
-    fa_bwd_kernel<D><<<unsigned(prm.n_kv_tiles) * unsigned(BH_kv), kBwdThreads, smem, stream>>>(tq, tk, tv, tdo,
-                                                                                                   tdq, tdk, tdv, prm);
+    // one CTA per (K/V head, key tile); dK from the shared-memory dS when K/V heads are shared
+    const unsigned grid = unsigned(prm.n_kv_tiles) * unsigned(BH_kv);
+    const int rs = prm.group > 1 ? launch_regs_checked<fa_bwd_kernel<D, true>>(grid, kBwdThreads, smem, stream,
+                                                                               kBwdLaunchRegs, tq, tk, tv, tdo, tdq,
+                                                                               tdk, tdv, prm)
+                                 : launch_regs_checked<fa_bwd_kernel<D, false>>(grid, kBwdThreads, smem, stream,
+                                                                                kBwdLaunchRegs, tq, tk, tv, tdo, tdq,
+                                                                                tdk, tdv, prm);
+    if (rs != FA_OK) return rs;
   }
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }

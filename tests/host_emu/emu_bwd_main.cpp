@@ -132,8 +132,13 @@ int main(int argc, char** argv) {
   emu_launch(unsigned(prm.n_kv_tiles) * unsigned(BH_kv), kB256Threads, sizeof(fa::smem_raw),
              [&] { fa_bwd256_kernel(tq, tk, tv, tdo, tdq, prm); }, fa::smem_raw);
 #else
-  emu_launch(unsigned(prm.n_kv_tiles) * unsigned(BH_kv), kBwdThreads, sizeof(fa::smem_raw),
-             [&] { fa_bwd_kernel<D>(tq, tk, tv, tdo, tdq, tdk, tdv, prm); }, fa::smem_raw);
+  // the form the host library launches: dK from the shared-memory dS when K/V heads are shared
+  if (prm.group > 1)
+    emu_launch(unsigned(prm.n_kv_tiles) * unsigned(BH_kv), kBwdThreads, sizeof(fa::smem_raw),
+               [&] { fa_bwd_kernel<D, true>(tq, tk, tv, tdo, tdq, tdk, tdv, prm); }, fa::smem_raw);
+  else
+    emu_launch(unsigned(prm.n_kv_tiles) * unsigned(BH_kv), kBwdThreads, sizeof(fa::smem_raw),
+               [&] { fa_bwd_kernel<D, false>(tq, tk, tv, tdo, tdq, tdk, tdv, prm); }, fa::smem_raw);
 #endif
   if (g_status != 0) { std::fprintf(stderr, "device status %d\n", g_status); return 3; }
   const long long rows = (long long)BH * N;
